@@ -1,0 +1,141 @@
+"""Python binding of libgdn (Gated DeltaNet recurrence on B200, sm_100a).
+
+Argument marshalling only: every step of the recurrence runs in the CUDA
+kernels of ``libgdn.so`` behind the C ABI of ``include/gdn.h``.  PyTorch
+provides device memory and streams.  There is no CPU fallback: if the native
+library is missing or no CUDA device is present, the calls raise.
+
+    out, s_final = chunk_fwd(q, k, v, g, beta, state_in)        # prefill
+    o = recurrent_step(q, k, v, g, beta, state)                 # decode, in place
+
+Gate mode is read from g's shape: [..., H] scalar per head, [..., H, dk] per
+key channel.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import torch
+
+_PKG = Path(__file__).resolve().parent
+LIB_PATH = _PKG / "libgdn.so"
+
+GDN_OK = 0
+GDN_ERR_INVALID_ARG = -1
+GDN_ERR_UNSUPPORTED = -2
+GDN_ERR_MISALIGNED = -3
+GDN_ERR_CUDA = -4
+GDN_ERR_NOMEM = -5
+GDN_ERR_TIMEOUT = -6
+GATE_SCALAR = 0
+GATE_CHANNEL = 1
+IO_BF16 = 0
+IO_F32 = 1
+
+SYMBOLS = ("gdn_chunk_fwd", "gdn_chunk_fwd_ex", "gdn_recurrent_step", "gdn_recurrent_step_ex",
+           "gdn_check", "gdn_status_string")
+
+_lib = None
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+def load() -> ctypes.CDLL:
+    """Load libgdn.so (raises if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not LIB_PATH.exists():
+        raise ImportError(f"{LIB_PATH} is missing; run `python -m gated_delta_rule_77_b200.build`")
+    lib = ctypes.CDLL(str(LIB_PATH))
+    vp, fp, i = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
+    lib.gdn_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i, i, i, i, i, i, vp]
+    lib.gdn_chunk_fwd_ex.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i, i, i, i, i, i, i, i, vp]
+    lib.gdn_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, vp]
+    lib.gdn_recurrent_step_ex.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, i, vp]
+    lib.gdn_check.argtypes = [vp]
+    lib.gdn_status_string.argtypes = [i]
+    lib.gdn_status_string.restype = ctypes.c_char_p
+    for name in SYMBOLS[:-1]:
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().gdn_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("every tensor must be a contiguous CUDA tensor")
+
+
+def _io_code(dtype):
+    if dtype == torch.bfloat16:
+        return IO_BF16
+    if dtype == torch.float32:
+        return IO_F32
+    raise ValueError(f"unsupported I/O dtype {dtype}")
+
+
+def chunk_fwd(q, k, v, g, beta, state_in=None, *, out=None, state_out=None,
+              return_state: bool = True, chunk_size: int = 0, stream=None):
+    """Chunkwise prefill.  q, k [B,T,H,dk]; v [B,T,H,dv]; g [B,T,H] or
+    [B,T,H,dk] fp32; beta [B,T,H] fp32; state_in [B,H,dk,dv] fp32 or None.
+    Returns (out [B,T,H,dv] in v's dtype, final state or None)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    gate = GATE_CHANNEL if g.dim() == 4 else GATE_SCALAR
+    if out is None:
+        out = torch.empty(B, T, H, dv, dtype=v.dtype, device=v.device)
+    if state_out is None and return_state:
+        state_out = torch.empty(B, H, dk, dv, dtype=torch.float32, device=v.device)
+    _check_cuda(q, k, v, g, beta, state_in, out, state_out)
+    rc = load().gdn_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in),
+                                 _ptr(out), _ptr(state_out), B, T, H, dk, dv, gate,
+                                 _io_code(q.dtype), int(chunk_size), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_chunk_fwd_ex")
+    return out, state_out
+
+
+def recurrent_step(q, k, v, g, beta, state, *, state_out=None, out=None, stream=None):
+    """One decode step.  q, k [B,H,dk]; v [B,H,dv]; g [B,H] or [B,H,dk];
+    beta [B,H]; state [B,H,dk,dv] fp32 (updated in place unless state_out is
+    given).  Returns out [B,H,dv] fp32."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    gate = GATE_CHANNEL if g.dim() == 3 else GATE_SCALAR
+    if state_out is None:
+        state_out = state
+    if out is None:
+        out = torch.empty(B, H, dv, dtype=torch.float32, device=v.device)
+    _check_cuda(q, k, v, g, beta, state, state_out, out)
+    rc = load().gdn_recurrent_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                      _ptr(state), _ptr(state_out), _ptr(out), B, H, dk, dv,
+                                      gate, _io_code(q.dtype), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_recurrent_step_ex")
+    return out
+
+
+def check(stream=None) -> int:
+    """Synchronise the stream and report a bounded-wait timeout, if any."""
+    return int(load().gdn_check(_stream(stream)))

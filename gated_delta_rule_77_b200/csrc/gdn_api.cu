@@ -1,0 +1,166 @@
+// gdn_api.cu -- the C ABI of libgdn (declared in include/gdn.h): argument
+// validation, dispatch to the kernels, status strings.
+//
+// Every check runs on the host before anything is launched, so an invalid
+// call has no side effect.  Calls never synchronise (except gdn_check).
+
+#include <stdint.h>
+
+#include "../../include/gdn.h"
+#include "gdn_internal.cuh"
+
+namespace {
+
+struct Range {
+    uintptr_t lo, hi;  // [lo, hi)
+};
+
+Range range_of(const void* p, size_t bytes) {
+    uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return Range{a, a + bytes};
+}
+
+bool overlaps(Range a, Range b) {
+    return a.lo < b.hi && b.lo < a.hi && a.lo != a.hi && b.lo != b.hi;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool dim_ok(int d) { return d == 64 || d == 128; }
+
+int to_status(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
+
+// Shared validation of the tensors of one call.  `T_tokens` is T for the
+// prefill and 1 for a decode step (its layout is the T = 1 case).
+int validate(const void* q, const void* k, const void* v, const float* g, const float* beta,
+             const float* state_in, const float* state_out, const void* out,
+             long B, long T_tokens, long H, int dk, int dv, int gate_mode, int io_dtype,
+             bool out_f32, bool state_in_required)
+{
+    // With no tokens the per-token tensors are never touched and may be null.
+    if (T_tokens != 0 && (!q || !k || !v || !g || !beta || !out)) return GDN_ERR_INVALID_ARG;
+    if (state_in_required && (!state_in || !state_out)) return GDN_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || T_tokens < 0 || dk < 1 || dv < 1) return GDN_ERR_INVALID_ARG;
+    if (gate_mode != GDN_GATE_SCALAR && gate_mode != GDN_GATE_CHANNEL) return GDN_ERR_INVALID_ARG;
+    if (io_dtype != GDN_IO_BF16 && io_dtype != GDN_IO_F32) return GDN_ERR_INVALID_ARG;
+    if (!dim_ok(dk) || !dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
+    // Keep every element index well inside 64-bit arithmetic and the TMA
+    // coordinate range.
+    if (B > (1L << 20) || H > (1L << 16) || T_tokens > (1L << 30)) return GDN_ERR_UNSUPPORTED;
+    const void* ptrs[] = {q, k, v, g, beta, state_in, state_out, out};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
+
+    const size_t esz = io_dtype == GDN_IO_F32 ? 4 : 2;
+    const size_t tok = (size_t)B * (size_t)T_tokens * (size_t)H;
+    const size_t st = (size_t)B * (size_t)H * (size_t)dk * (size_t)dv * 4;
+    const Range rq = range_of(q, tok * dk * esz), rk = range_of(k, tok * dk * esz),
+                rv = range_of(v, tok * dv * esz),
+                rg = range_of(g, tok * (gate_mode == GDN_GATE_CHANNEL ? dk : 1) * 4),
+                rb = range_of(beta, tok * 4),
+                ro = range_of(out, tok * dv * (out_f32 ? 4 : esz));
+    const Range rsi = state_in ? range_of(state_in, st) : Range{0, 0};
+    const Range rso = state_out ? range_of(state_out, st) : Range{0, 0};
+    // The output aliases nothing; the final state may only coincide exactly
+    // with the initial state.
+    for (Range r : {rq, rk, rv, rg, rb, rsi, rso})
+        if (overlaps(ro, r)) return GDN_ERR_INVALID_ARG;
+    for (Range r : {rq, rk, rv, rg, rb})
+        if (overlaps(rso, r)) return GDN_ERR_INVALID_ARG;
+    if (state_in && state_out && state_in != state_out && overlaps(rsi, rso))
+        return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* g,
+                     const float* beta, const float* state_in, void* out, float* state_out,
+                     int B, int T, int H, int dk, int dv, int gate_mode, int io_dtype,
+                     int chunk_size, gdn_stream_t stream_)
+{
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    int rc = validate(q, k, v, g, beta, state_in, state_out, out, B, T, H, dk, dv, gate_mode,
+                      io_dtype, io_dtype == GDN_IO_F32, false);
+    if (rc != GDN_OK) return rc;
+    const bool f32 = io_dtype == GDN_IO_F32;
+    if (f32) {
+        if (chunk_size != 0 && chunk_size != 1) return GDN_ERR_UNSUPPORTED;
+    } else if (chunk_size != 0 && chunk_size != 1 && chunk_size != 64) {
+        return GDN_ERR_UNSUPPORTED;
+    }
+    if (T == 0) {
+        if (!state_out) return GDN_OK;
+        const size_t st = (size_t)B * H * dk * dv * sizeof(float);
+        if (state_in == state_out) return GDN_OK;
+        cudaError_t e = state_in
+            ? cudaMemcpyAsync(state_out, state_in, st, cudaMemcpyDeviceToDevice, stream)
+            : cudaMemsetAsync(state_out, 0, st, stream);
+        return to_status(e);
+    }
+    gdn::Problem p{q, k, v, g, beta, state_in, state_out, out, B, T, H, dk, dv,
+                   gate_mode == GDN_GATE_CHANNEL, f32, f32};
+    if (!f32 && chunk_size != 1) {
+        cudaError_t e = gdn::launch_chunk_sm100(p, stream);
+        if (e != cudaErrorNotSupported) return to_status(e);
+        if (chunk_size == 64) return GDN_ERR_UNSUPPORTED;
+    }
+    return to_status(gdn::launch_recurrent(p, stream));
+}
+
+int gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                  const float* beta, const float* state_in, void* out, float* state_out,
+                  int B, int T, int H, int dk, int dv, int gate_mode, gdn_stream_t stream)
+{
+    return gdn_chunk_fwd_ex(q, k, v, g, beta, state_in, out, state_out, B, T, H, dk, dv,
+                            gate_mode, GDN_IO_BF16, 0, stream);
+}
+
+int gdn_recurrent_step_ex(const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, const float* state_in, float* state_out,
+                          void* out, int B, int H, int dk, int dv, int gate_mode,
+                          int io_dtype, gdn_stream_t stream_)
+{
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    int rc = validate(q, k, v, g, beta, state_in, state_out, out, B, 1, H, dk, dv, gate_mode,
+                      io_dtype, true, true);
+    if (rc != GDN_OK) return rc;
+    gdn::Problem p{q, k, v, g, beta, state_in, state_out, out, B, 1, H, dk, dv,
+                   gate_mode == GDN_GATE_CHANNEL, io_dtype == GDN_IO_F32, true};
+    return to_status(gdn::launch_recurrent(p, stream));
+}
+
+int gdn_recurrent_step(const void* q, const void* k, const void* v, const float* g,
+                       const float* beta, const float* state_in, float* state_out, void* out,
+                       int B, int H, int dk, int dv, int gate_mode, gdn_stream_t stream)
+{
+    return gdn_recurrent_step_ex(q, k, v, g, beta, state_in, state_out, out, B, H, dk, dv,
+                                 gate_mode, GDN_IO_BF16, stream);
+}
+
+int gdn_check(gdn_stream_t stream_)
+{
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    unsigned int status = 0;
+    cudaError_t e = gdn::read_and_clear_status(&status, stream);
+    if (e != cudaSuccess) return GDN_ERR_CUDA;
+    return status ? GDN_ERR_TIMEOUT : GDN_OK;
+}
+
+const char* gdn_status_string(int status)
+{
+    switch (status) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+        case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+        case GDN_ERR_MISALIGNED: return "GDN_ERR_MISALIGNED";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+        case GDN_ERR_NOMEM: return "GDN_ERR_NOMEM";
+        case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+        default: return "GDN_ERR_UNKNOWN";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,40 @@
+// gdn_internal.cuh -- declarations shared by the CUDA sources of libgdn.
+// Not part of the public ABI (that is include/gdn.h).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn {
+
+// Arguments of one recurrence call, already validated by the ABI layer.
+// Token-major layouts: q, k [B, T, H, dk]; v, out [B, T, H, dv];
+// g [B, T, H] or [B, T, H, dk]; beta [B, T, H]; states [B, H, dk, dv].
+// A decode step is the T = 1 case of the same layout ([B, H, d]).
+struct Problem {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* g;
+    const float* beta;
+    const float* state_in;   // may be null (zero state)
+    float* state_out;        // may be null (not written)
+    void* out;
+    int B, T, H, dk, dv;
+    bool per_channel;
+    bool io_f32;             // q, k, v in fp32 (else bf16)
+    bool out_f32;            // out in fp32 (else bf16)
+};
+
+// Token-serial fused recurrence (decode, and the fp32 / fallback prefill).
+cudaError_t launch_recurrent(const Problem& p, cudaStream_t stream);
+
+// Chunkwise tensor-core prefill (bf16 I/O, dk = dv = 128, chunk of 64).
+// Returns cudaErrorNotSupported for shapes it does not handle.
+cudaError_t launch_chunk_sm100(const Problem& p, cudaStream_t stream);
+
+// Device status word written by kernels that abandon a bounded wait.
+cudaError_t read_and_clear_status(unsigned int* status, cudaStream_t stream);
+
+}  // namespace gdn

@@ -1,0 +1,146 @@
+/*
+ * gdn.h -- C ABI of libgdn, a B200 (sm_100a) implementation of the Gated
+ * DeltaNet mixer recurrence.
+ *
+ * Method (Atomic-GDN2 model card, section 2.1 "Gated DeltaNet-2"):
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t,          alpha_t = exp(g_t)
+ *
+ * The caller passes the log-decay g (g <= 0); the library applies the
+ * exponential itself (same section: the kernel is handed g directly).  The
+ * gate is either one value per (token, head) -- GDN_GATE_SCALAR -- or one
+ * value per key channel -- GDN_GATE_CHANNEL, the GDN-2 / KDA form ("Gated
+ * DeltaNet" entity trail, finding of 2026-07-29).  No 1/sqrt(dk) query scale
+ * is applied.  The library neither clamps g nor normalises q and k; both are
+ * the caller's contract.
+ *
+ * Two execution modes compute the same mathematics (entity trail, finding of
+ * 2026-07-29: a fused recurrent mode for decode and a chunkwise mode for
+ * training / prefill):
+ *   gdn_chunk_fwd       chunkwise-parallel prefill over T tokens;
+ *   gdn_recurrent_step  one token per sequence, state updated in place.
+ *
+ * Memory and ownership
+ *   Every pointer is caller-owned DEVICE memory (e.g. a torch tensor's
+ *   data_ptr()), contiguous, row-major, 16-byte aligned.  The library never
+ *   frees caller memory.  Scratch space the prefill needs is taken
+ *   stream-ordered (cudaMallocAsync / cudaFreeAsync on `stream`).
+ *   The recurrent state is fp32, [B, H, dk, dv], row index = key channel --
+ *   the precision the source keeps the state in ("Hybrid layouts: three
+ *   DeltaNet, one attention", section 01 Concept: fp32 recurrent state).
+ *
+ * Streams and synchronisation
+ *   Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *   stream).  No call synchronises the host or the device.
+ *
+ * Errors
+ *   Every argument is validated on the host before anything is launched; an
+ *   invalid call returns a negative status and launches nothing.  A launch
+ *   failure returns GDN_ERR_CUDA.  A kernel that gives up on a bounded
+ *   internal wait records it in a device status word; gdn_check reports it.
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                        /* = cudaStream_t */
+typedef struct CUstream_st* gdn_stream_t;
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = -1,   /* null required pointer, bad size or enum    */
+    GDN_ERR_UNSUPPORTED = -2,   /* valid but not implemented (e.g. dk = 96)   */
+    GDN_ERR_MISALIGNED = -3,    /* a pointer is not 16-byte aligned           */
+    GDN_ERR_CUDA = -4,          /* a CUDA runtime call or launch failed       */
+    GDN_ERR_NOMEM = -5,         /* stream-ordered scratch allocation failed   */
+    GDN_ERR_TIMEOUT = -6        /* a kernel abandoned a bounded wait          */
+} gdn_status;
+
+enum { GDN_GATE_SCALAR = 0, GDN_GATE_CHANNEL = 1 };
+enum { GDN_IO_BF16 = 0, GDN_IO_F32 = 1 };
+
+/*
+ * gdn_chunk_fwd -- chunkwise prefill of T tokens for B sequences and H heads.
+ *
+ *   q, k      [B, T, H, dk]  bf16 (GDN_IO_BF16, the default)
+ *   v         [B, T, H, dv]  bf16
+ *   g         [B, T, H] (GDN_GATE_SCALAR) or [B, T, H, dk] (GDN_GATE_CHANNEL),
+ *             fp32, g <= 0.  The per-channel gate requires g >= -5, the
+ *             domain of the model card's gate parameterisation (section 2.1,
+ *             g = -min(softplus(.), 160/bs2) with bs2 = 32); the chunk
+ *             factorisation relies on that bound.  The scalar gate accepts
+ *             any g <= 0.
+ *   beta      [B, T, H] fp32
+ *   state_in  [B, H, dk, dv] fp32, or NULL for a zero initial state
+ *   out       [B, T, H, dv], same dtype as v; must not alias an input
+ *   state_out [B, H, dk, dv] fp32, or NULL (final state not written);
+ *             state_out == state_in is allowed
+ *   dk, dv    64 or 128 (else GDN_ERR_UNSUPPORTED); B, H >= 1; T >= 0.
+ *   gate_mode GDN_GATE_SCALAR or GDN_GATE_CHANNEL.
+ *   T == 0 writes state_out := state_in (or zeros) and returns GDN_OK; the
+ *   per-token pointers (q, k, v, g, beta, out) may then be NULL.
+ */
+GDN_API int gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                  const float* beta, const float* state_in, void* out, float* state_out,
+                  int B, int T, int H, int dk, int dv, int gate_mode, gdn_stream_t stream);
+
+/*
+ * gdn_chunk_fwd_ex -- gdn_chunk_fwd with an explicit I/O dtype and chunk size.
+ *   io_dtype   GDN_IO_BF16: q, k, v, out bf16 (tensor-core chunk path).
+ *              GDN_IO_F32 : q, k, v, out fp32 (fp32 CUDA-core path, for
+ *                           tolerances tighter than bf16 operands allow).
+ *   chunk_size 0 = default.  bf16: 0 or 64 = chunkwise tensor-core path
+ *              (dk = dv = 128; other dims fall back to the token-serial
+ *              path when chunk_size is 0), 1 = token-serial fused
+ *              recurrence.  fp32: 0 or 1 (token-serial).
+ */
+GDN_API int gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* g,
+                     const float* beta, const float* state_in, void* out, float* state_out,
+                     int B, int T, int H, int dk, int dv, int gate_mode, int io_dtype,
+                     int chunk_size, gdn_stream_t stream);
+
+/*
+ * gdn_recurrent_step -- one decode step for B sequences and H heads.
+ *
+ *   q, k      [B, H, dk] bf16;   v [B, H, dv] bf16
+ *   g         [B, H] or [B, H, dk] fp32 (g <= 0);   beta [B, H] fp32
+ *   state_in  [B, H, dk, dv] fp32 (required)
+ *   state_out [B, H, dk, dv] fp32 (required); == state_in updates in place
+ *   out       [B, H, dv] fp32 (fp32 so that the output keeps the state's
+ *             precision); must not alias an input
+ */
+GDN_API int gdn_recurrent_step(const void* q, const void* k, const void* v, const float* g,
+                       const float* beta, const float* state_in, float* state_out, void* out,
+                       int B, int H, int dk, int dv, int gate_mode, gdn_stream_t stream);
+
+/* gdn_recurrent_step_ex -- io_dtype selects bf16 or fp32 q, k, v; out is fp32. */
+GDN_API int gdn_recurrent_step_ex(const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, const float* state_in, float* state_out,
+                          void* out, int B, int H, int dk, int dv, int gate_mode,
+                          int io_dtype, gdn_stream_t stream);
+
+/*
+ * gdn_check -- synchronises `stream`, then reports GDN_ERR_TIMEOUT if any
+ * kernel of this library on the current device abandoned a bounded wait
+ * since the last gdn_check (and clears the record), GDN_ERR_CUDA on a CUDA
+ * error, else GDN_OK.  This is the only call that synchronises.
+ */
+GDN_API int gdn_check(gdn_stream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+GDN_API const char* gdn_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GDN_H */

@@ -1,0 +1,98 @@
+"""The C ABI on the host: the library loads, exports every declared symbol,
+and rejects invalid calls before launching anything (no GPU needed).
+
+Every call here fails validation on purpose, so no kernel is launched and
+no fake pointer is ever dereferenced.
+"""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+import gated_delta_rule_77_b200 as gdn
+
+HEADER = Path(__file__).resolve().parent.parent / "include" / "gdn.h"
+A = 0x10000          # 16-byte aligned fake device addresses, spaced apart
+MB = 1 << 20
+
+
+def declared_symbols():
+    text = HEADER.read_text()
+    return sorted(set(re.findall(r"GDN_API\s+[\w\s\*]+?\b(gdn_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_delta_rule_77_b200 import build
+    build.build()
+    return gdn.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert set(names) == set(gdn.SYMBOLS)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code, name in [(0, "GDN_OK"), (-1, "GDN_ERR_INVALID_ARG"), (-2, "GDN_ERR_UNSUPPORTED"),
+                       (-3, "GDN_ERR_MISALIGNED"), (-4, "GDN_ERR_CUDA"), (-5, "GDN_ERR_NOMEM"),
+                       (-6, "GDN_ERR_TIMEOUT"), (7, "GDN_ERR_UNKNOWN")]:
+        assert gdn.status_string(code) == name
+
+
+def _prefill(lib, q=A, k=A + 64 * MB, v=A + 128 * MB, g=A + 192 * MB, beta=A + 256 * MB,
+             s_in=A + 320 * MB, out=A + 384 * MB, s_out=A + 448 * MB, B=1, T=16, H=1, dk=128, dv=128,
+             gate=0, io=0, chunk=0):
+    c = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    return lib.gdn_chunk_fwd_ex(c(q), c(k), c(v), c(g), c(beta), c(s_in), c(out), c(s_out),
+                                B, T, H, dk, dv, gate, io, chunk, None)
+
+
+def _step(lib, q=A, k=A + 64 * MB, v=A + 128 * MB, g=A + 192 * MB, beta=A + 256 * MB,
+          s_in=A + 320 * MB, s_out=A + 320 * MB, out=A + 448 * MB, B=1, H=1, dk=128, dv=128, gate=1,
+          io=0):
+    c = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    return lib.gdn_recurrent_step_ex(c(q), c(k), c(v), c(g), c(beta), c(s_in), c(s_out), c(out),
+                                     B, H, dk, dv, gate, io, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(k=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(v=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(g=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(beta=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(out=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(B=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(H=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(T=-1), gdn.GDN_ERR_INVALID_ARG),
+    (dict(gate=2), gdn.GDN_ERR_INVALID_ARG),
+    (dict(io=5), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dk=96), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dv=32), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(chunk=48), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(io=1, chunk=64), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(q=A + 8), gdn.GDN_ERR_MISALIGNED),
+    (dict(s_out=A + 448 * MB + 4), gdn.GDN_ERR_MISALIGNED),
+    (dict(out=A + 16), gdn.GDN_ERR_INVALID_ARG),                     # out overlaps q
+    (dict(out=A + 320 * MB), gdn.GDN_ERR_INVALID_ARG),               # out overlaps state_in
+    (dict(s_out=A + 128 * MB), gdn.GDN_ERR_INVALID_ARG),             # state_out overlaps v
+    (dict(s_out=A + 320 * MB + 4096), gdn.GDN_ERR_INVALID_ARG),      # partial state overlap
+])
+def test_prefill_rejects(lib, kw, status):
+    assert _prefill(lib, **kw) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(s_in=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(s_out=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(out=A + 320 * MB), gdn.GDN_ERR_INVALID_ARG),               # out overlaps state
+    (dict(dk=100), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(gate=-1), gdn.GDN_ERR_INVALID_ARG),
+    (dict(v=A + 128 * MB + 2), gdn.GDN_ERR_MISALIGNED),
+])
+def test_step_rejects(lib, kw, status):
+    assert _step(lib, **kw) == status
