@@ -99,12 +99,12 @@ def chunk_fwd(q, k, v, g, beta, state_in=None, *, out=None, state_out=None,
               return_state: bool = True, chunk_size: int = 0, stream=None):
     """Chunkwise prefill.  q, k [B,T,H,dk]; v [B,T,H,dv]; g [B,T,H] or
     [B,T,H,dk] fp32; beta [B,T,H] fp32; state_in [B,H,dk,dv] fp32 or None.
-    Returns (out [B,T,H,dv] in v's dtype, final state or None)."""
+    Returns (out [B,T,H,dv] fp32, final state or None)."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     gate = GATE_CHANNEL if g.dim() == 4 else GATE_SCALAR
     if out is None:
-        out = torch.empty(B, T, H, dv, dtype=v.dtype, device=v.device)
+        out = torch.empty(B, T, H, dv, dtype=torch.float32, device=v.device)
     if state_out is None and return_state:
         state_out = torch.empty(B, H, dk, dv, dtype=torch.float32, device=v.device)
     _check_cuda(q, k, v, g, beta, state_in, out, state_out)

@@ -1,11 +1,753 @@
-// chunk_sm100.cu -- placeholder until the tensor-core chunk kernel lands.
+// chunk_sm100.cu -- chunkwise-parallel prefill of the Gated DeltaNet
+// recurrence on Blackwell tensor cores (tcgen05 + TMEM, operands fed by TMA).
+//
+// Method: Atomic-GDN2 model card, section 2.1 "Gated DeltaNet-2":
+//     S_t = (I - b_t k_t k_t^T) Diag(a_t) S_{t-1} + b_t k_t v_t^T,  o_t = S_t^T q_t,
+//     a_t = exp(g_t), g scalar per head or one value per key channel.
+// The chunkwise mode ("Gated DeltaNet" entity trail, finding of 2026-07-29)
+// computes the same mathematics with dense products inside a chunk.
+//
+// Chunk algebra (derived by unrolling the recurrence over a chunk of C = 64
+// tokens with initial state S; G_r = cumulative sum of g inside the chunk,
+// a scalar or a dk-vector; E_r = exp(G_r); u_r = b_r (v_r - S'_r^T k_r) is
+// the corrected value the delta rule writes at token r):
+//   A_rj = b_r k_r^T Diag(exp(G_r - G_j)) k_j          (j < r)
+//   T    = (I + A)^{-1},  T' = T Diag(b)                (unit lower triangular)
+//   W    = T' (K * E),    U = T' V - W S
+//   P_rj = q_r^T Diag(exp(G_r - G_j)) k_j              (j <= r)
+//   O    = (Q * E) S + P U
+//   S   <- Diag(E_last) S + (K * D)^T U,  D_r = exp(G_last - G_r)
+// The state S stays fp32 in registers across chunks.
+//
+// Per-channel decay inside A and P.  exp(G_r - G_j) per key channel is
+// factored through a reference token m at the centre of a 32-token block:
+// exp(G_r - G_m) * exp(G_m - G_j).  With g >= -5 (the gate domain of the
+// model card, section 2.1, g = -min(softplus(.), 160/bs2), bs2 = 32) every
+// factor lies within exp(+-80), inside fp32 and bf16 range, so A and P come
+// out of plain matrix products (K * F)(K / F)^T.  Rows of block 0 (tokens
+// 0-31) use reference 15, rows of block 1 use reference 47; both products
+// share the left operand [K * F ; Q * F] and differ in the right one.
+// The scalar gate needs no factorisation: exp(G_r - G_j) is applied exactly
+// to K K^T and Q K^T after the product, for any g <= 0.
+//
+// Precision.  The output o is a small difference of much larger terms
+// ((Q*E) S and P U; on the source's workloads max|o| ~ 9 rms(o)), so plain
+// bf16 operands would cost more than a 2e-2 * rms(o) error budget.  The
+// model card's kernel computes in "bf16x3" (section 3.2 Precision, section 5
+// compute mode): a value is carried as a bf16 hi part plus a bf16 lo part
+// and a product takes three bf16 MMAs (hi*hi + hi*lo + lo*hi).  Here that is
+// applied to the operands that need it: the factored operands of A and P,
+// T', P, U and K*D.  The state copy S, W and Q*E, whose magnitudes stay
+// moderate, are fp16 operands (4x finer than bf16).  Accumulation is fp32 in
+// TMEM and the output is written in fp32.
+//
+// Products (all 128-row tcgen05.mma; transposed forms put the 128-wide key or
+// value dimension on M):
+//   X   = [K*F;Q*F] (K/F)^T        M = 2C rows, N = 32 / 64 -> A and P (raw)
+//   W^T = (K*E)^T T'^T             M = dk, N = C, K = C
+//   U^T = V^T T'^T - S^T W^T       M = dv, N = C, K = C then dk
+//   O^T = S^T (Q*E)^T + U^T P^T    M = dv, N = C
+//   SN  = (K*D)^T U                M = dk, N = dv, K = C
+//
+// This version runs the phases of a chunk one after another in one CTA per
+// (batch, head); the next chunk's TMA loads overlap the end of the chunk.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "gdn_internal.cuh"
+#include "sm100_util.cuh"
 
 namespace gdn {
 
 __device__ unsigned int g_status_word = 0;
 
-cudaError_t launch_chunk_sm100(const Problem&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+using namespace sm100;
+
+constexpr int C = 64;      // chunk length
+constexpr int D = 128;     // dk = dv
+constexpr int NT = 256;    // threads per CTA
+
+// ---- shared-memory map (byte offsets from a 1024-aligned base) -------------
+// R_IN: raw K and Q of the chunk (TMA, bf16, 128B-swizzled rows):
+//   [half][K rows 0-63 | Q rows 0-63][128 B].  Dead once the derived tiles
+//   are built; then holds T' (hi, lo), the solve scratch and W^T.
+constexpr uint32_t R_IN = 0;                 // 32 KB
+constexpr uint32_t OFF_TH = R_IN;            //   8 KB T' hi [64 r][64 m]
+constexpr uint32_t OFF_TL = R_IN + 8192;     //   8 KB T' lo
+constexpr uint32_t OFF_Y = R_IN + 16384;     //   3 KB solve scratch
+constexpr uint32_t OFF_WT = R_IN + 16384;    //   16 KB W^T fp16 [128 i][64 r] (after solve)
+constexpr uint32_t R_V = 32768;              // 16 KB raw V [half][64][128 B]
+constexpr uint32_t R_S = 49152;              // 32 KB S fp16 [j half][128 i][64 j]
+constexpr uint32_t R_X = 81920;              // 112 KB, two uses per chunk:
+//  (a) X operands (per-channel gate), bf16 hi / lo:
+constexpr uint32_t OFF_AH = R_X;             //   32 KB [half][K*F 64 | Q*F 64][128 B]
+constexpr uint32_t OFF_AL = R_X + 32768;     //   32 KB
+constexpr uint32_t OFF_C0H = R_X + 65536;    //   8 KB [half][32][128 B]  K/F (ref 15)
+constexpr uint32_t OFF_C0L = R_X + 73728;    //   8 KB
+constexpr uint32_t OFF_C1H = R_X + 81920;    //   16 KB [half][64][128 B] K*exp(G_47 - G)
+constexpr uint32_t OFF_C1L = R_X + 98304;    //   16 KB
+//  (b) after X: derived tiles, P, solve input, U
+constexpr uint32_t OFF_KE = R_X;             //   16 KB K*E bf16  [half][64 r][128 B]
+constexpr uint32_t OFF_QE = R_X + 16384;     //   16 KB Q*E fp16
+constexpr uint32_t OFF_KDH = R_X + 32768;    //   16 KB K*D bf16 hi
+constexpr uint32_t OFF_KDL = R_X + 49152;    //   16 KB K*D bf16 lo
+constexpr uint32_t OFF_PH = R_X + 65536;     //   8 KB P hi [64 r][64 m]
+constexpr uint32_t OFF_PL = R_X + 73728;     //   8 KB P lo
+constexpr uint32_t OFF_A = R_X + 81920;      //   16 KB A fp32 [64][64]
+constexpr uint32_t OFF_TF = R_X + 98304;     //   16 KB T fp32 [64][64]
+constexpr uint32_t OFF_UH = R_X + 81920;     //   16 KB U^T hi [128 j][64 r] (after solve)
+constexpr uint32_t OFF_UL = R_X + 98304;     //   16 KB U^T lo
+constexpr uint32_t R_SMALL = R_X + 114688;
+constexpr uint32_t SM_GAM = R_SMALL;          // 64 f32: scalar G
+constexpr uint32_t SM_BETA = SM_GAM + 256;    // 64 f32
+constexpr uint32_t SM_REF0 = SM_BETA + 256;   // 128 f32: G at token 15 (channel)
+constexpr uint32_t SM_REF1 = SM_REF0 + 512;   // 128 f32: G at token 47
+constexpr uint32_t SM_LAST = SM_REF1 + 512;   // 128 f32: G at token 63
+constexpr uint32_t SM_BAR = SM_LAST + 512;    // 2 mbarriers
+constexpr uint32_t SM_TMEM = SM_BAR + 16;     // TMEM base address
+constexpr uint32_t SMEM_USED = SM_TMEM + 16;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
+
+// ---- TMEM columns (512 allocated) -------------------------------------------
+constexpr uint32_t TM_X = 0;      // X: 128 rows (A rows 0-63, P rows 64-127), N <= 96
+constexpr uint32_t TM_WT = 128;   // W^T: 128 x 64
+constexpr uint32_t TM_UT = 192;   // U^T: 128 x 64
+constexpr uint32_t TM_OT = 256;   // O^T: 128 x 64
+constexpr uint32_t TM_SN = 384;   // SN:  128 x 128
+
+struct Params {
+    const float* g;            // [B, T, H] or [B, T, H, D]
+    const float* beta;         // [B, T, H]
+    const float* state_in;     // [B, H, D, D] or null
+    float* state_out;          // [B, H, D, D] or null
+    float* out;                // [B, T, H, D] fp32
+    int T, H;
+};
+
+// fp32 64x64 matrix in shared memory, float4 groups xor-swizzled by row so
+// that row-parallel and column-parallel accesses both avoid bank conflicts.
+__device__ __forceinline__ uint32_t fidx(int r, int m) {
+    return static_cast<uint32_t>(r * 64 + ((((m >> 2) ^ r) & 15) << 2) + (m & 3));
+}
+
+// Eight fp32 values -> a 16-byte bf16 chunk (hi) and the bf16 rounding of the
+// remainder (lo), so that hi + lo reproduces each value to ~2^-16.
+__device__ __forceinline__ void store_split(uint8_t* hi_dst, uint8_t* lo_dst, const float* v) {
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        hi[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+        lo[e] = pack_bf16(v[2 * e] - bf16_lo(hi[e]), v[2 * e + 1] - bf16_hi(hi[e]));
+    }
+    *reinterpret_cast<uint4*>(hi_dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(lo_dst) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+}
+
+__device__ __forceinline__ void store_bf16x8(uint8_t* dst, const float* v) {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                                                pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+}
+
+__device__ __forceinline__ void store_f16x8(uint8_t* dst, const float* v) {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(pack_f16(v[0], v[1]), pack_f16(v[2], v[3]),
+                                                pack_f16(v[4], v[5]), pack_f16(v[6], v[7]));
+}
+
+__device__ __forceinline__ void load_bf16x8(const uint8_t* src, float* v) {
+    const uint4 w = *reinterpret_cast<const uint4*>(src);
+    const uint32_t x[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        v[2 * e] = bf16_lo(x[e]);
+        v[2 * e + 1] = bf16_hi(x[e]);
+    }
+}
+
+template <bool CHANNEL>
+__global__ void __launch_bounds__(NT, 1)
+chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const Params p)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(smem);
+    float* sGam = reinterpret_cast<float*>(smem + SM_GAM);
+    float* sBeta = reinterpret_cast<float*>(smem + SM_BETA);
+    float* sRef0 = reinterpret_cast<float*>(smem + SM_REF0);
+    float* sRef1 = reinterpret_cast<float*>(smem + SM_REF1);
+    float* sLast = reinterpret_cast<float*>(smem + SM_LAST);
+    float* sA = reinterpret_cast<float*>(smem + OFF_A);
+    float* sTf = reinterpret_cast<float*>(smem + OFF_TF);
+    float* sY = reinterpret_cast<float*>(smem + OFF_Y);
+    const uint32_t bar_tma = sbase + SM_BAR;
+    const uint32_t bar_mma = sbase + SM_BAR + 8;
+    uint32_t* sTmemBase = reinterpret_cast<uint32_t*>(smem + SM_TMEM);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int quad = warp & 3;      // TMEM lane quarter of this warp
+    const int half = warp >> 2;     // which half of the columns this warp takes
+    const int T = p.T;
+    const int H = p.H;
+    const int h = blockIdx.x % H;
+    const int b = blockIdx.x / H;
+    const int nchunks = (T + C - 1) / C;
+
+    // Element ownership for the gate prep and tile building: 16 channel
+    // chunks of 8 (ck) x 16 token groups of 4 (tg); the 16 token groups of a
+    // channel chunk sit in one half-warp so the cumulative sum is a shuffle scan.
+    const int ck = 2 * warp + (lane >> 4);
+    const int tg = lane & 15;
+    const int ckh = ck >> 3;       // 64-channel half of the tile
+    const int ckc = ck & 7;        // 16-byte chunk within a 128-byte row
+
+    if (tid == 0) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+        mbar_init(bar_tma, 1);
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(sbase + SM_TMEM, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *sTmemBase;
+
+    // ---- resident fp32 state: thread owns row i, columns [64*half, +64) ------
+    const int srow = quad * 32 + lane;
+    const int scol = half * 64;
+    float s[64];
+    const long sb = ((long)b * H + h) * (long)D * D;
+    if (p.state_in) {
+        const float4* src = reinterpret_cast<const float4*>(p.state_in + sb + (long)srow * D + scol);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            float4 t = src[c];
+            s[4 * c] = t.x; s[4 * c + 1] = t.y; s[4 * c + 2] = t.z; s[4 * c + 3] = t.w;
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) s[c] = 0.f;
+    }
+    // fp16 copy: MN-major tile [j half][128 i rows][64 j] (row i, 8 chunks).
+    auto write_state_f16 = [&]() {
+        uint8_t* dst = smem + R_S + half * 16384;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) store_f16x8(dst + swz(srow, c), &s[8 * c]);
+    };
+    write_state_f16();
+
+    auto issue_loads = [&](int chunk) {
+        const int t0 = chunk * C;
+        mbar_expect_tx(bar_tma, 3 * 16384);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            tma_load_4d(sbase + R_IN + hf * 16384, &tm_k, hf * 64, h, t0, b, bar_tma);
+            tma_load_4d(sbase + R_IN + hf * 16384 + 8192, &tm_q, hf * 64, h, t0, b, bar_tma);
+            tma_load_4d(sbase + R_V + hf * 8192, &tm_v, hf * 64, h, t0, b, bar_tma);
+        }
+    };
+
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) issue_loads(0);
+    int tma_waited = -1;   // last chunk whose loads were waited for
+
+    uint32_t mma_phase = 0;
+    bool ok = true;
+    auto mma_sync = [&]() {   // all threads wait for the last commit
+        ok = ok && mbar_wait(bar_mma, mma_phase, &g_status_word);
+        mma_phase ^= 1;
+        tc_fence_after();
+    };
+
+    for (int ci = 0; ci < nchunks; ++ci) {
+        const int t0 = ci * C;
+        const long tk0 = ((long)b * T + t0) * H + h;     // flat (b, t0, h)
+
+        // ---------------------------------------------------- gate prep --------
+        // Per-channel: this thread's 4 tokens x 8 channels of g, cumulated over
+        // the chunk (registers).  Scalar: warp 0 scans the 64 values.
+        float gam[4][8];
+        if (CHANNEL) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int t = t0 + 4 * tg + u;
+                if (t < T) {
+                    const float4* src = reinterpret_cast<const float4*>(
+                        p.g + (tk0 + (long)(4 * tg + u) * H) * D + 8 * ck);
+                    const float4 a = src[0], c = src[1];
+                    gam[u][0] = a.x; gam[u][1] = a.y; gam[u][2] = a.z; gam[u][3] = a.w;
+                    gam[u][4] = c.x; gam[u][5] = c.y; gam[u][6] = c.z; gam[u][7] = c.w;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) gam[u][e] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                gam[1][e] += gam[0][e];
+                gam[2][e] += gam[1][e];
+                gam[3][e] += gam[2][e];
+                float tot = gam[3][e];           // inclusive scan of group totals
+#pragma unroll
+                for (int o = 1; o < 16; o <<= 1) {
+                    const float x = __shfl_up_sync(0xffffffffu, tot, o, 16);
+                    if (tg >= o) tot += x;
+                }
+                const float excl = tot - gam[3][e];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) gam[u][e] += excl;
+            }
+            if (tg == 3 || tg == 11 || tg == 15) {
+                float* dst = tg == 3 ? sRef0 : (tg == 11 ? sRef1 : sLast);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) dst[8 * ck + e] = gam[3][e];
+            }
+        }
+        if (warp == 0) {
+            float b0 = 0.f, b1 = 0.f, g0 = 0.f, g1 = 0.f;
+            if (t0 + lane < T) {
+                b0 = p.beta[tk0 + (long)lane * H];
+                if (!CHANNEL) g0 = p.g[tk0 + (long)lane * H];
+            }
+            if (t0 + 32 + lane < T) {
+                b1 = p.beta[tk0 + (long)(32 + lane) * H];
+                if (!CHANNEL) g1 = p.g[tk0 + (long)(32 + lane) * H];
+            }
+            sBeta[lane] = b0;
+            sBeta[32 + lane] = b1;
+            if (!CHANNEL) {
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float x0 = __shfl_up_sync(0xffffffffu, g0, o);
+                    const float x1 = __shfl_up_sync(0xffffffffu, g1, o);
+                    if (lane >= o) { g0 += x0; g1 += x1; }
+                }
+                g1 += __shfl_sync(0xffffffffu, g0, 31);
+                sGam[lane] = g0;
+                sGam[32 + lane] = g1;
+            }
+        }
+        ok = ok && mbar_wait(bar_tma, ci & 1, &g_status_word);
+        tma_waited = ci;
+        if (__syncthreads_or(!ok)) break;
+
+        // ---------------------------------------------------- X = raw A and P --
+        if (CHANNEL) {
+            // Factored operands, bf16 hi + lo (see header).
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int r = 4 * tg + u;
+                const float* ref = r < 32 ? sRef0 : sRef1;
+                float kf[8], qf[8];
+                load_bf16x8(smem + R_IN + ckh * 16384 + swz(r, ckc), kf);
+                load_bf16x8(smem + R_IN + ckh * 16384 + 8192 + swz(r, ckc), qf);
+                float kr[8], qr[8], kc[8], kc1[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float x = gam[u][e] - ref[8 * ck + e];
+                    const float F = __expf(x);
+                    const float Fi = __expf(-x);
+                    kr[e] = kf[e] * F;
+                    qr[e] = qf[e] * F;
+                    kc[e] = kf[e] * Fi;
+                    kc1[e] = r < 32 ? kf[e] * __expf(sRef1[8 * ck + e] - gam[u][e]) : kc[e];
+                }
+                const uint32_t o128 = ckh * 16384 + swz(r, ckc);
+                const uint32_t o128q = ckh * 16384 + swz(64 + r, ckc);
+                store_split(smem + OFF_AH + o128, smem + OFF_AL + o128, kr);
+                store_split(smem + OFF_AH + o128q, smem + OFF_AL + o128q, qr);
+                if (r < 32) {
+                    const uint32_t o32 = ckh * 4096 + swz(r, ckc);
+                    store_split(smem + OFF_C0H + o32, smem + OFF_C0L + o32, kc);
+                }
+                const uint32_t o64 = ckh * 8192 + swz(r, ckc);
+                store_split(smem + OFF_C1H + o64, smem + OFF_C1L + o64, kc1);
+            }
+            fence_async_smem();
+            __syncthreads();
+        }
+        if (tid == 0) {
+            tc_fence_after();
+            if (CHANNEL) {
+                const uint32_t id0 = idesc_bf16(128, 32, false, false);
+                const uint32_t id1 = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t ka = (ks >> 2) * 16384 + (ks & 3) * 32;
+                    const uint32_t k0 = (ks >> 2) * 4096 + (ks & 3) * 32;
+                    const uint32_t k1 = (ks >> 2) * 8192 + (ks & 3) * 32;
+                    const uint64_t ah = sdesc_sw128(sbase + OFF_AH + ka, 16, 1024);
+                    const uint64_t al = sdesc_sw128(sbase + OFF_AL + ka, 16, 1024);
+                    const uint64_t b0h = sdesc_sw128(sbase + OFF_C0H + k0, 16, 1024);
+                    const uint64_t b0l = sdesc_sw128(sbase + OFF_C0L + k0, 16, 1024);
+                    const uint64_t b1h = sdesc_sw128(sbase + OFF_C1H + k1, 16, 1024);
+                    const uint64_t b1l = sdesc_sw128(sbase + OFF_C1L + k1, 16, 1024);
+                    mma_bf16(tmem + TM_X, ah, b0h, id0, ks > 0);
+                    mma_bf16(tmem + TM_X, ah, b0l, id0, 1);
+                    mma_bf16(tmem + TM_X, al, b0h, id0, 1);
+                    mma_bf16(tmem + TM_X + 32, ah, b1h, id1, ks > 0);
+                    mma_bf16(tmem + TM_X + 32, ah, b1l, id1, 1);
+                    mma_bf16(tmem + TM_X + 32, al, b1h, id1, 1);
+                }
+            } else {
+                // Exact: bf16 inputs, fp32 accumulation.
+                const uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint64_t a = sdesc_sw128(sbase + R_IN + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                    mma_bf16(tmem + TM_X, a, a, id, ks > 0);
+                }
+            }
+            mma_commit(bar_mma);
+        }
+        mma_sync();
+        if (__syncthreads_or(!ok)) break;
+
+        // ------------------------------- derived tiles; A and P from X ----------
+        // K*E (bf16), Q*E (fp16), K*D (bf16 hi + lo) into the freed X region.
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int r = 4 * tg + u;
+            float kf[8], qf[8], ke[8], qe[8], kd[8];
+            load_bf16x8(smem + R_IN + ckh * 16384 + swz(r, ckc), kf);
+            load_bf16x8(smem + R_IN + ckh * 16384 + 8192 + swz(r, ckc), qf);
+            if (CHANNEL) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float E = __expf(gam[u][e]);
+                    const float Dd = __expf(sLast[8 * ck + e] - gam[u][e]);
+                    ke[e] = kf[e] * E;
+                    qe[e] = qf[e] * E;
+                    kd[e] = kf[e] * Dd;
+                }
+            } else {
+                const float E = __expf(sGam[r]);
+                const float Dd = __expf(sGam[C - 1] - sGam[r]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    ke[e] = kf[e] * E;
+                    qe[e] = qf[e] * E;
+                    kd[e] = kf[e] * Dd;
+                }
+            }
+            const uint32_t o64 = ckh * 8192 + swz(r, ckc);
+            store_bf16x8(smem + OFF_KE + o64, ke);
+            store_f16x8(smem + OFF_QE + o64, qe);
+            store_split(smem + OFF_KDH + o64, smem + OFF_KDL + o64, kd);
+        }
+        if (warp < 4) {
+            const int L = warp * 32 + lane;       // TMEM lane = row of X
+            const bool is_p = L >= 64;
+            const int r = L & 63;
+            float x[64];
+            const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+            if (CHANNEL) {
+                if (r < 32) {
+                    tmem_ld32(lane_base + TM_X, *reinterpret_cast<float(*)[32]>(&x[0]));
+#pragma unroll
+                    for (int j = 32; j < 64; ++j) x[j] = 0.f;
+                } else {
+                    tmem_ld32(lane_base + TM_X + 32, *reinterpret_cast<float(*)[32]>(&x[0]));
+                    tmem_ld32(lane_base + TM_X + 64, *reinterpret_cast<float(*)[32]>(&x[32]));
+                }
+            } else {
+                tmem_ld32(lane_base + TM_X, *reinterpret_cast<float(*)[32]>(&x[0]));
+                tmem_ld32(lane_base + TM_X + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
+            }
+            tmem_wait_ld();
+            const float br = sBeta[r];
+            const float Gr = CHANNEL ? 0.f : sGam[r];
+            if (!is_p) {
+#pragma unroll
+                for (int j4 = 0; j4 < 16; ++j4) {
+                    float4 a4;
+                    float* a = &a4.x;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = 4 * j4 + e;
+                        float val = 0.f;
+                        if (j < r) val = br * x[j] * (CHANNEL ? 1.f : __expf(Gr - sGam[j]));
+                        a[e] = val;
+                    }
+                    *reinterpret_cast<float4*>(&sA[fidx(r, 4 * j4)]) = a4;
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    float pv[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int j = 8 * c + e;
+                        float val = 0.f;
+                        if (j <= r) val = x[j] * (CHANNEL ? 1.f : __expf(Gr - sGam[j]));
+                        pv[e] = val;
+                    }
+                    store_split(smem + OFF_PH + swz(r, c), smem + OFF_PL + swz(r, c), pv);
+                }
+            }
+        }
+        // Decay of the state over the whole chunk, per key row (own row).
+        const float e_last = __expf(CHANNEL ? sLast[srow] : sGam[C - 1]);
+        tc_fence_before();
+        __syncthreads();
+
+        // ---------------------------------------------------- T = (I + A)^{-1} --
+        // Diagonal 16x16 blocks by forward substitution (warp b, lane = column).
+        if (warp < 4 && lane < 16) {
+            const int o = warp * 16;
+            float t[16];
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) {
+                float acc = 0.f;
+#pragma unroll
+                for (int m = 0; m < rr; ++m) acc = fmaf(sA[fidx(o + rr, o + m)], t[m], acc);
+                t[rr] = (rr == lane) ? 1.f : -acc;
+            }
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) sTf[fidx(o + rr, o + lane)] = t[rr];
+        }
+        __syncthreads();
+        // Off-diagonal blocks: T_ab = -T_aa * sum_{m=b}^{a-1} A_am T_mb, by
+        // increasing distance a - b.
+#pragma unroll 1
+        for (int d = 1; d < 4; ++d) {
+            const int nel = (4 - d) * 256;
+            for (int e = tid; e < nel; e += NT) {
+                const int blk = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+                const int a = blk + d, bb = blk;
+                float acc = 0.f;
+                for (int m = 16 * bb; m < 16 * a; ++m)
+                    acc = fmaf(sA[fidx(16 * a + rr, m)], sTf[fidx(m, 16 * bb + cc)], acc);
+                sY[e] = acc;
+            }
+            __syncthreads();
+            for (int e = tid; e < nel; e += NT) {
+                const int blk = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+                const int a = blk + d, bb = blk;
+                float acc = 0.f;
+#pragma unroll
+                for (int n = 0; n < 16; ++n)
+                    acc = fmaf(sTf[fidx(16 * a + rr, 16 * a + n)], sY[(blk << 8) + (n << 4) + cc], acc);
+                sTf[fidx(16 * a + rr, 16 * bb + cc)] = -acc;
+            }
+            __syncthreads();
+        }
+        // T' = T Diag(beta) -> bf16 hi + lo, K-major [64 r][64 m].
+        for (int e = tid; e < 512; e += NT) {
+            const int r = e >> 3, c = e & 7;
+            float tv[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int m = 8 * c + q;
+                tv[q] = (m <= r) ? sTf[fidx(r, m)] * sBeta[m] : 0.f;
+            }
+            store_split(smem + OFF_TH + swz(r, c), smem + OFF_TL + swz(r, c), tv);
+        }
+        fence_async_smem();
+        __syncthreads();
+
+        // ---------------------------------------------------- W^T and T'V ------
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id = idesc_bf16(128, 64, true, false);
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t tb = part ? OFF_TL : OFF_TH;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t bt = sdesc_sw128(sbase + tb + ks * 32, 16, 1024);
+                    const uint32_t acc = (part | ks) != 0;
+                    mma_bf16(tmem + TM_WT, sdesc_sw128(sbase + OFF_KE + ks * 2048, 8192, 1024), bt, id, acc);
+                    mma_bf16(tmem + TM_UT, sdesc_sw128(sbase + R_V + ks * 2048, 8192, 1024), bt, id, acc);
+                }
+            }
+            mma_commit(bar_mma);
+        }
+        mma_sync();
+        if (__syncthreads_or(!ok)) break;
+
+        // W^T -> fp16, MN-major B operand [128 i][64 r].  Thread: row i, 32 r.
+        {
+            float w[32];
+            tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + TM_WT + half * 32, w);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) store_f16x8(smem + OFF_WT + swz(srow, half * 4 + c), &w[8 * c]);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ------------------------------- U^T -= S^T W^T ; O^T = S^T (QE)^T ------
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id_u = idesc_f16(128, 64, true, true, true);
+            const uint32_t id_o = idesc_f16(128, 64, true, false);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t a = sdesc_sw128(sbase + R_S + ks * 2048, 16384, 1024);
+                mma_bf16(tmem + TM_UT, a, sdesc_sw128(sbase + OFF_WT + ks * 2048, 8192, 1024), id_u, 1);
+                const uint64_t bq = sdesc_sw128(sbase + OFF_QE + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+                mma_bf16(tmem + TM_OT, a, bq, id_o, ks > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        mma_sync();
+        if (__syncthreads_or(!ok)) break;
+        // Raw K, Q, V, T' and W^T are no longer read: prefetch the next chunk.
+        if (tid == 0 && ci + 1 < nchunks) issue_loads(ci + 1);
+
+        // U^T -> bf16 hi + lo [128 j][64 r] (K-major B of SN, K-major A of O^T).
+        {
+            float u[32];
+            tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + TM_UT + half * 32, u);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                store_split(smem + OFF_UH + swz(srow, half * 4 + c), smem + OFF_UL + swz(srow, half * 4 + c),
+                            &u[8 * c]);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ------------------------------- SN = (K D)^T U ; O^T += U^T P^T --------
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id_s = idesc_bf16(128, 128, true, false);
+            const uint32_t id_o = idesc_bf16(128, 64, false, false);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t kdh = sdesc_sw128(sbase + OFF_KDH + ks * 2048, 8192, 1024);
+                const uint64_t kdl = sdesc_sw128(sbase + OFF_KDL + ks * 2048, 8192, 1024);
+                const uint64_t uh = sdesc_sw128(sbase + OFF_UH + ks * 32, 16, 1024);
+                const uint64_t ul = sdesc_sw128(sbase + OFF_UL + ks * 32, 16, 1024);
+                const uint64_t ph = sdesc_sw128(sbase + OFF_PH + ks * 32, 16, 1024);
+                const uint64_t pl = sdesc_sw128(sbase + OFF_PL + ks * 32, 16, 1024);
+                mma_bf16(tmem + TM_SN, kdh, uh, id_s, ks > 0);
+                mma_bf16(tmem + TM_SN, kdh, ul, id_s, 1);
+                mma_bf16(tmem + TM_SN, kdl, uh, id_s, 1);
+                mma_bf16(tmem + TM_OT, uh, ph, id_o, 1);
+                mma_bf16(tmem + TM_OT, uh, pl, id_o, 1);
+                mma_bf16(tmem + TM_OT, ul, ph, id_o, 1);
+            }
+            mma_commit(bar_mma);
+        }
+        mma_sync();
+        if (__syncthreads_or(!ok)) break;
+
+        // ---------------------------------------------------- state and output --
+        {
+            const uint32_t lb = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+            float sn[32];
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                tmem_ld32(lb + TM_SN + half * 64 + part * 32, sn);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; ++c) s[part * 32 + c] = fmaf(e_last, s[part * 32 + c], sn[c]);
+            }
+            write_state_f16();
+            float o[32];
+            tmem_ld32(lb + TM_OT + half * 32, o);
+            tmem_wait_ld();
+            const int j = srow;
+            const int nvalid = min(C, T - t0) - half * 32;
+#pragma unroll
+            for (int r = 0; r < 32; ++r) {
+                if (r < nvalid) p.out[(tk0 + (long)(half * 32 + r) * H) * D + j] = o[r];
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+    }
+
+    if (!ok && tid == 0) {
+        // Abandoned: drain what this CTA still has in flight (bounded) before
+        // its shared memory and TMEM go away.
+        if (tma_waited + 1 < nchunks) mbar_wait(bar_tma, (tma_waited + 1) & 1, &g_status_word);
+        mma_commit(bar_mma);
+        mbar_wait(bar_mma, mma_phase, &g_status_word);
+    }
+    if (ok && p.state_out) {
+        float4* dst = reinterpret_cast<float4*>(p.state_out + sb + (long)srow * D + scol);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) dst[c] = make_float4(s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---- host side ---------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 4-D map over a bf16 [B, T, H, 128] tensor; box {64 channels, 1, 64 tokens, 1},
+// 128-byte swizzle (the operand layout of the MMAs).
+bool make_map(CUtensorMap* map, const void* base, int H, int T, int B) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)C, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <bool CHANNEL>
+cudaError_t launch(const Problem& p, cudaStream_t stream) {
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(chunk_fwd_kernel<CHANNEL>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, p.q, p.H, p.T, p.B) || !make_map(&mk, p.k, p.H, p.T, p.B) ||
+        !make_map(&mv, p.v, p.H, p.T, p.B))
+        return cudaErrorInvalidValue;
+    Params prm{p.g, p.beta, p.state_in, p.state_out, static_cast<float*>(p.out), p.T, p.H};
+    chunk_fwd_kernel<CHANNEL><<<p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, prm);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_sm100(const Problem& p, cudaStream_t stream) {
+    if (p.io_f32 || !p.out_f32 || p.dk != D || p.dv != D) return cudaErrorNotSupported;
+    return p.per_channel ? launch<true>(p, stream) : launch<false>(p, stream);
+}
 
 cudaError_t read_and_clear_status(unsigned int* status, cudaStream_t stream) {
     cudaError_t e = cudaStreamSynchronize(stream);

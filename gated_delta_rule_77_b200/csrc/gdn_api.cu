@@ -47,9 +47,14 @@ int validate(const void* q, const void* k, const void* v, const float* g, const 
     // Keep every element index well inside 64-bit arithmetic and the TMA
     // coordinate range.
     if (B > (1L << 20) || H > (1L << 16) || T_tokens > (1L << 30)) return GDN_ERR_UNSUPPORTED;
-    const void* ptrs[] = {q, k, v, g, beta, state_in, state_out, out};
-    for (const void* p : ptrs)
+    // Rows read or written with vector loads / TMA need 16-byte alignment; a
+    // scalar gate and beta are read one float at a time.
+    const void* ptrs16[] = {q, k, v, state_in, state_out, out,
+                            gate_mode == GDN_GATE_CHANNEL ? g : nullptr};
+    for (const void* p : ptrs16)
         if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
+    for (const void* p : {(const void*)g, (const void*)beta})
+        if (p && (reinterpret_cast<uintptr_t>(p) & 3u)) return GDN_ERR_MISALIGNED;
 
     const size_t esz = io_dtype == GDN_IO_F32 ? 4 : 2;
     const size_t tok = (size_t)B * (size_t)T_tokens * (size_t)H;
@@ -83,7 +88,7 @@ int gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* g
 {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     int rc = validate(q, k, v, g, beta, state_in, state_out, out, B, T, H, dk, dv, gate_mode,
-                      io_dtype, io_dtype == GDN_IO_F32, false);
+                      io_dtype, true, false);
     if (rc != GDN_OK) return rc;
     const bool f32 = io_dtype == GDN_IO_F32;
     if (f32) {
@@ -101,7 +106,7 @@ int gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* g
         return to_status(e);
     }
     gdn::Problem p{q, k, v, g, beta, state_in, state_out, out, B, T, H, dk, dv,
-                   gate_mode == GDN_GATE_CHANNEL, f32, f32};
+                   gate_mode == GDN_GATE_CHANNEL, f32, true};
     if (!f32 && chunk_size != 1) {
         cudaError_t e = gdn::launch_chunk_sm100(p, stream);
         if (e != cudaErrorNotSupported) return to_status(e);

@@ -82,9 +82,11 @@ recurrent_kernel(const TIN* __restrict__ q, const TIN* __restrict__ k,
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const int h = blockIdx.y;
-    const int b = blockIdx.z;
-    const int col0 = blockIdx.x * COLS + lane * VW;   // first value column of this lane
+    const int nslices = dv / COLS;
+    const int slice = blockIdx.x % nslices;
+    const int h = (blockIdx.x / nslices) % H;
+    const int b = blockIdx.x / nslices / H;
+    const int col0 = slice * COLS + lane * VW;   // first value column of this lane
     const int row0 = warp * R;                        // first key row of this warp
 
     // Resident state slice: S[row0 + r][col0 + c].
@@ -175,7 +177,7 @@ recurrent_kernel(const TIN* __restrict__ q, const TIN* __restrict__ k,
 
 template <int DK, int COLS, int NWARPS, bool CHANNEL, typename TIN, typename TOUT>
 cudaError_t launch_typed(const Problem& p, cudaStream_t stream) {
-    dim3 grid(p.dv / COLS, p.H, p.B);
+    const unsigned grid = static_cast<unsigned>(p.dv / COLS) * p.H * p.B;
     recurrent_kernel<DK, COLS, NWARPS, CHANNEL, TIN, TOUT><<<grid, NWARPS * 32, 0, stream>>>(
         static_cast<const TIN*>(p.q), static_cast<const TIN*>(p.k), static_cast<const TIN*>(p.v),
         p.g, p.beta, p.state_in, p.state_out, static_cast<TOUT*>(p.out), p.T, p.H, p.dv);

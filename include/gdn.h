@@ -23,7 +23,9 @@
  *
  * Memory and ownership
  *   Every pointer is caller-owned DEVICE memory (e.g. a torch tensor's
- *   data_ptr()), contiguous, row-major, 16-byte aligned.  The library never
+ *   data_ptr()), contiguous and row-major.  q, k, v, out, the states and a
+ *   per-channel g must be 16-byte aligned; a scalar g and beta 4-byte
+ *   aligned (else GDN_ERR_MISALIGNED).  The library never
  *   frees caller memory.  Scratch space the prefill needs is taken
  *   stream-ordered (cudaMallocAsync / cudaFreeAsync on `stream`).
  *   The recurrent state is fp32, [B, H, dk, dv], row index = key channel --
@@ -82,7 +84,10 @@ enum { GDN_IO_BF16 = 0, GDN_IO_F32 = 1 };
  *             any g <= 0.
  *   beta      [B, T, H] fp32
  *   state_in  [B, H, dk, dv] fp32, or NULL for a zero initial state
- *   out       [B, T, H, dv], same dtype as v; must not alias an input
+ *   out       [B, T, H, dv] fp32; must not alias an input.  fp32 because the
+ *             output is a small difference of larger terms: on the source's
+ *             workloads max|o| is ~9 rms(o), so bf16 rounding of o alone
+ *             would take ~90% of a 2e-2 * rms(o) error budget.
  *   state_out [B, H, dk, dv] fp32, or NULL (final state not written);
  *             state_out == state_in is allowed
  *   dk, dv    64 or 128 (else GDN_ERR_UNSUPPORTED); B, H >= 1; T >= 0.
@@ -96,9 +101,10 @@ GDN_API int gdn_chunk_fwd(const void* q, const void* k, const void* v, const flo
 
 /*
  * gdn_chunk_fwd_ex -- gdn_chunk_fwd with an explicit I/O dtype and chunk size.
- *   io_dtype   GDN_IO_BF16: q, k, v, out bf16 (tensor-core chunk path).
- *              GDN_IO_F32 : q, k, v, out fp32 (fp32 CUDA-core path, for
+ *   io_dtype   GDN_IO_BF16: q, k, v bf16 (tensor-core chunk path).
+ *              GDN_IO_F32 : q, k, v fp32 (fp32 CUDA-core path, for
  *                           tolerances tighter than bf16 operands allow).
+ *              out is fp32 in both cases.
  *   chunk_size 0 = default.  bf16: 0 or 64 = chunkwise tensor-core path
  *              (dk = dv = 128; other dims fall back to the token-serial
  *              path when chunk_size is 0), 1 = token-serial fused

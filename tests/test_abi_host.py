@@ -93,6 +93,15 @@ def test_prefill_rejects(lib, kw, status):
     (dict(dk=100), gdn.GDN_ERR_UNSUPPORTED),
     (dict(gate=-1), gdn.GDN_ERR_INVALID_ARG),
     (dict(v=A + 128 * MB + 2), gdn.GDN_ERR_MISALIGNED),
+    (dict(beta=A + 256 * MB + 2), gdn.GDN_ERR_MISALIGNED),
+    (dict(g=A + 192 * MB + 4), gdn.GDN_ERR_MISALIGNED),
 ])
 def test_step_rejects(lib, kw, status):
     assert _step(lib, **kw) == status
+
+
+def test_scalar_gate_and_beta_need_only_4_byte_alignment(lib):
+    # A per-step slice of a [steps, B, H] tensor starts at a multiple of 4 bytes.
+    # With state_in = None the call is rejected for that reason, not alignment.
+    assert _step(lib, gate=0, g=A + 192 * MB + 4, beta=A + 256 * MB + 12, s_in=None) == \
+        gdn.GDN_ERR_INVALID_ARG

@@ -1,0 +1,150 @@
+"""GPU parity of the chunkwise tensor-core prefill (gdn_chunk_fwd, bf16 I/O,
+dk = dv = 128) against the fp64 oracle.
+
+Tolerance rule: max|got - ref| <= tol * rms(ref), tol = 2e-2 for bf16 I/O.
+Full-size workloads are checked on sampled (b, h) pairs, which the oracle
+computes exactly like the full problem (pairs are independent).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synth import CONFIGS, config_inputs, prefill_inputs
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-2
+
+
+def _gpu(gdn, x, chunk_size=0, with_s0=True):
+    dev = torch.device("cuda")
+    args = [x[n].to(dev) for n in ("q", "k", "v", "g", "beta")]
+    s0 = x["s0"].to(dev) if (with_s0 and x["s0"] is not None) else None
+    out, s = gdn.chunk_fwd(*args, s0, chunk_size=chunk_size)
+    torch.cuda.synchronize()
+    return out.float().cpu(), s.cpu()
+
+
+def _ref(x, per_channel, heads=None, with_s0=True):
+    s0 = x["s0"] if with_s0 else None
+    return oracle.run(x["q"], x["k"], x["v"], x["g"], x["beta"], s0, per_channel=per_channel,
+                      heads=heads)
+
+
+def _pairs(x, heads):
+    H = x["q"].shape[2]
+    return [divmod(bh, H) for bh in heads]
+
+
+def _check_pairs(got_o, got_s, ref_o, ref_s, pairs, tol=TOL):
+    for b, h in pairs:
+        eo = oracle.rel_err(got_o[b, :, h], ref_o[b, :, h])
+        es = oracle.rel_err(got_s[b, h], ref_s[b, h])
+        assert eo <= tol and es <= tol, f"(b={b}, h={h}): out {eo:.3e} state {es:.3e}"
+
+
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 150, 256])
+def test_small_shapes(gdn, gate, T):
+    x = prefill_inputs(2, T, 3, 128, 128, gate=gate, s0_std=0.1, seed=200 + T)
+    got_o, got_s = _gpu(gdn, x)
+    ref_o, ref_s = _ref(x, gate == "channel")
+    assert oracle.rel_err(got_o, ref_o) <= TOL
+    assert oracle.rel_err(got_s, ref_s) <= TOL
+
+
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+def test_zero_initial_state_and_no_state_out(gdn, gate):
+    x = prefill_inputs(1, 200, 2, 128, 128, gate=gate, seed=210)
+    dev = torch.device("cuda")
+    out, s = gdn.chunk_fwd(*(x[n].to(dev) for n in ("q", "k", "v", "g", "beta")), None,
+                           return_state=False)
+    torch.cuda.synchronize()
+    assert s is None
+    ref_o, _ = _ref(x, gate == "channel")
+    assert oracle.rel_err(out.float().cpu(), ref_o) <= TOL
+
+
+def test_in_place_state(gdn):
+    x = prefill_inputs(2, 130, 2, 128, 128, gate="channel", s0_std=0.1, seed=211)
+    dev = torch.device("cuda")
+    st = x["s0"].to(dev).clone()
+    out, s = gdn.chunk_fwd(*(x[n].to(dev) for n in ("q", "k", "v", "g", "beta")), st, state_out=st)
+    torch.cuda.synchronize()
+    ref_o, ref_s = _ref(x, True)
+    assert s.data_ptr() == st.data_ptr()
+    assert oracle.rel_err(out.float().cpu(), ref_o) <= TOL
+    assert oracle.rel_err(st.cpu(), ref_s) <= TOL
+
+
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+def test_chunk_size_independence(gdn, gate):
+    """Chunked (C = 64) and token-serial (C = 1) agree within tol/2 of each
+    other and each within tol of the oracle."""
+    x = prefill_inputs(2, 300, 2, 128, 128, gate=gate, s0_std=0.1, seed=212)
+    o64, s64 = _gpu(gdn, x, chunk_size=64)
+    o1, s1 = _gpu(gdn, x, chunk_size=1)
+    ref_o, ref_s = _ref(x, gate == "channel")
+    assert oracle.rel_err(o64, ref_o) <= TOL and oracle.rel_err(o1, ref_o) <= TOL
+    assert oracle.rel_err(o64, o1.double()) <= TOL / 2
+    assert oracle.rel_err(s64, s1.double()) <= TOL / 2
+
+
+def test_channel_gate_equal_channels_equals_scalar(gdn):
+    x = prefill_inputs(1, 192, 2, 128, 128, gate="scalar", s0_std=0.1, seed=213)
+    xc = dict(x)
+    xc["g"] = x["g"][..., None].expand(*x["g"].shape, 128).contiguous()
+    o_s, s_s = _gpu(gdn, x)
+    o_c, s_c = _gpu(gdn, xc)
+    assert oracle.rel_err(o_c, o_s.double()) <= TOL / 2
+    assert oracle.rel_err(s_c, s_s.double()) <= TOL / 2
+
+
+def test_frozen_state_special_case(gdn):
+    """beta = 0 and g = 0: the state is unchanged and o_t = S0^T q_t."""
+    x = prefill_inputs(1, 100, 2, 128, 128, gate="channel", s0_std=0.1, seed=214)
+    x["beta"].zero_()
+    x["g"].zero_()
+    got_o, got_s = _gpu(gdn, x)
+    ref = torch.einsum("bhij,bthi->bthj", x["s0"].double(), x["q"].double())
+    assert oracle.rel_err(got_o, ref) <= TOL
+    assert oracle.rel_err(got_s, x["s0"].double()) <= 1e-2
+
+
+def test_split_sequence_carries_state(gdn):
+    x = prefill_inputs(1, 256, 2, 128, 128, gate="channel", s0_std=0.1, seed=215)
+    o_all, s_all = _gpu(gdn, x)
+    a = {n: (x[n][:, :100].contiguous() if n != "s0" else x[n]) for n in x}
+    o1, s1 = _gpu(gdn, a)
+    bpart = {n: (x[n][:, 100:].contiguous() if n != "s0" else s1) for n in x}
+    o2, s2 = _gpu(gdn, bpart)
+    assert oracle.rel_err(torch.cat([o1, o2], 1), o_all.double()) <= TOL / 2
+    assert oracle.rel_err(s2, s_all.double()) <= TOL / 2
+
+
+def test_prefill_equals_decode_steps(gdn):
+    x = prefill_inputs(2, 70, 2, 128, 128, gate="channel", s0_std=0.1, seed=216)
+    o_p, s_p = _gpu(gdn, x)
+    dev = torch.device("cuda")
+    st = x["s0"].to(dev).clone()
+    outs = []
+    for t in range(70):
+        outs.append(gdn.recurrent_step(*(x[n][:, t].contiguous().to(dev)
+                                         for n in ("q", "k", "v", "g", "beta")), st))
+    torch.cuda.synchronize()
+    o_d = torch.stack(outs, 1).cpu()
+    assert oracle.rel_err(o_p, o_d.double()) <= TOL
+    assert oracle.rel_err(s_p, st.cpu().double()) <= TOL
+
+
+@pytest.mark.parametrize("index", [2, 3])
+def test_full_config_sampled_heads(gdn, index, oracle_threads):
+    cfg = CONFIGS[index]
+    x = config_inputs(cfg)
+    got_o, got_s = _gpu(gdn, x)
+    BH = cfg.B * cfg.H
+    heads = sorted({0, BH // 3, BH // 2 + 1, BH - 1})
+    ref_o, ref_s = oracle.run(x["q"], x["k"], x["v"], x["g"], x["beta"], x["s0"],
+                              per_channel=cfg.per_channel, heads=heads, threads=oracle_threads)
+    _check_pairs(got_o, got_s, ref_o, ref_s, _pairs(x, heads), cfg.tol)
+    assert torch.isfinite(got_o).all() and torch.isfinite(got_s).all()
