@@ -1,0 +1,410 @@
+"""Benchmark of the Gated DeltaNet hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one chunkwise prefill (gdn_chunk_fwd) of the GDN-2 layer workload:
+B=8 sequences, H=8 heads, T=2048 tokens, dk=dv=128, bf16 q/k/v, per-channel
+gate g in [-5, 0], beta = sigmoid(N(0,1)), zero initial state, fp32 state
+and output.  Inputs are synthetic (seeded recipe in synth/), resident in HBM
+when the timed region starts; they total 235 MB per step, more than the
+126 MB L2, so no L2 flush is needed between steps.
+
+The same run also measures the decode mode (gdn_recurrent_step) on its own
+workload -- B=64 sequences, H=16, d=128, per-channel gate, fp32 state
+carried in place -- with L2 flushed before every timed step (the 64 MiB
+state would otherwise stay in the 126 MB L2), reported under "decode".
+
+Under torchrun (N > 1) every rank runs the same per-GPU workload on its own
+GPU (weak scaling, no collective on the data path); the reported time is
+the max over ranks.  Prints one JSON line on rank 0.
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (the reference arm of this comparison).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+if str(ROOT) not in sys.path:
+    sys.path.insert(0, str(ROOT))
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from synth import CONFIGS, config_inputs  # noqa: E402
+
+PREFILL_CFG = CONFIGS[2]
+DECODE_CFG = CONFIGS[4]
+L2_BYTES = 126 * 1024 * 1024
+METRIC = "GDN prefill tokens/s + % tensor roofline; decode state GB/s vs HBM peak"
+PROFILE_SUMMARY = ROOT / "profiles" / "chunk_fwd_kernel_gdn2_layer_B8H8T2048.md"
+
+
+# ---------------------------------------------------------------- accounting --
+def prefill_bytes(cfg, with_state_in: bool) -> int:
+    """Algorithmic HBM bytes of one prefill call: every input read once,
+    every output written once (q,k,v bf16; g, beta fp32; out fp32; states)."""
+    th = cfg.B * cfg.T * cfg.H
+    per = 2 * cfg.dk + 2 * cfg.dk + 2 * cfg.dv + 4 * (cfg.dk if cfg.per_channel else 1) + 4 + 4 * cfg.dv
+    st = cfg.B * cfg.H * cfg.dk * cfg.dv * 4
+    return th * per + st * (2 if with_state_in else 1)
+
+
+def prefill_flops(cfg, C: int = 64) -> float:
+    """Algorithmic flops per token-head of the chunk algebra: 3 C dk + 2 C dv
+    + C^2 / 3 + 6 dk dv (the triangular halves only; wasted tile work and the
+    extra passes of split-precision operands are not counted)."""
+    per = 3 * C * cfg.dk + 2 * C * cfg.dv + C * C / 3 + 6 * cfg.dk * cfg.dv
+    return per * cfg.B * cfg.T * cfg.H
+
+
+def decode_bytes(cfg) -> int:
+    bh = cfg.B * cfg.H
+    state = 2 * bh * cfg.dk * cfg.dv * 4
+    qkv = bh * (2 * cfg.dk + cfg.dv) * 2
+    g = bh * (cfg.dk if cfg.per_channel else 1) * 4
+    return state + qkv + g + bh * 4 + bh * cfg.dv * 4
+
+
+def measured_peaks() -> dict:
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def ncu_traffic():
+    """dram read+write bytes per launch of the chunk kernel, from the committed
+    ncu summary (a 'traffic_bytes_per_launch: N' line), else None."""
+    if not PROFILE_SUMMARY.exists():
+        return None
+    for line in PROFILE_SUMMARY.read_text().splitlines():
+        if line.strip().startswith("traffic_bytes_per_launch:"):
+            try:
+                return float(line.split(":", 1)[1].strip())
+            except ValueError:
+                return None
+    return None
+
+
+# ---------------------------------------------------------------- clocks --------
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.index = index
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.error = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        except Exception as e:  # pragma: no cover - NVML missing
+            self.error = repr(e)
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+            except Exception as e:  # pragma: no cover
+                self.error = repr(e)
+                return
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self) -> dict:
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples),
+                **({"error": self.error} if self.error else {})}
+
+
+# ---------------------------------------------------------------- distributed ---
+def dist_setup(n_gpus: int, backend: str | None = None):
+    """Process-group set-up for torchrun launches; returns (rank, world, local).
+    NCCL on GPUs (one process per GPU), gloo otherwise or when asked."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    if world != n_gpus and rank == 0:
+        print(f"warning: --gpus {n_gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    return rank, world, local
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        if dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[torch.cuda.current_device()])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank scalar (timings are reported as the slowest rank)."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = torch.device("cuda") if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- CPU oracle ----
+def oracle_sample(cfg, n_pairs: int, threads: int):
+    """Times the fp64 oracle on the first n_pairs (b, h) pairs of the workload;
+    returns (seconds, equivalent tokens) where tokens = pairs * T / H."""
+    import oracle
+    x = config_inputs(cfg, B=max(1, -(-n_pairs // cfg.H)))
+    f = {k: (None if v is None else np.ascontiguousarray(v.double().numpy())) for k, v in x.items()}
+    heads = list(range(n_pairs))
+    t0 = time.perf_counter()
+    oracle.run(f["q"], f["k"], f["v"], f["g"], f["beta"], f["s0"], per_channel=cfg.per_channel,
+               heads=heads, threads=threads)
+    dt = time.perf_counter() - t0
+    return dt, n_pairs * cfg.T / cfg.H
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return 0
+    cfg = PREFILL_CFG
+    cores = cpu_cores()
+    n_pairs = min(cfg.B * cfg.H, cores)
+    for _ in range(args.warmup):
+        oracle_sample(cfg, n_pairs, cores)
+    total_t = 0.0
+    total_tok = 0.0
+    for _ in range(args.steps):
+        dt, tok = oracle_sample(cfg, n_pairs, cores)
+        total_t += dt
+        total_tok += tok
+    value = total_tok / total_t
+    sample = (f"{n_pairs} (b,h) pairs x T={cfg.T} per step of the {cfg.name} workload, fp64, "
+              f"one pair per thread")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(cfg),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def workload_config(cfg) -> dict:
+    return {"workload": "GDN-2 layer prefill (chunkwise, per-channel gate)", "B": cfg.B,
+            "H": cfg.H, "T": cfg.T, "dk": cfg.dk, "dv": cfg.dv, "gate": cfg.gate,
+            "inputs": "bf16 q/k/v, fp32 g/beta, zero initial state, fp32 state and output",
+            "chunk": 64,
+            "l2": f"inputs {prefill_bytes(cfg, False) / 1e6:.0f} MB per step > 126 MB L2 (no flush)"}
+
+
+# ---------------------------------------------------------------- GPU arm -------
+def time_events(fn, steps: int, stream) -> float:
+    """Seconds for `steps` calls of fn, CUDA events on the launching stream."""
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / 1e3
+
+
+def run_ours(args, rank: int, world: int, local: int):
+    import gated_delta_rule_77_b200 as gdn
+    gdn.load()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    peaks = measured_peaks()
+    cfg = PREFILL_CFG
+
+    x = config_inputs(cfg, seed=cfg.index + 1000 * rank)
+    q, k, v, g, beta = (x[n].to(dev) for n in ("q", "k", "v", "g", "beta"))
+    out = torch.empty(cfg.B, cfg.T, cfg.H, cfg.dv, dtype=torch.float32, device=dev)
+    s_out = torch.empty(cfg.B, cfg.H, cfg.dk, cfg.dv, dtype=torch.float32, device=dev)
+
+    def step():
+        gdn.chunk_fwd(q, k, v, g, beta, None, out=out, state_out=s_out, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        dt = time_events(step, args.steps, stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    dt = max_over_ranks(dt, world)
+    if gdn.check(stream) != gdn.GDN_OK:
+        raise RuntimeError("the chunk kernel reported an abandoned wait")
+
+    tokens = cfg.B * cfg.T * args.steps * world
+    value = tokens / dt
+    t_launch = dt / args.steps
+    nbytes = prefill_bytes(cfg, False)
+    nflops = prefill_flops(cfg)
+    achieved_gbs = nbytes / t_launch / 1e9
+    traffic = ncu_traffic()
+    roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": traffic,
+                "kernel": "chunk_fwd_kernel<per-channel>", "bytes_per_launch": nbytes,
+                "peak_source": peaks["source"]}
+    tflops = nflops / t_launch / 1e12
+    tensor = {"achieved_tflops": tflops, "peak_tflops": peaks["bf16_tflops"],
+              "frac": tflops / peaks["bf16_tflops"], "flops_per_launch": nflops,
+              "attainable_frac": min(1.0, (nbytes / (peaks["hbm_gbs"] * 1e9)) / t_launch)}
+
+    # End to end through the public API with pinned host buffers: H2D of the
+    # step's inputs, the call, D2H of the output, all inside the timed region.
+    host = {n: x[n].pin_memory() for n in ("q", "k", "v", "g", "beta")}
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    def e2e_step():
+        for n, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta)):
+            t.copy_(host[n], non_blocking=True)
+        gdn.chunk_fwd(q, k, v, g, beta, None, out=out, state_out=s_out, stream=stream)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_steps = max(1, min(args.steps, 10))
+    dt_e2e = max_over_ranks(time_events(e2e_step, e2e_steps, stream), world)
+    e2e = {"value": cfg.B * cfg.T * e2e_steps * world / dt_e2e, "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+
+    decode = run_decode(gdn, dev, stream, peaks, world, rank)
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cores = cpu_cores()
+            n_pairs = cfg.B * cfg.H
+            cdt, ctok = oracle_sample(cfg, n_pairs, cores)
+            cpu = {"value": ctok / cdt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                   "sample": f"the full workload once ({n_pairs} (b,h) pairs x T={cfg.T}), fp64, "
+                             f"{cdt:.1f} s wall on {cores} threads"}
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_launch,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic", "config": workload_config(cfg), "roofline": roofline,
+                "tensor": tensor, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": args.steps, "clocks": clk.summary(), "decode": decode}
+        print(json.dumps(line))
+    return 0
+
+
+def run_decode(gdn, dev, stream, peaks, world, rank, steps: int = 20, warmup: int = 3):
+    """Decode-mode step time with L2 flushed before each timed step."""
+    cfg = DECODE_CFG
+    x = config_inputs(cfg, steps=4, seed=cfg.index + 1000 * rank)
+    q, k, v, g, beta = (x[n].to(dev) for n in ("q", "k", "v", "g", "beta"))
+    state = x["s0"].to(dev)
+    out = torch.empty(cfg.B, cfg.H, cfg.dv, dtype=torch.float32, device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    times = []
+    for i in range(warmup + steps):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        gdn.recurrent_step(q[i % 4], k[i % 4], v[i % 4], g[i % 4], beta[i % 4], state, out=out,
+                           stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= warmup:
+            times.append(e0.elapsed_time(e1) / 1e3)
+    t = max_over_ranks(statistics.median(times), world)
+    nbytes = decode_bytes(cfg)
+    gbs = nbytes / t / 1e9
+    return {"metric": "decode state GB/s", "value": gbs, "unit": "GB/s",
+            "us_per_step": t * 1e6, "frac": gbs / peaks["hbm_gbs"], "peak": peaks["hbm_gbs"],
+            "bytes_per_step": nbytes, "tokens_per_s": cfg.B * world / t,
+            "config": {"workload": "recurrent decode step", "B": cfg.B, "H": cfg.H, "dk": cfg.dk,
+                       "dv": cfg.dv, "gate": cfg.gate, "state": "fp32 in place",
+                       "l2": "flushed before every timed step (state 64 MiB < L2)"},
+            "timing": f"median of {steps} single-step CUDA-event timings"}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            return run_reference(args, rank, world)
+        return run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

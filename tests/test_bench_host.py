@@ -1,0 +1,74 @@
+"""Host-side logic of bench.py (CPU only): algorithmic byte / flop accounting,
+the reference arm's JSON line, and the max-over-ranks timing with two gloo
+ranks."""
+import json
+import os
+import socket
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import bench
+from synth import CONFIGS
+
+
+def test_prefill_accounting_matches_hand_count():
+    cfg = CONFIGS[2]
+    th = 8 * 2048 * 8                       # token-heads
+    per = 256 + 256 + 256 + 512 + 4 + 512   # q, k, v bf16; g, beta, out fp32
+    assert bench.prefill_bytes(cfg, False) == th * per + 8 * 8 * 128 * 128 * 4
+    assert bench.prefill_flops(cfg) == pytest.approx(th * (3 * 64 * 128 + 2 * 64 * 128 + 64 * 64 / 3
+                                                            + 6 * 128 * 128))
+
+
+def test_decode_accounting_matches_hand_count():
+    # 2 x 64 MiB of state + q,k,v bf16 + per-channel g + beta + fp32 out
+    assert bench.decode_bytes(CONFIGS[4]) == 136_056_832
+
+
+def test_reference_arm_prints_contract_line(capsys, monkeypatch):
+    monkeypatch.setattr(bench, "cpu_cores", lambda: 2)
+    rc = bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"])
+    assert rc == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "dtype", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 2
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    r, w, _ = bench.dist_setup(world, backend="gloo")
+    try:
+        bench.barrier(w)
+        q.put((r, bench.max_over_ranks(float(10 + r), w)))
+    finally:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_two_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=10) for _ in range(2))
+    assert got == [(0, 11.0), (1, 11.0)]
