@@ -85,17 +85,24 @@ def measured_peaks() -> dict:
 
 
 def ncu_traffic():
-    """dram read+write bytes per launch of the chunk kernel, from the committed
-    ncu summary (a 'traffic_bytes_per_launch: N' line), else None."""
+    """dram read+write bytes per launch of the chunk kernel from the committed
+    ncu summary, or None when the kernel source changed since that capture
+    (the summary records the sha1 of the source it measured)."""
+    import hashlib
     if not PROFILE_SUMMARY.exists():
         return None
+    fields = {}
     for line in PROFILE_SUMMARY.read_text().splitlines():
-        if line.strip().startswith("traffic_bytes_per_launch:"):
-            try:
-                return float(line.split(":", 1)[1].strip())
-            except ValueError:
-                return None
-    return None
+        if ":" in line and not line.startswith(("|", " ", "#")):
+            key, val = line.split(":", 1)
+            fields[key.strip()] = val.strip()
+    src = ROOT / "gated_delta_rule_77_b200" / "csrc" / "chunk_sm100.cu"
+    if fields.get("kernel_source_sha1") != hashlib.sha1(src.read_bytes()).hexdigest():
+        return None
+    try:
+        return float(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 # ---------------------------------------------------------------- clocks --------
@@ -360,10 +367,13 @@ def run_decode(gdn, dev, stream, peaks, world, rank, steps: int = 20, warmup: in
     q, k, v, g, beta = (x[n].to(dev) for n in ("q", "k", "v", "g", "beta"))
     state = x["s0"].to(dev)
     out = torch.empty(cfg.B, cfg.H, cfg.dv, dtype=torch.float32, device=dev)
-    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    # Evict the state from L2 by reading a buffer twice its size: a read
+    # leaves L2 clean, so the timed step pays for its own traffic only.
+    flush = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
     times = []
     for i in range(warmup + steps):
-        flush.zero_()
+        torch.sum(flush, out=sink)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -381,7 +391,7 @@ def run_decode(gdn, dev, stream, peaks, world, rank, steps: int = 20, warmup: in
             "bytes_per_step": nbytes, "tokens_per_s": cfg.B * world / t,
             "config": {"workload": "recurrent decode step", "B": cfg.B, "H": cfg.H, "dk": cfg.dk,
                        "dv": cfg.dv, "gate": cfg.gate, "state": "fp32 in place",
-                       "l2": "flushed before every timed step (state 64 MiB < L2)"},
+                       "l2": "evicted before every timed step by reading 2x L2 (state 64 MiB < L2)"},
             "timing": f"median of {steps} single-step CUDA-event timings"}
 
 

@@ -77,7 +77,7 @@ constexpr int NT = 256;    // threads per CTA
 constexpr uint32_t R_IN = 0;                 // 32 KB
 constexpr uint32_t OFF_TH = R_IN;            //   8 KB T' hi [64 r][64 m]
 constexpr uint32_t OFF_TL = R_IN + 8192;     //   8 KB T' lo
-constexpr uint32_t OFF_Y = R_IN + 16384;     //   3 KB solve scratch
+constexpr uint32_t OFF_Y = R_IN + 16384;     //   3 KB solve scratch [16][48] fp32
 constexpr uint32_t OFF_WT = R_IN + 16384;    //   16 KB W^T fp16 [128 i][64 r] (after solve)
 constexpr uint32_t R_V = 32768;              // 16 KB raw V [half][64][128 B]
 constexpr uint32_t R_S = 49152;              // 32 KB S fp16 [j half][128 i][64 j]
@@ -97,7 +97,7 @@ constexpr uint32_t OFF_KDL = R_X + 49152;    //   16 KB K*D bf16 lo
 constexpr uint32_t OFF_PH = R_X + 65536;     //   8 KB P hi [64 r][64 m]
 constexpr uint32_t OFF_PL = R_X + 73728;     //   8 KB P lo
 constexpr uint32_t OFF_A = R_X + 81920;      //   16 KB A fp32 [64][64]
-constexpr uint32_t OFF_TF = R_X + 98304;     //   16 KB T fp32 [64][64]
+constexpr uint32_t OFF_TF = R_X + 98304;     //   16 KB T fp32 [64][64] row-major
 constexpr uint32_t OFF_UH = R_X + 81920;     //   16 KB U^T hi [128 j][64 r] (after solve)
 constexpr uint32_t OFF_UL = R_X + 98304;     //   16 KB U^T lo
 constexpr uint32_t R_SMALL = R_X + 114688;
@@ -166,14 +166,107 @@ __device__ __forceinline__ void load_bf16x8(const uint8_t* src, float* v) {
     }
 }
 
+
+// T = (I + A)^{-1} for a strictly lower triangular 64x64 fp32 A (layout fidx),
+// written to T (plain row-major [64][64]; entries above the diagonal inside the
+// 16x16 diagonal blocks are written as zero, other upper entries untouched).
+// Y: 16 x 48 fp32 scratch.  Called by all NT threads (contains barriers).
+//   (a) D_b = (I + A_bb)^{-1}, b = 0..3, by forward substitution: warp b,
+//       lane = column;
+//   (b) row blocks a = 1..3: T_{a,<a} = -D_a (A_{a,<a} T_{<a,<a}), both small
+//       products register-blocked by four columns.
+__device__ __forceinline__ void solve_unit_lower64(const float* sA, float* sT, float* sY, int tid) {
+    const int warp = tid >> 5, lane = tid & 31;
+    if (warp < 4 && lane < 16) {
+        const int o = warp * 16;
+        float t[16];
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) {
+            float a[16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 v = *reinterpret_cast<const float4*>(&sA[fidx(o + rr, o + 4 * q)]);
+                a[4 * q] = v.x; a[4 * q + 1] = v.y; a[4 * q + 2] = v.z; a[4 * q + 3] = v.w;
+            }
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};     // short dependency chains
+#pragma unroll
+            for (int m = 0; m < rr; ++m) acc[m & 3] = fmaf(a[m], t[m], acc[m & 3]);
+            t[rr] = (rr == lane) ? 1.f : -((acc[0] + acc[1]) + (acc[2] + acc[3]));
+        }
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) sT[(o + rr) * 64 + o + lane] = t[rr];
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int a = 1; a < 4; ++a) {
+        // Thread tile: rows {rp, rp + 8} x four columns [4 c4, 4 c4 + 4).
+        const int ncol4 = 4 * a;            // float4 column groups left of the diagonal block
+        const int nitem = 8 * ncol4;
+        const int rp = tid / ncol4, c4 = tid - (tid / ncol4) * ncol4;
+        if (tid < nitem) {
+            // Y[rr][4c4..] = sum_m A[16a+rr][m] T[m][4c4..]; T[m][c] = 0 for m < 4 c4.
+            float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            for (int m4 = c4; m4 < 4 * a; ++m4) {
+                const float4 a0 = *reinterpret_cast<const float4*>(&sA[fidx(16 * a + rp, 4 * m4)]);
+                const float4 a1 = *reinterpret_cast<const float4*>(&sA[fidx(16 * a + rp + 8, 4 * m4)]);
+                const float am[2][4] = {{a0.x, a0.y, a0.z, a0.w}, {a1.x, a1.y, a1.z, a1.w}};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float4 tv = *reinterpret_cast<const float4*>(&sT[(4 * m4 + e) * 64 + 4 * c4]);
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        y[i][0] = fmaf(am[i][e], tv.x, y[i][0]);
+                        y[i][1] = fmaf(am[i][e], tv.y, y[i][1]);
+                        y[i][2] = fmaf(am[i][e], tv.z, y[i][2]);
+                        y[i][3] = fmaf(am[i][e], tv.w, y[i][3]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+                *reinterpret_cast<float4*>(&sY[(rp + 8 * i) * 48 + 4 * c4]) =
+                    make_float4(y[i][0], y[i][1], y[i][2], y[i][3]);
+        }
+        __syncthreads();
+        if (tid < nitem) {
+            // T[16a+rr][4c4..] = -sum_n D_a[rr][n] Y[n][4c4..]
+            float t[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+            for (int n4 = 0; n4 < 4; ++n4) {
+                const float4 d0 = *reinterpret_cast<const float4*>(&sT[(16 * a + rp) * 64 + 16 * a + 4 * n4]);
+                const float4 d1 = *reinterpret_cast<const float4*>(&sT[(16 * a + rp + 8) * 64 + 16 * a + 4 * n4]);
+                const float dn[2][4] = {{d0.x, d0.y, d0.z, d0.w}, {d1.x, d1.y, d1.z, d1.w}};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float4 yv = *reinterpret_cast<const float4*>(&sY[(4 * n4 + e) * 48 + 4 * c4]);
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        t[i][0] = fmaf(dn[i][e], yv.x, t[i][0]);
+                        t[i][1] = fmaf(dn[i][e], yv.y, t[i][1]);
+                        t[i][2] = fmaf(dn[i][e], yv.z, t[i][2]);
+                        t[i][3] = fmaf(dn[i][e], yv.w, t[i][3]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+                *reinterpret_cast<float4*>(&sT[(16 * a + rp + 8 * i) * 64 + 4 * c4]) =
+                    make_float4(-t[i][0], -t[i][1], -t[i][2], -t[i][3]);
+        }
+        __syncthreads();
+    }
+}
+
 template <bool CHANNEL>
 __global__ void __launch_bounds__(NT, 1)
 chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const Params p)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    // 1024-byte aligned base (128B-swizzle atoms), derived by a pointer offset
+    // so that the compiler keeps the shared address space (LDS/STS, not
+    // generic loads and stores).
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(smem);
     float* sGam = reinterpret_cast<float*>(smem + SM_GAM);
     float* sBeta = reinterpret_cast<float*>(smem + SM_BETA);
@@ -199,8 +292,10 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int nchunks = (T + C - 1) / C;
 
     // Element ownership for the gate prep and tile building: 16 channel
-    // chunks of 8 (ck) x 16 token groups of 4 (tg); the 16 token groups of a
-    // channel chunk sit in one half-warp so the cumulative sum is a shuffle scan.
+    // chunks of 8 (ck) x 16 lanes (tg), lane tg owning tokens tg + 16 u,
+    // u = 0..3.  The 16 lanes of a channel chunk sit in one half-warp (the
+    // cumulative sum is a shuffle scan) and eight consecutive lanes touch eight
+    // consecutive rows of a 128B-swizzled tile (no shared-memory bank conflicts).
     const int ck = 2 * warp + (lane >> 4);
     const int tg = lane & 15;
     const int ckh = ck >> 3;       // 64-channel half of the tile
@@ -282,10 +377,10 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (CHANNEL) {
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int t = t0 + 4 * tg + u;
-                if (t < T) {
+                const int r = tg + 16 * u;
+                if (t0 + r < T) {
                     const float4* src = reinterpret_cast<const float4*>(
-                        p.g + (tk0 + (long)(4 * tg + u) * H) * D + 8 * ck);
+                        p.g + (tk0 + (long)r * H) * D + 8 * ck);
                     const float4 a = src[0], c = src[1];
                     gam[u][0] = a.x; gam[u][1] = a.y; gam[u][2] = a.z; gam[u][3] = a.w;
                     gam[u][4] = c.x; gam[u][5] = c.y; gam[u][6] = c.z; gam[u][7] = c.w;
@@ -294,25 +389,42 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     for (int e = 0; e < 8; ++e) gam[u][e] = 0.f;
                 }
             }
+            // Inclusive scan over the 16 lanes of each 16-token block, then add
+            // the totals of the preceding blocks.
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float x = __shfl_up_sync(0xffffffffu, gam[u][e], o, 16);
+                        if (tg >= o) gam[u][e] += x;
+                    }
+            }
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                gam[1][e] += gam[0][e];
-                gam[2][e] += gam[1][e];
-                gam[3][e] += gam[2][e];
-                float tot = gam[3][e];           // inclusive scan of group totals
+                float off = 0.f;
 #pragma unroll
-                for (int o = 1; o < 16; o <<= 1) {
-                    const float x = __shfl_up_sync(0xffffffffu, tot, o, 16);
-                    if (tg >= o) tot += x;
+                for (int u = 0; u < 4; ++u) {
+                    const float tot = __shfl_sync(0xffffffffu, gam[u][e], 15, 16);
+                    gam[u][e] += off;
+                    off += tot;
                 }
-                const float excl = tot - gam[3][e];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) gam[u][e] += excl;
             }
-            if (tg == 3 || tg == 11 || tg == 15) {
-                float* dst = tg == 3 ? sRef0 : (tg == 11 ? sRef1 : sLast);
+            if (ci + 1 < nchunks) {   // warm L2 with the next chunk's gate rows
 #pragma unroll
-                for (int e = 0; e < 8; ++e) dst[8 * ck + e] = gam[3][e];
+                for (int u = 0; u < 4; ++u) {
+                    const int r = C + tg + 16 * u;
+                    if (t0 + r < T) prefetch_l2(p.g + (tk0 + (long)r * H) * D + 8 * ck);
+                }
+            }
+            if (tg == 15) {   // G at tokens 15, 47 (block references) and 63
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    sRef0[8 * ck + e] = gam[0][e];
+                    sRef1[8 * ck + e] = gam[2][e];
+                    sLast[8 * ck + e] = gam[3][e];
+                }
             }
         }
         if (warp == 0) {
@@ -348,7 +460,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // Factored operands, bf16 hi + lo (see header).
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int r = 4 * tg + u;
+                const int r = tg + 16 * u;
                 const float* ref = r < 32 ? sRef0 : sRef1;
                 float kf[8], qf[8];
                 load_bf16x8(smem + R_IN + ckh * 16384 + swz(r, ckc), kf);
@@ -419,7 +531,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // K*E (bf16), Q*E (fp16), K*D (bf16 hi + lo) into the freed X region.
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const int r = 4 * tg + u;
+            const int r = tg + 16 * u;
             float kf[8], qf[8], ke[8], qe[8], kd[8];
             load_bf16x8(smem + R_IN + ckh * 16384 + swz(r, ckc), kf);
             load_bf16x8(smem + R_IN + ckh * 16384 + 8192 + swz(r, ckc), qf);
@@ -447,54 +559,58 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             store_f16x8(smem + OFF_QE + o64, qe);
             store_split(smem + OFF_KDH + o64, smem + OFF_KDL + o64, kd);
         }
-        if (warp < 4) {
-            const int L = warp * 32 + lane;       // TMEM lane = row of X
+        {
+            // Thread: row L = TMEM lane of X (A rows 0-63, P rows 64-127),
+            // columns j in [32*half, 32*half + 32).
+            const int L = quad * 32 + lane;
             const bool is_p = L >= 64;
             const int r = L & 63;
-            float x[64];
-            const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+            float x[32];
+            const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+            bool zero = false;
             if (CHANNEL) {
-                if (r < 32) {
-                    tmem_ld32(lane_base + TM_X, *reinterpret_cast<float(*)[32]>(&x[0]));
-#pragma unroll
-                    for (int j = 32; j < 64; ++j) x[j] = 0.f;
-                } else {
-                    tmem_ld32(lane_base + TM_X + 32, *reinterpret_cast<float(*)[32]>(&x[0]));
-                    tmem_ld32(lane_base + TM_X + 64, *reinterpret_cast<float(*)[32]>(&x[32]));
+                if (r < 32) {   // block 0: X columns 0-31 hold j = 0..31
+                    if (half == 0) tmem_ld32(lane_base + TM_X, x); else zero = true;
+                } else {        // block 1: X columns 32-95 hold j = 0..63
+                    tmem_ld32(lane_base + TM_X + 32 + half * 32, x);
                 }
             } else {
-                tmem_ld32(lane_base + TM_X, *reinterpret_cast<float(*)[32]>(&x[0]));
-                tmem_ld32(lane_base + TM_X + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
+                tmem_ld32(lane_base + TM_X + half * 32, x);
             }
             tmem_wait_ld();
+            if (zero) {
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) x[jj] = 0.f;
+            }
             const float br = sBeta[r];
             const float Gr = CHANNEL ? 0.f : sGam[r];
+            const int j0 = half * 32;
             if (!is_p) {
 #pragma unroll
-                for (int j4 = 0; j4 < 16; ++j4) {
-                    float4 a4;
-                    float* a = &a4.x;
+                for (int j4 = 0; j4 < 8; ++j4) {
+                    float a[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int j = 4 * j4 + e;
+                        const int j = j0 + 4 * j4 + e;
                         float val = 0.f;
-                        if (j < r) val = br * x[j] * (CHANNEL ? 1.f : __expf(Gr - sGam[j]));
+                        if (j < r) val = br * x[4 * j4 + e] * (CHANNEL ? 1.f : __expf(Gr - sGam[j]));
                         a[e] = val;
                     }
-                    *reinterpret_cast<float4*>(&sA[fidx(r, 4 * j4)]) = a4;
+                    *reinterpret_cast<float4*>(&sA[fidx(r, j0 + 4 * j4)]) = make_float4(a[0], a[1], a[2], a[3]);
                 }
             } else {
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
+                for (int c = 0; c < 4; ++c) {
                     float pv[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const int j = 8 * c + e;
+                        const int j = j0 + 8 * c + e;
                         float val = 0.f;
-                        if (j <= r) val = x[j] * (CHANNEL ? 1.f : __expf(Gr - sGam[j]));
+                        if (j <= r) val = x[8 * c + e] * (CHANNEL ? 1.f : __expf(Gr - sGam[j]));
                         pv[e] = val;
                     }
-                    store_split(smem + OFF_PH + swz(r, c), smem + OFF_PL + swz(r, c), pv);
+                    const int cc = half * 4 + c;
+                    store_split(smem + OFF_PH + swz(r, cc), smem + OFF_PL + swz(r, cc), pv);
                 }
             }
         }
@@ -504,54 +620,18 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         __syncthreads();
 
         // ---------------------------------------------------- T = (I + A)^{-1} --
-        // Diagonal 16x16 blocks by forward substitution (warp b, lane = column).
-        if (warp < 4 && lane < 16) {
-            const int o = warp * 16;
-            float t[16];
-#pragma unroll
-            for (int rr = 0; rr < 16; ++rr) {
-                float acc = 0.f;
-#pragma unroll
-                for (int m = 0; m < rr; ++m) acc = fmaf(sA[fidx(o + rr, o + m)], t[m], acc);
-                t[rr] = (rr == lane) ? 1.f : -acc;
-            }
-#pragma unroll
-            for (int rr = 0; rr < 16; ++rr) sTf[fidx(o + rr, o + lane)] = t[rr];
-        }
-        __syncthreads();
-        // Off-diagonal blocks: T_ab = -T_aa * sum_{m=b}^{a-1} A_am T_mb, by
-        // increasing distance a - b.
-#pragma unroll 1
-        for (int d = 1; d < 4; ++d) {
-            const int nel = (4 - d) * 256;
-            for (int e = tid; e < nel; e += NT) {
-                const int blk = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-                const int a = blk + d, bb = blk;
-                float acc = 0.f;
-                for (int m = 16 * bb; m < 16 * a; ++m)
-                    acc = fmaf(sA[fidx(16 * a + rr, m)], sTf[fidx(m, 16 * bb + cc)], acc);
-                sY[e] = acc;
-            }
-            __syncthreads();
-            for (int e = tid; e < nel; e += NT) {
-                const int blk = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-                const int a = blk + d, bb = blk;
-                float acc = 0.f;
-#pragma unroll
-                for (int n = 0; n < 16; ++n)
-                    acc = fmaf(sTf[fidx(16 * a + rr, 16 * a + n)], sY[(blk << 8) + (n << 4) + cc], acc);
-                sTf[fidx(16 * a + rr, 16 * bb + cc)] = -acc;
-            }
-            __syncthreads();
-        }
+        solve_unit_lower64(sA, sTf, sY, tid);
         // T' = T Diag(beta) -> bf16 hi + lo, K-major [64 r][64 m].
         for (int e = tid; e < 512; e += NT) {
             const int r = e >> 3, c = e & 7;
+            const float4 t0v = *reinterpret_cast<const float4*>(&sTf[r * 64 + 8 * c]);
+            const float4 t1v = *reinterpret_cast<const float4*>(&sTf[r * 64 + 8 * c + 4]);
+            const float tt[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
             float tv[8];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 const int m = 8 * c + q;
-                tv[q] = (m <= r) ? sTf[fidx(r, m)] * sBeta[m] : 0.f;
+                tv[q] = (m <= r) ? tt[q] * sBeta[m] : 0.f;
             }
             store_split(smem + OFF_TH + swz(r, c), smem + OFF_TL + swz(r, c), tv);
         }
