@@ -33,8 +33,8 @@ GATE_CHANNEL = 1
 IO_BF16 = 0
 IO_F32 = 1
 
-SYMBOLS = ("gdn_chunk_fwd", "gdn_chunk_fwd_ex", "gdn_recurrent_step", "gdn_recurrent_step_ex",
-           "gdn_check", "gdn_status_string")
+SYMBOLS = ("gdn_chunk_fwd", "gdn_chunk_fwd_ex", "gdn_chunk_fwd_segments", "gdn_recurrent_step",
+           "gdn_recurrent_step_ex", "gdn_check", "gdn_status_string")
 
 _lib = None
 
@@ -56,6 +56,7 @@ def load() -> ctypes.CDLL:
     vp, fp, i = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
     lib.gdn_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i, i, i, i, i, i, vp]
     lib.gdn_chunk_fwd_ex.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i, i, i, i, i, i, i, i, vp]
+    lib.gdn_chunk_fwd_segments.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i, i, i, i, i, i, i, vp]
     lib.gdn_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, vp]
     lib.gdn_recurrent_step_ex.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, i, vp]
     lib.gdn_check.argtypes = [vp]
@@ -96,9 +97,11 @@ def _io_code(dtype):
 
 
 def chunk_fwd(q, k, v, g, beta, state_in=None, *, out=None, state_out=None,
-              return_state: bool = True, chunk_size: int = 0, stream=None):
+              return_state: bool = True, chunk_size: int = 0, segments=None, stream=None):
     """Chunkwise prefill.  q, k [B,T,H,dk]; v [B,T,H,dv]; g [B,T,H] or
     [B,T,H,dk] fp32; beta [B,T,H] fp32; state_in [B,H,dk,dv] fp32 or None.
+    ``segments``: None = automatic; an int selects gdn_chunk_fwd_segments
+    (1 = no sequence parallelism, n > 1 = n time segments).
     Returns (out [B,T,H,dv] fp32, final state or None)."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -108,6 +111,13 @@ def chunk_fwd(q, k, v, g, beta, state_in=None, *, out=None, state_out=None,
     if state_out is None and return_state:
         state_out = torch.empty(B, H, dk, dv, dtype=torch.float32, device=v.device)
     _check_cuda(q, k, v, g, beta, state_in, out, state_out)
+    if segments is not None:
+        rc = load().gdn_chunk_fwd_segments(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                           _ptr(state_in), _ptr(out), _ptr(state_out), B, T, H,
+                                           dk, dv, gate, int(segments), _stream(stream))
+        if rc != GDN_OK:
+            raise GdnError(rc, "gdn_chunk_fwd_segments")
+        return out, state_out
     rc = load().gdn_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in),
                                  _ptr(out), _ptr(state_out), B, T, H, dk, dv, gate,
                                  _io_code(q.dtype), int(chunk_size), _stream(stream))

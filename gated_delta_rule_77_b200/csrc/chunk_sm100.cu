@@ -118,13 +118,21 @@ constexpr uint32_t TM_UT = 192;   // U^T: 128 x 64
 constexpr uint32_t TM_OT = 256;   // O^T: 128 x 64
 constexpr uint32_t TM_SN = 384;   // SN:  128 x 128
 
+// One launch covers B x nseg x H (batch, time segment, head) problems, and
+// optionally a second copy of them ("transition" CTAs, second half of the
+// grid) that run the same chunk recursion with v = 0 from the identity state:
+// the state map of a segment is affine, S_end = M S_start + S_end(0), and
+// those CTAs produce M (dk x dk).
 struct Params {
     const float* g;            // [B, T, H] or [B, T, H, D]
     const float* beta;         // [B, T, H]
-    const float* state_in;     // [B, H, D, D] or null
-    float* state_out;          // [B, H, D, D] or null
-    float* out;                // [B, T, H, D] fp32
-    int T, H;
+    const float* state_in;     // [B, in_segs, H, D, D] or null (zero state)
+    float* state_out;          // [B, out_segs, H, D, D] or null; out_segs == 1: last segment only
+    float* trans_out;          // [B, nseg, H, D, D] transitions, or null (no transition CTAs)
+    float* out;                // [B, T, H, D] fp32, or null (outputs not written)
+    int T, H, B;
+    int nseg, seg_len;         // time segments of seg_len tokens (a multiple of C)
+    int in_segs, out_segs;     // 1 or nseg
 };
 
 // fp32 64x64 matrix in shared memory, float4 groups xor-swizzled by row so
@@ -287,9 +295,15 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int half = warp >> 2;     // which half of the columns this warp takes
     const int T = p.T;
     const int H = p.H;
-    const int h = blockIdx.x % H;
-    const int b = blockIdx.x / H;
-    const int nchunks = (T + C - 1) / C;
+    const int per_mode = p.B * p.nseg * H;
+    const bool transition = static_cast<int>(blockIdx.x) >= per_mode;
+    const int rem = static_cast<int>(blockIdx.x) - (transition ? per_mode : 0);
+    const int h = rem % H;
+    const int seg = (rem / H) % p.nseg;
+    const int b = rem / (H * p.nseg);
+    const int t_begin = seg * p.seg_len;
+    const int t_end = min(T, t_begin + p.seg_len);
+    const int nchunks = t_end > t_begin ? (t_end - t_begin + C - 1) / C : 0;
 
     // Element ownership for the gate prep and tile building: 16 channel
     // chunks of 8 (ck) x 16 lanes (tg), lane tg owning tokens tg + 16 u,
@@ -322,9 +336,13 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int srow = quad * 32 + lane;
     const int scol = half * 64;
     float s[64];
-    const long sb = ((long)b * H + h) * (long)D * D;
-    if (p.state_in) {
-        const float4* src = reinterpret_cast<const float4*>(p.state_in + sb + (long)srow * D + scol);
+    const long DD = (long)D * D;
+    if (transition) {                       // identity: the chain yields M
+#pragma unroll
+        for (int c = 0; c < 64; ++c) s[c] = (srow == scol + c) ? 1.f : 0.f;
+    } else if (p.state_in) {
+        const long sin_b = (((long)b * p.in_segs + (p.in_segs == 1 ? 0 : seg)) * H + h) * DD;
+        const float4* src = reinterpret_cast<const float4*>(p.state_in + sin_b + (long)srow * D + scol);
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
             float4 t = src[c];
@@ -343,19 +361,19 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     write_state_f16();
 
     auto issue_loads = [&](int chunk) {
-        const int t0 = chunk * C;
-        mbar_expect_tx(bar_tma, 3 * 16384);
+        const int t0 = t_begin + chunk * C;
+        mbar_expect_tx(bar_tma, (transition ? 2 : 3) * 16384);
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
             tma_load_4d(sbase + R_IN + hf * 16384, &tm_k, hf * 64, h, t0, b, bar_tma);
             tma_load_4d(sbase + R_IN + hf * 16384 + 8192, &tm_q, hf * 64, h, t0, b, bar_tma);
-            tma_load_4d(sbase + R_V + hf * 8192, &tm_v, hf * 64, h, t0, b, bar_tma);
+            if (!transition) tma_load_4d(sbase + R_V + hf * 8192, &tm_v, hf * 64, h, t0, b, bar_tma);
         }
     };
 
     fence_async_smem();
     __syncthreads();
-    if (tid == 0) issue_loads(0);
+    if (tid == 0 && nchunks > 0) issue_loads(0);
     int tma_waited = -1;   // last chunk whose loads were waited for
 
     uint32_t mma_phase = 0;
@@ -367,7 +385,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     };
 
     for (int ci = 0; ci < nchunks; ++ci) {
-        const int t0 = ci * C;
+        const int t0 = t_begin + ci * C;
         const long tk0 = ((long)b * T + t0) * H + h;     // flat (b, t0, h)
 
         // ---------------------------------------------------- gate prep --------
@@ -378,7 +396,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int r = tg + 16 * u;
-                if (t0 + r < T) {
+                if (t0 + r < t_end) {
                     const float4* src = reinterpret_cast<const float4*>(
                         p.g + (tk0 + (long)r * H) * D + 8 * ck);
                     const float4 a = src[0], c = src[1];
@@ -415,7 +433,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int r = C + tg + 16 * u;
-                    if (t0 + r < T) prefetch_l2(p.g + (tk0 + (long)r * H) * D + 8 * ck);
+                    if (t0 + r < t_end) prefetch_l2(p.g + (tk0 + (long)r * H) * D + 8 * ck);
                 }
             }
             if (tg == 15) {   // G at tokens 15, 47 (block references) and 63
@@ -429,11 +447,11 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         if (warp == 0) {
             float b0 = 0.f, b1 = 0.f, g0 = 0.f, g1 = 0.f;
-            if (t0 + lane < T) {
+            if (t0 + lane < t_end) {
                 b0 = p.beta[tk0 + (long)lane * H];
                 if (!CHANNEL) g0 = p.g[tk0 + (long)lane * H];
             }
-            if (t0 + 32 + lane < T) {
+            if (t0 + 32 + lane < t_end) {
                 b1 = p.beta[tk0 + (long)(32 + lane) * H];
                 if (!CHANNEL) g1 = p.g[tk0 + (long)(32 + lane) * H];
             }
@@ -650,7 +668,8 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     const uint64_t bt = sdesc_sw128(sbase + tb + ks * 32, 16, 1024);
                     const uint32_t acc = (part | ks) != 0;
                     mma_bf16(tmem + TM_WT, sdesc_sw128(sbase + OFF_KE + ks * 2048, 8192, 1024), bt, id, acc);
-                    mma_bf16(tmem + TM_UT, sdesc_sw128(sbase + R_V + ks * 2048, 8192, 1024), bt, id, acc);
+                    if (!transition)
+                        mma_bf16(tmem + TM_UT, sdesc_sw128(sbase + R_V + ks * 2048, 8192, 1024), bt, id, acc);
                 }
             }
             mma_commit(bar_mma);
@@ -678,9 +697,13 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint64_t a = sdesc_sw128(sbase + R_S + ks * 2048, 16384, 1024);
-                mma_bf16(tmem + TM_UT, a, sdesc_sw128(sbase + OFF_WT + ks * 2048, 8192, 1024), id_u, 1);
-                const uint64_t bq = sdesc_sw128(sbase + OFF_QE + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
-                mma_bf16(tmem + TM_OT, a, bq, id_o, ks > 0);
+                // Transition CTAs have V = 0: U = -W S starts the accumulator.
+                mma_bf16(tmem + TM_UT, a, sdesc_sw128(sbase + OFF_WT + ks * 2048, 8192, 1024), id_u,
+                         transition ? (ks > 0) : 1);
+                if (!transition) {
+                    const uint64_t bq = sdesc_sw128(sbase + OFF_QE + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+                    mma_bf16(tmem + TM_OT, a, bq, id_o, ks > 0);
+                }
             }
             mma_commit(bar_mma);
         }
@@ -719,9 +742,11 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 mma_bf16(tmem + TM_SN, kdh, uh, id_s, ks > 0);
                 mma_bf16(tmem + TM_SN, kdh, ul, id_s, 1);
                 mma_bf16(tmem + TM_SN, kdl, uh, id_s, 1);
-                mma_bf16(tmem + TM_OT, uh, ph, id_o, 1);
-                mma_bf16(tmem + TM_OT, uh, pl, id_o, 1);
-                mma_bf16(tmem + TM_OT, ul, ph, id_o, 1);
+                if (!transition) {
+                    mma_bf16(tmem + TM_OT, uh, ph, id_o, 1);
+                    mma_bf16(tmem + TM_OT, uh, pl, id_o, 1);
+                    mma_bf16(tmem + TM_OT, ul, ph, id_o, 1);
+                }
             }
             mma_commit(bar_mma);
         }
@@ -744,10 +769,12 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             tmem_ld32(lb + TM_OT + half * 32, o);
             tmem_wait_ld();
             const int j = srow;
-            const int nvalid = min(C, T - t0) - half * 32;
+            const int nvalid = min(C, t_end - t0) - half * 32;
+            if (p.out != nullptr && !transition) {
 #pragma unroll
-            for (int r = 0; r < 32; ++r) {
-                if (r < nvalid) p.out[(tk0 + (long)(half * 32 + r) * H) * D + j] = o[r];
+                for (int r = 0; r < 32; ++r) {
+                    if (r < nvalid) p.out[(tk0 + (long)(half * 32 + r) * H) * D + j] = o[r];
+                }
             }
         }
         fence_async_smem();
@@ -762,8 +789,14 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         mma_commit(bar_mma);
         mbar_wait(bar_mma, mma_phase, &g_status_word);
     }
-    if (ok && p.state_out) {
-        float4* dst = reinterpret_cast<float4*>(p.state_out + sb + (long)srow * D + scol);
+    float* sdst = nullptr;
+    if (transition) {
+        sdst = p.trans_out + (((long)b * p.nseg + seg) * H + h) * DD;
+    } else if (p.state_out != nullptr && (p.out_segs != 1 || seg == p.nseg - 1)) {
+        sdst = p.state_out + (((long)b * p.out_segs + (p.out_segs == 1 ? 0 : seg)) * H + h) * DD;
+    }
+    if (ok && sdst) {
+        float4* dst = reinterpret_cast<float4*>(sdst + (long)srow * D + scol);
 #pragma unroll
         for (int c = 0; c < 16; ++c) dst[c] = make_float4(s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]);
     }
@@ -804,6 +837,97 @@ bool make_map(CUtensorMap* map, const void* base, int H, int T, int B) {
     return r == CUDA_SUCCESS;
 }
 
+// Serial combine of the segments' affine state maps, for one (batch, head)
+// and a 32-column slice of the state:
+//     S_start(0) = S0,   S_start(s + 1) = M_s S_start(s) + S_end(0)(s).
+// In place: on entry seg_states[s] holds S_end(0)(s), the end state of
+// segment s started from zero; on exit it holds S_start(s).  The state after
+// the last segment goes to state_out (may alias state_in).  fp32 throughout.
+constexpr int CB_COLS = 32;
+__global__ void __launch_bounds__(256)
+combine_segments_kernel(float* seg_states, const float* trans, const float* state_in,
+                        float* state_out, int H, int nseg)
+{
+    __shared__ __align__(16) float sS[D][CB_COLS];     // current state slice
+    const int nslice = D / CB_COLS;
+    const int slice = blockIdx.x % nslice;
+    const int bh = blockIdx.x / nslice;                // b * H + h
+    const int b = bh / H, h = bh % H;
+    const int c0 = slice * CB_COLS;
+    const int tid = threadIdx.x;
+    const int i = tid >> 1, jc = (tid & 1) * 16;       // row i, 16 columns
+    const long DD = (long)D * D;
+    for (int e = tid; e < D * CB_COLS; e += 256) {
+        const int r = e / CB_COLS, c = e % CB_COLS;
+        sS[r][c] = state_in ? state_in[(long)bh * DD + (long)r * D + c0 + c] : 0.f;
+    }
+    __syncthreads();
+    for (int sg = 0; sg < nseg; ++sg) {
+        const long base = (((long)b * nseg + sg) * H + h) * DD;
+        float* slot = seg_states + base + (long)i * D + c0 + jc;
+        float acc[16];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 v = reinterpret_cast<const float4*>(slot)[q];
+            acc[4 * q] = v.x; acc[4 * q + 1] = v.y; acc[4 * q + 2] = v.z; acc[4 * q + 3] = v.w;
+        }
+        const float4* mrow = reinterpret_cast<const float4*>(trans + base + (long)i * D);
+#pragma unroll 4
+        for (int k4 = 0; k4 < D / 4; ++k4) {
+            const float4 m = mrow[k4];
+            const float mk[4] = {m.x, m.y, m.z, m.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float* srow_k = &sS[4 * k4 + e][jc];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) acc[c] = fmaf(mk[e], srow_k[c], acc[c]);
+            }
+        }
+        float cur[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) cur[c] = sS[i][jc + c];
+        __syncthreads();                               // every read of sS is done
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            reinterpret_cast<float4*>(slot)[q] =
+                make_float4(cur[4 * q], cur[4 * q + 1], cur[4 * q + 2], cur[4 * q + 3]);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) sS[i][jc + c] = acc[c];
+        __syncthreads();
+    }
+    if (state_out) {
+        for (int e = tid; e < D * CB_COLS; e += 256) {
+            const int r = e / CB_COLS, c = e % CB_COLS;
+            state_out[(long)bh * DD + (long)r * D + c0 + c] = sS[r][c];
+        }
+    }
+}
+
+int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+    }
+    return n;
+}
+
+// Number of time segments per (batch, head).  Segmenting costs three chunk
+// passes (zero-start states, transitions, outputs) instead of one, so it pays
+// only when the (batch, head) pairs alone leave most SMs idle.
+int choose_segments(int requested, int BH, int nchunks) {
+    if (nchunks <= 1 || requested == 1) return 1;
+    int n = requested;
+    if (n <= 0) {
+        const int sms = sm_count();
+        if (nchunks < 64 || BH * 4 > sms) return 1;
+        n = sms / BH;
+    }
+    return n < nchunks ? n : nchunks;
+}
+
 template <bool CHANNEL>
 cudaError_t launch(const Problem& p, cudaStream_t stream) {
     static bool attr_set = false;
@@ -817,9 +941,41 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
     if (!make_map(&mq, p.q, p.H, p.T, p.B) || !make_map(&mk, p.k, p.H, p.T, p.B) ||
         !make_map(&mv, p.v, p.H, p.T, p.B))
         return cudaErrorInvalidValue;
-    Params prm{p.g, p.beta, p.state_in, p.state_out, static_cast<float*>(p.out), p.T, p.H};
-    chunk_fwd_kernel<CHANNEL><<<p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, prm);
-    return cudaGetLastError();
+    float* out = static_cast<float*>(p.out);
+    const int nchunks = (p.T + C - 1) / C;
+    int nseg = choose_segments(p.segments, p.B * p.H, nchunks);
+    if (nseg <= 1) {
+        Params prm{p.g, p.beta, p.state_in, p.state_out, nullptr, out, p.T, p.H, p.B,
+                   1, nchunks * C, 1, 1};
+        chunk_fwd_kernel<CHANNEL><<<p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, prm);
+        return cudaGetLastError();
+    }
+    // Segment-parallel path: per segment the zero-start end state and the
+    // transition (one launch, two kinds of CTA), a serial combine, then every
+    // segment again from its true start state for the outputs.
+    const int seg_len = ((nchunks + nseg - 1) / nseg) * C;
+    nseg = (p.T + seg_len - 1) / seg_len;
+    const size_t slab = (size_t)p.B * nseg * p.H * D * D;
+    float* ws = nullptr;
+    cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), 2 * slab * sizeof(float), stream);
+    if (e != cudaSuccess) return e;
+    float* seg_states = ws;
+    float* trans = ws + slab;
+    Params p1{p.g, p.beta, nullptr, seg_states, trans, nullptr, p.T, p.H, p.B, nseg, seg_len, 1, nseg};
+    chunk_fwd_kernel<CHANNEL><<<2 * p.B * nseg * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, p1);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) {
+        combine_segments_kernel<<<p.B * p.H * (D / CB_COLS), 256, 0, stream>>>(
+            seg_states, trans, p.state_in, p.state_out, p.H, nseg);
+        e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) {
+        Params p2{p.g, p.beta, seg_states, nullptr, nullptr, out, p.T, p.H, p.B, nseg, seg_len, nseg, 1};
+        chunk_fwd_kernel<CHANNEL><<<p.B * nseg * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, p2);
+        e = cudaGetLastError();
+    }
+    const cudaError_t ef = cudaFreeAsync(ws, stream);
+    return e != cudaSuccess ? e : ef;
 }
 
 }  // namespace

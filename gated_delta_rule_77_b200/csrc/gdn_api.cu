@@ -28,7 +28,10 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 bool dim_ok(int d) { return d == 64 || d == 128; }
 
-int to_status(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
+int to_status(cudaError_t e) {
+    if (e == cudaSuccess) return GDN_OK;
+    return e == cudaErrorMemoryAllocation ? GDN_ERR_NOMEM : GDN_ERR_CUDA;
+}
 
 // Shared validation of the tensors of one call.  `T_tokens` is T for the
 // prefill and 1 for a decode step (its layout is the T = 1 case).
@@ -81,21 +84,24 @@ int validate(const void* q, const void* k, const void* v, const float* g, const 
 
 extern "C" {
 
-int gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* g,
-                     const float* beta, const float* state_in, void* out, float* state_out,
-                     int B, int T, int H, int dk, int dv, int gate_mode, int io_dtype,
-                     int chunk_size, gdn_stream_t stream_)
+static int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, const float* state_in, void* out, float* state_out,
+                          int B, int T, int H, int dk, int dv, int gate_mode, int io_dtype,
+                          int chunk_size, int segments, gdn_stream_t stream_)
 {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     int rc = validate(q, k, v, g, beta, state_in, state_out, out, B, T, H, dk, dv, gate_mode,
                       io_dtype, true, false);
     if (rc != GDN_OK) return rc;
+    if (segments < 0) return GDN_ERR_INVALID_ARG;
     const bool f32 = io_dtype == GDN_IO_F32;
     if (f32) {
         if (chunk_size != 0 && chunk_size != 1) return GDN_ERR_UNSUPPORTED;
+        if (segments > 1) return GDN_ERR_UNSUPPORTED;
     } else if (chunk_size != 0 && chunk_size != 1 && chunk_size != 64) {
         return GDN_ERR_UNSUPPORTED;
     }
+    if (segments > 1 && (chunk_size == 1 || dk != 128 || dv != 128)) return GDN_ERR_UNSUPPORTED;
     if (T == 0) {
         if (!state_out) return GDN_OK;
         const size_t st = (size_t)B * H * dk * dv * sizeof(float);
@@ -106,13 +112,31 @@ int gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* g
         return to_status(e);
     }
     gdn::Problem p{q, k, v, g, beta, state_in, state_out, out, B, T, H, dk, dv,
-                   gate_mode == GDN_GATE_CHANNEL, f32, true};
+                   gate_mode == GDN_GATE_CHANNEL, f32, true, segments};
     if (!f32 && chunk_size != 1) {
         cudaError_t e = gdn::launch_chunk_sm100(p, stream);
         if (e != cudaErrorNotSupported) return to_status(e);
         if (chunk_size == 64) return GDN_ERR_UNSUPPORTED;
     }
     return to_status(gdn::launch_recurrent(p, stream));
+}
+
+int gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* g,
+                     const float* beta, const float* state_in, void* out, float* state_out,
+                     int B, int T, int H, int dk, int dv, int gate_mode, int io_dtype,
+                     int chunk_size, gdn_stream_t stream)
+{
+    return chunk_fwd_impl(q, k, v, g, beta, state_in, out, state_out, B, T, H, dk, dv, gate_mode,
+                          io_dtype, chunk_size, 0, stream);
+}
+
+int gdn_chunk_fwd_segments(const void* q, const void* k, const void* v, const float* g,
+                           const float* beta, const float* state_in, void* out, float* state_out,
+                           int B, int T, int H, int dk, int dv, int gate_mode, int num_segments,
+                           gdn_stream_t stream)
+{
+    return chunk_fwd_impl(q, k, v, g, beta, state_in, out, state_out, B, T, H, dk, dv, gate_mode,
+                          GDN_IO_BF16, 0, num_segments, stream);
 }
 
 int gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,

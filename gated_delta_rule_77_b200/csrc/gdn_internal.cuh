@@ -25,6 +25,7 @@ struct Problem {
     bool per_channel;
     bool io_f32;             // q, k, v in fp32 (else bf16)
     bool out_f32;            // out in fp32 (else bf16)
+    int segments = 0;        // chunk path: time segments per (b, h); 0 = automatic
 };
 
 // Token-serial fused recurrence (decode, and the fp32 / fallback prefill).

@@ -116,6 +116,27 @@ GDN_API int gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const 
                      int chunk_size, gdn_stream_t stream);
 
 /*
+ * gdn_chunk_fwd_segments -- gdn_chunk_fwd (bf16 q, k, v) with explicit
+ * sequence parallelism.  The state map of a stretch of tokens is affine,
+ * S_end = M S_start + S_end(0) (it follows from the formula of section 2.1),
+ * so a long sequence can be cut into num_segments time segments that run in
+ * parallel: every segment computes its end state from a zero start and its
+ * dk x dk transition M, a serial combine gives each segment its true start
+ * state, and the segments run again from those states for the outputs.
+ * This costs three chunk passes instead of one and pays off when B * H is
+ * small against the SM count and T is long.
+ *   num_segments 0 = automatic (what gdn_chunk_fwd does), 1 = none,
+ *                n > 1 = n segments (at most one per 64-token chunk;
+ *                dk = dv = 128 only).
+ * Scratch: 2 * B * n * H * dk * dv * 4 bytes, stream-ordered on `stream`
+ * (GDN_ERR_NOMEM if it cannot be had).  Other arguments as gdn_chunk_fwd.
+ */
+GDN_API int gdn_chunk_fwd_segments(const void* q, const void* k, const void* v, const float* g,
+                                   const float* beta, const float* state_in, void* out,
+                                   float* state_out, int B, int T, int H, int dk, int dv,
+                                   int gate_mode, int num_segments, gdn_stream_t stream);
+
+/*
  * gdn_recurrent_step -- one decode step for B sequences and H heads.
  *
  *   q, k      [B, H, dk] bf16;   v [B, H, dv] bf16

@@ -105,3 +105,13 @@ def test_scalar_gate_and_beta_need_only_4_byte_alignment(lib):
     # With state_in = None the call is rejected for that reason, not alignment.
     assert _step(lib, gate=0, g=A + 192 * MB + 4, beta=A + 256 * MB + 12, s_in=None) == \
         gdn.GDN_ERR_INVALID_ARG
+
+
+def test_segments_entry_point_rejects(lib):
+    c = ctypes.c_void_p
+    call = lambda segs, dk=128, B=1: lib.gdn_chunk_fwd_segments(  # noqa: E731
+        c(A), c(A + 64 * MB), c(A + 128 * MB), c(A + 192 * MB), c(A + 256 * MB), None,
+        c(A + 384 * MB), c(A + 448 * MB), B, 16, 1, dk, 128, 0, segs, None)
+    assert call(-1) == gdn.GDN_ERR_INVALID_ARG
+    assert call(4, dk=64) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(4, B=0) == gdn.GDN_ERR_INVALID_ARG
