@@ -28,13 +28,15 @@ GDN_ERR_MISALIGNED = -3
 GDN_ERR_CUDA = -4
 GDN_ERR_NOMEM = -5
 GDN_ERR_TIMEOUT = -6
+GDN_ERR_SCRATCH_LIMIT = -7
 GATE_SCALAR = 0
 GATE_CHANNEL = 1
 IO_BF16 = 0
 IO_F32 = 1
 
-SYMBOLS = ("gdn_chunk_fwd", "gdn_chunk_fwd_ex", "gdn_chunk_fwd_segments", "gdn_recurrent_step",
-           "gdn_recurrent_step_ex", "gdn_check", "gdn_status_string")
+SYMBOLS = ("gdn_chunk_fwd", "gdn_chunk_fwd_ex", "gdn_chunk_fwd_segments",
+           "gdn_chunk_fwd_segments_noalloc", "gdn_recurrent_step", "gdn_recurrent_step_ex",
+           "gdn_check", "gdn_status_string")
 
 _lib = None
 
@@ -57,6 +59,8 @@ def load() -> ctypes.CDLL:
     lib.gdn_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i, i, i, i, i, i, vp]
     lib.gdn_chunk_fwd_ex.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i, i, i, i, i, i, i, i, vp]
     lib.gdn_chunk_fwd_segments.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i, i, i, i, i, i, i, vp]
+    lib.gdn_chunk_fwd_segments_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i, i, i, i, i, i, i,
+                                                   vp]
     lib.gdn_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, vp]
     lib.gdn_recurrent_step_ex.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, i, vp]
     lib.gdn_check.argtypes = [vp]

@@ -55,6 +55,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 #include "gdn_internal.cuh"
 #include "sm100_util.cuh"
 
@@ -978,7 +980,90 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
     return e != cudaSuccess ? e : ef;
 }
 
+// ---- no-allocation variant of the segment-parallel path ---------------------
+// Scratch for callers that must not allocate: a fixed array in the library's
+// device image (every GPU that loads the library holds it until exit).
+// Host code may not use the array's name as a device address; the address is
+// looked up with cudaGetSymbolAddress once per device (see below).
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+
+cudaError_t noalloc_scratch_address(float** ptr) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    constexpr int kMaxDevices = 128;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    static std::mutex mu;
+    static float* addr[kMaxDevices] = {};
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {   // first call on this device, device current
+        void* a = nullptr;
+        e = cudaGetSymbolAddress(&a, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        addr[dev] = static_cast<float*>(a);
+    }
+    *ptr = addr[dev];
+    return cudaSuccess;
+}
+
+template <bool CHANNEL>
+cudaError_t launch_noalloc(const Problem& p, cudaStream_t stream, bool* over_limit) {
+    *over_limit = false;
+    const int nchunks = (p.T + C - 1) / C;
+    int nseg = choose_segments(p.segments, p.B * p.H, nchunks);
+    const int seg_len = ((nchunks + nseg - 1) / nseg) * C;
+    if (nseg > 1) nseg = (p.T + seg_len - 1) / seg_len;
+    const size_t slab = (size_t)p.B * nseg * p.H * D * D;
+    if (nseg > 1 && 2 * slab > kNoAllocScratchFloats) {
+        *over_limit = true;          // rejected before anything is launched
+        return cudaErrorInvalidValue;
+    }
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(chunk_fwd_kernel<CHANNEL>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, p.q, p.H, p.T, p.B) || !make_map(&mk, p.k, p.H, p.T, p.B) ||
+        !make_map(&mv, p.v, p.H, p.T, p.B))
+        return cudaErrorInvalidValue;
+    float* out = static_cast<float*>(p.out);
+    if (nseg <= 1) {
+        Params prm{p.g, p.beta, p.state_in, p.state_out, nullptr, out, p.T, p.H, p.B,
+                   1, nchunks * C, 1, 1};
+        chunk_fwd_kernel<CHANNEL><<<p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, prm);
+        return cudaGetLastError();
+    }
+    float* ws = nullptr;
+    cudaError_t e = noalloc_scratch_address(&ws);
+    if (e != cudaSuccess) return e;
+    // Every scratch element read below is written earlier in this call (pass
+    // 1 writes all end states and transitions), so nothing is cleared.
+    float* seg_states = ws;
+    float* trans = ws + slab;
+    Params p1{p.g, p.beta, nullptr, seg_states, trans, nullptr, p.T, p.H, p.B, nseg, seg_len, 1, nseg};
+    chunk_fwd_kernel<CHANNEL><<<2 * p.B * nseg * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, p1);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    combine_segments_kernel<<<p.B * p.H * (D / CB_COLS), 256, 0, stream>>>(
+        seg_states, trans, p.state_in, p.state_out, p.H, nseg);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    Params p2{p.g, p.beta, seg_states, nullptr, nullptr, out, p.T, p.H, p.B, nseg, seg_len, nseg, 1};
+    chunk_fwd_kernel<CHANNEL><<<p.B * nseg * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, p2);
+    return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_chunk_sm100_noalloc(const Problem& p, cudaStream_t stream, bool* over_limit) {
+    *over_limit = false;
+    if (p.io_f32 || !p.out_f32 || p.dk != D || p.dv != D) return cudaErrorNotSupported;
+    return p.per_channel ? launch_noalloc<true>(p, stream, over_limit)
+                         : launch_noalloc<false>(p, stream, over_limit);
+}
 
 cudaError_t launch_chunk_sm100(const Problem& p, cudaStream_t stream) {
     if (p.io_f32 || !p.out_f32 || p.dk != D || p.dv != D) return cudaErrorNotSupported;

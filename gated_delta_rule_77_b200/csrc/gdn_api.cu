@@ -147,6 +147,33 @@ int gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
                             gate_mode, GDN_IO_BF16, 0, stream);
 }
 
+int gdn_chunk_fwd_segments_noalloc(const void* q, const void* k, const void* v, const float* g,
+                                   const float* beta, const float* state_in, void* out,
+                                   float* state_out, int B, int T, int H, int dk, int dv,
+                                   int gate_mode, int num_segments, gdn_stream_t stream_)
+{
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    int rc = validate(q, k, v, g, beta, state_in, state_out, out, B, T, H, dk, dv, gate_mode,
+                      GDN_IO_BF16, true, false);
+    if (rc != GDN_OK) return rc;
+    if (num_segments < 0) return GDN_ERR_INVALID_ARG;
+    if (dk != 128 || dv != 128) return GDN_ERR_UNSUPPORTED;
+    if (T == 0) {
+        if (!state_out || state_in == state_out) return GDN_OK;
+        const size_t st = (size_t)B * H * dk * dv * sizeof(float);
+        cudaError_t e = state_in
+            ? cudaMemcpyAsync(state_out, state_in, st, cudaMemcpyDeviceToDevice, stream)
+            : cudaMemsetAsync(state_out, 0, st, stream);
+        return to_status(e);
+    }
+    gdn::Problem p{q, k, v, g, beta, state_in, state_out, out, B, T, H, dk, dv,
+                   gate_mode == GDN_GATE_CHANNEL, false, true, num_segments};
+    bool over_limit = false;
+    cudaError_t e = gdn::launch_chunk_sm100_noalloc(p, stream, &over_limit);
+    if (over_limit) return GDN_ERR_SCRATCH_LIMIT;
+    return to_status(e);
+}
+
 int gdn_recurrent_step_ex(const void* q, const void* k, const void* v, const float* g,
                           const float* beta, const float* state_in, float* state_out,
                           void* out, int B, int H, int dk, int dv, int gate_mode,
@@ -188,6 +215,7 @@ const char* gdn_status_string(int status)
         case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
         case GDN_ERR_NOMEM: return "GDN_ERR_NOMEM";
         case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+        case GDN_ERR_SCRATCH_LIMIT: return "GDN_ERR_SCRATCH_LIMIT";
         default: return "GDN_ERR_UNKNOWN";
     }
 }

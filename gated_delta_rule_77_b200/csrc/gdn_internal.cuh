@@ -35,6 +35,12 @@ cudaError_t launch_recurrent(const Problem& p, cudaStream_t stream);
 // Returns cudaErrorNotSupported for shapes it does not handle.
 cudaError_t launch_chunk_sm100(const Problem& p, cudaStream_t stream);
 
+// The segment-parallel chunk path with its scratch taken from a fixed
+// device array of kNoAllocScratchFloats floats instead of an allocation.
+// Sets *over_limit (and launches nothing) when the call needs more.
+constexpr size_t kNoAllocScratchFloats = size_t(8) * 1024 * 1024;   // 32 MiB
+cudaError_t launch_chunk_sm100_noalloc(const Problem& p, cudaStream_t stream, bool* over_limit);
+
 // Device status word written by kernels that abandon a bounded wait.
 cudaError_t read_and_clear_status(unsigned int* status, cudaStream_t stream);
 

@@ -65,7 +65,8 @@ typedef enum {
     GDN_ERR_MISALIGNED = -3,    /* a pointer is not 16-byte aligned           */
     GDN_ERR_CUDA = -4,          /* a CUDA runtime call or launch failed       */
     GDN_ERR_NOMEM = -5,         /* stream-ordered scratch allocation failed   */
-    GDN_ERR_TIMEOUT = -6        /* a kernel abandoned a bounded wait          */
+    GDN_ERR_TIMEOUT = -6,       /* a kernel abandoned a bounded wait          */
+    GDN_ERR_SCRATCH_LIMIT = -7  /* needs more than the fixed scratch array    */
 } gdn_status;
 
 enum { GDN_GATE_SCALAR = 0, GDN_GATE_CHANNEL = 1 };
@@ -135,6 +136,43 @@ GDN_API int gdn_chunk_fwd_segments(const void* q, const void* k, const void* v, 
                                    const float* beta, const float* state_in, void* out,
                                    float* state_out, int B, int T, int H, int dk, int dv,
                                    int gate_mode, int num_segments, gdn_stream_t stream);
+
+/*
+ * gdn_chunk_fwd_segments_noalloc -- gdn_chunk_fwd_segments for callers that
+ * must not have the library allocate device memory.  The source pages have
+ * no counterpart to this entry point: it is a convenience of this library's
+ * interface, computing exactly what gdn_chunk_fwd_segments computes.
+ *
+ * Who needs it: callers whose device memory already belongs to another
+ * allocator (e.g. a framework pool that has reserved all free memory, so a
+ * cudaMallocAsync inside the library could fail or fragment it), and callers
+ * whose step must never stall in an allocator or fail for lack of memory
+ * half-way through.  This variant calls no allocation or free routine: its
+ * scratch is a fixed 32 MiB array compiled into the library, which every GPU
+ * that loads libgdn holds until the process exits.
+ *
+ * Limit: the segmented path needs 2 * B * n * H * dk * dv * 4 bytes for n
+ * time segments (n as chosen by gdn_chunk_fwd_segments for num_segments);
+ * with dk = dv = 128 that is B * n * H <= 256.  A larger call returns
+ * GDN_ERR_SCRATCH_LIMIT and launches nothing.  With n = 1 no scratch is used.
+ * bf16 q, k, v and dk = dv = 128 only (else GDN_ERR_UNSUPPORTED).
+ *
+ * First call: the first call on a device, with that device current, looks up
+ * the device address of the array (once per device); make that first call
+ * before any stream capture.
+ *
+ * Sharing: all calls use the same array and leave their data in it.  A call
+ * writes every scratch element before it reads it, so nothing is cleared
+ * between calls -- but two calls whose kernels may run at the same time on
+ * one GPU (different streams without ordering between them) race on the
+ * array and give wrong results.  Order such calls on one stream.
+ * Other arguments as gdn_chunk_fwd_segments.
+ */
+GDN_API int gdn_chunk_fwd_segments_noalloc(const void* q, const void* k, const void* v,
+                                           const float* g, const float* beta,
+                                           const float* state_in, void* out, float* state_out,
+                                           int B, int T, int H, int dk, int dv, int gate_mode,
+                                           int num_segments, gdn_stream_t stream);
 
 /*
  * gdn_recurrent_step -- one decode step for B sequences and H heads.

@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 def test_status_strings(lib):
     for code, name in [(0, "GDN_OK"), (-1, "GDN_ERR_INVALID_ARG"), (-2, "GDN_ERR_UNSUPPORTED"),
                        (-3, "GDN_ERR_MISALIGNED"), (-4, "GDN_ERR_CUDA"), (-5, "GDN_ERR_NOMEM"),
-                       (-6, "GDN_ERR_TIMEOUT"), (7, "GDN_ERR_UNKNOWN")]:
+                       (-6, "GDN_ERR_TIMEOUT"), (-7, "GDN_ERR_SCRATCH_LIMIT"), (7, "GDN_ERR_UNKNOWN")]:
         assert gdn.status_string(code) == name
 
 
