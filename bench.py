@@ -373,7 +373,7 @@ def run_decode(gdn, dev, stream, peaks, world, rank, steps: int = 20, warmup: in
     sink = torch.empty((), dtype=torch.float32, device=dev)
     times = []
     for i in range(warmup + steps):
-        torch.sum(flush, out=sink)
+        torch.sum(flush, dim=0, out=sink)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
