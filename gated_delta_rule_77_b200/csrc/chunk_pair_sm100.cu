@@ -1,0 +1,752 @@
+// chunk_pair_sm100.cu -- chunkwise prefill with the work of one (batch, head)
+// split across a cluster of two CTAs on two SMs.
+//
+// Same chunk algebra as chunk_sm100.cu (Atomic-GDN2 model card, section 2.1;
+// chunkwise mode of the "Gated DeltaNet" entity trail, finding of
+// 2026-07-29):
+//   A_rj = b_r k_r^T Diag(exp(G_r - G_j)) k_j (j < r),  T' = (I + A)^{-1} Diag(b)
+//   P_rj = q_r^T Diag(exp(G_r - G_j)) k_j (j <= r)
+//   U = T' V - T' (K * E) S,  O = (Q * E) S + P U,  S <- Diag(E_last) S + (K * D)^T U
+// A, P and T' depend on the chunk's own inputs only; U, O and the new S
+// depend on the state.  The two halves run on different SMs and overlap:
+//
+//   CTA 0 ("prep"):  gate prep, X = [K*F; Q*F](K/F)^T on tcgen05, A and P,
+//                    the fp32 triangular solve, T' and P as bf16 hi + lo;
+//                    hands the 32 KB of T' and P to CTA 1 with a bulk copy
+//                    into CTA 1's shared memory (no multicast), then moves on
+//                    to the next chunk.
+//   CTA 1 ("chain"): owns the fp32 state; gate prep for E and D, the derived
+//                    operands K*E, Q*E, K*D, and the state-dependent products
+//                    W^T, U^T, O^T and SN; writes the outputs.
+//
+// Hand-off: CTA 1's "full" mbarrier (armed by CTA 0 with a remote
+// arrive.expect_tx, completed by the bulk copy's byte count) and CTA 0's
+// "empty" mbarrier (a remote arrive from CTA 1 once the products that read the
+// slot are complete).  CTA 0 therefore works on chunk c + 1 while CTA 1 works
+// on chunk c.  Every wait is bounded (kWaitBudgetNs); on expiry a CTA records
+// it in its status word, stops, drains its own copies and returns.
+//
+// Precision and operand formats are those of chunk_sm100.cu (bf16 hi + lo for
+// the factored A/P operands, T', P, U and K*D; fp16 for S, W and Q*E; fp32
+// accumulation in TMEM; fp32 output).
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "chunk_common.cuh"
+#include "gdn_internal.cuh"
+#include "sm100_util.cuh"
+
+namespace gdn {
+
+__device__ unsigned int g_pair_status_word = 0;
+
+namespace {
+
+using namespace sm100;
+using namespace chunk;
+
+constexpr int C = 64;
+constexpr int D = 128;
+constexpr int NT = 256;
+
+// ---- CTA 0 (prep) shared memory -----------------------------------------------
+constexpr uint32_t P_IN = 0;                  // 32 KB raw K, Q [half][K 64 | Q 64][128 B]
+constexpr uint32_t P_X = 32768;               // 112 KB:
+constexpr uint32_t P_AH = P_X;                //   X operands (per-channel): 32 KB
+constexpr uint32_t P_AL = P_X + 32768;        //   32 KB
+constexpr uint32_t P_C0H = P_X + 65536;       //   8 KB
+constexpr uint32_t P_C0L = P_X + 73728;       //   8 KB
+constexpr uint32_t P_C1H = P_X + 81920;       //   16 KB
+constexpr uint32_t P_C1L = P_X + 98304;       //   16 KB
+constexpr uint32_t P_STAGE = P_X;             //   after X: T' hi, T' lo, P hi, P lo (4 x 8 KB)
+constexpr uint32_t P_A = P_X + 32768;         //   16 KB A fp32 (fidx layout)
+constexpr uint32_t P_T = P_X + 49152;         //   16 KB T fp32 row-major
+constexpr uint32_t P_Y = P_X + 65536;         //   3 KB solve scratch
+constexpr uint32_t P_SMALL = P_X + 114688;
+constexpr uint32_t P_GAM = P_SMALL;           // 64 f32
+constexpr uint32_t P_BETA = P_GAM + 256;      // 64 f32
+constexpr uint32_t P_REF0 = P_BETA + 256;     // 128 f32
+constexpr uint32_t P_REF1 = P_REF0 + 512;     // 128 f32
+constexpr uint32_t P_BAR = P_REF1 + 512;      // tma, mma, empty
+constexpr uint32_t P_TMEM = P_BAR + 24;
+constexpr uint32_t P_USED = P_TMEM + 8;
+
+// ---- CTA 1 (chain) shared memory ----------------------------------------------
+constexpr uint32_t C_IN = 0;                  // 32 KB raw K, Q
+constexpr uint32_t C_V = 32768;               // 16 KB raw V
+constexpr uint32_t C_S = 49152;               // 32 KB S fp16 [j half][128 i][64 j]
+constexpr uint32_t C_KE = 81920;              // 16 KB K*E bf16; then W^T fp16 [128 i][64 r]
+constexpr uint32_t C_QE = 98304;              // 16 KB Q*E fp16
+constexpr uint32_t C_KDH = 114688;            // 16 KB K*D bf16 hi
+constexpr uint32_t C_KDL = 131072;            // 16 KB K*D bf16 lo
+constexpr uint32_t C_UH = 147456;             // 16 KB U^T hi [128 j][64 r]
+constexpr uint32_t C_UL = 163840;             // 16 KB U^T lo
+constexpr uint32_t C_SLOT = 180224;           // 32 KB T' hi, T' lo, P hi, P lo (from CTA 0)
+constexpr uint32_t C_TH = C_SLOT, C_TL = C_SLOT + 8192, C_PH = C_SLOT + 16384, C_PL = C_SLOT + 24576;
+constexpr uint32_t C_SMALL = C_SLOT + 32768;
+constexpr uint32_t C_GAM = C_SMALL;           // 64 f32
+constexpr uint32_t C_LAST = C_GAM + 256;      // 128 f32
+constexpr uint32_t C_BAR = C_LAST + 512;      // tma_kq, tma_v, mma, full
+constexpr uint32_t C_TMEM = C_BAR + 32;
+constexpr uint32_t C_USED = C_TMEM + 8;
+
+constexpr uint32_t SLOT_BYTES = 32768;
+constexpr uint32_t SMEM_BYTES = (P_USED > C_USED ? P_USED : C_USED) + 1024;
+
+// TMEM columns.  CTA 0: X (128 rows x up to 96).  CTA 1: W^T, U^T, O^T, SN.
+constexpr uint32_t TM_X = 0;
+constexpr uint32_t TM_WT = 0, TM_UT = 64, TM_OT = 128, TM_SN = 256;
+
+struct PairParams {
+    const float* g;            // [B, T, H] or [B, T, H, D]
+    const float* beta;         // [B, T, H]
+    const float* state_in;     // [B, H, D, D] or null
+    float* state_out;          // [B, H, D, D] or null
+    float* out;                // [B, T, H, D] fp32
+    int T, H;
+};
+
+template <bool CHANNEL>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
+chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const PairParams p)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(smem);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int quad = warp & 3;
+    const int half = warp >> 2;
+    const uint32_t rank = cluster_ctarank();
+    const int T = p.T;
+    const int H = p.H;
+    const int pair = blockIdx.x >> 1;
+    const int h = pair % H;
+    const int b = pair / H;
+    const int nchunks = (T + C - 1) / C;
+    // Gate-prep / tile-building ownership (see chunk_sm100.cu): channel chunk
+    // ck of 8 channels, lane tg owns tokens tg + 16 u.
+    const int ck = 2 * warp + (lane >> 4);
+    const int tg = lane & 15;
+    const int ckh = ck >> 3;
+    const int ckc = ck & 7;
+    bool ok = true;
+
+    // Both CTAs: barriers and TMEM, then a cluster barrier so that no remote
+    // arrive or copy can reach an uninitialised barrier.
+    const uint32_t bar0 = sbase + (rank == 0 ? P_BAR : C_BAR);
+    if (tid == 0) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        if (rank == 1) prefetch_tensormap(&tm_v);
+        for (int i = 0; i < (rank == 0 ? 3 : 4); ++i) mbar_init(bar0 + 8 * i, 1);
+        fence_mbar_init();
+    }
+    const uint32_t tmem_cols = rank == 0 ? 128 : 512;
+    if (warp == 0) {
+        tmem_alloc(sbase + (rank == 0 ? P_TMEM : C_TMEM), tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<uint32_t*>(smem + (rank == 0 ? P_TMEM : C_TMEM));
+    cluster_sync();
+
+    uint32_t mma_phase = 0;
+    auto mma_sync = [&]() {
+        ok = ok && mbar_wait(bar0 + 8 * (rank == 0 ? 1 : 2), mma_phase, &g_pair_status_word);
+        mma_phase ^= 1;
+        tc_fence_after();
+    };
+
+    // Per-channel cumulative log-decay of this thread's 4 tokens x 8 channels
+    // (registers); block references / last token stored by lane tg = 15.
+    auto gate_channel = [&](int t0, long tk0, float (&gam)[4][8], float* ref0, float* ref1,
+                            float* last) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int r = tg + 16 * u;
+            if (t0 + r < T) {
+                const float4* src = reinterpret_cast<const float4*>(p.g + (tk0 + (long)r * H) * D + 8 * ck);
+                const float4 a = src[0], c = src[1];
+                gam[u][0] = a.x; gam[u][1] = a.y; gam[u][2] = a.z; gam[u][3] = a.w;
+                gam[u][4] = c.x; gam[u][5] = c.y; gam[u][6] = c.z; gam[u][7] = c.w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) gam[u][e] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float x = __shfl_up_sync(0xffffffffu, gam[u][e], o, 16);
+                    if (tg >= o) gam[u][e] += x;
+                }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            float off = 0.f;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float tot = __shfl_sync(0xffffffffu, gam[u][e], 15, 16);
+                gam[u][e] += off;
+                off += tot;
+            }
+        }
+        if (t0 + C < T) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int r = C + tg + 16 * u;
+                if (t0 + r < T) prefetch_l2(p.g + (tk0 + (long)r * H) * D + 8 * ck);
+            }
+        }
+        if (tg == 15) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                if (ref0) ref0[8 * ck + e] = gam[0][e];
+                if (ref1) ref1[8 * ck + e] = gam[2][e];
+                if (last) last[8 * ck + e] = gam[3][e];
+            }
+        }
+    };
+    // Scalar gate: warp 0 scans the chunk's 64 values of g into sGam (and
+    // copies beta when sBeta is given).
+    auto gate_scalar = [&](int t0, long tk0, float* sGam, float* sBeta) {
+        if (warp != 0) return;
+        float b0 = 0.f, b1 = 0.f, g0 = 0.f, g1 = 0.f;
+        if (t0 + lane < T) {
+            if (sBeta) b0 = p.beta[tk0 + (long)lane * H];
+            if (!CHANNEL) g0 = p.g[tk0 + (long)lane * H];
+        }
+        if (t0 + 32 + lane < T) {
+            if (sBeta) b1 = p.beta[tk0 + (long)(32 + lane) * H];
+            if (!CHANNEL) g1 = p.g[tk0 + (long)(32 + lane) * H];
+        }
+        if (sBeta) {
+            sBeta[lane] = b0;
+            sBeta[32 + lane] = b1;
+        }
+        if (!CHANNEL) {
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float x0 = __shfl_up_sync(0xffffffffu, g0, o);
+                const float x1 = __shfl_up_sync(0xffffffffu, g1, o);
+                if (lane >= o) { g0 += x0; g1 += x1; }
+            }
+            g1 += __shfl_sync(0xffffffffu, g0, 31);
+            sGam[lane] = g0;
+            sGam[32 + lane] = g1;
+        }
+    };
+
+    if (rank == 0) {
+        // =========================================================== prep CTA ===
+        float* sGam = reinterpret_cast<float*>(smem + P_GAM);
+        float* sBeta = reinterpret_cast<float*>(smem + P_BETA);
+        float* sRef0 = reinterpret_cast<float*>(smem + P_REF0);
+        float* sRef1 = reinterpret_cast<float*>(smem + P_REF1);
+        float* sA = reinterpret_cast<float*>(smem + P_A);
+        float* sT = reinterpret_cast<float*>(smem + P_T);
+        float* sY = reinterpret_cast<float*>(smem + P_Y);
+        const uint32_t bar_tma = sbase + P_BAR, bar_empty = sbase + P_BAR + 16;
+        // CTA 1's slot and "full" barrier, as cluster addresses.
+        const uint32_t peer_slot = mapa_shared(sbase + C_SLOT, 1);
+        const uint32_t peer_full = mapa_shared(sbase + C_BAR + 24, 1);
+        auto issue_kq = [&](int chunk) {
+            const int t0 = chunk * C;
+            mbar_expect_tx(bar_tma, 2 * 16384);
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                tma_load_4d(sbase + P_IN + hf * 16384, &tm_k, hf * 64, h, t0, b, bar_tma);
+                tma_load_4d(sbase + P_IN + hf * 16384 + 8192, &tm_q, hf * 64, h, t0, b, bar_tma);
+            }
+        };
+        if (tid == 0 && nchunks > 0) issue_kq(0);
+        int kq_waited = -1;
+        bool copy_pending = false;
+
+        for (int ci = 0; ci < nchunks; ++ci) {
+            const int t0 = ci * C;
+            const long tk0 = ((long)b * T + t0) * H + h;
+            float gam[4][8];
+            if (CHANNEL) gate_channel(t0, tk0, gam, sRef0, sRef1, nullptr);
+            gate_scalar(t0, tk0, sGam, sBeta);
+            ok = ok && mbar_wait(bar_tma, ci & 1, &g_pair_status_word);
+            kq_waited = ci;
+            if (tid == 0 && copy_pending) {      // staging (in the X region) free again
+                bulk_wait_read_all();
+                copy_pending = false;
+            }
+            if (__syncthreads_or(!ok)) break;
+
+            if (CHANNEL) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int r = tg + 16 * u;
+                    const float* ref = r < 32 ? sRef0 : sRef1;
+                    float kf[8], qf[8];
+                    load_bf16x8(smem + P_IN + ckh * 16384 + swz(r, ckc), kf);
+                    load_bf16x8(smem + P_IN + ckh * 16384 + 8192 + swz(r, ckc), qf);
+                    float kr[8], qr[8], kc[8], kc1[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float x = gam[u][e] - ref[8 * ck + e];
+                        const float F = __expf(x);
+                        const float Fi = __expf(-x);
+                        kr[e] = kf[e] * F;
+                        qr[e] = qf[e] * F;
+                        kc[e] = kf[e] * Fi;
+                        kc1[e] = r < 32 ? kf[e] * __expf(sRef1[8 * ck + e] - gam[u][e]) : kc[e];
+                    }
+                    const uint32_t o128 = ckh * 16384 + swz(r, ckc);
+                    const uint32_t o128q = ckh * 16384 + swz(64 + r, ckc);
+                    store_split(smem + P_AH + o128, smem + P_AL + o128, kr);
+                    store_split(smem + P_AH + o128q, smem + P_AL + o128q, qr);
+                    if (r < 32) {
+                        const uint32_t o32 = ckh * 4096 + swz(r, ckc);
+                        store_split(smem + P_C0H + o32, smem + P_C0L + o32, kc);
+                    }
+                    const uint32_t o64 = ckh * 8192 + swz(r, ckc);
+                    store_split(smem + P_C1H + o64, smem + P_C1L + o64, kc1);
+                }
+                fence_async_smem();
+                __syncthreads();
+            }
+            if (tid == 0) {
+                tc_fence_after();
+                if (CHANNEL) {
+                    const uint32_t id0 = idesc_bf16(128, 32, false, false);
+                    const uint32_t id1 = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t ka = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        const uint32_t k0 = (ks >> 2) * 4096 + (ks & 3) * 32;
+                        const uint32_t k1 = (ks >> 2) * 8192 + (ks & 3) * 32;
+                        const uint64_t ah = sdesc_sw128(sbase + P_AH + ka, 16, 1024);
+                        const uint64_t al = sdesc_sw128(sbase + P_AL + ka, 16, 1024);
+                        const uint64_t b0h = sdesc_sw128(sbase + P_C0H + k0, 16, 1024);
+                        const uint64_t b0l = sdesc_sw128(sbase + P_C0L + k0, 16, 1024);
+                        const uint64_t b1h = sdesc_sw128(sbase + P_C1H + k1, 16, 1024);
+                        const uint64_t b1l = sdesc_sw128(sbase + P_C1L + k1, 16, 1024);
+                        mma_bf16(tmem + TM_X, ah, b0h, id0, ks > 0);
+                        mma_bf16(tmem + TM_X, ah, b0l, id0, 1);
+                        mma_bf16(tmem + TM_X, al, b0h, id0, 1);
+                        mma_bf16(tmem + TM_X + 32, ah, b1h, id1, ks > 0);
+                        mma_bf16(tmem + TM_X + 32, ah, b1l, id1, 1);
+                        mma_bf16(tmem + TM_X + 32, al, b1h, id1, 1);
+                    }
+                } else {
+                    const uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint64_t a = sdesc_sw128(sbase + P_IN + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                        mma_bf16(tmem + TM_X, a, a, id, ks > 0);
+                    }
+                }
+                mma_commit(sbase + P_BAR + 8);
+            }
+            mma_sync();
+            if (__syncthreads_or(!ok)) break;
+            // Raw K, Q and the X operands are consumed: prefetch the next chunk.
+            if (tid == 0 && ci + 1 < nchunks) issue_kq(ci + 1);
+
+            // A and P from X (see chunk_sm100.cu); P as bf16 hi + lo into the staging.
+            {
+                const int L = quad * 32 + lane;
+                const bool is_p = L >= 64;
+                const int r = L & 63;
+                float x[32];
+                const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+                bool zero = false;
+                if (CHANNEL) {
+                    if (r < 32) {
+                        if (half == 0) tmem_ld32(lane_base + TM_X, x); else zero = true;
+                    } else {
+                        tmem_ld32(lane_base + TM_X + 32 + half * 32, x);
+                    }
+                } else {
+                    tmem_ld32(lane_base + TM_X + half * 32, x);
+                }
+                tmem_wait_ld();
+                if (zero) {
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) x[jj] = 0.f;
+                }
+                const float br = sBeta[r];
+                const float Gr = CHANNEL ? 0.f : sGam[r];
+                const int j0 = half * 32;
+                if (!is_p) {
+#pragma unroll
+                    for (int j4 = 0; j4 < 8; ++j4) {
+                        float a[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = j0 + 4 * j4 + e;
+                            float val = 0.f;
+                            if (j < r) val = br * x[4 * j4 + e] * (CHANNEL ? 1.f : __expf(Gr - sGam[j]));
+                            a[e] = val;
+                        }
+                        *reinterpret_cast<float4*>(&sA[fidx(r, j0 + 4 * j4)]) = make_float4(a[0], a[1], a[2], a[3]);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        float pv[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int j = j0 + 8 * c + e;
+                            float val = 0.f;
+                            if (j <= r) val = x[8 * c + e] * (CHANNEL ? 1.f : __expf(Gr - sGam[j]));
+                            pv[e] = val;
+                        }
+                        const int cc = half * 4 + c;
+                        store_split(smem + P_STAGE + 16384 + swz(r, cc), smem + P_STAGE + 24576 + swz(r, cc), pv);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncthreads();
+            solve_unit_lower64(sA, sT, sY, tid);
+            for (int e = tid; e < 512; e += NT) {
+                const int r = e >> 3, c = e & 7;
+                const float4 t0v = *reinterpret_cast<const float4*>(&sT[r * 64 + 8 * c]);
+                const float4 t1v = *reinterpret_cast<const float4*>(&sT[r * 64 + 8 * c + 4]);
+                const float tt[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
+                float tv[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int m = 8 * c + q;
+                    tv[q] = (m <= r) ? tt[q] * sBeta[m] : 0.f;
+                }
+                store_split(smem + P_STAGE + swz(r, c), smem + P_STAGE + 8192 + swz(r, c), tv);
+            }
+            fence_async_smem();          // staging written by threads -> read by the bulk copy
+            __syncthreads();
+            if (tid == 0) {
+                // Wait until CTA 1 has consumed the previous chunk's slot.
+                ok = ok && mbar_wait_cluster(bar_empty, (ci & 1) ^ 1, &g_pair_status_word);
+                if (ok) {
+                    mbar_arrive_expect_tx_remote(peer_full, SLOT_BYTES);
+                    bulk_copy_to_peer(peer_slot, sbase + P_STAGE, SLOT_BYTES, peer_full);
+                    bulk_commit();
+                    copy_pending = true;
+                }
+            }
+            if (__syncthreads_or(!ok)) break;
+        }
+        if (tid == 0) {
+            bulk_wait_all();                 // own copies complete before exit
+            if (!ok && kq_waited + 1 < nchunks)
+                mbar_wait(bar_tma, (kq_waited + 1) & 1, &g_pair_status_word);
+        }
+    } else {
+        // ========================================================== chain CTA ===
+        float* sGam = reinterpret_cast<float*>(smem + C_GAM);
+        float* sLast = reinterpret_cast<float*>(smem + C_LAST);
+        const uint32_t bar_kq = sbase + C_BAR, bar_v = sbase + C_BAR + 8;
+        const uint32_t bar_full = sbase + C_BAR + 24;
+        const uint32_t bar_mma = sbase + C_BAR + 16;
+        const uint32_t peer_empty = mapa_shared(sbase + P_BAR + 16, 0);
+
+        const int srow = quad * 32 + lane;
+        const int scol = half * 64;
+        float s[64];
+        const long DD = (long)D * D;
+        if (p.state_in) {
+            const float4* src = reinterpret_cast<const float4*>(p.state_in + ((long)b * H + h) * DD +
+                                                                (long)srow * D + scol);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                float4 t = src[c];
+                s[4 * c] = t.x; s[4 * c + 1] = t.y; s[4 * c + 2] = t.z; s[4 * c + 3] = t.w;
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) s[c] = 0.f;
+        }
+        auto write_state_f16 = [&]() {
+            uint8_t* dst = smem + C_S + half * 16384;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) store_f16x8(dst + swz(srow, c), &s[8 * c]);
+        };
+        write_state_f16();
+        auto issue_kq = [&](int chunk) {
+            const int t0 = chunk * C;
+            mbar_expect_tx(bar_kq, 2 * 16384);
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                tma_load_4d(sbase + C_IN + hf * 16384, &tm_k, hf * 64, h, t0, b, bar_kq);
+                tma_load_4d(sbase + C_IN + hf * 16384 + 8192, &tm_q, hf * 64, h, t0, b, bar_kq);
+            }
+        };
+        auto issue_v = [&](int chunk) {
+            const int t0 = chunk * C;
+            mbar_expect_tx(bar_v, 16384);
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf)
+                tma_load_4d(sbase + C_V + hf * 8192, &tm_v, hf * 64, h, t0, b, bar_v);
+        };
+        fence_async_smem();
+        __syncthreads();
+        if (tid == 0 && nchunks > 0) {
+            issue_kq(0);
+            issue_v(0);
+        }
+        int kq_waited = -1, v_waited = -1, full_waited = -1;
+
+        for (int ci = 0; ci < nchunks; ++ci) {
+            const int t0 = ci * C;
+            const long tk0 = ((long)b * T + t0) * H + h;
+            float gam[4][8];
+            if (CHANNEL) gate_channel(t0, tk0, gam, nullptr, nullptr, sLast);
+            gate_scalar(t0, tk0, sGam, nullptr);
+            ok = ok && mbar_wait(bar_kq, ci & 1, &g_pair_status_word);
+            kq_waited = ci;
+            if (__syncthreads_or(!ok)) break;
+
+            // K*E (bf16), Q*E (fp16), K*D (bf16 hi + lo).
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int r = tg + 16 * u;
+                float kf[8], qf[8], ke[8], qe[8], kd[8];
+                load_bf16x8(smem + C_IN + ckh * 16384 + swz(r, ckc), kf);
+                load_bf16x8(smem + C_IN + ckh * 16384 + 8192 + swz(r, ckc), qf);
+                if (CHANNEL) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float E = __expf(gam[u][e]);
+                        const float Dd = __expf(sLast[8 * ck + e] - gam[u][e]);
+                        ke[e] = kf[e] * E;
+                        qe[e] = qf[e] * E;
+                        kd[e] = kf[e] * Dd;
+                    }
+                } else {
+                    const float E = __expf(sGam[r]);
+                    const float Dd = __expf(sGam[C - 1] - sGam[r]);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        ke[e] = kf[e] * E;
+                        qe[e] = qf[e] * E;
+                        kd[e] = kf[e] * Dd;
+                    }
+                }
+                const uint32_t o64 = ckh * 8192 + swz(r, ckc);
+                store_bf16x8(smem + C_KE + o64, ke);
+                store_f16x8(smem + C_QE + o64, qe);
+                store_split(smem + C_KDH + o64, smem + C_KDL + o64, kd);
+            }
+            const float e_last = __expf(CHANNEL ? sLast[srow] : sGam[C - 1]);
+            fence_async_smem();
+            __syncthreads();
+            if (tid == 0 && ci + 1 < nchunks) issue_kq(ci + 1);   // raw K, Q consumed
+
+            // T' and P of this chunk from CTA 0; V of this chunk.
+            if (tid == 0) {
+                ok = ok && mbar_wait_cluster(bar_full, ci & 1, &g_pair_status_word);
+                full_waited = ci;
+            }
+            ok = ok && mbar_wait(bar_v, ci & 1, &g_pair_status_word);
+            v_waited = ci;
+            if (__syncthreads_or(!ok)) break;
+
+            if (tid == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, 64, true, false);
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {
+                    const uint32_t tb = part ? C_TL : C_TH;
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t bt = sdesc_sw128(sbase + tb + ks * 32, 16, 1024);
+                        const uint32_t acc = (part | ks) != 0;
+                        mma_bf16(tmem + TM_WT, sdesc_sw128(sbase + C_KE + ks * 2048, 8192, 1024), bt, id, acc);
+                        mma_bf16(tmem + TM_UT, sdesc_sw128(sbase + C_V + ks * 2048, 8192, 1024), bt, id, acc);
+                    }
+                }
+                mma_commit(bar_mma);
+            }
+            mma_sync();
+            if (__syncthreads_or(!ok)) break;
+            if (tid == 0 && ci + 1 < nchunks) issue_v(ci + 1);      // V consumed
+
+            {   // W^T -> fp16 [128 i][64 r] over the consumed K*E tile
+                float w[32];
+                tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + TM_WT + half * 32, w);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 4; ++c) store_f16x8(smem + C_KE + swz(srow, half * 4 + c), &w[8 * c]);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+
+            if (tid == 0) {
+                tc_fence_after();
+                const uint32_t id_u = idesc_f16(128, 64, true, true, true);
+                const uint32_t id_o = idesc_f16(128, 64, true, false);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint64_t a = sdesc_sw128(sbase + C_S + ks * 2048, 16384, 1024);
+                    mma_bf16(tmem + TM_UT, a, sdesc_sw128(sbase + C_KE + ks * 2048, 8192, 1024), id_u, 1);
+                    const uint64_t bq = sdesc_sw128(sbase + C_QE + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+                    mma_bf16(tmem + TM_OT, a, bq, id_o, ks > 0);
+                }
+                mma_commit(bar_mma);
+            }
+            mma_sync();
+            if (__syncthreads_or(!ok)) break;
+
+            {   // U^T -> bf16 hi + lo [128 j][64 r]
+                float u[32];
+                tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + TM_UT + half * 32, u);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    store_split(smem + C_UH + swz(srow, half * 4 + c), smem + C_UL + swz(srow, half * 4 + c),
+                                &u[8 * c]);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+
+            if (tid == 0) {
+                tc_fence_after();
+                const uint32_t id_s = idesc_bf16(128, 128, true, false);
+                const uint32_t id_o = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t kdh = sdesc_sw128(sbase + C_KDH + ks * 2048, 8192, 1024);
+                    const uint64_t kdl = sdesc_sw128(sbase + C_KDL + ks * 2048, 8192, 1024);
+                    const uint64_t uh = sdesc_sw128(sbase + C_UH + ks * 32, 16, 1024);
+                    const uint64_t ul = sdesc_sw128(sbase + C_UL + ks * 32, 16, 1024);
+                    const uint64_t ph = sdesc_sw128(sbase + C_PH + ks * 32, 16, 1024);
+                    const uint64_t pl = sdesc_sw128(sbase + C_PL + ks * 32, 16, 1024);
+                    mma_bf16(tmem + TM_SN, kdh, uh, id_s, ks > 0);
+                    mma_bf16(tmem + TM_SN, kdh, ul, id_s, 1);
+                    mma_bf16(tmem + TM_SN, kdl, uh, id_s, 1);
+                    mma_bf16(tmem + TM_OT, uh, ph, id_o, 1);
+                    mma_bf16(tmem + TM_OT, uh, pl, id_o, 1);
+                    mma_bf16(tmem + TM_OT, ul, ph, id_o, 1);
+                }
+                mma_commit(bar_mma);
+            }
+            mma_sync();
+            if (__syncthreads_or(!ok)) break;
+            if (tid == 0) mbar_arrive_remote(peer_empty);          // slot consumed
+
+            {
+                const uint32_t lb = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+                float sn[32];
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {
+                    tmem_ld32(lb + TM_SN + half * 64 + part * 32, sn);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) s[part * 32 + c] = fmaf(e_last, s[part * 32 + c], sn[c]);
+                }
+                write_state_f16();
+                float o[32];
+                tmem_ld32(lb + TM_OT + half * 32, o);
+                tmem_wait_ld();
+                const int nvalid = min(C, T - t0) - half * 32;
+#pragma unroll
+                for (int r = 0; r < 32; ++r) {
+                    if (r < nvalid) p.out[(tk0 + (long)(half * 32 + r) * H) * D + srow] = o[r];
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+        }
+        if (tid == 0 && !ok) {   // drain this CTA's own loads and products (bounded)
+            if (kq_waited + 1 < nchunks) mbar_wait(bar_kq, (kq_waited + 1) & 1, &g_pair_status_word);
+            if (v_waited + 1 < nchunks) mbar_wait(bar_v, (v_waited + 1) & 1, &g_pair_status_word);
+            mma_commit(bar_mma);
+            mbar_wait(bar_mma, mma_phase, &g_pair_status_word);
+            (void)full_waited;
+        }
+        if (ok && p.state_out) {
+            float4* dst = reinterpret_cast<float4*>(p.state_out + ((long)b * H + h) * DD +
+                                                    (long)srow * D + scol);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) dst[c] = make_float4(s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]);
+        }
+    }
+
+    // Neither CTA leaves while the other may still touch its shared memory.
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, tmem_cols);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+bool make_map(CUtensorMap* map, const void* base, int H, int T, int B) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)C, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <bool CHANNEL>
+cudaError_t launch_pair(const Problem& p, cudaStream_t stream) {
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(chunk_pair_kernel<CHANNEL>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, p.q, p.H, p.T, p.B) || !make_map(&mk, p.k, p.H, p.T, p.B) ||
+        !make_map(&mv, p.v, p.H, p.T, p.B))
+        return cudaErrorInvalidValue;
+    PairParams prm{p.g, p.beta, p.state_in, p.state_out, static_cast<float*>(p.out), p.T, p.H};
+    chunk_pair_kernel<CHANNEL><<<2 * p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, prm);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_pair_sm100(const Problem& p, cudaStream_t stream) {
+    if (p.io_f32 || !p.out_f32 || p.dk != D || p.dv != D) return cudaErrorNotSupported;
+    return p.per_channel ? launch_pair<true>(p, stream) : launch_pair<false>(p, stream);
+}
+
+cudaError_t read_and_clear_pair_status(unsigned int* status) {
+    cudaError_t e = cudaMemcpyFromSymbol(status, g_pair_status_word, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_pair_status_word, &zero, sizeof(unsigned int));
+}
+
+}  // namespace gdn

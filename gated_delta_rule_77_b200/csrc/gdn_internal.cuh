@@ -41,6 +41,12 @@ cudaError_t launch_chunk_sm100(const Problem& p, cudaStream_t stream);
 constexpr size_t kNoAllocScratchFloats = size_t(8) * 1024 * 1024;   // 32 MiB
 cudaError_t launch_chunk_sm100_noalloc(const Problem& p, cudaStream_t stream, bool* over_limit);
 
+// The same chunk algebra with each (batch, head) on a cluster of two CTAs:
+// one computes A, P and T' for chunk c + 1 while the other runs the state
+// chain of chunk c.  Used for unsegmented calls when 2 * B * H <= #SMs.
+cudaError_t launch_chunk_pair_sm100(const Problem& p, cudaStream_t stream);
+cudaError_t read_and_clear_pair_status(unsigned int* status);
+
 // Device status word written by kernels that abandon a bounded wait.
 cudaError_t read_and_clear_status(unsigned int* status, cudaStream_t stream);
 

@@ -148,3 +148,21 @@ def test_full_config_sampled_heads(gdn, index, oracle_threads):
                               per_channel=cfg.per_channel, heads=heads, threads=oracle_threads)
     _check_pairs(got_o, got_s, ref_o, ref_s, _pairs(x, heads), cfg.tol)
     assert torch.isfinite(got_o).all() and torch.isfinite(got_s).all()
+
+
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+@pytest.mark.parametrize("T", [50, 64, 200, 700])
+def test_single_cta_and_cta_pair_kernels_agree(gdn, gate, T, monkeypatch):
+    """The one-CTA kernel and the two-CTA cluster kernel (chunk-local work on
+    one SM, state chain on the other) compute the same chunk algebra."""
+    x = prefill_inputs(2, T, 2, 128, 128, gate=gate, s0_std=0.1, seed=230 + T)
+    monkeypatch.setenv("GDN_CHUNK_KERNEL", "single")
+    o1, s1 = _gpu(gdn, x)
+    monkeypatch.setenv("GDN_CHUNK_KERNEL", "pair")
+    o2, s2 = _gpu(gdn, x)
+    ref_o, ref_s = _ref(x, gate == "channel")
+    for o, s in ((o1, s1), (o2, s2)):
+        assert oracle.rel_err(o, ref_o) <= TOL and oracle.rel_err(s, ref_s) <= TOL
+    assert oracle.rel_err(o2, o1.double()) <= TOL / 2
+    assert oracle.rel_err(s2, s1.double()) <= TOL / 2
+    assert gdn.check() == gdn.GDN_OK
