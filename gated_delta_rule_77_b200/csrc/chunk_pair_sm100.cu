@@ -68,7 +68,10 @@ constexpr uint32_t P_GAM = P_SMALL;           // 64 f32
 constexpr uint32_t P_BETA = P_GAM + 256;      // 64 f32
 constexpr uint32_t P_REF0 = P_BETA + 256;     // 128 f32
 constexpr uint32_t P_REF1 = P_REF0 + 512;     // 128 f32
-constexpr uint32_t P_BAR = P_REF1 + 512;      // tma, mma, empty
+constexpr uint32_t P_ER = P_REF1 + 512;       // 64 f32: exp(G_r - G_31)  (scalar gate)
+constexpr uint32_t P_FJ = P_ER + 256;         // 64 f32: exp(G_31 - G_j)
+constexpr uint32_t P_SAFE = P_FJ + 256;       // int: product form in range
+constexpr uint32_t P_BAR = P_SAFE + 16;       // tma, mma, empty
 constexpr uint32_t P_TMEM = P_BAR + 24;
 constexpr uint32_t P_USED = P_TMEM + 8;
 
@@ -219,7 +222,8 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     };
     // Scalar gate: warp 0 scans the chunk's 64 values of g into sGam (and
     // copies beta when sBeta is given).
-    auto gate_scalar = [&](int t0, long tk0, float* sGam, float* sBeta) {
+    auto gate_scalar = [&](int t0, long tk0, float* sGam, float* sBeta, float* sEr = nullptr,
+                           float* sFj = nullptr, int* sSafe = nullptr) {
         if (warp != 0) return;
         float b0 = 0.f, b1 = 0.f, g0 = 0.f, g1 = 0.f;
         if (t0 + lane < T) {
@@ -244,6 +248,23 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             g1 += __shfl_sync(0xffffffffu, g0, 31);
             sGam[lane] = g0;
             sGam[32 + lane] = g1;
+            if (sEr) {
+                // exp(G_r - G_j) = exp(G_r - G_31) exp(G_31 - G_j), exact in fp32
+                // while the chunk's total decay is at most 80 (both factors
+                // within exp(+-80)); otherwise the epilogue exponentiates directly.
+                const float m = __shfl_sync(0xffffffffu, g0, 31);
+                float mx = fmaxf(g0, g1), mn = fminf(g0, g1);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+                }
+                sEr[lane] = __expf(g0 - m);
+                sEr[32 + lane] = __expf(g1 - m);
+                sFj[lane] = __expf(m - g0);
+                sFj[32 + lane] = __expf(m - g1);
+                if (lane == 0) *sSafe = (mx - mn) <= 80.f;
+            }
         }
     };
 
@@ -253,6 +274,9 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         float* sBeta = reinterpret_cast<float*>(smem + P_BETA);
         float* sRef0 = reinterpret_cast<float*>(smem + P_REF0);
         float* sRef1 = reinterpret_cast<float*>(smem + P_REF1);
+        float* sEr = reinterpret_cast<float*>(smem + P_ER);
+        float* sFj = reinterpret_cast<float*>(smem + P_FJ);
+        int* sSafe = reinterpret_cast<int*>(smem + P_SAFE);
         float* sA = reinterpret_cast<float*>(smem + P_A);
         float* sT = reinterpret_cast<float*>(smem + P_T);
         float* sY = reinterpret_cast<float*>(smem + P_Y);
@@ -278,7 +302,7 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const long tk0 = ((long)b * T + t0) * H + h;
             float gam[4][8];
             if (CHANNEL) gate_channel(t0, tk0, gam, sRef0, sRef1, nullptr);
-            gate_scalar(t0, tk0, sGam, sBeta);
+            gate_scalar(t0, tk0, sGam, sBeta, sEr, sFj, sSafe);
             ok = ok && mbar_wait(bar_tma, ci & 1, &g_pair_status_word);
             kq_waited = ci;
             if (tid == 0 && copy_pending) {      // staging (in the X region) free again
@@ -382,6 +406,12 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
                 const float br = sBeta[r];
                 const float Gr = CHANNEL ? 0.f : sGam[r];
+                const bool prod = !CHANNEL && *sSafe;
+                const float er = CHANNEL ? 1.f : sEr[r];
+                auto decay = [&](int j) -> float {
+                    if (CHANNEL) return 1.f;
+                    return prod ? er * sFj[j] : __expf(Gr - sGam[j]);
+                };
                 const int j0 = half * 32;
                 if (!is_p) {
 #pragma unroll
@@ -391,7 +421,7 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         for (int e = 0; e < 4; ++e) {
                             const int j = j0 + 4 * j4 + e;
                             float val = 0.f;
-                            if (j < r) val = br * x[4 * j4 + e] * (CHANNEL ? 1.f : __expf(Gr - sGam[j]));
+                            if (j < r) val = br * x[4 * j4 + e] * decay(j);
                             a[e] = val;
                         }
                         *reinterpret_cast<float4*>(&sA[fidx(r, j0 + 4 * j4)]) = make_float4(a[0], a[1], a[2], a[3]);
@@ -404,7 +434,7 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         for (int e = 0; e < 8; ++e) {
                             const int j = j0 + 8 * c + e;
                             float val = 0.f;
-                            if (j <= r) val = x[8 * c + e] * (CHANNEL ? 1.f : __expf(Gr - sGam[j]));
+                            if (j <= r) val = x[8 * c + e] * decay(j);
                             pv[e] = val;
                         }
                         const int cc = half * 4 + c;

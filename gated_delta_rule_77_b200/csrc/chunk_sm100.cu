@@ -112,7 +112,10 @@ constexpr uint32_t SM_BETA = SM_GAM + 256;    // 64 f32
 constexpr uint32_t SM_REF0 = SM_BETA + 256;   // 128 f32: G at token 15 (channel)
 constexpr uint32_t SM_REF1 = SM_REF0 + 512;   // 128 f32: G at token 47
 constexpr uint32_t SM_LAST = SM_REF1 + 512;   // 128 f32: G at token 63
-constexpr uint32_t SM_BAR = SM_LAST + 512;    // 2 mbarriers
+constexpr uint32_t SM_ER = SM_LAST + 512;     // 64 f32: exp(G_r - G_31)  (scalar gate)
+constexpr uint32_t SM_FJ = SM_ER + 256;       // 64 f32: exp(G_31 - G_j)
+constexpr uint32_t SM_SAFE = SM_FJ + 256;     // int: product form in range
+constexpr uint32_t SM_BAR = SM_SAFE + 16;     // 2 mbarriers
 constexpr uint32_t SM_TMEM = SM_BAR + 16;     // TMEM base address
 constexpr uint32_t SMEM_USED = SM_TMEM + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
@@ -157,6 +160,9 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     float* sRef0 = reinterpret_cast<float*>(smem + SM_REF0);
     float* sRef1 = reinterpret_cast<float*>(smem + SM_REF1);
     float* sLast = reinterpret_cast<float*>(smem + SM_LAST);
+    float* sEr = reinterpret_cast<float*>(smem + SM_ER);
+    float* sFj = reinterpret_cast<float*>(smem + SM_FJ);
+    int* sSafe = reinterpret_cast<int*>(smem + SM_SAFE);
     float* sA = reinterpret_cast<float*>(smem + OFF_A);
     float* sTf = reinterpret_cast<float*>(smem + OFF_TF);
     float* sY = reinterpret_cast<float*>(smem + OFF_Y);
@@ -343,6 +349,21 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 g1 += __shfl_sync(0xffffffffu, g0, 31);
                 sGam[lane] = g0;
                 sGam[32 + lane] = g1;
+                // exp(G_r - G_j) = exp(G_r - G_31) exp(G_31 - G_j), exact in fp32
+                // while the chunk's total decay is at most 80; otherwise the
+                // epilogue exponentiates directly.
+                const float m = __shfl_sync(0xffffffffu, g0, 31);
+                float mx = fmaxf(g0, g1), mn = fminf(g0, g1);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+                }
+                sEr[lane] = __expf(g0 - m);
+                sEr[32 + lane] = __expf(g1 - m);
+                sFj[lane] = __expf(m - g0);
+                sFj[32 + lane] = __expf(m - g1);
+                if (lane == 0) *sSafe = (mx - mn) <= 80.f;
             }
         }
         ok = ok && mbar_wait(bar_tma, ci & 1, &g_status_word);
@@ -478,6 +499,12 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             const float br = sBeta[r];
             const float Gr = CHANNEL ? 0.f : sGam[r];
+            const bool prod = !CHANNEL && *sSafe;
+            const float er = CHANNEL ? 1.f : sEr[r];
+            auto decay = [&](int j) -> float {
+                if (CHANNEL) return 1.f;
+                return prod ? er * sFj[j] : __expf(Gr - sGam[j]);
+            };
             const int j0 = half * 32;
             if (!is_p) {
 #pragma unroll
@@ -487,7 +514,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     for (int e = 0; e < 4; ++e) {
                         const int j = j0 + 4 * j4 + e;
                         float val = 0.f;
-                        if (j < r) val = br * x[4 * j4 + e] * (CHANNEL ? 1.f : __expf(Gr - sGam[j]));
+                        if (j < r) val = br * x[4 * j4 + e] * decay(j);
                         a[e] = val;
                     }
                     *reinterpret_cast<float4*>(&sA[fidx(r, j0 + 4 * j4)]) = make_float4(a[0], a[1], a[2], a[3]);
@@ -500,7 +527,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     for (int e = 0; e < 8; ++e) {
                         const int j = j0 + 8 * c + e;
                         float val = 0.f;
-                        if (j <= r) val = x[8 * c + e] * (CHANNEL ? 1.f : __expf(Gr - sGam[j]));
+                        if (j <= r) val = x[8 * c + e] * decay(j);
                         pv[e] = val;
                     }
                     const int cc = half * 4 + c;

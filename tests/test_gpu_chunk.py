@@ -166,3 +166,18 @@ def test_single_cta_and_cta_pair_kernels_agree(gdn, gate, T, monkeypatch):
     assert oracle.rel_err(o2, o1.double()) <= TOL / 2
     assert oracle.rel_err(s2, s1.double()) <= TOL / 2
     assert gdn.check() == gdn.GDN_OK
+
+
+@pytest.mark.parametrize("kernel", ["single", "pair"])
+def test_scalar_gate_beyond_the_bounded_domain(gdn, kernel, monkeypatch):
+    """The scalar gate accepts any g <= 0: chunks whose total decay exceeds the
+    range of the factored form take exact per-element exponentials."""
+    x = prefill_inputs(1, 256, 2, 128, 128, gate="scalar", s0_std=0.1, seed=240)
+    gen = torch.Generator().manual_seed(241)
+    strong = -30.0 * torch.rand(x["g"].shape, generator=gen)
+    x["g"] = torch.where(torch.arange(256)[None, :, None] < 128, strong, x["g"]).contiguous()
+    monkeypatch.setenv("GDN_CHUNK_KERNEL", kernel)
+    got_o, got_s = _gpu(gdn, x)
+    ref_o, ref_s = _ref(x, False)
+    assert oracle.rel_err(got_o, ref_o) <= TOL
+    assert oracle.rel_err(got_s, ref_s) <= TOL
