@@ -45,7 +45,10 @@ PREFILL_CFG = CONFIGS[2]
 DECODE_CFG = CONFIGS[4]
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "GDN prefill tokens/s + % tensor roofline; decode state GB/s vs HBM peak"
-PROFILE_SUMMARY = ROOT / "profiles" / "chunk_fwd_kernel_gdn2_layer_B8H8T2048.md"
+PROFILE_SUMMARY = ROOT / "profiles" / "chunk_pair_kernel_gdn2_layer_B8H8T2048.md"
+# The sources the prefill kernel of this workload is compiled from (a cluster
+# of two CTAs per (batch, head): 2 * B * H = 128 <= 148 SMs).
+KERNEL_SOURCES = ("chunk_pair_sm100.cu", "chunk_common.cuh", "sm100_util.cuh")
 
 
 # ---------------------------------------------------------------- accounting --
@@ -84,11 +87,19 @@ def measured_peaks() -> dict:
             "source": "fallback"}
 
 
+def kernel_source_sha1() -> str:
+    """sha1 over the prefill kernel's source files, in KERNEL_SOURCES order."""
+    import hashlib
+    h = hashlib.sha1()
+    for name in KERNEL_SOURCES:
+        h.update((ROOT / "gated_delta_rule_77_b200" / "csrc" / name).read_bytes())
+    return h.hexdigest()
+
+
 def ncu_traffic():
     """dram read+write bytes per launch of the chunk kernel from the committed
     ncu summary, or None when the kernel source changed since that capture
-    (the summary records the sha1 of the source it measured)."""
-    import hashlib
+    (the summary records the sha1 of the sources it measured)."""
     if not PROFILE_SUMMARY.exists():
         return None
     fields = {}
@@ -96,8 +107,7 @@ def ncu_traffic():
         if ":" in line and not line.startswith(("|", " ", "#")):
             key, val = line.split(":", 1)
             fields[key.strip()] = val.strip()
-    src = ROOT / "gated_delta_rule_77_b200" / "csrc" / "chunk_sm100.cu"
-    if fields.get("kernel_source_sha1") != hashlib.sha1(src.read_bytes()).hexdigest():
+    if fields.get("kernel_source_sha1") != kernel_source_sha1():
         return None
     try:
         return float(fields["traffic_bytes_per_launch"])
@@ -309,7 +319,7 @@ def run_ours(args, rank: int, world: int, local: int):
     traffic = ncu_traffic()
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": traffic,
-                "kernel": "chunk_fwd_kernel<per-channel>", "bytes_per_launch": nbytes,
+                "kernel": "chunk_pair_kernel<per-channel>", "bytes_per_launch": nbytes,
                 "peak_source": peaks["source"]}
     tflops = nflops / t_launch / 1e12
     tensor = {"achieved_tflops": tflops, "peak_tflops": peaks["bf16_tflops"],

@@ -61,8 +61,8 @@ constexpr uint32_t P_C1H = P_X + 81920;       //   16 KB
 constexpr uint32_t P_C1L = P_X + 98304;       //   16 KB
 constexpr uint32_t P_STAGE = P_X;             //   after X: T' hi, T' lo, P hi, P lo (4 x 8 KB)
 constexpr uint32_t P_A = P_X + 32768;         //   16 KB A fp32 (fidx layout)
-constexpr uint32_t P_T = P_X + 49152;         //   16 KB T fp32 row-major
-constexpr uint32_t P_Y = P_X + 65536;         //   3 KB solve scratch
+constexpr uint32_t P_T = P_X + 49152;         //   16 KB T fp32 (tidx layout)
+constexpr uint32_t P_Y = P_X + 65536;         //   3.5 KB solve scratch [16][56]
 constexpr uint32_t P_SMALL = P_X + 114688;
 constexpr uint32_t P_GAM = P_SMALL;           // 64 f32
 constexpr uint32_t P_BETA = P_GAM + 256;      // 64 f32
@@ -169,8 +169,14 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
     // Per-channel cumulative log-decay of this thread's 4 tokens x 8 channels
     // (registers); block references / last token stored by lane tg = 15.
-    auto gate_channel = [&](int t0, long tk0, float (&gam)[4][8], float* ref0, float* ref1,
-                            float* last) {
+    // Loads are issued one chunk ahead (gate_load for chunk c + 1 once chunk c
+    // no longer needs its own values), so their latency is hidden behind the
+    // rest of the chunk; the scan (gate_channel) runs at the start of the
+    // chunk.  They are issued after a proxy fence, not before one: the fence
+    // waits for the thread's outstanding loads (measured on B200).
+    auto gate_load = [&](int chunk, float (&gam)[4][8]) {
+        const int t0 = chunk * C;
+        const long tk0 = ((long)b * T + t0) * H + h;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int r = tg + 16 * u;
@@ -184,6 +190,9 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 for (int e = 0; e < 8; ++e) gam[u][e] = 0.f;
             }
         }
+    };
+    auto gate_channel = [&](int t0, long tk0, float (&gam)[4][8], float* ref0, float* ref1,
+                            float* last) {
 #pragma unroll
         for (int o = 1; o < 16; o <<= 1) {
 #pragma unroll
@@ -204,10 +213,10 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 off += tot;
             }
         }
-        if (t0 + C < T) {
+        if (t0 + 2 * C < T) {     // warm L2 two chunks ahead
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int r = C + tg + 16 * u;
+                const int r = 2 * C + tg + 16 * u;
                 if (t0 + r < T) prefetch_l2(p.g + (tk0 + (long)r * H) * D + 8 * ck);
             }
         }
@@ -220,20 +229,28 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
         }
     };
-    // Scalar gate: warp 0 scans the chunk's 64 values of g into sGam (and
-    // copies beta when sBeta is given).
-    auto gate_scalar = [&](int t0, long tk0, float* sGam, float* sBeta, float* sEr = nullptr,
-                           float* sFj = nullptr, int* sSafe = nullptr) {
+    // Scalar gate and beta, warp 0: lane holds tokens lane and 32 + lane.
+    // gate_scalar_load reads them into registers; gate_scalar scans g into
+    // sGam (and stores beta when sBeta is given).
+    auto gate_scalar_load = [&](int chunk, bool with_beta, float (&bg)[4]) {
+        bg[0] = bg[1] = bg[2] = bg[3] = 0.f;
         if (warp != 0) return;
-        float b0 = 0.f, b1 = 0.f, g0 = 0.f, g1 = 0.f;
+        const int t0 = chunk * C;
+        const long tk0 = ((long)b * T + t0) * H + h;
         if (t0 + lane < T) {
-            if (sBeta) b0 = p.beta[tk0 + (long)lane * H];
-            if (!CHANNEL) g0 = p.g[tk0 + (long)lane * H];
+            if (with_beta) bg[0] = p.beta[tk0 + (long)lane * H];
+            if (!CHANNEL) bg[2] = p.g[tk0 + (long)lane * H];
         }
         if (t0 + 32 + lane < T) {
-            if (sBeta) b1 = p.beta[tk0 + (long)(32 + lane) * H];
-            if (!CHANNEL) g1 = p.g[tk0 + (long)(32 + lane) * H];
+            if (with_beta) bg[1] = p.beta[tk0 + (long)(32 + lane) * H];
+            if (!CHANNEL) bg[3] = p.g[tk0 + (long)(32 + lane) * H];
         }
+    };
+    auto gate_scalar = [&](const float (&bg)[4], float* sGam, float* sBeta, float* sEr = nullptr,
+                           float* sFj = nullptr, int* sSafe = nullptr) {
+        if (warp != 0) return;
+        const float b0 = bg[0], b1 = bg[1];
+        float g0 = bg[2], g1 = bg[3];
         if (sBeta) {
             sBeta[lane] = b0;
             sBeta[32 + lane] = b1;
@@ -296,13 +313,26 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (tid == 0 && nchunks > 0) issue_kq(0);
         int kq_waited = -1;
         bool copy_pending = false;
+        float gnext[4][8], bgnext[4];
+        if (CHANNEL && nchunks > 0) gate_load(0, gnext);
+        if (CHANNEL && nchunks > 0) gate_scalar_load(0, true, bgnext);
 
         for (int ci = 0; ci < nchunks; ++ci) {
             const int t0 = ci * C;
             const long tk0 = ((long)b * T + t0) * H + h;
             float gam[4][8];
-            if (CHANNEL) gate_channel(t0, tk0, gam, sRef0, sRef1, nullptr);
-            gate_scalar(t0, tk0, sGam, sBeta, sEr, sFj, sSafe);
+            if (CHANNEL) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) gam[u][e] = gnext[u][e];
+                gate_channel(t0, tk0, gam, sRef0, sRef1, nullptr);
+            }
+            // beta one chunk ahead with per-channel gates; in place with a
+            // scalar gate, where the early load measured slower.
+            if (!CHANNEL) gate_scalar_load(ci, true, bgnext);
+            gate_scalar(bgnext, sGam, sBeta, sEr, sFj, sSafe);
+            if (CHANNEL && ci + 1 < nchunks) gate_scalar_load(ci + 1, true, bgnext);
             ok = ok && mbar_wait(bar_tma, ci & 1, &g_pair_status_word);
             kq_waited = ci;
             if (tid == 0 && copy_pending) {      // staging (in the X region) free again
@@ -343,6 +373,7 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
                 fence_async_smem();
                 __syncthreads();
+                if (ci + 1 < nchunks) gate_load(ci + 1, gnext);
             }
             if (tid == 0) {
                 tc_fence_after();
@@ -444,11 +475,11 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             tc_fence_before();
             __syncthreads();
-            solve_unit_lower64(sA, sT, sY, tid);
+            solve_unit_lower64_mma(sA, sT, sY, tid);
             for (int e = tid; e < 512; e += NT) {
                 const int r = e >> 3, c = e & 7;
-                const float4 t0v = *reinterpret_cast<const float4*>(&sT[r * 64 + 8 * c]);
-                const float4 t1v = *reinterpret_cast<const float4*>(&sT[r * 64 + 8 * c + 4]);
+                const float4 t0v = *reinterpret_cast<const float4*>(&sT[tidx(r, 8 * c)]);
+                const float4 t1v = *reinterpret_cast<const float4*>(&sT[tidx(r, 8 * c + 4)]);
                 const float tt[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
                 float tv[8];
 #pragma unroll
@@ -531,13 +562,23 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             issue_v(0);
         }
         int kq_waited = -1, v_waited = -1, full_waited = -1;
+        float gnext[4][8], bgnext[4];
+        if (CHANNEL && nchunks > 0) gate_load(0, gnext);
 
         for (int ci = 0; ci < nchunks; ++ci) {
             const int t0 = ci * C;
             const long tk0 = ((long)b * T + t0) * H + h;
             float gam[4][8];
-            if (CHANNEL) gate_channel(t0, tk0, gam, nullptr, nullptr, sLast);
-            gate_scalar(t0, tk0, sGam, nullptr);
+            if (CHANNEL) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) gam[u][e] = gnext[u][e];
+                gate_channel(t0, tk0, gam, nullptr, nullptr, sLast);
+            } else {
+                gate_scalar_load(ci, false, bgnext);
+                gate_scalar(bgnext, sGam, nullptr);
+            }
             ok = ok && mbar_wait(bar_kq, ci & 1, &g_pair_status_word);
             kq_waited = ci;
             if (__syncthreads_or(!ok)) break;
@@ -577,6 +618,7 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             fence_async_smem();
             __syncthreads();
             if (tid == 0 && ci + 1 < nchunks) issue_kq(ci + 1);   // raw K, Q consumed
+            if (CHANNEL && ci + 1 < nchunks) gate_load(ci + 1, gnext);
 
             // T' and P of this chunk from CTA 0; V of this chunk.
             if (tid == 0) {
