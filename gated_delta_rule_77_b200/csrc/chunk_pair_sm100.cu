@@ -59,7 +59,6 @@ constexpr uint32_t P_C0H = P_X + 65536;       //   8 KB
 constexpr uint32_t P_C0L = P_X + 73728;       //   8 KB
 constexpr uint32_t P_C1H = P_X + 81920;       //   16 KB
 constexpr uint32_t P_C1L = P_X + 98304;       //   16 KB
-constexpr uint32_t P_STAGE = P_X;             //   after X: T' hi, T' lo, P hi, P lo (4 x 8 KB)
 constexpr uint32_t P_A = P_X + 32768;         //   16 KB A fp32 (fidx layout)
 constexpr uint32_t P_T = P_X + 49152;         //   16 KB T fp32 (tidx layout)
 constexpr uint32_t P_Y = P_X + 65536;         //   3.5 KB solve scratch [16][56]
@@ -73,7 +72,10 @@ constexpr uint32_t P_FJ = P_ER + 256;         // 64 f32: exp(G_31 - G_j)
 constexpr uint32_t P_SAFE = P_FJ + 256;       // int: product form in range
 constexpr uint32_t P_BAR = P_SAFE + 16;       // tma, mma, empty
 constexpr uint32_t P_TMEM = P_BAR + 24;
-constexpr uint32_t P_USED = P_TMEM + 8;
+// T' hi, T' lo, P hi, P lo (4 x 8 KB) for the bulk copy to CTA 1; apart from
+// the X region so that the copy of chunk c overlaps the X build of chunk c + 1.
+constexpr uint32_t P_STAGE = (P_TMEM + 8 + 1023) / 1024 * 1024;
+constexpr uint32_t P_USED = P_STAGE + 32768;
 
 // ---- CTA 1 (chain) shared memory ----------------------------------------------
 constexpr uint32_t C_IN = 0;                  // 32 KB raw K, Q
@@ -83,6 +85,7 @@ constexpr uint32_t C_KE = 81920;              // 16 KB K*E bf16; then W^T fp16 [
 constexpr uint32_t C_QE = 98304;              // 16 KB Q*E fp16
 constexpr uint32_t C_KDH = 114688;            // 16 KB K*D bf16 hi
 constexpr uint32_t C_KDL = 131072;            // 16 KB K*D bf16 lo
+constexpr uint32_t C_OST = C_KDH;             // after SN: 32 KB O fp32 [64 t][128 j] for the TMA store
 constexpr uint32_t C_UH = 147456;             // 16 KB U^T hi [128 j][64 r]
 constexpr uint32_t C_UL = 163840;             // 16 KB U^T lo
 constexpr uint32_t C_SLOT = 180224;           // 32 KB T' hi, T' lo, P hi, P lo (from CTA 0)
@@ -113,7 +116,8 @@ struct PairParams {
 template <bool CHANNEL>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
 chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const PairParams p)
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  const PairParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -145,7 +149,10 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (tid == 0) {
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
-        if (rank == 1) prefetch_tensormap(&tm_v);
+        if (rank == 1) {
+            prefetch_tensormap(&tm_v);
+            prefetch_tensormap(&tm_o);
+        }
         for (int i = 0; i < (rank == 0 ? 3 : 4); ++i) mbar_init(bar0 + 8 * i, 1);
         fence_mbar_init();
     }
@@ -335,10 +342,6 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (CHANNEL && ci + 1 < nchunks) gate_scalar_load(ci + 1, true, bgnext);
             ok = ok && mbar_wait(bar_tma, ci & 1, &g_pair_status_word);
             kq_waited = ci;
-            if (tid == 0 && copy_pending) {      // staging (in the X region) free again
-                bulk_wait_read_all();
-                copy_pending = false;
-            }
             if (__syncthreads_or(!ok)) break;
 
             if (CHANNEL) {
@@ -409,6 +412,10 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 mma_commit(sbase + P_BAR + 8);
             }
             mma_sync();
+            if (tid == 0 && copy_pending) {      // the staging is free again
+                bulk_wait_read_all();
+                copy_pending = false;
+            }
             if (__syncthreads_or(!ok)) break;
             // Raw K, Q and the X operands are consumed: prefetch the next chunk.
             if (tid == 0 && ci + 1 < nchunks) issue_kq(ci + 1);
@@ -581,6 +588,7 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             ok = ok && mbar_wait(bar_kq, ci & 1, &g_pair_status_word);
             kq_waited = ci;
+            if (tid == 0) bulk_wait_read_all();   // previous O store has read C_OST
             if (__syncthreads_or(!ok)) break;
 
             // K*E (bf16), Q*E (fp16), K*D (bf16 hi + lo).
@@ -728,16 +736,22 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 float o[32];
                 tmem_ld32(lb + TM_OT + half * 32, o);
                 tmem_wait_ld();
-                const int nvalid = min(C, T - t0) - half * 32;
+                // O^T (lane = value column) -> [token][column] fp32; one TMA
+                // store writes the chunk and drops rows past T.  Global stores
+                // from the threads would hold up the proxy fence below.
+                float* so = reinterpret_cast<float*>(smem + C_OST) + half * 32 * D + srow;
 #pragma unroll
-                for (int r = 0; r < 32; ++r) {
-                    if (r < nvalid) p.out[(tk0 + (long)(half * 32 + r) * H) * D + srow] = o[r];
-                }
+                for (int r = 0; r < 32; ++r) so[r * D] = o[r];
             }
             fence_async_smem();
             tc_fence_before();
             __syncthreads();
+            if (tid == 0) {
+                tma_store_4d(&tm_o, sbase + C_OST, 0, h, t0, b);
+                bulk_commit();
+            }
         }
+        if (tid == 0) bulk_wait_all();       // output stores complete before exit
         if (tid == 0 && !ok) {   // drain this CTA's own loads and products (bounded)
             if (kq_waited + 1 < nchunks) mbar_wait(bar_kq, (kq_waited + 1) & 1, &g_pair_status_word);
             if (v_waited + 1 < nchunks) mbar_wait(bar_v, (v_waited + 1) & 1, &g_pair_status_word);
@@ -776,6 +790,20 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
+// out [B, T, H, D] fp32, box = one chunk of one head, no swizzle.
+bool make_out_map(CUtensorMap* map, void* base, int H, int T, int B) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 4, (cuuint64_t)H * D * 4, (cuuint64_t)T * H * D * 4};
+    cuuint32_t box[4] = {(cuuint32_t)D, 1, (cuuint32_t)C, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool make_map(CUtensorMap* map, const void* base, int H, int T, int B) {
     auto fn = encode_fn();
     if (!fn) return false;
@@ -798,12 +826,12 @@ cudaError_t launch_pair(const Problem& p, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, p.q, p.H, p.T, p.B) || !make_map(&mk, p.k, p.H, p.T, p.B) ||
-        !make_map(&mv, p.v, p.H, p.T, p.B))
+        !make_map(&mv, p.v, p.H, p.T, p.B) || !make_out_map(&mo, p.out, p.H, p.T, p.B))
         return cudaErrorInvalidValue;
     PairParams prm{p.g, p.beta, p.state_in, p.state_out, static_cast<float*>(p.out), p.T, p.H};
-    chunk_pair_kernel<CHANNEL><<<2 * p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, prm);
+    chunk_pair_kernel<CHANNEL><<<2 * p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, prm);
     return cudaGetLastError();
 }
 

@@ -657,6 +657,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (__syncthreads_or(!ok)) break;
 
         // ---------------------------------------------------- state and output --
+        float o[32];
         {
             const uint32_t lb = tmem + (static_cast<uint32_t>(quad * 32) << 16);
             float sn[32];
@@ -668,21 +669,20 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 for (int c = 0; c < 32; ++c) s[part * 32 + c] = fmaf(e_last, s[part * 32 + c], sn[c]);
             }
             write_state_f16();
-            float o[32];
             tmem_ld32(lb + TM_OT + half * 32, o);
             tmem_wait_ld();
-            const int j = srow;
-            const int nvalid = min(C, t_end - t0) - half * 32;
-            if (p.out != nullptr && !transition) {
-#pragma unroll
-                for (int r = 0; r < 32; ++r) {
-                    if (r < nvalid) p.out[(tk0 + (long)(half * 32 + r) * H) * D + j] = o[r];
-                }
-            }
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
+        // Output stores after the fence, which would otherwise wait for them.
+        if (p.out != nullptr && !transition) {
+            const int nvalid = min(C, t_end - t0) - half * 32;
+#pragma unroll
+            for (int r = 0; r < 32; ++r) {
+                if (r < nvalid) p.out[(tk0 + (long)(half * 32 + r) * H) * D + srow] = o[r];
+            }
+        }
     }
 
     if (!ok && tid == 0) {

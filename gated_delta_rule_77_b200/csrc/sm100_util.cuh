@@ -151,6 +151,17 @@ __device__ __forceinline__ void bulk_wait_all() {
 }
 
 // ---- TMA ----------------------------------------------------------------------
+// Tiled store of a shared-memory box to global memory, tracked by this
+// thread's bulk groups (bulk_commit / bulk_wait_*).  Elements outside the
+// tensor's extent are not written.  Coordinates must not be negative.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t src, int c0, int c1,
+                                             int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+        ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
                                             int c2, int c3, uint32_t bar) {
     asm volatile(
