@@ -276,5 +276,148 @@ __device__ __forceinline__ void solve_unit_lower64_mma(const float* sA, float* s
     }
 }
 
+// Three-term TF32 product with three independent accumulators (hi*hi,
+// hi*lo, lo*hi), so that consecutive k-steps do not wait on each other.
+struct Acc3 {
+    float hh[4] = {0.f, 0.f, 0.f, 0.f};
+    float hl[4] = {0.f, 0.f, 0.f, 0.f};
+    float lh[4] = {0.f, 0.f, 0.f, 0.f};
+    __device__ __forceinline__ void add(const float (&a)[4], const float (&b)[2]) {
+        uint32_t ah[4], al[4], bh[2], bl[2];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) split_tf32(a[i], ah[i], al[i]);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) split_tf32(b[i], bh[i], bl[i]);
+        mma_tf32_16x8x8(hh, ah, bh);
+        mma_tf32_16x8x8(hl, ah, bl);
+        mma_tf32_16x8x8(lh, al, bh);
+    }
+    __device__ __forceinline__ float sum(int i) const { return hh[i] + (hl[i] + lh[i]); }
+};
+
+// T = (I + A)^{-1} for a strictly lower triangular 64x64 fp32 A (fidx
+// layout) by recursive doubling on 16-row blocks, with the inverse of a
+// block lower triangular matrix [[P, 0], [R, Q]] written as
+// [[P^-1, 0], [-Q^-1 R P^-1, Q^-1]]:
+//   1. the four 16x16 diagonal blocks by forward substitution (fp32);
+//   2. both 32x32 diagonal blocks: T_10 = -D_1 (A_10 D_0), T_32 = -D_3 (A_32 D_2);
+//   3. the lower-left 32x32 block: -T_BB (A_BA T_AA).
+// Five dependent stages instead of the seven of the row-block levels.  The
+// products run on mma.m16n8k8 (tf32, hi/lo splits, fp32-class accuracy); the
+// triangular operands' zero blocks are skipped.  T is written in the tidx
+// layout (entries above the diagonal of the diagonal 16x16 blocks are zero,
+// the rest of the upper triangle is not written).  Y scratch: [32][40] fp32.
+// Ends with a barrier.
+__device__ __forceinline__ void solve_unit_lower64_rd(const float* sA, float* sT, float* sY, int tid) {
+    const int warp = tid >> 5, lane = tid & 31;
+    const int grp = lane >> 2, tig = lane & 3;
+    if (warp < 4 && lane < 16) {
+        const int o = warp * 16;
+        float t[16];
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) {
+            float a[16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 v = *reinterpret_cast<const float4*>(&sA[fidx(o + rr, o + 4 * q)]);
+                a[4 * q] = v.x; a[4 * q + 1] = v.y; a[4 * q + 2] = v.z; a[4 * q + 3] = v.w;
+            }
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int m = 0; m < rr; ++m) acc[m & 3] = fmaf(a[m], t[m], acc[m & 3]);
+            t[rr] = (rr == lane) ? 1.f : -((acc[0] + acc[1]) + (acc[2] + acc[3]));
+        }
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) sT[tidx(o + rr, o + lane)] = t[rr];
+    }
+    __syncthreads();
+
+    // Stage 2, first product: Y_b = A[32b+16.., 32b..+16] D_{2b} (16x16 each),
+    // warps 0-3: b = warp >> 1, output columns 8 nt.. with nt = warp & 1.
+    if (warp < 4) {
+        const int bb = warp >> 1, nt = warp & 1, base = 32 * bb;
+        Acc3 acc;
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            if (ks < nt) continue;                       // D rows above its columns are zero
+            const int k0 = 8 * ks + tig;
+            const float af[4] = {sA[fidx(base + 16 + grp, base + k0)], sA[fidx(base + 24 + grp, base + k0)],
+                                 sA[fidx(base + 16 + grp, base + k0 + 4)], sA[fidx(base + 24 + grp, base + k0 + 4)]};
+            const float bf[2] = {sT[tidx(base + k0, base + 8 * nt + grp)],
+                                 sT[tidx(base + k0 + 4, base + 8 * nt + grp)]};
+            acc.add(af, bf);
+        }
+        const int c = 8 * nt + 2 * tig;
+        float* y = sY + (16 * bb) * 40;
+        *reinterpret_cast<float2*>(&y[grp * 40 + c]) = make_float2(acc.sum(0), acc.sum(1));
+        *reinterpret_cast<float2*>(&y[(grp + 8) * 40 + c]) = make_float2(acc.sum(2), acc.sum(3));
+    }
+    __syncthreads();
+    // Stage 2, second product: T[32b+16.., 32b..] = -D_{2b+1} Y_b.
+    if (warp < 4) {
+        const int bb = warp >> 1, nt = warp & 1, base = 32 * bb;
+        const float* y = sY + (16 * bb) * 40;
+        Acc3 acc;
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            const int k0 = 8 * ks + tig;
+            const int r0 = base + 16 + grp;
+            const float af[4] = {sT[tidx(r0, base + 16 + k0)], sT[tidx(r0 + 8, base + 16 + k0)],
+                                 sT[tidx(r0, base + 16 + k0 + 4)], sT[tidx(r0 + 8, base + 16 + k0 + 4)]};
+            const float bf[2] = {y[k0 * 40 + 8 * nt + grp], y[(k0 + 4) * 40 + 8 * nt + grp]};
+            acc.add(af, bf);
+        }
+        const int c = base + 8 * nt + 2 * tig;
+        const int r0 = base + 16 + grp, r1 = r0 + 8;
+        sT[tidx(r0, c)] = -acc.sum(0);
+        sT[tidx(r0, c + 1)] = -acc.sum(1);
+        sT[tidx(r1, c)] = -acc.sum(2);
+        sT[tidx(r1, c + 1)] = -acc.sum(3);
+    }
+    __syncthreads();
+
+    // Stage 3: Y = A[32.., 0..32] T[0..32, 0..32] (32x32), then
+    // T[32.., 0..32] = -T[32.., 32..] Y.  Warp = (row tile mt, column tile nt).
+    const int mt = warp >> 2, nt = warp & 3;
+    {
+        Acc3 acc;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            if (ks < nt) continue;                       // T_AA is lower triangular
+            const int k0 = 8 * ks + tig;
+            const int r0 = 32 + 16 * mt + grp;
+            const float af[4] = {sA[fidx(r0, k0)], sA[fidx(r0 + 8, k0)], sA[fidx(r0, k0 + 4)],
+                                 sA[fidx(r0 + 8, k0 + 4)]};
+            const float bf[2] = {sT[tidx(k0, 8 * nt + grp)], sT[tidx(k0 + 4, 8 * nt + grp)]};
+            acc.add(af, bf);
+        }
+        const int c = 8 * nt + 2 * tig;
+        float* y = sY + (16 * mt) * 40;
+        *reinterpret_cast<float2*>(&y[grp * 40 + c]) = make_float2(acc.sum(0), acc.sum(1));
+        *reinterpret_cast<float2*>(&y[(grp + 8) * 40 + c]) = make_float2(acc.sum(2), acc.sum(3));
+    }
+    __syncthreads();
+    {
+        Acc3 acc;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            if (ks > 2 * mt + 1) continue;               // T_BB is lower triangular
+            const int k0 = 8 * ks + tig;
+            const int r0 = 32 + 16 * mt + grp;
+            const float af[4] = {sT[tidx(r0, 32 + k0)], sT[tidx(r0 + 8, 32 + k0)],
+                                 sT[tidx(r0, 32 + k0 + 4)], sT[tidx(r0 + 8, 32 + k0 + 4)]};
+            const float bf[2] = {sY[k0 * 40 + 8 * nt + grp], sY[(k0 + 4) * 40 + 8 * nt + grp]};
+            acc.add(af, bf);
+        }
+        const int c = 8 * nt + 2 * tig;
+        const int r0 = 32 + 16 * mt + grp, r1 = r0 + 8;
+        sT[tidx(r0, c)] = -acc.sum(0);
+        sT[tidx(r0, c + 1)] = -acc.sum(1);
+        sT[tidx(r1, c)] = -acc.sum(2);
+        sT[tidx(r1, c + 1)] = -acc.sum(3);
+    }
+    __syncthreads();
+}
+
 }  // namespace chunk
 }  // namespace gdn
