@@ -53,116 +53,17 @@ __device__ __forceinline__ void load_bf16x8(const uint8_t* src, float* v) {
 }
 
 
-// T = (I + A)^{-1} for a strictly lower triangular 64x64 fp32 A (layout fidx),
-// written to T (plain row-major [64][64]; entries above the diagonal inside the
-// 16x16 diagonal blocks are written as zero, other upper entries untouched).
-// Y: 16 x 48 fp32 scratch.  Called by every thread of a CTA of at least 128
-// threads (contains barriers).
-//   (a) D_b = (I + A_bb)^{-1}, b = 0..3, by forward substitution: warp b,
-//       lane = column;
-//   (b) row blocks a = 1..3: T_{a,<a} = -D_a (A_{a,<a} T_{<a,<a}), both small
-//       products register-blocked by four columns.
-__device__ __forceinline__ void solve_unit_lower64(const float* sA, float* sT, float* sY, int tid) {
-    const int warp = tid >> 5, lane = tid & 31;
-    if (warp < 4 && lane < 16) {
-        const int o = warp * 16;
-        float t[16];
-#pragma unroll
-        for (int rr = 0; rr < 16; ++rr) {
-            float a[16];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 v = *reinterpret_cast<const float4*>(&sA[fidx(o + rr, o + 4 * q)]);
-                a[4 * q] = v.x; a[4 * q + 1] = v.y; a[4 * q + 2] = v.z; a[4 * q + 3] = v.w;
-            }
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};     // short dependency chains
-#pragma unroll
-            for (int m = 0; m < rr; ++m) acc[m & 3] = fmaf(a[m], t[m], acc[m & 3]);
-            t[rr] = (rr == lane) ? 1.f : -((acc[0] + acc[1]) + (acc[2] + acc[3]));
-        }
-#pragma unroll
-        for (int rr = 0; rr < 16; ++rr) sT[(o + rr) * 64 + o + lane] = t[rr];
-    }
-    __syncthreads();
-#pragma unroll 1
-    for (int a = 1; a < 4; ++a) {
-        // Thread tile: rows {rp, rp + 8} x four columns [4 c4, 4 c4 + 4).
-        const int ncol4 = 4 * a;            // float4 column groups left of the diagonal block
-        const int nitem = 8 * ncol4;
-        const int rp = tid / ncol4, c4 = tid - (tid / ncol4) * ncol4;
-        if (tid < nitem) {
-            // Y[rr][4c4..] = sum_m A[16a+rr][m] T[m][4c4..]; T[m][c] = 0 for m < 4 c4.
-            float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            for (int m4 = c4; m4 < 4 * a; ++m4) {
-                const float4 a0 = *reinterpret_cast<const float4*>(&sA[fidx(16 * a + rp, 4 * m4)]);
-                const float4 a1 = *reinterpret_cast<const float4*>(&sA[fidx(16 * a + rp + 8, 4 * m4)]);
-                const float am[2][4] = {{a0.x, a0.y, a0.z, a0.w}, {a1.x, a1.y, a1.z, a1.w}};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float4 tv = *reinterpret_cast<const float4*>(&sT[(4 * m4 + e) * 64 + 4 * c4]);
-#pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        y[i][0] = fmaf(am[i][e], tv.x, y[i][0]);
-                        y[i][1] = fmaf(am[i][e], tv.y, y[i][1]);
-                        y[i][2] = fmaf(am[i][e], tv.z, y[i][2]);
-                        y[i][3] = fmaf(am[i][e], tv.w, y[i][3]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < 2; ++i)
-                *reinterpret_cast<float4*>(&sY[(rp + 8 * i) * 48 + 4 * c4]) =
-                    make_float4(y[i][0], y[i][1], y[i][2], y[i][3]);
-        }
-        __syncthreads();
-        if (tid < nitem) {
-            // T[16a+rr][4c4..] = -sum_n D_a[rr][n] Y[n][4c4..]
-            float t[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-            for (int n4 = 0; n4 < 4; ++n4) {
-                const float4 d0 = *reinterpret_cast<const float4*>(&sT[(16 * a + rp) * 64 + 16 * a + 4 * n4]);
-                const float4 d1 = *reinterpret_cast<const float4*>(&sT[(16 * a + rp + 8) * 64 + 16 * a + 4 * n4]);
-                const float dn[2][4] = {{d0.x, d0.y, d0.z, d0.w}, {d1.x, d1.y, d1.z, d1.w}};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float4 yv = *reinterpret_cast<const float4*>(&sY[(4 * n4 + e) * 48 + 4 * c4]);
-#pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        t[i][0] = fmaf(dn[i][e], yv.x, t[i][0]);
-                        t[i][1] = fmaf(dn[i][e], yv.y, t[i][1]);
-                        t[i][2] = fmaf(dn[i][e], yv.z, t[i][2]);
-                        t[i][3] = fmaf(dn[i][e], yv.w, t[i][3]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < 2; ++i)
-                *reinterpret_cast<float4*>(&sT[(16 * a + rp + 8 * i) * 64 + 4 * c4]) =
-                    make_float4(-t[i][0], -t[i][1], -t[i][2], -t[i][3]);
-        }
-        __syncthreads();
-    }
-}
 
-
-}  // namespace chunk
-}  // namespace gdn
-
-namespace gdn {
-namespace chunk {
-
-// ---- T = (I + A)^{-1} with the off-diagonal products on mma.sync ------------
-// Same blocked algorithm as solve_unit_lower64, but the two small products of
-// every row-block level (Y = A_{a,<a} T_{<a,<a} and T_{a,<a} = -D_a Y) run on
-// the warp-level tensor-core instruction mma.m16n8k8 with tf32 operands, each
-// operand split as x = hi + lo (both tf32) and the product taken as
-// hi*hi + hi*lo + lo*hi, which keeps fp32-class accuracy (error ~2^-22
-// relative per term).  One warp per 8-column tile of the level's output.
+// ---- T = (I + A)^{-1}: tf32 tensor-core helpers ------------------------------
+// Products inside the triangular solve run on the warp-level tensor-core
+// instruction mma.m16n8k8 with tf32 operands, each operand split as
+// x = hi + lo (both tf32) and the product taken as hi*hi + hi*lo + lo*hi,
+// which keeps fp32-class accuracy (error ~2^-22 relative per term).
 //
 // T layout: row-major [64][64] fp32 with the column index xor-ed by
 // 8 * (row mod 4) (tidx), so that the fragment loads of four consecutive rows
 // at one column fall in different banks; 4- and 8-aligned column groups stay
-// contiguous.  Y scratch: [16][56] fp32.
+// contiguous.
 
 __device__ __forceinline__ uint32_t tidx(int r, int c) {
     return static_cast<uint32_t>(r * 64 + (c ^ ((r & 3) << 3)));
@@ -189,93 +90,6 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&
 }
 
 // d += A(16x8) B(8x8) with both operands split (three tf32 products).
-__device__ __forceinline__ void mma3_tf32(float (&d)[4], const float (&a)[4], const float (&b)[2]) {
-    uint32_t ah[4], al[4], bh[2], bl[2];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) split_tf32(a[i], ah[i], al[i]);
-#pragma unroll
-    for (int i = 0; i < 2; ++i) split_tf32(b[i], bh[i], bl[i]);
-    mma_tf32_16x8x8(d, al, bh);
-    mma_tf32_16x8x8(d, ah, bl);
-    mma_tf32_16x8x8(d, ah, bh);
-}
-
-// A: strictly lower 64x64 fp32 (fidx layout).  T: output in the tidx layout
-// (entries above the diagonal inside the 16x16 diagonal blocks written as zero,
-// other upper entries untouched).  Y: 16 x 56 fp32 scratch.  Called by every
-// thread of a CTA of at least 192 threads (contains barriers).
-__device__ __forceinline__ void solve_unit_lower64_mma(const float* sA, float* sT, float* sY, int tid) {
-    const int warp = tid >> 5, lane = tid & 31;
-    const int grp = lane >> 2, tig = lane & 3;
-    if (warp < 4 && lane < 16) {
-        const int o = warp * 16;
-        float t[16];
-#pragma unroll
-        for (int rr = 0; rr < 16; ++rr) {
-            float a[16];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 v = *reinterpret_cast<const float4*>(&sA[fidx(o + rr, o + 4 * q)]);
-                a[4 * q] = v.x; a[4 * q + 1] = v.y; a[4 * q + 2] = v.z; a[4 * q + 3] = v.w;
-            }
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int m = 0; m < rr; ++m) acc[m & 3] = fmaf(a[m], t[m], acc[m & 3]);
-            t[rr] = (rr == lane) ? 1.f : -((acc[0] + acc[1]) + (acc[2] + acc[3]));
-        }
-#pragma unroll
-        for (int rr = 0; rr < 16; ++rr) sT[tidx(o + rr, o + lane)] = t[rr];
-    }
-    __syncthreads();
-#pragma unroll 1
-    for (int a = 1; a < 4; ++a) {
-        const int nt = warp;                 // 8-column tile of the level's output
-        const bool active = nt < 2 * a;
-        if (active) {
-            // Y[:, 8nt..8nt+7] = sum over k-steps ks >= nt of A_{a, 8ks..} T_{8ks.., 8nt..}
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int ks = nt; ks < 2 * a; ++ks) {
-                const int k0 = 8 * ks + tig;
-                float af[4], bf[2];
-                af[0] = sA[fidx(16 * a + grp, k0)];
-                af[1] = sA[fidx(16 * a + grp + 8, k0)];
-                af[2] = sA[fidx(16 * a + grp, k0 + 4)];
-                af[3] = sA[fidx(16 * a + grp + 8, k0 + 4)];
-                bf[0] = sT[tidx(k0, 8 * nt + grp)];
-                bf[1] = sT[tidx(k0 + 4, 8 * nt + grp)];
-                mma3_tf32(d, af, bf);
-            }
-            const int c = 8 * nt + 2 * tig;
-            *reinterpret_cast<float2*>(&sY[grp * 56 + c]) = make_float2(d[0], d[1]);
-            *reinterpret_cast<float2*>(&sY[(grp + 8) * 56 + c]) = make_float2(d[2], d[3]);
-        }
-        __syncthreads();
-        if (active) {
-            // T[16a.., 8nt..] = -D_a Y[:, 8nt..],  D_a = T[16a.., 16a..]
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int ks = 0; ks < 2; ++ks) {
-                const int k0 = 8 * ks + tig;
-                float af[4], bf[2];
-                af[0] = sT[tidx(16 * a + grp, 16 * a + k0)];
-                af[1] = sT[tidx(16 * a + grp + 8, 16 * a + k0)];
-                af[2] = sT[tidx(16 * a + grp, 16 * a + k0 + 4)];
-                af[3] = sT[tidx(16 * a + grp + 8, 16 * a + k0 + 4)];
-                bf[0] = sY[k0 * 56 + 8 * nt + grp];
-                bf[1] = sY[(k0 + 4) * 56 + 8 * nt + grp];
-                mma3_tf32(d, af, bf);
-            }
-            const int c = 8 * nt + 2 * tig;
-            const int r0 = 16 * a + grp, r1 = r0 + 8;
-            sT[tidx(r0, c)] = -d[0];
-            sT[tidx(r0, c + 1)] = -d[1];
-            sT[tidx(r1, c)] = -d[2];
-            sT[tidx(r1, c + 1)] = -d[3];
-        }
-        __syncthreads();
-    }
-}
-
 // Three-term TF32 product with three independent accumulators (hi*hi,
 // hi*lo, lo*hi), so that consecutive k-steps do not wait on each other.
 struct Acc3 {

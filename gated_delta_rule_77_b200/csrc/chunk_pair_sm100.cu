@@ -85,16 +85,16 @@ constexpr uint32_t C_KE = 81920;              // 16 KB K*E bf16; then W^T fp16 [
 constexpr uint32_t C_QE = 98304;              // 16 KB Q*E fp16
 constexpr uint32_t C_KDH = 114688;            // 16 KB K*D bf16 hi
 constexpr uint32_t C_KDL = 131072;            // 16 KB K*D bf16 lo
-constexpr uint32_t C_OST = C_KDH;             // after SN: 32 KB O fp32 [64 t][128 j] for the TMA store
 constexpr uint32_t C_UH = 147456;             // 16 KB U^T hi [128 j][64 r]
 constexpr uint32_t C_UL = 163840;             // 16 KB U^T lo
+constexpr uint32_t C_OST = C_UH;              // after O: 32 KB O fp32 [64 t][128 j] for the TMA store
 constexpr uint32_t C_SLOT = 180224;           // 32 KB T' hi, T' lo, P hi, P lo (from CTA 0)
 constexpr uint32_t C_TH = C_SLOT, C_TL = C_SLOT + 8192, C_PH = C_SLOT + 16384, C_PL = C_SLOT + 24576;
 constexpr uint32_t C_SMALL = C_SLOT + 32768;
 constexpr uint32_t C_GAM = C_SMALL;           // 64 f32
 constexpr uint32_t C_LAST = C_GAM + 256;      // 128 f32
-constexpr uint32_t C_BAR = C_LAST + 512;      // tma_kq, tma_v, mma, full
-constexpr uint32_t C_TMEM = C_BAR + 32;
+constexpr uint32_t C_BAR = C_LAST + 512;      // tma_kq, tma_v, mma, full, out
+constexpr uint32_t C_TMEM = C_BAR + 40;
 constexpr uint32_t C_USED = C_TMEM + 8;
 
 constexpr uint32_t SLOT_BYTES = 32768;
@@ -153,7 +153,7 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             prefetch_tensormap(&tm_v);
             prefetch_tensormap(&tm_o);
         }
-        for (int i = 0; i < (rank == 0 ? 3 : 4); ++i) mbar_init(bar0 + 8 * i, 1);
+        for (int i = 0; i < (rank == 0 ? 3 : 5); ++i) mbar_init(bar0 + 8 * i, 1);
         fence_mbar_init();
     }
     const uint32_t tmem_cols = rank == 0 ? 128 : 512;
@@ -322,7 +322,7 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         bool copy_pending = false;
         float gnext[4][8], bgnext[4];
         if (CHANNEL && nchunks > 0) gate_load(0, gnext);
-        if (CHANNEL && nchunks > 0) gate_scalar_load(0, true, bgnext);
+        if (nchunks > 0) gate_scalar_load(0, true, bgnext);
 
         for (int ci = 0; ci < nchunks; ++ci) {
             const int t0 = ci * C;
@@ -335,9 +335,7 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     for (int e = 0; e < 8; ++e) gam[u][e] = gnext[u][e];
                 gate_channel(t0, tk0, gam, sRef0, sRef1, nullptr);
             }
-            // beta one chunk ahead with per-channel gates; in place with a
-            // scalar gate, where the early load measured slower.
-            if (!CHANNEL) gate_scalar_load(ci, true, bgnext);
+            // g and beta were loaded one chunk ahead.
             gate_scalar(bgnext, sGam, sBeta, sEr, sFj, sSafe);
             if (CHANNEL && ci + 1 < nchunks) gate_scalar_load(ci + 1, true, bgnext);
             ok = ok && mbar_wait(bar_tma, ci & 1, &g_pair_status_word);
@@ -419,6 +417,7 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (__syncthreads_or(!ok)) break;
             // Raw K, Q and the X operands are consumed: prefetch the next chunk.
             if (tid == 0 && ci + 1 < nchunks) issue_kq(ci + 1);
+            if (!CHANNEL && ci + 1 < nchunks) gate_scalar_load(ci + 1, true, bgnext);
 
             // A and P from X (see chunk_sm100.cu); P as bf16 hi + lo into the staging.
             {
@@ -522,6 +521,9 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const uint32_t bar_kq = sbase + C_BAR, bar_v = sbase + C_BAR + 8;
         const uint32_t bar_full = sbase + C_BAR + 24;
         const uint32_t bar_mma = sbase + C_BAR + 16;
+        // Products into O^T are committed apart (bar_out), so that the U
+        // epilogue and the state update do not wait for them.
+        const uint32_t bar_out = sbase + C_BAR + 32;
         const uint32_t peer_empty = mapa_shared(sbase + P_BAR + 16, 0);
 
         const int srow = quad * 32 + lane;
@@ -571,6 +573,7 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         int kq_waited = -1, v_waited = -1, full_waited = -1;
         float gnext[4][8], bgnext[4];
         if (CHANNEL && nchunks > 0) gate_load(0, gnext);
+        if (!CHANNEL && nchunks > 0) gate_scalar_load(0, false, bgnext);
 
         for (int ci = 0; ci < nchunks; ++ci) {
             const int t0 = ci * C;
@@ -583,12 +586,10 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     for (int e = 0; e < 8; ++e) gam[u][e] = gnext[u][e];
                 gate_channel(t0, tk0, gam, nullptr, nullptr, sLast);
             } else {
-                gate_scalar_load(ci, false, bgnext);
                 gate_scalar(bgnext, sGam, nullptr);
             }
             ok = ok && mbar_wait(bar_kq, ci & 1, &g_pair_status_word);
             kq_waited = ci;
-            if (tid == 0) bulk_wait_read_all();   // previous O store has read C_OST
             if (__syncthreads_or(!ok)) break;
 
             // K*E (bf16), Q*E (fp16), K*D (bf16 hi + lo).
@@ -626,7 +627,10 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             fence_async_smem();
             __syncthreads();
             if (tid == 0 && ci + 1 < nchunks) issue_kq(ci + 1);   // raw K, Q consumed
-            if (CHANNEL && ci + 1 < nchunks) gate_load(ci + 1, gnext);
+            if (ci + 1 < nchunks) {
+                if (CHANNEL) gate_load(ci + 1, gnext);
+                else gate_scalar_load(ci + 1, false, bgnext);
+            }
 
             // T' and P of this chunk from CTA 0; V of this chunk.
             if (tid == 0) {
@@ -676,12 +680,17 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint64_t a = sdesc_sw128(sbase + C_S + ks * 2048, 16384, 1024);
                     mma_bf16(tmem + TM_UT, a, sdesc_sw128(sbase + C_KE + ks * 2048, 8192, 1024), id_u, 1);
+                }
+                mma_commit(bar_mma);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint64_t a = sdesc_sw128(sbase + C_S + ks * 2048, 16384, 1024);
                     const uint64_t bq = sdesc_sw128(sbase + C_QE + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
                     mma_bf16(tmem + TM_OT, a, bq, id_o, ks > 0);
                 }
-                mma_commit(bar_mma);
             }
             mma_sync();
+            if (tid == 0) bulk_wait_read_all();   // the previous O store has read C_OST
             if (__syncthreads_or(!ok)) break;
 
             {   // U^T -> bf16 hi + lo [128 j][64 r]
@@ -707,32 +716,46 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     const uint64_t kdl = sdesc_sw128(sbase + C_KDL + ks * 2048, 8192, 1024);
                     const uint64_t uh = sdesc_sw128(sbase + C_UH + ks * 32, 16, 1024);
                     const uint64_t ul = sdesc_sw128(sbase + C_UL + ks * 32, 16, 1024);
-                    const uint64_t ph = sdesc_sw128(sbase + C_PH + ks * 32, 16, 1024);
-                    const uint64_t pl = sdesc_sw128(sbase + C_PL + ks * 32, 16, 1024);
                     mma_bf16(tmem + TM_SN, kdh, uh, id_s, ks > 0);
                     mma_bf16(tmem + TM_SN, kdh, ul, id_s, 1);
                     mma_bf16(tmem + TM_SN, kdl, uh, id_s, 1);
+                }
+                mma_commit(bar_mma);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t uh = sdesc_sw128(sbase + C_UH + ks * 32, 16, 1024);
+                    const uint64_t ul = sdesc_sw128(sbase + C_UL + ks * 32, 16, 1024);
+                    const uint64_t ph = sdesc_sw128(sbase + C_PH + ks * 32, 16, 1024);
+                    const uint64_t pl = sdesc_sw128(sbase + C_PL + ks * 32, 16, 1024);
                     mma_bf16(tmem + TM_OT, uh, ph, id_o, 1);
                     mma_bf16(tmem + TM_OT, uh, pl, id_o, 1);
                     mma_bf16(tmem + TM_OT, ul, ph, id_o, 1);
                 }
-                mma_commit(bar_mma);
+                mma_commit(bar_out);
             }
             mma_sync();
             if (__syncthreads_or(!ok)) break;
-            if (tid == 0) mbar_arrive_remote(peer_empty);          // slot consumed
 
             {
                 const uint32_t lb = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-                float sn[32];
-#pragma unroll
-                for (int part = 0; part < 2; ++part) {
-                    tmem_ld32(lb + TM_SN + half * 64 + part * 32, sn);
+                {
+                    float sn0[32], sn1[32];
+                    tmem_ld32(lb + TM_SN + half * 64, sn0);
+                    tmem_ld32(lb + TM_SN + half * 64 + 32, sn1);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) s[part * 32 + c] = fmaf(e_last, s[part * 32 + c], sn[c]);
+                    for (int c = 0; c < 32; ++c) {
+                        s[c] = fmaf(e_last, s[c], sn0[c]);
+                        s[32 + c] = fmaf(e_last, s[32 + c], sn1[c]);
+                    }
                 }
                 write_state_f16();
+                // Products into O^T complete (they read P in the slot and U^T):
+                // the slot goes back to CTA 0.  The arrive is made by a thread
+                // of the last warp, which has no global loads in flight.
+                ok = ok && mbar_wait(bar_out, ci & 1, &g_pair_status_word);
+                if (tid == NT - 32 && ok) mbar_arrive_remote_relaxed(peer_empty);
+                tc_fence_after();
                 float o[32];
                 tmem_ld32(lb + TM_OT + half * 32, o);
                 tmem_wait_ld();
@@ -745,7 +768,7 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             fence_async_smem();
             tc_fence_before();
-            __syncthreads();
+            if (__syncthreads_or(!ok)) break;
             if (tid == 0) {
                 tma_store_4d(&tm_o, sbase + C_OST, 0, h, t0, b);
                 bulk_commit();

@@ -83,7 +83,7 @@ constexpr int NT = 256;    // threads per CTA
 constexpr uint32_t R_IN = 0;                 // 32 KB
 constexpr uint32_t OFF_TH = R_IN;            //   8 KB T' hi [64 r][64 m]
 constexpr uint32_t OFF_TL = R_IN + 8192;     //   8 KB T' lo
-constexpr uint32_t OFF_Y = R_IN + 16384;     //   3 KB solve scratch [16][48] fp32
+constexpr uint32_t OFF_Y = R_IN + 16384;     //   5 KB solve scratch [32][40] fp32
 constexpr uint32_t OFF_WT = R_IN + 16384;    //   16 KB W^T fp16 [128 i][64 r] (after solve)
 constexpr uint32_t R_V = 32768;              // 16 KB raw V [half][64][128 B]
 constexpr uint32_t R_S = 49152;              // 32 KB S fp16 [j half][128 i][64 j]
@@ -103,7 +103,7 @@ constexpr uint32_t OFF_KDL = R_X + 49152;    //   16 KB K*D bf16 lo
 constexpr uint32_t OFF_PH = R_X + 65536;     //   8 KB P hi [64 r][64 m]
 constexpr uint32_t OFF_PL = R_X + 73728;     //   8 KB P lo
 constexpr uint32_t OFF_A = R_X + 81920;      //   16 KB A fp32 [64][64]
-constexpr uint32_t OFF_TF = R_X + 98304;     //   16 KB T fp32 [64][64] row-major
+constexpr uint32_t OFF_TF = R_X + 98304;     //   16 KB T fp32 [64][64] (tidx layout)
 constexpr uint32_t OFF_UH = R_X + 81920;     //   16 KB U^T hi [128 j][64 r] (after solve)
 constexpr uint32_t OFF_UL = R_X + 98304;     //   16 KB U^T lo
 constexpr uint32_t R_SMALL = R_X + 114688;
@@ -541,12 +541,12 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         __syncthreads();
 
         // ---------------------------------------------------- T = (I + A)^{-1} --
-        solve_unit_lower64(sA, sTf, sY, tid);
+        solve_unit_lower64_rd(sA, sTf, sY, tid);
         // T' = T Diag(beta) -> bf16 hi + lo, K-major [64 r][64 m].
         for (int e = tid; e < 512; e += NT) {
             const int r = e >> 3, c = e & 7;
-            const float4 t0v = *reinterpret_cast<const float4*>(&sTf[r * 64 + 8 * c]);
-            const float4 t1v = *reinterpret_cast<const float4*>(&sTf[r * 64 + 8 * c + 4]);
+            const float4 t0v = *reinterpret_cast<const float4*>(&sTf[tidx(r, 8 * c)]);
+            const float4 t1v = *reinterpret_cast<const float4*>(&sTf[tidx(r, 8 * c + 4)]);
             const float tt[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
             float tv[8];
 #pragma unroll

@@ -120,6 +120,14 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
                  : "memory");
 }
 
+// Relaxed remote arrive: for a thread that only signals that asynchronous
+// reads it has already observed complete (through another mbarrier) are done,
+// and that publishes no writes of its own to the waiting CTA.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+                 : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t cluster_bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;"
                  ::"r"(cluster_bar), "r"(bytes)
