@@ -501,7 +501,7 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 // Wait until CTA 1 has consumed the previous chunk's slot.
                 ok = ok && mbar_wait_cluster(bar_empty, (ci & 1) ^ 1, &g_pair_status_word);
                 if (ok) {
-                    mbar_arrive_expect_tx_remote(peer_full, SLOT_BYTES);
+                    mbar_arrive_expect_tx_remote_relaxed(peer_full, SLOT_BYTES);
                     bulk_copy_to_peer(peer_slot, sbase + P_STAGE, SLOT_BYTES, peer_full);
                     bulk_commit();
                     copy_pending = true;

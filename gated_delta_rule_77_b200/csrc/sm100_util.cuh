@@ -128,6 +128,15 @@ __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_bar)
                  : "memory");
 }
 
+// Relaxed remote arrive.expect_tx: arms another CTA's mbarrier for a bulk
+// copy whose bytes complete it; the data travels by the copy, not by this
+// thread's writes, so no release is needed.
+__device__ __forceinline__ void mbar_arrive_expect_tx_remote_relaxed(uint32_t cluster_bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;"
+                 ::"r"(cluster_bar), "r"(bytes)
+                 : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t cluster_bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;"
                  ::"r"(cluster_bar), "r"(bytes)
