@@ -42,6 +42,47 @@ __device__ __forceinline__ void store_f16x8(uint8_t* dst, const float* v) {
                                                 pack_f16(v[4], v[5]), pack_f16(v[6], v[7]));
 }
 
+// ---- paired fp32 arithmetic (sm_100 add/sub/mul .f32x2: one instruction for
+// two lanes of a register pair) ------------------------------------------------
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, d;\n\t"
+        "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, d;\n\t"
+        "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// 2^x on the special-function unit (approximate, denormals flushed).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// log2(e): exp(x) = 2^(x log2 e).
+constexpr float kLog2e = 1.44269504088896340736f;
+
+// Four pairs -> bf16 hi and bf16 rounding of the remainder (lo), as store_split.
+__device__ __forceinline__ void store_split2(uint8_t* hi_dst, uint8_t* lo_dst, const float2* v) {
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        hi[e] = pack_bf16(v[e].x, v[e].y);
+        const float2 r = sub2(v[e], make_float2(bf16_lo(hi[e]), bf16_hi(hi[e])));
+        lo[e] = pack_bf16(r.x, r.y);
+    }
+    *reinterpret_cast<uint4*>(hi_dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(lo_dst) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+}
+
 __device__ __forceinline__ void load_bf16x8(const uint8_t* src, float* v) {
     const uint4 w = *reinterpret_cast<const uint4*>(src);
     const uint32_t x[4] = {w.x, w.y, w.z, w.w};

@@ -343,34 +343,50 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (__syncthreads_or(!ok)) break;
 
             if (CHANNEL) {
+                // Channel pairs on the paired fp32 instructions.  Tokens
+                // tg + 16u with u < 2 are before token 32 (reference 15).
+                const float2 l2e = make_float2(kLog2e, kLog2e);
+                float2 ref0[4], ref1[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    ref0[e] = make_float2(sRef0[8 * ck + 2 * e], sRef0[8 * ck + 2 * e + 1]);
+                    ref1[e] = make_float2(sRef1[8 * ck + 2 * e], sRef1[8 * ck + 2 * e + 1]);
+                }
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int r = tg + 16 * u;
-                    const float* ref = r < 32 ? sRef0 : sRef1;
                     float kf[8], qf[8];
                     load_bf16x8(smem + P_IN + ckh * 16384 + swz(r, ckc), kf);
                     load_bf16x8(smem + P_IN + ckh * 16384 + 8192 + swz(r, ckc), qf);
-                    float kr[8], qr[8], kc[8], kc1[8];
+                    float2 kr[4], qr[4], kc[4], kc1[4];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float x = gam[u][e] - ref[8 * ck + e];
-                        const float F = __expf(x);
-                        const float Fi = __expf(-x);
-                        kr[e] = kf[e] * F;
-                        qr[e] = qf[e] * F;
-                        kc[e] = kf[e] * Fi;
-                        kc1[e] = r < 32 ? kf[e] * __expf(sRef1[8 * ck + e] - gam[u][e]) : kc[e];
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 k2 = make_float2(kf[2 * e], kf[2 * e + 1]);
+                        const float2 q2 = make_float2(qf[2 * e], qf[2 * e + 1]);
+                        const float2 g2 = make_float2(gam[u][2 * e], gam[u][2 * e + 1]);
+                        const float2 xl = mul2(sub2(g2, u < 2 ? ref0[e] : ref1[e]), l2e);
+                        const float2 F = make_float2(ex2_approx(xl.x), ex2_approx(xl.y));
+                        const float2 Fi = make_float2(ex2_approx(-xl.x), ex2_approx(-xl.y));
+                        kr[e] = mul2(k2, F);
+                        qr[e] = mul2(q2, F);
+                        kc[e] = mul2(k2, Fi);
+                        if (u < 2) {
+                            const float2 yl = mul2(sub2(ref1[e], g2), l2e);
+                            kc1[e] = mul2(k2, make_float2(ex2_approx(yl.x), ex2_approx(yl.y)));
+                        } else {
+                            kc1[e] = kc[e];
+                        }
                     }
                     const uint32_t o128 = ckh * 16384 + swz(r, ckc);
                     const uint32_t o128q = ckh * 16384 + swz(64 + r, ckc);
-                    store_split(smem + P_AH + o128, smem + P_AL + o128, kr);
-                    store_split(smem + P_AH + o128q, smem + P_AL + o128q, qr);
-                    if (r < 32) {
+                    store_split2(smem + P_AH + o128, smem + P_AL + o128, kr);
+                    store_split2(smem + P_AH + o128q, smem + P_AL + o128q, qr);
+                    if (u < 2) {
                         const uint32_t o32 = ckh * 4096 + swz(r, ckc);
-                        store_split(smem + P_C0H + o32, smem + P_C0L + o32, kc);
+                        store_split2(smem + P_C0H + o32, smem + P_C0L + o32, kc);
                     }
                     const uint32_t o64 = ckh * 8192 + swz(r, ckc);
-                    store_split(smem + P_C1H + o64, smem + P_C1L + o64, kc1);
+                    store_split2(smem + P_C1H + o64, smem + P_C1L + o64, kc1);
                 }
                 fence_async_smem();
                 __syncthreads();
@@ -592,36 +608,50 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             kq_waited = ci;
             if (__syncthreads_or(!ok)) break;
 
-            // K*E (bf16), Q*E (fp16), K*D (bf16 hi + lo).
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int r = tg + 16 * u;
-                float kf[8], qf[8], ke[8], qe[8], kd[8];
-                load_bf16x8(smem + C_IN + ckh * 16384 + swz(r, ckc), kf);
-                load_bf16x8(smem + C_IN + ckh * 16384 + 8192 + swz(r, ckc), qf);
+            // K*E (bf16), Q*E (fp16), K*D (bf16 hi + lo), on channel pairs.
+            {
+                const float2 l2e = make_float2(kLog2e, kLog2e);
+                float2 last2[4];
                 if (CHANNEL) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float E = __expf(gam[u][e]);
-                        const float Dd = __expf(sLast[8 * ck + e] - gam[u][e]);
-                        ke[e] = kf[e] * E;
-                        qe[e] = qf[e] * E;
-                        kd[e] = kf[e] * Dd;
-                    }
-                } else {
-                    const float E = __expf(sGam[r]);
-                    const float Dd = __expf(sGam[C - 1] - sGam[r]);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        ke[e] = kf[e] * E;
-                        qe[e] = qf[e] * E;
-                        kd[e] = kf[e] * Dd;
-                    }
+                    for (int e = 0; e < 4; ++e)
+                        last2[e] = make_float2(sLast[8 * ck + 2 * e], sLast[8 * ck + 2 * e + 1]);
                 }
-                const uint32_t o64 = ckh * 8192 + swz(r, ckc);
-                store_bf16x8(smem + C_KE + o64, ke);
-                store_f16x8(smem + C_QE + o64, qe);
-                store_split(smem + C_KDH + o64, smem + C_KDL + o64, kd);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int r = tg + 16 * u;
+                    float kf[8], qf[8], ke[8], qe[8];
+                    float2 kd[4];
+                    load_bf16x8(smem + C_IN + ckh * 16384 + swz(r, ckc), kf);
+                    load_bf16x8(smem + C_IN + ckh * 16384 + 8192 + swz(r, ckc), qf);
+                    float2 E2 = make_float2(0.f, 0.f), D2 = E2;
+                    if (!CHANNEL) {
+                        const float E = ex2_approx(sGam[r] * kLog2e);
+                        const float Dd = ex2_approx((sGam[C - 1] - sGam[r]) * kLog2e);
+                        E2 = make_float2(E, E);
+                        D2 = make_float2(Dd, Dd);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 k2 = make_float2(kf[2 * e], kf[2 * e + 1]);
+                        const float2 q2 = make_float2(qf[2 * e], qf[2 * e + 1]);
+                        if (CHANNEL) {
+                            const float2 g2 = make_float2(gam[u][2 * e], gam[u][2 * e + 1]);
+                            const float2 el = mul2(g2, l2e);
+                            const float2 dl = mul2(sub2(last2[e], g2), l2e);
+                            E2 = make_float2(ex2_approx(el.x), ex2_approx(el.y));
+                            D2 = make_float2(ex2_approx(dl.x), ex2_approx(dl.y));
+                        }
+                        const float2 ke2 = mul2(k2, E2), qe2 = mul2(q2, E2);
+                        ke[2 * e] = ke2.x; ke[2 * e + 1] = ke2.y;
+                        qe[2 * e] = qe2.x; qe[2 * e + 1] = qe2.y;
+                        kd[e] = mul2(k2, D2);
+                    }
+                    const uint32_t o64 = ckh * 8192 + swz(r, ckc);
+                    store_bf16x8(smem + C_KE + o64, ke);
+                    store_f16x8(smem + C_QE + o64, qe);
+                    store_split2(smem + C_KDH + o64, smem + C_KDL + o64, kd);
+                }
             }
             const float e_last = __expf(CHANNEL ? sLast[srow] : sGam[C - 1]);
             fence_async_smem();
