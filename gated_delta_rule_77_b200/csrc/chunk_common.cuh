@@ -19,6 +19,33 @@ __device__ __forceinline__ uint32_t fidx(int r, int m) {
     return static_cast<uint32_t>(r * 64 + ((((m >> 2) ^ r) & 15) << 2) + (m & 3));
 }
 
+// ---- paired fp32 arithmetic (sm_100 add/sub/mul .f32x2: one instruction for
+// two lanes of a register pair) ------------------------------------------------
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, d;\n\t"
+        "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+        "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+        "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, d;\n\t"
+        "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
 // Eight fp32 values -> a 16-byte bf16 chunk (hi) and the bf16 rounding of the
 // remainder (lo), so that hi + lo reproduces each value to ~2^-16.
 __device__ __forceinline__ void store_split(uint8_t* hi_dst, uint8_t* lo_dst, const float* v) {
@@ -26,7 +53,8 @@ __device__ __forceinline__ void store_split(uint8_t* hi_dst, uint8_t* lo_dst, co
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
         hi[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
-        lo[e] = pack_bf16(v[2 * e] - bf16_lo(hi[e]), v[2 * e + 1] - bf16_hi(hi[e]));
+        const float2 r = sub2(make_float2(v[2 * e], v[2 * e + 1]), make_float2(bf16_lo(hi[e]), bf16_hi(hi[e])));
+        lo[e] = pack_bf16(r.x, r.y);
     }
     *reinterpret_cast<uint4*>(hi_dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
     *reinterpret_cast<uint4*>(lo_dst) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
@@ -40,25 +68,6 @@ __device__ __forceinline__ void store_bf16x8(uint8_t* dst, const float* v) {
 __device__ __forceinline__ void store_f16x8(uint8_t* dst, const float* v) {
     *reinterpret_cast<uint4*>(dst) = make_uint4(pack_f16(v[0], v[1]), pack_f16(v[2], v[3]),
                                                 pack_f16(v[4], v[5]), pack_f16(v[6], v[7]));
-}
-
-// ---- paired fp32 arithmetic (sm_100 add/sub/mul .f32x2: one instruction for
-// two lanes of a register pair) ------------------------------------------------
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 a, b, d;\n\t"
-        "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
-        "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 a, b, d;\n\t"
-        "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
-        "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
 }
 
 // 2^x on the special-function unit (approximate, denormals flushed).

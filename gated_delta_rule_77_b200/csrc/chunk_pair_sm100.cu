@@ -773,10 +773,12 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     tmem_ld32(lb + TM_SN + half * 64, sn0);
                     tmem_ld32(lb + TM_SN + half * 64 + 32, sn1);
                     tmem_wait_ld();
+                    const float2 e2 = make_float2(e_last, e_last);
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        s[c] = fmaf(e_last, s[c], sn0[c]);
-                        s[32 + c] = fmaf(e_last, s[32 + c], sn1[c]);
+                    for (int c = 0; c < 32; c += 2) {
+                        float2 a = fma2(e2, make_float2(s[c], s[c + 1]), make_float2(sn0[c], sn0[c + 1]));
+                        float2 z = fma2(e2, make_float2(s[32 + c], s[33 + c]), make_float2(sn1[c], sn1[c + 1]));
+                        s[c] = a.x; s[c + 1] = a.y; s[32 + c] = z.x; s[33 + c] = z.y;
                     }
                 }
                 write_state_f16();
