@@ -166,12 +166,13 @@ struct Acc3 {
 //   1. the four 16x16 diagonal blocks by forward substitution (fp32);
 //   2. both 32x32 diagonal blocks: T_10 = -D_1 (A_10 D_0), T_32 = -D_3 (A_32 D_2);
 //   3. the lower-left 32x32 block: -T_BB (A_BA T_AA).
-// Five dependent stages instead of the seven of the row-block levels.  The
+// The part of Y = A_BA T_AA that needs only the diagonal blocks D_0, D_1 runs
+// during stage 2 on warps 4-7; only the term with T_10 waits for it.  The
 // products run on mma.m16n8k8 (tf32, hi/lo splits, fp32-class accuracy); the
 // triangular operands' zero blocks are skipped.  T is written in the tidx
 // layout (entries above the diagonal of the diagonal 16x16 blocks are zero,
-// the rest of the upper triangle is not written).  Y scratch: [32][40] fp32.
-// Ends with a barrier.
+// the rest of the upper triangle is not written).  Scratch sY: two [32][40]
+// fp32 tiles (10 KB).  Needs 8 warps; ends with a barrier.
 __device__ __forceinline__ void solve_unit_lower64_rd(const float* sA, float* sT, float* sY, int tid) {
     const int warp = tid >> 5, lane = tid & 31;
     const int grp = lane >> 2, tig = lane & 3;
@@ -196,9 +197,34 @@ __device__ __forceinline__ void solve_unit_lower64_rd(const float* sA, float* sT
     }
     __syncthreads();
 
+    float* sY3 = sY + 32 * 40;           // Y = A_BA T_AA, [32][40]
     // Stage 2, first product: Y_b = A[32b+16.., 32b..+16] D_{2b} (16x16 each),
     // warps 0-3: b = warp >> 1, output columns 8 nt.. with nt = warp & 1.
-    if (warp < 4) {
+    // Warps 4-7: the D_0 / D_1 terms of Y = A_BA T_AA, row tile mt = (warp-4)>>1,
+    // column tiles nt = 2((warp-4)&1) and +1.
+    if (warp >= 4) {
+        const int w = warp - 4, mt = w >> 1;
+        float* y = sY3 + (16 * mt) * 40;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int nt = 2 * (w & 1) + q;
+            Acc3 acc;
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+                const int ks = 2 * (nt >> 1) + kk;       // 8-row group inside D_0 or D_1
+                if (ks < nt) continue;
+                const int k0 = 8 * ks + tig;
+                const int r0 = 32 + 16 * mt + grp;
+                const float af[4] = {sA[fidx(r0, k0)], sA[fidx(r0 + 8, k0)], sA[fidx(r0, k0 + 4)],
+                                     sA[fidx(r0 + 8, k0 + 4)]};
+                const float bf[2] = {sT[tidx(k0, 8 * nt + grp)], sT[tidx(k0 + 4, 8 * nt + grp)]};
+                acc.add(af, bf);
+            }
+            const int c = 8 * nt + 2 * tig;
+            *reinterpret_cast<float2*>(&y[grp * 40 + c]) = make_float2(acc.sum(0), acc.sum(1));
+            *reinterpret_cast<float2*>(&y[(grp + 8) * 40 + c]) = make_float2(acc.sum(2), acc.sum(3));
+        }
+    } else {
         const int bb = warp >> 1, nt = warp & 1, base = 32 * bb;
         Acc3 acc;
 #pragma unroll
@@ -240,14 +266,13 @@ __device__ __forceinline__ void solve_unit_lower64_rd(const float* sA, float* sT
     }
     __syncthreads();
 
-    // Stage 3: Y = A[32.., 0..32] T[0..32, 0..32] (32x32), then
-    // T[32.., 0..32] = -T[32.., 32..] Y.  Warp = (row tile mt, column tile nt).
-    const int mt = warp >> 2, nt = warp & 3;
-    {
+    // Stage 3: the T_10 term, Y[:, 0..16] += A[32.., 16..32] T_10 (warps 0-3:
+    // mt = warp >> 1, nt = warp & 1), then T[32.., 0..32] = -T[32.., 32..] Y.
+    if (warp < 4) {
+        const int mt = warp >> 1, nt = warp & 1;
         Acc3 acc;
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            if (ks < nt) continue;                       // T_AA is lower triangular
+        for (int ks = 2; ks < 4; ++ks) {
             const int k0 = 8 * ks + tig;
             const int r0 = 32 + 16 * mt + grp;
             const float af[4] = {sA[fidx(r0, k0)], sA[fidx(r0 + 8, k0)], sA[fidx(r0, k0 + 4)],
@@ -256,11 +281,14 @@ __device__ __forceinline__ void solve_unit_lower64_rd(const float* sA, float* sT
             acc.add(af, bf);
         }
         const int c = 8 * nt + 2 * tig;
-        float* y = sY + (16 * mt) * 40;
-        *reinterpret_cast<float2*>(&y[grp * 40 + c]) = make_float2(acc.sum(0), acc.sum(1));
-        *reinterpret_cast<float2*>(&y[(grp + 8) * 40 + c]) = make_float2(acc.sum(2), acc.sum(3));
+        float* y = sY3 + (16 * mt) * 40;
+        float2* y0 = reinterpret_cast<float2*>(&y[grp * 40 + c]);
+        float2* y1 = reinterpret_cast<float2*>(&y[(grp + 8) * 40 + c]);
+        *y0 = make_float2(y0->x + acc.sum(0), y0->y + acc.sum(1));
+        *y1 = make_float2(y1->x + acc.sum(2), y1->y + acc.sum(3));
     }
     __syncthreads();
+    const int mt = warp >> 2, nt = warp & 3;
     {
         Acc3 acc;
 #pragma unroll
@@ -270,7 +298,7 @@ __device__ __forceinline__ void solve_unit_lower64_rd(const float* sA, float* sT
             const int r0 = 32 + 16 * mt + grp;
             const float af[4] = {sT[tidx(r0, 32 + k0)], sT[tidx(r0 + 8, 32 + k0)],
                                  sT[tidx(r0, 32 + k0 + 4)], sT[tidx(r0 + 8, 32 + k0 + 4)]};
-            const float bf[2] = {sY[k0 * 40 + 8 * nt + grp], sY[(k0 + 4) * 40 + 8 * nt + grp]};
+            const float bf[2] = {sY3[k0 * 40 + 8 * nt + grp], sY3[(k0 + 4) * 40 + 8 * nt + grp]};
             acc.add(af, bf);
         }
         const int c = 8 * nt + 2 * tig;

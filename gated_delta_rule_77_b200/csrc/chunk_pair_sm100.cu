@@ -61,7 +61,7 @@ constexpr uint32_t P_C1H = P_X + 81920;       //   16 KB
 constexpr uint32_t P_C1L = P_X + 98304;       //   16 KB
 constexpr uint32_t P_A = P_X + 32768;         //   16 KB A fp32 (fidx layout)
 constexpr uint32_t P_T = P_X + 49152;         //   16 KB T fp32 (tidx layout)
-constexpr uint32_t P_Y = P_X + 65536;         //   5 KB solve scratch [32][40]
+constexpr uint32_t P_Y = P_X + 65536;         //   10 KB solve scratch 2 x [32][40]
 constexpr uint32_t P_SMALL = P_X + 114688;
 constexpr uint32_t P_GAM = P_SMALL;           // 64 f32
 constexpr uint32_t P_BETA = P_GAM + 256;      // 64 f32

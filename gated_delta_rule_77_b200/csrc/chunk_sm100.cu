@@ -83,7 +83,7 @@ constexpr int NT = 256;    // threads per CTA
 constexpr uint32_t R_IN = 0;                 // 32 KB
 constexpr uint32_t OFF_TH = R_IN;            //   8 KB T' hi [64 r][64 m]
 constexpr uint32_t OFF_TL = R_IN + 8192;     //   8 KB T' lo
-constexpr uint32_t OFF_Y = R_IN + 16384;     //   5 KB solve scratch [32][40] fp32
+constexpr uint32_t OFF_Y = R_IN + 16384;     //   10 KB solve scratch 2 x [32][40] fp32
 constexpr uint32_t OFF_WT = R_IN + 16384;    //   16 KB W^T fp16 [128 i][64 r] (after solve)
 constexpr uint32_t R_V = 32768;              // 16 KB raw V [half][64][128 B]
 constexpr uint32_t R_S = 49152;              // 32 KB S fp16 [j half][128 i][64 j]
