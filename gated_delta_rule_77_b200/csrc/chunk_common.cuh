@@ -172,7 +172,8 @@ struct Acc3 {
 // triangular operands' zero blocks are skipped.  T is written in the tidx
 // layout (entries above the diagonal of the diagonal 16x16 blocks are zero,
 // the rest of the upper triangle is not written).  Scratch sY: two [32][40]
-// fp32 tiles (10 KB).  Needs 8 warps; ends with a barrier.
+// fp32 tiles (10 KB).  Works on warps 0-7 of a CTA of at least 8 warps (any
+// further warps only take part in the barriers); ends with a barrier.
 __device__ __forceinline__ void solve_unit_lower64_rd(const float* sA, float* sT, float* sY, int tid) {
     const int warp = tid >> 5, lane = tid & 31;
     const int grp = lane >> 2, tig = lane & 3;
@@ -202,7 +203,7 @@ __device__ __forceinline__ void solve_unit_lower64_rd(const float* sA, float* sT
     // warps 0-3: b = warp >> 1, output columns 8 nt.. with nt = warp & 1.
     // Warps 4-7: the D_0 / D_1 terms of Y = A_BA T_AA, row tile mt = (warp-4)>>1,
     // column tiles nt = 2((warp-4)&1) and +1.
-    if (warp >= 4) {
+    if (warp >= 4 && warp < 8) {
         const int w = warp - 4, mt = w >> 1;
         float* y = sY3 + (16 * mt) * 40;
 #pragma unroll
@@ -224,7 +225,7 @@ __device__ __forceinline__ void solve_unit_lower64_rd(const float* sA, float* sT
             *reinterpret_cast<float2*>(&y[grp * 40 + c]) = make_float2(acc.sum(0), acc.sum(1));
             *reinterpret_cast<float2*>(&y[(grp + 8) * 40 + c]) = make_float2(acc.sum(2), acc.sum(3));
         }
-    } else {
+    } else if (warp < 4) {
         const int bb = warp >> 1, nt = warp & 1, base = 32 * bb;
         Acc3 acc;
 #pragma unroll
@@ -289,7 +290,7 @@ __device__ __forceinline__ void solve_unit_lower64_rd(const float* sA, float* sT
     }
     __syncthreads();
     const int mt = warp >> 2, nt = warp & 3;
-    {
+    if (warp < 8) {
         Acc3 acc;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {

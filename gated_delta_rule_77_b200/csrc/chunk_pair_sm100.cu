@@ -55,10 +55,13 @@ constexpr uint32_t P_IN = 0;                  // 32 KB raw K, Q [half][K 64 | Q 
 constexpr uint32_t P_X = 32768;               // 112 KB:
 constexpr uint32_t P_AH = P_X;                //   X operands (per-channel): 32 KB
 constexpr uint32_t P_AL = P_X + 32768;        //   32 KB
-constexpr uint32_t P_C0H = P_X + 65536;       //   8 KB
-constexpr uint32_t P_C0L = P_X + 73728;       //   8 KB
-constexpr uint32_t P_C1H = P_X + 81920;       //   16 KB
-constexpr uint32_t P_C1L = P_X + 98304;       //   16 KB
+// B operand of X, hi and lo, [64-channel half][96 rows][128 B]: rows 0-31 =
+// K/F of tokens 0-31 (reference 15), rows 32-95 = K*exp(G_47 - G) of tokens
+// 0-63, so that one N = 96 product per k-step covers both (fewer operand
+// reads from shared memory than separate N = 32 and N = 64 products).
+constexpr uint32_t P_CBH = P_X + 65536;       //   24 KB
+constexpr uint32_t P_CBL = P_X + 90112;       //   24 KB
+constexpr uint32_t CB_HALF = 96 * 128;
 constexpr uint32_t P_A = P_X + 32768;         //   16 KB A fp32 (fidx layout)
 constexpr uint32_t P_T = P_X + 49152;         //   16 KB T fp32 (tidx layout)
 constexpr uint32_t P_Y = P_X + 65536;         //   10 KB solve scratch 2 x [32][40]
@@ -382,11 +385,11 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     store_split2(smem + P_AH + o128, smem + P_AL + o128, kr);
                     store_split2(smem + P_AH + o128q, smem + P_AL + o128q, qr);
                     if (u < 2) {
-                        const uint32_t o32 = ckh * 4096 + swz(r, ckc);
-                        store_split2(smem + P_C0H + o32, smem + P_C0L + o32, kc);
+                        const uint32_t o32 = ckh * CB_HALF + swz(r, ckc);
+                        store_split2(smem + P_CBH + o32, smem + P_CBL + o32, kc);
                     }
-                    const uint32_t o64 = ckh * 8192 + swz(r, ckc);
-                    store_split2(smem + P_C1H + o64, smem + P_C1L + o64, kc1);
+                    const uint32_t o64 = ckh * CB_HALF + swz(32 + r, ckc);
+                    store_split2(smem + P_CBH + o64, smem + P_CBL + o64, kc1);
                 }
                 fence_async_smem();
                 __syncthreads();
@@ -395,25 +398,18 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (tid == 0) {
                 tc_fence_after();
                 if (CHANNEL) {
-                    const uint32_t id0 = idesc_bf16(128, 32, false, false);
-                    const uint32_t id1 = idesc_bf16(128, 64, false, false);
+                    const uint32_t id = idesc_bf16(128, 96, false, false);
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {
                         const uint32_t ka = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        const uint32_t k0 = (ks >> 2) * 4096 + (ks & 3) * 32;
-                        const uint32_t k1 = (ks >> 2) * 8192 + (ks & 3) * 32;
+                        const uint32_t kb = (ks >> 2) * CB_HALF + (ks & 3) * 32;
                         const uint64_t ah = sdesc_sw128(sbase + P_AH + ka, 16, 1024);
                         const uint64_t al = sdesc_sw128(sbase + P_AL + ka, 16, 1024);
-                        const uint64_t b0h = sdesc_sw128(sbase + P_C0H + k0, 16, 1024);
-                        const uint64_t b0l = sdesc_sw128(sbase + P_C0L + k0, 16, 1024);
-                        const uint64_t b1h = sdesc_sw128(sbase + P_C1H + k1, 16, 1024);
-                        const uint64_t b1l = sdesc_sw128(sbase + P_C1L + k1, 16, 1024);
-                        mma_bf16(tmem + TM_X, ah, b0h, id0, ks > 0);
-                        mma_bf16(tmem + TM_X, ah, b0l, id0, 1);
-                        mma_bf16(tmem + TM_X, al, b0h, id0, 1);
-                        mma_bf16(tmem + TM_X + 32, ah, b1h, id1, ks > 0);
-                        mma_bf16(tmem + TM_X + 32, ah, b1l, id1, 1);
-                        mma_bf16(tmem + TM_X + 32, al, b1h, id1, 1);
+                        const uint64_t bh = sdesc_sw128(sbase + P_CBH + kb, 16, 1024);
+                        const uint64_t bl = sdesc_sw128(sbase + P_CBL + kb, 16, 1024);
+                        mma_bf16(tmem + TM_X, ah, bh, id, ks > 0);
+                        mma_bf16(tmem + TM_X, ah, bl, id, 1);
+                        mma_bf16(tmem + TM_X, al, bh, id, 1);
                     }
                 } else {
                     const uint32_t id = idesc_bf16(128, 64, false, false);
