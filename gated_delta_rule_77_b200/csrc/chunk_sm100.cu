@@ -91,10 +91,9 @@ constexpr uint32_t R_X = 81920;              // 112 KB, two uses per chunk:
 //  (a) X operands (per-channel gate), bf16 hi / lo:
 constexpr uint32_t OFF_AH = R_X;             //   32 KB [half][K*F 64 | Q*F 64][128 B]
 constexpr uint32_t OFF_AL = R_X + 32768;     //   32 KB
-constexpr uint32_t OFF_C0H = R_X + 65536;    //   8 KB [half][32][128 B]  K/F (ref 15)
-constexpr uint32_t OFF_C0L = R_X + 73728;    //   8 KB
-constexpr uint32_t OFF_C1H = R_X + 81920;    //   16 KB [half][64][128 B] K*exp(G_47 - G)
-constexpr uint32_t OFF_C1L = R_X + 98304;    //   16 KB
+constexpr uint32_t OFF_CBH = R_X + 65536;    //   24 KB [half][96][128 B]: rows 0-31 K/F (ref 15),
+constexpr uint32_t OFF_CBL = R_X + 90112;    //   24 KB   rows 32-95 K*exp(G_47 - G); one N = 96 B
+constexpr uint32_t CB_HALF = 96 * 128;
 //  (b) after X: derived tiles, P, solve input, U
 constexpr uint32_t OFF_KE = R_X;             //   16 KB K*E bf16  [half][64 r][128 B]
 constexpr uint32_t OFF_QE = R_X + 16384;     //   16 KB Q*E fp16
@@ -115,8 +114,8 @@ constexpr uint32_t SM_LAST = SM_REF1 + 512;   // 128 f32: G at token 63
 constexpr uint32_t SM_ER = SM_LAST + 512;     // 64 f32: exp(G_r - G_31)  (scalar gate)
 constexpr uint32_t SM_FJ = SM_ER + 256;       // 64 f32: exp(G_31 - G_j)
 constexpr uint32_t SM_SAFE = SM_FJ + 256;     // int: product form in range
-constexpr uint32_t SM_BAR = SM_SAFE + 16;     // 2 mbarriers
-constexpr uint32_t SM_TMEM = SM_BAR + 16;     // TMEM base address
+constexpr uint32_t SM_BAR = SM_SAFE + 16;     // 3 mbarriers: loads, products, products into O
+constexpr uint32_t SM_TMEM = SM_BAR + 24;     // TMEM base address
 constexpr uint32_t SMEM_USED = SM_TMEM + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 
@@ -168,6 +167,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     float* sY = reinterpret_cast<float*>(smem + OFF_Y);
     const uint32_t bar_tma = sbase + SM_BAR;
     const uint32_t bar_mma = sbase + SM_BAR + 8;
+    const uint32_t bar_out = sbase + SM_BAR + 16;   // O^T products, committed apart
     uint32_t* sTmemBase = reinterpret_cast<uint32_t*>(smem + SM_TMEM);
 
     const int tid = threadIdx.x;
@@ -186,6 +186,9 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int t_begin = seg * p.seg_len;
     const int t_end = min(T, t_begin + p.seg_len);
     const int nchunks = t_end > t_begin ? (t_end - t_begin + C - 1) / C : 0;
+    // Outputs are formed only where they are written (not by transition CTAs
+    // nor by the zero-start pass of the segment path).
+    const bool want_o = !transition && p.out != nullptr;
 
     // Element ownership for the gate prep and tile building: 16 channel
     // chunks of 8 (ck) x 16 lanes (tg), lane tg owning tokens tg + 16 u,
@@ -203,6 +206,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         prefetch_tensormap(&tm_v);
         mbar_init(bar_tma, 1);
         mbar_init(bar_mma, 1);
+        mbar_init(bar_out, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -266,6 +270,44 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tc_fence_after();
     };
 
+    // g (per-channel: this thread's 4 tokens x 8 channels) and, in warp 0,
+    // beta and the scalar g are loaded into registers one chunk ahead, issued
+    // after a shared-memory proxy fence (which would wait for them).
+    auto load_gate = [&](int chunk, float (&gn)[4][8]) {
+        const int tc0 = t_begin + chunk * C;
+        const long tkc = ((long)b * T + tc0) * H + h;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int r = tg + 16 * u;
+            if (tc0 + r < t_end) {
+                const float4* src = reinterpret_cast<const float4*>(p.g + (tkc + (long)r * H) * D + 8 * ck);
+                const float4 a = src[0], c = src[1];
+                gn[u][0] = a.x; gn[u][1] = a.y; gn[u][2] = a.z; gn[u][3] = a.w;
+                gn[u][4] = c.x; gn[u][5] = c.y; gn[u][6] = c.z; gn[u][7] = c.w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) gn[u][e] = 0.f;
+            }
+        }
+    };
+    auto load_beta = [&](int chunk, float (&bg)[4]) {   // warp 0: lane, 32 + lane
+        bg[0] = bg[1] = bg[2] = bg[3] = 0.f;
+        if (warp != 0) return;
+        const int tc0 = t_begin + chunk * C;
+        const long tkc = ((long)b * T + tc0) * H + h;
+        if (tc0 + lane < t_end) {
+            bg[0] = p.beta[tkc + (long)lane * H];
+            if (!CHANNEL) bg[2] = p.g[tkc + (long)lane * H];
+        }
+        if (tc0 + 32 + lane < t_end) {
+            bg[1] = p.beta[tkc + (long)(32 + lane) * H];
+            if (!CHANNEL) bg[3] = p.g[tkc + (long)(32 + lane) * H];
+        }
+    };
+    float gnext[4][8], bgnext[4];
+    if (CHANNEL && nchunks > 0) load_gate(0, gnext);
+    if (nchunks > 0) load_beta(0, bgnext);
+
     for (int ci = 0; ci < nchunks; ++ci) {
         const int t0 = t_begin + ci * C;
         const long tk0 = ((long)b * T + t0) * H + h;     // flat (b, t0, h)
@@ -276,19 +318,9 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         float gam[4][8];
         if (CHANNEL) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int r = tg + 16 * u;
-                if (t0 + r < t_end) {
-                    const float4* src = reinterpret_cast<const float4*>(
-                        p.g + (tk0 + (long)r * H) * D + 8 * ck);
-                    const float4 a = src[0], c = src[1];
-                    gam[u][0] = a.x; gam[u][1] = a.y; gam[u][2] = a.z; gam[u][3] = a.w;
-                    gam[u][4] = c.x; gam[u][5] = c.y; gam[u][6] = c.z; gam[u][7] = c.w;
-                } else {
+            for (int u = 0; u < 4; ++u)
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) gam[u][e] = 0.f;
-                }
-            }
+                for (int e = 0; e < 8; ++e) gam[u][e] = gnext[u][e];
             // Inclusive scan over the 16 lanes of each 16-token block, then add
             // the totals of the preceding blocks.
 #pragma unroll
@@ -311,10 +343,10 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     off += tot;
                 }
             }
-            if (ci + 1 < nchunks) {   // warm L2 with the next chunk's gate rows
+            if (ci + 2 < nchunks) {   // warm L2 two chunks ahead
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const int r = C + tg + 16 * u;
+                    const int r = 2 * C + tg + 16 * u;
                     if (t0 + r < t_end) prefetch_l2(p.g + (tk0 + (long)r * H) * D + 8 * ck);
                 }
             }
@@ -328,15 +360,8 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
         }
         if (warp == 0) {
-            float b0 = 0.f, b1 = 0.f, g0 = 0.f, g1 = 0.f;
-            if (t0 + lane < t_end) {
-                b0 = p.beta[tk0 + (long)lane * H];
-                if (!CHANNEL) g0 = p.g[tk0 + (long)lane * H];
-            }
-            if (t0 + 32 + lane < t_end) {
-                b1 = p.beta[tk0 + (long)(32 + lane) * H];
-                if (!CHANNEL) g1 = p.g[tk0 + (long)(32 + lane) * H];
-            }
+            const float b0 = bgnext[0], b1 = bgnext[1];
+            float g0 = bgnext[2], g1 = bgnext[3];
             sBeta[lane] = b0;
             sBeta[32 + lane] = b1;
             if (!CHANNEL) {
@@ -373,60 +398,70 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // ---------------------------------------------------- X = raw A and P --
         if (CHANNEL) {
             // Factored operands, bf16 hi + lo (see header).
+            // Channel pairs on the paired fp32 instructions; tokens tg + 16u
+            // with u < 2 are before token 32 (reference 15).
+            const float2 l2e = make_float2(kLog2e, kLog2e);
+            float2 ref0[4], ref1[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                ref0[e] = make_float2(sRef0[8 * ck + 2 * e], sRef0[8 * ck + 2 * e + 1]);
+                ref1[e] = make_float2(sRef1[8 * ck + 2 * e], sRef1[8 * ck + 2 * e + 1]);
+            }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int r = tg + 16 * u;
-                const float* ref = r < 32 ? sRef0 : sRef1;
                 float kf[8], qf[8];
                 load_bf16x8(smem + R_IN + ckh * 16384 + swz(r, ckc), kf);
                 load_bf16x8(smem + R_IN + ckh * 16384 + 8192 + swz(r, ckc), qf);
-                float kr[8], qr[8], kc[8], kc1[8];
+                float2 kr[4], qr[4], kc[4], kc1[4];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float x = gam[u][e] - ref[8 * ck + e];
-                    const float F = __expf(x);
-                    const float Fi = __expf(-x);
-                    kr[e] = kf[e] * F;
-                    qr[e] = qf[e] * F;
-                    kc[e] = kf[e] * Fi;
-                    kc1[e] = r < 32 ? kf[e] * __expf(sRef1[8 * ck + e] - gam[u][e]) : kc[e];
+                for (int e = 0; e < 4; ++e) {
+                    const float2 k2 = make_float2(kf[2 * e], kf[2 * e + 1]);
+                    const float2 q2 = make_float2(qf[2 * e], qf[2 * e + 1]);
+                    const float2 g2 = make_float2(gam[u][2 * e], gam[u][2 * e + 1]);
+                    const float2 xl = mul2(sub2(g2, u < 2 ? ref0[e] : ref1[e]), l2e);
+                    const float2 F = make_float2(ex2_approx(xl.x), ex2_approx(xl.y));
+                    const float2 Fi = make_float2(ex2_approx(-xl.x), ex2_approx(-xl.y));
+                    kr[e] = mul2(k2, F);
+                    qr[e] = mul2(q2, F);
+                    kc[e] = mul2(k2, Fi);
+                    if (u < 2) {
+                        const float2 yl = mul2(sub2(ref1[e], g2), l2e);
+                        kc1[e] = mul2(k2, make_float2(ex2_approx(yl.x), ex2_approx(yl.y)));
+                    } else {
+                        kc1[e] = kc[e];
+                    }
                 }
                 const uint32_t o128 = ckh * 16384 + swz(r, ckc);
                 const uint32_t o128q = ckh * 16384 + swz(64 + r, ckc);
-                store_split(smem + OFF_AH + o128, smem + OFF_AL + o128, kr);
-                store_split(smem + OFF_AH + o128q, smem + OFF_AL + o128q, qr);
-                if (r < 32) {
-                    const uint32_t o32 = ckh * 4096 + swz(r, ckc);
-                    store_split(smem + OFF_C0H + o32, smem + OFF_C0L + o32, kc);
+                store_split2(smem + OFF_AH + o128, smem + OFF_AL + o128, kr);
+                store_split2(smem + OFF_AH + o128q, smem + OFF_AL + o128q, qr);
+                if (u < 2) {
+                    const uint32_t o32 = ckh * CB_HALF + swz(r, ckc);
+                    store_split2(smem + OFF_CBH + o32, smem + OFF_CBL + o32, kc);
                 }
-                const uint32_t o64 = ckh * 8192 + swz(r, ckc);
-                store_split(smem + OFF_C1H + o64, smem + OFF_C1L + o64, kc1);
+                const uint32_t o64 = ckh * CB_HALF + swz(32 + r, ckc);
+                store_split2(smem + OFF_CBH + o64, smem + OFF_CBL + o64, kc1);
             }
             fence_async_smem();
             __syncthreads();
+            if (ci + 1 < nchunks) load_gate(ci + 1, gnext);
         }
         if (tid == 0) {
             tc_fence_after();
             if (CHANNEL) {
-                const uint32_t id0 = idesc_bf16(128, 32, false, false);
-                const uint32_t id1 = idesc_bf16(128, 64, false, false);
+                const uint32_t id = idesc_bf16(128, 96, false, false);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t ka = (ks >> 2) * 16384 + (ks & 3) * 32;
-                    const uint32_t k0 = (ks >> 2) * 4096 + (ks & 3) * 32;
-                    const uint32_t k1 = (ks >> 2) * 8192 + (ks & 3) * 32;
+                    const uint32_t kb = (ks >> 2) * CB_HALF + (ks & 3) * 32;
                     const uint64_t ah = sdesc_sw128(sbase + OFF_AH + ka, 16, 1024);
                     const uint64_t al = sdesc_sw128(sbase + OFF_AL + ka, 16, 1024);
-                    const uint64_t b0h = sdesc_sw128(sbase + OFF_C0H + k0, 16, 1024);
-                    const uint64_t b0l = sdesc_sw128(sbase + OFF_C0L + k0, 16, 1024);
-                    const uint64_t b1h = sdesc_sw128(sbase + OFF_C1H + k1, 16, 1024);
-                    const uint64_t b1l = sdesc_sw128(sbase + OFF_C1L + k1, 16, 1024);
-                    mma_bf16(tmem + TM_X, ah, b0h, id0, ks > 0);
-                    mma_bf16(tmem + TM_X, ah, b0l, id0, 1);
-                    mma_bf16(tmem + TM_X, al, b0h, id0, 1);
-                    mma_bf16(tmem + TM_X + 32, ah, b1h, id1, ks > 0);
-                    mma_bf16(tmem + TM_X + 32, ah, b1l, id1, 1);
-                    mma_bf16(tmem + TM_X + 32, al, b1h, id1, 1);
+                    const uint64_t bh = sdesc_sw128(sbase + OFF_CBH + kb, 16, 1024);
+                    const uint64_t bl = sdesc_sw128(sbase + OFF_CBL + kb, 16, 1024);
+                    mma_bf16(tmem + TM_X, ah, bh, id, ks > 0);
+                    mma_bf16(tmem + TM_X, ah, bl, id, 1);
+                    mma_bf16(tmem + TM_X, al, bh, id, 1);
                 }
             } else {
                 // Exact: bf16 inputs, fp32 accumulation.
@@ -441,38 +476,53 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         mma_sync();
         if (__syncthreads_or(!ok)) break;
+        if (ci + 1 < nchunks) load_beta(ci + 1, bgnext);
 
         // ------------------------------- derived tiles; A and P from X ----------
         // K*E (bf16), Q*E (fp16), K*D (bf16 hi + lo) into the freed X region.
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int r = tg + 16 * u;
-            float kf[8], qf[8], ke[8], qe[8], kd[8];
-            load_bf16x8(smem + R_IN + ckh * 16384 + swz(r, ckc), kf);
-            load_bf16x8(smem + R_IN + ckh * 16384 + 8192 + swz(r, ckc), qf);
+        {
+            const float2 l2e = make_float2(kLog2e, kLog2e);
+            float2 last2[4];
             if (CHANNEL) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float E = __expf(gam[u][e]);
-                    const float Dd = __expf(sLast[8 * ck + e] - gam[u][e]);
-                    ke[e] = kf[e] * E;
-                    qe[e] = qf[e] * E;
-                    kd[e] = kf[e] * Dd;
-                }
-            } else {
-                const float E = __expf(sGam[r]);
-                const float Dd = __expf(sGam[C - 1] - sGam[r]);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    ke[e] = kf[e] * E;
-                    qe[e] = qf[e] * E;
-                    kd[e] = kf[e] * Dd;
-                }
+                for (int e = 0; e < 4; ++e)
+                    last2[e] = make_float2(sLast[8 * ck + 2 * e], sLast[8 * ck + 2 * e + 1]);
             }
-            const uint32_t o64 = ckh * 8192 + swz(r, ckc);
-            store_bf16x8(smem + OFF_KE + o64, ke);
-            store_f16x8(smem + OFF_QE + o64, qe);
-            store_split(smem + OFF_KDH + o64, smem + OFF_KDL + o64, kd);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int r = tg + 16 * u;
+                float kf[8], qf[8], ke[8], qe[8];
+                float2 kd[4];
+                load_bf16x8(smem + R_IN + ckh * 16384 + swz(r, ckc), kf);
+                load_bf16x8(smem + R_IN + ckh * 16384 + 8192 + swz(r, ckc), qf);
+                float2 E2 = make_float2(0.f, 0.f), D2 = E2;
+                if (!CHANNEL) {
+                    const float E = ex2_approx(sGam[r] * kLog2e);
+                    const float Dd = ex2_approx((sGam[C - 1] - sGam[r]) * kLog2e);
+                    E2 = make_float2(E, E);
+                    D2 = make_float2(Dd, Dd);
+                }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 k2 = make_float2(kf[2 * e], kf[2 * e + 1]);
+                    const float2 q2 = make_float2(qf[2 * e], qf[2 * e + 1]);
+                    if (CHANNEL) {
+                        const float2 g2 = make_float2(gam[u][2 * e], gam[u][2 * e + 1]);
+                        const float2 el = mul2(g2, l2e);
+                        const float2 dl = mul2(sub2(last2[e], g2), l2e);
+                        E2 = make_float2(ex2_approx(el.x), ex2_approx(el.y));
+                        D2 = make_float2(ex2_approx(dl.x), ex2_approx(dl.y));
+                    }
+                    const float2 ke2 = mul2(k2, E2), qe2 = mul2(q2, E2);
+                    ke[2 * e] = ke2.x; ke[2 * e + 1] = ke2.y;
+                    qe[2 * e] = qe2.x; qe[2 * e + 1] = qe2.y;
+                    kd[e] = mul2(k2, D2);
+                }
+                const uint32_t o64 = ckh * 8192 + swz(r, ckc);
+                store_bf16x8(smem + OFF_KE + o64, ke);
+                store_f16x8(smem + OFF_QE + o64, qe);
+                store_split2(smem + OFF_KDH + o64, smem + OFF_KDL + o64, kd);
+            }
         }
         {
             // Thread: row L = TMEM lane of X (A rows 0-63, P rows 64-127),
@@ -603,12 +653,16 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 // Transition CTAs have V = 0: U = -W S starts the accumulator.
                 mma_bf16(tmem + TM_UT, a, sdesc_sw128(sbase + OFF_WT + ks * 2048, 8192, 1024), id_u,
                          transition ? (ks > 0) : 1);
-                if (!transition) {
+            }
+            mma_commit(bar_mma);
+            if (want_o) {
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint64_t a = sdesc_sw128(sbase + R_S + ks * 2048, 16384, 1024);
                     const uint64_t bq = sdesc_sw128(sbase + OFF_QE + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
                     mma_bf16(tmem + TM_OT, a, bq, id_o, ks > 0);
                 }
             }
-            mma_commit(bar_mma);
         }
         mma_sync();
         if (__syncthreads_or(!ok)) break;
@@ -640,18 +694,24 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const uint64_t kdl = sdesc_sw128(sbase + OFF_KDL + ks * 2048, 8192, 1024);
                 const uint64_t uh = sdesc_sw128(sbase + OFF_UH + ks * 32, 16, 1024);
                 const uint64_t ul = sdesc_sw128(sbase + OFF_UL + ks * 32, 16, 1024);
-                const uint64_t ph = sdesc_sw128(sbase + OFF_PH + ks * 32, 16, 1024);
-                const uint64_t pl = sdesc_sw128(sbase + OFF_PL + ks * 32, 16, 1024);
                 mma_bf16(tmem + TM_SN, kdh, uh, id_s, ks > 0);
                 mma_bf16(tmem + TM_SN, kdh, ul, id_s, 1);
                 mma_bf16(tmem + TM_SN, kdl, uh, id_s, 1);
-                if (!transition) {
+            }
+            mma_commit(bar_mma);
+            if (want_o) {
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t uh = sdesc_sw128(sbase + OFF_UH + ks * 32, 16, 1024);
+                    const uint64_t ul = sdesc_sw128(sbase + OFF_UL + ks * 32, 16, 1024);
+                    const uint64_t ph = sdesc_sw128(sbase + OFF_PH + ks * 32, 16, 1024);
+                    const uint64_t pl = sdesc_sw128(sbase + OFF_PL + ks * 32, 16, 1024);
                     mma_bf16(tmem + TM_OT, uh, ph, id_o, 1);
                     mma_bf16(tmem + TM_OT, uh, pl, id_o, 1);
                     mma_bf16(tmem + TM_OT, ul, ph, id_o, 1);
                 }
+                mma_commit(bar_out);
             }
-            mma_commit(bar_mma);
         }
         mma_sync();
         if (__syncthreads_or(!ok)) break;
@@ -660,23 +720,32 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         float o[32];
         {
             const uint32_t lb = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-            float sn[32];
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                tmem_ld32(lb + TM_SN + half * 64 + part * 32, sn);
+            {
+                float sn0[32], sn1[32];
+                tmem_ld32(lb + TM_SN + half * 64, sn0);
+                tmem_ld32(lb + TM_SN + half * 64 + 32, sn1);
                 tmem_wait_ld();
+                const float2 e2 = make_float2(e_last, e_last);
 #pragma unroll
-                for (int c = 0; c < 32; ++c) s[part * 32 + c] = fmaf(e_last, s[part * 32 + c], sn[c]);
+                for (int c = 0; c < 32; c += 2) {
+                    const float2 a = fma2(e2, make_float2(s[c], s[c + 1]), make_float2(sn0[c], sn0[c + 1]));
+                    const float2 z = fma2(e2, make_float2(s[32 + c], s[33 + c]), make_float2(sn1[c], sn1[c + 1]));
+                    s[c] = a.x; s[c + 1] = a.y; s[32 + c] = z.x; s[33 + c] = z.y;
+                }
             }
             write_state_f16();
-            tmem_ld32(lb + TM_OT + half * 32, o);
-            tmem_wait_ld();
+            if (want_o) {
+                ok = ok && mbar_wait(bar_out, ci & 1, &g_status_word);
+                tc_fence_after();
+                tmem_ld32(lb + TM_OT + half * 32, o);
+                tmem_wait_ld();
+            }
         }
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
+        if (__syncthreads_or(!ok)) break;
         // Output stores after the fence, which would otherwise wait for them.
-        if (p.out != nullptr && !transition) {
+        if (want_o) {
             const int nvalid = min(C, t_end - t0) - half * 32;
 #pragma unroll
             for (int r = 0; r < 32; ++r) {
