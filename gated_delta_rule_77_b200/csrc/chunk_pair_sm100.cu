@@ -586,6 +586,9 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         float gnext[4][8], bgnext[4];
         if (CHANNEL && nchunks > 0) gate_load(0, gnext);
         if (!CHANNEL && nchunks > 0) gate_scalar_load(0, false, bgnext);
+        // Per-channel: chunk 0's scan here; the scan of chunk c + 1 runs
+        // while the products SN of chunk c are on the tensor core.
+        if (CHANNEL && nchunks > 0) gate_channel(0, (long)b * T * H + h, gnext, nullptr, nullptr, sLast);
 
         for (int ci = 0; ci < nchunks; ++ci) {
             const int t0 = ci * C;
@@ -595,8 +598,7 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) gam[u][e] = gnext[u][e];
-                gate_channel(t0, tk0, gam, nullptr, nullptr, sLast);
+                    for (int e = 0; e < 8; ++e) gam[u][e] = gnext[u][e];   // already scanned
             } else {
                 gate_scalar(bgnext, sGam, nullptr);
             }
@@ -759,6 +761,8 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
                 mma_commit(bar_out);
             }
+            if (CHANNEL && ci + 1 < nchunks)   // sLast of this chunk is no longer read
+                gate_channel(t0 + C, tk0 + (long)C * H, gnext, nullptr, nullptr, sLast);
             mma_sync();
             if (__syncthreads_or(!ok)) break;
 
