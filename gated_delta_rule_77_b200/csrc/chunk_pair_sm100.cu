@@ -73,12 +73,15 @@ constexpr uint32_t P_REF1 = P_REF0 + 512;     // 128 f32
 constexpr uint32_t P_ER = P_REF1 + 512;       // 64 f32: exp(G_r - G_31)  (scalar gate)
 constexpr uint32_t P_FJ = P_ER + 256;         // 64 f32: exp(G_31 - G_j)
 constexpr uint32_t P_SAFE = P_FJ + 256;       // int: product form in range
-constexpr uint32_t P_BAR = P_SAFE + 16;       // tma, mma, empty
-constexpr uint32_t P_TMEM = P_BAR + 24;
+constexpr uint32_t P_BAR = P_SAFE + 16;       // tma, mma, empty, g
+constexpr uint32_t P_TMEM = P_BAR + 32;
 // T' hi, T' lo, P hi, P lo (4 x 8 KB) for the bulk copy to CTA 1; apart from
 // the X region so that the copy of chunk c overlaps the X build of chunk c + 1.
 constexpr uint32_t P_STAGE = (P_TMEM + 8 + 1023) / 1024 * 1024;
-constexpr uint32_t P_USED = P_STAGE + 32768;
+// Per-channel g of the next chunk, by TMA: four [64 tokens][32 channels] fp32
+// boxes, 128-byte swizzled (8 KB each).
+constexpr uint32_t P_G = P_STAGE + 32768;
+constexpr uint32_t P_USED = P_G + 32768;
 
 // ---- CTA 1 (chain) shared memory ----------------------------------------------
 constexpr uint32_t C_IN = 0;                  // 32 KB raw K, Q
@@ -120,7 +123,7 @@ template <bool CHANNEL>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
 chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                  const PairParams p)
+                  const __grid_constant__ CUtensorMap tm_g, const PairParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -156,7 +159,8 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             prefetch_tensormap(&tm_v);
             prefetch_tensormap(&tm_o);
         }
-        for (int i = 0; i < (rank == 0 ? 3 : 5); ++i) mbar_init(bar0 + 8 * i, 1);
+        if (rank == 0 && CHANNEL) prefetch_tensormap(&tm_g);
+        for (int i = 0; i < (rank == 0 ? 4 : 5); ++i) mbar_init(bar0 + 8 * i, 1);
         fence_mbar_init();
     }
     const uint32_t tmem_cols = rank == 0 ? 128 : 512;
@@ -201,8 +205,7 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
         }
     };
-    auto gate_channel = [&](int t0, long tk0, float (&gam)[4][8], float* ref0, float* ref1,
-                            float* last) {
+    auto gate_scan = [&](float (&gam)[4][8], float* ref0, float* ref1, float* last) {
 #pragma unroll
         for (int o = 1; o < 16; o <<= 1) {
 #pragma unroll
@@ -223,13 +226,6 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 off += tot;
             }
         }
-        if (t0 + 2 * C < T) {     // warm L2 two chunks ahead
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int r = 2 * C + tg + 16 * u;
-                if (t0 + r < T) prefetch_l2(p.g + (tk0 + (long)r * H) * D + 8 * ck);
-            }
-        }
         if (tg == 15) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -238,6 +234,17 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (last) last[8 * ck + e] = gam[3][e];
             }
         }
+    };
+    auto gate_channel = [&](int t0, long tk0, float (&gam)[4][8], float* ref0, float* ref1,
+                            float* last) {
+        if (t0 + 2 * C < T) {     // warm L2 two chunks ahead
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int r = 2 * C + tg + 16 * u;
+                if (t0 + r < T) prefetch_l2(p.g + (tk0 + (long)r * H) * D + 8 * ck);
+            }
+        }
+        gate_scan(gam, ref0, ref1, last);
     };
     // Scalar gate and beta, warp 0: lane holds tokens lane and 32 + lane.
     // gate_scalar_load reads them into registers; gate_scalar scans g into
@@ -308,6 +315,7 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         float* sT = reinterpret_cast<float*>(smem + P_T);
         float* sY = reinterpret_cast<float*>(smem + P_Y);
         const uint32_t bar_tma = sbase + P_BAR, bar_empty = sbase + P_BAR + 16;
+        const uint32_t bar_g = sbase + P_BAR + 24;
         // CTA 1's slot and "full" barrier, as cluster addresses.
         const uint32_t peer_slot = mapa_shared(sbase + C_SLOT, 1);
         const uint32_t peer_full = mapa_shared(sbase + C_BAR + 24, 1);
@@ -320,25 +328,50 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 tma_load_4d(sbase + P_IN + hf * 16384 + 8192, &tm_q, hf * 64, h, t0, b, bar_tma);
             }
         };
+        // Per-channel g: chunk c + 1 arrives by TMA while chunk c's operands
+        // are built, and is scanned while chunk c's X product runs.
+        auto issue_g = [&](int chunk) {
+            mbar_expect_tx(bar_g, 32768);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                tma_load_4d(sbase + P_G + i * 8192, &tm_g, 32 * i, h, chunk * C, b, bar_g);
+        };
+        int g_issued = 0, g_waited = 0;          // g loads issued / waited for
+        auto scan_g = [&](float (&gn)[4][8]) {   // wait, read this thread's values, scan
+            ok = ok && mbar_wait(bar_g, g_waited & 1, &g_pair_status_word);
+            ++g_waited;
+            const uint8_t* box = smem + P_G + (ck >> 2) * 8192;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int r = tg + 16 * u;
+                const float4 a = *reinterpret_cast<const float4*>(box + swz(r, 2 * (ck & 3)));
+                const float4 c = *reinterpret_cast<const float4*>(box + swz(r, 2 * (ck & 3) + 1));
+                gn[u][0] = a.x; gn[u][1] = a.y; gn[u][2] = a.z; gn[u][3] = a.w;
+                gn[u][4] = c.x; gn[u][5] = c.y; gn[u][6] = c.z; gn[u][7] = c.w;
+            }
+            gate_scan(gn, sRef0, sRef1, nullptr);
+        };
         if (tid == 0 && nchunks > 0) issue_kq(0);
         int kq_waited = -1;
         bool copy_pending = false;
         float gnext[4][8], bgnext[4];
-        if (CHANNEL && nchunks > 0) gate_load(0, gnext);
+        if (CHANNEL && nchunks > 0) {
+            if (tid == 0) { issue_g(0); g_issued = 1; }
+            scan_g(gnext);
+            __syncthreads();                      // chunk 0's g has been read
+            if (tid == 0 && nchunks > 1) { issue_g(1); g_issued = 2; }
+        }
         if (nchunks > 0) gate_scalar_load(0, true, bgnext);
 
         for (int ci = 0; ci < nchunks; ++ci) {
-            const int t0 = ci * C;
-            const long tk0 = ((long)b * T + t0) * H + h;
             float gam[4][8];
-            if (CHANNEL) {
+            if (CHANNEL) {   // scanned one chunk ahead; sRef0/1 hold this chunk's
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
 #pragma unroll
                     for (int e = 0; e < 8; ++e) gam[u][e] = gnext[u][e];
-                gate_channel(t0, tk0, gam, sRef0, sRef1, nullptr);
             }
-            // g and beta were loaded one chunk ahead.
+            // beta (and a scalar g) were loaded one chunk ahead.
             gate_scalar(bgnext, sGam, sBeta, sEr, sFj, sSafe);
             if (CHANNEL && ci + 1 < nchunks) gate_scalar_load(ci + 1, true, bgnext);
             ok = ok && mbar_wait(bar_tma, ci & 1, &g_pair_status_word);
@@ -393,7 +426,6 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
                 fence_async_smem();
                 __syncthreads();
-                if (ci + 1 < nchunks) gate_load(ci + 1, gnext);
             }
             if (tid == 0) {
                 tc_fence_after();
@@ -421,14 +453,19 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
                 mma_commit(sbase + P_BAR + 8);
             }
+            // While X runs: the next chunk's g (the X build of this chunk has
+            // read sRef0/1 already).
+            if (CHANNEL && ci + 1 < nchunks) scan_g(gnext);
             mma_sync();
             if (tid == 0 && copy_pending) {      // the staging is free again
                 bulk_wait_read_all();
                 copy_pending = false;
             }
             if (__syncthreads_or(!ok)) break;
-            // Raw K, Q and the X operands are consumed: prefetch the next chunk.
+            // Raw K, Q and the X operands are consumed: prefetch the next chunk;
+            // the g tile has been read by every thread.
             if (tid == 0 && ci + 1 < nchunks) issue_kq(ci + 1);
+            if (CHANNEL && tid == 0 && ci + 2 < nchunks) { issue_g(ci + 2); g_issued = ci + 3; }
             if (!CHANNEL && ci + 1 < nchunks) gate_scalar_load(ci + 1, true, bgnext);
 
             // A and P from X (see chunk_sm100.cu); P as bf16 hi + lo into the staging.
@@ -525,6 +562,8 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             bulk_wait_all();                 // own copies complete before exit
             if (!ok && kq_waited + 1 < nchunks)
                 mbar_wait(bar_tma, (kq_waited + 1) & 1, &g_pair_status_word);
+            for (int i = g_waited; !ok && i < g_issued; ++i)   // g tiles still in flight
+                mbar_wait(bar_g, i & 1, &g_pair_status_word);
         }
     } else {
         // ========================================================== chain CTA ===
@@ -859,6 +898,20 @@ bool make_out_map(CUtensorMap* map, void* base, int H, int T, int B) {
     return r == CUDA_SUCCESS;
 }
 
+// g [B, T, H, D] fp32 (per-channel gate), box 32 channels x 64 tokens, 128B swizzle.
+bool make_g_map(CUtensorMap* map, const float* base, int H, int T, int B) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 4, (cuuint64_t)H * D * 4, (cuuint64_t)T * H * D * 4};
+    cuuint32_t box[4] = {32, 1, (cuuint32_t)C, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool make_map(CUtensorMap* map, const void* base, int H, int T, int B) {
     auto fn = encode_fn();
     if (!fn) return false;
@@ -881,12 +934,17 @@ cudaError_t launch_pair(const Problem& p, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    CUtensorMap mq, mk, mv, mo;
+    CUtensorMap mq, mk, mv, mo, mg;
     if (!make_map(&mq, p.q, p.H, p.T, p.B) || !make_map(&mk, p.k, p.H, p.T, p.B) ||
         !make_map(&mv, p.v, p.H, p.T, p.B) || !make_out_map(&mo, p.out, p.H, p.T, p.B))
         return cudaErrorInvalidValue;
+    if (CHANNEL) {
+        if (!make_g_map(&mg, p.g, p.H, p.T, p.B)) return cudaErrorInvalidValue;
+    } else {
+        mg = mq;                                   // not read with a scalar gate
+    }
     PairParams prm{p.g, p.beta, p.state_in, p.state_out, static_cast<float*>(p.out), p.T, p.H};
-    chunk_pair_kernel<CHANNEL><<<2 * p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, prm);
+    chunk_pair_kernel<CHANNEL><<<2 * p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mg, prm);
     return cudaGetLastError();
 }
 
