@@ -96,6 +96,7 @@ constexpr uint32_t OFF_CBL = R_X + 90112;    //   24 KB   rows 32-95 K*exp(G_47 
 constexpr uint32_t CB_HALF = 96 * 128;
 //  (b) after X: derived tiles, P, solve input, U
 constexpr uint32_t OFF_KE = R_X;             //   16 KB K*E bf16  [half][64 r][128 B]
+constexpr uint32_t OFF_OST = R_X;            //   at the chunk's end: 32 KB O fp32 [64 t][128 j] (TMA store)
 constexpr uint32_t OFF_QE = R_X + 16384;     //   16 KB Q*E fp16
 constexpr uint32_t OFF_KDH = R_X + 32768;    //   16 KB K*D bf16 hi
 constexpr uint32_t OFF_KDL = R_X + 49152;    //   16 KB K*D bf16 lo
@@ -146,7 +147,8 @@ struct Params {
 template <bool CHANNEL>
 __global__ void __launch_bounds__(NT, 1)
 chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                 const __grid_constant__ CUtensorMap tm_v, const Params p)
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                 const Params p)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base (128B-swizzle atoms), derived by a pointer offset
@@ -204,6 +206,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
+        if (p.out != nullptr) prefetch_tensormap(&tm_o);
         mbar_init(bar_tma, 1);
         mbar_init(bar_mma, 1);
         mbar_init(bar_out, 1);
@@ -393,6 +396,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         ok = ok && mbar_wait(bar_tma, ci & 1, &g_status_word);
         tma_waited = ci;
+        if (tid == 0) bulk_wait_read_all();   // the previous output store has read OFF_OST
         if (__syncthreads_or(!ok)) break;
 
         // ---------------------------------------------------- X = raw A and P --
@@ -739,20 +743,23 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 tc_fence_after();
                 tmem_ld32(lb + TM_OT + half * 32, o);
                 tmem_wait_ld();
+                // O^T (lane = value column) -> [token][column] fp32 over the
+                // consumed K*E / Q*E tiles; one TMA store per chunk, rows past
+                // T dropped.  Thread stores would hold up the next proxy fence.
+                float* so = reinterpret_cast<float*>(smem + OFF_OST) + half * 32 * D + srow;
+#pragma unroll
+                for (int r = 0; r < 32; ++r) so[r * D] = o[r];
             }
         }
         fence_async_smem();
         tc_fence_before();
         if (__syncthreads_or(!ok)) break;
-        // Output stores after the fence, which would otherwise wait for them.
-        if (want_o) {
-            const int nvalid = min(C, t_end - t0) - half * 32;
-#pragma unroll
-            for (int r = 0; r < 32; ++r) {
-                if (r < nvalid) p.out[(tk0 + (long)(half * 32 + r) * H) * D + srow] = o[r];
-            }
+        if (want_o && tid == 0) {
+            tma_store_4d(&tm_o, sbase + OFF_OST, 0, h, t0, b);
+            bulk_commit();
         }
     }
+    if (tid == 0) bulk_wait_all();     // output stores complete before exit
 
     if (!ok && tid == 0) {
         // Abandoned: drain what this CTA still has in flight (bounded) before
@@ -796,6 +803,20 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // 4-D map over a bf16 [B, T, H, 128] tensor; box {64 channels, 1, 64 tokens, 1},
 // 128-byte swizzle (the operand layout of the MMAs).
+// out [B, T, H, 128] fp32, box = one chunk of one head, no swizzle.
+bool make_out_map(CUtensorMap* map, const void* base, int H, int T, int B) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 4, (cuuint64_t)H * D * 4, (cuuint64_t)T * H * D * 4};
+    cuuint32_t box[4] = {(cuuint32_t)D, 1, (cuuint32_t)C, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box,
+                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool make_map(CUtensorMap* map, const void* base, int H, int T, int B) {
     auto fn = encode_fn();
     if (!fn) return false;
@@ -909,9 +930,9 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, p.q, p.H, p.T, p.B) || !make_map(&mk, p.k, p.H, p.T, p.B) ||
-        !make_map(&mv, p.v, p.H, p.T, p.B))
+        !make_map(&mv, p.v, p.H, p.T, p.B) || !make_out_map(&mo, p.out, p.H, p.T, p.B))
         return cudaErrorInvalidValue;
     float* out = static_cast<float*>(p.out);
     const int nchunks = (p.T + C - 1) / C;
@@ -925,7 +946,7 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
         if (pair) return launch_chunk_pair_sm100(p, stream);
         Params prm{p.g, p.beta, p.state_in, p.state_out, nullptr, out, p.T, p.H, p.B,
                    1, nchunks * C, 1, 1};
-        chunk_fwd_kernel<CHANNEL><<<p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, prm);
+        chunk_fwd_kernel<CHANNEL><<<p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, prm);
         return cudaGetLastError();
     }
     // Segment-parallel path: per segment the zero-start end state and the
@@ -940,7 +961,7 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
     float* seg_states = ws;
     float* trans = ws + slab;
     Params p1{p.g, p.beta, nullptr, seg_states, trans, nullptr, p.T, p.H, p.B, nseg, seg_len, 1, nseg};
-    chunk_fwd_kernel<CHANNEL><<<2 * p.B * nseg * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, p1);
+    chunk_fwd_kernel<CHANNEL><<<2 * p.B * nseg * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, p1);
     e = cudaGetLastError();
     if (e == cudaSuccess) {
         combine_segments_kernel<<<p.B * p.H * (D / CB_COLS), 256, 0, stream>>>(
@@ -949,7 +970,7 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
     }
     if (e == cudaSuccess) {
         Params p2{p.g, p.beta, seg_states, nullptr, nullptr, out, p.T, p.H, p.B, nseg, seg_len, nseg, 1};
-        chunk_fwd_kernel<CHANNEL><<<p.B * nseg * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, p2);
+        chunk_fwd_kernel<CHANNEL><<<p.B * nseg * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, p2);
         e = cudaGetLastError();
     }
     const cudaError_t ef = cudaFreeAsync(ws, stream);
@@ -1001,15 +1022,15 @@ cudaError_t launch_noalloc(const Problem& p, cudaStream_t stream, bool* over_lim
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, p.q, p.H, p.T, p.B) || !make_map(&mk, p.k, p.H, p.T, p.B) ||
-        !make_map(&mv, p.v, p.H, p.T, p.B))
+        !make_map(&mv, p.v, p.H, p.T, p.B) || !make_out_map(&mo, p.out, p.H, p.T, p.B))
         return cudaErrorInvalidValue;
     float* out = static_cast<float*>(p.out);
     if (nseg <= 1) {
         Params prm{p.g, p.beta, p.state_in, p.state_out, nullptr, out, p.T, p.H, p.B,
                    1, nchunks * C, 1, 1};
-        chunk_fwd_kernel<CHANNEL><<<p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, prm);
+        chunk_fwd_kernel<CHANNEL><<<p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, prm);
         return cudaGetLastError();
     }
     float* ws = nullptr;
@@ -1020,7 +1041,7 @@ cudaError_t launch_noalloc(const Problem& p, cudaStream_t stream, bool* over_lim
     float* seg_states = ws;
     float* trans = ws + slab;
     Params p1{p.g, p.beta, nullptr, seg_states, trans, nullptr, p.T, p.H, p.B, nseg, seg_len, 1, nseg};
-    chunk_fwd_kernel<CHANNEL><<<2 * p.B * nseg * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, p1);
+    chunk_fwd_kernel<CHANNEL><<<2 * p.B * nseg * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, p1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     combine_segments_kernel<<<p.B * p.H * (D / CB_COLS), 256, 0, stream>>>(
@@ -1028,7 +1049,7 @@ cudaError_t launch_noalloc(const Problem& p, cudaStream_t stream, bool* over_lim
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     Params p2{p.g, p.beta, seg_states, nullptr, nullptr, out, p.T, p.H, p.B, nseg, seg_len, nseg, 1};
-    chunk_fwd_kernel<CHANNEL><<<p.B * nseg * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, p2);
+    chunk_fwd_kernel<CHANNEL><<<p.B * nseg * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, p2);
     return cudaGetLastError();
 }
 
