@@ -478,8 +478,13 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             mma_commit(bar_mma);
         }
-        mma_sync();
-        if (__syncthreads_or(!ok)) break;
+        // Per-channel X reads its operands from R_X, where the derived tiles
+        // go: wait first.  With a scalar gate X reads only the raw K and Q, so
+        // the derived tiles are built while it runs.
+        if (CHANNEL) {
+            mma_sync();
+            if (__syncthreads_or(!ok)) break;
+        }
         if (ci + 1 < nchunks) load_beta(ci + 1, bgnext);
 
         // ------------------------------- derived tiles; A and P from X ----------
@@ -528,7 +533,13 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 store_split2(smem + OFF_KDH + o64, smem + OFF_KDL + o64, kd);
             }
         }
-        {
+        if (!CHANNEL) {
+            mma_sync();
+            if (__syncthreads_or(!ok)) break;
+        }
+        // P (rows 64-127, warps of lane quadrants 2 and 3) only where outputs
+        // are formed.
+        if (quad < 2 || want_o) {
             // Thread: row L = TMEM lane of X (A rows 0-63, P rows 64-127),
             // columns j in [32*half, 32*half + 32).
             const int L = quad * 32 + lane;
