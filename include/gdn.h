@@ -27,7 +27,10 @@
  *   per-channel g must be 16-byte aligned; a scalar g and beta 4-byte
  *   aligned (else GDN_ERR_MISALIGNED).  The library never
  *   frees caller memory.  Scratch space the prefill needs is taken
- *   stream-ordered (cudaMallocAsync / cudaFreeAsync on `stream`).
+ *   stream-ordered on `stream` (cudaMallocFromPoolAsync / cudaFreeAsync)
+ *   from a memory pool the library creates per device, which keeps its
+ *   memory for reuse by later calls (at most the largest scratch in use at
+ *   once) until the process ends.
  *   The recurrent state is fp32, [B, H, dk, dv], row index = key channel --
  *   the precision the source keeps the state in ("Hybrid layouts: three
  *   DeltaNet, one attention", section 01 Concept: fp32 recurrent state).
@@ -130,7 +133,8 @@ GDN_API int gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const 
  *                n > 1 = n segments (at most one per 64-token chunk;
  *                dk = dv = 128 only).
  * Scratch: 2 * B * n * H * dk * dv * 4 bytes, stream-ordered on `stream`
- * (GDN_ERR_NOMEM if it cannot be had).  Other arguments as gdn_chunk_fwd.
+ * from the library's pool (GDN_ERR_NOMEM if it cannot be had).  Other
+ * arguments as gdn_chunk_fwd.
  */
 GDN_API int gdn_chunk_fwd_segments(const void* q, const void* k, const void* v, const float* g,
                                    const float* beta, const float* state_in, void* out,
@@ -145,7 +149,7 @@ GDN_API int gdn_chunk_fwd_segments(const void* q, const void* k, const void* v, 
  *
  * Who needs it: callers whose device memory already belongs to another
  * allocator (e.g. a framework pool that has reserved all free memory, so a
- * cudaMallocAsync inside the library could fail or fragment it), and callers
+ * stream-ordered allocation inside the library could fail or fragment it), and callers
  * whose step must never stall in an allocator or fail for lack of memory
  * half-way through.  This variant calls no allocation or free routine: its
  * scratch is a fixed 32 MiB array compiled into the library, which every GPU
