@@ -33,10 +33,12 @@ GATE_SCALAR = 0
 GATE_CHANNEL = 1
 IO_BF16 = 0
 IO_F32 = 1
+ACT_NONE = 0
+ACT_SILU = 1
 
 SYMBOLS = ("gdn_chunk_fwd", "gdn_chunk_fwd_ex", "gdn_chunk_fwd_segments",
            "gdn_chunk_fwd_segments_noalloc", "gdn_recurrent_step", "gdn_recurrent_step_ex",
-           "gdn_check", "gdn_status_string")
+           "gdn_prologue", "gdn_recurrent_step_prologue", "gdn_check", "gdn_status_string")
 
 _lib = None
 
@@ -63,6 +65,10 @@ def load() -> ctypes.CDLL:
                                                    vp]
     lib.gdn_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, vp]
     lib.gdn_recurrent_step_ex.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, i, vp]
+    lib.gdn_prologue.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, vp, vp, vp, fp, fp, i, i, i, i, i,
+                                 i, i, vp]
+    lib.gdn_recurrent_step_prologue.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, fp, fp, vp, i, i, i,
+                                                i, i, i, vp]
     lib.gdn_check.argtypes = [vp]
     lib.gdn_status_string.argtypes = [i]
     lib.gdn_status_string.restype = ctypes.c_char_p
@@ -147,6 +153,72 @@ def recurrent_step(q, k, v, g, beta, state, *, state_out=None, out=None, stream=
                                       gate, _io_code(q.dtype), _stream(stream))
     if rc != GDN_OK:
         raise GdnError(rc, "gdn_recurrent_step_ex")
+    return out
+
+
+def _act_code(activation):
+    if activation == "silu":
+        return ACT_SILU
+    if activation == "none":
+        return ACT_NONE
+    raise ValueError(f"unknown activation {activation!r}")
+
+
+def prologue(q_raw, k_raw, v_raw, g_raw, beta_raw, conv_w, ring=None, pos0=None, *,
+             activation: str = "silu", stream=None):
+    """The layer's input prologue over T tokens (gdn_prologue).  q_raw, k_raw
+    [B,T,H,dk] bf16; v_raw [B,T,H,dv] bf16; g_raw [B,T,H] or [B,T,H,dk] fp32;
+    beta_raw [B,T,H] fp32; conv_w [H, 2dk+dv, 4] fp32; ring [B,H,4,2dk+dv]
+    fp32 (updated in place) or None; pos0 [B] int32 or None.  Returns
+    (q, k, v, g, beta), ready for chunk_fwd."""
+    B, T, H, dk = q_raw.shape
+    dv = v_raw.shape[-1]
+    gate = GATE_CHANNEL if g_raw.dim() == 4 else GATE_SCALAR
+    dev = q_raw.device
+    q = torch.empty(B, T, H, dk, dtype=torch.bfloat16, device=dev)
+    k = torch.empty_like(q)
+    v = torch.empty(B, T, H, dv, dtype=torch.bfloat16, device=dev)
+    g = torch.empty(g_raw.shape, dtype=torch.float32, device=dev)
+    beta = torch.empty(B, T, H, dtype=torch.float32, device=dev)
+    _check_cuda(q_raw, k_raw, v_raw, g_raw, beta_raw, conv_w, ring, pos0)
+    if q_raw.dtype != torch.bfloat16 or v_raw.dtype != torch.bfloat16:
+        raise ValueError("q_raw, k_raw and v_raw must be bf16")
+    if pos0 is not None and pos0.dtype != torch.int32:
+        raise ValueError("pos0 must be int32")
+    rc = load().gdn_prologue(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(g_raw), _ptr(beta_raw),
+                             _ptr(conv_w), _ptr(ring), _ptr(pos0), _ptr(q), _ptr(k), _ptr(v),
+                             _ptr(g), _ptr(beta), B, T, H, dk, dv, gate, _act_code(activation),
+                             _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_prologue")
+    return q, k, v, g, beta
+
+
+def recurrent_step_prologue(q_raw, k_raw, v_raw, g_raw, beta_raw, conv_w, ring, state, pos=None, *,
+                            activation: str = "silu", state_out=None, out=None, stream=None):
+    """One decode step with the prologue fused in (gdn_recurrent_step_prologue).
+    q_raw, k_raw [B,H,dk] bf16; v_raw [B,H,dv] bf16; g_raw [B,H] or [B,H,dk];
+    beta_raw [B,H]; ring [B,H,4,2dk+dv] fp32 (slot pos mod 4 written);
+    state [B,H,dk,dv] fp32 (in place unless state_out); pos [B] int32 or
+    None.  Returns out [B,H,dv] fp32."""
+    B, H, dk = q_raw.shape
+    dv = v_raw.shape[-1]
+    gate = GATE_CHANNEL if g_raw.dim() == 3 else GATE_SCALAR
+    if state_out is None:
+        state_out = state
+    if out is None:
+        out = torch.empty(B, H, dv, dtype=torch.float32, device=v_raw.device)
+    _check_cuda(q_raw, k_raw, v_raw, g_raw, beta_raw, conv_w, ring, state, state_out, out, pos)
+    if q_raw.dtype != torch.bfloat16 or v_raw.dtype != torch.bfloat16:
+        raise ValueError("q_raw, k_raw and v_raw must be bf16")
+    if pos is not None and pos.dtype != torch.int32:
+        raise ValueError("pos must be int32")
+    rc = load().gdn_recurrent_step_prologue(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(g_raw),
+                                            _ptr(beta_raw), _ptr(conv_w), _ptr(ring), _ptr(pos),
+                                            _ptr(state), _ptr(state_out), _ptr(out), B, H, dk, dv,
+                                            gate, _act_code(activation), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_recurrent_step_prologue")
     return out
 
 

@@ -80,9 +80,113 @@ int validate(const void* q, const void* k, const void* v, const float* g, const 
     return GDN_OK;
 }
 
+// Validation shared by the two prologue entries.  Tensors are listed with
+// their sizes; inputs and outputs may not overlap (the ring included).
+int validate_prologue(const void* q_raw, const void* k_raw, const void* v_raw, const float* g_raw,
+                      const float* beta_raw, const float* conv_w, const float* ring,
+                      const int* pos, long B, long T, long H, int dk, int dv, int gate_mode,
+                      int activation, const void* const* outs, const size_t* out_bytes, int n_out)
+{
+    if (B < 1 || H < 1 || T < 0 || dk < 1 || dv < 1) return GDN_ERR_INVALID_ARG;
+    if (gate_mode != GDN_GATE_SCALAR && gate_mode != GDN_GATE_CHANNEL) return GDN_ERR_INVALID_ARG;
+    if (activation != GDN_ACT_NONE && activation != GDN_ACT_SILU) return GDN_ERR_INVALID_ARG;
+    if (!conv_w) return GDN_ERR_INVALID_ARG;
+    if (T != 0) {
+        if (!q_raw || !k_raw || !v_raw || !g_raw || !beta_raw) return GDN_ERR_INVALID_ARG;
+        for (int i = 0; i < n_out; ++i)
+            if (!outs[i]) return GDN_ERR_INVALID_ARG;
+    }
+    if (!dim_ok(dk) || !dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
+    // The prefill grid is (tiles, H, B): both within the 65535 grid limit.
+    if (B > 65535 || H > 65535 || T > (1L << 30)) return GDN_ERR_UNSUPPORTED;
+    const bool ch = gate_mode == GDN_GATE_CHANNEL;
+    const void* p16[] = {q_raw, k_raw, v_raw, conv_w, ring, ch ? g_raw : nullptr};
+    for (const void* p : p16)
+        if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
+    for (const void* p : {(const void*)g_raw, (const void*)beta_raw, (const void*)pos})
+        if (p && (reinterpret_cast<uintptr_t>(p) & 3u)) return GDN_ERR_MISALIGNED;
+    for (int i = 0; i < n_out; ++i)
+        if (outs[i] && !aligned16(outs[i])) return GDN_ERR_MISALIGNED;
+
+    const size_t tok = (size_t)B * (size_t)T * (size_t)H;
+    const size_t CH = 2 * (size_t)dk + dv;
+    Range in[] = {range_of(q_raw, tok * dk * 2), range_of(k_raw, tok * dk * 2),
+                  range_of(v_raw, tok * dv * 2), range_of(g_raw, tok * (ch ? dk : 1) * 4),
+                  range_of(beta_raw, tok * 4), range_of(conv_w, (size_t)H * CH * 16),
+                  range_of(pos, pos ? (size_t)B * 4 : 0),
+                  range_of(ring, ring ? (size_t)B * H * 4 * CH * 4 : 0)};
+    const int n_in = sizeof(in) / sizeof(in[0]);
+    for (int i = 0; i < n_out; ++i) {
+        const Range ro = range_of(outs[i], out_bytes[i]);
+        for (int j = 0; j < n_in; ++j)
+            if (overlaps(ro, in[j])) return GDN_ERR_INVALID_ARG;
+        for (int j = 0; j < i; ++j)
+            if (overlaps(ro, range_of(outs[j], out_bytes[j]))) return GDN_ERR_INVALID_ARG;
+    }
+    // The ring is written: it may not overlap the other inputs either.
+    for (int j = 0; j < n_in - 1; ++j)
+        if (overlaps(in[n_in - 1], in[j])) return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+int gdn_prologue(const void* q_raw, const void* k_raw, const void* v_raw, const float* g_raw,
+                 const float* beta_raw, const float* conv_w, float* ring, const int* pos0, void* q,
+                 void* k, void* v, float* g, float* beta, int B, int T, int H, int dk, int dv,
+                 int gate_mode, int activation, gdn_stream_t stream_)
+{
+    const size_t tok = (size_t)(B > 0 ? B : 0) * (size_t)(T > 0 ? T : 0) * (size_t)(H > 0 ? H : 0);
+    const bool ch = gate_mode == GDN_GATE_CHANNEL;
+    const void* outs[] = {q, k, v, g, beta};
+    const size_t bytes[] = {tok * (size_t)dk * 2, tok * (size_t)dk * 2, tok * (size_t)dv * 2,
+                            tok * (ch ? (size_t)dk : 1) * 4, tok * 4};
+    int rc = validate_prologue(q_raw, k_raw, v_raw, g_raw, beta_raw, conv_w, ring, pos0, B, T, H,
+                               dk, dv, gate_mode, activation, outs, bytes, 5);
+    if (rc != GDN_OK) return rc;
+    if (T == 0) return GDN_OK;
+    gdn::PrologueArgs a{static_cast<const __nv_bfloat16*>(q_raw),
+                        static_cast<const __nv_bfloat16*>(k_raw),
+                        static_cast<const __nv_bfloat16*>(v_raw),
+                        g_raw, beta_raw, conv_w, ring, pos0, activation == GDN_ACT_SILU,
+                        static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k),
+                        static_cast<__nv_bfloat16*>(v), g, beta, B, T, H, dk, dv, ch};
+    cudaError_t e = gdn::launch_prologue(a, reinterpret_cast<cudaStream_t>(stream_));
+    return e == cudaErrorNotSupported ? GDN_ERR_UNSUPPORTED : to_status(e);
+}
+
+int gdn_recurrent_step_prologue(const void* q_raw, const void* k_raw, const void* v_raw,
+                                const float* g_raw, const float* beta_raw, const float* conv_w,
+                                float* ring, const int* pos, const float* state_in,
+                                float* state_out, void* out, int B, int H, int dk, int dv,
+                                int gate_mode, int activation, gdn_stream_t stream_)
+{
+    if (!ring || !state_in || !state_out) return GDN_ERR_INVALID_ARG;
+    const size_t bh = (size_t)(B > 0 ? B : 0) * (size_t)(H > 0 ? H : 0);
+    const size_t st = bh * (size_t)(dk > 0 ? dk : 0) * (size_t)(dv > 0 ? dv : 0) * 4;
+    // state_out may coincide with state_in exactly (in-place update); it is
+    // then checked once.
+    const void* outs[] = {out, state_out};
+    const size_t bytes[] = {bh * (size_t)(dv > 0 ? dv : 0) * 4, st};
+    int rc = validate_prologue(q_raw, k_raw, v_raw, g_raw, beta_raw, conv_w, ring, pos, B, 1, H,
+                               dk, dv, gate_mode, activation, outs, bytes, 2);
+    if (rc != GDN_OK) return rc;
+    if (!aligned16(state_in)) return GDN_ERR_MISALIGNED;
+    const Range rsi = range_of(state_in, st);
+    if (overlaps(rsi, range_of(out, bytes[0]))) return GDN_ERR_INVALID_ARG;
+    if (state_in != state_out && overlaps(rsi, range_of(state_out, st))) return GDN_ERR_INVALID_ARG;
+    if (overlaps(rsi, range_of(ring, bh * 4 * (2 * (size_t)dk + dv) * 4))) return GDN_ERR_INVALID_ARG;
+    gdn::StepPrologueArgs a{static_cast<const __nv_bfloat16*>(q_raw),
+                            static_cast<const __nv_bfloat16*>(k_raw),
+                            static_cast<const __nv_bfloat16*>(v_raw),
+                            g_raw, beta_raw, conv_w, ring, pos, activation == GDN_ACT_SILU,
+                            state_in, state_out, static_cast<float*>(out), B, H, dk, dv,
+                            gate_mode == GDN_GATE_CHANNEL};
+    cudaError_t e = gdn::launch_step_prologue(a, reinterpret_cast<cudaStream_t>(stream_));
+    return e == cudaErrorNotSupported ? GDN_ERR_UNSUPPORTED : to_status(e);
+}
 
 static int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g,
                           const float* beta, const float* state_in, void* out, float* state_out,

@@ -47,6 +47,48 @@ cudaError_t launch_chunk_sm100_noalloc(const Problem& p, cudaStream_t stream, bo
 cudaError_t launch_chunk_pair_sm100(const Problem& p, cudaStream_t stream);
 cudaError_t read_and_clear_pair_status(unsigned int* status);
 
+// The layer's input prologue (prologue.cu): width-4 causal convolution over
+// q | k | v with a 4-slot history ring, SiLU or none, q/k L2 norm, beta and
+// gate maps.  Prefill writes bf16 q, k, v and fp32 g, beta; the decode form is
+// fused into the recurrent step.
+struct PrologueArgs {
+    const __nv_bfloat16* q_raw;
+    const __nv_bfloat16* k_raw;
+    const __nv_bfloat16* v_raw;
+    const float* g_raw;
+    const float* beta_raw;
+    const float* conv_w;     // [H, 2 dk + dv, 4]
+    float* ring;             // [B, H, 4, 2 dk + dv] or null
+    const int* pos0;         // [B] or null (0)
+    bool silu;
+    __nv_bfloat16* q;
+    __nv_bfloat16* k;
+    __nv_bfloat16* v;
+    float* g;
+    float* beta;
+    int B, T, H, dk, dv;
+    bool per_channel;
+};
+cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream);
+
+struct StepPrologueArgs {
+    const __nv_bfloat16* q_raw;
+    const __nv_bfloat16* k_raw;
+    const __nv_bfloat16* v_raw;
+    const float* g_raw;
+    const float* beta_raw;
+    const float* conv_w;
+    float* ring;
+    const int* pos;          // [B] or null (0)
+    bool silu;
+    const float* state_in;
+    float* state_out;
+    float* out;              // [B, H, dv] fp32
+    int B, H, dk, dv;
+    bool per_channel;
+};
+cudaError_t launch_step_prologue(const StepPrologueArgs& a, cudaStream_t stream);
+
 // Device status word written by kernels that abandon a bounded wait.
 cudaError_t read_and_clear_status(unsigned int* status, cudaStream_t stream);
 

@@ -199,6 +199,77 @@ GDN_API int gdn_recurrent_step_ex(const void* q, const void* k, const void* v, c
                           int io_dtype, gdn_stream_t stream);
 
 /*
+ * The layer's input prologue: what turns the projected inputs of a Gated
+ * DeltaNet layer into the recurrence's q, k, v, g and beta.
+ *   - A causal depthwise convolution of width 4 over the token axis on every
+ *     channel of q | k | v (the DeltaNet layers' kernel-4 convolution, Qwen3.5
+ *     27B page, section on the hybrid layout; causal q/k/v convolutions,
+ *     HANDOFF timeline page, v2 entry):
+ *         y_t[c] = sum_{j=0..3} conv_w[h, c, j] * x_{t-3+j}[c],
+ *     tap 3 on the current token.  The inputs before a sequence's first
+ *     token come from a 4-slot history ring (slot p mod 4 holds the raw input
+ *     of position p) or are zero.
+ *   - An activation after the convolution: GDN_ACT_SILU, y / (1 + exp(-y)),
+ *     or GDN_ACT_NONE.  The pages name none; SiLU is the usual one.
+ *   - q and k L2-normalised per head: x * (sum x^2 + 1e-6)^(-1/2).
+ *   - beta = sigmoid(beta_raw); g = -min(softplus(g_raw), 5) (Atomic-GDN2
+ *     model card, section 2.1: the bound 160 / bs2 with bs2 = 32).
+ * Everything is computed in fp32 from the bf16 / fp32 inputs.
+ */
+enum { GDN_ACT_NONE = 0, GDN_ACT_SILU = 1 };
+
+/*
+ * gdn_prologue -- the prologue over T tokens (prefill), one fused pass.
+ *
+ *   q_raw, k_raw [B, T, H, dk] bf16;  v_raw [B, T, H, dv] bf16
+ *   g_raw      [B, T, H] (GDN_GATE_SCALAR) or [B, T, H, dk] (GDN_GATE_CHANNEL) fp32
+ *   beta_raw   [B, T, H] fp32
+ *   conv_w     [H, 2 dk + dv, 4] fp32, channels in the order q | k | v
+ *   ring       [B, H, 4, 2 dk + dv] fp32 (read for the three positions
+ *              before token 0, then slots (pos0 + t) mod 4 of the last
+ *              min(T, 4) tokens are overwritten with their raw inputs), or
+ *              NULL: zero history, nothing written
+ *   pos0       [B] int32 device memory: the position of each row's token 0,
+ *              or NULL for all 0.  A position p < 0 reads as zero history.
+ *   q, k       [B, T, H, dk] bf16 out;  v [B, T, H, dv] bf16 out
+ *   g          same shape as g_raw, fp32 out;  beta [B, T, H] fp32 out
+ *   dk, dv     64 or 128; B, H >= 1; T >= 0 (T == 0 does nothing)
+ *   activation GDN_ACT_NONE or GDN_ACT_SILU
+ * The outputs are what gdn_chunk_fwd takes.  No output may overlap an input,
+ * another output or the ring (inputs of a tile are read by its neighbour).
+ * conv_w, the q/k/v tensors, the ring and a per-channel g must be 16-byte
+ * aligned; a scalar g, beta and pos0 4-byte aligned.
+ */
+GDN_API int gdn_prologue(const void* q_raw, const void* k_raw, const void* v_raw,
+                         const float* g_raw, const float* beta_raw, const float* conv_w,
+                         float* ring, const int* pos0, void* q, void* k, void* v, float* g,
+                         float* beta, int B, int T, int H, int dk, int dv, int gate_mode,
+                         int activation, gdn_stream_t stream);
+
+/*
+ * gdn_recurrent_step_prologue -- one decode step with the prologue fused
+ * into it: the raw inputs of one token per sequence go through the
+ * convolution (history from the ring), the activation, the L2 norms and the
+ * gate maps inside the decode kernel, which then applies gdn_recurrent_step.
+ *
+ *   q_raw, k_raw [B, H, dk] bf16;  v_raw [B, H, dv] bf16
+ *   g_raw      [B, H] or [B, H, dk] fp32;  beta_raw [B, H] fp32
+ *   conv_w     [H, 2 dk + dv, 4] fp32
+ *   ring       [B, H, 4, 2 dk + dv] fp32, required: slots pos - 3 .. pos - 1
+ *              are read, slot pos mod 4 takes this token's raw input
+ *   pos        [B] int32 device memory (the token's position), or NULL for 0
+ *   state_in, state_out, out as gdn_recurrent_step (state_out == state_in
+ *              updates in place)
+ *   dk 64 or 128; dv 64 or 128.
+ */
+GDN_API int gdn_recurrent_step_prologue(const void* q_raw, const void* k_raw, const void* v_raw,
+                                        const float* g_raw, const float* beta_raw,
+                                        const float* conv_w, float* ring, const int* pos,
+                                        const float* state_in, float* state_out, void* out,
+                                        int B, int H, int dk, int dv, int gate_mode,
+                                        int activation, gdn_stream_t stream);
+
+/*
  * gdn_check -- synchronises `stream`, then reports GDN_ERR_TIMEOUT if any
  * kernel of this library on the current device abandoned a bounded wait
  * since the last gdn_check (and clears the record), GDN_ERR_CUDA on a CUDA

@@ -152,3 +152,30 @@ def config_inputs(cfg: Config, seed: int | None = None, **overrides):
     return prefill_inputs(B, overrides.get("T", cfg.T), H, cfg.dk, cfg.dv, gate=cfg.gate,
                           io=cfg.torch_io, s0_std=cfg.s0_std, g_zero_frac=cfg.g_zero_frac,
                           seed=seed)
+
+
+def prologue_inputs(B, T, H, dk, dv, *, gate="channel", ring=True, pos0_max=1000, seed=0):
+    """Raw inputs of the layer's input prologue (layout [B, T, H, ...]).
+
+    Recipe: q_raw, k_raw, v_raw ~ N(0, 1) rounded to bf16 (the projections'
+    outputs); g_raw ~ N(0, 2) (so that the softplus bound of 5 is active on
+    a fraction of tokens); beta_raw ~ N(0, 1); conv taps ~ U(-0.5, 0.5) (the
+    default initialisation bound 1/sqrt(width) of a width-4 depthwise
+    convolution); the history ring holds bf16-representable N(0, 1) values,
+    and pos0 ~ U{0 .. pos0_max} (a ring position not a multiple of 4 in
+    general).  Drawn in that order from ``manual_seed(seed)``.
+    """
+    gen = torch.Generator().manual_seed(int(seed))
+    q = _randn_sliced(gen, (B,), T, (H, dk), 1).to(torch.bfloat16)
+    k = _randn_sliced(gen, (B,), T, (H, dk), 1).to(torch.bfloat16)
+    v = _randn_sliced(gen, (B,), T, (H, dv), 1).to(torch.bfloat16)
+    g_tail = (H, dk) if gate == "channel" else (H,)
+    g = _randn_sliced(gen, (B,), T, g_tail, 1) * 2.0
+    beta = _randn_sliced(gen, (B,), T, (H,), 1)
+    w = torch.rand(H, 2 * dk + dv, 4, generator=gen) - 0.5
+    C = 2 * dk + dv
+    r = torch.randn(B, H, 4, C, generator=gen).to(torch.bfloat16).float() if ring else None
+    pos0 = torch.randint(0, pos0_max + 1, (B,), generator=gen, dtype=torch.int32)
+    return dict(q_raw=q.contiguous(), k_raw=k.contiguous(), v_raw=v.contiguous(), g_raw=g.contiguous(),
+                beta_raw=beta.contiguous(), conv_w=w.contiguous(), ring=r, pos0=pos0)
+

@@ -115,3 +115,66 @@ def test_segments_entry_point_rejects(lib):
     assert call(-1) == gdn.GDN_ERR_INVALID_ARG
     assert call(4, dk=64) == gdn.GDN_ERR_UNSUPPORTED
     assert call(4, B=0) == gdn.GDN_ERR_INVALID_ARG
+
+
+def _pro(lib, qr=A, kr=A + 64 * MB, vr=A + 128 * MB, gr=A + 192 * MB, br=A + 256 * MB,
+         w=A + 300 * MB, ring=A + 310 * MB, pos=A + 319 * MB, q=A + 320 * MB, k=A + 384 * MB,
+         v=A + 448 * MB, g=A + 512 * MB, beta=A + 576 * MB, B=1, T=16, H=1, dk=128, dv=128, gate=0,
+         act=1):
+    c = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    return lib.gdn_prologue(c(qr), c(kr), c(vr), c(gr), c(br), c(w), c(ring), c(pos), c(q), c(k),
+                            c(v), c(g), c(beta), B, T, H, dk, dv, gate, act, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(qr=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(w=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(q=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(beta=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(act=2), gdn.GDN_ERR_INVALID_ARG),
+    (dict(gate=3), gdn.GDN_ERR_INVALID_ARG),
+    (dict(T=-1), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dk=32), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dv=256), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(w=A + 300 * MB + 8), gdn.GDN_ERR_MISALIGNED),      # conv taps are read as float4
+    (dict(ring=A + 310 * MB + 4), gdn.GDN_ERR_MISALIGNED),
+    (dict(gate=1, gr=A + 192 * MB + 8), gdn.GDN_ERR_MISALIGNED),
+    (dict(pos=A + 319 * MB + 2), gdn.GDN_ERR_MISALIGNED),
+    (dict(q=A + 32), gdn.GDN_ERR_INVALID_ARG),               # q overlaps q_raw (no in-place)
+    (dict(v=A + 384 * MB + 64), gdn.GDN_ERR_INVALID_ARG),    # v overlaps k
+    (dict(ring=A + 128 * MB), gdn.GDN_ERR_INVALID_ARG),      # ring overlaps v_raw
+    (dict(beta=A + 310 * MB), gdn.GDN_ERR_INVALID_ARG),      # beta overlaps the ring
+])
+def test_prologue_rejects(lib, kw, status):
+    assert _pro(lib, **kw) == status
+
+
+def test_prologue_with_no_tokens_launches_nothing(lib):
+    # T = 0: every per-token pointer may be null and nothing is launched.
+    assert _pro(lib, T=0, qr=None, kr=None, vr=None, gr=None, br=None, q=None, k=None, v=None,
+                g=None, beta=None) == gdn.GDN_OK
+
+
+def _step_pro(lib, qr=A, kr=A + 64 * MB, vr=A + 128 * MB, gr=A + 192 * MB, br=A + 256 * MB,
+              w=A + 300 * MB, ring=A + 310 * MB, pos=A + 319 * MB, s_in=A + 320 * MB,
+              s_out=A + 320 * MB, out=A + 448 * MB, B=1, H=1, dk=128, dv=128, gate=1, act=1):
+    c = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    return lib.gdn_recurrent_step_prologue(c(qr), c(kr), c(vr), c(gr), c(br), c(w), c(ring),
+                                           c(pos), c(s_in), c(s_out), c(out), B, H, dk, dv, gate,
+                                           act, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(ring=None), gdn.GDN_ERR_INVALID_ARG),              # the ring is required
+    (dict(s_in=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(out=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(B=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(act=-1), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dk=96), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(s_in=A + 320 * MB + 4, s_out=A + 320 * MB + 4), gdn.GDN_ERR_MISALIGNED),
+    (dict(out=A + 320 * MB), gdn.GDN_ERR_INVALID_ARG),       # out overlaps the state
+    (dict(s_out=A + 320 * MB + 1024), gdn.GDN_ERR_INVALID_ARG),   # partial state overlap
+    (dict(s_in=A + 310 * MB, s_out=A + 310 * MB), gdn.GDN_ERR_INVALID_ARG),  # state on the ring
+])
+def test_step_prologue_rejects(lib, kw, status):
+    assert _step_pro(lib, **kw) == status
