@@ -14,6 +14,11 @@ workload -- B=64 sequences, H=16, d=128, per-channel gate, fp32 state
 carried in place -- with L2 flushed before every timed step (the 64 MiB
 state would otherwise stay in the 126 MB L2), reported under "decode".
 
+The layer's input prologue is measured beside them under "prologue": the
+prefill pass (gdn_prologue) on the GDN-2 layer shape, and the decode step
+with the prologue fused in (gdn_recurrent_step_prologue) on the decode
+shape, each against the HBM bandwidth.
+
 Under torchrun (N > 1) every rank runs the same per-GPU workload on its own
 GPU (weak scaling, no collective on the data path); the reported time is
 the max over ranks.  Prints one JSON line on rank 0.
@@ -39,7 +44,7 @@ if str(ROOT) not in sys.path:
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from synth import CONFIGS, config_inputs  # noqa: E402
+from synth import CONFIGS, config_inputs, prologue_inputs  # noqa: E402
 
 PREFILL_CFG = CONFIGS[2]
 DECODE_CFG = CONFIGS[4]
@@ -381,6 +386,7 @@ def run_ours(args, rank: int, world: int, local: int):
            "overlap": "two buffer sets; uploads, calls and downloads on three streams"}
 
     decode = run_decode(gdn, dev, stream, peaks, world, rank)
+    prologue = run_prologue(gdn, dev, stream, peaks, world, rank)
 
     line = None
     if rank == 0:
@@ -397,9 +403,85 @@ def run_ours(args, rank: int, world: int, local: int):
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic", "config": workload_config(cfg), "roofline": roofline,
                 "tensor": tensor, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": args.steps, "clocks": clk.summary(), "decode": decode}
+                "gpu_launches": args.steps, "clocks": clk.summary(), "decode": decode,
+                "prologue": prologue}
         print(json.dumps(line))
     return 0
+
+
+def prologue_bytes(B, T, H, dk, dv, per_channel: bool) -> int:
+    """Algorithmic HBM bytes of one prologue pass: per token-head the raw
+    q, k, v (bf16) read and q, k, v written (bf16), g read and written (fp32,
+    dk values per channel gate or 1), beta read and written (fp32); per
+    (b, h) three ring slots read and min(T, 4) written (fp32); the taps once."""
+    C = 2 * dk + dv
+    gate = dk if per_channel else 1
+    per_tok = 2 * (2 * C) + 2 * 4 * gate + 2 * 4
+    return B * T * H * per_tok + B * H * (3 + min(T, 4)) * C * 4 + H * C * 4 * 4
+
+
+def run_prologue(gdn, dev, stream, peaks, world, rank, steps: int = 20, warmup: int = 3):
+    """The prologue's two forms, each timed alone (median of single-launch
+    CUDA-event timings).  The prefill pass moves 337 MB, more than L2; the
+    decode step's state is evicted from L2 before every timed step."""
+    pc = PREFILL_CFG
+    x = prologue_inputs(pc.B, pc.T, pc.H, pc.dk, pc.dv, gate=pc.gate, seed=pc.index + 1000 * rank)
+    xd = {n: (None if t is None else t.to(dev)) for n, t in x.items()}
+    args = [xd[n] for n in ("q_raw", "k_raw", "v_raw", "g_raw", "beta_raw", "conv_w")]
+    times = []
+    for i in range(warmup + steps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        gdn.prologue(*args, xd["ring"], xd["pos0"], stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= warmup:
+            times.append(e0.elapsed_time(e1) / 1e3)
+    t_pre = max_over_ranks(statistics.median(times), world)
+    b_pre = prologue_bytes(pc.B, pc.T, pc.H, pc.dk, pc.dv, pc.per_channel)
+    del xd, args
+
+    dc = DECODE_CFG
+    y = prologue_inputs(dc.B, 4, dc.H, dc.dk, dc.dv, gate=dc.gate, seed=dc.index + 1000 * rank)
+    yd = {n: t.to(dev) for n, t in y.items()}
+    state = torch.zeros(dc.B, dc.H, dc.dk, dc.dv, dtype=torch.float32, device=dev)
+    out = torch.empty(dc.B, dc.H, dc.dv, dtype=torch.float32, device=dev)
+    steps_in = [[yd[n][:, j].contiguous() for n in ("q_raw", "k_raw", "v_raw", "g_raw",
+                                                    "beta_raw")] for j in range(4)]
+    pos = [yd["pos0"] + j for j in range(warmup + steps)]
+    flush = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    times = []
+    for i in range(warmup + steps):
+        torch.sum(flush, dim=0, out=sink)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        gdn.recurrent_step_prologue(*steps_in[i % 4], yd["conv_w"], yd["ring"], state, pos[i],
+                                    out=out, stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= warmup:
+            times.append(e0.elapsed_time(e1) / 1e3)
+    t_dec = max_over_ranks(statistics.median(times), world)
+    C = 2 * dc.dk + dc.dv
+    b_dec = (decode_bytes(dc) + dc.B * dc.H * (3 + 1) * C * 4 + dc.H * C * 16)
+    hbm = peaks["hbm_gbs"]
+    return {
+        "prefill_pass": {"kernel": "prologue_kernel + prologue_ring_kernel",
+                         "us": t_pre * 1e6, "bytes": b_pre, "GB/s": b_pre / t_pre / 1e9,
+                         "frac": b_pre / t_pre / 1e9 / hbm, "peak": hbm,
+                         "config": {"workload": "input prologue of the GDN-2 layer prefill",
+                                    "B": pc.B, "T": pc.T, "H": pc.H, "dk": pc.dk, "dv": pc.dv,
+                                    "gate": pc.gate, "activation": "silu", "ring": True}},
+        "decode_fused": {"kernel": "recurrent_prologue_kernel", "us_per_step": t_dec * 1e6,
+                         "bytes": b_dec, "GB/s": b_dec / t_dec / 1e9,
+                         "frac": b_dec / t_dec / 1e9 / hbm, "peak": hbm,
+                         "config": {"workload": "decode step with the prologue fused in",
+                                    "B": dc.B, "H": dc.H, "dk": dc.dk, "dv": dc.dv,
+                                    "gate": dc.gate, "l2": "evicted before every timed step"}},
+        "timing": f"median of {steps} single-launch CUDA-event timings each"}
 
 
 def run_decode(gdn, dev, stream, peaks, world, rank, steps: int = 20, warmup: int = 3):

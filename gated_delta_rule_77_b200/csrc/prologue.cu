@@ -26,12 +26,46 @@
 namespace gdn {
 namespace {
 
-constexpr int TT = 32;   // tokens per CTA of the prefill prologue
+constexpr int TT = 16;   // tokens per CTA of the prefill prologue (a multiple of 8)
 
-__device__ __forceinline__ float act_fn(float y, bool silu) { return silu ? y / (1.f + expf(-y)) : y; }
+__device__ __forceinline__ float ex2_fast(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+constexpr float kLog2eP = 1.4426950408889634f;
+
+// SiLU y / (1 + e^-y) with the hardware 2^x and a fast divide (relative
+// error a few 1e-7, far below the bf16 rounding of the results).  The limits
+// hold: e^-y overflows to inf for y < -88 (result -0), underflows to 0 for
+// large y (result y).
+__device__ __forceinline__ float act_fn(float y, bool silu) {
+    return silu ? __fdividef(y, 1.f + ex2_fast(-y * kLog2eP)) : y;
+}
 __device__ __forceinline__ float sigmoid_fn(float x) { return 1.f / (1.f + expf(-x)); }
+
+// log(1 + u) for u in [0, 1] from log(1 + u) = 2 atanh(s), s = u / (2 + u)
+// in [0, 1/3], and the odd series atanh(s) = s + s^3/3 + s^5/5 + ...; eight
+// terms leave a remainder below (1/3)^16 / 17 < 1.5e-9 of the sum.  Relative
+// accuracy holds down to the smallest u (s ~ u/2), where log1p matters for
+// a gate near 0.
+__device__ __forceinline__ float log1p_unit(float u) {
+    const float s = __fdividef(u, 2.f + u);
+    const float z = s * s;
+    float t = 1.f / 15.f;
+    t = fmaf(t, z, 1.f / 13.f);
+    t = fmaf(t, z, 1.f / 11.f);
+    t = fmaf(t, z, 1.f / 9.f);
+    t = fmaf(t, z, 1.f / 7.f);
+    t = fmaf(t, z, 1.f / 5.f);
+    t = fmaf(t, z, 1.f / 3.f);
+    t = fmaf(t, z, 1.f);
+    return 2.f * s * t;
+}
+
+// g = -min(softplus(x), 5) with softplus(x) = max(x, 0) + log1p(e^-|x|).
 __device__ __forceinline__ float gate_fn(float x) {
-    const float sp = x > 30.f ? x : log1pf(expf(x));
+    const float sp = fmaxf(x, 0.f) + log1p_unit(ex2_fast(-fabsf(x) * kLog2eP));
     return -fminf(sp, 5.f);
 }
 
@@ -47,11 +81,28 @@ __device__ __forceinline__ float2 raw_pair(const __nv_bfloat16* q, const __nv_bf
     return __bfloat1622float2(x);
 }
 
-// One CTA: TT tokens of one (batch, head); one thread per pair of channels of
-// q | k | v (CP = (2 dk + dv) / 2 threads).  Sliding window of the last three
-// raw inputs in registers; the L2 norms of q and k through warp shuffles and
-// one shared-memory exchange between the warps of a tensor.
-template <int DK, int DV, bool CHANNEL>
+// 16 bytes (8 channels) of the raw row q | k | v of one token.
+__device__ __forceinline__ uint4 raw16(const __nv_bfloat16* q, const __nv_bfloat16* k,
+                                       const __nv_bfloat16* v, long tok, int c, int dk, int dv) {
+    const __nv_bfloat16* src;
+    long i;
+    if (c < dk) { src = q; i = tok * dk + c; }
+    else if (c < 2 * dk) { src = k; i = tok * dk + (c - dk); }
+    else { src = v; i = tok * dv + (c - 2 * dk); }
+    return *reinterpret_cast<const uint4*>(src + i);
+}
+
+// One CTA: TT tokens of one (batch, head).
+//   1. Stage: every thread issues its 16-byte loads of the raw rows of the
+//      tile (and the three rows before it, from the inputs or the ring) and
+//      of the gate, before any is used; the rows go to shared memory.
+//   2. Convolve: one thread per pair of channels slides the 4-tap window
+//      down the tile; the activations stay in registers.  The sums of
+//      squares of q and k per token go through warp shuffles and one
+//      exchange in shared memory.
+//   3. Normalise, write the bf16 results over the staged rows (each thread
+//      its own channels), and store the rows back with 16-byte stores.
+template <int DK, int DV, bool CHANNEL, int TT>
 __global__ void __launch_bounds__((2 * DK + DV) / 2)
 prologue_kernel(const __nv_bfloat16* __restrict__ q_raw, const __nv_bfloat16* __restrict__ k_raw,
                 const __nv_bfloat16* __restrict__ v_raw, const float* __restrict__ g_raw,
@@ -61,47 +112,116 @@ prologue_kernel(const __nv_bfloat16* __restrict__ q_raw, const __nv_bfloat16* __
                 float* __restrict__ g, float* __restrict__ beta, int T, int H)
 {
     constexpr int CH = 2 * DK + DV;
+    constexpr int NT = CH / 2;                  // threads
     constexpr int QW = DK / 64;                 // warps per q (and per k)
-    __shared__ float s_ss[2][QW][TT];           // per-warp sums of squares, q and k
+    constexpr int CPR = CH / 8;                 // 16-byte chunks per token row
+    constexpr int NX = TT * CPR;                // chunks of the tile
+    constexpr int PX = (NX + NT - 1) / NT;      // chunks per thread
+    constexpr int NG = CHANNEL ? TT * DK / 4 : 0;   // float4 of the per-channel gate
+    constexpr int PG = CHANNEL ? (NG + NT - 1) / NT : 0;
+    static_assert(3 * CPR <= NT && TT <= NT, "staging layout");
+
+    __shared__ __align__(16) __nv_bfloat16 s_x[TT][CH];   // raw rows, then results
+    __shared__ __align__(16) float s_h[3][CH];            // the three rows before the tile
+    __shared__ float s_ss[2][QW][TT];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int t0 = tile * TT;
-    const int c = 2 * tid;                      // first channel of this thread
-    const int p0 = pos0 ? pos0[b] : 0;
+    const int t0 = blockIdx.x * TT, h = blockIdx.y, b = blockIdx.z;
+    const int nt = min(TT, T - t0);
+    auto tok_of = [&](int t) -> long { return ((long)b * T + t) * H + h; };
 
-    const float* w = conv_w + ((long)h * CH + c) * 4;
-    const float4 w0 = *reinterpret_cast<const float4*>(w);        // taps of channel c
-    const float4 w1 = *reinterpret_cast<const float4*>(w + 4);    // taps of channel c + 1
-
-    // Window: raw inputs at t0 - 3, t0 - 2, t0 - 1.
-    float2 win[3];
+    // ---- 1. stage (all loads first) ----
+    uint4 xb[PX];
 #pragma unroll
-    for (int i = 0; i < 3; ++i) {
-        const int t = t0 - 3 + i;
+    for (int j = 0; j < PX; ++j) {
+        const int idx = tid + j * NT;
+        const int i = idx / CPR, cc = (idx % CPR) * 8;
+        xb[j] = make_uint4(0u, 0u, 0u, 0u);
+        if (idx < NX && i < nt) xb[j] = raw16(q_raw, k_raw, v_raw, tok_of(t0 + i), cc, DK, DV);
+    }
+    float hb[8];
+    const int hr = tid / CPR, hc = (tid % CPR) * 8;
+    if (tid < 3 * CPR) {
+        const int t = t0 - 3 + hr;
         if (t >= 0) {
-            win[i] = raw_pair(q_raw, k_raw, v_raw, ((long)b * T + t) * H + h, c, DK, DV);
+            const uint4 u = raw16(q_raw, k_raw, v_raw, tok_of(t), hc, DK, DV);
+            const __nv_bfloat162* e = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float2 f = __bfloat1622float2(e[m]);
+                hb[2 * m] = f.x; hb[2 * m + 1] = f.y;
+            }
         } else {
-            const int p = p0 + t;
-            win[i] = make_float2(0.f, 0.f);
-            if (ring && p >= 0) {
-                const float* r = ring + (((long)b * H + h) * 4 + (p & 3)) * CH + c;
-                win[i] = make_float2(r[0], r[1]);
+            const int p = (pos0 ? pos0[b] : 0) + t;
+#pragma unroll
+            for (int m = 0; m < 8; ++m) hb[m] = 0.f;
+            if (ring != nullptr && p >= 0) {
+                const float* r = ring + (((long)b * H + h) * 4 + (p & 3)) * CH + hc;
+                const float4 f0 = *reinterpret_cast<const float4*>(r);
+                const float4 f1 = *reinterpret_cast<const float4*>(r + 4);
+                hb[0] = f0.x; hb[1] = f0.y; hb[2] = f0.z; hb[3] = f0.w;
+                hb[4] = f1.x; hb[5] = f1.y; hb[6] = f1.z; hb[7] = f1.w;
             }
         }
     }
-    const int nt = min(TT, T - t0);
+    float4 gb[PG > 0 ? PG : 1];
+    if constexpr (CHANNEL) {
+#pragma unroll
+        for (int j = 0; j < PG; ++j) {
+            const int idx = tid + j * NT;
+            const int i = idx / (DK / 4), c4 = (idx % (DK / 4)) * 4;
+            gb[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (idx < NG && i < nt)
+                gb[j] = *reinterpret_cast<const float4*>(g_raw + tok_of(t0 + i) * DK + c4);
+        }
+    }
+    float braw = 0.f, graw = 0.f;
+    if (tid < nt) {
+        braw = beta_raw[tok_of(t0 + tid)];
+        if (!CHANNEL) graw = g_raw[tok_of(t0 + tid)];
+    }
+
+#pragma unroll
+    for (int j = 0; j < PX; ++j) {
+        const int idx = tid + j * NT;
+        if (idx < NX) *reinterpret_cast<uint4*>(&s_x[idx / CPR][(idx % CPR) * 8]) = xb[j];
+    }
+    if (tid < 3 * CPR) {
+        *reinterpret_cast<float4*>(&s_h[hr][hc]) = make_float4(hb[0], hb[1], hb[2], hb[3]);
+        *reinterpret_cast<float4*>(&s_h[hr][hc + 4]) = make_float4(hb[4], hb[5], hb[6], hb[7]);
+    }
+    // The gate maps need nothing staged: apply and store them now.
+    if constexpr (CHANNEL) {
+#pragma unroll
+        for (int j = 0; j < PG; ++j) {
+            const int idx = tid + j * NT;
+            const int i = idx / (DK / 4), c4 = (idx % (DK / 4)) * 4;
+            if (idx < NG && i < nt)
+                *reinterpret_cast<float4*>(g + tok_of(t0 + i) * DK + c4) =
+                    make_float4(gate_fn(gb[j].x), gate_fn(gb[j].y), gate_fn(gb[j].z), gate_fn(gb[j].w));
+        }
+    }
+    if (tid < nt) {
+        beta[tok_of(t0 + tid)] = sigmoid_fn(braw);
+        if (!CHANNEL) g[tok_of(t0 + tid)] = gate_fn(graw);
+    }
+    __syncthreads();
+
+    // ---- 2. convolve ----
+    const int c = 2 * tid;
+    const float4 w0 = *reinterpret_cast<const float4*>(conv_w + ((long)h * CH + c) * 4);
+    const float4 w1 = *reinterpret_cast<const float4*>(conv_w + ((long)h * CH + c + 1) * 4);
+    float2 win[3];
+#pragma unroll
+    for (int r = 0; r < 3; ++r) win[r] = make_float2(s_h[r][c], s_h[r][c + 1]);
     float2 y[TT];
 #pragma unroll
     for (int i = 0; i < TT; ++i) {
-        y[i] = make_float2(0.f, 0.f);
-        if (i < nt) {
-            const float2 x = raw_pair(q_raw, k_raw, v_raw, ((long)b * T + t0 + i) * H + h, c, DK, DV);
-            float a0 = w0.x * win[0].x + w0.y * win[1].x + w0.z * win[2].x + w0.w * x.x;
-            float a1 = w1.x * win[0].y + w1.y * win[1].y + w1.z * win[2].y + w1.w * x.y;
-            y[i] = make_float2(act_fn(a0, silu), act_fn(a1, silu));
-            win[0] = win[1]; win[1] = win[2]; win[2] = x;
-        }
+        const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&s_x[i][c]));
+        const float a0 = w0.x * win[0].x + w0.y * win[1].x + w0.z * win[2].x + w0.w * x.x;
+        const float a1 = w1.x * win[0].y + w1.y * win[1].y + w1.z * win[2].y + w1.w * x.y;
+        y[i] = make_float2(act_fn(a0, silu), act_fn(a1, silu));
+        win[0] = win[1]; win[1] = win[2]; win[2] = x;
     }
     const int tensor = warp / QW;               // 0 q, 1 k, >= 2 v
     if (tensor < 2) {
@@ -113,21 +233,11 @@ prologue_kernel(const __nv_bfloat16* __restrict__ q_raw, const __nv_bfloat16* __
             if (lane == 0) s_ss[tensor][warp % QW][i] = ss;
         }
     }
-    // beta and a scalar g: the v threads (which follow the DK threads of q and
-    // k), one token each.
-    if (tensor >= 2) {
-        const int i = tid - DK;
-        if (i < nt) {
-            const long tok = ((long)b * T + t0 + i) * H + h;
-            beta[tok] = sigmoid_fn(beta_raw[tok]);
-            if (!CHANNEL) g[tok] = gate_fn(g_raw[tok]);
-        }
-    }
     __syncthreads();
+
+    // ---- 3. normalise, write over the staged rows, store ----
 #pragma unroll
     for (int i = 0; i < TT; ++i) {
-        if (i >= nt) break;
-        const long tok = ((long)b * T + t0 + i) * H + h;
         float2 o = y[i];
         if (tensor < 2) {
             float ss = 0.f;
@@ -136,17 +246,19 @@ prologue_kernel(const __nv_bfloat16* __restrict__ q_raw, const __nv_bfloat16* __
             const float inv = rsqrtf(ss + 1e-6f);
             o.x *= inv; o.y *= inv;
         }
-        const __nv_bfloat162 ob = __floats2bfloat162_rn(o.x, o.y);
-        if (tensor == 0) {
-            *reinterpret_cast<__nv_bfloat162*>(q + tok * DK + c) = ob;
-            if (CHANNEL) {   // the q threads also map the per-channel gate
-                const float2 gr = *reinterpret_cast<const float2*>(g_raw + tok * DK + c);
-                *reinterpret_cast<float2*>(g + tok * DK + c) = make_float2(gate_fn(gr.x), gate_fn(gr.y));
-            }
-        } else if (tensor == 1) {
-            *reinterpret_cast<__nv_bfloat162*>(k + tok * DK + (c - DK)) = ob;
-        } else {
-            *reinterpret_cast<__nv_bfloat162*>(v + tok * DV + (c - 2 * DK)) = ob;
+        *reinterpret_cast<__nv_bfloat162*>(&s_x[i][c]) = __floats2bfloat162_rn(o.x, o.y);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < PX; ++j) {
+        const int idx = tid + j * NT;
+        const int i = idx / CPR, cc = (idx % CPR) * 8;
+        if (idx < NX && i < nt) {
+            const uint4 u = *reinterpret_cast<const uint4*>(&s_x[i][cc]);
+            const long tok = tok_of(t0 + i);
+            __nv_bfloat16* dst = cc < DK ? q + tok * DK + cc
+                               : cc < 2 * DK ? k + tok * DK + (cc - DK) : v + tok * DV + (cc - 2 * DK);
+            *reinterpret_cast<uint4*>(dst) = u;
         }
     }
 }
@@ -180,7 +292,7 @@ __global__ void prologue_ring_kernel(const __nv_bfloat16* __restrict__ q_raw,
 // 0, v columns by the slice that owns them), so no CTA writes what another
 // reads in the same call.
 template <int DK, int COLS, int NWARPS, bool CHANNEL>
-__global__ void __launch_bounds__(NWARPS * 32)
+__global__ void __launch_bounds__(NWARPS * 32, 5)   // 5 CTAs per SM: measured faster than 4
 recurrent_prologue_kernel(const __nv_bfloat16* __restrict__ q_raw, const __nv_bfloat16* __restrict__ k_raw,
                           const __nv_bfloat16* __restrict__ v_raw, const float* __restrict__ g_raw,
                           const float* __restrict__ beta_raw, const float* __restrict__ conv_w,
@@ -211,30 +323,39 @@ recurrent_prologue_kernel(const __nv_bfloat16* __restrict__ q_raw, const __nv_bf
     const long tok = (long)b * H + h;
     const long ring_bh = ((long)b * H + h) * 4;
 
+    // The state slice first (8-byte loads, the bulk of the traffic), then the
+    // prologue's loads, none of which waits on another: the ring is read in
+    // all four slots and the three history slots are picked afterwards.
     float s[R][VW];
     const long sbase = ((long)b * H + h) * DK * (long)dv;
-    if (state_in != nullptr) {
 #pragma unroll
-        for (int r = 0; r < R; ++r)
-#pragma unroll
-            for (int c = 0; c < VW; ++c) s[r][c] = state_in[sbase + (long)(row0 + r) * dv + col0 + c];
-    } else {
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-#pragma unroll
-            for (int c = 0; c < VW; ++c) s[r][c] = 0.f;
+    for (int r = 0; r < R; ++r) {
+        if constexpr (VW == 2) {
+            float2 t = make_float2(0.f, 0.f);
+            if (state_in != nullptr)
+                t = *reinterpret_cast<const float2*>(state_in + sbase + (long)(row0 + r) * dv + col0);
+            s[r][0] = t.x; s[r][1] = t.y;
+        } else {
+            s[r][0] = state_in != nullptr ? state_in[sbase + (long)(row0 + r) * dv + col0] : 0.f;
+        }
     }
 
-    // Convolution of one channel: taps 0..2 from the ring, tap 3 the input.
+    // Convolution of one channel: taps 0..2 from ring slots p-3 .. p-1 (zero
+    // before position 0), tap 3 the input.
     auto conv1 = [&](int ch, float x) -> float {
         const float4 w = *reinterpret_cast<const float4*>(conv_w + ((long)h * CH + ch) * 4);
-        float hst[3] = {0.f, 0.f, 0.f};
+        float sl[4] = {0.f, 0.f, 0.f, 0.f};
         if (ring) {
 #pragma unroll
-            for (int j = 0; j < 3; ++j) {
-                const int pp = p - 3 + j;
-                if (pp >= 0) hst[j] = ring[(ring_bh + (pp & 3)) * CH + ch];
-            }
+            for (int j = 0; j < 4; ++j) sl[j] = ring[(ring_bh + j) * CH + ch];
+        }
+        float hst[3];
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+            const int pp = p - 3 + j;
+            const int m = pp & 3;
+            const float val = m == 0 ? sl[0] : m == 1 ? sl[1] : m == 2 ? sl[2] : sl[3];
+            hst[j] = pp >= 0 ? val : 0.f;
         }
         return act_fn(w.x * hst[0] + w.y * hst[1] + w.z * hst[2] + w.w * x, silu);
     };
@@ -341,11 +462,11 @@ cudaError_t launch_prologue_t(const PrologueArgs& a, cudaStream_t stream) {
     constexpr int threads = (2 * DK + DV) / 2;
     if (a.T > 0) {
         if (a.per_channel)
-            prologue_kernel<DK, DV, true><<<grid, threads, 0, stream>>>(
+            prologue_kernel<DK, DV, true, TT><<<grid, threads, 0, stream>>>(
                 a.q_raw, a.k_raw, a.v_raw, a.g_raw, a.beta_raw, a.conv_w, a.ring, a.pos0, a.silu,
                 a.q, a.k, a.v, a.g, a.beta, a.T, a.H);
         else
-            prologue_kernel<DK, DV, false><<<grid, threads, 0, stream>>>(
+            prologue_kernel<DK, DV, false, TT><<<grid, threads, 0, stream>>>(
                 a.q_raw, a.k_raw, a.v_raw, a.g_raw, a.beta_raw, a.conv_w, a.ring, a.pos0, a.silu,
                 a.q, a.k, a.v, a.g, a.beta, a.T, a.H);
         cudaError_t e = cudaGetLastError();
@@ -359,10 +480,13 @@ cudaError_t launch_prologue_t(const PrologueArgs& a, cudaStream_t stream) {
     return cudaSuccess;
 }
 
+constexpr int STEP_COLS = 64;   // value columns per CTA of the fused decode step
+constexpr int STEP_WARPS = 4;
+
 template <int DK, bool CHANNEL>
 cudaError_t launch_step_t(const StepPrologueArgs& a, cudaStream_t stream) {
-    const unsigned grid = static_cast<unsigned>(a.dv / 64) * a.H * a.B;
-    recurrent_prologue_kernel<DK, 64, 4, CHANNEL><<<grid, 128, 0, stream>>>(
+    const unsigned grid = static_cast<unsigned>(a.dv / STEP_COLS) * a.H * a.B;
+    recurrent_prologue_kernel<DK, STEP_COLS, STEP_WARPS, CHANNEL><<<grid, STEP_WARPS * 32, 0, stream>>>(
         a.q_raw, a.k_raw, a.v_raw, a.g_raw, a.beta_raw, a.conv_w, a.ring, a.pos, a.silu, a.state_in,
         a.state_out, a.out, a.H, a.dv);
     return cudaGetLastError();
