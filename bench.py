@@ -387,6 +387,7 @@ def run_ours(args, rank: int, world: int, local: int):
 
     decode = run_decode(gdn, dev, stream, peaks, world, rank)
     prologue = run_prologue(gdn, dev, stream, peaks, world, rank)
+    multitoken = run_multitoken(gdn, dev, stream, peaks, world, rank)
 
     line = None
     if rank == 0:
@@ -404,7 +405,7 @@ def run_ours(args, rank: int, world: int, local: int):
                 "data": "synthetic", "config": workload_config(cfg), "roofline": roofline,
                 "tensor": tensor, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": args.steps, "clocks": clk.summary(), "decode": decode,
-                "prologue": prologue}
+                "prologue": prologue, "multi_token_decode": multitoken}
         print(json.dumps(line))
     return 0
 
@@ -482,6 +483,46 @@ def run_prologue(gdn, dev, stream, peaks, world, rank, steps: int = 20, warmup: 
                                     "B": dc.B, "H": dc.H, "dk": dc.dk, "dv": dc.dv,
                                     "gate": dc.gate, "l2": "evicted before every timed step"}},
         "timing": f"median of {steps} single-launch CUDA-event timings each"}
+
+
+def run_multitoken(gdn, dev, stream, peaks, world, rank, T: int = 4, steps: int = 20,
+                   warmup: int = 3):
+    """Multi-token decode (T draft tokens per sequence, state after every
+    token kept) on the decode shape, L2 evicted before every timed call."""
+    from synth import prefill_inputs
+    cfg = DECODE_CFG
+    x = prefill_inputs(cfg.B, T, cfg.H, cfg.dk, cfg.dv, gate=cfg.gate, s0_std=cfg.s0_std,
+                       seed=cfg.index + 1000 * rank)
+    d = {n: x[n].to(dev) for n in ("q", "k", "v", "g", "beta", "s0")}
+    snap = torch.empty(cfg.B, T, cfg.H, cfg.dk, cfg.dv, dtype=torch.float32, device=dev)
+    out = torch.empty(cfg.B, T, cfg.H, cfg.dv, dtype=torch.float32, device=dev)
+    flush = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    times = []
+    for i in range(warmup + steps):
+        torch.sum(flush, dim=0, out=sink)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        gdn.recurrent_steps(d["q"], d["k"], d["v"], d["g"], d["beta"], d["s0"], snapshots=snap,
+                            out=out, stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= warmup:
+            times.append(e0.elapsed_time(e1) / 1e3)
+    t = max_over_ranks(statistics.median(times), world)
+    bh = cfg.B * cfg.H
+    st = cfg.dk * cfg.dv * 4
+    per_tok = 2 * (2 * cfg.dk + cfg.dv) + 4 * (cfg.dk if cfg.per_channel else 1) + 4 + 4 * cfg.dv
+    nbytes = bh * (st + T * st + T * per_tok)
+    gbs = nbytes / t / 1e9
+    return {"metric": "multi-token decode GB/s", "value": gbs, "unit": "GB/s",
+            "us_per_call": t * 1e6, "frac": gbs / peaks["hbm_gbs"], "peak": peaks["hbm_gbs"],
+            "bytes_per_call": nbytes, "tokens_per_s": cfg.B * T * world / t,
+            "config": {"workload": "multi-token decode with per-token state snapshots",
+                       "B": cfg.B, "H": cfg.H, "T": T, "dk": cfg.dk, "dv": cfg.dv,
+                       "gate": cfg.gate, "l2": "evicted before every timed call"},
+            "timing": f"median of {steps} single-call CUDA-event timings"}
 
 
 def run_decode(gdn, dev, stream, peaks, world, rank, steps: int = 20, warmup: int = 3):

@@ -38,7 +38,8 @@ ACT_SILU = 1
 
 SYMBOLS = ("gdn_chunk_fwd", "gdn_chunk_fwd_ex", "gdn_chunk_fwd_segments",
            "gdn_chunk_fwd_segments_noalloc", "gdn_recurrent_step", "gdn_recurrent_step_ex",
-           "gdn_prologue", "gdn_recurrent_step_prologue", "gdn_check", "gdn_status_string")
+           "gdn_recurrent_steps", "gdn_state_select", "gdn_prologue", "gdn_recurrent_step_prologue",
+           "gdn_check", "gdn_status_string")
 
 _lib = None
 
@@ -65,6 +66,8 @@ def load() -> ctypes.CDLL:
                                                    vp]
     lib.gdn_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, vp]
     lib.gdn_recurrent_step_ex.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, i, vp]
+    lib.gdn_recurrent_steps.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, vp, i, i, i, i, i, i, vp]
+    lib.gdn_state_select.argtypes = [fp, vp, fp, i, i, i, i, i, vp]
     lib.gdn_prologue.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, vp, vp, vp, fp, fp, i, i, i, i, i,
                                  i, i, vp]
     lib.gdn_recurrent_step_prologue.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, fp, fp, vp, i, i, i,
@@ -154,6 +157,43 @@ def recurrent_step(q, k, v, g, beta, state, *, state_out=None, out=None, stream=
     if rc != GDN_OK:
         raise GdnError(rc, "gdn_recurrent_step_ex")
     return out
+
+
+def recurrent_steps(q, k, v, g, beta, state, *, state_out=None, snapshots=True, out=None,
+                    stream=None):
+    """T successive decode tokens per sequence (speculative verification).
+    q, k [B,T,H,dk] bf16; v [B,T,H,dv] bf16; g [B,T,H] or [B,T,H,dk];
+    beta [B,T,H]; state [B,H,dk,dv] fp32, read only unless state_out is
+    ``state`` itself.  ``snapshots``: True allocates [B,T,H,dk,dv], a tensor
+    is written, None skips them.  Returns (out [B,T,H,dv] fp32, snapshots)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    gate = GATE_CHANNEL if g.dim() == 4 else GATE_SCALAR
+    if snapshots is True:
+        snapshots = torch.empty(B, T, H, dk, dv, dtype=torch.float32, device=v.device)
+    if out is None:
+        out = torch.empty(B, T, H, dv, dtype=torch.float32, device=v.device)
+    _check_cuda(q, k, v, g, beta, state, state_out, snapshots, out)
+    rc = load().gdn_recurrent_steps(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
+                                    _ptr(state_out), _ptr(snapshots), _ptr(out), B, T, H, dk, dv,
+                                    gate, _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_recurrent_steps")
+    return out, snapshots
+
+
+def state_select(snapshots, num_accepted, state, *, stream=None):
+    """state[b] := snapshots[b, num_accepted[b] - 1] where 1 <= n_b <= T
+    (num_accepted: int32 [B] on the device); other rows unchanged."""
+    B, T, H, dk, dv = snapshots.shape
+    _check_cuda(snapshots, num_accepted, state)
+    if num_accepted.dtype != torch.int32:
+        raise ValueError("num_accepted must be int32")
+    rc = load().gdn_state_select(_ptr(snapshots), _ptr(num_accepted), _ptr(state), B, T, H, dk, dv,
+                                 _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_state_select")
+    return state
 
 
 def _act_code(activation):

@@ -300,6 +300,54 @@ int gdn_recurrent_step(const void* q, const void* k, const void* v, const float*
                                  gate_mode, GDN_IO_BF16, stream);
 }
 
+int gdn_recurrent_steps(const void* q, const void* k, const void* v, const float* g,
+                        const float* beta, const float* state_in, float* state_out,
+                        float* snapshots, void* out, int B, int T, int H, int dk, int dv,
+                        int gate_mode, gdn_stream_t stream_)
+{
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (!state_in || T < 1) return GDN_ERR_INVALID_ARG;
+    if (!state_out && !snapshots) return GDN_ERR_INVALID_ARG;   // nothing would be kept
+    int rc = validate(q, k, v, g, beta, state_in, state_out, out, B, T, H, dk, dv, gate_mode,
+                      GDN_IO_BF16, true, false);
+    if (rc != GDN_OK) return rc;
+    if (snapshots) {
+        if (!aligned16(snapshots)) return GDN_ERR_MISALIGNED;
+        const size_t tok = (size_t)B * T * H;
+        const size_t st = (size_t)B * H * dk * dv * 4;
+        const Range rs = range_of(snapshots, tok * dk * dv * 4);
+        const bool ch = gate_mode == GDN_GATE_CHANNEL;
+        const Range others[] = {range_of(q, tok * dk * 2), range_of(k, tok * dk * 2),
+                                range_of(v, tok * dv * 2), range_of(g, tok * (ch ? dk : 1) * 4),
+                                range_of(beta, tok * 4), range_of(out, tok * dv * 4),
+                                range_of(state_in, st),
+                                state_out ? range_of(state_out, st) : Range{0, 0}};
+        for (Range r : others)
+            if (overlaps(rs, r)) return GDN_ERR_INVALID_ARG;
+    }
+    gdn::Problem p{q, k, v, g, beta, state_in, state_out, out, B, T, H, dk, dv,
+                   gate_mode == GDN_GATE_CHANNEL, false, true};
+    p.snapshots = snapshots;
+    return to_status(gdn::launch_recurrent(p, stream));
+}
+
+int gdn_state_select(const float* snapshots, const int* num_accepted, float* state, int B, int T,
+                     int H, int dk, int dv, gdn_stream_t stream_)
+{
+    if (!snapshots || !num_accepted || !state) return GDN_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || T < 1) return GDN_ERR_INVALID_ARG;
+    if (!dim_ok(dk) || !dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
+    if (B > 65535 || H > 65535 || (long)B * H > 2147483647L) return GDN_ERR_UNSUPPORTED;
+    if (!aligned16(snapshots) || !aligned16(state)) return GDN_ERR_MISALIGNED;
+    if (reinterpret_cast<uintptr_t>(num_accepted) & 3u) return GDN_ERR_MISALIGNED;
+    const size_t st = (size_t)B * H * dk * dv * 4;
+    const Range rst = range_of(state, st);
+    if (overlaps(rst, range_of(snapshots, st * T)) || overlaps(rst, range_of(num_accepted, (size_t)B * 4)))
+        return GDN_ERR_INVALID_ARG;
+    return to_status(gdn::launch_state_select(snapshots, num_accepted, state, B, T, H, dk, dv,
+                                              reinterpret_cast<cudaStream_t>(stream_)));
+}
+
 int gdn_check(gdn_stream_t stream_)
 {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);

@@ -26,10 +26,16 @@ struct Problem {
     bool io_f32;             // q, k, v in fp32 (else bf16)
     bool out_f32;            // out in fp32 (else bf16)
     int segments = 0;        // chunk path: time segments per (b, h); 0 = automatic
+    float* snapshots = nullptr;   // token-serial path: S after every token, [B, T, H, dk, dv]
 };
 
 // Token-serial fused recurrence (decode, and the fp32 / fallback prefill).
 cudaError_t launch_recurrent(const Problem& p, cudaStream_t stream);
+
+// state_out[b] := snapshots[b, n_b - 1] for 1 <= n_b <= T (n = num_accepted,
+// device memory); other rows are left as they are.
+cudaError_t launch_state_select(const float* snapshots, const int* num_accepted, float* state_out,
+                                int B, int T, int H, int dk, int dv, cudaStream_t stream);
 
 // Chunkwise tensor-core prefill (bf16 I/O, dk = dv = 128, chunk of 64).
 // Returns cudaErrorNotSupported for shapes it does not handle.

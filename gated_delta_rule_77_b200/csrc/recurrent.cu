@@ -19,6 +19,10 @@
 // adjacent columns (one vector load per row); the state stays in registers
 // for all T tokens.  The two column reductions go through shared memory once
 // per token; the rank-1 update and the output are then local.
+//
+// Multi-token decode (speculative verification of T draft tokens): with a
+// snapshot buffer every token's updated state slice is also stored, so that
+// the caller can resume from the state after any accepted prefix.
 
 #include "gdn_internal.cuh"
 
@@ -68,7 +72,7 @@ __global__ void __launch_bounds__(NWARPS * 32)
 recurrent_kernel(const TIN* __restrict__ q, const TIN* __restrict__ k,
                  const TIN* __restrict__ v, const float* __restrict__ g,
                  const float* __restrict__ beta, const float* state_in, float* state_out,
-                 TOUT* __restrict__ out, int T, int H, int dv)
+                 TOUT* __restrict__ out, float* __restrict__ snap, int T, int H, int dv)
 {
     constexpr int VW = COLS / 32;
     constexpr int R = DK / NWARPS;
@@ -167,6 +171,11 @@ recurrent_kernel(const TIN* __restrict__ q, const TIN* __restrict__ k,
 #pragma unroll
             for (int c = 0; c < VW; ++c) s[r][c] = fmaf(ki, u[c], s[r][c]);
         }
+        if (snap != nullptr) {   // S after token t: snapshot [b, t, h]
+            float* dst = snap + tok * DK * (long)dv;
+#pragma unroll
+            for (int r = 0; r < R; ++r) store_vec<VW>(dst + (long)(row0 + r) * dv + col0, s[r]);
+        }
     }
 
     if (state_out != nullptr) {
@@ -180,7 +189,7 @@ cudaError_t launch_typed(const Problem& p, cudaStream_t stream) {
     const unsigned grid = static_cast<unsigned>(p.dv / COLS) * p.H * p.B;
     recurrent_kernel<DK, COLS, NWARPS, CHANNEL, TIN, TOUT><<<grid, NWARPS * 32, 0, stream>>>(
         static_cast<const TIN*>(p.q), static_cast<const TIN*>(p.k), static_cast<const TIN*>(p.v),
-        p.g, p.beta, p.state_in, p.state_out, static_cast<TOUT*>(p.out), p.T, p.H, p.dv);
+        p.g, p.beta, p.state_in, p.state_out, static_cast<TOUT*>(p.out), p.snapshots, p.T, p.H, p.dv);
     return cudaGetLastError();
 }
 
@@ -190,7 +199,9 @@ cudaError_t launch_dk(const Problem& p, cudaStream_t stream) {
     // state per thread (32 independent 8-byte loads in flight per thread);
     // measured fastest of 32/64/128-column slices x 4/8/16 warps on B200.
     // Long token loops (prefill) use 32-column slices for more CTAs per head.
-    if (p.T == 1) return launch_typed<DK, 64, 4, CHANNEL, TIN, TOUT>(p, stream);
+    // A few tokens over many heads (multi-token decode) keep the decode tiling.
+    const long ctas64 = (long)p.B * p.H * (p.dv / 64);
+    if (p.T == 1 || (p.T <= 16 && ctas64 >= 2 * 148)) return launch_typed<DK, 64, 4, CHANNEL, TIN, TOUT>(p, stream);
     return launch_typed<DK, 32, DK / 16, CHANNEL, TIN, TOUT>(p, stream);
 }
 
@@ -206,7 +217,28 @@ cudaError_t launch_io(const Problem& p, cudaStream_t stream) {
                          : launch_gate<false, TIN, TOUT>(p, stream);
 }
 
+// One CTA per (b, h): copies snapshot n_b - 1 of row b into the state.
+__global__ void state_select_kernel(const float4* __restrict__ snap, const int* __restrict__ nacc,
+                                    float4* __restrict__ state, int T, int H, long n4)
+{
+    const int h = blockIdx.x % H, b = blockIdx.x / H;
+    const int n = nacc[b];
+    if (n < 1 || n > T) return;
+    const float4* src = snap + (((long)b * T + (n - 1)) * H + h) * n4;
+    float4* dst = state + ((long)b * H + h) * n4;
+    for (long i = threadIdx.x; i < n4; i += blockDim.x) dst[i] = src[i];
+}
+
 }  // namespace
+
+cudaError_t launch_state_select(const float* snapshots, const int* num_accepted, float* state_out,
+                                int B, int T, int H, int dk, int dv, cudaStream_t stream) {
+    const long n4 = (long)dk * dv / 4;
+    state_select_kernel<<<(unsigned)(B * H), 256, 0, stream>>>(
+        reinterpret_cast<const float4*>(snapshots), num_accepted, reinterpret_cast<float4*>(state_out),
+        T, H, n4);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_recurrent(const Problem& p, cudaStream_t stream) {
     if (p.io_f32) {

@@ -199,6 +199,40 @@ GDN_API int gdn_recurrent_step_ex(const void* q, const void* k, const void* v, c
                           int io_dtype, gdn_stream_t stream);
 
 /*
+ * gdn_recurrent_steps -- T successive tokens per sequence through the decode
+ * kernel (speculative verification of T draft tokens; the fused recurrent
+ * mode of the "Gated DeltaNet" entity trail, finding of 2026-07-29), with the
+ * state after every token optionally kept.
+ *
+ *   q, k      [B, T, H, dk] bf16;  v [B, T, H, dv] bf16 (token-major, as the
+ *             prefill)
+ *   g         [B, T, H] or [B, T, H, dk] fp32 (g <= 0);  beta [B, T, H] fp32
+ *   state_in  [B, H, dk, dv] fp32 (required)
+ *   state_out [B, H, dk, dv] fp32: the state after all T tokens, or NULL;
+ *             == state_in updates in place
+ *   snapshots [B, T, H, dk, dv] fp32: snapshots[b, t, h] = S_t, the state of
+ *             (b, h) after token t, or NULL.  At least one of state_out and
+ *             snapshots is required.
+ *   out       [B, T, H, dv] fp32
+ *   T >= 1; dk, dv 64 or 128.  Results equal T calls of gdn_recurrent_step
+ *   (same arithmetic, same order).
+ */
+GDN_API int gdn_recurrent_steps(const void* q, const void* k, const void* v, const float* g,
+                                const float* beta, const float* state_in, float* state_out,
+                                float* snapshots, void* out, int B, int T, int H, int dk, int dv,
+                                int gate_mode, gdn_stream_t stream);
+
+/*
+ * gdn_state_select -- commit the accepted prefix of a verification step:
+ * state[b] := snapshots[b, n_b - 1] for every sequence b whose accepted
+ * count n_b = num_accepted[b] (int32, device memory) lies in 1 .. T; rows
+ * with any other count are left as they are.  snapshots as written by
+ * gdn_recurrent_steps; state [B, H, dk, dv] fp32 must not overlap them.
+ */
+GDN_API int gdn_state_select(const float* snapshots, const int* num_accepted, float* state,
+                             int B, int T, int H, int dk, int dv, gdn_stream_t stream);
+
+/*
  * The layer's input prologue: what turns the projected inputs of a Gated
  * DeltaNet layer into the recurrence's q, k, v, g and beta.
  *   - A causal depthwise convolution of width 4 over the token axis on every

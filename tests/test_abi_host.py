@@ -178,3 +178,45 @@ def _step_pro(lib, qr=A, kr=A + 64 * MB, vr=A + 128 * MB, gr=A + 192 * MB, br=A 
 ])
 def test_step_prologue_rejects(lib, kw, status):
     assert _step_pro(lib, **kw) == status
+
+
+def _steps(lib, q=A, k=A + 64 * MB, v=A + 128 * MB, g=A + 192 * MB, beta=A + 256 * MB,
+           s_in=A + 320 * MB, s_out=A + 320 * MB, snap=A + 512 * MB, out=A + 448 * MB, B=1, T=4, H=1,
+           dk=128, dv=128, gate=1):
+    c = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    return lib.gdn_recurrent_steps(c(q), c(k), c(v), c(g), c(beta), c(s_in), c(s_out), c(snap),
+                                   c(out), B, T, H, dk, dv, gate, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(s_in=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(s_out=None, snap=None), gdn.GDN_ERR_INVALID_ARG),      # nothing would be kept
+    (dict(T=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(q=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dv=48), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(snap=A + 512 * MB + 4), gdn.GDN_ERR_MISALIGNED),
+    (dict(snap=A + 448 * MB), gdn.GDN_ERR_INVALID_ARG),          # snapshots overlap out
+    (dict(snap=A + 320 * MB), gdn.GDN_ERR_INVALID_ARG),          # snapshots overlap the state
+    (dict(out=A + 320 * MB + 64), gdn.GDN_ERR_INVALID_ARG),      # out overlaps the state
+])
+def test_recurrent_steps_rejects(lib, kw, status):
+    assert _steps(lib, **kw) == status
+
+
+def _select(lib, snap=A, nacc=A + 300 * MB, state=A + 320 * MB, B=2, T=4, H=2, dk=128, dv=128):
+    c = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    return lib.gdn_state_select(c(snap), c(nacc), c(state), B, T, H, dk, dv, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(snap=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(nacc=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(state=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(T=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dk=32), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(state=A + 320 * MB + 8), gdn.GDN_ERR_MISALIGNED),
+    (dict(nacc=A + 300 * MB + 2), gdn.GDN_ERR_MISALIGNED),
+    (dict(state=A + 1024), gdn.GDN_ERR_INVALID_ARG),             # state overlaps the snapshots
+])
+def test_state_select_rejects(lib, kw, status):
+    assert _select(lib, **kw) == status
