@@ -38,7 +38,7 @@ ACT_SILU = 1
 
 SYMBOLS = ("gdn_chunk_fwd", "gdn_chunk_fwd_ex", "gdn_chunk_fwd_segments",
            "gdn_chunk_fwd_segments_noalloc", "gdn_recurrent_step", "gdn_recurrent_step_ex",
-           "gdn_recurrent_steps", "gdn_state_select", "gdn_prologue", "gdn_recurrent_step_prologue",
+           "gdn_chunk_bwd", "gdn_recurrent_steps", "gdn_state_select", "gdn_prologue", "gdn_recurrent_step_prologue",
            "gdn_check", "gdn_status_string")
 
 _lib = None
@@ -66,6 +66,8 @@ def load() -> ctypes.CDLL:
                                                    vp]
     lib.gdn_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, vp]
     lib.gdn_recurrent_step_ex.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, i, vp]
+    lib.gdn_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, fp, fp, fp, fp, fp, fp, i, i, i,
+                                  i, i, i, vp]
     lib.gdn_recurrent_steps.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, vp, i, i, i, i, i, i, vp]
     lib.gdn_state_select.argtypes = [fp, vp, fp, i, i, i, i, i, vp]
     lib.gdn_prologue.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, vp, vp, vp, fp, fp, i, i, i, i, i,
@@ -156,6 +158,32 @@ def recurrent_step(q, k, v, g, beta, state, *, state_out=None, out=None, stream=
                                       gate, _io_code(q.dtype), _stream(stream))
     if rc != GDN_OK:
         raise GdnError(rc, "gdn_recurrent_step_ex")
+    return out
+
+
+def chunk_bwd(q, k, v, g, beta, state_in, d_out, d_state_out=None, *, stream=None):
+    """Gradients of the prefill (gdn_chunk_bwd) for the loss
+    sum(d_out * out) + sum(d_state_out * state_out).  Returns a dict of fp32
+    tensors dq, dk, dv, dg, dbeta and ds0 (the initial state's gradient)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    gate = GATE_CHANNEL if g.dim() == 4 else GATE_SCALAR
+    dev = q.device
+    out = dict(dq=torch.empty(B, T, H, dk, dtype=torch.float32, device=dev),
+               dk=torch.empty(B, T, H, dk, dtype=torch.float32, device=dev),
+               dv=torch.empty(B, T, H, dv, dtype=torch.float32, device=dev),
+               dg=torch.empty(g.shape, dtype=torch.float32, device=dev),
+               dbeta=torch.empty(B, T, H, dtype=torch.float32, device=dev),
+               ds0=torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev))
+    _check_cuda(q, k, v, g, beta, state_in, d_out, d_state_out)
+    if q.dtype != torch.bfloat16:
+        raise ValueError("q, k, v must be bf16")
+    rc = load().gdn_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in),
+                              _ptr(d_out), _ptr(d_state_out), _ptr(out["dq"]), _ptr(out["dk"]),
+                              _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]), _ptr(out["ds0"]),
+                              B, T, H, dk, dv, gate, _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_chunk_bwd")
     return out
 
 

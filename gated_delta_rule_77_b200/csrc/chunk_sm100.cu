@@ -841,41 +841,6 @@ bool make_map(CUtensorMap* map, const void* base, int H, int T, int B) {
     return r == CUDA_SUCCESS;
 }
 
-// Stream-ordered workspace from a memory pool owned by this library, one per
-// device, that keeps its memory between calls (release threshold: no limit).
-// The device's default pool returns its memory to the system at every
-// synchronisation unless its owner configured it otherwise, and mapping it
-// again on the next call cost milliseconds.  Held: the largest workspace in
-// use at once.
-cudaError_t workspace_alloc(void** ptr, size_t bytes, cudaStream_t stream) {
-    static std::mutex mu;
-    static cudaMemPool_t pools[64] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    {
-        std::lock_guard<std::mutex> lock(mu);
-        if (!pools[dev]) {
-            cudaMemPoolProps props = {};
-            props.allocType = cudaMemAllocationTypePinned;
-            props.location.type = cudaMemLocationTypeDevice;
-            props.location.id = dev;
-            cudaMemPool_t pool = nullptr;
-            e = cudaMemPoolCreate(&pool, &props);
-            if (e != cudaSuccess) return e;
-            cuuint64_t keep = ~cuuint64_t(0);
-            e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
-            if (e != cudaSuccess) {
-                cudaMemPoolDestroy(pool);
-                return e;
-            }
-            pools[dev] = pool;
-        }
-    }
-    return cudaMallocFromPoolAsync(ptr, bytes, pools[dev], stream);
-}
-
 // Serial combine of the segments' affine state maps, for one (batch, head)
 // and a 32-column slice of the state:
 //     S_start(0) = S0,   S_start(s + 1) = M_s S_start(s) + S_end(0)(s).
@@ -1100,6 +1065,41 @@ cudaError_t launch_noalloc(const Problem& p, cudaStream_t stream, bool* over_lim
 }
 
 }  // namespace
+
+// Stream-ordered workspace from a memory pool owned by this library, one per
+// device, that keeps its memory between calls (release threshold: no limit).
+// The device's default pool returns its memory to the system at every
+// synchronisation unless its owner configured it otherwise, and mapping it
+// again on the next call cost milliseconds.  Held: the largest workspace in
+// use at once.
+cudaError_t workspace_alloc(void** ptr, size_t bytes, cudaStream_t stream) {
+    static std::mutex mu;
+    static cudaMemPool_t pools[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!pools[dev]) {
+            cudaMemPoolProps props = {};
+            props.allocType = cudaMemAllocationTypePinned;
+            props.location.type = cudaMemLocationTypeDevice;
+            props.location.id = dev;
+            cudaMemPool_t pool = nullptr;
+            e = cudaMemPoolCreate(&pool, &props);
+            if (e != cudaSuccess) return e;
+            cuuint64_t keep = ~cuuint64_t(0);
+            e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+            if (e != cudaSuccess) {
+                cudaMemPoolDestroy(pool);
+                return e;
+            }
+            pools[dev] = pool;
+        }
+    }
+    return cudaMallocFromPoolAsync(ptr, bytes, pools[dev], stream);
+}
 
 cudaError_t launch_chunk_sm100_noalloc(const Problem& p, cudaStream_t stream, bool* over_limit) {
     *over_limit = false;

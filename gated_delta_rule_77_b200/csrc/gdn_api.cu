@@ -348,6 +348,54 @@ int gdn_state_select(const float* snapshots, const int* num_accepted, float* sta
                                               reinterpret_cast<cudaStream_t>(stream_)));
 }
 
+int gdn_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                  const float* state_in, const float* d_out, const float* d_state_out, float* dq,
+                  float* dk, float* dv, float* dg, float* dbeta, float* d_state_in, int B, int T,
+                  int H, int Dk, int Dv, int gate_mode, gdn_stream_t stream_)
+{
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (B < 1 || H < 1 || T < 0 || Dk < 1 || Dv < 1) return GDN_ERR_INVALID_ARG;
+    if (gate_mode != GDN_GATE_SCALAR && gate_mode != GDN_GATE_CHANNEL) return GDN_ERR_INVALID_ARG;
+    if (T > 0 && (!q || !k || !v || !g || !beta || !d_out || !dq || !dk || !dv || !dg || !dbeta))
+        return GDN_ERR_INVALID_ARG;
+    if (!dim_ok(Dk) || !dim_ok(Dv)) return GDN_ERR_UNSUPPORTED;
+    if (B > 65535 || H > 65535 || T > (1L << 30)) return GDN_ERR_UNSUPPORTED;
+    const bool ch = gate_mode == GDN_GATE_CHANNEL;
+    const void* p16[] = {q, k, v, d_out, state_in, d_state_out, dq, dk, dv, d_state_in,
+                         ch ? (const void*)g : nullptr, ch ? (const void*)dg : nullptr};
+    for (const void* ptr : p16)
+        if (ptr && !aligned16(ptr)) return GDN_ERR_MISALIGNED;
+    for (const void* ptr : {(const void*)g, (const void*)beta, (const void*)dg, (const void*)dbeta})
+        if (ptr && (reinterpret_cast<uintptr_t>(ptr) & 3u)) return GDN_ERR_MISALIGNED;
+    const size_t tok = (size_t)B * T * H;
+    const size_t st = (size_t)B * H * Dk * Dv * 4;
+    const size_t gw = ch ? (size_t)Dk : 1;
+    const Range in[] = {range_of(q, tok * Dk * 2), range_of(k, tok * Dk * 2), range_of(v, tok * Dv * 2),
+                        range_of(g, tok * gw * 4), range_of(beta, tok * 4), range_of(d_out, tok * Dv * 4),
+                        state_in ? range_of(state_in, st) : Range{0, 0},
+                        d_state_out ? range_of(d_state_out, st) : Range{0, 0}};
+    const Range out[] = {range_of(dq, tok * Dk * 4), range_of(dk, tok * Dk * 4), range_of(dv, tok * Dv * 4),
+                         range_of(dg, tok * gw * 4), range_of(dbeta, tok * 4),
+                         d_state_in ? range_of(d_state_in, st) : Range{0, 0}};
+    for (int i = 0; i < 6; ++i) {
+        for (Range r : in)
+            if (overlaps(out[i], r)) return GDN_ERR_INVALID_ARG;
+        for (int j = 0; j < i; ++j)
+            if (overlaps(out[i], out[j])) return GDN_ERR_INVALID_ARG;
+    }
+    if (T == 0) {   // the state passes through unchanged
+        if (!d_state_in) return GDN_OK;
+        cudaError_t e = d_state_out ? cudaMemcpyAsync(d_state_in, d_state_out, st, cudaMemcpyDeviceToDevice, stream)
+                                    : cudaMemsetAsync(d_state_in, 0, st, stream);
+        return to_status(e);
+    }
+    gdn::BwdProblem p{static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                      static_cast<const __nv_bfloat16*>(v), g, beta, state_in, d_out, d_state_out,
+                      dq, dk, dv, dg, dbeta, d_state_in, B, T, H, Dk, Dv, ch};
+    cudaError_t e = gdn::launch_chunk_bwd(p, stream);
+    return e == cudaErrorNotSupported ? GDN_ERR_UNSUPPORTED : to_status(e);
+}
+
 int gdn_check(gdn_stream_t stream_)
 {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);

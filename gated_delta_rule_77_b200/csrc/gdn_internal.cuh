@@ -37,6 +37,32 @@ cudaError_t launch_recurrent(const Problem& p, cudaStream_t stream);
 cudaError_t launch_state_select(const float* snapshots, const int* num_accepted, float* state_out,
                                 int B, int T, int H, int dk, int dv, cudaStream_t stream);
 
+// Gradients of the chunkwise recurrence (chunk_bwd.cu).  bf16 q, k, v; fp32
+// everything else; gradients in fp32.
+struct BwdProblem {
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* k;
+    const __nv_bfloat16* v;
+    const float* g;
+    const float* beta;
+    const float* state_in;      // may be null (zero)
+    const float* d_out;         // [B, T, H, dv]
+    const float* d_state_out;   // [B, H, dk, dv] or null (zero)
+    float* dq;
+    float* dk;
+    float* dv;
+    float* dg;
+    float* dbeta;
+    float* d_state_in;          // may be null (not written)
+    int B, T, H, Dk, Dv;
+    bool per_channel;
+};
+cudaError_t launch_chunk_bwd(const BwdProblem& p, cudaStream_t stream);
+
+// Stream-ordered scratch from the library's per-device memory pool (freed
+// with cudaFreeAsync on the same stream).
+cudaError_t workspace_alloc(void** ptr, size_t bytes, cudaStream_t stream);
+
 // Chunkwise tensor-core prefill (bf16 I/O, dk = dv = 128, chunk of 64).
 // Returns cudaErrorNotSupported for shapes it does not handle.
 cudaError_t launch_chunk_sm100(const Problem& p, cudaStream_t stream);

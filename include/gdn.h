@@ -199,6 +199,34 @@ GDN_API int gdn_recurrent_step_ex(const void* q, const void* k, const void* v, c
                           int io_dtype, gdn_stream_t stream);
 
 /*
+ * gdn_chunk_bwd -- gradients of the chunkwise prefill (training).
+ *
+ * For the loss sum(d_out * out) + sum(d_state_out * state_out) of the call
+ * gdn_chunk_fwd(q, k, v, g, beta, state_in) -> (out, state_out), writes the
+ * gradients of every input.  The forward is recomputed inside (chunks of 32
+ * tokens: the start state of every chunk, then the state gradient backward
+ * over the chunks, then each chunk's token gradients in parallel), in fp32.
+ * Reverse mode of the model card's recurrence (section 2.1) in its chunkwise
+ * form; the gate enters through a = exp(g) as in the forward.
+ *
+ *   q, k, v, g, beta, state_in  as gdn_chunk_fwd (bf16 q, k, v; per-channel
+ *               g in [-5, 0]; state_in may be NULL = zero)
+ *   d_out       [B, T, H, dv] fp32
+ *   d_state_out [B, H, dk, dv] fp32, or NULL (zero)
+ *   dq, dk      [B, T, H, dk] fp32;  dv [B, T, H, dv] fp32
+ *   dg          g's shape, fp32;  dbeta [B, T, H] fp32
+ *   d_state_in  [B, H, dk, dv] fp32, or NULL (not written)
+ *   No output may overlap an input or another output.  Scratch: about
+ *   (T / 32) * B * H * (2 dk dv + 3 * 32 dk + 32 dv + 32^2 + dk) * 4 bytes,
+ *   stream-ordered from the library's pool.
+ */
+GDN_API int gdn_chunk_bwd(const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, const float* state_in, const float* d_out,
+                          const float* d_state_out, float* dq, float* dk, float* dv, float* dg,
+                          float* dbeta, float* d_state_in, int B, int T, int H, int Dk, int Dv,
+                          int gate_mode, gdn_stream_t stream);
+
+/*
  * gdn_recurrent_steps -- T successive tokens per sequence through the decode
  * kernel (speculative verification of T draft tokens; the fused recurrent
  * mode of the "Gated DeltaNet" entity trail, finding of 2026-07-29), with the

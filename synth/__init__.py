@@ -179,3 +179,13 @@ def prologue_inputs(B, T, H, dk, dv, *, gate="channel", ring=True, pos0_max=1000
     return dict(q_raw=q.contiguous(), k_raw=k.contiguous(), v_raw=v.contiguous(), g_raw=g.contiguous(),
                 beta_raw=beta.contiguous(), conv_w=w.contiguous(), ring=r, pos0=pos0)
 
+
+def grad_inputs(B, T, H, dk, dv, *, seed=0, d_state=True):
+    """Incoming gradients of a prefill call: d_out [B, T, H, dv] ~ N(0, 1) and
+    d_state_out [B, H, dk, dv] ~ N(0, 1) (or None), fp32, drawn in that order
+    from ``manual_seed(seed)``."""
+    gen = torch.Generator().manual_seed(int(seed))
+    d_out = _randn_sliced(gen, (B,), T, (H, dv), 1)
+    ds = torch.randn(B, H, dk, dv, generator=gen) if d_state else None
+    return d_out.contiguous(), ds
+

@@ -220,3 +220,29 @@ def _select(lib, snap=A, nacc=A + 300 * MB, state=A + 320 * MB, B=2, T=4, H=2, d
 ])
 def test_state_select_rejects(lib, kw, status):
     assert _select(lib, **kw) == status
+
+
+def _bwd(lib, q=A, k=A + 64 * MB, v=A + 128 * MB, g=A + 192 * MB, beta=A + 256 * MB, s_in=None,
+         do=A + 320 * MB, ds_out=None, dq=A + 512 * MB, dk=A + 576 * MB, dv=A + 640 * MB,
+         dg=A + 704 * MB, dbeta=A + 768 * MB, ds_in=None, B=1, T=16, H=1, Dk=128, Dv=128, gate=1):
+    c = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    return lib.gdn_chunk_bwd(c(q), c(k), c(v), c(g), c(beta), c(s_in), c(do), c(ds_out), c(dq), c(dk),
+                             c(dv), c(dg), c(dbeta), c(ds_in), B, T, H, Dk, Dv, gate, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(do=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dg=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(T=-1), gdn.GDN_ERR_INVALID_ARG),
+    (dict(gate=7), gdn.GDN_ERR_INVALID_ARG),
+    (dict(Dk=48), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(H=70000), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(do=A + 320 * MB + 4), gdn.GDN_ERR_MISALIGNED),
+    (dict(dg=A + 704 * MB + 4), gdn.GDN_ERR_MISALIGNED),          # per-channel dg: 16 bytes
+    (dict(dq=A + 64), gdn.GDN_ERR_INVALID_ARG),                   # dq overlaps q
+    (dict(dv=A + 576 * MB + 32), gdn.GDN_ERR_INVALID_ARG),        # dv overlaps dk
+    (dict(ds_in=A + 320 * MB), gdn.GDN_ERR_INVALID_ARG),          # d_state_in overlaps d_out
+])
+def test_chunk_bwd_rejects(lib, kw, status):
+    assert _bwd(lib, **kw) == status
