@@ -388,6 +388,7 @@ def run_ours(args, rank: int, world: int, local: int):
     decode = run_decode(gdn, dev, stream, peaks, world, rank)
     prologue = run_prologue(gdn, dev, stream, peaks, world, rank)
     multitoken = run_multitoken(gdn, dev, stream, peaks, world, rank)
+    backward = run_backward(gdn, dev, stream, peaks, world, rank)
 
     line = None
     if rank == 0:
@@ -405,7 +406,7 @@ def run_ours(args, rank: int, world: int, local: int):
                 "data": "synthetic", "config": workload_config(cfg), "roofline": roofline,
                 "tensor": tensor, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": args.steps, "clocks": clk.summary(), "decode": decode,
-                "prologue": prologue, "multi_token_decode": multitoken}
+                "prologue": prologue, "multi_token_decode": multitoken, "backward": backward}
         print(json.dumps(line))
     return 0
 
@@ -483,6 +484,52 @@ def run_prologue(gdn, dev, stream, peaks, world, rank, steps: int = 20, warmup: 
                                     "B": dc.B, "H": dc.H, "dk": dc.dk, "dv": dc.dv,
                                     "gate": dc.gate, "l2": "evicted before every timed step"}},
         "timing": f"median of {steps} single-launch CUDA-event timings each"}
+
+
+def backward_flops(cfg, C: int = 32) -> float:
+    """fp32 multiply-adds x 2 of the chunkwise backward per launch, counted
+    from its products per 32-token chunk: 10 C dk dv (state-sized products in
+    the two chains and the gradient pass) + C^2 (9 dk + 7 dv) (chunk-local
+    products), plus the C^3 / 3 solve twice."""
+    n_chunks = cfg.B * cfg.H * -(-cfg.T // C)
+    macs = 10 * C * cfg.dk * cfg.dv + C * C * (9 * cfg.dk + 7 * cfg.dv) + 2 * C ** 3 / 3
+    return 2.0 * macs * n_chunks
+
+
+def run_backward(gdn, dev, stream, peaks, world, rank, steps: int = 10, warmup: int = 3):
+    """gdn_chunk_bwd on the GDN-2 layer shape.  Its products run on the
+    tensor cores (mma.sync, bf16 operands split hi + lo, three passes), so
+    the roofline is the measured dense bf16 peak, against the algorithmic
+    flops of one pass."""
+    from synth import grad_inputs, prefill_inputs
+    cfg = PREFILL_CFG
+    x = prefill_inputs(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, gate=cfg.gate, s0_std=0.1,
+                       seed=cfg.index + 1000 * rank)
+    do, dsT = grad_inputs(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, seed=cfg.index + 1000 * rank)
+    d = {n: x[n].to(dev) for n in ("q", "k", "v", "g", "beta", "s0")}
+    do, dsT = do.to(dev), dsT.to(dev)
+    times = []
+    for i in range(warmup + steps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        gdn.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["s0"], do, dsT, stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= warmup:
+            times.append(e0.elapsed_time(e1) / 1e3)
+    t = max_over_ranks(statistics.median(times), world)
+    fl = backward_flops(cfg)
+    peak = peaks["bf16_tflops"]
+    return {"metric": "prefill backward tokens/s", "value": cfg.B * cfg.T * world / t,
+            "unit": "tokens/s", "ms_per_call": t * 1e3,
+            "roofline": {"bound": "tensor", "achieved": fl / t / 1e12, "peak": peak,
+                         "unit": "TFLOP/s", "frac": fl / t / 1e12 / peak, "flops_per_call": fl,
+                         "peak_source": peaks["source"]},
+            "config": {"workload": "GDN-2 layer prefill gradients (dq, dk, dv, dg, dbeta, dS0)",
+                       "B": cfg.B, "H": cfg.H, "T": cfg.T, "dk": cfg.dk, "dv": cfg.dv,
+                       "gate": cfg.gate, "chunk": 32},
+            "timing": f"median of {steps} single-call CUDA-event timings"}
 
 
 def run_multitoken(gdn, dev, stream, peaks, world, rank, T: int = 4, steps: int = 20,

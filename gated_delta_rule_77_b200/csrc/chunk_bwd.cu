@@ -58,39 +58,78 @@ namespace {
 constexpr int BC = 32;          // chunk length
 constexpr int BM = 16;          // reference token of the per-channel decay
 constexpr int BNT = 256;        // threads per CTA
-constexpr int CP = BC + 1;      // padded row length of a C x C matrix
+constexpr int CP = BC + 4;      // padded row of a C x C tile (4 mod 32: see wmm)
 
-// out(r, c) for r < 32, c < N: warp w owns rows 4w .. 4w+3, lane l the
-// columns l, l + 32, ..., so that a row-major B operand is read by
-// consecutive lanes and a transposed one (row stride = 1 mod 32) without
-// bank conflicts; the A operand is one address per warp (a broadcast).
-template <int N, int K, typename FA, typename FB>
-__device__ __forceinline__ void mm32(float (&acc)[4][N / 32], FA a, FB b) {
-    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-#pragma unroll 4
-    for (int kk = 0; kk < K; ++kk) {
-        float av[4], bv[N / 32];
+// Products on the tensor cores with mma.sync m16n8k16 (bf16 in, fp32
+// accumulate).  Every fp32 operand is split as x = hi + lo with hi, lo in
+// bf16 (16 significant bits together) and a product is hi*hi + hi*lo + lo*hi,
+// about 2^-16 relative: fp32-grade for these gradients.
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 r = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&r);
+}
+
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+                 "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// acc[j] += A[rb .. rb+15][0 .. K) * B[0 .. K)[cb + 8j .. cb + 8j + 7] for one
+// warp, through element accessors a(r, k) and b(k, n).  Fragment layout of
+// m16n8k16 (g = lane / 4, t = lane % 4): A rows g and g + 8, columns 2t, 2t+1
+// and 2t+8, 2t+9; B columns n = g, rows 2t, 2t+1, 2t+8, 2t+9; the result
+// acc[j][e] sits at row rb + g + 8 (e / 2), column cb + 8j + 2t + e % 2.
+// With fp32 tiles of row stride 4 mod 32 the B reads of a row-major tile
+// (bank 8t + g) are conflict-free and the others at most 2-way.
+template <int NT, int K, typename FA, typename FB>
+__device__ __forceinline__ void wmm(float (&acc)[NT][4], int rb, int cb, FA a, FB b) {
+    const int l = threadIdx.x & 31, g = l >> 2, t = l & 3;
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 16) {
+        uint32_t ah[4], al[4];
+        split2(a(rb + g, k0 + 2 * t), a(rb + g, k0 + 2 * t + 1), ah[0], al[0]);
+        split2(a(rb + g + 8, k0 + 2 * t), a(rb + g + 8, k0 + 2 * t + 1), ah[1], al[1]);
+        split2(a(rb + g, k0 + 2 * t + 8), a(rb + g, k0 + 2 * t + 9), ah[2], al[2]);
+        split2(a(rb + g + 8, k0 + 2 * t + 8), a(rb + g + 8, k0 + 2 * t + 9), ah[3], al[3]);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) av[i] = a(4 * w + i, kk);
-#pragma unroll
-        for (int j = 0; j < N / 32; ++j) bv[j] = b(kk, l + 32 * j);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < N / 32; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        for (int j = 0; j < NT; ++j) {
+            const int n = cb + 8 * j + g;
+            uint32_t bh0, bl0, bh1, bl1;
+            split2(b(k0 + 2 * t, n), b(k0 + 2 * t + 1, n), bh0, bl0);
+            split2(b(k0 + 2 * t + 8, n), b(k0 + 2 * t + 9, n), bh1, bl1);
+            mma16816(acc[j], ah, bh0, bh1);
+            mma16816(acc[j], ah, bl0, bl1);
+            mma16816(acc[j], al, bh0, bh1);
+        }
     }
 }
 
-template <int N>
-__device__ __forceinline__ void zero4(float (&acc)[4][N]) {
+template <int NT>
+__device__ __forceinline__ void zero_acc(float (&acc)[NT][4]) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int j = 0; j < NT; ++j)
 #pragma unroll
-        for (int j = 0; j < N; ++j) acc[i][j] = 0.f;
+        for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
 }
 
+// The 32 x N outputs of a chunk are split over the 8 warps as 2 x 4 blocks
+// of 16 rows x N/4 columns (N/32 tiles of 8 columns per warp).
+template <int N>
+struct Tile32 {
+    static constexpr int NT = N / 32;
+    int rb, cb;
+    __device__ Tile32() : rb(((threadIdx.x >> 5) >> 2) * 16), cb(((threadIdx.x >> 5) & 3) * (N / 4)) {}
+    __device__ int row(int e) const { return rb + ((threadIdx.x & 31) >> 2) + 8 * (e >> 1); }
+    __device__ int col(int j, int e) const { return cb + 8 * j + 2 * (threadIdx.x & 3) + (e & 1); }
+};
+
 // Scratch of one (b, h, chunk) for the chains (fp32): W, Kh, Qt [C][DK],
-// Ut [C][DV], P [C][C], E_last [DK].
+// Ut [C][DV], P [C][C], E_last [DK].  Every part starts on a 16-byte boundary.
 template <int DK, int DV>
 struct ChunkScratch {
     static constexpr long kW = 0;
@@ -103,10 +142,10 @@ struct ChunkScratch {
 };
 
 // Shared-memory tiles of the chunk-local part common to the prep and the
-// gradient kernels.
+// gradient kernels.  Rows of fp32 tiles are padded to 4 mod 32 floats.
 template <int DK, int CHANNEL>
-struct Local {
-    static constexpr int KP = DK + 1;            // padded row of a C x DK tile
+struct __align__(16) Local {
+    static constexpr int KP = DK + 4;
     float KL[BC][KP];      // channel: L (.) K ; scalar: K
     float KR[BC][KP];      // channel: R (.) K ; scalar: K
     float QL[BC][KP];      // channel: L (.) Q ; scalar: Q
@@ -128,20 +167,28 @@ __device__ void chunk_local(Local<DK, CHANNEL>& s, const __nv_bfloat16* __restri
                             const float* __restrict__ beta, int b, int h, int t0, int T, int H)
 {
     const int tid = threadIdx.x;
-    for (int idx = tid; idx < BC * DK; idx += BNT) {
-        const int r = idx / DK, c = idx % DK;
+    constexpr int IL = BC * DK / 2 / BNT;    // pairs of channels per thread
+    float2 kv[IL], qv[IL], gv[IL];
+#pragma unroll
+    for (int it = 0; it < IL; ++it) {        // every load first
+        const int idx = tid + it * BNT;
+        const int r = idx / (DK / 2), c = 2 * (idx % (DK / 2));
         const int t = t0 + r;
-        float kv = 0.f, qv = 0.f;
+        kv[it] = qv[it] = gv[it] = make_float2(0.f, 0.f);
         if (t < T) {
             const long tok = ((long)b * T + t) * H + h;
-            kv = __bfloat162float(k[tok * DK + c]);
-            qv = __bfloat162float(q[tok * DK + c]);
-            if (CHANNEL) s.Gam[r][c] = g[tok * DK + c];
-        } else if (CHANNEL) {
-            s.Gam[r][c] = 0.f;
+            kv[it] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(k + tok * DK + c));
+            qv[it] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(q + tok * DK + c));
+            if (CHANNEL) gv[it] = *reinterpret_cast<const float2*>(g + tok * DK + c);
         }
-        s.KL[r][c] = kv;
-        s.QL[r][c] = qv;
+    }
+#pragma unroll
+    for (int it = 0; it < IL; ++it) {
+        const int idx = tid + it * BNT;
+        const int r = idx / (DK / 2), c = 2 * (idx % (DK / 2));
+        s.KL[r][c] = kv[it].x; s.KL[r][c + 1] = kv[it].y;
+        s.QL[r][c] = qv[it].x; s.QL[r][c + 1] = qv[it].y;
+        if (CHANNEL) { s.Gam[r][c] = gv[it].x; s.Gam[r][c + 1] = gv[it].y; }
     }
     if (tid < BC) {
         const int t = t0 + tid;
@@ -186,20 +233,20 @@ __device__ void chunk_local(Local<DK, CHANNEL>& s, const __nv_bfloat16* __restri
     __syncthreads();
     // Abar = KL KR^T (strictly lower), P = QL KR^T (lower), decay applied.
     {
-        float aa[4][1], pp[4][1];
-        zero4(aa);
-        zero4(pp);
-        mm32<BC, DK>(aa, [&](int r, int kk) { return s.KL[r][kk]; },
-                     [&](int kk, int j) { return s.KR[j][kk]; });
-        mm32<BC, DK>(pp, [&](int r, int kk) { return s.QL[r][kk]; },
-                     [&](int kk, int j) { return s.KR[j][kk]; });
-        const int w = tid >> 5, j = tid & 31;
+        const Tile32<BC> tl;
+        float aa[1][4], pp[1][4];
+        zero_acc(aa);
+        zero_acc(pp);
+        wmm<1, DK>(aa, tl.rb, tl.cb, [&](int r, int kk) { return s.KL[r][kk]; },
+                   [&](int kk, int j) { return s.KR[j][kk]; });
+        wmm<1, DK>(pp, tl.rb, tl.cb, [&](int r, int kk) { return s.QL[r][kk]; },
+                   [&](int kk, int j) { return s.KR[j][kk]; });
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = 4 * w + i;
+        for (int e = 0; e < 4; ++e) {
+            const int r = tl.row(e), j = tl.col(0, e);
             const float dec = CHANNEL ? 1.f : s.D[r][j];
-            s.Abar[r][j] = j < r ? aa[i][0] * dec : 0.f;
-            s.P[r][j] = j <= r ? pp[i][0] * dec : 0.f;
+            s.Abar[r][j] = j < r ? aa[0][e] * dec : 0.f;
+            s.P[r][j] = j <= r ? pp[0][e] * dec : 0.f;
         }
     }
     __syncthreads();
@@ -233,50 +280,49 @@ bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     using L = Local<DK, CHANNEL>;
     using SC = ChunkScratch<DK, DV>;
     L& s = *reinterpret_cast<L*>(smem_raw);
-    float (*sV)[DV + 1] = reinterpret_cast<float (*)[DV + 1]>(smem_raw + sizeof(L));
+    float (*sV)[DV + 4] = reinterpret_cast<float (*)[DV + 4]>(smem_raw + sizeof(L));
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t0 = c * BC, tid = threadIdx.x;
-    for (int idx = tid; idx < BC * DV; idx += BNT) {
-        const int r = idx / DV, j = idx % DV;
+    for (int idx = tid; idx < BC * DV / 2; idx += BNT) {
+        const int r = idx / (DV / 2), j = 2 * (idx % (DV / 2));
         const int t = t0 + r;
-        sV[r][j] = t < T ? __bfloat162float(v[(((long)b * T + t) * H + h) * DV + j]) : 0.f;
+        float2 x = make_float2(0.f, 0.f);
+        if (t < T)
+            x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(v + (((long)b * T + t) * H + h) * DV + j));
+        sV[r][j] = x.x;
+        sV[r][j + 1] = x.y;
     }
     chunk_local<DK, CHANNEL>(s, q, k, g, beta, b, h, t0, T, H);
     float* out = scratch + (((long)b * H + h) * N + c) * SC::kSize;
-
-    // Kt = E (.) K and Qt = E (.) Q, Kh = exp(G_last - G) (.) K.
-    auto e_of = [&](int r, int cc) -> float {   // E_rc = exp(G_rc)
-        return CHANNEL ? expf(s.Gam[r][cc]) : expf(s.Gam[r][0]);
-    };
-    const int w = tid >> 5, l = tid & 31;
-    {
-        float acc[4][DK / 32];
-        zero4(acc);
-        if (CHANNEL) {
-            mm32<DK, BC>(acc, [&](int r, int j) { return s.Tm[r][j] * s.beta[j]; },
-                         [&](int j, int cc) { return s.KL[j][cc]; });
-        } else {
-            mm32<DK, BC>(acc, [&](int r, int j) { return s.Tm[r][j] * s.beta[j] * expf(s.Gam[j][0]); },
-                         [&](int j, int cc) { return s.KL[j][cc]; });
-        }
+    {   // W = T Diag(b) Kt, Kt = E (.) K (channel: (L (.) K) E_m)
+        const Tile32<DK> tl;
+        float acc[DK / 32][4];
+        zero_acc(acc);
+        if (CHANNEL)
+            wmm<DK / 32, BC>(acc, tl.rb, tl.cb, [&](int r, int j) { return s.Tm[r][j] * s.beta[j]; },
+                             [&](int j, int cc) { return s.KL[j][cc]; });
+        else
+            wmm<DK / 32, BC>(acc, tl.rb, tl.cb,
+                             [&](int r, int j) { return s.Tm[r][j] * s.beta[j] * expf(s.Gam[j][0]); },
+                             [&](int j, int cc) { return s.KL[j][cc]; });
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int j = 0; j < DK / 32; ++j)
 #pragma unroll
-            for (int jj = 0; jj < DK / 32; ++jj) {
-                const int r = 4 * w + i, cc = l + 32 * jj;
-                // channel: W = T Diag(b) (L (.) K) scaled by E_m per channel
-                out[SC::kW + r * DK + cc] = CHANNEL ? acc[i][jj] * expf(s.Gm[cc]) : acc[i][jj];
+            for (int e = 0; e < 4; ++e) {
+                const int r = tl.row(e), cc = tl.col(j, e);
+                out[SC::kW + r * DK + cc] = CHANNEL ? acc[j][e] * expf(s.Gm[cc]) : acc[j][e];
             }
     }
-    {
-        float acc[4][DV / 32];
-        zero4(acc);
-        mm32<DV, BC>(acc, [&](int r, int j) { return s.Tm[r][j] * s.beta[j]; },
-                     [&](int j, int cc) { return sV[j][cc]; });
+    {   // Ut = T Diag(b) V
+        const Tile32<DV> tl;
+        float acc[DV / 32][4];
+        zero_acc(acc);
+        wmm<DV / 32, BC>(acc, tl.rb, tl.cb, [&](int r, int j) { return s.Tm[r][j] * s.beta[j]; },
+                         [&](int j, int cc) { return sV[j][cc]; });
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int j = 0; j < DV / 32; ++j)
 #pragma unroll
-            for (int jj = 0; jj < DV / 32; ++jj) out[SC::kUt + (4 * w + i) * DV + l + 32 * jj] = acc[i][jj];
+            for (int e = 0; e < 4; ++e) out[SC::kUt + tl.row(e) * DV + tl.col(j, e)] = acc[j][e];
     }
     for (int idx = tid; idx < BC * DK; idx += BNT) {
         const int r = idx / DK, cc = idx % DK;
@@ -286,7 +332,7 @@ bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
             qt = s.QL[r][cc] * expf(s.Gm[cc]);
         } else {
             kh = s.KL[r][cc] * expf(s.Gl[0] - s.Gam[r][0]);
-            qt = s.QL[r][cc] * e_of(r, cc);
+            qt = s.QL[r][cc] * expf(s.Gam[r][0]);
         }
         out[SC::kKh + idx] = kh;
         out[SC::kQt + idx] = qt;
@@ -295,165 +341,226 @@ bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     for (int cc = tid; cc < DK; cc += BNT) out[SC::kEl + cc] = expf(CHANNEL ? s.Gl[cc] : s.Gl[0]);
 }
 
-// Shared memory of the two chains (per 32-column slice of the state).
+// ---------------------------------------------------------------- chains ---
+constexpr int SW = 64;          // value columns per chain CTA
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                 :: "r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Per-chunk operands of a chain, double-buffered.
 template <int DK>
-struct ChainSmem {
-    float W[BC][DK + 1];
-    float Kh[BC][DK + 1];
-    float Qt[BC][DK + 1];
-    float P[BC][CP];
-    float dO[BC][33];
-    float Z[BC][33];
-    float S[DK][33];
+struct __align__(16) ChainBuf {
+    float W[BC][DK + 4];
+    float Kh[BC][DK + 4];
+    float Qt[BC][DK + 4];      // backward chain only
+    float P[BC][CP];           // backward chain only
+    float X[BC][SW + 4];       // Ut slice (forward) or dO slice (backward)
     float El[DK];
 };
+template <int DK>
+struct ChainSmem {
+    ChainBuf<DK> buf[2];
+    float S[DK][SW + 4];       // state (forward) or state gradient (backward) slice
+    float Z[BC][SW + 4];
+};
+
+// Issues the copies of chunk c's operands into a buffer (one commit group).
+// Tokens past T get a zero dO row.
+template <int DK, int DV, bool BACKWARD>
+__device__ void chain_fetch(ChainBuf<DK>& bf, const float* __restrict__ scratch, const float* __restrict__ d_out,
+                            long bh, int c, int N, int col0, int b, int h, int T, int H)
+{
+    using SC = ChunkScratch<DK, DV>;
+    const float* src = scratch + (bh * N + c) * SC::kSize;
+    constexpr int R4 = DK / 4;                       // 16-byte pieces per row
+    for (int idx = threadIdx.x; idx < BC * R4; idx += BNT) {
+        const int r = idx / R4, q4 = 4 * (idx % R4);
+        cp_async16(&bf.W[r][q4], src + SC::kW + r * DK + q4);
+        cp_async16(&bf.Kh[r][q4], src + SC::kKh + r * DK + q4);
+        if (BACKWARD) cp_async16(&bf.Qt[r][q4], src + SC::kQt + r * DK + q4);
+    }
+    if (BACKWARD)
+        for (int idx = threadIdx.x; idx < BC * BC / 4; idx += BNT) {
+            const int r = idx / (BC / 4), q4 = 4 * (idx % (BC / 4));
+            cp_async16(&bf.P[r][q4], src + SC::kP + r * BC + q4);
+        }
+    for (int idx = threadIdx.x; idx < BC * SW / 4; idx += BNT) {
+        const int r = idx / (SW / 4), q4 = 4 * (idx % (SW / 4));
+        if (!BACKWARD) {
+            cp_async16(&bf.X[r][q4], src + SC::kUt + r * DV + col0 + q4);
+        } else {
+            const int t = c * BC + r;
+            if (t < T)
+                cp_async16(&bf.X[r][q4], d_out + (((long)b * T + t) * H + h) * DV + col0 + q4);
+            else
+                *reinterpret_cast<float4*>(&bf.X[r][q4]) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    for (int idx = threadIdx.x; idx < DK / 4; idx += BNT) cp_async16(&bf.El[4 * idx], src + SC::kEl + 4 * idx);
+    cp_async_commit();
+}
+
+// The DK x SW state slice over the 8 warps: DK/16 row blocks x (8 / (DK/16))
+// column groups.
+template <int DK>
+struct TileS {
+    static constexpr int RB = DK / 16, CG = 8 / RB, NT = SW / CG / 8;
+    int rb, cb;
+    __device__ TileS() : rb(((threadIdx.x >> 5) / CG) * 16), cb(((threadIdx.x >> 5) % CG) * (SW / CG)) {}
+    __device__ int row(int e) const { return rb + ((threadIdx.x & 31) >> 2) + 8 * (e >> 1); }
+    __device__ int col(int j, int e) const { return cb + 8 * j + 2 * (threadIdx.x & 3) + (e & 1); }
+};
+
+// Copies the smem slice to [DK][DV] rows at dst (columns col0 ..).
+template <int DK, int DV>
+__device__ __forceinline__ void store_slice(float* __restrict__ dst, const float (*S)[SW + 4], int col0) {
+    for (int idx = threadIdx.x; idx < DK * SW / 4; idx += BNT) {
+        const int r = idx / (SW / 4), q4 = 4 * (idx % (SW / 4));
+        *reinterpret_cast<float4*>(dst + (long)r * DV + col0 + q4) = *reinterpret_cast<const float4*>(&S[r][q4]);
+    }
+}
 
 // Pass 2: chunk start states, forward over the chunks of one (b, h) for a
-// slice of 32 value columns.  grid (DV / 32, H, B).
+// slice of SW value columns.  grid (DV / SW, H, B).
 template <int DK, int DV>
 __global__ void __launch_bounds__(BNT)
 bwd_state_chain_kernel(const float* __restrict__ scratch, const float* __restrict__ state_in,
-                       float* __restrict__ states, int H, int N)
+                       float* __restrict__ states, int T, int H, int N)
 {
-    using SC = ChunkScratch<DK, DV>;
-    constexpr int RW = DK / 8;                     // state rows per warp
     extern __shared__ __align__(16) unsigned char smem_raw[];
     ChainSmem<DK>& cs = *reinterpret_cast<ChainSmem<DK>*>(smem_raw);
-    auto& sW = cs.W;
-    auto& sKh = cs.Kh;
-    auto& sZ = cs.Z;
-    auto& sS = cs.S;
-    auto& sEl = cs.El;
     const int sl = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
-    const int col = sl * 32 + l;
+    const int col0 = sl * SW;
     const long bh = (long)b * H + h;
-    float st[RW];
-#pragma unroll
-    for (int i = 0; i < RW; ++i)
-        st[i] = state_in ? state_in[(bh * DK + RW * w + i) * DV + col] : 0.f;
+    for (int idx = threadIdx.x; idx < DK * SW; idx += BNT) {
+        const int r = idx / SW, j = idx % SW;
+        cs.S[r][j] = state_in ? state_in[(bh * DK + r) * DV + col0 + j] : 0.f;
+    }
+    chain_fetch<DK, DV, false>(cs.buf[0], scratch, nullptr, bh, 0, N, col0, b, h, T, H);
+    const Tile32<SW> tz;
+    const TileS<DK> ts;
     for (int c = 0; c < N; ++c) {
-        const float* src = scratch + (bh * N + c) * SC::kSize;
-        float* dst = states + ((bh * N + c) * DK) * (long)DV;
-#pragma unroll
-        for (int i = 0; i < RW; ++i) {
-            dst[(long)(RW * w + i) * DV + col] = st[i];
-            sS[RW * w + i][l] = st[i];
-        }
-        for (int idx = tid; idx < BC * DK; idx += BNT) {
-            sW[idx / DK][idx % DK] = src[SC::kW + idx];
-            sKh[idx / DK][idx % DK] = src[SC::kKh + idx];
-        }
-        for (int cc = tid; cc < DK; cc += BNT) sEl[cc] = src[SC::kEl + cc];
+        ChainBuf<DK>& bf = cs.buf[c & 1];
+        if (c + 1 < N) chain_fetch<DK, DV, false>(cs.buf[(c + 1) & 1], scratch, nullptr, bh, c + 1, N, col0, b, h, T, H);
+        else cp_async_commit();
+        cp_async_wait1();
         __syncthreads();
-        // Z = Ut - W S  (C x 32)
-        float z[4][1];
-        zero4(z);
-        mm32<32, DK>(z, [&](int r, int kk) { return sW[r][kk]; }, [&](int kk, int j) { return sS[kk][j]; });
+        store_slice<DK, DV>(states + (bh * N + c) * DK * (long)DV, cs.S, col0);
+        {   // Z = Ut - W S
+            float acc[SW / 32][4];
+            zero_acc(acc);
+            wmm<SW / 32, DK>(acc, tz.rb, tz.cb, [&](int r, int kk) { return bf.W[r][kk]; },
+                             [&](int kk, int n) { return cs.S[kk][n]; });
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            sZ[4 * w + i][l] = src[SC::kUt + (4 * w + i) * DV + col] - z[i][0];
+            for (int j = 0; j < SW / 32; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = tz.row(e), n = tz.col(j, e);
+                    cs.Z[r][n] = bf.X[r][n] - acc[j][e];
+                }
+        }
         __syncthreads();
-        // S = Diag(E_last) S + Kh^T Z
+        {   // S = Diag(E_last) S + Kh^T Z
+            float acc[TileS<DK>::NT][4];
+            zero_acc(acc);
+            wmm<TileS<DK>::NT, BC>(acc, ts.rb, ts.cb, [&](int r, int j) { return bf.Kh[j][r]; },
+                                   [&](int j, int n) { return cs.Z[j][n]; });
 #pragma unroll
-        for (int i = 0; i < RW; ++i) {
-            const int r = RW * w + i;
-            float acc = 0.f;
-#pragma unroll 8
-            for (int j = 0; j < BC; ++j) acc = fmaf(sKh[j][r], sZ[j][l], acc);
-            st[i] = fmaf(sEl[r], st[i], acc);
+            for (int j = 0; j < TileS<DK>::NT; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = ts.row(e), n = ts.col(j, e);
+                    cs.S[r][n] = fmaf(bf.El[r], cs.S[r][n], acc[j][e]);
+                }
         }
         __syncthreads();
     }
 }
 
 // Pass 3: dS at every chunk end, backward over the chunks of one (b, h) for
-// a slice of 32 value columns; writes d(state_in).  grid (DV / 32, H, B).
+// a slice of SW value columns; writes d(state_in).  grid (DV / SW, H, B).
 template <int DK, int DV>
 __global__ void __launch_bounds__(BNT)
 bwd_dstate_chain_kernel(const float* __restrict__ scratch, const float* __restrict__ d_out,
                         const float* __restrict__ d_state_out, float* __restrict__ dstates,
                         float* __restrict__ d_state_in, int T, int H, int N)
 {
-    using SC = ChunkScratch<DK, DV>;
-    constexpr int RW = DK / 8;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     ChainSmem<DK>& cs = *reinterpret_cast<ChainSmem<DK>*>(smem_raw);
-    auto& sW = cs.W;
-    auto& sKh = cs.Kh;
-    auto& sQt = cs.Qt;
-    auto& sP = cs.P;
-    auto& sdO = cs.dO;
-    auto& sZ = cs.Z;
-    auto& sS = cs.S;
-    auto& sEl = cs.El;
     const int sl = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
-    const int col = sl * 32 + l;
+    const int col0 = sl * SW;
     const long bh = (long)b * H + h;
-    float ds[RW];
-#pragma unroll
-    for (int i = 0; i < RW; ++i)
-        ds[i] = d_state_out ? d_state_out[(bh * DK + RW * w + i) * DV + col] : 0.f;
+    for (int idx = threadIdx.x; idx < DK * SW; idx += BNT) {
+        const int r = idx / SW, j = idx % SW;
+        cs.S[r][j] = d_state_out ? d_state_out[(bh * DK + r) * DV + col0 + j] : 0.f;
+    }
+    chain_fetch<DK, DV, true>(cs.buf[(N - 1) & 1], scratch, d_out, bh, N - 1, N, col0, b, h, T, H);
+    const Tile32<SW> tz;
+    const TileS<DK> ts;
     for (int c = N - 1; c >= 0; --c) {
-        const float* src = scratch + (bh * N + c) * SC::kSize;
-        float* dst = dstates + ((bh * N + c) * DK) * (long)DV;
+        ChainBuf<DK>& bf = cs.buf[c & 1];
+        if (c > 0) chain_fetch<DK, DV, true>(cs.buf[(c - 1) & 1], scratch, d_out, bh, c - 1, N, col0, b, h, T, H);
+        else cp_async_commit();
+        cp_async_wait1();
+        __syncthreads();
+        store_slice<DK, DV>(dstates + (bh * N + c) * DK * (long)DV, cs.S, col0);
+        {   // Z = Kh dS_next + P^T dO
+            float acc[SW / 32][4];
+            zero_acc(acc);
+            wmm<SW / 32, DK>(acc, tz.rb, tz.cb, [&](int r, int kk) { return bf.Kh[r][kk]; },
+                             [&](int kk, int n) { return cs.S[kk][n]; });
+            wmm<SW / 32, BC>(acc, tz.rb, tz.cb, [&](int r, int j) { return bf.P[j][r]; },
+                             [&](int j, int n) { return bf.X[j][n]; });
 #pragma unroll
-        for (int i = 0; i < RW; ++i) {
-            dst[(long)(RW * w + i) * DV + col] = ds[i];
-            sS[RW * w + i][l] = ds[i];
-        }
-        for (int idx = tid; idx < BC * DK; idx += BNT) {
-            sW[idx / DK][idx % DK] = src[SC::kW + idx];
-            sKh[idx / DK][idx % DK] = src[SC::kKh + idx];
-            sQt[idx / DK][idx % DK] = src[SC::kQt + idx];
-        }
-        for (int idx = tid; idx < BC * BC; idx += BNT) sP[idx / BC][idx % BC] = src[SC::kP + idx];
-        for (int cc = tid; cc < DK; cc += BNT) sEl[cc] = src[SC::kEl + cc];
+            for (int j = 0; j < SW / 32; ++j)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int t = c * BC + 4 * w + i;
-            sdO[4 * w + i][l] = t < T ? d_out[(((long)b * T + t) * H + h) * DV + col] : 0.f;
+                for (int e = 0; e < 4; ++e) cs.Z[tz.row(e)][tz.col(j, e)] = acc[j][e];
         }
         __syncthreads();
-        // Z = Kh dS_next + P^T dO  (C x 32)
-        float z[4][1];
-        zero4(z);
-        mm32<32, DK>(z, [&](int r, int kk) { return sKh[r][kk]; }, [&](int kk, int j) { return sS[kk][j]; });
-        mm32<32, BC>(z, [&](int r, int j) { return sP[j][r]; }, [&](int j, int cc) { return sdO[j][cc]; });
+        {   // dS = Diag(E_last) dS_next + Qt^T dO - W^T Z
+            float acc[TileS<DK>::NT][4];
+            zero_acc(acc);
+            wmm<TileS<DK>::NT, BC>(acc, ts.rb, ts.cb, [&](int r, int j) { return bf.Qt[j][r]; },
+                                   [&](int j, int n) { return bf.X[j][n]; });
+            wmm<TileS<DK>::NT, BC>(acc, ts.rb, ts.cb, [&](int r, int j) { return -bf.W[j][r]; },
+                                   [&](int j, int n) { return cs.Z[j][n]; });
 #pragma unroll
-        for (int i = 0; i < 4; ++i) sZ[4 * w + i][l] = z[i][0];
-        __syncthreads();
-        // dS = Diag(E_last) dS_next + Qt^T dO - W^T Z
+            for (int j = 0; j < TileS<DK>::NT; ++j)
 #pragma unroll
-        for (int i = 0; i < RW; ++i) {
-            const int r = RW * w + i;
-            float acc = 0.f;
-#pragma unroll 8
-            for (int j = 0; j < BC; ++j) acc = fmaf(sQt[j][r], sdO[j][l], fmaf(-sW[j][r], sZ[j][l], acc));
-            ds[i] = fmaf(sEl[r], ds[i], acc);
+                for (int e = 0; e < 4; ++e) {
+                    const int r = ts.row(e), n = ts.col(j, e);
+                    cs.S[r][n] = fmaf(bf.El[r], cs.S[r][n], acc[j][e]);
+                }
         }
         __syncthreads();
     }
     if (d_state_in) {
-#pragma unroll
-        for (int i = 0; i < RW; ++i) d_state_in[(bh * DK + RW * w + i) * DV + col] = ds[i];
+        for (int idx = threadIdx.x; idx < DK * SW; idx += BNT) {
+            const int r = idx / SW, j = idx % SW;
+            d_state_in[(bh * DK + r) * DV + col0 + j] = cs.S[r][j];
+        }
     }
 }
 
-// Shared memory of the gradient kernel beyond the chunk-local tiles.
+// ------------------------------------------------------- token gradients ---
 template <int DK, int DV, int CHANNEL>
-struct GradSmem {
+struct __align__(16) GradSmem {
     Local<DK, CHANNEL> loc;
-    float V[BC][DV + 1];       // v, then E2 = V - Kt S
-    float dO[BC][DV + 1];      // dO, then dU, then Y
-    float U[BC][DV + 1];
-    float Big[DK][DV + 1];     // S, dS_next, S again, then dG [C][DK]
+    float V[BC][DV + 4];       // v, then E2 = V - Kt S
+    float dO[BC][DV + 4];      // dO, then dU, then Y
+    float U[BC][DV + 4];
+    float Big[DK][DV + 4];     // S, dS_next, S again, then dG [C][DK]
     float dP[BC][CP];          // lower(dO U^T), no decay
     float Gm2[BC][CP];         // -strictlower(Y U^T), no decay
     float rowdot[DK];          // rowsum(dS_next (.) S)
-    float last[8][DK];         // per-warp column sums of Kh (.) dKh
+    float last[DK];            // column sums of Kh (.) dKh
     float db[BC];
+    float rowg[BC];            // scalar gate: dG per token
     float eM[CHANNEL ? DK : BC];    // channel: exp(G_m); scalar: E_r = exp(G_r)
     float eH[CHANNEL ? DK : BC];    // channel: exp(G_last - G_m); scalar: exp(G_last - G_r)
 };
@@ -479,15 +586,45 @@ bwd_grads_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     const float* gS = states + n * DK * (long)DV;
     const float* gdS = dstates + n * DK * (long)DV;
     auto tok_of = [&](int r) -> long { return ((long)b * T + t0 + r) * H + h; };
+    constexpr int IT = DK * DV / 4 / BNT;   // 16-byte pieces of a state per thread
+    // Asynchronous copy of a state into Big (one commit group).
+    auto fetch_big = [&](const float* src) {
+#pragma unroll
+        for (int it = 0; it < IT; ++it) {
+            const int idx = tid + it * BNT;
+            const int r = idx / (DV / 4), q4 = 4 * (idx % (DV / 4));
+            cp_async16(&m.Big[r][q4], src + (long)r * DV + q4);
+        }
+        cp_async_commit();
+    };
 
-    for (int idx = tid; idx < BC * DV; idx += BNT) {
-        const int r = idx / DV, j = idx % DV;
-        const bool in = t0 + r < T;
-        m.V[r][j] = in ? __bfloat162float(v[tok_of(r) * DV + j]) : 0.f;
-        m.dO[r][j] = in ? d_out[tok_of(r) * DV + j] : 0.f;
+    fetch_big(gS);
+    {
+        constexpr int IV = BC * DV / 2 / BNT;
+        float2 vv[IV], oo[IV];
+#pragma unroll
+        for (int it = 0; it < IV; ++it) {
+            const int idx = tid + it * BNT;
+            const int r = idx / (DV / 2), j = 2 * (idx % (DV / 2));
+            vv[it] = make_float2(0.f, 0.f);
+            oo[it] = make_float2(0.f, 0.f);
+            if (t0 + r < T) {
+                vv[it] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(v + tok_of(r) * DV + j));
+                oo[it] = *reinterpret_cast<const float2*>(d_out + tok_of(r) * DV + j);
+            }
+        }
+#pragma unroll
+        for (int it = 0; it < IV; ++it) {
+            const int idx = tid + it * BNT;
+            const int r = idx / (DV / 2), j = 2 * (idx % (DV / 2));
+            m.V[r][j] = vv[it].x; m.V[r][j + 1] = vv[it].y;
+            m.dO[r][j] = oo[it].x; m.dO[r][j + 1] = oo[it].y;
+        }
     }
-    for (int idx = tid; idx < DK * DV; idx += BNT) m.Big[idx / DV][idx % DV] = gS[idx];
+    for (int cc = tid; cc < DK; cc += BNT) m.last[cc] = 0.f;
     chunk_local<DK, CHANNEL>(s, q, k, g, beta, b, h, t0, T, H);   // ends with a barrier
+    cp_async_wait0();
+    __syncthreads();
     if (CHANNEL) {
         for (int cc = tid; cc < DK; cc += BNT) {
             m.eM[cc] = expf(s.Gm[cc]);
@@ -499,282 +636,279 @@ bwd_grads_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     }
     __syncthreads();
 
-    // Per-element factors of this thread's outputs (rows 4w + i, columns
-    // l + 32 jj of a C x DK tile).
     auto Kt = [&](int r, int cc) { return CHANNEL ? s.KL[r][cc] * m.eM[cc] : s.KL[r][cc] * m.eM[r]; };
     auto Qt = [&](int r, int cc) { return CHANNEL ? s.QL[r][cc] * m.eM[cc] : s.QL[r][cc] * m.eM[r]; };
     auto Kh = [&](int r, int cc) { return CHANNEL ? s.KR[r][cc] * m.eH[cc] : s.KL[r][cc] * m.eH[r]; };
     auto Eo = [&](int r, int cc) { return CHANNEL ? expf(s.Gam[r][cc]) : m.eM[r]; };
     auto Eho = [&](int r, int cc) { return CHANNEL ? expf(s.Gl[cc] - s.Gam[r][cc]) : m.eH[r]; };
 
-    float dQa[4][NK], dKa[4][NK], dGa[4][NK];
-    zero4(dQa);
-    zero4(dKa);
-    zero4(dGa);
+    const Tile32<DK> tk;     // C x DK outputs: this thread's elements
+    const Tile32<DV> tv;     // C x DV outputs
+    const Tile32<BC> tc;     // C x C outputs
+    float dQa[NK][4], dKa[NK][4], dGa[NK][4];
+    zero_acc(dQa);
+    zero_acc(dKa);
+    zero_acc(dGa);
 
-    // E2 = V - Kt S (in place in V); dQt = dO S^T.
-    {
-        float acc[4][NV];
-        zero4(acc);
-        mm32<DV, DK>(acc, Kt, [&](int kk, int j) { return m.Big[kk][j]; });
+    {   // E2 = V - Kt S (in place in V)
+        float acc[NV][4];
+        zero_acc(acc);
+        wmm<NV, DK>(acc, tv.rb, tv.cb, Kt, [&](int kk, int j) { return m.Big[kk][j]; });
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int j = 0; j < NV; ++j)
 #pragma unroll
-            for (int jj = 0; jj < NV; ++jj) m.V[4 * w + i][l + 32 * jj] -= acc[i][jj];
+            for (int e = 0; e < 4; ++e) m.V[tv.row(e)][tv.col(j, e)] -= acc[j][e];
     }
-    {
-        float acc[4][NK];
-        zero4(acc);
-        mm32<DK, DV>(acc, [&](int r, int j) { return m.dO[r][j]; }, [&](int j, int cc) { return m.Big[cc][j]; });
+    {   // dQt = dO S^T
+        float acc[NK][4];
+        zero_acc(acc);
+        wmm<NK, DV>(acc, tk.rb, tk.cb, [&](int r, int j) { return m.dO[r][j]; },
+                    [&](int j, int cc) { return m.Big[cc][j]; });
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int j = 0; j < NK; ++j)
 #pragma unroll
-            for (int jj = 0; jj < NK; ++jj) {
-                const int r = 4 * w + i, cc = l + 32 * jj;
-                dQa[i][jj] += Eo(r, cc) * acc[i][jj];
-                dGa[i][jj] += Qt(r, cc) * acc[i][jj];
+            for (int e = 0; e < 4; ++e) {
+                const int r = tk.row(e), cc = tk.col(j, e);
+                dQa[j][e] += Eo(r, cc) * acc[j][e];
+                dGa[j][e] += Qt(r, cc) * acc[j][e];
             }
     }
     __syncthreads();
-    // U = T Diag(b) E2.
+    // dS_next replaces S; rowsum(dS_next (.) S) on the way.  Every load is
+    // issued before the first use; piece it of a thread lies in row
+    // (tid + it * BNT) / (DV / 4), so the rows of a warp are reduced by
+    // shuffles once the pieces of a row are summed.
     {
-        float acc[4][NV];
-        zero4(acc);
-        mm32<DV, BC>(acc, [&](int r, int j) { return s.Tm[r][j] * s.beta[j]; },
-                     [&](int j, int cc) { return m.V[j][cc]; });
+        float4 x[IT];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int it = 0; it < IT; ++it) {
+            const int idx = tid + it * BNT;
+            x[it] = *reinterpret_cast<const float4*>(gdS + (long)(idx / (DV / 4)) * DV + 4 * (idx % (DV / 4)));
+        }
 #pragma unroll
-            for (int jj = 0; jj < NV; ++jj) m.U[4 * w + i][l + 32 * jj] = acc[i][jj];
-    }
-    // rowsum(dS_next (.) S), one row per warp at a time.
-    for (int r = w; r < DK; r += 8) {
-        float acc = 0.f;
-        for (int j = l; j < DV; j += 32) acc = fmaf(gdS[(long)r * DV + j], m.Big[r][j], acc);
+        for (int it = 0; it < IT; ++it) {
+            const int idx = tid + it * BNT;
+            const int r = idx / (DV / 4), q4 = 4 * (idx % (DV / 4));
+            float4& sv = *reinterpret_cast<float4*>(&m.Big[r][q4]);
+            float d = x[it].x * sv.x + x[it].y * sv.y + x[it].z * sv.z + x[it].w * sv.w;
+            sv = x[it];
+            // the DV / 4 lanes that share row r are consecutive: reduce over them
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (l == 0) m.rowdot[r] = acc;
+            for (int o = DV / 8; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+            if ((tid % (DV / 4)) == 0) m.rowdot[r] = d;
+        }
     }
     __syncthreads();
-    // dP = lower(dO U^T); dS_next replaces S.
-    {
-        float acc[4][1];
-        zero4(acc);
-        mm32<BC, DV>(acc, [&](int r, int j) { return m.dO[r][j]; }, [&](int j, int jj) { return m.U[jj][j]; });
+    {   // U = T Diag(b) E2
+        float acc[NV][4];
+        zero_acc(acc);
+        wmm<NV, BC>(acc, tv.rb, tv.cb, [&](int r, int j) { return s.Tm[r][j] * s.beta[j]; },
+                    [&](int j, int cc) { return m.V[j][cc]; });
 #pragma unroll
-        for (int i = 0; i < 4; ++i) m.dP[4 * w + i][l] = l <= 4 * w + i ? acc[i][0] : 0.f;
+        for (int j = 0; j < NV; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) m.U[tv.row(e)][tv.col(j, e)] = acc[j][e];
     }
-    for (int idx = tid; idx < DK * DV; idx += BNT) m.Big[idx / DV][idx % DV] = gdS[idx];
     __syncthreads();
-    // dKh = U dS_next^T.
-    {
-        float acc[4][NK];
-        zero4(acc);
-        mm32<DK, DV>(acc, [&](int r, int j) { return m.U[r][j]; }, [&](int j, int cc) { return m.Big[cc][j]; });
+    {   // dP = lower(dO U^T)
+        float acc[1][4];
+        zero_acc(acc);
+        wmm<1, DV>(acc, tc.rb, tc.cb, [&](int r, int j) { return m.dO[r][j]; },
+                   [&](int j, int jj) { return m.U[jj][j]; });
 #pragma unroll
-        for (int jj = 0; jj < NK; ++jj) {
-            const int cc = l + 32 * jj;
-            float colsum = 0.f;
+        for (int e = 0; e < 4; ++e) {
+            const int r = tc.row(e), jj = tc.col(0, e);
+            m.dP[r][jj] = jj <= r ? acc[0][e] : 0.f;
+        }
+    }
+    {   // dKh = U dS_next^T
+        float acc[NK][4];
+        zero_acc(acc);
+        wmm<NK, DV>(acc, tk.rb, tk.cb, [&](int r, int j) { return m.U[r][j]; },
+                    [&](int j, int cc) { return m.Big[cc][j]; });
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = 4 * w + i;
+        for (int j = 0; j < NK; ++j) {
+            float colsum[2] = {0.f, 0.f};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = tk.row(e), cc = tk.col(j, e);
                 const float kh = Kh(r, cc);
-                dKa[i][jj] += Eho(r, cc) * acc[i][jj];
-                dGa[i][jj] -= kh * acc[i][jj];
-                colsum = fmaf(kh, acc[i][jj], colsum);
+                dKa[j][e] += Eho(r, cc) * acc[j][e];
+                dGa[j][e] -= kh * acc[j][e];
+                colsum[e & 1] = fmaf(kh, acc[j][e], colsum[e & 1]);
             }
-            m.last[w][cc] = colsum;
+            atomicAdd(&m.last[tk.col(j, 0)], colsum[0]);
+            atomicAdd(&m.last[tk.col(j, 1)], colsum[1]);
         }
     }
-    // dU = Kh dS_next + P^T dO (into dO once every thread is done with dO).
-    {
-        float acc[4][NV];
-        zero4(acc);
-        mm32<DV, DK>(acc, Kh, [&](int kk, int j) { return m.Big[kk][j]; });
-        mm32<DV, BC>(acc, [&](int r, int j) { return s.P[j][r]; }, [&](int j, int cc) { return m.dO[j][cc]; });
+    {   // dU = Kh dS_next + P^T dO  (into dO once every thread is done with dO)
+        float acc[NV][4];
+        zero_acc(acc);
+        wmm<NV, DK>(acc, tv.rb, tv.cb, Kh, [&](int kk, int j) { return m.Big[kk][j]; });
+        wmm<NV, BC>(acc, tv.rb, tv.cb, [&](int r, int j) { return s.P[j][r]; },
+                    [&](int j, int cc) { return m.dO[j][cc]; });
         __syncthreads();
+        fetch_big(gS);   // S again: dS_next is no longer read
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int j = 0; j < NV; ++j)
 #pragma unroll
-            for (int jj = 0; jj < NV; ++jj) m.dO[4 * w + i][l + 32 * jj] = acc[i][jj];
+            for (int e = 0; e < 4; ++e) m.dO[tv.row(e)][tv.col(j, e)] = acc[j][e];
         __syncthreads();
     }
-    // Y = T^T dU (into dO).
-    {
-        float acc[4][NV];
-        zero4(acc);
-        mm32<DV, BC>(acc, [&](int r, int j) { return s.Tm[j][r]; }, [&](int j, int cc) { return m.dO[j][cc]; });
+    {   // Y = T^T dU (into dO); dV = Diag(b) Y
+        float acc[NV][4];
+        zero_acc(acc);
+        wmm<NV, BC>(acc, tv.rb, tv.cb, [&](int r, int j) { return s.Tm[j][r]; },
+                    [&](int j, int cc) { return m.dO[j][cc]; });
         __syncthreads();
-        float dbp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = 4 * w + i;
+        for (int j = 0; j < NV; ++j)
 #pragma unroll
-            for (int jj = 0; jj < NV; ++jj) {
-                const int cc = l + 32 * jj;
-                m.dO[r][cc] = acc[i][jj];
-                dbp[i] = fmaf(acc[i][jj], m.V[r][cc], dbp[i]);
-                if (t0 + r < T) dv[tok_of(r) * DV + cc] = s.beta[r] * acc[i][jj];
+            for (int e = 0; e < 4; ++e) {
+                const int r = tv.row(e), cc = tv.col(j, e);
+                m.dO[r][cc] = acc[j][e];
+                if (t0 + r < T) dv[tok_of(r) * DV + cc] = s.beta[r] * acc[j][e];
             }
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) dbp[i] += __shfl_xor_sync(0xffffffffu, dbp[i], o);
-            if (l == 0) m.db[4 * w + i] = dbp[i];
-        }
         __syncthreads();
     }
-    // G = -strictlower(Y U^T); db += rowsum(G (.) Abar).  S replaces dS_next.
-    {
-        float acc[4][1];
-        zero4(acc);
-        mm32<BC, DV>(acc, [&](int r, int j) { return m.dO[r][j]; }, [&](int j, int jj) { return m.U[jj][j]; });
+    {   // G = -strictlower(Y U^T)
+        float acc[1][4];
+        zero_acc(acc);
+        wmm<1, DV>(acc, tc.rb, tc.cb, [&](int r, int j) { return m.dO[r][j]; },
+                   [&](int j, int jj) { return m.U[jj][j]; });
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = 4 * w + i;
-            const float gv = l < r ? -acc[i][0] : 0.f;
-            m.Gm2[r][l] = gv;
-            float x = gv * s.Abar[r][l];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-            if (l == 0) m.db[r] += x;
+        for (int e = 0; e < 4; ++e) {
+            const int r = tc.row(e), jj = tc.col(0, e);
+            m.Gm2[r][jj] = jj < r ? -acc[0][e] : 0.f;
         }
     }
     __syncthreads();
-    for (int idx = tid; idx < DK * DV; idx += BNT) m.Big[idx / DV][idx % DV] = gS[idx];
+    // db_r = Y_r . E2_r + sum_j G_rj Abar_rj, one warp per 4 rows.
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = 4 * w + i;
+        float x = m.Gm2[r][l] * s.Abar[r][l];
+        for (int j = l; j < DV; j += 32) x = fmaf(m.dO[r][j], m.V[r][j], x);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        if (l == 0) m.db[r] = x;
+    }
+    cp_async_wait0();
     __syncthreads();
-    // dKt = -Diag(b) Y S^T.
-    {
-        float acc[4][NK];
-        zero4(acc);
-        mm32<DK, DV>(acc, [&](int r, int j) { return -s.beta[r] * m.dO[r][j]; },
-                     [&](int j, int cc) { return m.Big[cc][j]; });
+    {   // dKt = -Diag(b) Y S^T
+        float acc[NK][4];
+        zero_acc(acc);
+        wmm<NK, DV>(acc, tk.rb, tk.cb, [&](int r, int j) { return -s.beta[r] * m.dO[r][j]; },
+                    [&](int j, int cc) { return m.Big[cc][j]; });
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int j = 0; j < NK; ++j)
 #pragma unroll
-            for (int jj = 0; jj < NK; ++jj) {
-                const int r = 4 * w + i, cc = l + 32 * jj;
-                dKa[i][jj] += Eo(r, cc) * acc[i][jj];
-                dGa[i][jj] += Kt(r, cc) * acc[i][jj];
+            for (int e = 0; e < 4; ++e) {
+                const int r = tk.row(e), cc = tk.col(j, e);
+                dKa[j][e] += Eo(r, cc) * acc[j][e];
+                dGa[j][e] += Kt(r, cc) * acc[j][e];
             }
     }
-    // The decay-weighted products of A and P: rows and columns.
+    // The decay-weighted products of A and P, rows and columns.
     auto decay = [&](int r, int j) { return CHANNEL ? 1.f : s.D[r][j]; };
     auto Lf = [&](int r, int cc) { return expf(s.Gam[r][cc] - s.Gm[cc]); };
     {   // t_row = (b G) KR ; t_col = (b G)^T KL
-        float tr[4][NK], tc[4][NK];
-        zero4(tr);
-        zero4(tc);
-        mm32<DK, BC>(tr, [&](int r, int j) { return s.beta[r] * m.Gm2[r][j] * decay(r, j); },
-                     [&](int j, int cc) { return s.KR[j][cc]; });
-        mm32<DK, BC>(tc, [&](int r, int j) { return s.beta[j] * m.Gm2[j][r] * decay(j, r); },
-                     [&](int j, int cc) { return s.KL[j][cc]; });
+        float tr[NK][4], tcl[NK][4];
+        zero_acc(tr);
+        zero_acc(tcl);
+        wmm<NK, BC>(tr, tk.rb, tk.cb, [&](int r, int j) { return s.beta[r] * m.Gm2[r][j] * decay(r, j); },
+                    [&](int j, int cc) { return s.KR[j][cc]; });
+        wmm<NK, BC>(tcl, tk.rb, tk.cb, [&](int r, int j) { return s.beta[j] * m.Gm2[j][r] * decay(j, r); },
+                    [&](int j, int cc) { return s.KL[j][cc]; });
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int j = 0; j < NK; ++j)
 #pragma unroll
-            for (int jj = 0; jj < NK; ++jj) {
-                const int r = 4 * w + i, cc = l + 32 * jj;
+            for (int e = 0; e < 4; ++e) {
+                const int r = tk.row(e), cc = tk.col(j, e);
                 if (CHANNEL) {
                     const float L = Lf(r, cc), R = 1.f / L;
-                    dKa[i][jj] += L * tr[i][jj] + R * tc[i][jj];
-                    dGa[i][jj] += s.KL[r][cc] * tr[i][jj] - s.KR[r][cc] * tc[i][jj];
+                    dKa[j][e] += L * tr[j][e] + R * tcl[j][e];
+                    dGa[j][e] += s.KL[r][cc] * tr[j][e] - s.KR[r][cc] * tcl[j][e];
                 } else {
-                    dKa[i][jj] += tr[i][jj] + tc[i][jj];
+                    dKa[j][e] += tr[j][e] + tcl[j][e];
                 }
             }
     }
     {   // p_row = dP KR ; p_col = dP^T QL
-        float pr[4][NK], pc[4][NK];
-        zero4(pr);
-        zero4(pc);
-        mm32<DK, BC>(pr, [&](int r, int j) { return m.dP[r][j] * decay(r, j); },
-                     [&](int j, int cc) { return s.KR[j][cc]; });
-        mm32<DK, BC>(pc, [&](int r, int j) { return m.dP[j][r] * decay(j, r); },
-                     [&](int j, int cc) { return s.QL[j][cc]; });
+        float pr[NK][4], pc[NK][4];
+        zero_acc(pr);
+        zero_acc(pc);
+        wmm<NK, BC>(pr, tk.rb, tk.cb, [&](int r, int j) { return m.dP[r][j] * decay(r, j); },
+                    [&](int j, int cc) { return s.KR[j][cc]; });
+        wmm<NK, BC>(pc, tk.rb, tk.cb, [&](int r, int j) { return m.dP[j][r] * decay(j, r); },
+                    [&](int j, int cc) { return s.QL[j][cc]; });
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int j = 0; j < NK; ++j)
 #pragma unroll
-            for (int jj = 0; jj < NK; ++jj) {
-                const int r = 4 * w + i, cc = l + 32 * jj;
+            for (int e = 0; e < 4; ++e) {
+                const int r = tk.row(e), cc = tk.col(j, e);
                 if (CHANNEL) {
                     const float L = Lf(r, cc), R = 1.f / L;
-                    dQa[i][jj] += L * pr[i][jj];
-                    dKa[i][jj] += R * pc[i][jj];
-                    dGa[i][jj] += s.QL[r][cc] * pr[i][jj] - s.KR[r][cc] * pc[i][jj];
+                    dQa[j][e] += L * pr[j][e];
+                    dKa[j][e] += R * pc[j][e];
+                    dGa[j][e] += s.QL[r][cc] * pr[j][e] - s.KR[r][cc] * pc[j][e];
                 } else {
-                    dQa[i][jj] += pr[i][jj];
-                    dKa[i][jj] += pc[i][jj];
+                    dQa[j][e] += pr[j][e];
+                    dKa[j][e] += pc[j][e];
                 }
             }
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int r = 4 * w + i;
-        if (t0 + r < T) {
+    for (int j = 0; j < NK; ++j)
 #pragma unroll
-            for (int jj = 0; jj < NK; ++jj) {
-                dq[tok_of(r) * DK + l + 32 * jj] = dQa[i][jj];
-                dk[tok_of(r) * DK + l + 32 * jj] = dKa[i][jj];
+        for (int e = 0; e < 4; e += 2) {     // the two adjacent columns of a row
+            const int r = tk.row(e), cc = tk.col(j, e);
+            if (t0 + r < T) {
+                *reinterpret_cast<float2*>(dq + tok_of(r) * DK + cc) = make_float2(dQa[j][e], dQa[j][e + 1]);
+                *reinterpret_cast<float2*>(dk + tok_of(r) * DK + cc) = make_float2(dKa[j][e], dKa[j][e + 1]);
             }
         }
-    }
     __syncthreads();   // every read of Big (S) is done
-    // dG per token and channel, then the reverse in-chunk cumulative sum.
     float* sdG = &m.Big[0][0];               // [C][DK]
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int j = 0; j < NK; ++j)
 #pragma unroll
-        for (int jj = 0; jj < NK; ++jj) sdG[(4 * w + i) * DK + l + 32 * jj] = dGa[i][jj];
+        for (int e = 0; e < 4; ++e) sdG[tk.row(e) * DK + tk.col(j, e)] = dGa[j][e];
     __syncthreads();
     if (CHANNEL) {
         for (int cc = tid; cc < DK; cc += BNT) {
-            float lastc = 0.f;
-#pragma unroll
-            for (int ww = 0; ww < 8; ++ww) lastc += m.last[ww][cc];
-            float acc = expf(s.Gl[cc]) * m.rowdot[cc] + lastc;   // at the last token
+            float acc = expf(s.Gl[cc]) * m.rowdot[cc] + m.last[cc];   // at the last token
             for (int r = BC - 1; r >= 0; --r) {
                 acc += sdG[r * DK + cc];
                 if (t0 + r < T) dg[tok_of(r) * DK + cc] = acc;
             }
         }
     } else {
-        // Scalar gate: the channel sums of the per-element terms, the row and
+        // Scalar gate: channel sums of the per-element terms, the row minus
         // column sums of (b G) (.) Abar and dP (.) P, and the last-token term.
-        float* rowv = &m.last[0][0];            // reuse: [C] after the sums below
-        __shared__ float s_lastsum;
-        if (w == 0) {
-            float x = 0.f;
-            for (int cc = l; cc < DK; cc += 32) {
-                float lastc = 0.f;
-#pragma unroll
-                for (int ww = 0; ww < 8; ++ww) lastc += m.last[ww][cc];
-                x += expf(s.Gl[0]) * m.rowdot[cc] + lastc;
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-            if (l == 0) s_lastsum = x;
-        }
-        __syncthreads();
-        // One warp per 4 rows: per-element channel sums and the C x C terms.
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int r = 4 * w + i;
             float x = 0.f;
             for (int cc = l; cc < DK; cc += 32) x += sdG[r * DK + cc];
-            const float ga = s.beta[r] * m.Gm2[r][l] * s.Abar[r][l] + m.dP[r][l] * s.P[r][l];
-            const float gb = s.beta[l] * m.Gm2[l][r] * s.Abar[l][r] + m.dP[l][r] * s.P[l][r];
-            x += ga - gb;
+            x += s.beta[r] * m.Gm2[r][l] * s.Abar[r][l] + m.dP[r][l] * s.P[r][l];
+            x -= s.beta[l] * m.Gm2[l][r] * s.Abar[l][r] + m.dP[l][r] * s.P[l][r];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-            if (l == 0) rowv[r] = x;
+            if (l == 0) m.rowg[r] = x;
         }
         __syncthreads();
-        if (tid == 0) {
-            float acc = s_lastsum;
-            for (int r = BC - 1; r >= 0; --r) {
-                acc += rowv[r];
-                if (t0 + r < T) dg[tok_of(r)] = acc;
+        if (w == 0) {
+            float x = 0.f;
+            for (int cc = l; cc < DK; cc += 32) x += expf(s.Gl[0]) * m.rowdot[cc] + m.last[cc];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+            if (l == 0) {
+                float acc = x;
+                for (int r = BC - 1; r >= 0; --r) {
+                    acc += m.rowg[r];
+                    if (t0 + r < T) dg[tok_of(r)] = acc;
+                }
             }
         }
     }
@@ -794,12 +928,13 @@ cudaError_t launch_bwd_t(const BwdProblem& p, cudaStream_t stream) {
     float* scratch = ws;
     float* states = ws + nchunks * SC::kSize;
     float* dstates = states + nchunks * (long)DK * DV;
-    const dim3 grid_c(N, p.H, p.B), grid_s(DV / 32, p.H, p.B);
-    const size_t prep_smem = sizeof(Local<DK, CHANNEL>) + sizeof(float) * BC * (DV + 1);
+    const dim3 grid_c(N, p.H, p.B), grid_s(DV / SW, p.H, p.B);
+    const size_t prep_smem = sizeof(Local<DK, CHANNEL>) + sizeof(float) * BC * (DV + 4);
     const size_t grad_smem = sizeof(GradSmem<DK, DV, CHANNEL>);
     const size_t chain_smem = sizeof(ChainSmem<DK>);
     static_assert(sizeof(GradSmem<DK, DV, CHANNEL>) <= 227 * 1024, "gradient tiles exceed shared memory");
-    static_assert(sizeof(Local<DK, CHANNEL>) + sizeof(float) * BC * (DV + 1) <= 227 * 1024, "prep tiles");
+    static_assert(sizeof(ChainSmem<DK>) <= 227 * 1024, "chain tiles exceed shared memory");
+    static_assert(sizeof(Local<DK, CHANNEL>) % 16 == 0 && sizeof(ChainBuf<DK>) % 16 == 0, "16-byte tiles");
     auto kp = bwd_prep_kernel<DK, DV, CHANNEL>;
     auto kg = bwd_grads_kernel<DK, DV, CHANNEL>;
     auto ks = bwd_state_chain_kernel<DK, DV>;
@@ -813,7 +948,7 @@ cudaError_t launch_bwd_t(const BwdProblem& p, cudaStream_t stream) {
         e = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)chain_smem);
     if (e == cudaSuccess) {
         kp<<<grid_c, BNT, prep_smem, stream>>>(p.q, p.k, p.v, p.g, p.beta, scratch, p.T, p.H, N);
-        ks<<<grid_s, BNT, chain_smem, stream>>>(scratch, p.state_in, states, p.H, N);
+        ks<<<grid_s, BNT, chain_smem, stream>>>(scratch, p.state_in, states, p.T, p.H, N);
         kd<<<grid_s, BNT, chain_smem, stream>>>(scratch, p.d_out, p.d_state_out, dstates, p.d_state_in,
                                                 p.T, p.H, N);
         kg<<<grid_c, BNT, grad_smem, stream>>>(p.q, p.k, p.v, p.g, p.beta, p.d_out, states, dstates,
