@@ -389,6 +389,7 @@ def run_ours(args, rank: int, world: int, local: int):
     prologue = run_prologue(gdn, dev, stream, peaks, world, rank)
     multitoken = run_multitoken(gdn, dev, stream, peaks, world, rank)
     backward = run_backward(gdn, dev, stream, peaks, world, rank)
+    decoupled = run_decoupled(gdn, dev, stream, peaks, world, rank)
 
     line = None
     if rank == 0:
@@ -406,7 +407,8 @@ def run_ours(args, rank: int, world: int, local: int):
                 "data": "synthetic", "config": workload_config(cfg), "roofline": roofline,
                 "tensor": tensor, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": args.steps, "clocks": clk.summary(), "decode": decode,
-                "prologue": prologue, "multi_token_decode": multitoken, "backward": backward}
+                "prologue": prologue, "multi_token_decode": multitoken, "backward": backward,
+                "decoupled_decode": decoupled}
         print(json.dumps(line))
     return 0
 
@@ -570,6 +572,43 @@ def run_multitoken(gdn, dev, stream, peaks, world, rank, T: int = 4, steps: int 
                        "B": cfg.B, "H": cfg.H, "T": T, "dk": cfg.dk, "dv": cfg.dv,
                        "gate": cfg.gate, "l2": "evicted before every timed call"},
             "timing": f"median of {steps} single-call CUDA-event timings"}
+
+
+def run_decoupled(gdn, dev, stream, peaks, world, rank, steps: int = 20, warmup: int = 3):
+    """One decode step with separate erase and write gates on the decode
+    shape (state in place, L2 evicted before every timed step)."""
+    from synth import prefill_inputs, write_gate
+    cfg = DECODE_CFG
+    x = prefill_inputs(cfg.B, 1, cfg.H, cfg.dk, cfg.dv, gate=cfg.gate, s0_std=cfg.s0_std,
+                       seed=cfg.index + 1000 * rank)
+    d = {n: x[n].to(dev) for n in ("q", "k", "v", "g", "beta", "s0")}
+    bw = write_gate(cfg.B, 1, cfg.H, seed=cfg.index + 1000 * rank).to(dev)
+    out = torch.empty(cfg.B, 1, cfg.H, cfg.dv, dtype=torch.float32, device=dev)
+    state = d["s0"]
+    flush = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    times = []
+    for i in range(warmup + steps):
+        torch.sum(flush, dim=0, out=sink)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        gdn.recurrent_steps(d["q"], d["k"], d["v"], d["g"], d["beta"], state, state_out=state,
+                            snapshots=None, out=out, beta_write=bw, stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= warmup:
+            times.append(e0.elapsed_time(e1) / 1e3)
+    t = max_over_ranks(statistics.median(times), world)
+    nbytes = decode_bytes(cfg) + cfg.B * cfg.H * 4
+    gbs = nbytes / t / 1e9
+    return {"metric": "decoupled-gate decode state GB/s", "value": gbs, "unit": "GB/s",
+            "us_per_step": t * 1e6, "frac": gbs / peaks["hbm_gbs"], "peak": peaks["hbm_gbs"],
+            "bytes_per_step": nbytes,
+            "config": {"workload": "decode step, separate erase and write gates", "B": cfg.B,
+                       "H": cfg.H, "dk": cfg.dk, "dv": cfg.dv, "gate": cfg.gate,
+                       "l2": "evicted before every timed step"},
+            "timing": f"median of {steps} single-step CUDA-event timings"}
 
 
 def run_decode(gdn, dev, stream, peaks, world, rank, steps: int = 20, warmup: int = 3):

@@ -38,7 +38,7 @@ ACT_SILU = 1
 
 SYMBOLS = ("gdn_chunk_fwd", "gdn_chunk_fwd_ex", "gdn_chunk_fwd_segments",
            "gdn_chunk_fwd_segments_noalloc", "gdn_recurrent_step", "gdn_recurrent_step_ex",
-           "gdn_chunk_bwd", "gdn_recurrent_steps", "gdn_state_select", "gdn_prologue", "gdn_recurrent_step_prologue",
+           "gdn_chunk_bwd", "gdn_recurrent_steps", "gdn_recurrent_steps_decoupled", "gdn_state_select", "gdn_prologue", "gdn_recurrent_step_prologue",
            "gdn_check", "gdn_status_string")
 
 _lib = None
@@ -69,6 +69,8 @@ def load() -> ctypes.CDLL:
     lib.gdn_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, fp, fp, fp, fp, fp, fp, i, i, i,
                                   i, i, i, vp]
     lib.gdn_recurrent_steps.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, vp, i, i, i, i, i, i, vp]
+    lib.gdn_recurrent_steps_decoupled.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, fp, vp, i, i, i, i,
+                                                  i, i, vp]
     lib.gdn_state_select.argtypes = [fp, vp, fp, i, i, i, i, i, vp]
     lib.gdn_prologue.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, vp, vp, vp, fp, fp, i, i, i, i, i,
                                  i, i, vp]
@@ -188,20 +190,32 @@ def chunk_bwd(q, k, v, g, beta, state_in, d_out, d_state_out=None, *, stream=Non
 
 
 def recurrent_steps(q, k, v, g, beta, state, *, state_out=None, snapshots=True, out=None,
-                    stream=None):
+                    beta_write=None, stream=None):
     """T successive decode tokens per sequence (speculative verification).
     q, k [B,T,H,dk] bf16; v [B,T,H,dv] bf16; g [B,T,H] or [B,T,H,dk];
     beta [B,T,H]; state [B,H,dk,dv] fp32, read only unless state_out is
     ``state`` itself.  ``snapshots``: True allocates [B,T,H,dk,dv], a tensor
-    is written, None skips them.  Returns (out [B,T,H,dv] fp32, snapshots)."""
+    is written, None skips them.  ``beta_write`` [B,T,H]: a separate write
+    gate (gdn_recurrent_steps_decoupled; ``beta`` is then the erase gate).
+    Returns (out [B,T,H,dv] fp32, snapshots)."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     gate = GATE_CHANNEL if g.dim() == 4 else GATE_SCALAR
     if snapshots is True:
         snapshots = torch.empty(B, T, H, dk, dv, dtype=torch.float32, device=v.device)
+    elif snapshots is False:
+        snapshots = None
     if out is None:
         out = torch.empty(B, T, H, dv, dtype=torch.float32, device=v.device)
-    _check_cuda(q, k, v, g, beta, state, state_out, snapshots, out)
+    _check_cuda(q, k, v, g, beta, state, state_out, snapshots, out, beta_write)
+    if beta_write is not None:
+        rc = load().gdn_recurrent_steps_decoupled(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                                  _ptr(beta_write), _ptr(state), _ptr(state_out),
+                                                  _ptr(snapshots), _ptr(out), B, T, H, dk, dv, gate,
+                                                  _stream(stream))
+        if rc != GDN_OK:
+            raise GdnError(rc, "gdn_recurrent_steps_decoupled")
+        return out, snapshots
     rc = load().gdn_recurrent_steps(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
                                     _ptr(state_out), _ptr(snapshots), _ptr(out), B, T, H, dk, dv,
                                     gate, _stream(stream))

@@ -300,10 +300,10 @@ int gdn_recurrent_step(const void* q, const void* k, const void* v, const float*
                                  gate_mode, GDN_IO_BF16, stream);
 }
 
-int gdn_recurrent_steps(const void* q, const void* k, const void* v, const float* g,
-                        const float* beta, const float* state_in, float* state_out,
-                        float* snapshots, void* out, int B, int T, int H, int dk, int dv,
-                        int gate_mode, gdn_stream_t stream_)
+static int recurrent_steps_impl(const void* q, const void* k, const void* v, const float* g,
+                                const float* beta, const float* beta_write, const float* state_in,
+                                float* state_out, float* snapshots, void* out, int B, int T, int H,
+                                int dk, int dv, int gate_mode, gdn_stream_t stream_)
 {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     if (!state_in || T < 1) return GDN_ERR_INVALID_ARG;
@@ -328,7 +328,38 @@ int gdn_recurrent_steps(const void* q, const void* k, const void* v, const float
     gdn::Problem p{q, k, v, g, beta, state_in, state_out, out, B, T, H, dk, dv,
                    gate_mode == GDN_GATE_CHANNEL, false, true};
     p.snapshots = snapshots;
+    p.beta_write = beta_write;
     return to_status(gdn::launch_recurrent(p, stream));
+}
+
+int gdn_recurrent_steps(const void* q, const void* k, const void* v, const float* g,
+                        const float* beta, const float* state_in, float* state_out,
+                        float* snapshots, void* out, int B, int T, int H, int dk, int dv,
+                        int gate_mode, gdn_stream_t stream_)
+{
+    return recurrent_steps_impl(q, k, v, g, beta, nullptr, state_in, state_out, snapshots, out, B, T,
+                                H, dk, dv, gate_mode, stream_);
+}
+
+int gdn_recurrent_steps_decoupled(const void* q, const void* k, const void* v, const float* g,
+                                  const float* beta_erase, const float* beta_write,
+                                  const float* state_in, float* state_out, float* snapshots,
+                                  void* out, int B, int T, int H, int dk, int dv, int gate_mode,
+                                  gdn_stream_t stream_)
+{
+    if (!beta_write) return GDN_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(beta_write) & 3u) return GDN_ERR_MISALIGNED;
+    if (B >= 1 && T >= 1 && H >= 1) {
+        const size_t tok = (size_t)B * T * H;
+        const Range rw = range_of(beta_write, tok * 4);
+        const Range outs[] = {range_of(out, tok * (size_t)(dv > 0 ? dv : 0) * 4),
+                              state_out ? range_of(state_out, (size_t)B * H * dk * dv * 4) : Range{0, 0},
+                              snapshots ? range_of(snapshots, tok * (size_t)dk * dv * 4) : Range{0, 0}};
+        for (Range r : outs)
+            if (overlaps(rw, r)) return GDN_ERR_INVALID_ARG;
+    }
+    return recurrent_steps_impl(q, k, v, g, beta_erase, beta_write, state_in, state_out, snapshots,
+                                out, B, T, H, dk, dv, gate_mode, stream_);
 }
 
 int gdn_state_select(const float* snapshots, const int* num_accepted, float* state, int B, int T,

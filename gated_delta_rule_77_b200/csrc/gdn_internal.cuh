@@ -27,6 +27,7 @@ struct Problem {
     bool out_f32;            // out in fp32 (else bf16)
     int segments = 0;        // chunk path: time segments per (b, h); 0 = automatic
     float* snapshots = nullptr;   // token-serial path: S after every token, [B, T, H, dk, dv]
+    const float* beta_write = nullptr;   // token-serial path: separate write gate, [B, T, H]
 };
 
 // Token-serial fused recurrence (decode, and the fp32 / fallback prefill).

@@ -20,6 +20,10 @@
 // for all T tokens.  The two column reductions go through shared memory once
 // per token; the rank-1 update and the output are then local.
 //
+// Decoupled erase and write gates (a reading of Gated DeltaNet-2, "Gated
+// DeltaNet" entity trail, finding of 2026-05-22): with a write gate bw the
+// update is S = S' - be k (k^T S') + bw k v^T, i.e. u = bw v - be x.
+//
 // Multi-token decode (speculative verification of T draft tokens): with a
 // snapshot buffer every token's updated state slice is also stored, so that
 // the caller can resume from the state after any accepted prefix.
@@ -72,7 +76,8 @@ __global__ void __launch_bounds__(NWARPS * 32)
 recurrent_kernel(const TIN* __restrict__ q, const TIN* __restrict__ k,
                  const TIN* __restrict__ v, const float* __restrict__ g,
                  const float* __restrict__ beta, const float* state_in, float* state_out,
-                 TOUT* __restrict__ out, float* __restrict__ snap, int T, int H, int dv)
+                 TOUT* __restrict__ out, float* __restrict__ snap, const float* __restrict__ beta_w,
+                 int T, int H, int dv)
 {
     constexpr int VW = COLS / 32;
     constexpr int R = DK / NWARPS;
@@ -119,6 +124,7 @@ recurrent_kernel(const TIN* __restrict__ q, const TIN* __restrict__ k,
 #pragma unroll
         for (int c = 0; c < VW; ++c) vv[c] = ld_in(v, tok * dv + col0 + c);
         const float bt = beta[tok];
+        const float bw = beta_w != nullptr ? beta_w[tok] : bt;
         float a_scalar = 1.f;
         if constexpr (!CHANNEL) a_scalar = expf(g[tok]);
         __syncthreads();
@@ -162,7 +168,7 @@ recurrent_kernel(const TIN* __restrict__ q, const TIN* __restrict__ k,
                 x += s_red[buf][0][w][lane * VW + c];
                 cc += s_red[buf][1][w][lane * VW + c];
             }
-            u[c] = bt * (vv[c] - x);
+            u[c] = beta_w != nullptr ? fmaf(bw, vv[c], -bt * x) : bt * (vv[c] - x);
             if (warp == 0) st_out(out, tok * dv + col0 + c, fmaf(u[c], kq_all, cc));
         }
 #pragma unroll
@@ -189,7 +195,7 @@ cudaError_t launch_typed(const Problem& p, cudaStream_t stream) {
     const unsigned grid = static_cast<unsigned>(p.dv / COLS) * p.H * p.B;
     recurrent_kernel<DK, COLS, NWARPS, CHANNEL, TIN, TOUT><<<grid, NWARPS * 32, 0, stream>>>(
         static_cast<const TIN*>(p.q), static_cast<const TIN*>(p.k), static_cast<const TIN*>(p.v),
-        p.g, p.beta, p.state_in, p.state_out, static_cast<TOUT*>(p.out), p.snapshots, p.T, p.H, p.dv);
+        p.g, p.beta, p.state_in, p.state_out, static_cast<TOUT*>(p.out), p.snapshots, p.beta_write, p.T, p.H, p.dv);
     return cudaGetLastError();
 }
 

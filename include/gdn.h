@@ -251,6 +251,25 @@ GDN_API int gdn_recurrent_steps(const void* q, const void* k, const void* v, con
                                 int gate_mode, gdn_stream_t stream);
 
 /*
+ * gdn_recurrent_steps_decoupled -- gdn_recurrent_steps with separate erase
+ * and write gates: S_t = (I - be_t k_t k_t^T) Diag(a_t) S_{t-1}
+ * + bw_t k_t v_t^T.  This is a reading of Gated DeltaNet-2's decoupled
+ * erase / write ("Gated DeltaNet" entity trail, finding of 2026-05-22),
+ * which gives no formula; be = bw is gdn_recurrent_steps.
+ *
+ *   beta_erase [B, T, H] fp32 (the erase gate; the beta of the other calls)
+ *   beta_write [B, T, H] fp32 (required; must not overlap an output)
+ *   every other argument as gdn_recurrent_steps (any T >= 1: one decode step,
+ *   draft tokens, or a token-serial prefill).
+ */
+GDN_API int gdn_recurrent_steps_decoupled(const void* q, const void* k, const void* v,
+                                          const float* g, const float* beta_erase,
+                                          const float* beta_write, const float* state_in,
+                                          float* state_out, float* snapshots, void* out, int B,
+                                          int T, int H, int dk, int dv, int gate_mode,
+                                          gdn_stream_t stream);
+
+/*
  * gdn_state_select -- commit the accepted prefix of a verification step:
  * state[b] := snapshots[b, n_b - 1] for every sequence b whose accepted
  * count n_b = num_accepted[b] (int32, device memory) lies in 1 .. T; rows

@@ -189,3 +189,11 @@ def grad_inputs(B, T, H, dk, dv, *, seed=0, d_state=True):
     ds = torch.randn(B, H, dk, dv, generator=gen) if d_state else None
     return d_out.contiguous(), ds
 
+
+def write_gate(B, T, H, *, seed=0):
+    """A separate write gate for the decoupled form: sigmoid(N(0, 1)) per
+    (b, t, h), fp32, from ``manual_seed(seed)`` (the erase gate is the
+    recipe's beta)."""
+    gen = torch.Generator().manual_seed(int(seed))
+    return torch.sigmoid(_randn_sliced(gen, (B,), T, (H,), 1)).contiguous()
+

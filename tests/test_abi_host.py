@@ -246,3 +246,16 @@ def _bwd(lib, q=A, k=A + 64 * MB, v=A + 128 * MB, g=A + 192 * MB, beta=A + 256 *
 ])
 def test_chunk_bwd_rejects(lib, kw, status):
     assert _bwd(lib, **kw) == status
+
+
+def test_decoupled_steps_rejects(lib):
+    c = ctypes.c_void_p
+    call = lambda bw, out=A + 448 * MB, T=4: lib.gdn_recurrent_steps_decoupled(  # noqa: E731
+        c(A), c(A + 64 * MB), c(A + 128 * MB), c(A + 192 * MB), c(A + 256 * MB),
+        None if bw is None else c(bw), c(A + 320 * MB), c(A + 320 * MB), None, c(out),
+        1, T, 1, 128, 128, 1, None)
+    assert call(None) == gdn.GDN_ERR_INVALID_ARG                  # the write gate is required
+    assert call(A + 300 * MB + 2) == gdn.GDN_ERR_MISALIGNED
+    assert call(A + 448 * MB) == gdn.GDN_ERR_INVALID_ARG          # overlaps out
+    assert call(A + 300 * MB, T=0) == gdn.GDN_ERR_INVALID_ARG
+    assert call(A + 300 * MB, out=A + 16) == gdn.GDN_ERR_INVALID_ARG   # out overlaps q
