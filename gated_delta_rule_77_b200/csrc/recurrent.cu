@@ -71,7 +71,9 @@ __device__ __forceinline__ void st_out(__nv_bfloat16* p, long i, float x) {
     p[i] = __float2bfloat16_rn(x);
 }
 
-template <int DK, int COLS, int NWARPS, bool CHANNEL, typename TIN, typename TOUT>
+// EXT: the snapshot buffer and the separate write gate may be used (a
+// separate instantiation, so that the plain decode step carries neither).
+template <int DK, int COLS, int NWARPS, bool CHANNEL, typename TIN, typename TOUT, bool EXT>
 __global__ void __launch_bounds__(NWARPS * 32)
 recurrent_kernel(const TIN* __restrict__ q, const TIN* __restrict__ k,
                  const TIN* __restrict__ v, const float* __restrict__ g,
@@ -124,7 +126,7 @@ recurrent_kernel(const TIN* __restrict__ q, const TIN* __restrict__ k,
 #pragma unroll
         for (int c = 0; c < VW; ++c) vv[c] = ld_in(v, tok * dv + col0 + c);
         const float bt = beta[tok];
-        const float bw = beta_w != nullptr ? beta_w[tok] : bt;
+        const float bw = (EXT && beta_w != nullptr) ? beta_w[tok] : bt;
         float a_scalar = 1.f;
         if constexpr (!CHANNEL) a_scalar = expf(g[tok]);
         __syncthreads();
@@ -168,7 +170,7 @@ recurrent_kernel(const TIN* __restrict__ q, const TIN* __restrict__ k,
                 x += s_red[buf][0][w][lane * VW + c];
                 cc += s_red[buf][1][w][lane * VW + c];
             }
-            u[c] = beta_w != nullptr ? fmaf(bw, vv[c], -bt * x) : bt * (vv[c] - x);
+            u[c] = (EXT && beta_w != nullptr) ? fmaf(bw, vv[c], -bt * x) : bt * (vv[c] - x);
             if (warp == 0) st_out(out, tok * dv + col0 + c, fmaf(u[c], kq_all, cc));
         }
 #pragma unroll
@@ -177,7 +179,7 @@ recurrent_kernel(const TIN* __restrict__ q, const TIN* __restrict__ k,
 #pragma unroll
             for (int c = 0; c < VW; ++c) s[r][c] = fmaf(ki, u[c], s[r][c]);
         }
-        if (snap != nullptr) {   // S after token t: snapshot [b, t, h]
+        if (EXT && snap != nullptr) {   // S after token t: snapshot [b, t, h]
             float* dst = snap + tok * DK * (long)dv;
 #pragma unroll
             for (int r = 0; r < R; ++r) store_vec<VW>(dst + (long)(row0 + r) * dv + col0, s[r]);
@@ -193,7 +195,14 @@ recurrent_kernel(const TIN* __restrict__ q, const TIN* __restrict__ k,
 template <int DK, int COLS, int NWARPS, bool CHANNEL, typename TIN, typename TOUT>
 cudaError_t launch_typed(const Problem& p, cudaStream_t stream) {
     const unsigned grid = static_cast<unsigned>(p.dv / COLS) * p.H * p.B;
-    recurrent_kernel<DK, COLS, NWARPS, CHANNEL, TIN, TOUT><<<grid, NWARPS * 32, 0, stream>>>(
+    if (p.snapshots != nullptr || p.beta_write != nullptr) {
+        recurrent_kernel<DK, COLS, NWARPS, CHANNEL, TIN, TOUT, true><<<grid, NWARPS * 32, 0, stream>>>(
+            static_cast<const TIN*>(p.q), static_cast<const TIN*>(p.k), static_cast<const TIN*>(p.v),
+            p.g, p.beta, p.state_in, p.state_out, static_cast<TOUT*>(p.out), p.snapshots, p.beta_write,
+            p.T, p.H, p.dv);
+        return cudaGetLastError();
+    }
+    recurrent_kernel<DK, COLS, NWARPS, CHANNEL, TIN, TOUT, false><<<grid, NWARPS * 32, 0, stream>>>(
         static_cast<const TIN*>(p.q), static_cast<const TIN*>(p.k), static_cast<const TIN*>(p.v),
         p.g, p.beta, p.state_in, p.state_out, static_cast<TOUT*>(p.out), p.snapshots, p.beta_write, p.T, p.H, p.dv);
     return cudaGetLastError();
