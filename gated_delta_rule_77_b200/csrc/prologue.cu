@@ -21,6 +21,7 @@
 
 #include <math.h>
 
+#include "chunk_common.cuh"
 #include "gdn_internal.cuh"
 
 namespace gdn {
@@ -67,6 +68,32 @@ __device__ __forceinline__ float log1p_unit(float u) {
 __device__ __forceinline__ float gate_fn(float x) {
     const float sp = fmaxf(x, 0.f) + log1p_unit(ex2_fast(-fabsf(x) * kLog2eP));
     return -fminf(sp, 5.f);
+}
+
+// The same two at a time, with paired fp32 (f32x2) arithmetic.
+using chunk::add2;
+using chunk::fma2;
+using chunk::mul2;
+__device__ __forceinline__ float2 gate_fn2(float2 x) {
+    const float2 u = make_float2(ex2_fast(-fabsf(x.x) * kLog2eP), ex2_fast(-fabsf(x.y) * kLog2eP));
+    const float2 s2 = make_float2(__fdividef(u.x, 2.f + u.x), __fdividef(u.y, 2.f + u.y));
+    const float2 z = mul2(s2, s2);
+    float2 t = make_float2(1.f / 15.f, 1.f / 15.f);
+    t = fma2(t, z, make_float2(1.f / 13.f, 1.f / 13.f));
+    t = fma2(t, z, make_float2(1.f / 11.f, 1.f / 11.f));
+    t = fma2(t, z, make_float2(1.f / 9.f, 1.f / 9.f));
+    t = fma2(t, z, make_float2(1.f / 7.f, 1.f / 7.f));
+    t = fma2(t, z, make_float2(1.f / 5.f, 1.f / 5.f));
+    t = fma2(t, z, make_float2(1.f / 3.f, 1.f / 3.f));
+    t = fma2(t, z, make_float2(1.f, 1.f));
+    const float2 l = mul2(mul2(s2, make_float2(2.f, 2.f)), t);
+    return make_float2(-fminf(fmaxf(x.x, 0.f) + l.x, 5.f), -fminf(fmaxf(x.y, 0.f) + l.y, 5.f));
+}
+__device__ __forceinline__ float2 act_fn2(float2 y, bool silu) {
+    if (!silu) return y;
+    const float2 m = mul2(y, make_float2(-kLog2eP, -kLog2eP));
+    const float2 d = add2(make_float2(ex2_fast(m.x), ex2_fast(m.y)), make_float2(1.f, 1.f));
+    return mul2(y, make_float2(__fdividef(1.f, d.x), __fdividef(1.f, d.y)));
 }
 
 // Channels c of q | k | v for token t of row b, head h (bf16 inputs).
@@ -198,7 +225,11 @@ prologue_kernel(const __nv_bfloat16* __restrict__ q_raw, const __nv_bfloat16* __
             const int i = idx / (DK / 4), c4 = (idx % (DK / 4)) * 4;
             if (idx < NG && i < nt)
                 *reinterpret_cast<float4*>(g + tok_of(t0 + i) * DK + c4) =
-                    make_float4(gate_fn(gb[j].x), gate_fn(gb[j].y), gate_fn(gb[j].z), gate_fn(gb[j].w));
+                    [&] {
+                        const float2 lo = gate_fn2(make_float2(gb[j].x, gb[j].y));
+                        const float2 hi = gate_fn2(make_float2(gb[j].z, gb[j].w));
+                        return make_float4(lo.x, lo.y, hi.x, hi.y);
+                    }();
         }
     }
     if (tid < nt) {
@@ -214,24 +245,41 @@ prologue_kernel(const __nv_bfloat16* __restrict__ q_raw, const __nv_bfloat16* __
     float2 win[3];
 #pragma unroll
     for (int r = 0; r < 3; ++r) win[r] = make_float2(s_h[r][c], s_h[r][c + 1]);
+    // Taps of the two channels side by side, for paired arithmetic.
+    const float2 ta = make_float2(w0.x, w1.x), tb = make_float2(w0.y, w1.y);
+    const float2 tc = make_float2(w0.z, w1.z), td = make_float2(w0.w, w1.w);
     float2 y[TT];
 #pragma unroll
     for (int i = 0; i < TT; ++i) {
         const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&s_x[i][c]));
-        const float a0 = w0.x * win[0].x + w0.y * win[1].x + w0.z * win[2].x + w0.w * x.x;
-        const float a1 = w1.x * win[0].y + w1.y * win[1].y + w1.z * win[2].y + w1.w * x.y;
-        y[i] = make_float2(act_fn(a0, silu), act_fn(a1, silu));
+        const float2 a = fma2(ta, win[0], fma2(tb, win[1], fma2(tc, win[2], mul2(td, x))));
+        y[i] = act_fn2(a, silu);
         win[0] = win[1]; win[1] = win[2]; win[2] = x;
     }
     const int tensor = warp / QW;               // 0 q, 1 k, >= 2 v
     if (tensor < 2) {
+        // Sums of squares of the TT = 16 tokens over the warp's 32 lanes by a
+        // transposing butterfly: at each step a lane keeps half of its
+        // remaining tokens and adds its partner's partial for them, so that
+        // 8 + 4 + 2 + 1 + 1 shuffles leave lanes 2j and 2j + 1 with the
+        // warp's total for one token.
+        static_assert(TT == 16, "the butterfly below is written for 16 tokens");
+        float v[TT];
 #pragma unroll
-        for (int i = 0; i < TT; ++i) {
-            float ss = y[i].x * y[i].x + y[i].y * y[i].y;
+        for (int i = 0; i < TT; ++i) v[i] = fmaf(y[i].x, y[i].x, y[i].y * y[i].y);
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-            if (lane == 0) s_ss[tensor][warp % QW][i] = ss;
+        for (int half = 8, bit = 16; half >= 1; half >>= 1, bit >>= 1) {
+            const bool up = (lane & bit) != 0;
+#pragma unroll
+            for (int i = 0; i < half; ++i) {
+                const float send = up ? v[i] : v[i + half];
+                const float keep = up ? v[i + half] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+            }
         }
+        v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+        const int tok = 8 * ((lane >> 4) & 1) + 4 * ((lane >> 3) & 1) + 2 * ((lane >> 2) & 1) + ((lane >> 1) & 1);
+        if ((lane & 1) == 0) s_ss[tensor][warp % QW][tok] = v[0];
     }
     __syncthreads();
 
