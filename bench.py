@@ -48,6 +48,7 @@ from synth import CONFIGS, config_inputs, prologue_inputs  # noqa: E402
 
 PREFILL_CFG = CONFIGS[2]
 DECODE_CFG = CONFIGS[4]
+LONG_CFG = CONFIGS[5]
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "GDN prefill tokens/s + % tensor roofline; decode state GB/s vs HBM peak"
 PROFILE_SUMMARY = ROOT / "profiles" / "chunk_pair_kernel_gdn2_layer_B8H8T2048.md"
@@ -390,6 +391,7 @@ def run_ours(args, rank: int, world: int, local: int):
     multitoken = run_multitoken(gdn, dev, stream, peaks, world, rank)
     backward = run_backward(gdn, dev, stream, peaks, world, rank)
     decoupled = run_decoupled(gdn, dev, stream, peaks, world, rank)
+    long_context = run_long_context(gdn, dev, stream, peaks, world, rank)
 
     line = None
     if rank == 0:
@@ -408,7 +410,7 @@ def run_ours(args, rank: int, world: int, local: int):
                 "tensor": tensor, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": args.steps, "clocks": clk.summary(), "decode": decode,
                 "prologue": prologue, "multi_token_decode": multitoken, "backward": backward,
-                "decoupled_decode": decoupled}
+                "decoupled_decode": decoupled, "long_context": long_context}
         print(json.dumps(line))
     return 0
 
@@ -571,6 +573,40 @@ def run_multitoken(gdn, dev, stream, peaks, world, rank, T: int = 4, steps: int 
             "config": {"workload": "multi-token decode with per-token state snapshots",
                        "B": cfg.B, "H": cfg.H, "T": T, "dk": cfg.dk, "dv": cfg.dv,
                        "gate": cfg.gate, "l2": "evicted before every timed call"},
+            "timing": f"median of {steps} single-call CUDA-event timings"}
+
+
+def run_long_context(gdn, dev, stream, peaks, world, rank, steps: int = 3, warmup: int = 2):
+    """The long-context prefill (one sequence of 262,144 tokens, 16 heads,
+    scalar gate with 10% g = 0) through the automatic segment-parallel path;
+    inputs 3.4 GB, far above L2."""
+    cfg = LONG_CFG
+    x = config_inputs(cfg, seed=cfg.index + 1000 * rank)
+    q, k, v, g, beta = (x[n].to(dev) for n in ("q", "k", "v", "g", "beta"))
+    del x
+    out = torch.empty(cfg.B, cfg.T, cfg.H, cfg.dv, dtype=torch.float32, device=dev)
+    s_out = torch.empty(cfg.B, cfg.H, cfg.dk, cfg.dv, dtype=torch.float32, device=dev)
+    times = []
+    for i in range(warmup + steps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        gdn.chunk_fwd(q, k, v, g, beta, None, out=out, state_out=s_out, stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= warmup:
+            times.append(e0.elapsed_time(e1) / 1e3)
+    if gdn.check(stream) != gdn.GDN_OK:
+        raise RuntimeError("the long-context prefill reported an abandoned wait")
+    t = max_over_ranks(statistics.median(times), world)
+    nbytes = prefill_bytes(cfg, False)
+    return {"metric": "long-context prefill tokens/s", "value": cfg.B * cfg.T * world / t,
+            "unit": "tokens/s", "ms_per_call": t * 1e3,
+            "roofline": {"bound": "hbm", "achieved": nbytes / t / 1e9, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": nbytes / t / 1e9 / peaks["hbm_gbs"],
+                         "bytes_per_call": nbytes},
+            "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "T": cfg.T, "dk": cfg.dk,
+                       "dv": cfg.dv, "gate": cfg.gate, "path": "segment-parallel (automatic)"},
             "timing": f"median of {steps} single-call CUDA-event timings"}
 
 
