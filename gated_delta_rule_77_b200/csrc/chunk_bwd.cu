@@ -73,7 +73,7 @@ __device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_
 }
 
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
                  "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
                  : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
                  : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -96,16 +96,21 @@ __device__ __forceinline__ void wmm(float (&acc)[NT][4], int rb, int cb, FA a, F
         split2(a(rb + g + 8, k0 + 2 * t), a(rb + g + 8, k0 + 2 * t + 1), ah[1], al[1]);
         split2(a(rb + g, k0 + 2 * t + 8), a(rb + g, k0 + 2 * t + 9), ah[2], al[2]);
         split2(a(rb + g + 8, k0 + 2 * t + 8), a(rb + g + 8, k0 + 2 * t + 9), ah[3], al[3]);
+        uint32_t bh0[NT], bl0[NT], bh1[NT], bl1[NT];
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
             const int n = cb + 8 * j + g;
-            uint32_t bh0, bl0, bh1, bl1;
-            split2(b(k0 + 2 * t, n), b(k0 + 2 * t + 1, n), bh0, bl0);
-            split2(b(k0 + 2 * t + 8, n), b(k0 + 2 * t + 9, n), bh1, bl1);
-            mma16816(acc[j], ah, bh0, bh1);
-            mma16816(acc[j], ah, bl0, bl1);
-            mma16816(acc[j], al, bh0, bh1);
+            split2(b(k0 + 2 * t, n), b(k0 + 2 * t + 1, n), bh0[j], bl0[j]);
+            split2(b(k0 + 2 * t + 8, n), b(k0 + 2 * t + 9, n), bh1[j], bl1[j]);
         }
+        // The three products of a tile accumulate in one register set: issue
+        // them NT apart so that consecutive MMAs are independent.
+#pragma unroll
+        for (int j = 0; j < NT; ++j) mma16816(acc[j], ah, bh0[j], bh1[j]);
+#pragma unroll
+        for (int j = 0; j < NT; ++j) mma16816(acc[j], ah, bl0[j], bl1[j]);
+#pragma unroll
+        for (int j = 0; j < NT; ++j) mma16816(acc[j], al, bh0[j], bh1[j]);
     }
 }
 
