@@ -644,12 +644,27 @@ bwd_grads_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     auto Kt = [&](int r, int cc) { return CHANNEL ? s.KL[r][cc] * m.eM[cc] : s.KL[r][cc] * m.eM[r]; };
     auto Qt = [&](int r, int cc) { return CHANNEL ? s.QL[r][cc] * m.eM[cc] : s.QL[r][cc] * m.eM[r]; };
     auto Kh = [&](int r, int cc) { return CHANNEL ? s.KR[r][cc] * m.eH[cc] : s.KL[r][cc] * m.eH[r]; };
-    auto Eo = [&](int r, int cc) { return CHANNEL ? expf(s.Gam[r][cc]) : m.eM[r]; };
-    auto Eho = [&](int r, int cc) { return CHANNEL ? expf(s.Gl[cc] - s.Gam[r][cc]) : m.eH[r]; };
+    // Per-element decay factors of this thread's C x DK elements (channel
+    // gate): L = exp(G - G_m) once, then E = L e^{G_m}, exp(G_last - G) =
+    // e^{G_last - G_m} / L and R = 1 / L (see Lr, Rr below).
 
     const Tile32<DK> tk;     // C x DK outputs: this thread's elements
     const Tile32<DV> tv;     // C x DV outputs
     const Tile32<BC> tc;     // C x C outputs
+    float Lr[CHANNEL ? NK : 1][4], Rr[CHANNEL ? NK : 1][4];
+    if (CHANNEL) {
+#pragma unroll
+        for (int j = 0; j < NK; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = tk.row(e), cc = tk.col(j, e);
+                Lr[j][e] = expf(s.Gam[r][cc] - s.Gm[cc]);
+                Rr[j][e] = __fdividef(1.f, Lr[j][e]);
+            }
+    }
+    // E and exp(G_last - G) of element (j, e) of this thread.
+    auto Ej = [&](int j, int e, int r, int cc) { return CHANNEL ? Lr[j][e] * m.eM[cc] : m.eM[r]; };
+    auto Ehj = [&](int j, int e, int r, int cc) { return CHANNEL ? m.eH[cc] * Rr[j][e] : m.eH[r]; };
     float dQa[NK][4], dKa[NK][4], dGa[NK][4];
     zero_acc(dQa);
     zero_acc(dKa);
@@ -674,7 +689,7 @@ bwd_grads_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int r = tk.row(e), cc = tk.col(j, e);
-                dQa[j][e] += Eo(r, cc) * acc[j][e];
+                dQa[j][e] += Ej(j, e, r, cc) * acc[j][e];
                 dGa[j][e] += Qt(r, cc) * acc[j][e];
             }
     }
@@ -738,7 +753,7 @@ bwd_grads_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
             for (int e = 0; e < 4; ++e) {
                 const int r = tk.row(e), cc = tk.col(j, e);
                 const float kh = Kh(r, cc);
-                dKa[j][e] += Eho(r, cc) * acc[j][e];
+                dKa[j][e] += Ehj(j, e, r, cc) * acc[j][e];
                 dGa[j][e] -= kh * acc[j][e];
                 colsum[e & 1] = fmaf(kh, acc[j][e], colsum[e & 1]);
             }
@@ -810,13 +825,12 @@ bwd_grads_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int r = tk.row(e), cc = tk.col(j, e);
-                dKa[j][e] += Eo(r, cc) * acc[j][e];
+                dKa[j][e] += Ej(j, e, r, cc) * acc[j][e];
                 dGa[j][e] += Kt(r, cc) * acc[j][e];
             }
     }
     // The decay-weighted products of A and P, rows and columns.
     auto decay = [&](int r, int j) { return CHANNEL ? 1.f : s.D[r][j]; };
-    auto Lf = [&](int r, int cc) { return expf(s.Gam[r][cc] - s.Gm[cc]); };
     {   // t_row = (b G) KR ; t_col = (b G)^T KL
         float tr[NK][4], tcl[NK][4];
         zero_acc(tr);
@@ -831,7 +845,7 @@ bwd_grads_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
             for (int e = 0; e < 4; ++e) {
                 const int r = tk.row(e), cc = tk.col(j, e);
                 if (CHANNEL) {
-                    const float L = Lf(r, cc), R = 1.f / L;
+                    const float L = Lr[j][e], R = Rr[j][e];
                     dKa[j][e] += L * tr[j][e] + R * tcl[j][e];
                     dGa[j][e] += s.KL[r][cc] * tr[j][e] - s.KR[r][cc] * tcl[j][e];
                 } else {
@@ -853,7 +867,7 @@ bwd_grads_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
             for (int e = 0; e < 4; ++e) {
                 const int r = tk.row(e), cc = tk.col(j, e);
                 if (CHANNEL) {
-                    const float L = Lf(r, cc), R = 1.f / L;
+                    const float L = Lr[j][e], R = Rr[j][e];
                     dQa[j][e] += L * pr[j][e];
                     dKa[j][e] += R * pc[j][e];
                     dGa[j][e] += s.QL[r][cc] * pr[j][e] - s.KR[r][cc] * pc[j][e];
