@@ -114,6 +114,55 @@ __device__ __forceinline__ void wmm(float (&acc)[NT][4], int rb, int cb, FA a, F
     }
 }
 
+// ldmatrix of four 8 x 8 bf16 matrices (lane i gives the row address of
+// matrix i / 8), plain or transposed.
+__device__ __forceinline__ void ldsm4(uint32_t (&r)[4], const void* p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))) : "memory");
+}
+__device__ __forceinline__ void ldsm4t(uint32_t (&r)[4], const void* p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))) : "memory");
+}
+
+// wmm with the B operand already split: bf16 tiles bh (hi) and bl (lo) of
+// row length LD.  TRANS: B(k, n) = tile[k][n]; otherwise B(k, n) =
+// tile[n][k].  Each ldmatrix.x4 brings both fragment registers of two
+// 8-column tiles (NT even).  Rows must start on 16-byte boundaries.
+template <int NT, int K, bool TRANS, int LD, typename FA>
+__device__ __forceinline__ void wmm_sb(float (&acc)[NT][4], int rb, int cb, FA a,
+                                       const __nv_bfloat16* bh, const __nv_bfloat16* bl) {
+    static_assert(NT % 2 == 0, "pairs of 8-column tiles");
+    const int l = threadIdx.x & 31, g = l >> 2, t = l & 3;
+    const int mi = l >> 3, rr = l & 7;
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 16) {
+        uint32_t ah[4], al[4];
+        split2(a(rb + g, k0 + 2 * t), a(rb + g, k0 + 2 * t + 1), ah[0], al[0]);
+        split2(a(rb + g + 8, k0 + 2 * t), a(rb + g + 8, k0 + 2 * t + 1), ah[1], al[1]);
+        split2(a(rb + g, k0 + 2 * t + 8), a(rb + g, k0 + 2 * t + 9), ah[2], al[2]);
+        split2(a(rb + g + 8, k0 + 2 * t + 8), a(rb + g + 8, k0 + 2 * t + 9), ah[3], al[3]);
+        uint32_t bhv[NT / 2][4], blv[NT / 2][4];
+#pragma unroll
+        for (int jp = 0; jp < NT / 2; ++jp) {
+            const int n0 = cb + 16 * jp;
+            long off;
+            if (TRANS) off = (long)(k0 + rr + 8 * (mi & 1)) * LD + n0 + 8 * (mi >> 1);
+            else off = (long)(n0 + rr + 8 * (mi >> 1)) * LD + k0 + 8 * (mi & 1);
+            if (TRANS) { ldsm4t(bhv[jp], bh + off); ldsm4t(blv[jp], bl + off); }
+            else { ldsm4(bhv[jp], bh + off); ldsm4(blv[jp], bl + off); }
+        }
+#pragma unroll
+        for (int j = 0; j < NT; ++j) mma16816(acc[j], ah, bhv[j / 2][2 * (j & 1)], bhv[j / 2][2 * (j & 1) + 1]);
+#pragma unroll
+        for (int j = 0; j < NT; ++j) mma16816(acc[j], ah, blv[j / 2][2 * (j & 1)], blv[j / 2][2 * (j & 1) + 1]);
+#pragma unroll
+        for (int j = 0; j < NT; ++j) mma16816(acc[j], al, bhv[j / 2][2 * (j & 1)], bhv[j / 2][2 * (j & 1) + 1]);
+    }
+}
+
 template <int NT>
 __device__ __forceinline__ void zero_acc(float (&acc)[NT][4]) {
 #pragma unroll
@@ -559,7 +608,8 @@ struct __align__(16) GradSmem {
     float V[BC][DV + 4];       // v, then E2 = V - Kt S
     float dO[BC][DV + 4];      // dO, then dU, then Y
     float U[BC][DV + 4];
-    float Big[DK][DV + 4];     // S, dS_next, S again, then dG [C][DK]
+    __nv_bfloat16 BigH[DK][DV + 8];   // S, dS_next, S again (bf16 hi); then dG [C][DK] fp32
+    __nv_bfloat16 BigL[DK][DV + 8];   // the matching bf16 lo
     float dP[BC][CP];          // lower(dO U^T), no decay
     float Gm2[BC][CP];         // -strictlower(Y U^T), no decay
     float rowdot[DK];          // rowsum(dS_next (.) S)
@@ -592,18 +642,39 @@ bwd_grads_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     const float* gdS = dstates + n * DK * (long)DV;
     auto tok_of = [&](int r) -> long { return ((long)b * T + t0 + r) * H + h; };
     constexpr int IT = DK * DV / 4 / BNT;   // 16-byte pieces of a state per thread
-    // Asynchronous copy of a state into Big (one commit group).
-    auto fetch_big = [&](const float* src) {
+    constexpr int LDB = DV + 8;
+    // A state into BigH / BigL as bf16 hi + lo; every load is issued first.
+    auto put4 = [&](int r, int q4, float4 x) {
+        uint32_t h0, l0, h1, l1;
+        split2(x.x, x.y, h0, l0);
+        split2(x.z, x.w, h1, l1);
+        *reinterpret_cast<uint2*>(&m.BigH[r][q4]) = make_uint2(h0, h1);
+        *reinterpret_cast<uint2*>(&m.BigL[r][q4]) = make_uint2(l0, l1);
+    };
+    auto get4 = [&](int r, int q4) -> float4 {   // hi + lo back in fp32
+        const uint2 hh = *reinterpret_cast<const uint2*>(&m.BigH[r][q4]);
+        const uint2 ll = *reinterpret_cast<const uint2*>(&m.BigL[r][q4]);
+        const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hh.x));
+        const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hh.y));
+        const float2 b0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ll.x));
+        const float2 b1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ll.y));
+        return make_float4(a0.x + b0.x, a0.y + b0.y, a1.x + b1.x, a1.y + b1.y);
+    };
+    auto load_big = [&](const float* src) {
+        float4 x[IT];
 #pragma unroll
         for (int it = 0; it < IT; ++it) {
             const int idx = tid + it * BNT;
-            const int r = idx / (DV / 4), q4 = 4 * (idx % (DV / 4));
-            cp_async16(&m.Big[r][q4], src + (long)r * DV + q4);
+            x[it] = *reinterpret_cast<const float4*>(src + (long)(idx / (DV / 4)) * DV + 4 * (idx % (DV / 4)));
         }
-        cp_async_commit();
+#pragma unroll
+        for (int it = 0; it < IT; ++it) {
+            const int idx = tid + it * BNT;
+            put4(idx / (DV / 4), 4 * (idx % (DV / 4)), x[it]);
+        }
     };
 
-    fetch_big(gS);
+    load_big(gS);
     {
         constexpr int IV = BC * DV / 2 / BNT;
         float2 vv[IV], oo[IV];
@@ -628,8 +699,6 @@ bwd_grads_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     }
     for (int cc = tid; cc < DK; cc += BNT) m.last[cc] = 0.f;
     chunk_local<DK, CHANNEL>(s, q, k, g, beta, b, h, t0, T, H);   // ends with a barrier
-    cp_async_wait0();
-    __syncthreads();
     if (CHANNEL) {
         for (int cc = tid; cc < DK; cc += BNT) {
             m.eM[cc] = expf(s.Gm[cc]);
@@ -673,7 +742,7 @@ bwd_grads_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     {   // E2 = V - Kt S (in place in V)
         float acc[NV][4];
         zero_acc(acc);
-        wmm<NV, DK>(acc, tv.rb, tv.cb, Kt, [&](int kk, int j) { return m.Big[kk][j]; });
+        wmm_sb<NV, DK, true, LDB>(acc, tv.rb, tv.cb, Kt, &m.BigH[0][0], &m.BigL[0][0]);
 #pragma unroll
         for (int j = 0; j < NV; ++j)
 #pragma unroll
@@ -682,8 +751,8 @@ bwd_grads_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     {   // dQt = dO S^T
         float acc[NK][4];
         zero_acc(acc);
-        wmm<NK, DV>(acc, tk.rb, tk.cb, [&](int r, int j) { return m.dO[r][j]; },
-                    [&](int j, int cc) { return m.Big[cc][j]; });
+        wmm_sb<NK, DV, false, LDB>(acc, tk.rb, tk.cb, [&](int r, int j) { return m.dO[r][j]; },
+                                   &m.BigH[0][0], &m.BigL[0][0]);
 #pragma unroll
         for (int j = 0; j < NK; ++j)
 #pragma unroll
@@ -709,9 +778,9 @@ bwd_grads_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         for (int it = 0; it < IT; ++it) {
             const int idx = tid + it * BNT;
             const int r = idx / (DV / 4), q4 = 4 * (idx % (DV / 4));
-            float4& sv = *reinterpret_cast<float4*>(&m.Big[r][q4]);
+            const float4 sv = get4(r, q4);
             float d = x[it].x * sv.x + x[it].y * sv.y + x[it].z * sv.z + x[it].w * sv.w;
-            sv = x[it];
+            put4(r, q4, x[it]);
             // the DV / 4 lanes that share row r are consecutive: reduce over them
 #pragma unroll
             for (int o = DV / 8; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
@@ -744,8 +813,8 @@ bwd_grads_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     {   // dKh = U dS_next^T
         float acc[NK][4];
         zero_acc(acc);
-        wmm<NK, DV>(acc, tk.rb, tk.cb, [&](int r, int j) { return m.U[r][j]; },
-                    [&](int j, int cc) { return m.Big[cc][j]; });
+        wmm_sb<NK, DV, false, LDB>(acc, tk.rb, tk.cb, [&](int r, int j) { return m.U[r][j]; },
+                                   &m.BigH[0][0], &m.BigL[0][0]);
 #pragma unroll
         for (int j = 0; j < NK; ++j) {
             float colsum[2] = {0.f, 0.f};
@@ -764,11 +833,10 @@ bwd_grads_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     {   // dU = Kh dS_next + P^T dO  (into dO once every thread is done with dO)
         float acc[NV][4];
         zero_acc(acc);
-        wmm<NV, DK>(acc, tv.rb, tv.cb, Kh, [&](int kk, int j) { return m.Big[kk][j]; });
+        wmm_sb<NV, DK, true, LDB>(acc, tv.rb, tv.cb, Kh, &m.BigH[0][0], &m.BigL[0][0]);
         wmm<NV, BC>(acc, tv.rb, tv.cb, [&](int r, int j) { return s.P[j][r]; },
                     [&](int j, int cc) { return m.dO[j][cc]; });
         __syncthreads();
-        fetch_big(gS);   // S again: dS_next is no longer read
 #pragma unroll
         for (int j = 0; j < NV; ++j)
 #pragma unroll
@@ -813,13 +881,13 @@ bwd_grads_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
         if (l == 0) m.db[r] = x;
     }
-    cp_async_wait0();
+    load_big(gS);    // S again: dS_next is no longer read
     __syncthreads();
     {   // dKt = -Diag(b) Y S^T
         float acc[NK][4];
         zero_acc(acc);
-        wmm<NK, DV>(acc, tk.rb, tk.cb, [&](int r, int j) { return -s.beta[r] * m.dO[r][j]; },
-                    [&](int j, int cc) { return m.Big[cc][j]; });
+        wmm_sb<NK, DV, false, LDB>(acc, tk.rb, tk.cb, [&](int r, int j) { return -s.beta[r] * m.dO[r][j]; },
+                                   &m.BigH[0][0], &m.BigL[0][0]);
 #pragma unroll
         for (int j = 0; j < NK; ++j)
 #pragma unroll
@@ -888,7 +956,8 @@ bwd_grads_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
             }
         }
     __syncthreads();   // every read of Big (S) is done
-    float* sdG = &m.Big[0][0];               // [C][DK]
+    float* sdG = reinterpret_cast<float*>(&m.BigH[0][0]);   // [C][DK] fp32
+    static_assert(sizeof(float) * BC * DK <= sizeof(__nv_bfloat16) * DK * (DV + 8), "dG fits in BigH");
 #pragma unroll
     for (int j = 0; j < NK; ++j)
 #pragma unroll
