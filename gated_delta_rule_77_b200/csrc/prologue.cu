@@ -420,13 +420,10 @@ recurrent_prologue_kernel(const __nv_bfloat16* __restrict__ q_raw, const __nv_bf
             ring[(ring_bh + (p & 3)) * CH + DK + tid] = xk;
         }
     }
-    float sq = yq * yq, sk = yk * yk;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        sq += __shfl_xor_sync(0xffffffffu, sq, o);
-        sk += __shfl_xor_sync(0xffffffffu, sk, o);
+    if (tid < DK) {           // unnormalised: the norms are applied after the reductions
+        s_q[tid] = yq;
+        s_k[tid] = yk;
     }
-    if (lane == 0) { s_ss[0][warp] = sq; s_ss[1][warp] = sk; }
     float vv[VW];
 #pragma unroll
     for (int c = 0; c < VW; ++c) {
@@ -438,29 +435,24 @@ recurrent_prologue_kernel(const __nv_bfloat16* __restrict__ q_raw, const __nv_bf
     float a_scalar = 1.f;
     if (!CHANNEL) a_scalar = expf(gate_fn(g_raw[tok]));
     __syncthreads();
-    {
-        float nq = 0.f, nk = 0.f;
-#pragma unroll
-        for (int w = 0; w < NWARPS; ++w) { nq += s_ss[0][w]; nk += s_ss[1][w]; }
-        if (tid < DK) {
-            s_q[tid] = yq * rsqrtf(nq + 1e-6f);
-            s_k[tid] = yk * rsqrtf(nk + 1e-6f);
-        }
-    }
-    __syncthreads();
 
-    // The decode step (as recurrent.cu): S' = Diag(a) S, x = S'^T k,
-    // c = S'^T q, u = b (v - x), S = S' + k u^T, o = c + u (k . q).
+    // The decode step (as recurrent.cu) with q = yq / |yq|, k = yk / |yk|.
+    // The norms are scalars of the head, so they are applied after the
+    // column reductions: x = S'^T yk / |yk|, c = S'^T yq / |yq|, and their
+    // sums of squares ride along in the same exchange.  S' = Diag(a) S,
+    // u = b (v - x), S = S' + k u^T, o = c + u (k . q).
     float px[VW], pc[VW];
 #pragma unroll
     for (int c = 0; c < VW; ++c) { px[c] = 0.f; pc[c] = 0.f; }
-    float kq = 0.f;
+    float kq = 0.f, ssk = 0.f, ssq = 0.f;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
         const float ki = s_k[row0 + r];
         const float qi = s_q[row0 + r];
         const float ai = CHANNEL ? s_a[row0 + r] : a_scalar;
         kq = fmaf(ki, qi, kq);
+        ssk = fmaf(ki, ki, ssk);
+        ssq = fmaf(qi, qi, ssq);
 #pragma unroll
         for (int c = 0; c < VW; ++c) {
             s[r][c] *= ai;
@@ -473,11 +465,20 @@ recurrent_prologue_kernel(const __nv_bfloat16* __restrict__ q_raw, const __nv_bf
         s_red[0][warp][lane * VW + c] = px[c];
         s_red[1][warp][lane * VW + c] = pc[c];
     }
-    if (lane == 0) s_kq[warp] = kq;
+    if (lane == 0) {
+        s_kq[warp] = kq;
+        s_ss[0][warp] = ssq;
+        s_ss[1][warp] = ssk;
+    }
     __syncthreads();
-    float kq_all = 0.f;
+    float kq_all = 0.f, nq = 0.f, nk = 0.f;
 #pragma unroll
-    for (int w = 0; w < NWARPS; ++w) kq_all += s_kq[w];
+    for (int w = 0; w < NWARPS; ++w) {
+        kq_all += s_kq[w];
+        nq += s_ss[0][w];
+        nk += s_ss[1][w];
+    }
+    const float iq = rsqrtf(nq + 1e-6f), ik = rsqrtf(nk + 1e-6f);
     float u[VW];
 #pragma unroll
     for (int c = 0; c < VW; ++c) {
@@ -487,12 +488,12 @@ recurrent_prologue_kernel(const __nv_bfloat16* __restrict__ q_raw, const __nv_bf
             x += s_red[0][w][lane * VW + c];
             cc += s_red[1][w][lane * VW + c];
         }
-        u[c] = bt * (vv[c] - x);
-        if (warp == 0) out[tok * dv + col0 + c] = fmaf(u[c], kq_all, cc);
+        u[c] = bt * (vv[c] - x * ik);
+        if (warp == 0) out[tok * dv + col0 + c] = fmaf(u[c], kq_all * ik * iq, cc * iq);
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-        const float ki = s_k[row0 + r];
+        const float ki = s_k[row0 + r] * ik;
 #pragma unroll
         for (int c = 0; c < VW; ++c) s[r][c] = fmaf(ki, u[c], s[r][c]);
     }
