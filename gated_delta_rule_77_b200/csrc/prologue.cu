@@ -376,16 +376,21 @@ recurrent_prologue_kernel(const __nv_bfloat16* __restrict__ q_raw, const __nv_bf
     // all four slots and the three history slots are picked afterwards.
     float s[R][VW];
     const long sbase = ((long)b * H + h) * DK * (long)dv;
+    if (state_in != nullptr) {      // one test outside the loop: every load issued back to back
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-        if constexpr (VW == 2) {
-            float2 t = make_float2(0.f, 0.f);
-            if (state_in != nullptr)
-                t = *reinterpret_cast<const float2*>(state_in + sbase + (long)(row0 + r) * dv + col0);
-            s[r][0] = t.x; s[r][1] = t.y;
-        } else {
-            s[r][0] = state_in != nullptr ? state_in[sbase + (long)(row0 + r) * dv + col0] : 0.f;
+        for (int r = 0; r < R; ++r) {
+            if constexpr (VW == 2) {
+                const float2 t = *reinterpret_cast<const float2*>(state_in + sbase + (long)(row0 + r) * dv + col0);
+                s[r][0] = t.x; s[r][1] = t.y;
+            } else {
+                s[r][0] = state_in[sbase + (long)(row0 + r) * dv + col0];
+            }
         }
+    } else {
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int c = 0; c < VW; ++c) s[r][c] = 0.f;
     }
 
     // Convolution of one channel: taps 0..2 from ring slots p-3 .. p-1 (zero
