@@ -14,10 +14,15 @@ workload -- B=64 sequences, H=16, d=128, per-channel gate, fp32 state
 carried in place -- with L2 flushed before every timed step (the 64 MiB
 state would otherwise stay in the 126 MB L2), reported under "decode".
 
-The layer's input prologue is measured beside them under "prologue": the
-prefill pass (gdn_prologue) on the GDN-2 layer shape, and the decode step
-with the prologue fused in (gdn_recurrent_step_prologue) on the decode
-shape, each against the HBM bandwidth.
+Measured beside them, each as its own object of the same JSON line:
+  "prologue"            the input prologue: the prefill pass (gdn_prologue) on
+                        the GDN-2 layer shape and the decode step with the
+                        prologue fused in (gdn_recurrent_step_prologue);
+  "multi_token_decode"  4 draft tokens with per-token state snapshots;
+  "backward"            the prefill gradients (gdn_chunk_bwd), GDN-2 layer shape;
+  "decoupled_decode"    a decode step with separate erase and write gates;
+  "long_context"        one sequence of 262,144 tokens over 16 heads through
+                        the segment-parallel path.
 
 Under torchrun (N > 1) every rank runs the same per-GPU workload on its own
 GPU (weak scaling, no collective on the data path); the reported time is
