@@ -60,6 +60,7 @@
 #include <mutex>
 
 #include "chunk_common.cuh"
+#include "warp_mma.cuh"
 #include "gdn_internal.cuh"
 #include "sm100_util.cuh"
 
@@ -142,13 +143,18 @@ struct Params {
     int T, H, B;
     int nseg, seg_len;         // time segments of seg_len tokens (a multiple of C)
     int in_segs, out_segs;     // 1 or nseg
+    // Transition CTAs with a buffer here also form outputs: with v = 0 from
+    // the identity their "output" is w_t = M_t^T q_t ([B, T, H, D] fp32),
+    // M_t the state map from the segment start to token t, so that the true
+    // output is the zero-start one plus S_start^T w_t.
+    float* wout = nullptr;
 };
 
 template <bool CHANNEL>
 __global__ void __launch_bounds__(NT, 1)
 chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                 const Params p)
+                 const __grid_constant__ CUtensorMap tm_w, const Params p)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base (128B-swizzle atoms), derived by a pointer offset
@@ -190,7 +196,8 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int nchunks = t_end > t_begin ? (t_end - t_begin + C - 1) / C : 0;
     // Outputs are formed only where they are written (not by transition CTAs
     // nor by the zero-start pass of the segment path).
-    const bool want_o = !transition && p.out != nullptr;
+    const bool want_o = transition ? p.wout != nullptr : p.out != nullptr;
+    const CUtensorMap* tm_store = transition ? &tm_w : &tm_o;
 
     // Element ownership for the gate prep and tile building: 16 channel
     // chunks of 8 (ck) x 16 lanes (tg), lane tg owning tokens tg + 16 u,
@@ -206,7 +213,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
-        if (p.out != nullptr) prefetch_tensormap(&tm_o);
+        if (want_o) prefetch_tensormap(tm_store);
         mbar_init(bar_tma, 1);
         mbar_init(bar_mma, 1);
         mbar_init(bar_out, 1);
@@ -766,7 +773,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tc_fence_before();
         if (__syncthreads_or(!ok)) break;
         if (want_o && tid == 0) {
-            tma_store_4d(&tm_o, sbase + OFF_OST, 0, h, t0, b);
+            tma_store_4d(tm_store, sbase + OFF_OST, 0, h, t0, b);
             bulk_commit();
         }
     }
@@ -907,6 +914,96 @@ combine_segments_kernel(float* seg_states, const float* trans, const float* stat
     }
 }
 
+// Segment correction: out[b, t, h, :] += S_start(b, seg(t), h)^T w[b, t, h, :]
+// for every token of a segment, after the combine has produced the true start
+// states.  One CTA per group of CORR_TILES 64-token tiles of one (batch,
+// segment, head); the start state is held as bf16 hi + lo and read with
+// ldmatrix, each tile of w (tokens x key channels) is the split A operand,
+// on mma.sync (warp_mma.cuh).
+constexpr int CORR_TILES = 16;
+struct __align__(16) CorrSmem {
+    __nv_bfloat16 sh[D][D + 8];
+    __nv_bfloat16 sl[D][D + 8];
+    float w[C][D + 4];
+};
+__global__ void __launch_bounds__(256)
+segment_correction_kernel(const float* __restrict__ seg_states, const float* __restrict__ wbuf,
+                          float* __restrict__ out, int T, int H, int nseg, int seg_len)
+{
+    using namespace wmma16;
+    extern __shared__ __align__(16) unsigned char corr_raw[];
+    CorrSmem& m = *reinterpret_cast<CorrSmem*>(corr_raw);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int h = blockIdx.y % H, seg = blockIdx.y / H, b = blockIdx.z;
+    const int t_begin = seg * seg_len, t_end = min(T, t_begin + seg_len);
+    const int tile0 = blockIdx.x * CORR_TILES;
+    if (t_begin + tile0 * C >= t_end) return;
+    const float* src = seg_states + (((long)b * nseg + seg) * H + h) * (long)(D * D);
+    for (int idx = tid; idx < D * D / 4; idx += 256) {
+        const int r = idx / (D / 4), q4 = 4 * (idx % (D / 4));
+        const float4 x = *reinterpret_cast<const float4*>(src + (long)r * D + q4);
+        uint32_t h0, l0, h1, l1;
+        split2(x.x, x.y, h0, l0);
+        split2(x.z, x.w, h1, l1);
+        *reinterpret_cast<uint2*>(&m.sh[r][q4]) = make_uint2(h0, h1);
+        *reinterpret_cast<uint2*>(&m.sl[r][q4]) = make_uint2(l0, l1);
+    }
+    const int rb = (warp >> 1) * 16, cb = (warp & 1) * 64;
+    const int l = tid & 31, g = l >> 2, t4 = l & 3;
+    // Software pipeline in registers: tile i + 1's w and tile i's outputs are
+    // loaded while tile i's products run.
+    constexpr int WPT = C * D / 4 / 256;     // float4 of a w tile per thread
+    float4 wreg[WPT];
+    auto load_w = [&](int t0) {
+#pragma unroll
+        for (int it = 0; it < WPT; ++it) {
+            const int idx = tid + it * 256;
+            const int r = idx / (D / 4), q4 = 4 * (idx % (D / 4));
+            wreg[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (t0 + r < t_end) wreg[it] = *reinterpret_cast<const float4*>(wbuf + (((long)b * T + t0 + r) * H + h) * D + q4);
+        }
+    };
+    load_w(t_begin + tile0 * C);
+    for (int i = 0; i < CORR_TILES; ++i) {
+        const int t0 = t_begin + (tile0 + i) * C;
+        if (t0 >= t_end) break;
+        __syncthreads();                     // the previous tile's w is consumed
+#pragma unroll
+        for (int it = 0; it < WPT; ++it) {
+            const int idx = tid + it * 256;
+            *reinterpret_cast<float4*>(&m.w[idx / (D / 4)][4 * (idx % (D / 4))]) = wreg[it];
+        }
+        __syncthreads();
+        // This tile's outputs, then the next tile's w, both in flight during the products.
+        float2 ov[8][2];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int e2 = 0; e2 < 2; ++e2) {
+                const int r = rb + g + 8 * e2;
+                ov[j][e2] = make_float2(0.f, 0.f);
+                if (t0 + r < t_end)
+                    ov[j][e2] = *reinterpret_cast<const float2*>(out + (((long)b * T + t0 + r) * H + h) * D + cb + 8 * j + 2 * t4);
+            }
+        const int tn = t0 + C;
+        if (i + 1 < CORR_TILES && tn < t_end) load_w(tn);
+        float acc[8][4];
+        zero_acc(acc);
+        wmm_sb<8, D, true, D + 8>(acc, rb, cb, [&](int r, int k) { return m.w[r][k]; },
+                                  &m.sh[0][0], &m.sl[0][0]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int e2 = 0; e2 < 2; ++e2) {
+                const int r = rb + g + 8 * e2;
+                if (t0 + r < t_end) {
+                    float2* o = reinterpret_cast<float2*>(out + (((long)b * T + t0 + r) * H + h) * D + cb + 8 * j + 2 * t4);
+                    *o = make_float2(ov[j][e2].x + acc[j][2 * e2], ov[j][e2].y + acc[j][2 * e2 + 1]);
+                }
+            }
+    }
+}
+
 int sm_count() {
     static int n = 0;
     if (n == 0) {
@@ -957,22 +1054,33 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
         if (pair) return launch_chunk_pair_sm100(p, stream);
         Params prm{p.g, p.beta, p.state_in, p.state_out, nullptr, out, p.T, p.H, p.B,
                    1, nchunks * C, 1, 1};
-        chunk_fwd_kernel<CHANNEL><<<p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, prm);
+        chunk_fwd_kernel<CHANNEL><<<p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mo, prm);
         return cudaGetLastError();
     }
-    // Segment-parallel path: per segment the zero-start end state and the
-    // transition (one launch, two kinds of CTA), a serial combine, then every
-    // segment again from its true start state for the outputs.
+    // Segment-parallel path in two chunk passes.  One launch runs every
+    // segment from a zero state, writing its outputs and end state, and, in a
+    // second set of CTAs, the transition M with v = 0 from the identity,
+    // writing w_t = M_t^T q_t per token.  A serial combine turns the end
+    // states into true start states; the correction then adds S_start^T w_t
+    // to every output (the state map is affine: S_t = M_t S_start + S_t(0)).
     const int seg_len = ((nchunks + nseg - 1) / nseg) * C;
     nseg = (p.T + seg_len - 1) / seg_len;
     const size_t slab = (size_t)p.B * nseg * p.H * D * D;
+    const size_t wlen = (size_t)p.B * p.T * p.H * D;
     float* ws = nullptr;
-    cudaError_t e = workspace_alloc(reinterpret_cast<void**>(&ws), 2 * slab * sizeof(float), stream);
+    cudaError_t e = workspace_alloc(reinterpret_cast<void**>(&ws), (2 * slab + wlen) * sizeof(float), stream);
     if (e != cudaSuccess) return e;
     float* seg_states = ws;
     float* trans = ws + slab;
-    Params p1{p.g, p.beta, nullptr, seg_states, trans, nullptr, p.T, p.H, p.B, nseg, seg_len, 1, nseg};
-    chunk_fwd_kernel<CHANNEL><<<2 * p.B * nseg * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, p1);
+    float* wbuf = ws + 2 * slab;
+    CUtensorMap mw;
+    if (!make_out_map(&mw, wbuf, p.H, p.T, p.B)) {
+        const cudaError_t ef = cudaFreeAsync(ws, stream);
+        return ef != cudaSuccess ? ef : cudaErrorInvalidValue;
+    }
+    Params p1{p.g, p.beta, nullptr, seg_states, trans, out, p.T, p.H, p.B, nseg, seg_len, 1, nseg};
+    p1.wout = wbuf;
+    chunk_fwd_kernel<CHANNEL><<<2 * p.B * nseg * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mw, p1);
     e = cudaGetLastError();
     if (e == cudaSuccess) {
         combine_segments_kernel<<<p.B * p.H * (D / CB_COLS), 256, 0, stream>>>(
@@ -980,9 +1088,18 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
         e = cudaGetLastError();
     }
     if (e == cudaSuccess) {
-        Params p2{p.g, p.beta, seg_states, nullptr, nullptr, out, p.T, p.H, p.B, nseg, seg_len, nseg, 1};
-        chunk_fwd_kernel<CHANNEL><<<p.B * nseg * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, p2);
-        e = cudaGetLastError();
+        static bool corr_attr = false;
+        if (!corr_attr) {
+            e = cudaFuncSetAttribute(segment_correction_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)sizeof(CorrSmem));
+            corr_attr = e == cudaSuccess;
+        }
+        if (e == cudaSuccess) {
+            const int groups = (seg_len / C + CORR_TILES - 1) / CORR_TILES;
+            segment_correction_kernel<<<dim3(groups, nseg * p.H, p.B), 256, sizeof(CorrSmem), stream>>>(
+                seg_states, wbuf, out, p.T, p.H, nseg, seg_len);
+            e = cudaGetLastError();
+        }
     }
     const cudaError_t ef = cudaFreeAsync(ws, stream);
     return e != cudaSuccess ? e : ef;
@@ -1041,7 +1158,7 @@ cudaError_t launch_noalloc(const Problem& p, cudaStream_t stream, bool* over_lim
     if (nseg <= 1) {
         Params prm{p.g, p.beta, p.state_in, p.state_out, nullptr, out, p.T, p.H, p.B,
                    1, nchunks * C, 1, 1};
-        chunk_fwd_kernel<CHANNEL><<<p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, prm);
+        chunk_fwd_kernel<CHANNEL><<<p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mo, prm);
         return cudaGetLastError();
     }
     float* ws = nullptr;
@@ -1052,7 +1169,7 @@ cudaError_t launch_noalloc(const Problem& p, cudaStream_t stream, bool* over_lim
     float* seg_states = ws;
     float* trans = ws + slab;
     Params p1{p.g, p.beta, nullptr, seg_states, trans, nullptr, p.T, p.H, p.B, nseg, seg_len, 1, nseg};
-    chunk_fwd_kernel<CHANNEL><<<2 * p.B * nseg * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, p1);
+    chunk_fwd_kernel<CHANNEL><<<2 * p.B * nseg * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mo, p1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     combine_segments_kernel<<<p.B * p.H * (D / CB_COLS), 256, 0, stream>>>(
@@ -1060,7 +1177,7 @@ cudaError_t launch_noalloc(const Problem& p, cudaStream_t stream, bool* over_lim
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     Params p2{p.g, p.beta, seg_states, nullptr, nullptr, out, p.T, p.H, p.B, nseg, seg_len, nseg, 1};
-    chunk_fwd_kernel<CHANNEL><<<p.B * nseg * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, p2);
+    chunk_fwd_kernel<CHANNEL><<<p.B * nseg * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mo, p2);
     return cudaGetLastError();
 }
 
