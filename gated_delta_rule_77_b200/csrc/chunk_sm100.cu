@@ -1015,9 +1015,10 @@ int sm_count() {
     return n;
 }
 
-// Number of time segments per (batch, head).  Segmenting costs three chunk
-// passes (zero-start states, transitions, outputs) instead of one, so it pays
-// only when the (batch, head) pairs alone leave most SMs idle.
+// Number of time segments per (batch, head).  Segmenting costs two chunk
+// passes (zero-start states and outputs, transitions) and a correction
+// instead of one pass, so it pays only when the (batch, head) pairs alone
+// leave most SMs idle.
 int choose_segments(int requested, int BH, int nchunks) {
     if (nchunks <= 1 || requested == 1) return 1;
     int n = requested;

@@ -124,17 +124,19 @@ GDN_API int gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const 
  * sequence parallelism.  The state map of a stretch of tokens is affine,
  * S_end = M S_start + S_end(0) (it follows from the formula of section 2.1),
  * so a long sequence can be cut into num_segments time segments that run in
- * parallel: every segment computes its end state from a zero start and its
- * dk x dk transition M, a serial combine gives each segment its true start
- * state, and the segments run again from those states for the outputs.
- * This costs three chunk passes instead of one and pays off when B * H is
- * small against the SM count and T is long.
+ * parallel: every segment computes its outputs and end state from a zero
+ * start, and its dk x dk transition M with w_t = M_t^T q_t per token; a serial
+ * combine gives each segment its true start state, and a correction adds
+ * S_start^T w_t to every output.  This costs two chunk passes instead of one
+ * and pays off when B * H is small against the SM count and T is long.
+ * (gdn_chunk_fwd_segments_noalloc runs the segments a third time from their
+ * true starts instead, since w does not fit its fixed scratch.)
  *   num_segments 0 = automatic (what gdn_chunk_fwd does), 1 = none,
  *                n > 1 = n segments (at most one per 64-token chunk;
  *                dk = dv = 128 only).
- * Scratch: 2 * B * n * H * dk * dv * 4 bytes, stream-ordered on `stream`
- * from the library's pool (GDN_ERR_NOMEM if it cannot be had).  Other
- * arguments as gdn_chunk_fwd.
+ * Scratch: (2 * B * n * H * dk * dv + B * T * H * dk) * 4 bytes,
+ * stream-ordered on `stream` from the library's pool (GDN_ERR_NOMEM if it
+ * cannot be had).  Other arguments as gdn_chunk_fwd.
  */
 GDN_API int gdn_chunk_fwd_segments(const void* q, const void* k, const void* v, const float* g,
                                    const float* beta, const float* state_in, void* out,
