@@ -917,16 +917,21 @@ combine_segments_kernel(float* seg_states, const float* trans, const float* stat
 // Segment correction: out[b, t, h, :] += S_start(b, seg(t), h)^T w[b, t, h, :]
 // for every token of a segment, after the combine has produced the true start
 // states.  One CTA per group of CORR_TILES 64-token tiles of one (batch,
-// segment, head); the start state is held as bf16 hi + lo and read with
-// ldmatrix, each tile of w (tokens x key channels) is the split A operand,
-// on mma.sync (warp_mma.cuh).
+// segment, head).  The term is a correction of the zero-start output: its
+// products run single-pass in fp16 (about 2^-11 relative, inside the
+// prefill's error budget), the start state as one fp16 tile read with
+// ldmatrix, and the tiles of w (tokens x key channels) arrive through two
+// cp.async stages while the previous tile's products run.
 constexpr int CORR_TILES = 16;
 struct __align__(16) CorrSmem {
-    __nv_bfloat16 sh[D][D + 8];
-    __nv_bfloat16 sl[D][D + 8];
-    float w[C][D + 4];
+    __half s[D][D + 8];
+    float w[2][C][D + 4];
 };
-__global__ void __launch_bounds__(256)
+__device__ __forceinline__ void corr_cp16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                 :: "r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))), "l"(src) : "memory");
+}
+__global__ void __launch_bounds__(256, 2)
 segment_correction_kernel(const float* __restrict__ seg_states, const float* __restrict__ wbuf,
                           float* __restrict__ out, int T, int H, int nseg, int seg_len)
 {
@@ -938,43 +943,34 @@ segment_correction_kernel(const float* __restrict__ seg_states, const float* __r
     const int t_begin = seg * seg_len, t_end = min(T, t_begin + seg_len);
     const int tile0 = blockIdx.x * CORR_TILES;
     if (t_begin + tile0 * C >= t_end) return;
+    // Tile i's w into stage i & 1 (one commit group; rows past the segment zero).
+    auto fetch = [&](int i) {
+        const int t0 = t_begin + (tile0 + i) * C;
+        if (i < CORR_TILES && t0 < t_end) {
+            for (int idx = tid; idx < C * D / 4; idx += 256) {
+                const int r = idx / (D / 4), q4 = 4 * (idx % (D / 4));
+                float* dst = &m.w[i & 1][r][q4];
+                if (t0 + r < t_end) corr_cp16(dst, wbuf + (((long)b * T + t0 + r) * H + h) * D + q4);
+                else *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    fetch(0);
     const float* src = seg_states + (((long)b * nseg + seg) * H + h) * (long)(D * D);
     for (int idx = tid; idx < D * D / 4; idx += 256) {
         const int r = idx / (D / 4), q4 = 4 * (idx % (D / 4));
         const float4 x = *reinterpret_cast<const float4*>(src + (long)r * D + q4);
-        uint32_t h0, l0, h1, l1;
-        split2(x.x, x.y, h0, l0);
-        split2(x.z, x.w, h1, l1);
-        *reinterpret_cast<uint2*>(&m.sh[r][q4]) = make_uint2(h0, h1);
-        *reinterpret_cast<uint2*>(&m.sl[r][q4]) = make_uint2(l0, l1);
+        *reinterpret_cast<uint2*>(&m.s[r][q4]) = make_uint2(pack_f16x2(x.x, x.y), pack_f16x2(x.z, x.w));
     }
     const int rb = (warp >> 1) * 16, cb = (warp & 1) * 64;
     const int l = tid & 31, g = l >> 2, t4 = l & 3;
-    // Software pipeline in registers: tile i + 1's w and tile i's outputs are
-    // loaded while tile i's products run.
-    constexpr int WPT = C * D / 4 / 256;     // float4 of a w tile per thread
-    float4 wreg[WPT];
-    auto load_w = [&](int t0) {
-#pragma unroll
-        for (int it = 0; it < WPT; ++it) {
-            const int idx = tid + it * 256;
-            const int r = idx / (D / 4), q4 = 4 * (idx % (D / 4));
-            wreg[it] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (t0 + r < t_end) wreg[it] = *reinterpret_cast<const float4*>(wbuf + (((long)b * T + t0 + r) * H + h) * D + q4);
-        }
-    };
-    load_w(t_begin + tile0 * C);
     for (int i = 0; i < CORR_TILES; ++i) {
         const int t0 = t_begin + (tile0 + i) * C;
         if (t0 >= t_end) break;
-        __syncthreads();                     // the previous tile's w is consumed
-#pragma unroll
-        for (int it = 0; it < WPT; ++it) {
-            const int idx = tid + it * 256;
-            *reinterpret_cast<float4*>(&m.w[idx / (D / 4)][4 * (idx % (D / 4))]) = wreg[it];
-        }
-        __syncthreads();
-        // This tile's outputs, then the next tile's w, both in flight during the products.
+        fetch(i + 1);                                   // the other stage is free (barrier below)
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+        __syncthreads();                                // tile i's w is in
         float2 ov[8][2];
 #pragma unroll
         for (int j = 0; j < 8; ++j)
@@ -985,12 +981,10 @@ segment_correction_kernel(const float* __restrict__ seg_states, const float* __r
                 if (t0 + r < t_end)
                     ov[j][e2] = *reinterpret_cast<const float2*>(out + (((long)b * T + t0 + r) * H + h) * D + cb + 8 * j + 2 * t4);
             }
-        const int tn = t0 + C;
-        if (i + 1 < CORR_TILES && tn < t_end) load_w(tn);
         float acc[8][4];
         zero_acc(acc);
-        wmm_sb<8, D, true, D + 8>(acc, rb, cb, [&](int r, int k) { return m.w[r][k]; },
-                                  &m.sh[0][0], &m.sl[0][0]);
+        const float (*wt)[D + 4] = m.w[i & 1];
+        wmm_f16<8, D, true, D + 8>(acc, rb, cb, [&](int r, int k) { return wt[r][k]; }, &m.s[0][0]);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
 #pragma unroll
@@ -1001,7 +995,9 @@ segment_correction_kernel(const float* __restrict__ seg_states, const float* __r
                     *o = make_float2(ov[j][e2].x + acc[j][2 * e2], ov[j][e2].y + acc[j][2 * e2 + 1]);
                 }
             }
+        __syncthreads();                                // stage i & 1 is consumed
     }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 int sm_count() {

@@ -5,6 +5,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace gdn {
@@ -110,6 +111,46 @@ __device__ __forceinline__ void wmm_sb(float (&acc)[NT][4], int rb, int cb, FA a
         for (int j = 0; j < NT; ++j) mma16816(acc[j], ah, blv[j / 2][2 * (j & 1)], blv[j / 2][2 * (j & 1) + 1]);
 #pragma unroll
         for (int j = 0; j < NT; ++j) mma16816(acc[j], al, bhv[j / 2][2 * (j & 1)], bhv[j / 2][2 * (j & 1) + 1]);
+    }
+}
+
+// Single-pass fp16 variant (about 2^-11 relative per product), for terms
+// whose error budget allows it: A from fp32 through an accessor, converted
+// to fp16 pairs; B from an fp16 tile of row length LD via ldmatrix (TRANS:
+// B(k, n) = tile[k][n], else tile[n][k]).
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    const __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+__device__ __forceinline__ void mma16816_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+template <int NT, int K, bool TRANS, int LD, typename FA>
+__device__ __forceinline__ void wmm_f16(float (&acc)[NT][4], int rb, int cb, FA a, const __half* bt) {
+    static_assert(NT % 2 == 0, "pairs of 8-column tiles");
+    const int l = threadIdx.x & 31, g = l >> 2, t = l & 3;
+    const int mi = l >> 3, rr = l & 7;
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 16) {
+        uint32_t af[4];
+        af[0] = pack_f16x2(a(rb + g, k0 + 2 * t), a(rb + g, k0 + 2 * t + 1));
+        af[1] = pack_f16x2(a(rb + g + 8, k0 + 2 * t), a(rb + g + 8, k0 + 2 * t + 1));
+        af[2] = pack_f16x2(a(rb + g, k0 + 2 * t + 8), a(rb + g, k0 + 2 * t + 9));
+        af[3] = pack_f16x2(a(rb + g + 8, k0 + 2 * t + 8), a(rb + g + 8, k0 + 2 * t + 9));
+#pragma unroll
+        for (int jp = 0; jp < NT / 2; ++jp) {
+            const int n0 = cb + 16 * jp;
+            long off;
+            if (TRANS) off = (long)(k0 + rr + 8 * (mi & 1)) * LD + n0 + 8 * (mi >> 1);
+            else off = (long)(n0 + rr + 8 * (mi >> 1)) * LD + k0 + 8 * (mi & 1);
+            uint32_t bv[4];
+            if (TRANS) ldsm4t(bv, bt + off); else ldsm4(bv, bt + off);
+            mma16816_f16(acc[2 * jp], af, bv[0], bv[1]);
+            mma16816_f16(acc[2 * jp + 1], af, bv[2], bv[3]);
+        }
     }
 }
 
