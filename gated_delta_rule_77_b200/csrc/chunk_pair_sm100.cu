@@ -1,5 +1,5 @@
 // chunk_pair_sm100.cu -- chunkwise prefill with the work of one (batch, head)
-// split across a cluster of two CTAs on two SMs.
+// split between a "prep" CTA and a "chain" CTA on two SMs.
 //
 // Same chunk algebra as chunk_sm100.cu (Atomic-GDN2 model card, section 2.1;
 // chunkwise mode of the "Gated DeltaNet" entity trail, finding of
@@ -19,12 +19,28 @@
 //                    operands K*E, Q*E, K*D, and the state-dependent products
 //                    W^T, U^T, O^T and SN; writes the outputs.
 //
-// Hand-off: CTA 1's "full" mbarrier (armed by CTA 0 with a remote
-// arrive.expect_tx, completed by the bulk copy's byte count) and CTA 0's
-// "empty" mbarrier (a remote arrive from CTA 1 once the products that read the
-// slot are complete).  CTA 0 therefore works on chunk c + 1 while CTA 1 works
-// on chunk c.  Every wait is bounded (kWaitBudgetNs); on expiry a CTA records
-// it in its status word, stops, drains its own copies and returns.
+// Two launch forms share the code of both roles:
+//
+// chunk_pair_kernel, a cluster of two CTAs per (batch, head).  Hand-off: CTA
+//   1's "full" mbarrier (armed by CTA 0 with a remote arrive.expect_tx,
+//   completed by the bulk copy's byte count) and CTA 0's "empty" mbarrier (a
+//   remote arrive from CTA 1 once the products that read the slot are
+//   complete).  CTA 0 therefore works on chunk c + 1 while CTA 1 works on
+//   chunk c.
+//
+// chunk_pool_kernel, a cooperative grid of one CTA per SM: B*H chain CTAs and
+//   every other SM a prep CTA.  The prep CTAs share the (batch, head, chunk)
+//   tasks, chunk-major (task i: chunk i / (B*H), pair i % (B*H); CTA j takes
+//   tasks j, j + n_prep, ...), store each 32 KB slot to a global buffer with
+//   one bulk copy and set the task's flag (release).  A chain CTA polls the
+//   flag of its next chunk (acquire; tried early in the chunk, when the slot is
+//   also prefetched into L2) and fetches the slot with one bulk copy onto its
+//   "full" mbarrier as soon as the previous slot is consumed.  With more prep
+//   CTAs than chains, the chain no longer waits on a single prep CTA, and the
+//   SMs that a cluster per pair leaves idle do prep work.
+//
+// Every wait is bounded (kWaitBudgetNs); on expiry a CTA records it in its
+// status word, stops, drains its own copies and returns.
 //
 // Precision and operand formats are those of chunk_sm100.cu (bf16 hi + lo for
 // the factored A/P operands, T', P, U and K*D; fp16 for S, W and Q*E; fp32
@@ -101,7 +117,8 @@ constexpr uint32_t C_GAM = C_SMALL;           // 64 f32
 constexpr uint32_t C_LAST = C_GAM + 256;      // 128 f32
 constexpr uint32_t C_BAR = C_LAST + 512;      // tma_kq, tma_v, mma, full, out
 constexpr uint32_t C_TMEM = C_BAR + 40;
-constexpr uint32_t C_USED = C_TMEM + 8;
+constexpr uint32_t C_FETCHED = C_TMEM + 8;    // int: slots fetched (pool form)
+constexpr uint32_t C_USED = C_FETCHED + 8;
 
 constexpr uint32_t SLOT_BYTES = 32768;
 constexpr uint32_t SMEM_BYTES = (P_USED > C_USED ? P_USED : C_USED) + 1024;
@@ -116,14 +133,15 @@ struct PairParams {
     const float* state_in;     // [B, H, D, D] or null
     float* state_out;          // [B, H, D, D] or null
     float* out;                // [B, T, H, D] fp32
-    int T, H;
+    int T, H, B;
+    uint8_t* slots;            // pool form: [B*H][chunks][SLOT_BYTES]
+    unsigned int* flags;       // pool form: [B*H][chunks], zero at launch
 };
 
-template <bool CHANNEL>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
-chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                  const __grid_constant__ CUtensorMap tm_g, const PairParams p)
+template <bool CHANNEL, bool POOL>
+__device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                                          const CUtensorMap& tm_v, const CUtensorMap& tm_o,
+                                          const CUtensorMap& tm_g, const PairParams& p)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -134,10 +152,13 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int lane = tid & 31;
     const int quad = warp & 3;
     const int half = warp >> 2;
-    const uint32_t rank = cluster_ctarank();
     const int T = p.T;
     const int H = p.H;
-    const int pair = blockIdx.x >> 1;
+    const int nbh = p.B * H;
+    // Role: rank 0 = prep, 1 = chain.  Pool form: CTAs 0 .. B*H-1 are the
+    // chains (one per pair), the rest prep CTAs.
+    const uint32_t rank = POOL ? ((int)blockIdx.x < nbh ? 1u : 0u) : cluster_ctarank();
+    const int pair = POOL ? (rank ? (int)blockIdx.x : 0) : (int)(blockIdx.x >> 1);
     const int h = pair % H;
     const int b = pair / H;
     const int nchunks = (T + C - 1) / C;
@@ -172,7 +193,7 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<uint32_t*>(smem + (rank == 0 ? P_TMEM : C_TMEM));
-    cluster_sync();
+    if (!POOL) cluster_sync();
 
     uint32_t mma_phase = 0;
     auto mma_sync = [&]() {
@@ -249,11 +270,11 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // Scalar gate and beta, warp 0: lane holds tokens lane and 32 + lane.
     // gate_scalar_load reads them into registers; gate_scalar scans g into
     // sGam (and stores beta when sBeta is given).
-    auto gate_scalar_load = [&](int chunk, bool with_beta, float (&bg)[4]) {
+    auto gate_scalar_load = [&](int bb, int hh, int chunk, bool with_beta, float (&bg)[4]) {
         bg[0] = bg[1] = bg[2] = bg[3] = 0.f;
         if (warp != 0) return;
         const int t0 = chunk * C;
-        const long tk0 = ((long)b * T + t0) * H + h;
+        const long tk0 = ((long)bb * T + t0) * H + hh;
         if (t0 + lane < T) {
             if (with_beta) bg[0] = p.beta[tk0 + (long)lane * H];
             if (!CHANNEL) bg[2] = p.g[tk0 + (long)lane * H];
@@ -316,25 +337,59 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         float* sY = reinterpret_cast<float*>(smem + P_Y);
         const uint32_t bar_tma = sbase + P_BAR, bar_empty = sbase + P_BAR + 16;
         const uint32_t bar_g = sbase + P_BAR + 24;
-        // CTA 1's slot and "full" barrier, as cluster addresses.
-        const uint32_t peer_slot = mapa_shared(sbase + C_SLOT, 1);
-        const uint32_t peer_full = mapa_shared(sbase + C_BAR + 24, 1);
-        auto issue_kq = [&](int chunk) {
-            const int t0 = chunk * C;
+        // Cluster form: CTA 1's slot and "full" barrier, as cluster addresses.
+        const uint32_t peer_slot = POOL ? 0u : mapa_shared(sbase + C_SLOT, 1);
+        const uint32_t peer_full = POOL ? 0u : mapa_shared(sbase + C_BAR + 24, 1);
+        // The items this CTA prepares, in order: the chunks of its pair
+        // (cluster form) or its share of the chunk-major task list (pool).
+        const int nprep = POOL ? (int)gridDim.x - nbh : 1;
+        const int pid = POOL ? (int)blockIdx.x - nbh : 0;
+        const int ntasks = nbh * nchunks;
+        const int nitems = POOL ? (pid < ntasks ? (ntasks - pid + nprep - 1) / nprep : 0) : nchunks;
+        auto item = [&](int j, int& ib, int& ih, int& ic) {
+            if (POOL) {
+                const int task = pid + j * nprep;
+                ic = task / nbh;
+                const int pr = task - ic * nbh;
+                ib = pr / H;
+                ih = pr - ib * H;
+            } else {
+                ib = b; ih = h; ic = j;
+            }
+        };
+        auto issue_kq = [&](int j) {
+            int ib, ih, ic;
+            item(j, ib, ih, ic);
             mbar_expect_tx(bar_tma, 2 * 16384);
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-                tma_load_4d(sbase + P_IN + hf * 16384, &tm_k, hf * 64, h, t0, b, bar_tma);
-                tma_load_4d(sbase + P_IN + hf * 16384 + 8192, &tm_q, hf * 64, h, t0, b, bar_tma);
+                tma_load_4d(sbase + P_IN + hf * 16384, &tm_k, hf * 64, ih, ic * C, ib, bar_tma);
+                tma_load_4d(sbase + P_IN + hf * 16384 + 8192, &tm_q, hf * 64, ih, ic * C, ib, bar_tma);
             }
         };
-        // Per-channel g: chunk c + 1 arrives by TMA while chunk c's operands
-        // are built, and is scanned while chunk c's X product runs.
-        auto issue_g = [&](int chunk) {
+        // Per-channel g: item j + 1's arrives by TMA while item j's operands
+        // are built, and is scanned while item j's X product runs.
+        auto issue_g = [&](int j) {
+            int ib, ih, ic;
+            item(j, ib, ih, ic);
             mbar_expect_tx(bar_g, 32768);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                tma_load_4d(sbase + P_G + i * 8192, &tm_g, 32 * i, h, chunk * C, b, bar_g);
+                tma_load_4d(sbase + P_G + i * 8192, &tm_g, 32 * i, ih, ic * C, ib, bar_g);
+        };
+        auto beta_load = [&](int j, float (&bg)[4]) {
+            int ib, ih, ic;
+            item(j, ib, ih, ic);
+            gate_scalar_load(ib, ih, ic, true, bg);
+        };
+        // Pool form: the slot of the last item stored, published (its flag
+        // set) once the store is complete.
+        unsigned int* pending_flag = nullptr;
+        auto publish = [&]() {
+            bulk_wait_all();
+            fence_proxy_async_global();
+            flag_release(pending_flag, 1u);
+            pending_flag = nullptr;
         };
         int g_issued = 0, g_waited = 0;          // g loads issued / waited for
         auto scan_g = [&](float (&gn)[4][8]) {   // wait, read this thread's values, scan
@@ -351,19 +406,19 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             gate_scan(gn, sRef0, sRef1, nullptr);
         };
-        if (tid == 0 && nchunks > 0) issue_kq(0);
+        if (tid == 0 && nitems > 0) issue_kq(0);
         int kq_waited = -1;
         bool copy_pending = false;
         float gnext[4][8], bgnext[4];
-        if (CHANNEL && nchunks > 0) {
+        if (CHANNEL && nitems > 0) {
             if (tid == 0) { issue_g(0); g_issued = 1; }
             scan_g(gnext);
-            __syncthreads();                      // chunk 0's g has been read
-            if (tid == 0 && nchunks > 1) { issue_g(1); g_issued = 2; }
+            __syncthreads();                      // item 0's g has been read
+            if (tid == 0 && nitems > 1) { issue_g(1); g_issued = 2; }
         }
-        if (nchunks > 0) gate_scalar_load(0, true, bgnext);
+        if (nitems > 0) beta_load(0, bgnext);
 
-        for (int ci = 0; ci < nchunks; ++ci) {
+        for (int ci = 0; ci < nitems; ++ci) {
             float gam[4][8];
             if (CHANNEL) {   // scanned one chunk ahead; sRef0/1 hold this chunk's
 #pragma unroll
@@ -373,7 +428,7 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             // beta (and a scalar g) were loaded one chunk ahead.
             gate_scalar(bgnext, sGam, sBeta, sEr, sFj, sSafe);
-            if (CHANNEL && ci + 1 < nchunks) gate_scalar_load(ci + 1, true, bgnext);
+            if (CHANNEL && ci + 1 < nitems) beta_load(ci + 1, bgnext);
             ok = ok && mbar_wait(bar_tma, ci & 1, &g_pair_status_word);
             kq_waited = ci;
             if (__syncthreads_or(!ok)) break;
@@ -455,18 +510,18 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             // While X runs: the next chunk's g (the X build of this chunk has
             // read sRef0/1 already).
-            if (CHANNEL && ci + 1 < nchunks) scan_g(gnext);
+            if (CHANNEL && ci + 1 < nitems) scan_g(gnext);
             mma_sync();
             if (tid == 0 && copy_pending) {      // the staging is free again
-                bulk_wait_read_all();
+                if (POOL) publish(); else bulk_wait_read_all();
                 copy_pending = false;
             }
             if (__syncthreads_or(!ok)) break;
-            // Raw K, Q and the X operands are consumed: prefetch the next chunk;
+            // Raw K, Q and the X operands are consumed: prefetch the next item;
             // the g tile has been read by every thread.
-            if (tid == 0 && ci + 1 < nchunks) issue_kq(ci + 1);
-            if (CHANNEL && tid == 0 && ci + 2 < nchunks) { issue_g(ci + 2); g_issued = ci + 3; }
-            if (!CHANNEL && ci + 1 < nchunks) gate_scalar_load(ci + 1, true, bgnext);
+            if (tid == 0 && ci + 1 < nitems) issue_kq(ci + 1);
+            if (CHANNEL && tid == 0 && ci + 2 < nitems) { issue_g(ci + 2); g_issued = ci + 3; }
+            if (!CHANNEL && ci + 1 < nitems) beta_load(ci + 1, bgnext);
 
             // A and P from X (see chunk_sm100.cu); P as bf16 hi + lo into the staging.
             {
@@ -546,7 +601,7 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             fence_async_smem();          // staging written by threads -> read by the bulk copy
             __syncthreads();
-            if (tid == 0) {
+            if (tid == 0 && !POOL) {
                 // Wait until CTA 1 has consumed the previous chunk's slot.
                 ok = ok && mbar_wait_cluster(bar_empty, (ci & 1) ^ 1, &g_pair_status_word);
                 if (ok) {
@@ -556,11 +611,29 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     copy_pending = true;
                 }
             }
+            if (tid == 0 && POOL) {
+                // The slot to the task's place in the global buffer; its flag
+                // is set once the store is complete (at once for the first
+                // item, which the chains wait for; otherwise after the next
+                // item's X product, when the store has long finished).
+                int ib, ih, ic;
+                item(ci, ib, ih, ic);
+                const size_t task = (size_t)(ib * H + ih) * nchunks + ic;
+                bulk_store_global(p.slots + task * SLOT_BYTES, sbase + P_STAGE, SLOT_BYTES);
+                bulk_commit();
+                pending_flag = p.flags + task;
+                copy_pending = true;
+                if (ci == 0) {
+                    publish();
+                    copy_pending = false;
+                }
+            }
             if (__syncthreads_or(!ok)) break;
         }
         if (tid == 0) {
             bulk_wait_all();                 // own copies complete before exit
-            if (!ok && kq_waited + 1 < nchunks)
+            if (POOL && pending_flag) publish();
+            if (!ok && kq_waited + 1 < nitems)
                 mbar_wait(bar_tma, (kq_waited + 1) & 1, &g_pair_status_word);
             for (int i = g_waited; !ok && i < g_issued; ++i)   // g tiles still in flight
                 mbar_wait(bar_g, i & 1, &g_pair_status_word);
@@ -575,7 +648,35 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         // Products into O^T are committed apart (bar_out), so that the U
         // epilogue and the state update do not wait for them.
         const uint32_t bar_out = sbase + C_BAR + 32;
-        const uint32_t peer_empty = mapa_shared(sbase + P_BAR + 16, 0);
+        const uint32_t peer_empty = POOL ? 0u : mapa_shared(sbase + P_BAR + 16, 0);
+        // Pool form: chunk c's slot is fetched from the global buffer with one
+        // bulk copy onto bar_full once chunk c - 1's products have read the
+        // previous slot.  Its flag is tried early in chunk c - 1 by the same
+        // thread, without blocking; when set, the slot is also prefetched into
+        // L2 (prep CTAs may run far ahead of the chains, and slots written
+        // long before have left L2).  The count of fetches issued is kept in
+        // shared memory for the drain on an abandoned wait.
+        int* sFetched = reinterpret_cast<int*>(smem + C_FETCHED);
+        int acquired = -1;              // chunk whose flag this thread has acquired
+        auto try_acquire = [&](int chunk) {
+            const size_t task = (size_t)pair * nchunks + chunk;
+            if (flag_acquire(p.flags + task) == 0) return;
+            fence_proxy_async_global();
+            bulk_prefetch_l2(p.slots + task * SLOT_BYTES, SLOT_BYTES);
+            acquired = chunk;
+        };
+        auto fetch_slot = [&](int chunk) {
+            const size_t task = (size_t)pair * nchunks + chunk;
+            if (acquired != chunk) {
+                ok = ok && flag_wait(p.flags + task, &g_pair_status_word);
+                if (!ok) return;
+                fence_proxy_async_global();
+            }
+            mbar_expect_tx(bar_full, SLOT_BYTES);
+            bulk_load_global(sbase + C_SLOT, p.slots + task * SLOT_BYTES, SLOT_BYTES, bar_full);
+            *sFetched = chunk + 1;
+        };
+        if (POOL && tid == 0) *sFetched = 0;
 
         const int srow = quad * 32 + lane;
         const int scol = half * 64;
@@ -624,10 +725,13 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         int kq_waited = -1, v_waited = -1, full_waited = -1;
         float gnext[4][8], bgnext[4];
         if (CHANNEL && nchunks > 0) gate_load(0, gnext);
-        if (!CHANNEL && nchunks > 0) gate_scalar_load(0, false, bgnext);
+        if (!CHANNEL && nchunks > 0) gate_scalar_load(b, h, 0, false, bgnext);
         // Per-channel: chunk 0's scan here; the scan of chunk c + 1 runs
         // while the products SN of chunk c are on the tensor core.
         if (CHANNEL && nchunks > 0) gate_channel(0, (long)b * T * H + h, gnext, nullptr, nullptr, sLast);
+        // The first slot: its flag is waited for after this thread's gate
+        // loads have been issued and used.
+        if (POOL && tid == 0 && nchunks > 0) fetch_slot(0);
 
         for (int ci = 0; ci < nchunks; ++ci) {
             const int t0 = ci * C;
@@ -696,12 +800,13 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (tid == 0 && ci + 1 < nchunks) issue_kq(ci + 1);   // raw K, Q consumed
             if (ci + 1 < nchunks) {
                 if (CHANNEL) gate_load(ci + 1, gnext);
-                else gate_scalar_load(ci + 1, false, bgnext);
+                else gate_scalar_load(b, h, ci + 1, false, bgnext);
             }
 
-            // T' and P of this chunk from CTA 0; V of this chunk.
+            // T' and P of this chunk from the prep side; V of this chunk.
             if (tid == 0) {
-                ok = ok && mbar_wait_cluster(bar_full, ci & 1, &g_pair_status_word);
+                ok = ok && (POOL ? mbar_wait(bar_full, ci & 1, &g_pair_status_word)
+                                 : mbar_wait_cluster(bar_full, ci & 1, &g_pair_status_word));
                 full_waited = ci;
             }
             ok = ok && mbar_wait(bar_v, ci & 1, &g_pair_status_word);
@@ -724,6 +829,8 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
                 mma_commit(bar_mma);
             }
+            // Pool form: the next chunk's flag, tried while these products run.
+            if (POOL && tid == NT - 32 && ci + 1 < nchunks) try_acquire(ci + 1);
             mma_sync();
             if (__syncthreads_or(!ok)) break;
             if (tid == 0 && ci + 1 < nchunks) issue_v(ci + 1);      // V consumed
@@ -822,10 +929,13 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
                 write_state_f16();
                 // Products into O^T complete (they read P in the slot and U^T):
-                // the slot goes back to CTA 0.  The arrive is made by a thread
-                // of the last warp, which has no global loads in flight.
+                // the slot is free.  Cluster form: it goes back to CTA 0 (the
+                // arrive is made by a thread of the last warp, which has no
+                // global loads in flight).  Pool form: the same thread fetches
+                // the next chunk's slot.
                 ok = ok && mbar_wait(bar_out, ci & 1, &g_pair_status_word);
-                if (tid == NT - 32 && ok) mbar_arrive_remote_relaxed(peer_empty);
+                if (!POOL && tid == NT - 32 && ok) mbar_arrive_remote_relaxed(peer_empty);
+                if (POOL && tid == NT - 32 && ok && ci + 1 < nchunks) fetch_slot(ci + 1);
                 tc_fence_after();
                 float o[32];
                 tmem_ld32(lb + TM_OT + half * 32, o);
@@ -846,14 +956,16 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
         }
         if (tid == 0) bulk_wait_all();       // output stores complete before exit
-        if (tid == 0 && !ok) {   // drain this CTA's own loads and products (bounded)
+        const bool failed = __syncthreads_or(!ok);
+        if (tid == 0 && failed) {   // drain this CTA's own loads and products (bounded)
             if (kq_waited + 1 < nchunks) mbar_wait(bar_kq, (kq_waited + 1) & 1, &g_pair_status_word);
             if (v_waited + 1 < nchunks) mbar_wait(bar_v, (v_waited + 1) & 1, &g_pair_status_word);
+            if (POOL && *sFetched > full_waited + 1)   // a slot fetch still in flight
+                mbar_wait(bar_full, (full_waited + 1) & 1, &g_pair_status_word);
             mma_commit(bar_mma);
             mbar_wait(bar_mma, mma_phase, &g_pair_status_word);
-            (void)full_waited;
         }
-        if (ok && p.state_out) {
+        if (!failed && p.state_out) {
             float4* dst = reinterpret_cast<float4*>(p.state_out + ((long)b * H + h) * DD +
                                                     (long)srow * D + scol);
 #pragma unroll
@@ -861,14 +973,33 @@ chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
     }
 
-    // Neither CTA leaves while the other may still touch its shared memory.
+    // Neither CTA of a cluster leaves while the other may still touch its
+    // shared memory.
     tc_fence_before();
     __syncthreads();
-    cluster_sync();
+    if (!POOL) cluster_sync();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, tmem_cols);
     }
+}
+
+template <bool CHANNEL>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
+chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  const __grid_constant__ CUtensorMap tm_g, const PairParams p)
+{
+    pair_body<CHANNEL, false>(tm_q, tm_k, tm_v, tm_o, tm_g, p);
+}
+
+template <bool CHANNEL>
+__global__ void __launch_bounds__(NT, 1)
+chunk_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  const __grid_constant__ CUtensorMap tm_g, const PairParams p)
+{
+    pair_body<CHANNEL, true>(tm_q, tm_k, tm_v, tm_o, tm_g, p);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -926,11 +1057,14 @@ bool make_map(CUtensorMap* map, const void* base, int H, int T, int B) {
 }
 
 template <bool CHANNEL>
-cudaError_t launch_pair(const Problem& p, cudaStream_t stream) {
+cudaError_t launch_pair(const Problem& p, cudaStream_t stream, int pool_ctas) {
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(chunk_pair_kernel<CHANNEL>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(chunk_pool_kernel<CHANNEL>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
@@ -943,16 +1077,55 @@ cudaError_t launch_pair(const Problem& p, cudaStream_t stream) {
     } else {
         mg = mq;                                   // not read with a scalar gate
     }
-    PairParams prm{p.g, p.beta, p.state_in, p.state_out, static_cast<float*>(p.out), p.T, p.H};
-    chunk_pair_kernel<CHANNEL><<<2 * p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mg, prm);
-    return cudaGetLastError();
+    PairParams prm{p.g, p.beta, p.state_in, p.state_out, static_cast<float*>(p.out), p.T, p.H, p.B,
+                   nullptr, nullptr};
+    const int nbh = p.B * p.H;
+    const int nchunks = (p.T + C - 1) / C;
+    if (pool_ctas <= nbh || nchunks == 0) {
+        chunk_pair_kernel<CHANNEL><<<2 * nbh, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mg, prm);
+        return cudaGetLastError();
+    }
+    // Pool form: flags, then the slots (1 KB aligned), from the stream-ordered
+    // workspace; the flags are cleared on the stream before the launch.
+    const size_t ntasks = (size_t)nbh * nchunks;
+    const size_t flag_bytes = (ntasks * sizeof(unsigned int) + 1023) / 1024 * 1024;
+    uint8_t* ws = nullptr;
+    cudaError_t e = workspace_alloc(reinterpret_cast<void**>(&ws), flag_bytes + ntasks * SLOT_BYTES, stream);
+    if (e != cudaSuccess) return e;
+    prm.flags = reinterpret_cast<unsigned int*>(ws);
+    prm.slots = ws + flag_bytes;
+    e = cudaMemsetAsync(ws, 0, ntasks * sizeof(unsigned int), stream);
+    if (e == cudaSuccess) {
+        // Cooperative: every CTA is resident at once (the chains wait on prep
+        // CTAs), or the launch fails instead of starting.
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(pool_ctas);
+        cfg.blockDim = dim3(NT);
+        cfg.dynamicSmemBytes = SMEM_BYTES;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, chunk_pool_kernel<CHANNEL>, mq, mk, mv, mo, mg, prm);
+        if (e == cudaErrorCooperativeLaunchTooLarge) {   // fewer SMs free: a cluster per pair
+            (void)cudaGetLastError();
+            prm.slots = nullptr;
+            prm.flags = nullptr;
+            chunk_pair_kernel<CHANNEL><<<2 * nbh, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mg, prm);
+            e = cudaGetLastError();
+        }
+    }
+    const cudaError_t ef = cudaFreeAsync(ws, stream);
+    return e != cudaSuccess ? e : ef;
 }
 
 }  // namespace
 
-cudaError_t launch_chunk_pair_sm100(const Problem& p, cudaStream_t stream) {
+cudaError_t launch_chunk_pair_sm100(const Problem& p, cudaStream_t stream, int pool_ctas) {
     if (p.io_f32 || !p.out_f32 || p.dk != D || p.dv != D) return cudaErrorNotSupported;
-    return p.per_channel ? launch_pair<true>(p, stream) : launch_pair<false>(p, stream);
+    return p.per_channel ? launch_pair<true>(p, stream, pool_ctas) : launch_pair<false>(p, stream, pool_ctas);
 }
 
 cudaError_t read_and_clear_pair_status(unsigned int* status) {

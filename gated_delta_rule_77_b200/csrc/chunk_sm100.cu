@@ -1043,12 +1043,15 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
     const int nchunks = (p.T + C - 1) / C;
     int nseg = choose_segments(p.segments, p.B * p.H, nchunks);
     if (nseg <= 1) {
-        // Two SMs per (batch, head) when they fit: chunk-local work overlaps the
-        // state chain.  GDN_CHUNK_KERNEL=single|pair overrides (tests, tuning).
+        // Chunk-local work and the state chain on different SMs when two per
+        // (batch, head) fit: by default one prep pool over all SMs; a cluster
+        // per pair with GDN_CHUNK_KERNEL=pair, one CTA per pair with =single
+        // (tests, tuning).
         const char* force = getenv("GDN_CHUNK_KERNEL");
-        const bool pair = force ? (strcmp(force, "pair") == 0)
-                                : (2 * p.B * p.H <= sm_count());
-        if (pair) return launch_chunk_pair_sm100(p, stream);
+        const bool split = force ? (strcmp(force, "pair") == 0 || strcmp(force, "pool") == 0)
+                                 : (2 * p.B * p.H <= sm_count());
+        const bool pool = !force || strcmp(force, "pool") == 0;
+        if (split) return launch_chunk_pair_sm100(p, stream, pool ? sm_count() : 0);
         Params prm{p.g, p.beta, p.state_in, p.state_out, nullptr, out, p.T, p.H, p.B,
                    1, nchunks * C, 1, 1};
         chunk_fwd_kernel<CHANNEL><<<p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mo, prm);

@@ -74,10 +74,14 @@ cudaError_t launch_chunk_sm100(const Problem& p, cudaStream_t stream);
 constexpr size_t kNoAllocScratchFloats = size_t(8) * 1024 * 1024;   // 32 MiB
 cudaError_t launch_chunk_sm100_noalloc(const Problem& p, cudaStream_t stream, bool* over_limit);
 
-// The same chunk algebra with each (batch, head) on a cluster of two CTAs:
-// one computes A, P and T' for chunk c + 1 while the other runs the state
-// chain of chunk c.  Used for unsegmented calls when 2 * B * H <= #SMs.
-cudaError_t launch_chunk_pair_sm100(const Problem& p, cudaStream_t stream);
+// The same chunk algebra with the chunk-local work (A, P, T') and the state
+// chain of each (batch, head) on different SMs.  pool_ctas <= B * H: a
+// cluster of two CTAs per pair (one prepares chunk c + 1 while the other runs
+// the chain of chunk c).  pool_ctas > B * H: one cooperative grid of that
+// many CTAs, B * H chains and the rest prep CTAs that share every pair's
+// chunks through a global slot buffer.  Used for unsegmented calls when
+// 2 * B * H <= #SMs.
+cudaError_t launch_chunk_pair_sm100(const Problem& p, cudaStream_t stream, int pool_ctas);
 cudaError_t read_and_clear_pair_status(unsigned int* status);
 
 // The layer's input prologue (prologue.cu): width-4 causal convolution over

@@ -154,6 +154,64 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t
         : "memory");
 }
 
+// Bulk copy (no multicast) of this CTA's shared memory to global memory,
+// tracked by this thread's bulk groups.  Addresses 16-byte aligned, size a
+// multiple of 16.
+__device__ __forceinline__ void bulk_store_global(void* dst, uint32_t src_local, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 ::"l"(reinterpret_cast<uint64_t>(dst)), "r"(src_local), "r"(bytes)
+                 : "memory");
+}
+
+// Bulk copy (no multicast) of global memory into this CTA's shared memory;
+// completion is counted in bytes on this CTA's mbarrier.
+__device__ __forceinline__ void bulk_load_global(uint32_t dst_local, const void* src, uint32_t bytes,
+                                                 uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst_local), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+// Asks for `bytes` of global memory to be brought into L2 (no data returned).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
+                 ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+                 : "memory");
+}
+
+// Orders this thread's global accesses between the generic and async proxies.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// A flag in global memory that another CTA of the same launch sets.
+__device__ __forceinline__ void flag_release(unsigned int* flag, unsigned int v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(flag)), "r"(v)
+                 : "memory");
+}
+
+__device__ __forceinline__ unsigned int flag_acquire(const unsigned int* flag) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(reinterpret_cast<uint64_t>(flag))
+                 : "memory");
+    return v;
+}
+
+// Bounded wait until *flag != 0 (acquire).  Returns false (and sets bit 0 of
+// *status) if the budget runs out.
+__device__ __forceinline__ bool flag_wait(const unsigned int* flag, unsigned int* status) {
+    if (flag_acquire(flag) != 0) return true;
+    const unsigned long long t0 = globaltimer();
+    while (flag_acquire(flag) == 0) {
+        if (globaltimer() - t0 > kWaitBudgetNs) {
+            atomicOr(status, 1u);
+            return false;
+        }
+        __nanosleep(64);
+    }
+    return true;
+}
+
 __device__ __forceinline__ void bulk_commit() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

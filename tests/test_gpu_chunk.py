@@ -152,23 +152,53 @@ def test_full_config_sampled_heads(gdn, index, oracle_threads):
 
 @pytest.mark.parametrize("gate", ["scalar", "channel"])
 @pytest.mark.parametrize("T", [50, 64, 200, 700])
-def test_single_cta_and_cta_pair_kernels_agree(gdn, gate, T, monkeypatch):
-    """The one-CTA kernel and the two-CTA cluster kernel (chunk-local work on
-    one SM, state chain on the other) compute the same chunk algebra."""
+def test_single_cta_pair_and_pool_kernels_agree(gdn, gate, T, monkeypatch):
+    """The one-CTA kernel, the two-CTA cluster kernel (chunk-local work on one
+    SM, state chain on the other) and the prep-pool kernel (chains fed by
+    prep CTAs on every other SM through a global slot buffer) compute the same
+    chunk algebra.  With 4 pairs and few chunks, most prep CTAs of the pool
+    get no task at all."""
     x = prefill_inputs(2, T, 2, 128, 128, gate=gate, s0_std=0.1, seed=230 + T)
-    monkeypatch.setenv("GDN_CHUNK_KERNEL", "single")
-    o1, s1 = _gpu(gdn, x)
-    monkeypatch.setenv("GDN_CHUNK_KERNEL", "pair")
-    o2, s2 = _gpu(gdn, x)
+    got = {}
+    for kernel in ("single", "pair", "pool"):
+        monkeypatch.setenv("GDN_CHUNK_KERNEL", kernel)
+        got[kernel] = _gpu(gdn, x)
     ref_o, ref_s = _ref(x, gate == "channel")
-    for o, s in ((o1, s1), (o2, s2)):
+    for o, s in got.values():
         assert oracle.rel_err(o, ref_o) <= TOL and oracle.rel_err(s, ref_s) <= TOL
-    assert oracle.rel_err(o2, o1.double()) <= TOL / 2
-    assert oracle.rel_err(s2, s1.double()) <= TOL / 2
+    o1, s1 = got["single"]
+    for kernel in ("pair", "pool"):
+        o2, s2 = got[kernel]
+        assert oracle.rel_err(o2, o1.double()) <= TOL / 2, kernel
+        assert oracle.rel_err(s2, s1.double()) <= TOL / 2, kernel
+    # The pool hands over the cluster kernel's T' and P: the same products.
+    assert oracle.rel_err(got["pool"][0], got["pair"][0].double()) <= 1e-6
+    assert oracle.rel_err(got["pool"][1], got["pair"][1].double()) <= 1e-6
     assert gdn.check() == gdn.GDN_OK
 
 
-@pytest.mark.parametrize("kernel", ["single", "pair"])
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+@pytest.mark.parametrize("B,H,T", [(2, 37, 300), (3, 5, 1000), (1, 1, 129)])
+def test_pool_kernel_pair_counts(gdn, gate, B, H, T, monkeypatch):
+    """Pool form at B*H = 74 (as many chains as prep CTAs on 148 SMs), at an
+    odd pair count with many chunks per prep CTA, and with one pair: sampled
+    pairs against the oracle, all pairs against the cluster kernel (the same
+    products in the same order)."""
+    x = prefill_inputs(B, T, H, 128, 128, gate=gate, s0_std=0.1, seed=250 + B * H)
+    monkeypatch.setenv("GDN_CHUNK_KERNEL", "pool")
+    o_pool, s_pool = _gpu(gdn, x)
+    monkeypatch.setenv("GDN_CHUNK_KERNEL", "pair")
+    o_pair, s_pair = _gpu(gdn, x)
+    BH = B * H
+    heads = sorted({0, BH // 2, BH - 1})
+    ref_o, ref_s = _ref(x, gate == "channel", heads=heads)
+    _check_pairs(o_pool, s_pool, ref_o, ref_s, _pairs(x, heads))
+    assert oracle.rel_err(o_pool, o_pair.double()) <= 1e-6
+    assert oracle.rel_err(s_pool, s_pair.double()) <= 1e-6
+    assert gdn.check() == gdn.GDN_OK
+
+
+@pytest.mark.parametrize("kernel", ["single", "pair", "pool"])
 def test_scalar_gate_beyond_the_bounded_domain(gdn, kernel, monkeypatch):
     """The scalar gate accepts any g <= 0: chunks whose total decay exceeds the
     range of the factored form take exact per-element exponentials."""
