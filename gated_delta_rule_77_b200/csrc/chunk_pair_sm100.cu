@@ -93,7 +93,8 @@ constexpr uint32_t P_BAR = P_SAFE + 16;       // tma, mma, empty, g
 constexpr uint32_t P_TMEM = P_BAR + 32;
 // T' hi, T' lo, P hi, P lo (4 x 8 KB) for the bulk copy to CTA 1; apart from
 // the X region so that the copy of chunk c overlaps the X build of chunk c + 1.
-constexpr uint32_t P_STAGE = (P_TMEM + 8 + 1023) / 1024 * 1024;
+constexpr uint32_t P_LAST = P_TMEM + 16;      // 128 f32: G of the chunk's last token (pool form)
+constexpr uint32_t P_STAGE = (P_LAST + 512 + 1023) / 1024 * 1024;
 // Per-channel g of the next chunk, by TMA: four [64 tokens][32 channels] fp32
 // boxes, 128-byte swizzled (8 KB each).
 constexpr uint32_t P_G = P_STAGE + 32768;
@@ -115,12 +116,25 @@ constexpr uint32_t C_TH = C_SLOT, C_TL = C_SLOT + 8192, C_PH = C_SLOT + 16384, C
 constexpr uint32_t C_SMALL = C_SLOT + 32768;
 constexpr uint32_t C_GAM = C_SMALL;           // 64 f32
 constexpr uint32_t C_LAST = C_GAM + 256;      // 128 f32
-constexpr uint32_t C_BAR = C_LAST + 512;      // tma_kq, tma_v, mma, full, out
-constexpr uint32_t C_TMEM = C_BAR + 40;
-constexpr uint32_t C_FETCHED = C_TMEM + 8;    // int: slots fetched (pool form)
-constexpr uint32_t C_USED = C_FETCHED + 8;
+constexpr uint32_t C_BAR = C_LAST + 512;      // tma_kq, tma_v, mma, full, out, full_b, full_c
+constexpr uint32_t C_TMEM = C_BAR + 56;
+constexpr uint32_t C_FETCHED = C_TMEM + 8;    // 3 int: record parts fetched (pool form)
+constexpr uint32_t C_USED = C_FETCHED + 16;
 
 constexpr uint32_t SLOT_BYTES = 32768;
+
+// Pool form: one task's record in the global buffer, in three parts that the
+// chain fetches apart, each as soon as the previous chunk's products that read
+// the same shared-memory tiles are complete.  Tiles are the images of the
+// chain's shared-memory tiles (same swizzle), so each part is a plain copy.
+constexpr uint32_t TA_T = 0;                  // part A: T' hi, T' lo (16 KB)
+constexpr uint32_t TA_KE = 16384;             //         K*E bf16 (16 KB)
+constexpr uint32_t TB_QE = 32768;             // part B: Q*E fp16 (16 KB)
+constexpr uint32_t TC_P = 49152;              // part C: P hi, P lo (16 KB)
+constexpr uint32_t TC_KD = 65536;             //         K*D bf16 hi, lo (32 KB)
+constexpr uint32_t TC_EL = 98304;             //         exp(G_last) per channel (512 B)
+constexpr uint32_t TASK_BYTES = 98816;
+constexpr uint32_t PART_A = TB_QE - TA_T, PART_B = TC_P - TB_QE, PART_C = TASK_BYTES - TC_P;
 constexpr uint32_t SMEM_BYTES = (P_USED > C_USED ? P_USED : C_USED) + 1024;
 
 // TMEM columns.  CTA 0: X (128 rows x up to 96).  CTA 1: W^T, U^T, O^T, SN.
@@ -134,7 +148,7 @@ struct PairParams {
     float* state_out;          // [B, H, D, D] or null
     float* out;                // [B, T, H, D] fp32
     int T, H, B;
-    uint8_t* slots;            // pool form: [B*H][chunks][SLOT_BYTES]
+    uint8_t* slots;            // pool form: [B*H][chunks][TASK_BYTES]
     unsigned int* flags;       // pool form: [B*H][chunks], zero at launch
 };
 
@@ -181,7 +195,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             prefetch_tensormap(&tm_o);
         }
         if (rank == 0 && CHANNEL) prefetch_tensormap(&tm_g);
-        for (int i = 0; i < (rank == 0 ? 4 : 5); ++i) mbar_init(bar0 + 8 * i, 1);
+        for (int i = 0; i < (rank == 0 ? 4 : 7); ++i) mbar_init(bar0 + 8 * i, 1);
         fence_mbar_init();
     }
     const uint32_t tmem_cols = rank == 0 ? 128 : 512;
@@ -335,6 +349,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
         float* sA = reinterpret_cast<float*>(smem + P_A);
         float* sT = reinterpret_cast<float*>(smem + P_T);
         float* sY = reinterpret_cast<float*>(smem + P_Y);
+        float* sLastP = reinterpret_cast<float*>(smem + P_LAST);
         const uint32_t bar_tma = sbase + P_BAR, bar_empty = sbase + P_BAR + 16;
         const uint32_t bar_g = sbase + P_BAR + 24;
         // Cluster form: CTA 1's slot and "full" barrier, as cluster addresses.
@@ -404,7 +419,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                 gn[u][0] = a.x; gn[u][1] = a.y; gn[u][2] = a.z; gn[u][3] = a.w;
                 gn[u][4] = c.x; gn[u][5] = c.y; gn[u][6] = c.z; gn[u][7] = c.w;
             }
-            gate_scan(gn, sRef0, sRef1, nullptr);
+            gate_scan(gn, sRef0, sRef1, POOL ? sLastP : nullptr);
         };
         if (tid == 0 && nitems > 0) issue_kq(0);
         int kq_waited = -1;
@@ -419,7 +434,15 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
         if (nitems > 0) beta_load(0, bgnext);
 
         for (int ci = 0; ci < nitems; ++ci) {
+            uint8_t* gslot = nullptr;           // pool form: this item's record
+            if (POOL) {
+                int ib, ih, ic;
+                item(ci, ib, ih, ic);
+                gslot = p.slots + ((size_t)(ib * H + ih) * nchunks + ic) * TASK_BYTES;
+            }
             float gam[4][8];
+            float2 last2[4];                    // pool form: G of the last token, this thread's channels
+            float my_last = 0.f;                // pool form: G of the last token, channel tid
             if (CHANNEL) {   // scanned one chunk ahead; sRef0/1 hold this chunk's
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
@@ -442,7 +465,9 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                 for (int e = 0; e < 4; ++e) {
                     ref0[e] = make_float2(sRef0[8 * ck + 2 * e], sRef0[8 * ck + 2 * e + 1]);
                     ref1[e] = make_float2(sRef1[8 * ck + 2 * e], sRef1[8 * ck + 2 * e + 1]);
+                    if (POOL) last2[e] = make_float2(sLastP[8 * ck + 2 * e], sLastP[8 * ck + 2 * e + 1]);
                 }
+                if (POOL) my_last = tid < D ? sLastP[tid] : 0.f;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int r = tg + 16 * u;
@@ -510,7 +535,59 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             }
             // While X runs: the next chunk's g (the X build of this chunk has
             // read sRef0/1 already).
+            if (POOL && CHANNEL) {    // the chain's operands K*E, Q*E and K*D, exp(G_last)
+                const float2 l2e = make_float2(kLog2e, kLog2e);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int r = tg + 16 * u;
+                    float kf[8], qf[8], ke[8], qe[8];
+                    float2 kd[4];
+                    load_bf16x8(smem + P_IN + ckh * 16384 + swz(r, ckc), kf);
+                    load_bf16x8(smem + P_IN + ckh * 16384 + 8192 + swz(r, ckc), qf);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 k2 = make_float2(kf[2 * e], kf[2 * e + 1]);
+                        const float2 q2 = make_float2(qf[2 * e], qf[2 * e + 1]);
+                        const float2 g2 = make_float2(gam[u][2 * e], gam[u][2 * e + 1]);
+                        const float2 el = mul2(g2, l2e);
+                        const float2 dl = mul2(sub2(last2[e], g2), l2e);
+                        const float2 E2 = make_float2(ex2_approx(el.x), ex2_approx(el.y));
+                        const float2 D2 = make_float2(ex2_approx(dl.x), ex2_approx(dl.y));
+                        const float2 ke2 = mul2(k2, E2), qe2 = mul2(q2, E2);
+                        ke[2 * e] = ke2.x; ke[2 * e + 1] = ke2.y;
+                        qe[2 * e] = qe2.x; qe[2 * e + 1] = qe2.y;
+                        kd[e] = mul2(k2, D2);
+                    }
+                    const uint32_t oc = ckh * 8192 + swz(r, ckc);
+                    store_bf16x8(gslot + TA_KE + oc, ke);
+                    store_f16x8(gslot + TB_QE + oc, qe);
+                    store_split2(gslot + TC_KD + oc, gslot + TC_KD + 16384 + oc, kd);
+                }
+                if (tid < D) reinterpret_cast<float*>(gslot + TC_EL)[tid] = __expf(my_last);
+            }
             if (CHANNEL && ci + 1 < nitems) scan_g(gnext);
+            if (POOL && !CHANNEL) {   // the chain's operands K*E, Q*E and K*D, exp(G_last)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int r = tg + 16 * u;
+                    float kf[8], qf[8], ke[8], qe[8], kd[8];
+                    load_bf16x8(smem + P_IN + ckh * 16384 + swz(r, ckc), kf);
+                    load_bf16x8(smem + P_IN + ckh * 16384 + 8192 + swz(r, ckc), qf);
+                    const float E = ex2_approx(sGam[r] * kLog2e);
+                    const float Dd = ex2_approx((sGam[C - 1] - sGam[r]) * kLog2e);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        ke[e] = kf[e] * E;
+                        qe[e] = qf[e] * E;
+                        kd[e] = kf[e] * Dd;
+                    }
+                    const uint32_t oc = ckh * 8192 + swz(r, ckc);
+                    store_bf16x8(gslot + TA_KE + oc, ke);
+                    store_f16x8(gslot + TB_QE + oc, qe);
+                    store_split(gslot + TC_KD + oc, gslot + TC_KD + 16384 + oc, kd);
+                }
+                if (tid < D) reinterpret_cast<float*>(gslot + TC_EL)[tid] = __expf(sGam[C - 1]);
+            }
             mma_sync();
             if (tid == 0 && copy_pending) {      // the staging is free again
                 if (POOL) publish(); else bulk_wait_read_all();
@@ -612,14 +689,17 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                 }
             }
             if (tid == 0 && POOL) {
-                // The slot to the task's place in the global buffer; its flag
-                // is set once the store is complete (at once for the first
-                // item, which the chains wait for; otherwise after the next
-                // item's X product, when the store has long finished).
+                // T' and P to the task's record in the global buffer (its
+                // other tiles were stored by every thread before the barrier
+                // above); the flag is set once the stores are complete (at
+                // once for the first item, which the chains wait for;
+                // otherwise after the next item's X product, when the stores
+                // have long finished).
                 int ib, ih, ic;
                 item(ci, ib, ih, ic);
                 const size_t task = (size_t)(ib * H + ih) * nchunks + ic;
-                bulk_store_global(p.slots + task * SLOT_BYTES, sbase + P_STAGE, SLOT_BYTES);
+                bulk_store_global(gslot + TA_T, sbase + P_STAGE, 16384);            // T'
+                bulk_store_global(gslot + TC_P, sbase + P_STAGE + 16384, 16384);    // P
                 bulk_commit();
                 pending_flag = p.flags + task;
                 copy_pending = true;
@@ -649,34 +729,53 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
         // epilogue and the state update do not wait for them.
         const uint32_t bar_out = sbase + C_BAR + 32;
         const uint32_t peer_empty = POOL ? 0u : mapa_shared(sbase + P_BAR + 16, 0);
-        // Pool form: chunk c's slot is fetched from the global buffer with one
-        // bulk copy onto bar_full once chunk c - 1's products have read the
-        // previous slot.  Its flag is tried early in chunk c - 1 by the same
-        // thread, without blocking; when set, the slot is also prefetched into
-        // L2 (prep CTAs may run far ahead of the chains, and slots written
-        // long before have left L2).  The count of fetches issued is kept in
-        // shared memory for the drain on an abandoned wait.
+        // Pool form: chunk c's record is fetched from the global buffer in
+        // three parts, each onto its own mbarrier, as soon as chunk c - 1's
+        // products that read the same tiles are complete: part A (T', K*E)
+        // after the W and U~ products, part B (Q*E) after the SN products (the
+        // O products that read Q*E precede them), part C (P, K*D, exp(G_last))
+        // once the chunk's output is staged.  The record's flag is tried early
+        // in chunk c - 1 by the fetching thread, without blocking; when set,
+        // the record is also prefetched into L2 (prep CTAs may run far ahead
+        // of the chains, and records written long before have left L2).  The
+        // counts of parts fetched are kept in shared memory for the drain on
+        // an abandoned wait.  The chain then needs no raw K, Q or gate, and W^T
+        // goes to the raw K, Q tile instead of over K*E.
+        const uint32_t bar_full_b = sbase + C_BAR + 40, bar_full_c = sbase + C_BAR + 48;
+        const uint32_t C_W = POOL ? C_IN : C_KE;
         int* sFetched = reinterpret_cast<int*>(smem + C_FETCHED);
         int acquired = -1;              // chunk whose flag this thread has acquired
+        auto record = [&](int chunk) { return p.slots + ((size_t)pair * nchunks + chunk) * TASK_BYTES; };
         auto try_acquire = [&](int chunk) {
-            const size_t task = (size_t)pair * nchunks + chunk;
-            if (flag_acquire(p.flags + task) == 0) return;
+            if (flag_acquire(p.flags + (size_t)pair * nchunks + chunk) == 0) return;
             fence_proxy_async_global();
-            bulk_prefetch_l2(p.slots + task * SLOT_BYTES, SLOT_BYTES);
+            bulk_prefetch_l2(record(chunk), TASK_BYTES);
             acquired = chunk;
         };
-        auto fetch_slot = [&](int chunk) {
-            const size_t task = (size_t)pair * nchunks + chunk;
+        auto fetch_part = [&](int chunk, int part) {
             if (acquired != chunk) {
-                ok = ok && flag_wait(p.flags + task, &g_pair_status_word);
+                ok = ok && flag_wait(p.flags + (size_t)pair * nchunks + chunk, &g_pair_status_word);
                 if (!ok) return;
                 fence_proxy_async_global();
+                acquired = chunk;
             }
-            mbar_expect_tx(bar_full, SLOT_BYTES);
-            bulk_load_global(sbase + C_SLOT, p.slots + task * SLOT_BYTES, SLOT_BYTES, bar_full);
-            *sFetched = chunk + 1;
+            const uint8_t* rec = record(chunk);
+            if (part == 0) {
+                mbar_expect_tx(bar_full, PART_A);
+                bulk_load_global(sbase + C_TH, rec + TA_T, 16384, bar_full);
+                bulk_load_global(sbase + C_KE, rec + TA_KE, 16384, bar_full);
+            } else if (part == 1) {
+                mbar_expect_tx(bar_full_b, PART_B);
+                bulk_load_global(sbase + C_QE, rec + TB_QE, 16384, bar_full_b);
+            } else {
+                mbar_expect_tx(bar_full_c, PART_C);
+                bulk_load_global(sbase + C_PH, rec + TC_P, 16384, bar_full_c);
+                bulk_load_global(sbase + C_KDH, rec + TC_KD, 32768, bar_full_c);
+                bulk_load_global(sbase + C_LAST, rec + TC_EL, 512, bar_full_c);
+            }
+            sFetched[part] = chunk + 1;
         };
-        if (POOL && tid == 0) *sFetched = 0;
+        if (POOL && tid == 0) sFetched[0] = sFetched[1] = sFetched[2] = 0;
 
         const int srow = quad * 32 + lane;
         const int scol = half * 64;
@@ -719,23 +818,27 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
         fence_async_smem();
         __syncthreads();
         if (tid == 0 && nchunks > 0) {
-            issue_kq(0);
+            if (!POOL) issue_kq(0);
             issue_v(0);
         }
-        int kq_waited = -1, v_waited = -1, full_waited = -1;
+        int kq_waited = -1, v_waited = -1, full_waited = -1, b_waited = -1, c_waited = -1;
         float gnext[4][8], bgnext[4];
-        if (CHANNEL && nchunks > 0) gate_load(0, gnext);
-        if (!CHANNEL && nchunks > 0) gate_scalar_load(b, h, 0, false, bgnext);
+        if (!POOL && CHANNEL && nchunks > 0) gate_load(0, gnext);
+        if (!POOL && !CHANNEL && nchunks > 0) gate_scalar_load(b, h, 0, false, bgnext);
         // Per-channel: chunk 0's scan here; the scan of chunk c + 1 runs
         // while the products SN of chunk c are on the tensor core.
-        if (CHANNEL && nchunks > 0) gate_channel(0, (long)b * T * H + h, gnext, nullptr, nullptr, sLast);
-        // The first slot: its flag is waited for after this thread's gate
-        // loads have been issued and used.
-        if (POOL && tid == 0 && nchunks > 0) fetch_slot(0);
+        if (!POOL && CHANNEL && nchunks > 0) gate_channel(0, (long)b * T * H + h, gnext, nullptr, nullptr, sLast);
+        if (POOL && tid == 0 && nchunks > 0) {
+            fetch_part(0, 0);
+            fetch_part(0, 1);
+            fetch_part(0, 2);
+        }
 
         for (int ci = 0; ci < nchunks; ++ci) {
             const int t0 = ci * C;
             const long tk0 = ((long)b * T + t0) * H + h;
+            float e_last = 0.f;
+          if (!POOL) {   // the operands K*E, Q*E, K*D from raw K, Q and the gate
             float gam[4][8];
             if (CHANNEL) {
 #pragma unroll
@@ -794,7 +897,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                     store_split2(smem + C_KDH + o64, smem + C_KDL + o64, kd);
                 }
             }
-            const float e_last = __expf(CHANNEL ? sLast[srow] : sGam[C - 1]);
+            e_last = __expf(CHANNEL ? sLast[srow] : sGam[C - 1]);
             fence_async_smem();
             __syncthreads();
             if (tid == 0 && ci + 1 < nchunks) issue_kq(ci + 1);   // raw K, Q consumed
@@ -802,8 +905,10 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                 if (CHANNEL) gate_load(ci + 1, gnext);
                 else gate_scalar_load(b, h, ci + 1, false, bgnext);
             }
+          }
 
-            // T' and P of this chunk from the prep side; V of this chunk.
+            // T' (with P, or pool form: with K*E) of this chunk from the prep
+            // side; V of this chunk.
             if (tid == 0) {
                 ok = ok && (POOL ? mbar_wait(bar_full, ci & 1, &g_pair_status_word)
                                  : mbar_wait_cluster(bar_full, ci & 1, &g_pair_status_word));
@@ -834,17 +939,22 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             mma_sync();
             if (__syncthreads_or(!ok)) break;
             if (tid == 0 && ci + 1 < nchunks) issue_v(ci + 1);      // V consumed
+            if (POOL && tid == NT - 32 && ci + 1 < nchunks) fetch_part(ci + 1, 0);   // T', K*E consumed
 
-            {   // W^T -> fp16 [128 i][64 r] over the consumed K*E tile
+            {   // W^T -> fp16 [128 i][64 r] (over the consumed K*E tile, or pool form: raw K, Q's)
                 float w[32];
                 tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + TM_WT + half * 32, w);
                 tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 4; ++c) store_f16x8(smem + C_KE + swz(srow, half * 4 + c), &w[8 * c]);
+                for (int c = 0; c < 4; ++c) store_f16x8(smem + C_W + swz(srow, half * 4 + c), &w[8 * c]);
+            }
+            if (POOL && tid == 0) {          // Q*E of this chunk, for the O products below
+                ok = ok && mbar_wait(bar_full_b, ci & 1, &g_pair_status_word);
+                b_waited = ci;
             }
             fence_async_smem();
             tc_fence_before();
-            __syncthreads();
+            if (__syncthreads_or(!ok)) break;
 
             if (tid == 0) {
                 tc_fence_after();
@@ -853,7 +963,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint64_t a = sdesc_sw128(sbase + C_S + ks * 2048, 16384, 1024);
-                    mma_bf16(tmem + TM_UT, a, sdesc_sw128(sbase + C_KE + ks * 2048, 8192, 1024), id_u, 1);
+                    mma_bf16(tmem + TM_UT, a, sdesc_sw128(sbase + C_W + ks * 2048, 8192, 1024), id_u, 1);
                 }
                 mma_commit(bar_mma);
 #pragma unroll
@@ -876,9 +986,13 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                     store_split(smem + C_UH + swz(srow, half * 4 + c), smem + C_UL + swz(srow, half * 4 + c),
                                 &u[8 * c]);
             }
+            if (POOL && tid == 0) {          // P and K*D of this chunk, for the products below
+                ok = ok && mbar_wait(bar_full_c, ci & 1, &g_pair_status_word);
+                c_waited = ci;
+            }
             fence_async_smem();
             tc_fence_before();
-            __syncthreads();
+            if (__syncthreads_or(!ok)) break;
 
             if (tid == 0) {
                 tc_fence_after();
@@ -907,10 +1021,15 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                 }
                 mma_commit(bar_out);
             }
-            if (CHANNEL && ci + 1 < nchunks)   // sLast of this chunk is no longer read
+            if (!POOL && CHANNEL && ci + 1 < nchunks)   // sLast of this chunk is no longer read
                 gate_channel(t0 + C, tk0 + (long)C * H, gnext, nullptr, nullptr, sLast);
             mma_sync();
             if (__syncthreads_or(!ok)) break;
+            if (POOL && tid == NT - 32 && ci + 1 < nchunks) fetch_part(ci + 1, 1);   // Q*E consumed
+            if (POOL) {   // exp(G_last) arrived with part C
+                ok = ok && mbar_wait(bar_full_c, ci & 1, &g_pair_status_word);
+                e_last = sLast[srow];
+            }
 
             {
                 const uint32_t lb = tmem + (static_cast<uint32_t>(quad * 32) << 16);
@@ -931,11 +1050,9 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                 // Products into O^T complete (they read P in the slot and U^T):
                 // the slot is free.  Cluster form: it goes back to CTA 0 (the
                 // arrive is made by a thread of the last warp, which has no
-                // global loads in flight).  Pool form: the same thread fetches
-                // the next chunk's slot.
+                // global loads in flight).
                 ok = ok && mbar_wait(bar_out, ci & 1, &g_pair_status_word);
                 if (!POOL && tid == NT - 32 && ok) mbar_arrive_remote_relaxed(peer_empty);
-                if (POOL && tid == NT - 32 && ok && ci + 1 < nchunks) fetch_slot(ci + 1);
                 tc_fence_after();
                 float o[32];
                 tmem_ld32(lb + TM_OT + half * 32, o);
@@ -954,14 +1071,22 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                 tma_store_4d(&tm_o, sbase + C_OST, 0, h, t0, b);
                 bulk_commit();
             }
+            // Pool form: P, K*D and exp(G_last) are consumed (every thread has
+            // read its decay before the barrier above).
+            if (POOL && tid == NT - 32 && ci + 1 < nchunks) fetch_part(ci + 1, 2);
         }
         if (tid == 0) bulk_wait_all();       // output stores complete before exit
         const bool failed = __syncthreads_or(!ok);
         if (tid == 0 && failed) {   // drain this CTA's own loads and products (bounded)
-            if (kq_waited + 1 < nchunks) mbar_wait(bar_kq, (kq_waited + 1) & 1, &g_pair_status_word);
+            if (!POOL && kq_waited + 1 < nchunks) mbar_wait(bar_kq, (kq_waited + 1) & 1, &g_pair_status_word);
             if (v_waited + 1 < nchunks) mbar_wait(bar_v, (v_waited + 1) & 1, &g_pair_status_word);
-            if (POOL && *sFetched > full_waited + 1)   // a slot fetch still in flight
-                mbar_wait(bar_full, (full_waited + 1) & 1, &g_pair_status_word);
+            if (POOL) {   // record parts still in flight (at most one of each)
+                const int waited[3] = {full_waited, b_waited, c_waited};
+                const uint32_t bars[3] = {bar_full, bar_full_b, bar_full_c};
+                for (int q = 0; q < 3; ++q)
+                    for (int i = waited[q] + 1; i < sFetched[q]; ++i)
+                        mbar_wait(bars[q], i & 1, &g_pair_status_word);
+            }
             mma_commit(bar_mma);
             mbar_wait(bar_mma, mma_phase, &g_pair_status_word);
         }
@@ -1090,7 +1215,7 @@ cudaError_t launch_pair(const Problem& p, cudaStream_t stream, int pool_ctas) {
     const size_t ntasks = (size_t)nbh * nchunks;
     const size_t flag_bytes = (ntasks * sizeof(unsigned int) + 1023) / 1024 * 1024;
     uint8_t* ws = nullptr;
-    cudaError_t e = workspace_alloc(reinterpret_cast<void**>(&ws), flag_bytes + ntasks * SLOT_BYTES, stream);
+    cudaError_t e = workspace_alloc(reinterpret_cast<void**>(&ws), flag_bytes + ntasks * TASK_BYTES, stream);
     if (e != cudaSuccess) return e;
     prm.flags = reinterpret_cast<unsigned int*>(ws);
     prm.slots = ws + flag_bytes;
