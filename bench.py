@@ -56,7 +56,7 @@ DECODE_CFG = CONFIGS[4]
 LONG_CFG = CONFIGS[5]
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "GDN prefill tokens/s + % tensor roofline; decode state GB/s vs HBM peak"
-PROFILE_SUMMARY = ROOT / "profiles" / "chunk_pair_kernel_gdn2_layer_B8H8T2048.md"
+PROFILE_SUMMARY = ROOT / "profiles" / "chunk_pool_kernel_gdn2_layer_B8H8T2048.md"
 # The sources the prefill kernel of this workload is compiled from (a cluster
 # of two CTAs per (batch, head): 2 * B * H = 128 <= 148 SMs).
 KERNEL_SOURCES = ("chunk_pair_sm100.cu", "chunk_common.cuh", "sm100_util.cuh")
@@ -330,7 +330,7 @@ def run_ours(args, rank: int, world: int, local: int):
     traffic = ncu_traffic()
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": traffic,
-                "kernel": "chunk_pair_kernel<per-channel>", "bytes_per_launch": nbytes,
+                "kernel": "chunk_pool_kernel<per-channel>", "bytes_per_launch": nbytes,
                 "peak_source": peaks["source"]}
     tflops = nflops / t_launch / 1e12
     tensor = {"achieved_tflops": tflops, "peak_tflops": peaks["bf16_tflops"],

@@ -133,7 +133,8 @@ constexpr uint32_t TB_QE = 32768;             // part B: Q*E fp16 (16 KB)
 constexpr uint32_t TC_P = 49152;              // part C: P hi, P lo (16 KB)
 constexpr uint32_t TC_KD = 65536;             //         K*D bf16 hi, lo (32 KB)
 constexpr uint32_t TC_EL = 98304;             //         exp(G_last) per channel (512 B)
-constexpr uint32_t TASK_BYTES = 98816;
+constexpr uint32_t TASK_BYTES = 98816;         // 772 lines of 128 bytes
+static_assert(TASK_BYTES % 128 == 0, "records are whole L2 lines (discarded after use)");
 constexpr uint32_t PART_A = TB_QE - TA_T, PART_B = TC_P - TB_QE, PART_C = TASK_BYTES - TC_P;
 constexpr uint32_t SMEM_BYTES = (P_USED > C_USED ? P_USED : C_USED) + 1024;
 
@@ -776,6 +777,10 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             sFetched[part] = chunk + 1;
         };
         if (POOL && tid == 0) sFetched[0] = sFetched[1] = sFetched[2] = 0;
+        auto discard_record = [&](int chunk) {
+            const uint8_t* rec = record(chunk);
+            for (uint32_t off = tid * 128u; off < TASK_BYTES; off += NT * 128u) discard_l2_line(rec + off);
+        };
 
         const int srow = quad * 32 + lane;
         const int scol = half * 64;
@@ -1023,6 +1028,10 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             }
             if (!POOL && CHANNEL && ci + 1 < nchunks)   // sLast of this chunk is no longer read
                 gate_channel(t0 + C, tk0 + (long)C * H, gnext, nullptr, nullptr, sLast);
+            // Pool form, while these products run: the previous chunk's record
+            // has been read for the last time, so its lines leave L2 without
+            // a write-back (three lines per thread).
+            if (POOL && ci > 0) discard_record(ci - 1);
             mma_sync();
             if (__syncthreads_or(!ok)) break;
             if (POOL && tid == NT - 32 && ci + 1 < nchunks) fetch_part(ci + 1, 1);   // Q*E consumed
@@ -1090,6 +1099,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             mma_commit(bar_mma);
             mbar_wait(bar_mma, mma_phase, &g_pair_status_word);
         }
+        if (POOL && !failed && nchunks > 0) discard_record(nchunks - 1);   // every product has completed
         if (!failed && p.state_out) {
             float4* dst = reinterpret_cast<float4*>(p.state_out + ((long)b * H + h) * DD +
                                                     (long)srow * D + scol);

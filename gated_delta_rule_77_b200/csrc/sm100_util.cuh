@@ -179,6 +179,12 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes
                  : "memory");
 }
 
+// Drops a 128-byte line from L2 without writing it back: its contents become
+// undefined.  For scratch that has been read for the last time.
+__device__ __forceinline__ void discard_l2_line(const void* line) {
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(reinterpret_cast<uint64_t>(line)) : "memory");
+}
+
 // Orders this thread's global accesses between the generic and async proxies.
 __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
