@@ -533,9 +533,16 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                     }
                 }
                 mma_commit(sbase + P_BAR + 8);
+                // Pool form: the previous item's record, whose stores have long
+                // completed, is published here, before this thread issues new
+                // global stores (a release waits for the thread's own stores).
+                if (POOL && copy_pending) {
+                    publish();
+                    copy_pending = false;
+                }
             }
-            // While X runs: the next chunk's g (the X build of this chunk has
-            // read sRef0/1 already).
+            // While X runs: the chain's operands (pool form) and the next
+            // chunk's g (the X build of this chunk has read sRef0/1 already).
             if (POOL && CHANNEL) {    // the chain's operands K*E, Q*E and K*D, exp(G_last)
                 const float2 l2e = make_float2(kLog2e, kLog2e);
 #pragma unroll
@@ -590,8 +597,8 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                 if (tid < D) reinterpret_cast<float*>(gslot + TC_EL)[tid] = __expf(sGam[C - 1]);
             }
             mma_sync();
-            if (tid == 0 && copy_pending) {      // the staging is free again
-                if (POOL) publish(); else bulk_wait_read_all();
+            if (!POOL && tid == 0 && copy_pending) {      // the staging is free again
+                bulk_wait_read_all();
                 copy_pending = false;
             }
             if (__syncthreads_or(!ok)) break;
@@ -694,8 +701,8 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                 // other tiles were stored by every thread before the barrier
                 // above); the flag is set once the stores are complete (at
                 // once for the first item, which the chains wait for;
-                // otherwise after the next item's X product, when the stores
-                // have long finished).
+                // otherwise once the next item's X product is issued, when
+                // the stores have long finished).
                 int ib, ih, ic;
                 item(ci, ib, ih, ic);
                 const size_t task = (size_t)(ib * H + ih) * nchunks + ic;
