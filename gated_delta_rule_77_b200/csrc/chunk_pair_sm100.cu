@@ -408,9 +408,34 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             pending_flag = nullptr;
         };
         int g_issued = 0, g_waited = 0;          // g loads issued / waited for
-        auto scan_g = [&](float (&gn)[4][8]) {   // wait, read this thread's values, scan
+        // Wait for a g tile, scan it in place (thread c < 128 runs the 64
+        // tokens of channel c in order; a row of a box is 32 channels on 32
+        // banks), then read this thread's values.  Every thread calls it.
+        auto scan_g = [&](float (&gn)[4][8]) {
             ok = ok && mbar_wait(bar_g, g_waited & 1, &g_pair_status_word);
             ++g_waited;
+            if (tid < D) {
+                uint8_t* col = smem + P_G + (tid >> 5) * 8192 + (tid & 3) * 4;
+                const uint32_t cchunk = (tid & 31) >> 2;
+                float acc = 0.f;
+#pragma unroll
+                for (int t0 = 0; t0 < C; t0 += 16) {
+                    float v[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = *reinterpret_cast<const float*>(col + swz(t0 + i, cchunk));
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        acc += v[i];
+                        v[i] = acc;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) *reinterpret_cast<float*>(col + swz(t0 + i, cchunk)) = v[i];
+                    if (t0 == 0) sRef0[tid] = v[15];          // token 15
+                    if (t0 == 32) sRef1[tid] = v[15];         // token 47
+                    if (POOL && t0 == 48) sLastP[tid] = v[15];   // token 63
+                }
+            }
+            __syncthreads();
             const uint8_t* box = smem + P_G + (ck >> 2) * 8192;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -420,7 +445,6 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                 gn[u][0] = a.x; gn[u][1] = a.y; gn[u][2] = a.z; gn[u][3] = a.w;
                 gn[u][4] = c.x; gn[u][5] = c.y; gn[u][6] = c.z; gn[u][7] = c.w;
             }
-            gate_scan(gn, sRef0, sRef1, POOL ? sLastP : nullptr);
         };
         if (tid == 0 && nitems > 0) issue_kq(0);
         int kq_waited = -1;
