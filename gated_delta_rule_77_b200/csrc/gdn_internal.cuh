@@ -79,7 +79,7 @@ cudaError_t launch_chunk_sm100_noalloc(const Problem& p, cudaStream_t stream, bo
 // cluster of two CTAs per pair (one prepares chunk c + 1 while the other runs
 // the chain of chunk c).  pool_ctas > B * H: one cooperative grid of that
 // many CTAs, B * H chains and the rest prep CTAs that share every pair's
-// chunks through a global slot buffer.  Used for unsegmented calls when
+// chunks through a global buffer of task records.  Used for unsegmented calls when
 // 2 * B * H <= #SMs.
 cudaError_t launch_chunk_pair_sm100(const Problem& p, cudaStream_t stream, int pool_ctas);
 cudaError_t read_and_clear_pair_status(unsigned int* status);
