@@ -127,15 +127,19 @@ constexpr uint32_t SLOT_BYTES = 32768;
 // chain fetches apart, each as soon as the previous chunk's products that read
 // the same shared-memory tiles are complete.  Tiles are the images of the
 // chain's shared-memory tiles (same swizzle), so each part is a plain copy.
-constexpr uint32_t TA_T = 0;                  // part A: T' hi, T' lo (16 KB)
+// With per-channel gates the prep CTAs bound the launch, so part A carries T
+// itself (fp32, as the solve leaves it) and beta, and the chain forms T' =
+// T Diag(beta) as bf16 hi + lo; with a scalar gate it carries T'.
+constexpr uint32_t TA_T = 0;                  // part A: T' hi, T' lo, or T fp32 (16 KB)
 constexpr uint32_t TA_KE = 16384;             //         K*E bf16 (16 KB)
 constexpr uint32_t TB_QE = 32768;             // part B: Q*E fp16 (16 KB)
 constexpr uint32_t TC_P = 49152;              // part C: P hi, P lo (16 KB)
 constexpr uint32_t TC_KD = 65536;             //         K*D bf16 hi, lo (32 KB)
 constexpr uint32_t TC_EL = 98304;             //         exp(G_last) per channel (512 B)
-constexpr uint32_t TASK_BYTES = 98816;         // 772 lines of 128 bytes
+constexpr uint32_t TA_BETA = 98816;           // part A: beta (256 B; per-channel gates)
+constexpr uint32_t TASK_BYTES = 99072;         // 774 lines of 128 bytes
 static_assert(TASK_BYTES % 128 == 0, "records are whole L2 lines (discarded after use)");
-constexpr uint32_t PART_A = TB_QE - TA_T, PART_B = TC_P - TB_QE, PART_C = TASK_BYTES - TC_P;
+constexpr uint32_t PART_A = TB_QE - TA_T, PART_B = TC_P - TB_QE, PART_C = TA_BETA - TC_P;
 constexpr uint32_t SMEM_BYTES = (P_USED > C_USED ? P_USED : C_USED) + 1024;
 
 // TMEM columns.  CTA 0: X (128 rows x up to 96).  CTA 1: W^T, U^T, O^T, SN.
@@ -695,7 +699,13 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             tc_fence_before();
             __syncthreads();
             solve_unit_lower64_rd(sA, sT, sY, tid);
-            for (int e = tid; e < 512; e += NT) {
+            if (POOL && CHANNEL) {   // T and beta as they are; the chain forms T'
+                const float4* src = reinterpret_cast<const float4*>(sT);
+                float4* dst = reinterpret_cast<float4*>(smem + P_STAGE);
+                for (int e = tid; e < 1024; e += NT) dst[e] = src[e];
+                if (tid < C) reinterpret_cast<float*>(gslot + TA_BETA)[tid] = sBeta[tid];
+            }
+            for (int e = tid; !(POOL && CHANNEL) && e < 512; e += NT) {
                 const int r = e >> 3, c = e & 7;
                 const float4 t0v = *reinterpret_cast<const float4*>(&sT[tidx(r, 8 * c)]);
                 const float4 t1v = *reinterpret_cast<const float4*>(&sT[tidx(r, 8 * c + 4)]);
@@ -775,6 +785,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
         // goes to the raw K, Q tile instead of over K*E.
         const uint32_t bar_full_b = sbase + C_BAR + 40, bar_full_c = sbase + C_BAR + 48;
         const uint32_t C_W = POOL ? C_IN : C_KE;
+        const uint32_t C_TF = C_IN + 16384;    // pool form, per-channel: T fp32 (tidx layout)
         int* sFetched = reinterpret_cast<int*>(smem + C_FETCHED);
         int acquired = -1;              // chunk whose flag this thread has acquired
         auto record = [&](int chunk) { return p.slots + ((size_t)pair * nchunks + chunk) * TASK_BYTES; };
@@ -793,9 +804,10 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             }
             const uint8_t* rec = record(chunk);
             if (part == 0) {
-                mbar_expect_tx(bar_full, PART_A);
-                bulk_load_global(sbase + C_TH, rec + TA_T, 16384, bar_full);
+                mbar_expect_tx(bar_full, CHANNEL ? PART_A + 256 : PART_A);
+                bulk_load_global(sbase + (CHANNEL ? C_TF : C_TH), rec + TA_T, 16384, bar_full);
                 bulk_load_global(sbase + C_KE, rec + TA_KE, 16384, bar_full);
+                if (CHANNEL) bulk_load_global(sbase + C_GAM, rec + TA_BETA, 256, bar_full);
             } else if (part == 1) {
                 mbar_expect_tx(bar_full_b, PART_B);
                 bulk_load_global(sbase + C_QE, rec + TB_QE, 16384, bar_full_b);
@@ -945,10 +957,28 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
 
             // T' (with P, or pool form: with K*E) of this chunk from the prep
             // side; V of this chunk.
-            if (tid == 0) {
+            if (tid == 0 || (POOL && CHANNEL)) {   // pool, per-channel: every thread reads T
                 ok = ok && (POOL ? mbar_wait(bar_full, ci & 1, &g_pair_status_word)
                                  : mbar_wait_cluster(bar_full, ci & 1, &g_pair_status_word));
                 full_waited = ci;
+            }
+            if (POOL && CHANNEL && ok) {   // T' = T Diag(beta) as bf16 hi + lo (lower triangle)
+                const float* sTc = reinterpret_cast<const float*>(smem + C_TF);
+                const float* sBc = reinterpret_cast<const float*>(smem + C_GAM);
+                for (int e = tid; e < 512; e += NT) {
+                    const int r = e >> 3, c = e & 7;
+                    const float4 t0v = *reinterpret_cast<const float4*>(&sTc[tidx(r, 8 * c)]);
+                    const float4 t1v = *reinterpret_cast<const float4*>(&sTc[tidx(r, 8 * c + 4)]);
+                    const float tt[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
+                    float tv[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const int m = 8 * c + q;
+                        tv[q] = (m <= r) ? tt[q] * sBc[m] : 0.f;
+                    }
+                    store_split(smem + C_TH + swz(r, c), smem + C_TL + swz(r, c), tv);
+                }
+                fence_async_smem();
             }
             ok = ok && mbar_wait(bar_v, ci & 1, &g_pair_status_word);
             v_waited = ci;
