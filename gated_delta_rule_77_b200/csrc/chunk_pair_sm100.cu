@@ -8,7 +8,9 @@
 //   P_rj = q_r^T Diag(exp(G_r - G_j)) k_j (j <= r)
 //   U = T' V - T' (K * E) S,  O = (Q * E) S + P U,  S <- Diag(E_last) S + (K * D)^T U
 // A, P and T' depend on the chunk's own inputs only; U, O and the new S
-// depend on the state.  The two halves run on different SMs and overlap:
+// depend on the state.  The two halves run on different SMs and overlap
+// (roles as in the cluster form; the pool form below moves the chain's
+// operand build to the prep side):
 //
 //   CTA 0 ("prep"):  gate prep, X = [K*F; Q*F](K/F)^T on tcgen05, A and P,
 //                    the fp32 triangular solve, T' and P as bf16 hi + lo;
@@ -31,13 +33,17 @@
 // chunk_pool_kernel, a cooperative grid of one CTA per SM: B*H chain CTAs and
 //   every other SM a prep CTA.  The prep CTAs share the (batch, head, chunk)
 //   tasks, chunk-major (task i: chunk i / (B*H), pair i % (B*H); CTA j takes
-//   tasks j, j + n_prep, ...), store each 32 KB slot to a global buffer with
-//   one bulk copy and set the task's flag (release).  A chain CTA polls the
-//   flag of its next chunk (acquire; tried early in the chunk, when the slot is
-//   also prefetched into L2) and fetches the slot with one bulk copy onto its
-//   "full" mbarrier as soon as the previous slot is consumed.  With more prep
-//   CTAs than chains, the chain no longer waits on a single prep CTA, and the
-//   SMs that a cluster per pair leaves idle do prep work.
+//   tasks j, j + n_prep, ...).  Each writes its task's record to a global
+//   buffer: T' (or, with per-channel gates, T and beta), P, and the chain's
+//   operands K*E, Q*E, K*D and exp(G_last), as images of the chain's
+//   shared-memory tiles; then it sets the task's flag (release).  A chain
+//   tries the flag of its next chunk early (acquire), prefetches the record
+//   into L2, and fetches it in three bulk copies, each as soon as the
+//   previous chunk's products that read the same tiles are complete.  It
+//   discards each record from L2 after its last read.  With more prep CTAs
+//   than chains, no chain waits on a single prep CTA, the SMs that a cluster
+//   per pair leaves idle do prep work, and the chain needs no raw K, Q or
+//   gate.
 //
 // Every wait is bounded (kWaitBudgetNs); on expiry a CTA records it in its
 // status word, stops, drains its own copies and returns.
@@ -402,8 +408,8 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             item(j, ib, ih, ic);
             gate_scalar_load(ib, ih, ic, true, bg);
         };
-        // Pool form: the slot of the last item stored, published (its flag
-        // set) once the store is complete.
+        // Pool form: the record of the last item stored, published (its flag
+        // set) once its stores are complete.
         unsigned int* pending_flag = nullptr;
         auto publish = [&]() {
             bulk_wait_all();
@@ -740,7 +746,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                 int ib, ih, ic;
                 item(ci, ib, ih, ic);
                 const size_t task = (size_t)(ib * H + ih) * nchunks + ic;
-                bulk_store_global(gslot + TA_T, sbase + P_STAGE, 16384);            // T'
+                bulk_store_global(gslot + TA_T, sbase + P_STAGE, 16384);            // T' or T
                 bulk_store_global(gslot + TC_P, sbase + P_STAGE + 16384, 16384);    // P
                 bulk_commit();
                 pending_flag = p.flags + task;
@@ -1281,7 +1287,7 @@ cudaError_t launch_pair(const Problem& p, cudaStream_t stream, int pool_ctas) {
         chunk_pair_kernel<CHANNEL><<<2 * nbh, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mg, prm);
         return cudaGetLastError();
     }
-    // Pool form: flags, then the slots (1 KB aligned), from the stream-ordered
+    // Pool form: flags, then the records (1 KB aligned), from the stream-ordered
     // workspace; the flags are cleared on the stream before the launch.
     const size_t ntasks = (size_t)nbh * nchunks;
     const size_t flag_bytes = (ntasks * sizeof(unsigned int) + 1023) / 1024 * 1024;
