@@ -1051,7 +1051,16 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
         const bool split = force ? (strcmp(force, "pair") == 0 || strcmp(force, "pool") == 0)
                                  : (2 * p.B * p.H <= sm_count());
         const bool pool = !force || strcmp(force, "pool") == 0;
-        if (split) return launch_chunk_pair_sm100(p, stream, pool ? sm_count() : 0);
+        if (split) {
+            cudaError_t e = launch_chunk_pair_sm100(p, stream, pool ? sm_count() : 0);
+            if (pool && e == cudaErrorMemoryAllocation) {
+                // No room for the pool's task records (nothing was launched):
+                // the cluster form needs no scratch.
+                (void)cudaGetLastError();
+                e = launch_chunk_pair_sm100(p, stream, 0);
+            }
+            return e;
+        }
         Params prm{p.g, p.beta, p.state_in, p.state_out, nullptr, out, p.T, p.H, p.B,
                    1, nchunks * C, 1, 1};
         chunk_fwd_kernel<CHANNEL><<<p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mo, prm);

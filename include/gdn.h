@@ -99,11 +99,12 @@ enum { GDN_IO_BF16 = 0, GDN_IO_F32 = 1 };
  *   T == 0 writes state_out := state_in (or zeros) and returns GDN_OK; the
  *   per-token pointers (q, k, v, g, beta, out) may then be NULL.
  * Scratch: with dk = dv = 128 and 2 * B * H <= the SM count, each chunk's
- * chunk-local results (T', P and the chain's operand tiles: 98,816 bytes)
- * pass from prep CTAs to the state chains through
- * B * H * ceil(T / 64) * (98,816 + 4) bytes of stream-ordered scratch on
- * `stream` from the library's pool (GDN_ERR_NOMEM if it cannot be had); it
- * is freed on `stream` when the call's kernel completes.
+ * chunk-local results (T' or T and beta, P and the chain's operand tiles:
+ * 99,072 bytes) pass from prep CTAs to the state chains through
+ * B * H * ceil(T / 64) * (99,072 + 4) bytes of stream-ordered scratch on
+ * `stream` from the library's pool, freed on `stream` when the call's kernel
+ * completes.  If it cannot be had, the call runs the cluster form of the
+ * same kernel, which needs none.
  */
 GDN_API int gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
                   const float* beta, const float* state_in, void* out, float* state_out,
