@@ -2,34 +2,34 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = one chunkwise prefill (gdn_chunk_fwd) of the GDN-2 layer workload:
-B=8 sequences, H=8 heads, T=2048 tokens, dk=dv=128, bf16 q/k/v, per-channel
-gate g in [-5, 0], beta = sigmoid(N(0,1)), zero initial state, fp32 state
-and output.  Inputs are synthetic (seeded recipe in synth/), resident in HBM
-when the timed region starts; they total 235 MB per step, more than the
-126 MB L2, so no L2 flush is needed between steps.
+One step = one chunkwise prefill (gdn_chunk_fwd) of the largest workload that
+fits one GPU, the long-context prefill: B=1 sequence of T=262,144 tokens,
+H=16 heads, dk=dv=128, bf16 q/k/v, scalar gate per head with 10% of tokens
+g=0 and the rest g=-min(softplus(N(0,1)),5), beta=sigmoid(N(0,1)), zero
+initial state, fp32 state carried across chunks, fp32 output.  Inputs are
+synthetic (seeded recipe in synth/) and resident in HBM when the timed region
+starts; at 3.4 GB per step they are far above the 126 MB L2, so no flush is
+needed.  The library picks its segment-parallel path for this shape.
 
-The same run also measures the decode mode (gdn_recurrent_step) on its own
-workload -- B=64 sequences, H=16, d=128, per-channel gate, fp32 state
-carried in place -- with L2 flushed before every timed step (the 64 MiB
-state would otherwise stay in the 126 MB L2), reported under "decode".
-
-Measured beside them, each as its own object of the same JSON line:
-  "prologue"            the input prologue: the prefill pass (gdn_prologue) on
-                        the GDN-2 layer shape and the decode step with the
-                        prologue fused in (gdn_recurrent_step_prologue);
-  "multi_token_decode"  4 draft tokens with per-token state snapshots;
-  "backward"            the prefill gradients (gdn_chunk_bwd), GDN-2 layer shape;
-  "decoupled_decode"    a decode step with separate erase and write gates;
-  "long_context"        one sequence of 262,144 tokens over 16 heads through
-                        the segment-parallel path.
+The JSON line also carries, as compact objects:
+  "prefill"  the two other prefill workloads (GDN-2 layer B8 H8 T2048 with a
+             per-channel gate; scalar gate B4 H12 T8192 with S0 != 0), each
+             with its HBM roofline fraction and the fp64 oracle's tokens/s;
+  "next"     the prologue pass, the prefill backward, 4-token decode with
+             snapshots and the decoupled-gate decode step;
+  "decode"   the decode mode (gdn_recurrent_step): B=64, H=16, d=128,
+             per-channel gate, 1024 successive steps captured in one CUDA
+             graph, each step on one of 6 rotating 64 MiB states (384 MiB,
+             more than 2x L2), so that every step's state read and the
+             write-back of its update cross HBM inside the timed region;
+             median per step over 5 graph replays.
 
 Under torchrun (N > 1) every rank runs the same per-GPU workload on its own
-GPU (weak scaling, no collective on the data path); the reported time is
-the max over ranks.  Prints one JSON line on rank 0.
+GPU (weak scaling, no collective on the data path); the reported time is the
+max over ranks.  Prints one JSON line on rank 0.
 
 --impl reference times the fp64 CPU oracle on the host cores on a bounded
-sample of the same workload (the reference arm of this comparison).
+sample of the headline workload (the reference arm of this comparison).
 """
 from __future__ import annotations
 
@@ -51,25 +51,42 @@ import torch  # noqa: E402
 
 from synth import CONFIGS, config_inputs, prologue_inputs  # noqa: E402
 
-PREFILL_CFG = CONFIGS[2]
+HEAD_CFG = CONFIGS[5]          # the headline: the largest single-GPU workload
+LAYER_CFG = CONFIGS[2]
+TRAIN_CFG = CONFIGS[3]
 DECODE_CFG = CONFIGS[4]
-LONG_CFG = CONFIGS[5]
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "GDN prefill tokens/s + % tensor roofline; decode state GB/s vs HBM peak"
-PROFILE_SUMMARY = ROOT / "profiles" / "chunk_pool_kernel_gdn2_layer_B8H8T2048.md"
-# The sources the prefill kernel of this workload is compiled from (a cluster
-# of two CTAs per (batch, head): 2 * B * H = 128 <= 148 SMs).
-KERNEL_SOURCES = ("chunk_pair_sm100.cu", "chunk_common.cuh", "sm100_util.cuh")
+TRAFFIC_FILE = ROOT / "profiles" / "traffic.json"
+
+
+def _r(x, n=4):
+    """Round to n significant digits (keeps the JSON line short)."""
+    if x is None or not isinstance(x, float) or x == 0 or not np.isfinite(x):
+        return x
+    return float(f"{x:.{n}g}")
 
 
 # ---------------------------------------------------------------- accounting --
-def prefill_bytes(cfg, with_state_in: bool) -> int:
-    """Algorithmic HBM bytes of one prefill call: every input read once,
-    every output written once (q,k,v bf16; g, beta fp32; out fp32; states)."""
+def prefill_bytes(cfg, with_state_in: bool, out_elem_bytes: int = 4) -> int:
+    """HBM bytes of one prefill call with every input read once and every
+    output written once: q, k, v bf16; g (dk values per channel gate, else 1)
+    and beta fp32; out at out_elem_bytes per element; the final state, and the
+    initial state when one is read (64 KiB per (b, h) each)."""
     th = cfg.B * cfg.T * cfg.H
-    per = 2 * cfg.dk + 2 * cfg.dk + 2 * cfg.dv + 4 * (cfg.dk if cfg.per_channel else 1) + 4 + 4 * cfg.dv
+    per = 2 * cfg.dk + 2 * cfg.dk + 2 * cfg.dv + 4 * (cfg.dk if cfg.per_channel else 1) + 4
+    per += out_elem_bytes * cfg.dv
     st = cfg.B * cfg.H * cfg.dk * cfg.dv * 4
     return th * per + st * (2 if with_state_in else 1)
+
+
+def algorithmic_bytes(cfg) -> int:
+    """The algorithmic bytes of a prefill workload: the per-token-head figure
+    (q, k, v 768 B, g 4 or 512 B, beta 4 B, out 256 B as bf16) times the
+    token-heads, plus the states read and written once.  The library writes
+    its output in fp32 (512 B per token-head); that extra write is not
+    counted, so the roofline fraction is conservative."""
+    return prefill_bytes(cfg, cfg.s0_std > 0, out_elem_bytes=2)
 
 
 def prefill_flops(cfg, C: int = 64) -> float:
@@ -98,32 +115,44 @@ def measured_peaks() -> dict:
             "source": "fallback"}
 
 
-def kernel_source_sha1() -> str:
-    """sha1 over the prefill kernel's source files, in KERNEL_SOURCES order."""
+def source_sha1(names) -> str:
+    """sha1 over the named kernel sources (gated_delta_rule_77_b200/csrc), in order."""
     import hashlib
     h = hashlib.sha1()
-    for name in KERNEL_SOURCES:
+    for name in names:
         h.update((ROOT / "gated_delta_rule_77_b200" / "csrc" / name).read_bytes())
     return h.hexdigest()
 
 
-def ncu_traffic():
-    """dram read+write bytes per launch of the chunk kernel from the committed
-    ncu summary, or None when the kernel source changed since that capture
-    (the summary records the sha1 of the sources it measured)."""
-    if not PROFILE_SUMMARY.exists():
+def ncu_traffic(key: str):
+    """DRAM read + write bytes per launch of a workload's dominant kernel, from
+    the committed ncu figures (profiles/traffic.json), or None when the kernel
+    sources changed since that capture (the entry records their sha1)."""
+    if not TRAFFIC_FILE.exists():
         return None
-    fields = {}
-    for line in PROFILE_SUMMARY.read_text().splitlines():
-        if ":" in line and not line.startswith(("|", " ", "#")):
-            key, val = line.split(":", 1)
-            fields[key.strip()] = val.strip()
-    if fields.get("kernel_source_sha1") != kernel_source_sha1():
+    entry = json.loads(TRAFFIC_FILE.read_text()).get(key)
+    if not entry:
         return None
     try:
-        return float(fields["traffic_bytes_per_launch"])
-    except (KeyError, ValueError):
+        if source_sha1(entry["sources"]) != entry["sources_sha1"]:
+            return None
+        return float(entry["dram_bytes_per_launch"])
+    except (KeyError, OSError, ValueError):
         return None
+
+
+def chunk_path_kernels(cfg, sms: int = 148) -> list:
+    """The kernels one gdn_chunk_fwd call launches for a workload (bf16 I/O,
+    d = 128), following the library's choice of path: the segment-parallel
+    path when B*H*4 <= #SMs and T >= 64 chunks, else the prep pool when
+    2*B*H <= #SMs, else one CTA per (batch, head)."""
+    bh = cfg.B * cfg.H
+    if bh * 4 <= sms and -(-cfg.T // 64) >= 64:
+        return ["chunk_fwd_kernel (zero-start + transition CTAs)", "combine_segments_kernel",
+                "segment_correction_kernel"]
+    if 2 * bh <= sms:
+        return ["chunk_pool_kernel"]
+    return ["chunk_fwd_kernel"]
 
 
 # ---------------------------------------------------------------- clocks --------
@@ -219,18 +248,20 @@ def max_over_ranks(x: float, world: int) -> float:
 
 
 # ---------------------------------------------------------------- CPU oracle ----
-def oracle_sample(cfg, n_pairs: int, threads: int):
-    """Times the fp64 oracle on the first n_pairs (b, h) pairs of the workload;
-    returns (seconds, equivalent tokens) where tokens = pairs * T / H."""
+def oracle_sample(cfg, threads: int, n_pairs: int | None = None, T: int | None = None):
+    """Times the fp64 oracle on a sample of a workload: the first n_pairs
+    (b, h) pairs over the first T tokens (defaults: all).  Returns
+    (seconds, tokens) where tokens = pairs * T / H (sequence tokens)."""
     import oracle
-    x = config_inputs(cfg, B=max(1, -(-n_pairs // cfg.H)))
+    n_pairs = n_pairs or cfg.B * cfg.H
+    T = T or cfg.T
+    x = config_inputs(cfg, B=max(1, -(-n_pairs // cfg.H)), T=T)
     f = {k: (None if v is None else np.ascontiguousarray(v.double().numpy())) for k, v in x.items()}
-    heads = list(range(n_pairs))
     t0 = time.perf_counter()
     oracle.run(f["q"], f["k"], f["v"], f["g"], f["beta"], f["s0"], per_channel=cfg.per_channel,
-               heads=heads, threads=threads)
+               heads=list(range(n_pairs)), threads=threads)
     dt = time.perf_counter() - t0
-    return dt, n_pairs * cfg.T / cfg.H
+    return dt, n_pairs * T / cfg.H
 
 
 def cpu_cores() -> int:
@@ -240,23 +271,29 @@ def cpu_cores() -> int:
         return os.cpu_count() or 1
 
 
+# The oracle's bounded sample of the headline workload: every head over the
+# first 16,384 tokens (1/16 of the sequence; the recurrence costs the same per
+# token everywhere).
+HEAD_SAMPLE_T = 16384
+
+
 def run_reference(args, rank: int, world: int):
     if rank != 0:
         return 0
-    cfg = PREFILL_CFG
+    cfg = HEAD_CFG
     cores = cpu_cores()
-    n_pairs = min(cfg.B * cfg.H, cores)
+    T = args.sample_tokens or HEAD_SAMPLE_T
     for _ in range(args.warmup):
-        oracle_sample(cfg, n_pairs, cores)
+        oracle_sample(cfg, cores, T=T // 4)
     total_t = 0.0
     total_tok = 0.0
     for _ in range(args.steps):
-        dt, tok = oracle_sample(cfg, n_pairs, cores)
+        dt, tok = oracle_sample(cfg, cores, T=T)
         total_t += dt
         total_tok += tok
     value = total_tok / total_t
-    sample = (f"{n_pairs} (b,h) pairs x T={cfg.T} per step of the {cfg.name} workload, fp64, "
-              f"one pair per thread")
+    sample = (f"all {cfg.B * cfg.H} (b,h) pairs over the first {T} of {cfg.T} tokens per step, "
+              f"fp64, one pair per thread")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True,
@@ -271,14 +308,13 @@ def run_reference(args, rank: int, world: int):
 
 
 def workload_config(cfg) -> dict:
-    return {"workload": "GDN-2 layer prefill (chunkwise, per-channel gate)", "B": cfg.B,
+    return {"workload": "long-context prefill (chunkwise, scalar gate, 10% g=0)", "B": cfg.B,
             "H": cfg.H, "T": cfg.T, "dk": cfg.dk, "dv": cfg.dv, "gate": cfg.gate,
-            "inputs": "bf16 q/k/v, fp32 g/beta, zero initial state, fp32 state and output",
-            "chunk": 64,
-            "l2": f"inputs {prefill_bytes(cfg, False) / 1e6:.0f} MB per step > 126 MB L2 (no flush)"}
+            "inputs": "bf16 q/k/v, fp32 g/beta, zero S0, fp32 state and output",
+            "chunk": 64, "l2": "inputs 3.4 GB per step > 126 MB L2 (no flush)"}
 
 
-# ---------------------------------------------------------------- GPU arm -------
+# ---------------------------------------------------------------- timing helpers -
 def time_events(fn, steps: int, stream) -> float:
     """Seconds for `steps` calls of fn, CUDA events on the launching stream."""
     e0 = torch.cuda.Event(enable_timing=True)
@@ -291,6 +327,97 @@ def time_events(fn, steps: int, stream) -> float:
     return e0.elapsed_time(e1) / 1e3
 
 
+def median_single(fn, stream, steps: int, warmup: int) -> float:
+    """Median seconds of single calls, each bracketed by CUDA events."""
+    times = []
+    for i in range(warmup + steps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        e1.synchronize()
+        if i >= warmup:
+            times.append(e0.elapsed_time(e1) / 1e3)
+    return statistics.median(times)
+
+
+def graph_steps(step, n: int, stream, replays: int = 5) -> tuple[float, str]:
+    """Per-step seconds of n successive calls step(i, stream) captured in one
+    CUDA graph: the median over `replays` replays of (replay time / n), CUDA
+    events on the replay stream.  If capture is refused, the n calls are
+    timed as plain back-to-back launches instead (same median rule)."""
+    s = torch.cuda.Stream()
+    s.wait_stream(stream)
+    with torch.cuda.stream(s):
+        for i in range(3):                   # warm-up outside the graph
+            step(i, s)
+    s.synchronize()
+    how = f"{n} steps in one CUDA graph, median of {replays} replays"
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=s):
+            for i in range(n):
+                step(i, s)
+        run = graph.replay
+        graph.replay()
+    except Exception as e:   # capture refused: plain launches
+        torch.cuda.synchronize()
+        graph = None
+        how = f"{n} back-to-back launches (graph capture failed: {type(e).__name__}), median of {replays}"
+
+        def run():
+            for i in range(n):
+                step(i, s)
+    s.synchronize()
+    times = []
+    for _ in range(replays):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        with torch.cuda.stream(s):
+            run()
+        e1.record(s)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1) / 1e3 / n)
+    del graph
+    return statistics.median(times), how
+
+
+# ---------------------------------------------------------------- GPU arm -------
+def run_only(args, local: int):
+    """One workload alone, for profiling under ncu (no JSON line): the
+    headline prefill (optionally at a shorter T), a prefill workload, or the
+    decode graph."""
+    import dataclasses
+    import gated_delta_rule_77_b200 as gdn
+    gdn.load()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    peaks = measured_peaks()
+    if args.only == "decode":
+        print(json.dumps(run_decode(gdn, dev, stream, peaks, 1, 0, n_steps=64)))
+        return 0
+    cfg = {"long": HEAD_CFG, "layer": LAYER_CFG, "train": TRAIN_CFG}[args.only]
+    if args.T:
+        cfg = dataclasses.replace(cfg, T=args.T)
+    x = config_inputs(cfg)
+    q, k, v, g, beta = (x[n].to(dev) for n in ("q", "k", "v", "g", "beta"))
+    s0 = x["s0"].to(dev) if x["s0"] is not None else None
+    out = torch.empty(cfg.B, cfg.T, cfg.H, cfg.dv, dtype=torch.float32, device=dev)
+    s_out = torch.empty(cfg.B, cfg.H, cfg.dk, cfg.dv, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        gdn.chunk_fwd(q, k, v, g, beta, s0, out=out, state_out=s_out, stream=stream)
+    t = time_events(lambda: gdn.chunk_fwd(q, k, v, g, beta, s0, out=out, state_out=s_out,
+                                          stream=stream), args.steps, stream) / args.steps
+    if gdn.check(stream) != gdn.GDN_OK:
+        raise RuntimeError("the prefill reported an abandoned wait")
+    print(json.dumps({"only": args.only, "T": cfg.T, "us_per_call": t * 1e6,
+                      "frac": algorithmic_bytes(cfg) / t / 1e9 / peaks["hbm_gbs"]}))
+    return 0
+
+
 def run_ours(args, rank: int, world: int, local: int):
     import gated_delta_rule_77_b200 as gdn
     gdn.load()
@@ -298,7 +425,7 @@ def run_ours(args, rank: int, world: int, local: int):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
     peaks = measured_peaks()
-    cfg = PREFILL_CFG
+    cfg = HEAD_CFG
 
     x = config_inputs(cfg, seed=cfg.index + 1000 * rank)
     q, k, v, g, beta = (x[n].to(dev) for n in ("q", "k", "v", "g", "beta"))
@@ -319,105 +446,164 @@ def run_ours(args, rank: int, world: int, local: int):
     barrier(world)
     dt = max_over_ranks(dt, world)
     if gdn.check(stream) != gdn.GDN_OK:
-        raise RuntimeError("the chunk kernel reported an abandoned wait")
+        raise RuntimeError("the prefill reported an abandoned wait")
 
-    tokens = cfg.B * cfg.T * args.steps * world
-    value = tokens / dt
-    t_launch = dt / args.steps
-    nbytes = prefill_bytes(cfg, False)
+    value = cfg.B * cfg.T * args.steps * world / dt
+    t_call = dt / args.steps
+    nbytes = algorithmic_bytes(cfg)
     nflops = prefill_flops(cfg)
-    achieved_gbs = nbytes / t_launch / 1e9
-    traffic = ncu_traffic()
-    roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": traffic,
-                "kernel": "chunk_pool_kernel<per-channel>", "bytes_per_launch": nbytes,
+    gbs = nbytes / t_call / 1e9
+    roofline = {"bound": "hbm", "achieved": _r(gbs), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": _r(gbs / peaks["hbm_gbs"]), "traffic": ncu_traffic("long_context"),
+                "bytes_per_call": nbytes, "kernels": chunk_path_kernels(cfg),
                 "peak_source": peaks["source"]}
-    tflops = nflops / t_launch / 1e12
-    tensor = {"achieved_tflops": tflops, "peak_tflops": peaks["bf16_tflops"],
-              "frac": tflops / peaks["bf16_tflops"], "flops_per_launch": nflops,
-              "attainable_frac": min(1.0, (nbytes / (peaks["hbm_gbs"] * 1e9)) / t_launch)}
+    tflops = nflops / t_call / 1e12
+    tensor = {"achieved_tflops": _r(tflops), "frac_burst": _r(tflops / peaks["bf16_tflops"]),
+              "attainable_frac": _r(min(1.0, (nbytes / (peaks["hbm_gbs"] * 1e9)) / t_call)),
+              "flops_per_call": nflops}
+    e2e = run_e2e(gdn, dev, stream, x, out, s_out, world, (q, k, v, g, beta))
+    del x
 
-    # End to end through the public API with pinned host buffers: every step
-    # copies its inputs host -> device, runs the call and copies its output
-    # device -> host, all inside the timed region.  Two device buffer sets and
-    # separate copy streams let step i + 1's upload and step i's download
-    # overlap step i's compute (PCIe is full duplex); the timed region runs
-    # from before the first upload to after the last download.
-    host = {n: x[n].pin_memory() for n in ("q", "k", "v", "g", "beta")}
+    layer = run_prefill(gdn, LAYER_CFG, dev, stream, peaks, world, rank)
+    train = run_prefill(gdn, TRAIN_CFG, dev, stream, peaks, world, rank)
+    decode = run_decode(gdn, dev, stream, peaks, world, rank)
+    nxt = {"prologue": run_prologue(gdn, dev, stream, peaks, world, rank),
+           "backward": run_backward(gdn, dev, stream, peaks, world, rank),
+           "multi_token_decode": run_multitoken(gdn, dev, stream, peaks, world, rank),
+           "decoupled_decode": run_decoupled(gdn, dev, stream, peaks, world, rank)}
+
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cores = cpu_cores()
+            cdt, ctok = oracle_sample(cfg, cores, T=HEAD_SAMPLE_T)
+            cpu = {"value": _r(ctok / cdt), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                   "sample": f"all 16 heads over the first {HEAD_SAMPLE_T} tokens, fp64, "
+                             f"{cdt:.1f} s on {min(cores, 16)} threads"}
+            for sub, c in ((layer, LAYER_CFG), (train, TRAIN_CFG)):
+                cdt, ctok = oracle_sample(c, cores)
+                sub["cpu_tok_s"] = _r(ctok / cdt)
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_call,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic", "config": workload_config(cfg), "roofline": roofline,
+                "tensor": tensor, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": len(roofline["kernels"]) * args.steps, "clocks": clk.summary(),
+                "next": nxt, "prefill": {"gdn2_layer_B8H8T2048": layer,
+                                         "scalar_B4H12T8192": train},
+                "decode": decode}
+        print(json.dumps(line))
+    return 0
+
+
+def run_e2e(gdn, dev, stream, x, out, s_out, world, dev_inputs, steps: int = 3):
+    """The headline metric end to end through the public API: every step
+    copies its inputs host -> device from pinned memory, runs the call and
+    copies the output and final state device -> host, all inside the timed
+    region.  Two device buffer sets and separate copy streams let step i + 1's
+    upload and step i's download overlap step i's call."""
+    cfg = HEAD_CFG
+    names = ("q", "k", "v", "g", "beta")
+    host = {n: x[n].pin_memory() for n in names}
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    s_h = torch.empty(s_out.shape, dtype=s_out.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_h.numel() * out_h.element_size()
-    sets = [dict(q=q, k=k, v=v, g=g, beta=beta, out=out, s_out=s_out)]
+    d2h = out_h.numel() * out_h.element_size() + s_h.numel() * s_h.element_size()
+    sets = [dict(zip(names, dev_inputs), out=out, s_out=s_out)]
     sets.append({n: torch.empty_like(t) for n, t in sets[0].items()})
     up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev_in = [torch.cuda.Event() for _ in sets]      # inputs of a set uploaded
-    ev_done = [torch.cuda.Event() for _ in sets]    # call on a set finished
-    ev_out = [torch.cuda.Event() for _ in sets]     # output of a set downloaded
-    for i in range(2):                              # all events start recorded
+    ev_in = [torch.cuda.Event() for _ in sets]
+    ev_done = [torch.cuda.Event() for _ in sets]
+    ev_out = [torch.cuda.Event() for _ in sets]
+    for i in range(2):
         ev_done[i].record(stream)
         ev_out[i].record(stream)
 
     def e2e_step(i):
         st = sets[i % 2]
-        up.wait_event(ev_done[i % 2])               # the set's previous call read its inputs
+        up.wait_event(ev_done[i % 2])
         with torch.cuda.stream(up):
-            for n in ("q", "k", "v", "g", "beta"):
+            for n in names:
                 st[n].copy_(host[n], non_blocking=True)
         ev_in[i % 2].record(up)
         stream.wait_event(ev_in[i % 2])
-        stream.wait_event(ev_out[i % 2])            # the set's previous output was downloaded
+        stream.wait_event(ev_out[i % 2])
         gdn.chunk_fwd(st["q"], st["k"], st["v"], st["g"], st["beta"], None, out=st["out"],
                       state_out=st["s_out"], stream=stream)
         ev_done[i % 2].record(stream)
         down.wait_event(ev_done[i % 2])
         with torch.cuda.stream(down):
             out_h.copy_(st["out"], non_blocking=True)
+            s_h.copy_(st["s_out"], non_blocking=True)
         ev_out[i % 2].record(down)
 
     for i in range(2):
         e2e_step(i)
     torch.cuda.synchronize()
     barrier(world)
-    e2e_steps = max(2, min(args.steps, 10))
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(up)
-    for i in range(e2e_steps):
+    for i in range(steps):
         e2e_step(i)
     e1.record(down)
     e1.synchronize()
-    dt_e2e = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
-    e2e = {"value": cfg.B * cfg.T * e2e_steps * world / dt_e2e, "unit": "tokens/s",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-           "overlap": "two buffer sets; uploads, calls and downloads on three streams"}
+    dt = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+    del sets
+    return {"value": _r(cfg.B * cfg.T * steps * world / dt), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": _r(1e3 * dt / steps), "overlap": "2 buffer sets, 3 streams"}
 
-    decode = run_decode(gdn, dev, stream, peaks, world, rank)
-    prologue = run_prologue(gdn, dev, stream, peaks, world, rank)
-    multitoken = run_multitoken(gdn, dev, stream, peaks, world, rank)
-    backward = run_backward(gdn, dev, stream, peaks, world, rank)
-    decoupled = run_decoupled(gdn, dev, stream, peaks, world, rank)
-    long_context = run_long_context(gdn, dev, stream, peaks, world, rank)
 
-    line = None
-    if rank == 0:
-        cpu = None
-        if world == 1 and not args.no_cpu_baseline:
-            cores = cpu_cores()
-            n_pairs = cfg.B * cfg.H
-            cdt, ctok = oracle_sample(cfg, n_pairs, cores)
-            cpu = {"value": ctok / cdt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                   "sample": f"the full workload once ({n_pairs} (b,h) pairs x T={cfg.T}), fp64, "
-                             f"{cdt:.1f} s wall on {cores} threads"}
-        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_launch,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-                "data": "synthetic", "config": workload_config(cfg), "roofline": roofline,
-                "tensor": tensor, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": args.steps, "clocks": clk.summary(), "decode": decode,
-                "prologue": prologue, "multi_token_decode": multitoken, "backward": backward,
-                "decoupled_decode": decoupled, "long_context": long_context}
-        print(json.dumps(line))
-    return 0
+def run_prefill(gdn, cfg, dev, stream, peaks, world, rank, steps: int = 20, warmup: int = 3):
+    """A prefill workload timed as back-to-back calls (inputs exceed L2)."""
+    x = config_inputs(cfg, seed=cfg.index + 1000 * rank)
+    q, k, v, g, beta = (x[n].to(dev) for n in ("q", "k", "v", "g", "beta"))
+    s0 = x["s0"].to(dev) if x["s0"] is not None else None
+    del x
+    out = torch.empty(cfg.B, cfg.T, cfg.H, cfg.dv, dtype=torch.float32, device=dev)
+    s_out = torch.empty(cfg.B, cfg.H, cfg.dk, cfg.dv, dtype=torch.float32, device=dev)
+
+    def step():
+        gdn.chunk_fwd(q, k, v, g, beta, s0, out=out, state_out=s_out, stream=stream)
+
+    for _ in range(warmup):
+        step()
+    t = max_over_ranks(time_events(step, steps, stream) / steps, world)
+    if gdn.check(stream) != gdn.GDN_OK:
+        raise RuntimeError("the prefill reported an abandoned wait")
+    nbytes = algorithmic_bytes(cfg)
+    gbs = nbytes / t / 1e9
+    key = "gdn2_layer" if cfg is LAYER_CFG else "scalar_train"
+    return {"tok_s": _r(cfg.B * cfg.T * world / t), "us": _r(t * 1e6), "GB/s": _r(gbs),
+            "frac": _r(gbs / peaks["hbm_gbs"]),
+            "tensor_frac": _r(prefill_flops(cfg) / t / 1e12 / peaks["bf16_tflops"]),
+            "traffic": ncu_traffic(key), "kernels": chunk_path_kernels(cfg)}
+
+
+def run_decode(gdn, dev, stream, peaks, world, rank, n_steps: int = 1024, n_states: int = 6,
+               n_inputs: int = 128):
+    """1024 successive decode steps on rotating states (see the module
+    docstring); inputs cycle over 128 distinct steps (170 MB, above L2)."""
+    cfg = DECODE_CFG
+    x = config_inputs(cfg, steps=n_inputs, seed=cfg.index + 1000 * rank)
+    q, k, v, g, beta = (x[n].to(dev) for n in ("q", "k", "v", "g", "beta"))
+    states = [x["s0"].to(dev) for _ in range(n_states)]
+    outs = [torch.empty(cfg.B, cfg.H, cfg.dv, dtype=torch.float32, device=dev) for _ in range(2)]
+
+    def step(i, s):
+        j = i % n_inputs
+        gdn.recurrent_step(q[j], k[j], v[j], g[j], beta[j], states[i % n_states],
+                           out=outs[i % 2], stream=s)
+
+    t, how = graph_steps(step, n_steps, stream)
+    t = max_over_ranks(t, world)
+    nbytes = decode_bytes(cfg)
+    gbs = nbytes / t / 1e9
+    return {"GB/s": _r(gbs), "frac": _r(gbs / peaks["hbm_gbs"]), "us_per_step": _r(t * 1e6),
+            "bytes_per_step": nbytes, "tok_s": _r(cfg.B * world / t),
+            "traffic": ncu_traffic("decode"),
+            "how": f"{how}; {n_states} rotating 64 MiB states (>2x L2)"}
 
 
 def prologue_bytes(B, T, H, dk, dv, per_channel: bool) -> int:
@@ -431,68 +617,41 @@ def prologue_bytes(B, T, H, dk, dv, per_channel: bool) -> int:
     return B * T * H * per_tok + B * H * (3 + min(T, 4)) * C * 4 + H * C * 4 * 4
 
 
-def run_prologue(gdn, dev, stream, peaks, world, rank, steps: int = 20, warmup: int = 3):
-    """The prologue's two forms, each timed alone (median of single-launch
-    CUDA-event timings).  The prefill pass moves 337 MB, more than L2; the
-    decode step's state is evicted from L2 before every timed step."""
-    pc = PREFILL_CFG
+def run_prologue(gdn, dev, stream, peaks, world, rank):
+    """The prologue's prefill pass at the GDN-2 layer shape (337 MB, above L2;
+    median of single launches) and the decode step with the prologue fused in
+    (rotating states in one graph, as the plain decode)."""
+    pc = LAYER_CFG
     x = prologue_inputs(pc.B, pc.T, pc.H, pc.dk, pc.dv, gate=pc.gate, seed=pc.index + 1000 * rank)
     xd = {n: (None if t is None else t.to(dev)) for n, t in x.items()}
     args = [xd[n] for n in ("q_raw", "k_raw", "v_raw", "g_raw", "beta_raw", "conv_w")]
-    times = []
-    for i in range(warmup + steps):
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        gdn.prologue(*args, xd["ring"], xd["pos0"], stream=stream)
-        e1.record(stream)
-        e1.synchronize()
-        if i >= warmup:
-            times.append(e0.elapsed_time(e1) / 1e3)
-    t_pre = max_over_ranks(statistics.median(times), world)
+    t_pre = max_over_ranks(median_single(
+        lambda: gdn.prologue(*args, xd["ring"], xd["pos0"], stream=stream), stream, 20, 3), world)
     b_pre = prologue_bytes(pc.B, pc.T, pc.H, pc.dk, pc.dv, pc.per_channel)
     del xd, args
 
     dc = DECODE_CFG
-    y = prologue_inputs(dc.B, 4, dc.H, dc.dk, dc.dv, gate=dc.gate, seed=dc.index + 1000 * rank)
+    n_in, n_states = 16, 6
+    y = prologue_inputs(dc.B, n_in, dc.H, dc.dk, dc.dv, gate=dc.gate, seed=dc.index + 1000 * rank)
     yd = {n: t.to(dev) for n, t in y.items()}
-    state = torch.zeros(dc.B, dc.H, dc.dk, dc.dv, dtype=torch.float32, device=dev)
-    out = torch.empty(dc.B, dc.H, dc.dv, dtype=torch.float32, device=dev)
     steps_in = [[yd[n][:, j].contiguous() for n in ("q_raw", "k_raw", "v_raw", "g_raw",
-                                                    "beta_raw")] for j in range(4)]
-    pos = [yd["pos0"] + j for j in range(warmup + steps)]
-    flush = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
-    sink = torch.empty((), dtype=torch.float32, device=dev)
-    times = []
-    for i in range(warmup + steps):
-        torch.sum(flush, dim=0, out=sink)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        gdn.recurrent_step_prologue(*steps_in[i % 4], yd["conv_w"], yd["ring"], state, pos[i],
-                                    out=out, stream=stream)
-        e1.record(stream)
-        e1.synchronize()
-        if i >= warmup:
-            times.append(e0.elapsed_time(e1) / 1e3)
-    t_dec = max_over_ranks(statistics.median(times), world)
+                                                    "beta_raw")] for j in range(n_in)]
+    states = [torch.zeros(dc.B, dc.H, dc.dk, dc.dv, dtype=torch.float32, device=dev)
+              for _ in range(n_states)]
+    rings = [yd["ring"].clone() for _ in range(n_states)]
+    out = torch.empty(dc.B, dc.H, dc.dv, dtype=torch.float32, device=dev)
+
+    def step(i, s):
+        gdn.recurrent_step_prologue(*steps_in[i % n_in], yd["conv_w"], rings[i % n_states],
+                                    states[i % n_states], yd["pos0"], out=out, stream=s)
+
+    t_dec, how = graph_steps(step, 256, stream)
+    t_dec = max_over_ranks(t_dec, world)
     C = 2 * dc.dk + dc.dv
-    b_dec = (decode_bytes(dc) + dc.B * dc.H * (3 + 1) * C * 4 + dc.H * C * 16)
+    b_dec = decode_bytes(dc) + dc.B * dc.H * (3 + 1) * C * 4 + dc.H * C * 16
     hbm = peaks["hbm_gbs"]
-    return {
-        "prefill_pass": {"kernel": "prologue_kernel + prologue_ring_kernel",
-                         "us": t_pre * 1e6, "bytes": b_pre, "GB/s": b_pre / t_pre / 1e9,
-                         "frac": b_pre / t_pre / 1e9 / hbm, "peak": hbm,
-                         "config": {"workload": "input prologue of the GDN-2 layer prefill",
-                                    "B": pc.B, "T": pc.T, "H": pc.H, "dk": pc.dk, "dv": pc.dv,
-                                    "gate": pc.gate, "activation": "silu", "ring": True}},
-        "decode_fused": {"kernel": "recurrent_prologue_kernel", "us_per_step": t_dec * 1e6,
-                         "bytes": b_dec, "GB/s": b_dec / t_dec / 1e9,
-                         "frac": b_dec / t_dec / 1e9 / hbm, "peak": hbm,
-                         "config": {"workload": "decode step with the prologue fused in",
-                                    "B": dc.B, "H": dc.H, "dk": dc.dk, "dv": dc.dv,
-                                    "gate": dc.gate, "l2": "evicted before every timed step"}},
-        "timing": f"median of {steps} single-launch CUDA-event timings each"}
+    return {"prefill_pass_us": _r(t_pre * 1e6), "prefill_pass_frac": _r(b_pre / t_pre / 1e9 / hbm),
+            "decode_fused_us": _r(t_dec * 1e6), "decode_fused_frac": _r(b_dec / t_dec / 1e9 / hbm)}
 
 
 def backward_flops(cfg, C: int = 32) -> float:
@@ -505,195 +664,87 @@ def backward_flops(cfg, C: int = 32) -> float:
     return 2.0 * macs * n_chunks
 
 
-def run_backward(gdn, dev, stream, peaks, world, rank, steps: int = 10, warmup: int = 3):
-    """gdn_chunk_bwd on the GDN-2 layer shape.  Its products run on the
-    tensor cores (mma.sync, bf16 operands split hi + lo, three passes), so
-    the roofline is the measured dense bf16 peak, against the algorithmic
-    flops of one pass."""
+def run_backward(gdn, dev, stream, peaks, world, rank):
+    """gdn_chunk_bwd on the GDN-2 layer shape (median of single calls);
+    roofline: the measured dense bf16 peak against one pass's flops."""
     from synth import grad_inputs, prefill_inputs
-    cfg = PREFILL_CFG
+    cfg = LAYER_CFG
     x = prefill_inputs(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, gate=cfg.gate, s0_std=0.1,
                        seed=cfg.index + 1000 * rank)
     do, dsT = grad_inputs(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, seed=cfg.index + 1000 * rank)
     d = {n: x[n].to(dev) for n in ("q", "k", "v", "g", "beta", "s0")}
     do, dsT = do.to(dev), dsT.to(dev)
-    times = []
-    for i in range(warmup + steps):
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        gdn.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["s0"], do, dsT, stream=stream)
-        e1.record(stream)
-        e1.synchronize()
-        if i >= warmup:
-            times.append(e0.elapsed_time(e1) / 1e3)
-    t = max_over_ranks(statistics.median(times), world)
+    t = max_over_ranks(median_single(
+        lambda: gdn.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["s0"], do, dsT,
+                              stream=stream), stream, 10, 3), world)
     fl = backward_flops(cfg)
-    peak = peaks["bf16_tflops"]
-    return {"metric": "prefill backward tokens/s", "value": cfg.B * cfg.T * world / t,
-            "unit": "tokens/s", "ms_per_call": t * 1e3,
-            "roofline": {"bound": "tensor", "achieved": fl / t / 1e12, "peak": peak,
-                         "unit": "TFLOP/s", "frac": fl / t / 1e12 / peak, "flops_per_call": fl,
-                         "peak_source": peaks["source"]},
-            "config": {"workload": "GDN-2 layer prefill gradients (dq, dk, dv, dg, dbeta, dS0)",
-                       "B": cfg.B, "H": cfg.H, "T": cfg.T, "dk": cfg.dk, "dv": cfg.dv,
-                       "gate": cfg.gate, "chunk": 32},
-            "timing": f"median of {steps} single-call CUDA-event timings"}
+    return {"ms": _r(t * 1e3), "tok_s": _r(cfg.B * cfg.T * world / t),
+            "tensor_frac": _r(fl / t / 1e12 / peaks["bf16_tflops"])}
 
 
-def run_multitoken(gdn, dev, stream, peaks, world, rank, T: int = 4, steps: int = 20,
-                   warmup: int = 3):
-    """Multi-token decode (T draft tokens per sequence, state after every
-    token kept) on the decode shape, L2 evicted before every timed call."""
+def run_multitoken(gdn, dev, stream, peaks, world, rank, T: int = 4, n_sets: int = 3):
+    """4 draft tokens with per-token snapshots on the decode shape: 64 calls in
+    one graph over 3 rotating (state, snapshot) sets (960 MiB)."""
     from synth import prefill_inputs
     cfg = DECODE_CFG
     x = prefill_inputs(cfg.B, T, cfg.H, cfg.dk, cfg.dv, gate=cfg.gate, s0_std=cfg.s0_std,
                        seed=cfg.index + 1000 * rank)
-    d = {n: x[n].to(dev) for n in ("q", "k", "v", "g", "beta", "s0")}
-    snap = torch.empty(cfg.B, T, cfg.H, cfg.dk, cfg.dv, dtype=torch.float32, device=dev)
+    d = {n: x[n].to(dev) for n in ("q", "k", "v", "g", "beta")}
+    states = [x["s0"].to(dev) for _ in range(n_sets)]
+    snaps = [torch.empty(cfg.B, T, cfg.H, cfg.dk, cfg.dv, dtype=torch.float32, device=dev)
+             for _ in range(n_sets)]
     out = torch.empty(cfg.B, T, cfg.H, cfg.dv, dtype=torch.float32, device=dev)
-    flush = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
-    sink = torch.empty((), dtype=torch.float32, device=dev)
-    times = []
-    for i in range(warmup + steps):
-        torch.sum(flush, dim=0, out=sink)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        gdn.recurrent_steps(d["q"], d["k"], d["v"], d["g"], d["beta"], d["s0"], snapshots=snap,
-                            out=out, stream=stream)
-        e1.record(stream)
-        e1.synchronize()
-        if i >= warmup:
-            times.append(e0.elapsed_time(e1) / 1e3)
-    t = max_over_ranks(statistics.median(times), world)
+
+    def step(i, s):
+        gdn.recurrent_steps(d["q"], d["k"], d["v"], d["g"], d["beta"], states[i % n_sets],
+                            snapshots=snaps[i % n_sets], out=out, stream=s)
+
+    t, _ = graph_steps(step, 64, stream)
+    t = max_over_ranks(t, world)
     bh = cfg.B * cfg.H
     st = cfg.dk * cfg.dv * 4
     per_tok = 2 * (2 * cfg.dk + cfg.dv) + 4 * (cfg.dk if cfg.per_channel else 1) + 4 + 4 * cfg.dv
     nbytes = bh * (st + T * st + T * per_tok)
     gbs = nbytes / t / 1e9
-    return {"metric": "multi-token decode GB/s", "value": gbs, "unit": "GB/s",
-            "us_per_call": t * 1e6, "frac": gbs / peaks["hbm_gbs"], "peak": peaks["hbm_gbs"],
-            "bytes_per_call": nbytes, "tokens_per_s": cfg.B * T * world / t,
-            "config": {"workload": "multi-token decode with per-token state snapshots",
-                       "B": cfg.B, "H": cfg.H, "T": T, "dk": cfg.dk, "dv": cfg.dv,
-                       "gate": cfg.gate, "l2": "evicted before every timed call"},
-            "timing": f"median of {steps} single-call CUDA-event timings"}
+    return {"us": _r(t * 1e6), "frac": _r(gbs / peaks["hbm_gbs"])}
 
 
-def run_long_context(gdn, dev, stream, peaks, world, rank, steps: int = 3, warmup: int = 2):
-    """The long-context prefill (one sequence of 262,144 tokens, 16 heads,
-    scalar gate with 10% g = 0) through the automatic segment-parallel path;
-    inputs 3.4 GB, far above L2."""
-    cfg = LONG_CFG
-    x = config_inputs(cfg, seed=cfg.index + 1000 * rank)
-    q, k, v, g, beta = (x[n].to(dev) for n in ("q", "k", "v", "g", "beta"))
-    del x
-    out = torch.empty(cfg.B, cfg.T, cfg.H, cfg.dv, dtype=torch.float32, device=dev)
-    s_out = torch.empty(cfg.B, cfg.H, cfg.dk, cfg.dv, dtype=torch.float32, device=dev)
-    times = []
-    for i in range(warmup + steps):
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        gdn.chunk_fwd(q, k, v, g, beta, None, out=out, state_out=s_out, stream=stream)
-        e1.record(stream)
-        e1.synchronize()
-        if i >= warmup:
-            times.append(e0.elapsed_time(e1) / 1e3)
-    if gdn.check(stream) != gdn.GDN_OK:
-        raise RuntimeError("the long-context prefill reported an abandoned wait")
-    t = max_over_ranks(statistics.median(times), world)
-    nbytes = prefill_bytes(cfg, False)
-    return {"metric": "long-context prefill tokens/s", "value": cfg.B * cfg.T * world / t,
-            "unit": "tokens/s", "ms_per_call": t * 1e3,
-            "roofline": {"bound": "hbm", "achieved": nbytes / t / 1e9, "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": nbytes / t / 1e9 / peaks["hbm_gbs"],
-                         "bytes_per_call": nbytes},
-            "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "T": cfg.T, "dk": cfg.dk,
-                       "dv": cfg.dv, "gate": cfg.gate, "path": "segment-parallel (automatic)"},
-            "timing": f"median of {steps} single-call CUDA-event timings"}
-
-
-def run_decoupled(gdn, dev, stream, peaks, world, rank, steps: int = 20, warmup: int = 3):
-    """One decode step with separate erase and write gates on the decode
-    shape (state in place, L2 evicted before every timed step)."""
+def run_decoupled(gdn, dev, stream, peaks, world, rank, n_states: int = 6):
+    """The decoupled-gate decode step: 256 steps in one graph over 6 rotating
+    states (as the plain decode)."""
     from synth import prefill_inputs, write_gate
     cfg = DECODE_CFG
     x = prefill_inputs(cfg.B, 1, cfg.H, cfg.dk, cfg.dv, gate=cfg.gate, s0_std=cfg.s0_std,
                        seed=cfg.index + 1000 * rank)
-    d = {n: x[n].to(dev) for n in ("q", "k", "v", "g", "beta", "s0")}
+    d = {n: x[n].to(dev) for n in ("q", "k", "v", "g", "beta")}
     bw = write_gate(cfg.B, 1, cfg.H, seed=cfg.index + 1000 * rank).to(dev)
+    states = [x["s0"].to(dev) for _ in range(n_states)]
     out = torch.empty(cfg.B, 1, cfg.H, cfg.dv, dtype=torch.float32, device=dev)
-    state = d["s0"]
-    flush = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
-    sink = torch.empty((), dtype=torch.float32, device=dev)
-    times = []
-    for i in range(warmup + steps):
-        torch.sum(flush, dim=0, out=sink)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        gdn.recurrent_steps(d["q"], d["k"], d["v"], d["g"], d["beta"], state, state_out=state,
-                            snapshots=None, out=out, beta_write=bw, stream=stream)
-        e1.record(stream)
-        e1.synchronize()
-        if i >= warmup:
-            times.append(e0.elapsed_time(e1) / 1e3)
-    t = max_over_ranks(statistics.median(times), world)
+
+    def step(i, s):
+        st = states[i % n_states]
+        gdn.recurrent_steps(d["q"], d["k"], d["v"], d["g"], d["beta"], st, state_out=st,
+                            snapshots=None, out=out, beta_write=bw, stream=s)
+
+    t, _ = graph_steps(step, 256, stream)
+    t = max_over_ranks(t, world)
     nbytes = decode_bytes(cfg) + cfg.B * cfg.H * 4
     gbs = nbytes / t / 1e9
-    return {"metric": "decoupled-gate decode state GB/s", "value": gbs, "unit": "GB/s",
-            "us_per_step": t * 1e6, "frac": gbs / peaks["hbm_gbs"], "peak": peaks["hbm_gbs"],
-            "bytes_per_step": nbytes,
-            "config": {"workload": "decode step, separate erase and write gates", "B": cfg.B,
-                       "H": cfg.H, "dk": cfg.dk, "dv": cfg.dv, "gate": cfg.gate,
-                       "l2": "evicted before every timed step"},
-            "timing": f"median of {steps} single-step CUDA-event timings"}
-
-
-def run_decode(gdn, dev, stream, peaks, world, rank, steps: int = 20, warmup: int = 3):
-    """Decode-mode step time with L2 flushed before each timed step."""
-    cfg = DECODE_CFG
-    x = config_inputs(cfg, steps=4, seed=cfg.index + 1000 * rank)
-    q, k, v, g, beta = (x[n].to(dev) for n in ("q", "k", "v", "g", "beta"))
-    state = x["s0"].to(dev)
-    out = torch.empty(cfg.B, cfg.H, cfg.dv, dtype=torch.float32, device=dev)
-    # Evict the state from L2 by reading a buffer twice its size: a read
-    # leaves L2 clean, so the timed step pays for its own traffic only.
-    flush = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
-    sink = torch.empty((), dtype=torch.float32, device=dev)
-    times = []
-    for i in range(warmup + steps):
-        torch.sum(flush, dim=0, out=sink)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        gdn.recurrent_step(q[i % 4], k[i % 4], v[i % 4], g[i % 4], beta[i % 4], state, out=out,
-                           stream=stream)
-        e1.record(stream)
-        e1.synchronize()
-        if i >= warmup:
-            times.append(e0.elapsed_time(e1) / 1e3)
-    t = max_over_ranks(statistics.median(times), world)
-    nbytes = decode_bytes(cfg)
-    gbs = nbytes / t / 1e9
-    return {"metric": "decode state GB/s", "value": gbs, "unit": "GB/s",
-            "us_per_step": t * 1e6, "frac": gbs / peaks["hbm_gbs"], "peak": peaks["hbm_gbs"],
-            "bytes_per_step": nbytes, "tokens_per_s": cfg.B * world / t,
-            "config": {"workload": "recurrent decode step", "B": cfg.B, "H": cfg.H, "dk": cfg.dk,
-                       "dv": cfg.dv, "gate": cfg.gate, "state": "fp32 in place",
-                       "l2": "evicted before every timed step by reading 2x L2 (state 64 MiB < L2)"},
-            "timing": f"median of {steps} single-step CUDA-event timings"}
+    return {"us": _r(t * 1e6), "frac": _r(gbs / peaks["hbm_gbs"])}
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sample-tokens", type=int, default=None,
+                    help="reference arm: tokens per step of the oracle's sample (default 16384)")
+    ap.add_argument("--only", choices=["long", "layer", "train", "decode"], default=None,
+                    help="profiling: run one workload alone and print its time, no JSON line")
+    ap.add_argument("--T", type=int, default=None, help="with --only: a shorter sequence length")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -701,6 +752,8 @@ def main(argv=None):
     try:
         if args.impl == "reference":
             return run_reference(args, rank, world)
+        if args.only:
+            return run_only(args, local)
         return run_ours(args, rank, world, local)
     finally:
         if world > 1:

@@ -36,7 +36,8 @@
 // decay-weighted products then become plain products of (L (.) K), (R (.) K),
 // (L (.) Q).  A scalar gate (any g <= 0) uses the exact C x C ratio matrix.
 //
-// Passes (all fp32 arithmetic on bf16 / fp32 inputs, CUDA cores):
+// Passes (fp32 state and accumulation; the products on the tensor cores as
+// mma.sync m16n8k16 with fp32 operands split into bf16 hi + lo, three passes):
 //   1. bwd_prep_kernel      per chunk: T, W = T Diag(b) Kt, Ut = T Diag(b) V,
 //                           Kh, Qt, P, E_last -> scratch;
 //   2. bwd_state_chain      per (b, h, 32-column slice), forward over chunks:

@@ -59,6 +59,8 @@
 #include "gdn_internal.cuh"
 #include "sm100_util.cuh"
 
+#include <cstdlib>
+
 namespace gdn {
 
 __device__ unsigned int g_pair_status_word = 0;
@@ -105,6 +107,9 @@ constexpr uint32_t P_STAGE = (P_LAST + 512 + 1023) / 1024 * 1024;
 // boxes, 128-byte swizzled (8 KB each).
 constexpr uint32_t P_G = P_STAGE + 32768;
 constexpr uint32_t P_USED = P_G + 32768;
+// Pool form, scalar gate: K*E bf16 [half][64 r][128 B] for the prep's own
+// W^T product (the per-channel X operands' space, unused with a scalar gate).
+constexpr uint32_t P_KE = P_X;
 
 // ---- CTA 1 (chain) shared memory ----------------------------------------------
 constexpr uint32_t C_IN = 0;                  // 32 KB raw K, Q
@@ -128,6 +133,11 @@ constexpr uint32_t C_FETCHED = C_TMEM + 8;    // 3 int: record parts fetched (po
 constexpr uint32_t C_USED = C_FETCHED + 16;
 
 constexpr uint32_t SLOT_BYTES = 32768;
+
+// Pool form: task records kept per (batch, head) at once (a ring; >= 4 for
+// progress, see PairParams).
+constexpr int kPoolRing = 8;
+static_assert(kPoolRing >= 4, "the record ring needs at least 4 slots");
 
 // Pool form: one task's record in the global buffer, in three parts that the
 // chain fetches apart, each as soon as the previous chunk's products that read
@@ -159,8 +169,27 @@ struct PairParams {
     float* state_out;          // [B, H, D, D] or null
     float* out;                // [B, T, H, D] fp32
     int T, H, B;
-    uint8_t* slots;            // pool form: [B*H][chunks][TASK_BYTES]
-    unsigned int* flags;       // pool form: [B*H][chunks], zero at launch
+    // Pool form: a ring of `ring` task records per (batch, head); record
+    // slot c % ring holds chunk c.  flags[pair][slot] = c + 1 once chunk c's
+    // record is stored (release); consumed[pair] = n once the chain has read
+    // (and discarded from L2) the records of chunks 0 .. n - 1, so a prep CTA
+    // may rewrite slot c % ring when consumed >= c - ring + 1.  All zero at
+    // launch.  The chain publishes consumed = c - 1 while it works on chunk
+    // c + 1 (it has read chunk c - 1's record by then).  With ring >= 4 this
+    // cannot deadlock: the unfinished task of lowest index (chunk-major
+    // order) waits only for its chain to reach chunk c - ring + 2, which
+    // needs records of lower index only.
+    uint8_t* slots;            // [B*H][ring][TASK_BYTES]
+    unsigned int* flags;       // [B*H][ring]
+    unsigned int* consumed;    // [B*H]
+    int ring;
+    // Failure-detection test hooks (pool form): the budget of a chain's wait
+    // for a record's flag, and one task whose flag is never set (-1: none).
+    // A chain that waits for that flag gives up when the budget runs out,
+    // records the timeout in the status word and returns; prep CTAs never
+    // wait for chains, so the launch still ends.
+    unsigned long long flag_budget_ns;
+    long long withheld_task;
 };
 
 template <bool CHANNEL, bool POOL>
@@ -383,9 +412,11 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                 ib = b; ih = h; ic = j;
             }
         };
+        int kq_issued = 0;                    // K, Q loads issued (tid 0), for the drain
         auto issue_kq = [&](int j) {
             int ib, ih, ic;
             item(j, ib, ih, ic);
+            ++kq_issued;
             mbar_expect_tx(bar_tma, 2 * 16384);
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
@@ -411,10 +442,12 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
         // Pool form: the record of the last item stored, published (its flag
         // set) once its stores are complete.
         unsigned int* pending_flag = nullptr;
+        unsigned int pending_value = 0;
+        long long pending_task = -1;
         auto publish = [&]() {
             bulk_wait_all();
             fence_proxy_async_global();
-            flag_release(pending_flag, 1u);
+            if (pending_task != p.withheld_task) flag_release(pending_flag, pending_value);
             pending_flag = nullptr;
         };
         int g_issued = 0, g_waited = 0;          // g loads issued / waited for
@@ -468,12 +501,18 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
         }
         if (nitems > 0) beta_load(0, bgnext);
 
+        bool next_slot_free = false;           // tid 0: the next item's slot found free
         for (int ci = 0; ci < nitems; ++ci) {
-            uint8_t* gslot = nullptr;           // pool form: this item's record
+            const bool slot_free = next_slot_free;
+            next_slot_free = false;
+            uint8_t* gslot = nullptr;           // pool form: this item's record slot
+            int item_pair = 0, item_chunk = 0;
             if (POOL) {
                 int ib, ih, ic;
                 item(ci, ib, ih, ic);
-                gslot = p.slots + ((size_t)(ib * H + ih) * nchunks + ic) * TASK_BYTES;
+                item_pair = ib * H + ih;
+                item_chunk = ic;
+                gslot = p.slots + ((size_t)item_pair * p.ring + ic % p.ring) * TASK_BYTES;
             }
             float gam[4][8];
             float2 last2[4];                    // pool form: G of the last token, this thread's channels
@@ -489,6 +528,15 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             if (CHANNEL && ci + 1 < nitems) beta_load(ci + 1, bgnext);
             ok = ok && mbar_wait(bar_tma, ci & 1, &g_pair_status_word);
             kq_waited = ci;
+            if (POOL && tid == 0 && item_chunk >= p.ring) {
+                // The slot's previous record (chunk - ring) must have been
+                // read by its chain before anything is stored into it
+                // (usually found so already while the previous item's X ran).
+                if (!slot_free)
+                    ok = ok && flag_wait_until(p.consumed + item_pair, (unsigned)(item_chunk - p.ring + 1),
+                                               &g_pair_status_word);
+                fence_proxy_async_global();
+            }
             if (__syncthreads_or(!ok)) break;
 
             if (CHANNEL) {
@@ -574,6 +622,14 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                     publish();
                     copy_pending = false;
                 }
+                // Pool form: the next item's record slot, tried while X runs
+                // (the acquire's cost is hidden there).
+                if (POOL && ci + 1 < nitems) {
+                    int nb, nh, nc;
+                    item(ci + 1, nb, nh, nc);
+                    next_slot_free = nc < p.ring ||
+                        (int)(flag_acquire(p.consumed + nb * H + nh) - (unsigned)(nc - p.ring + 1)) >= 0;
+                }
             }
             // While X runs: the chain's operands (pool form) and the next
             // chunk's g (the X build of this chunk has read sRef0/1 already).
@@ -608,7 +664,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                 if (tid < D) reinterpret_cast<float*>(gslot + TC_EL)[tid] = __expf(my_last);
             }
             if (CHANNEL && ci + 1 < nitems) scan_g(gnext);
-            if (POOL && !CHANNEL) {   // the chain's operands K*E, Q*E and K*D, exp(G_last)
+            if (POOL && !CHANNEL) {   // the chain's operands Q*E and K*D, exp(G_last); K*E here
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int r = tg + 16 * u;
@@ -624,7 +680,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                         kd[e] = kf[e] * Dd;
                     }
                     const uint32_t oc = ckh * 8192 + swz(r, ckc);
-                    store_bf16x8(gslot + TA_KE + oc, ke);
+                    store_bf16x8(smem + P_KE + oc, ke);     // for this CTA's W^T product
                     store_f16x8(gslot + TB_QE + oc, qe);
                     store_split(gslot + TC_KD + oc, gslot + TC_KD + 16384 + oc, kd);
                 }
@@ -726,6 +782,34 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             }
             fence_async_smem();          // staging written by threads -> read by the bulk copy
             __syncthreads();
+            if (POOL && !CHANNEL) {
+                // Scalar gate: W^T = (K*E)^T T'^T here, so that the chain,
+                // the bound with a scalar gate, receives W ready-made (fp16,
+                // the image of its operand tile) and runs one product round
+                // trip less per chunk.
+                if (tid == 0) {
+                    tc_fence_after();
+                    const uint32_t id = idesc_bf16(128, 64, true, false);
+#pragma unroll
+                    for (int part = 0; part < 2; ++part) {
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks) {
+                            const uint64_t bt = sdesc_sw128(sbase + P_STAGE + part * 8192 + ks * 32, 16, 1024);
+                            mma_bf16(tmem + TM_X, sdesc_sw128(sbase + P_KE + ks * 2048, 8192, 1024), bt, id,
+                                     (part | ks) != 0);
+                        }
+                    }
+                    mma_commit(sbase + P_BAR + 8);
+                }
+                mma_sync();
+                float w[32];
+                tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + TM_X + half * 32, w);
+                tmem_wait_ld();
+                const int wrow = quad * 32 + lane;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) store_f16x8(gslot + TA_KE + swz(wrow, half * 4 + c), &w[8 * c]);
+                tc_fence_before();
+            }
             if (tid == 0 && !POOL) {
                 // Wait until CTA 1 has consumed the previous chunk's slot.
                 ok = ok && mbar_wait_cluster(bar_empty, (ci & 1) ^ 1, &g_pair_status_word);
@@ -743,13 +827,12 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                 // once for the first item, which the chains wait for;
                 // otherwise once the next item's X product is issued, when
                 // the stores have long finished).
-                int ib, ih, ic;
-                item(ci, ib, ih, ic);
-                const size_t task = (size_t)(ib * H + ih) * nchunks + ic;
                 bulk_store_global(gslot + TA_T, sbase + P_STAGE, 16384);            // T' or T
                 bulk_store_global(gslot + TC_P, sbase + P_STAGE + 16384, 16384);    // P
                 bulk_commit();
-                pending_flag = p.flags + task;
+                pending_flag = p.flags + (size_t)item_pair * p.ring + item_chunk % p.ring;
+                pending_value = (unsigned)item_chunk + 1u;
+                pending_task = (long long)item_pair * nchunks + item_chunk;
                 copy_pending = true;
                 if (ci == 0) {
                     publish();
@@ -761,7 +844,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
         if (tid == 0) {
             bulk_wait_all();                 // own copies complete before exit
             if (POOL && pending_flag) publish();
-            if (!ok && kq_waited + 1 < nitems)
+            if (!ok && kq_issued > kq_waited + 1)
                 mbar_wait(bar_tma, (kq_waited + 1) & 1, &g_pair_status_word);
             for (int i = g_waited; !ok && i < g_issued; ++i)   // g tiles still in flight
                 mbar_wait(bar_g, i & 1, &g_pair_status_word);
@@ -791,19 +874,27 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
         // goes to the raw K, Q tile instead of over K*E.
         const uint32_t bar_full_b = sbase + C_BAR + 40, bar_full_c = sbase + C_BAR + 48;
         const uint32_t C_W = POOL ? C_IN : C_KE;
+        // Pool form, scalar gate: W^T arrives in the record (part A, over the
+        // K*E tile) and the chain skips its own W^T product.
+        constexpr bool W_READY = POOL && !CHANNEL;
+        const uint32_t C_WB = W_READY ? C_KE : C_W;
         const uint32_t C_TF = C_IN + 16384;    // pool form, per-channel: T fp32 (tidx layout)
         int* sFetched = reinterpret_cast<int*>(smem + C_FETCHED);
         int acquired = -1;              // chunk whose flag this thread has acquired
-        auto record = [&](int chunk) { return p.slots + ((size_t)pair * nchunks + chunk) * TASK_BYTES; };
+        auto record = [&](int chunk) {
+            return p.slots + ((size_t)pair * p.ring + chunk % p.ring) * TASK_BYTES;
+        };
+        auto flag_of = [&](int chunk) { return p.flags + (size_t)pair * p.ring + chunk % p.ring; };
         auto try_acquire = [&](int chunk) {
-            if (flag_acquire(p.flags + (size_t)pair * nchunks + chunk) == 0) return;
+            if (flag_acquire(flag_of(chunk)) != (unsigned)chunk + 1u) return;
             fence_proxy_async_global();
             bulk_prefetch_l2(record(chunk), TASK_BYTES);
             acquired = chunk;
         };
         auto fetch_part = [&](int chunk, int part) {
             if (acquired != chunk) {
-                ok = ok && flag_wait(p.flags + (size_t)pair * nchunks + chunk, &g_pair_status_word);
+                ok = ok && flag_wait_until(flag_of(chunk), (unsigned)chunk + 1u, &g_pair_status_word,
+                                           p.flag_budget_ns);
                 if (!ok) return;
                 fence_proxy_async_global();
                 acquired = chunk;
@@ -853,8 +944,10 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             for (int c = 0; c < 8; ++c) store_f16x8(dst + swz(srow, c), &s[8 * c]);
         };
         write_state_f16();
+        int kq_issued = 0, v_issued = 0;   // loads issued (tid 0), for the drain
         auto issue_kq = [&](int chunk) {
             const int t0 = chunk * C;
+            ++kq_issued;
             mbar_expect_tx(bar_kq, 2 * 16384);
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
@@ -864,6 +957,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
         };
         auto issue_v = [&](int chunk) {
             const int t0 = chunk * C;
+            ++v_issued;
             mbar_expect_tx(bar_v, 16384);
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf)
@@ -887,8 +981,11 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             fetch_part(0, 1);
             fetch_part(0, 2);
         }
+        // A first record that never came: no chunk starts (every thread
+        // learns it here, before any wait of the loop).
+        const bool started = !POOL || !__syncthreads_or(!ok);
 
-        for (int ci = 0; ci < nchunks; ++ci) {
+        for (int ci = 0; started && ci < nchunks; ++ci) {
             const int t0 = ci * C;
             const long tk0 = ((long)b * T + t0) * H + h;
             float e_last = 0.f;
@@ -990,6 +1087,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             v_waited = ci;
             if (__syncthreads_or(!ok)) break;
 
+          if (!W_READY) {
             if (tid == 0) {
                 tc_fence_after();
                 const uint32_t id = idesc_bf16(128, 64, true, false);
@@ -1020,32 +1118,57 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
 #pragma unroll
                 for (int c = 0; c < 4; ++c) store_f16x8(smem + C_W + swz(srow, half * 4 + c), &w[8 * c]);
             }
-            if (POOL && tid == 0) {          // Q*E of this chunk, for the O products below
+          }
+            if (POOL && !W_READY && tid == 0) {   // Q*E of this chunk, for the O products below
                 ok = ok && mbar_wait(bar_full_b, ci & 1, &g_pair_status_word);
                 b_waited = ci;
             }
             fence_async_smem();
             tc_fence_before();
-            if (__syncthreads_or(!ok)) break;
+            if (!W_READY && __syncthreads_or(!ok)) break;
+            // Pool form with W^T in the record: the next chunk's flag, tried
+            // while the products below run.
+            if (W_READY && tid == NT - 32 && ci + 1 < nchunks) try_acquire(ci + 1);
 
             if (tid == 0) {
                 tc_fence_after();
                 const uint32_t id_u = idesc_f16(128, 64, true, true, true);
                 const uint32_t id_o = idesc_f16(128, 64, true, false);
+                if (W_READY) {   // U~^T = V^T T'^T first (W^T came with the record)
+                    const uint32_t id = idesc_bf16(128, 64, true, false);
+#pragma unroll
+                    for (int part = 0; part < 2; ++part) {
+                        const uint32_t tb = part ? C_TL : C_TH;
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            mma_bf16(tmem + TM_UT, sdesc_sw128(sbase + C_V + ks * 2048, 8192, 1024),
+                                     sdesc_sw128(sbase + tb + ks * 32, 16, 1024), id, (part | ks) != 0);
+                    }
+                }
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint64_t a = sdesc_sw128(sbase + C_S + ks * 2048, 16384, 1024);
-                    mma_bf16(tmem + TM_UT, a, sdesc_sw128(sbase + C_W + ks * 2048, 8192, 1024), id_u, 1);
+                    mma_bf16(tmem + TM_UT, a, sdesc_sw128(sbase + C_WB + ks * 2048, 8192, 1024), id_u, 1);
                 }
                 mma_commit(bar_mma);
+                if (W_READY) {           // Q*E of this chunk, for the O products below
+                    ok = ok && mbar_wait(bar_full_b, ci & 1, &g_pair_status_word);
+                    b_waited = ci;
+                }
+              if (ok) {
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint64_t a = sdesc_sw128(sbase + C_S + ks * 2048, 16384, 1024);
                     const uint64_t bq = sdesc_sw128(sbase + C_QE + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
                     mma_bf16(tmem + TM_OT, a, bq, id_o, ks > 0);
                 }
+              }
             }
             mma_sync();
+            if (W_READY) {   // V, T' and W^T are consumed (the U~ and U products are complete)
+                if (tid == 0 && ci + 1 < nchunks) issue_v(ci + 1);
+                if (tid == NT - 32 && ci + 1 < nchunks) fetch_part(ci + 1, 0);
+            }
             if (tid == 0) bulk_wait_read_all();   // the previous O store has read C_OST
             if (__syncthreads_or(!ok)) break;
 
@@ -1099,6 +1222,11 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             // has been read for the last time, so its lines leave L2 without
             // a write-back (three lines per thread).
             if (POOL && ci > 0) discard_record(ci - 1);
+            // Records of chunks < ci - 1 are read and were discarded in the
+            // previous chunk, before its barriers: their slots may be reused.
+            // (Released here, where this thread waits for the products anyway:
+            // the release's fence costs the chain nothing.)
+            if (POOL && tid == 32 && ci > 1) flag_release(p.consumed + pair, (unsigned)(ci - 1));
             mma_sync();
             if (__syncthreads_or(!ok)) break;
             if (POOL && tid == NT - 32 && ci + 1 < nchunks) fetch_part(ci + 1, 1);   // Q*E consumed
@@ -1154,8 +1282,8 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
         if (tid == 0) bulk_wait_all();       // output stores complete before exit
         const bool failed = __syncthreads_or(!ok);
         if (tid == 0 && failed) {   // drain this CTA's own loads and products (bounded)
-            if (!POOL && kq_waited + 1 < nchunks) mbar_wait(bar_kq, (kq_waited + 1) & 1, &g_pair_status_word);
-            if (v_waited + 1 < nchunks) mbar_wait(bar_v, (v_waited + 1) & 1, &g_pair_status_word);
+            if (!POOL && kq_issued > kq_waited + 1) mbar_wait(bar_kq, (kq_waited + 1) & 1, &g_pair_status_word);
+            if (v_issued > v_waited + 1) mbar_wait(bar_v, (v_waited + 1) & 1, &g_pair_status_word);
             if (POOL) {   // record parts still in flight (at most one of each)
                 const int waited[3] = {full_waited, b_waited, c_waited};
                 const uint32_t bars[3] = {bar_full, bar_full_b, bar_full_c};
@@ -1165,6 +1293,9 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             }
             mma_commit(bar_mma);
             mbar_wait(bar_mma, mma_phase, &g_pair_status_word);
+            // Nothing of this chain reads its records any more: prep CTAs
+            // waiting for its slots go on (their records are never read).
+            if (POOL) flag_release(p.consumed + pair, 0x7fffffffu);
         }
         if (POOL && !failed && nchunks > 0) discard_record(nchunks - 1);   // every product has completed
         if (!failed && p.state_out) {
@@ -1205,15 +1336,16 @@ chunk_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
+    // Same entry point for every device; initialised once, thread-safely.
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
         void* ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
+            return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+        return nullptr;
+    }();
     return fn;
 }
 
@@ -1260,15 +1392,11 @@ bool make_map(CUtensorMap* map, const void* base, int H, int T, int B) {
 
 template <bool CHANNEL>
 cudaError_t launch_pair(const Problem& p, cudaStream_t stream, int pool_ctas) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(chunk_pair_kernel<CHANNEL>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    {
+        cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(chunk_pair_kernel<CHANNEL>), SMEM_BYTES);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(chunk_pool_kernel<CHANNEL>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+            e = set_smem_limit(reinterpret_cast<const void*>(chunk_pool_kernel<CHANNEL>), SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     CUtensorMap mq, mk, mv, mo, mg;
     if (!make_map(&mq, p.q, p.H, p.T, p.B) || !make_map(&mk, p.k, p.H, p.T, p.B) ||
@@ -1280,23 +1408,38 @@ cudaError_t launch_pair(const Problem& p, cudaStream_t stream, int pool_ctas) {
         mg = mq;                                   // not read with a scalar gate
     }
     PairParams prm{p.g, p.beta, p.state_in, p.state_out, static_cast<float*>(p.out), p.T, p.H, p.B,
-                   nullptr, nullptr};
+                   nullptr, nullptr, nullptr, 0, kWaitBudgetNs, -1};
+    // Test hooks of the pool form's flag wait (failure detection): a task
+    // whose record is never published, and a short budget for the chains'
+    // flag waits.  Unset in normal use.
+    if (const char* w = getenv("GDN_TEST_WITHHOLD_TASK")) prm.withheld_task = atoll(w);
+    if (const char* b = getenv("GDN_TEST_FLAG_BUDGET_NS")) {
+        const long long ns = atoll(b);
+        if (ns > 0) prm.flag_budget_ns = (unsigned long long)ns;
+    }
     const int nbh = p.B * p.H;
     const int nchunks = (p.T + C - 1) / C;
     if (pool_ctas <= nbh || nchunks == 0) {
         chunk_pair_kernel<CHANNEL><<<2 * nbh, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mg, prm);
         return cudaGetLastError();
     }
-    // Pool form: flags, then the records (1 KB aligned), from the stream-ordered
-    // workspace; the flags are cleared on the stream before the launch.
-    const size_t ntasks = (size_t)nbh * nchunks;
-    const size_t flag_bytes = (ntasks * sizeof(unsigned int) + 1023) / 1024 * 1024;
+    // Pool form: per (batch, head) a ring of kPoolRing task records, its
+    // flags and its consumed counter, from the stream-ordered workspace
+    // (flags and counters first, 1 KB aligned, cleared on the stream before
+    // the launch).  The scratch is kPoolRing * 99,072 + 4 * (kPoolRing + 1)
+    // bytes per (batch, head), whatever T.
+    const int ring = nchunks < kPoolRing ? nchunks : kPoolRing;
+    const size_t nslots = (size_t)nbh * ring;
+    const size_t counter_words = nslots + (size_t)nbh;
+    const size_t flag_bytes = (counter_words * sizeof(unsigned int) + 1023) / 1024 * 1024;
     uint8_t* ws = nullptr;
-    cudaError_t e = workspace_alloc(reinterpret_cast<void**>(&ws), flag_bytes + ntasks * TASK_BYTES, stream);
+    cudaError_t e = workspace_alloc(reinterpret_cast<void**>(&ws), flag_bytes + nslots * TASK_BYTES, stream);
     if (e != cudaSuccess) return e;
     prm.flags = reinterpret_cast<unsigned int*>(ws);
+    prm.consumed = prm.flags + nslots;
+    prm.ring = ring;
     prm.slots = ws + flag_bytes;
-    e = cudaMemsetAsync(ws, 0, ntasks * sizeof(unsigned int), stream);
+    e = cudaMemsetAsync(ws, 0, counter_words * sizeof(unsigned int), stream);
     if (e == cudaSuccess) {
         // Cooperative: every CTA is resident at once (the chains wait on prep
         // CTAs), or the launch fails instead of starting.
@@ -1315,6 +1458,7 @@ cudaError_t launch_pair(const Problem& p, cudaStream_t stream, int pool_ctas) {
             (void)cudaGetLastError();
             prm.slots = nullptr;
             prm.flags = nullptr;
+            prm.consumed = nullptr;
             chunk_pair_kernel<CHANNEL><<<2 * nbh, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mg, prm);
             e = cudaGetLastError();
         }

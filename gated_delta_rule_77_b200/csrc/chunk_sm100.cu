@@ -57,7 +57,9 @@
 
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "chunk_common.cuh"
 #include "warp_mma.cuh"
@@ -118,7 +120,13 @@ constexpr uint32_t SM_FJ = SM_ER + 256;       // 64 f32: exp(G_31 - G_j)
 constexpr uint32_t SM_SAFE = SM_FJ + 256;     // int: product form in range
 constexpr uint32_t SM_BAR = SM_SAFE + 16;     // 3 mbarriers: loads, products, products into O
 constexpr uint32_t SM_TMEM = SM_BAR + 24;     // TMEM base address
-constexpr uint32_t SMEM_USED = SM_TMEM + 16;
+constexpr uint32_t SM_RED = SM_TMEM + 16;     // 8 f32: per-warp max |M| (transition CTAs)
+constexpr uint32_t SMEM_USED = SM_RED + 32;
+
+// A transition CTA stops once every entry of its M is at most this: from
+// there on the dropped part of the correction is below 2^-53 |S_start|
+// (see Params::trans_len).
+constexpr float kTransitionDrop = 0x1p-60f;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 
 // ---- TMEM columns (512 allocated) -------------------------------------------
@@ -144,10 +152,31 @@ struct Params {
     int nseg, seg_len;         // time segments of seg_len tokens (a multiple of C)
     int in_segs, out_segs;     // 1 or nseg
     // Transition CTAs with a buffer here also form outputs: with v = 0 from
-    // the identity their "output" is w_t = M_t^T q_t ([B, T, H, D] fp32),
+    // the identity their "output" is w_t = M_t^T q_t ([B, T, H, D] fp16),
     // M_t the state map from the segment start to token t, so that the true
-    // output is the zero-start one plus S_start^T w_t.
-    float* wout = nullptr;
+    // output is the zero-start one plus S_start^T w_t.  (fp16: the
+    // correction that reads w multiplies in fp16 anyway.)
+    __half* wout = nullptr;
+    // Segment 0 from the true initial state: its zero-start CTA reads
+    // state_in (the others start from zero) and it has no transition CTA, so
+    // that transition CTAs cover segments trans_first .. nseg - 1.
+    int trans_first = 0;
+    bool in_first_only = false;
+    // Early end of the transitions (scalar gate; [B, nseg, H] chunks run;
+    // null: run every chunk).  Every step of the recurrence is a contraction
+    // when g <= 0, beta in [0, 1] and |k| = 1 (the model card's input domain,
+    // section 2.1): |I - b k k^T|_2 <= 1 while 0 <= b |k|^2 <= 2, and
+    // |exp(g)| <= 1.  So once max |M_ij| <= kTransitionDrop after a chunk,
+    // every later M_t' has |M_t'|_2 <= 128 kTransitionDrop = 2^-53, and
+    // dropping it changes an output by at most 2^-53 |S_start|_2 |q| --
+    // below fp32 resolution.  A transition CTA checks the domain on the
+    // tokens it runs (g <= 0 and 0 <= b (K K^T)_rr <= 2, from the diagonal of
+    // the product it forms anyway) and, before stopping, beta and g of the
+    // tokens it would skip; it never stops once a token is outside.  It then
+    // records how many chunks it ran and writes M = 0 and w only for those
+    // chunks; the correction reads the count.  With decaying gates M falls
+    // below the threshold within a chunk or two.
+    int* trans_len = nullptr;
 };
 
 template <bool CHANNEL>
@@ -177,6 +206,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t bar_mma = sbase + SM_BAR + 8;
     const uint32_t bar_out = sbase + SM_BAR + 16;   // O^T products, committed apart
     uint32_t* sTmemBase = reinterpret_cast<uint32_t*>(smem + SM_TMEM);
+    float* sRed = reinterpret_cast<float*>(smem + SM_RED);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -188,9 +218,10 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int per_mode = p.B * p.nseg * H;
     const bool transition = static_cast<int>(blockIdx.x) >= per_mode;
     const int rem = static_cast<int>(blockIdx.x) - (transition ? per_mode : 0);
+    const int nseg_here = transition ? p.nseg - p.trans_first : p.nseg;
     const int h = rem % H;
-    const int seg = (rem / H) % p.nseg;
-    const int b = rem / (H * p.nseg);
+    const int seg = (transition ? p.trans_first : 0) + (rem / H) % nseg_here;
+    const int b = rem / (H * nseg_here);
     const int t_begin = seg * p.seg_len;
     const int t_end = min(T, t_begin + p.seg_len);
     const int nchunks = t_end > t_begin ? (t_end - t_begin + C - 1) / C : 0;
@@ -236,7 +267,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (transition) {                       // identity: the chain yields M
 #pragma unroll
         for (int c = 0; c < 64; ++c) s[c] = (srow == scol + c) ? 1.f : 0.f;
-    } else if (p.state_in) {
+    } else if (p.state_in && (!p.in_first_only || seg == 0)) {
         const long sin_b = (((long)b * p.in_segs + (p.in_segs == 1 ? 0 : seg)) * H + h) * DD;
         const float4* src = reinterpret_cast<const float4*>(p.state_in + sin_b + (long)srow * D + scol);
 #pragma unroll
@@ -271,6 +302,13 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
     if (tid == 0 && nchunks > 0) issue_loads(0);
     int tma_waited = -1;   // last chunk whose loads were waited for
+    int tma_issued = nchunks > 0 ? 1 : 0;   // chunks whose loads were issued (tid 0)
+    // Transition CTAs that may stop early: this thread has seen a token
+    // outside the contracting domain (sticky), and the chunks run so far.
+    const bool may_stop = !CHANNEL && transition && p.trans_len != nullptr;
+    bool outside = false;
+    bool stopped = false;
+    int chunks_run = nchunks;
 
     uint32_t mma_phase = 0;
     bool ok = true;
@@ -374,6 +412,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             float g0 = bgnext[2], g1 = bgnext[3];
             sBeta[lane] = b0;
             sBeta[32 + lane] = b1;
+            if (!CHANNEL && may_stop && !(g0 <= 0.f && g1 <= 0.f)) outside = true;
             if (!CHANNEL) {
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
@@ -579,6 +618,12 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             };
             const int j0 = half * 32;
             if (!is_p) {
+                if (may_stop && half == (r >> 5)) {   // this thread holds (K K^T)_rr = |k_r|^2
+                    float xd = 0.f;
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) xd = jj == (r & 31) ? x[jj] : xd;
+                    if (!(br >= 0.f && br * xd <= 2.f)) outside = true;
+                }
 #pragma unroll
                 for (int j4 = 0; j4 < 8; ++j4) {
                     float a[4];
@@ -689,7 +734,10 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         mma_sync();
         if (__syncthreads_or(!ok)) break;
         // Raw K, Q, V, T' and W^T are no longer read: prefetch the next chunk.
-        if (tid == 0 && ci + 1 < nchunks) issue_loads(ci + 1);
+        if (tid == 0 && ci + 1 < nchunks) {
+            issue_loads(ci + 1);
+            ++tma_issued;
+        }
 
         // U^T -> bf16 hi + lo [128 j][64 r] (K-major B of SN, K-major A of O^T).
         {
@@ -764,31 +812,77 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 // O^T (lane = value column) -> [token][column] fp32 over the
                 // consumed K*E / Q*E tiles; one TMA store per chunk, rows past
                 // T dropped.  Thread stores would hold up the next proxy fence.
-                float* so = reinterpret_cast<float*>(smem + OFF_OST) + half * 32 * D + srow;
+                if (transition) {   // w in fp16
+                    __half* sh = reinterpret_cast<__half*>(smem + OFF_OST) + half * 32 * D + srow;
 #pragma unroll
-                for (int r = 0; r < 32; ++r) so[r * D] = o[r];
+                    for (int r = 0; r < 32; ++r) sh[r * D] = __float2half_rn(o[r]);
+                } else {
+                    float* so = reinterpret_cast<float*>(smem + OFF_OST) + half * 32 * D + srow;
+#pragma unroll
+                    for (int r = 0; r < 32; ++r) so[r * D] = o[r];
+                }
             }
         }
         fence_async_smem();
         tc_fence_before();
+        if (may_stop) {   // this chunk's max |M| (or +inf outside the domain), per warp
+            float m = 0.f;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) m = fmaxf(m, fabsf(s[c]));
+            if (outside) m = __int_as_float(0x7f800000);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (lane == 0) sRed[warp] = m;
+        }
         if (__syncthreads_or(!ok)) break;
         if (want_o && tid == 0) {
             tma_store_4d(tm_store, sbase + OFF_OST, 0, h, t0, b);
             bulk_commit();
         }
+        if (may_stop && ci + 1 < nchunks) {
+            // Read by every thread between this barrier and the next chunk's
+            // first one; rewritten only at the next chunk's end.
+            float m = sRed[0];
+#pragma unroll
+            for (int w = 1; w < NT / 32; ++w) m = fmaxf(m, sRed[w]);
+            if (m <= kTransitionDrop) {
+                // The tokens not run must be inside the domain too: scan their
+                // beta and g (8 bytes a token); unit keys are the caller's
+                // contract.
+                bool bad = false;
+                for (long t = t0 + C + tid; t < t_end; t += NT) {
+                    const long i = ((long)b * T + t) * H + h;
+                    const float bt = p.beta[i], gt = p.g[i];
+                    bad |= !(bt >= 0.f && bt <= 1.f && gt <= 0.f);
+                }
+                if (!__syncthreads_or(bad)) {
+                    stopped = true;
+                    chunks_run = ci + 1;
+                    break;
+                }
+                outside = true;   // some later token is outside: run every chunk
+            }
+        }
     }
     if (tid == 0) bulk_wait_all();     // output stores complete before exit
+    if (tid == 0 && stopped && tma_issued > tma_waited + 1)   // the next chunk's loads
+        mbar_wait(bar_tma, (tma_waited + 1) & 1, &g_status_word);
+    if (tid == 0 && may_stop && ok) p.trans_len[((long)b * p.nseg + seg) * H + h] = chunks_run;
 
     if (!ok && tid == 0) {
         // Abandoned: drain what this CTA still has in flight (bounded) before
         // its shared memory and TMEM go away.
-        if (tma_waited + 1 < nchunks) mbar_wait(bar_tma, (tma_waited + 1) & 1, &g_status_word);
+        if (tma_issued > tma_waited + 1) mbar_wait(bar_tma, (tma_waited + 1) & 1, &g_status_word);
         mma_commit(bar_mma);
         mbar_wait(bar_mma, mma_phase, &g_status_word);
     }
     float* sdst = nullptr;
     if (transition) {
         sdst = p.trans_out + (((long)b * p.nseg + seg) * H + h) * DD;
+        if (stopped) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) s[c] = 0.f;   // the dropped transition
+        }
     } else if (p.state_out != nullptr && (p.out_segs != 1 || seg == p.nseg - 1)) {
         sdst = p.state_out + (((long)b * p.out_segs + (p.out_segs == 1 ? 0 : seg)) * H + h) * DD;
     }
@@ -807,15 +901,17 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
 // ---- host side ---------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
+    // The driver entry point is the same for every device; a function-local
+    // static is initialised once, thread-safely.
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
         void* ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
+            return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+        return nullptr;
+    }();
     return fn;
 }
 
@@ -830,6 +926,20 @@ bool make_out_map(CUtensorMap* map, const void* base, int H, int T, int B) {
     cuuint32_t box[4] = {(cuuint32_t)D, 1, (cuuint32_t)C, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box,
+                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// w [B, T, H, D] fp16, box = one chunk of one head, no swizzle.
+bool make_half_map(CUtensorMap* map, const void* base, int H, int T, int B) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
+    cuuint32_t box[4] = {(cuuint32_t)D, 1, (cuuint32_t)C, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(base), dims, strides, box,
                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -852,12 +962,14 @@ bool make_map(CUtensorMap* map, const void* base, int H, int T, int B) {
 // and a 32-column slice of the state:
 //     S_start(0) = S0,   S_start(s + 1) = M_s S_start(s) + S_end(0)(s).
 // In place: on entry seg_states[s] holds S_end(0)(s), the end state of
-// segment s started from zero; on exit it holds S_start(s).  The state after
+// segment s started from zero; on exit it holds S_start(s).  With seg0_true,
+// seg_states[0] already holds the true end state of segment 0 (it ran from
+// S0), so S_start(1) = seg_states[0] and M_0 is not read.  The state after
 // the last segment goes to state_out (may alias state_in).  fp32 throughout.
 constexpr int CB_COLS = 32;
 __global__ void __launch_bounds__(256)
 combine_segments_kernel(float* seg_states, const float* trans, const float* state_in,
-                        float* state_out, int H, int nseg)
+                        float* state_out, int H, int nseg, int seg0_true)
 {
     __shared__ __align__(16) float sS[D][CB_COLS];     // current state slice
     const int nslice = D / CB_COLS;
@@ -884,7 +996,7 @@ combine_segments_kernel(float* seg_states, const float* trans, const float* stat
         }
         const float4* mrow = reinterpret_cast<const float4*>(trans + base + (long)i * D);
 #pragma unroll 4
-        for (int k4 = 0; k4 < D / 4; ++k4) {
+        for (int k4 = 0; k4 < ((sg == 0 && seg0_true) ? 0 : D / 4); ++k4) {
             const float4 m = mrow[k4];
             const float mk[4] = {m.x, m.y, m.z, m.w};
 #pragma unroll
@@ -925,33 +1037,38 @@ combine_segments_kernel(float* seg_states, const float* trans, const float* stat
 constexpr int CORR_TILES = 16;
 struct __align__(16) CorrSmem {
     __half s[D][D + 8];
-    float w[2][C][D + 4];
+    __half w[2][C][D + 8];
 };
 __device__ __forceinline__ void corr_cp16(void* dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
                  :: "r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))), "l"(src) : "memory");
 }
 __global__ void __launch_bounds__(256, 2)
-segment_correction_kernel(const float* __restrict__ seg_states, const float* __restrict__ wbuf,
-                          float* __restrict__ out, int T, int H, int nseg, int seg_len)
+segment_correction_kernel(const float* __restrict__ seg_states, const __half* __restrict__ wbuf,
+                          float* __restrict__ out, int T, int H, int nseg, int seg_len, int seg_first,
+                          const int* __restrict__ trans_len)
 {
     using namespace wmma16;
     extern __shared__ __align__(16) unsigned char corr_raw[];
     CorrSmem& m = *reinterpret_cast<CorrSmem*>(corr_raw);
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int h = blockIdx.y % H, seg = blockIdx.y / H, b = blockIdx.z;
-    const int t_begin = seg * seg_len, t_end = min(T, t_begin + seg_len);
+    const int h = blockIdx.y % H, seg = seg_first + (int)blockIdx.y / H, b = blockIdx.z;
+    const int t_begin = seg * seg_len;
+    // Tokens past the chunks the segment's transition ran have w = 0 (it
+    // stopped once M had decayed below fp32 resolution): nothing to add.
+    const int t_end = min(min(T, t_begin + seg_len),
+                          trans_len ? t_begin + trans_len[((long)b * nseg + seg) * H + h] * C : T);
     const int tile0 = blockIdx.x * CORR_TILES;
     if (t_begin + tile0 * C >= t_end) return;
     // Tile i's w into stage i & 1 (one commit group; rows past the segment zero).
     auto fetch = [&](int i) {
         const int t0 = t_begin + (tile0 + i) * C;
         if (i < CORR_TILES && t0 < t_end) {
-            for (int idx = tid; idx < C * D / 4; idx += 256) {
-                const int r = idx / (D / 4), q4 = 4 * (idx % (D / 4));
-                float* dst = &m.w[i & 1][r][q4];
-                if (t0 + r < t_end) corr_cp16(dst, wbuf + (((long)b * T + t0 + r) * H + h) * D + q4);
-                else *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int idx = tid; idx < C * D / 8; idx += 256) {
+                const int r = idx / (D / 8), q8 = 8 * (idx % (D / 8));
+                __half* dst = &m.w[i & 1][r][q8];
+                if (t0 + r < t_end) corr_cp16(dst, wbuf + (((long)b * T + t0 + r) * H + h) * D + q8);
+                else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
             }
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
@@ -983,8 +1100,7 @@ segment_correction_kernel(const float* __restrict__ seg_states, const float* __r
             }
         float acc[8][4];
         zero_acc(acc);
-        const float (*wt)[D + 4] = m.w[i & 1];
-        wmm_f16<8, D, true, D + 8>(acc, rb, cb, [&](int r, int k) { return wt[r][k]; }, &m.s[0][0]);
+        wmm_f16_ah<8, D, true, D + 8, D + 8>(acc, rb, cb, &m.w[i & 1][0][0], &m.s[0][0]);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
 #pragma unroll
@@ -1000,48 +1116,35 @@ segment_correction_kernel(const float* __restrict__ seg_states, const float* __r
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
-int sm_count() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-            n = 148;
-    }
-    return n;
-}
-
-// Number of time segments per (batch, head).  Segmenting costs two chunk
-// passes (zero-start states and outputs, transitions) and a correction
-// instead of one pass, so it pays only when the (batch, head) pairs alone
-// leave most SMs idle.
-int choose_segments(int requested, int BH, int nchunks) {
+// Number of time segments per (batch, head).  Segmenting costs a second
+// chunk recursion per segment (the transition) and a correction, so it pays
+// only when the (batch, head) pairs alone leave most SMs idle.  Automatic
+// choice: one segment per SM (B*H*n <= #SMs) where the transitions are
+// expected to end early (scalar gate, cheap_transitions); otherwise the
+// largest n whose B*H*(2n - 1) CTAs fit in one wave; at least 3 segments.
+int choose_segments(int requested, int BH, int nchunks, bool cheap_transitions) {
     if (nchunks <= 1 || requested == 1) return 1;
     int n = requested;
     if (n <= 0) {
         const int sms = sm_count();
         if (nchunks < 64 || BH * 4 > sms) return 1;
-        n = sms / BH;
+        n = cheap_transitions ? sms / BH : (sms / BH + 1) / 2;
+        if (n < 3) return 1;
     }
     return n < nchunks ? n : nchunks;
 }
 
 template <bool CHANNEL>
 cudaError_t launch(const Problem& p, cudaStream_t stream) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(chunk_fwd_kernel<CHANNEL>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    cudaError_t ea = set_smem_limit(reinterpret_cast<const void*>(chunk_fwd_kernel<CHANNEL>), SMEM_BYTES);
+    if (ea != cudaSuccess) return ea;
     CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, p.q, p.H, p.T, p.B) || !make_map(&mk, p.k, p.H, p.T, p.B) ||
         !make_map(&mv, p.v, p.H, p.T, p.B) || !make_out_map(&mo, p.out, p.H, p.T, p.B))
         return cudaErrorInvalidValue;
     float* out = static_cast<float*>(p.out);
     const int nchunks = (p.T + C - 1) / C;
-    int nseg = choose_segments(p.segments, p.B * p.H, nchunks);
+    int nseg = choose_segments(p.segments, p.B * p.H, nchunks, !CHANNEL);
     if (nseg <= 1) {
         // Chunk-local work and the state chain on different SMs when two per
         // (batch, head) fit: by default one prep pool over all SMs; a cluster
@@ -1055,8 +1158,9 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
             cudaError_t e = launch_chunk_pair_sm100(p, stream, pool ? sm_count() : 0);
             if (pool && e == cudaErrorMemoryAllocation) {
                 // No room for the pool's task records (nothing was launched):
-                // the cluster form needs no scratch.
-                (void)cudaGetLastError();
+                // the cluster form needs no scratch.  The failed allocation
+                // is the pending error, if any, that is cleared here.
+                if (cudaPeekAtLastError() == cudaErrorMemoryAllocation) (void)cudaGetLastError();
                 e = launch_chunk_pair_sm100(p, stream, 0);
             }
             return e;
@@ -1066,47 +1170,51 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
         chunk_fwd_kernel<CHANNEL><<<p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mo, prm);
         return cudaGetLastError();
     }
-    // Segment-parallel path in two chunk passes.  One launch runs every
-    // segment from a zero state, writing its outputs and end state, and, in a
-    // second set of CTAs, the transition M with v = 0 from the identity,
-    // writing w_t = M_t^T q_t per token.  A serial combine turns the end
-    // states into true start states; the correction then adds S_start^T w_t
-    // to every output (the state map is affine: S_t = M_t S_start + S_t(0)).
+    // Segment-parallel path in two chunk passes.  One launch runs segment 0
+    // from the true initial state and every other segment from a zero state,
+    // writing outputs and end states, and, in a second set of CTAs, the
+    // transitions M of segments 1 .. n-1 with v = 0 from the identity,
+    // writing w_t = M_t^T q_t per token (fp16).  A serial combine turns the
+    // end states into true start states; the correction then adds
+    // S_start^T w_t to the outputs of segments 1 .. n-1 (the state map is
+    // affine: S_t = M_t S_start + S_t(0)).
     const int seg_len = ((nchunks + nseg - 1) / nseg) * C;
     nseg = (p.T + seg_len - 1) / seg_len;
     const size_t slab = (size_t)p.B * nseg * p.H * D * D;
     const size_t wlen = (size_t)p.B * p.T * p.H * D;
     float* ws = nullptr;
-    cudaError_t e = workspace_alloc(reinterpret_cast<void**>(&ws), (2 * slab + wlen) * sizeof(float), stream);
+    const size_t nlen = ((size_t)p.B * nseg * p.H + 3) / 4 * 4;   // ints, 16-byte multiple
+    cudaError_t e = workspace_alloc(reinterpret_cast<void**>(&ws),
+                                    2 * slab * sizeof(float) + nlen * sizeof(int) + wlen * sizeof(__half),
+                                    stream);
     if (e != cudaSuccess) return e;
     float* seg_states = ws;
     float* trans = ws + slab;
-    float* wbuf = ws + 2 * slab;
+    int* trans_len = reinterpret_cast<int*>(ws + 2 * slab);
+    __half* wbuf = reinterpret_cast<__half*>(trans_len + nlen);
     CUtensorMap mw;
-    if (!make_out_map(&mw, wbuf, p.H, p.T, p.B)) {
+    if (!make_half_map(&mw, wbuf, p.H, p.T, p.B)) {
         const cudaError_t ef = cudaFreeAsync(ws, stream);
         return ef != cudaSuccess ? ef : cudaErrorInvalidValue;
     }
-    Params p1{p.g, p.beta, nullptr, seg_states, trans, out, p.T, p.H, p.B, nseg, seg_len, 1, nseg};
+    Params p1{p.g, p.beta, p.state_in, seg_states, trans, out, p.T, p.H, p.B, nseg, seg_len, 1, nseg};
     p1.wout = wbuf;
-    chunk_fwd_kernel<CHANNEL><<<2 * p.B * nseg * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mw, p1);
+    p1.trans_first = 1;
+    p1.in_first_only = true;
+    p1.trans_len = trans_len;
+    chunk_fwd_kernel<CHANNEL><<<p.B * (2 * nseg - 1) * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mw, p1);
     e = cudaGetLastError();
     if (e == cudaSuccess) {
         combine_segments_kernel<<<p.B * p.H * (D / CB_COLS), 256, 0, stream>>>(
-            seg_states, trans, p.state_in, p.state_out, p.H, nseg);
+            seg_states, trans, p.state_in, p.state_out, p.H, nseg, 1);
         e = cudaGetLastError();
     }
     if (e == cudaSuccess) {
-        static bool corr_attr = false;
-        if (!corr_attr) {
-            e = cudaFuncSetAttribute(segment_correction_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)sizeof(CorrSmem));
-            corr_attr = e == cudaSuccess;
-        }
+        e = set_smem_limit(reinterpret_cast<const void*>(segment_correction_kernel), (int)sizeof(CorrSmem));
         if (e == cudaSuccess) {
             const int groups = (seg_len / C + CORR_TILES - 1) / CORR_TILES;
-            segment_correction_kernel<<<dim3(groups, nseg * p.H, p.B), 256, sizeof(CorrSmem), stream>>>(
-                seg_states, wbuf, out, p.T, p.H, nseg, seg_len);
+            segment_correction_kernel<<<dim3(groups, (nseg - 1) * p.H, p.B), 256, sizeof(CorrSmem), stream>>>(
+                seg_states, wbuf, out, p.T, p.H, nseg, seg_len, 1, CHANNEL ? nullptr : trans_len);
             e = cudaGetLastError();
         }
     }
@@ -1144,7 +1252,7 @@ template <bool CHANNEL>
 cudaError_t launch_noalloc(const Problem& p, cudaStream_t stream, bool* over_limit) {
     *over_limit = false;
     const int nchunks = (p.T + C - 1) / C;
-    int nseg = choose_segments(p.segments, p.B * p.H, nchunks);
+    int nseg = choose_segments(p.segments, p.B * p.H, nchunks, true);
     const int seg_len = ((nchunks + nseg - 1) / nseg) * C;
     if (nseg > 1) nseg = (p.T + seg_len - 1) / seg_len;
     const size_t slab = (size_t)p.B * nseg * p.H * D * D;
@@ -1152,13 +1260,8 @@ cudaError_t launch_noalloc(const Problem& p, cudaStream_t stream, bool* over_lim
         *over_limit = true;          // rejected before anything is launched
         return cudaErrorInvalidValue;
     }
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(chunk_fwd_kernel<CHANNEL>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    cudaError_t ea = set_smem_limit(reinterpret_cast<const void*>(chunk_fwd_kernel<CHANNEL>), SMEM_BYTES);
+    if (ea != cudaSuccess) return ea;
     CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, p.q, p.H, p.T, p.B) || !make_map(&mk, p.k, p.H, p.T, p.B) ||
         !make_map(&mv, p.v, p.H, p.T, p.B) || !make_out_map(&mo, p.out, p.H, p.T, p.B))
@@ -1182,7 +1285,7 @@ cudaError_t launch_noalloc(const Problem& p, cudaStream_t stream, bool* over_lim
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     combine_segments_kernel<<<p.B * p.H * (D / CB_COLS), 256, 0, stream>>>(
-        seg_states, trans, p.state_in, p.state_out, p.H, nseg);
+        seg_states, trans, p.state_in, p.state_out, p.H, nseg, 0);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     Params p2{p.g, p.beta, seg_states, nullptr, nullptr, out, p.T, p.H, p.B, nseg, seg_len, nseg, 1};
@@ -1199,6 +1302,9 @@ cudaError_t launch_noalloc(const Problem& p, cudaStream_t stream, bool* over_lim
 // again on the next call cost milliseconds.  Held: the largest workspace in
 // use at once.
 cudaError_t workspace_alloc(void** ptr, size_t bytes, cudaStream_t stream) {
+    // Test hook: scratch that cannot be had, as on a full device (nothing is
+    // allocated or launched).  Unset in normal use.
+    if (getenv("GDN_TEST_FAIL_WORKSPACE")) return cudaErrorMemoryAllocation;
     static std::mutex mu;
     static cudaMemPool_t pools[64] = {};
     int dev = 0;
@@ -1225,6 +1331,35 @@ cudaError_t workspace_alloc(void** ptr, size_t bytes, cudaStream_t stream) {
         }
     }
     return cudaMallocFromPoolAsync(ptr, bytes, pools[dev], stream);
+}
+
+cudaError_t set_smem_limit(const void* kernel, int bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    static std::mutex mu;
+    static std::map<std::pair<int, const void*>, int> done;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = done.find({dev, kernel});
+    if (it != done.end() && it->second >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done[{dev, kernel}] = bytes;
+    return e;
+}
+
+int sm_count() {
+    constexpr int kMaxDevices = 128;
+    static std::mutex mu;
+    static int n[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    std::lock_guard<std::mutex> lock(mu);
+    if (n[dev] == 0) {
+        int c = 0;
+        n[dev] = cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && c > 0
+                     ? c : 148;
+    }
+    return n[dev];
 }
 
 cudaError_t launch_chunk_sm100_noalloc(const Problem& p, cudaStream_t stream, bool* over_limit) {

@@ -64,6 +64,14 @@ cudaError_t launch_chunk_bwd(const BwdProblem& p, cudaStream_t stream);
 // with cudaFreeAsync on the same stream).
 cudaError_t workspace_alloc(void** ptr, size_t bytes, cudaStream_t stream);
 
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current
+// device.  The attribute belongs to the device that is current when it is
+// set, so it is set once per (device, kernel), under a lock.
+cudaError_t set_smem_limit(const void* kernel, int bytes);
+
+// Number of SMs of the current device (looked up once per device).
+int sm_count();
+
 // Chunkwise tensor-core prefill (bf16 I/O, dk = dv = 128, chunk of 64).
 // Returns cudaErrorNotSupported for shapes it does not handle.
 cudaError_t launch_chunk_sm100(const Problem& p, cudaStream_t stream);

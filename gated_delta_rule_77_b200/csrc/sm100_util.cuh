@@ -204,12 +204,31 @@ __device__ __forceinline__ unsigned int flag_acquire(const unsigned int* flag) {
 }
 
 // Bounded wait until *flag != 0 (acquire).  Returns false (and sets bit 0 of
-// *status) if the budget runs out.
-__device__ __forceinline__ bool flag_wait(const unsigned int* flag, unsigned int* status) {
+// *status) if `budget_ns` runs out.
+__device__ __forceinline__ bool flag_wait(const unsigned int* flag, unsigned int* status,
+                                          unsigned long long budget_ns = kWaitBudgetNs) {
     if (flag_acquire(flag) != 0) return true;
     const unsigned long long t0 = globaltimer();
     while (flag_acquire(flag) == 0) {
-        if (globaltimer() - t0 > kWaitBudgetNs) {
+        if (globaltimer() - t0 > budget_ns) {
+            atomicOr(status, 1u);
+            return false;
+        }
+        __nanosleep(64);
+    }
+    return true;
+}
+
+// Bounded wait until the counter *flag has reached `value` (acquire); the
+// counter only grows, and is compared with wrap-around.  Returns false (and
+// sets bit 0 of *status) if `budget_ns` runs out.
+__device__ __forceinline__ bool flag_wait_until(const unsigned int* flag, unsigned int value,
+                                                unsigned int* status,
+                                                unsigned long long budget_ns = kWaitBudgetNs) {
+    if ((int)(flag_acquire(flag) - value) >= 0) return true;
+    const unsigned long long t0 = globaltimer();
+    while ((int)(flag_acquire(flag) - value) < 0) {
+        if (globaltimer() - t0 > budget_ns) {
             atomicOr(status, 1u);
             return false;
         }

@@ -154,6 +154,36 @@ __device__ __forceinline__ void wmm_f16(float (&acc)[NT][4], int rb, int cb, FA 
     }
 }
 
+// As wmm_f16, with A read as fp16 pairs straight from a row-major half
+// array (leading dimension LDA) instead of through an accessor.
+template <int NT, int K, bool TRANS, int LD, int LDA>
+__device__ __forceinline__ void wmm_f16_ah(float (&acc)[NT][4], int rb, int cb, const __half* a,
+                                           const __half* bt) {
+    static_assert(NT % 2 == 0, "pairs of 8-column tiles");
+    const int l = threadIdx.x & 31, g = l >> 2, t = l & 3;
+    const int mi = l >> 3, rr = l & 7;
+    auto a2 = [&](int r, int k) { return *reinterpret_cast<const uint32_t*>(a + (long)r * LDA + k); };
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 16) {
+        uint32_t af[4];
+        af[0] = a2(rb + g, k0 + 2 * t);
+        af[1] = a2(rb + g + 8, k0 + 2 * t);
+        af[2] = a2(rb + g, k0 + 2 * t + 8);
+        af[3] = a2(rb + g + 8, k0 + 2 * t + 8);
+#pragma unroll
+        for (int jp = 0; jp < NT / 2; ++jp) {
+            const int n0 = cb + 16 * jp;
+            long off;
+            if (TRANS) off = (long)(k0 + rr + 8 * (mi & 1)) * LD + n0 + 8 * (mi >> 1);
+            else off = (long)(n0 + rr + 8 * (mi >> 1)) * LD + k0 + 8 * (mi & 1);
+            uint32_t bv[4];
+            if (TRANS) ldsm4t(bv, bt + off); else ldsm4(bv, bt + off);
+            mma16816_f16(acc[2 * jp], af, bv[0], bv[1]);
+            mma16816_f16(acc[2 * jp + 1], af, bv[2], bv[3]);
+        }
+    }
+}
+
 template <int NT>
 __device__ __forceinline__ void zero_acc(float (&acc)[NT][4]) {
 #pragma unroll

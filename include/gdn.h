@@ -100,11 +100,14 @@ enum { GDN_IO_BF16 = 0, GDN_IO_F32 = 1 };
  *   per-token pointers (q, k, v, g, beta, out) may then be NULL.
  * Scratch: with dk = dv = 128 and 2 * B * H <= the SM count, each chunk's
  * chunk-local results (T' or T and beta, P and the chain's operand tiles:
- * 99,072 bytes) pass from prep CTAs to the state chains through
- * B * H * ceil(T / 64) * (99,072 + 4) bytes of stream-ordered scratch on
- * `stream` from the library's pool, freed on `stream` when the call's kernel
- * completes.  If it cannot be had, the call runs the cluster form of the
- * same kernel, which needs none.
+ * 99,072 bytes) pass from prep CTAs to the state chains through a ring of
+ * at most 8 such records per (batch, head): at most
+ * B * H * (8 * 99,072 + 36) bytes (about 0.8 MB per (batch, head), whatever
+ * T) of stream-ordered scratch on `stream` from the library's pool, freed on
+ * `stream` when the call's kernel completes.  If it cannot be had, the call
+ * runs the cluster form of the same kernel, which needs none.
+ * After a call that gdn_check reports as GDN_ERR_TIMEOUT, out and state_out
+ * are undefined.
  */
 GDN_API int gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
                   const float* beta, const float* state_in, void* out, float* state_out,
@@ -175,8 +178,11 @@ GDN_API int gdn_chunk_fwd_segments(const void* q, const void* k, const void* v, 
  * before any stream capture.
  *
  * Sharing: all calls use the same array and leave their data in it.  A call
- * writes every scratch element before it reads it, so nothing is cleared
- * between calls -- but two calls whose kernels may run at the same time on
+ * that completes writes every scratch element before it reads it, so nothing
+ * is cleared between calls; after a call that gdn_check reports as
+ * GDN_ERR_TIMEOUT (a bounded wait gave up), out and state_out are undefined,
+ * since later kernels of that call may read scratch the abandoned pass never
+ * wrote.  Two calls whose kernels may run at the same time on
  * one GPU (different streams without ordering between them) race on the
  * array and give wrong results.  Order such calls on one stream.
  * Other arguments as gdn_chunk_fwd_segments.

@@ -22,6 +22,22 @@ def test_prefill_accounting_matches_hand_count():
                                                             + 6 * 128 * 128))
 
 
+def test_algorithmic_bytes_match_the_per_token_head_figures():
+    # q, k, v 768 B + g 4 B (scalar) + beta 4 B + out 256 B (bf16) per
+    # token-head, plus the final state (64 KiB per (b, h)); S0 = 0 is not read.
+    assert bench.algorithmic_bytes(CONFIGS[5]) == 262144 * 16 * 1032 + 16 * 65536
+    # Per-channel g is 512 B per token-head.
+    assert bench.algorithmic_bytes(CONFIGS[2]) == 8 * 2048 * 8 * 1540 + 64 * 65536
+    # S0 != 0 is read as well as S_T written.
+    assert bench.algorithmic_bytes(CONFIGS[3]) == 4 * 8192 * 12 * 1032 + 2 * 48 * 65536
+
+
+def test_chunk_path_kernels_follow_the_dispatch_rule():
+    assert len(bench.chunk_path_kernels(CONFIGS[5])) == 3            # 16 pairs: segments
+    assert bench.chunk_path_kernels(CONFIGS[2]) == ["chunk_pool_kernel"]
+    assert bench.chunk_path_kernels(CONFIGS[3]) == ["chunk_pool_kernel"]
+
+
 def test_decode_accounting_matches_hand_count():
     # 2 x 64 MiB of state + q,k,v bf16 + per-channel g + beta + fp32 out
     assert bench.decode_bytes(CONFIGS[4]) == 136_056_832
@@ -29,7 +45,8 @@ def test_decode_accounting_matches_hand_count():
 
 def test_reference_arm_prints_contract_line(capsys, monkeypatch):
     monkeypatch.setattr(bench, "cpu_cores", lambda: 2)
-    rc = bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"])
+    rc = bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3",
+                     "--sample-tokens", "512"])
     assert rc == 0
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
@@ -38,6 +55,7 @@ def test_reference_arm_prints_contract_line(capsys, monkeypatch):
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 2
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["config"]["T"] == 262144 and line["config"]["H"] == 16
 
 
 def _free_port():

@@ -210,3 +210,58 @@ def test_scalar_gate_beyond_the_bounded_domain(gdn, kernel, monkeypatch):
     ref_o, ref_s = _ref(x, False)
     assert oracle.rel_err(got_o, ref_o) <= TOL
     assert oracle.rel_err(got_s, ref_s) <= TOL
+
+
+def _gate_at_bound(x, pattern):
+    """Per-channel g at the edge of its domain [-5, 0] (model card, section 2.1:
+    g = -min(softplus(.), 160 / bs2), bs2 = 32).  "floor": g = -5 on every token
+    and channel, so a 64-token chunk decays by exp(-320) and every factor of
+    the factored decay sits at exp(+-80) or below.  "runs": runs of 7 tokens
+    alternate between -5 and 0, shifted per channel, so one chunk mixes full
+    decay and no decay; channels 0-7 stay at -5 and channels 8-15 at 0."""
+    B, T, H, dk = x["g"].shape
+    if pattern == "floor":
+        g = torch.full((B, T, H, dk), -5.0)
+    else:
+        t = torch.arange(T)[:, None]
+        c = torch.arange(dk)[None, :]
+        g = torch.where(((t // 7) + c) % 2 == 0, -5.0, 0.0)
+        g[:, 0:8] = -5.0
+        g[:, 8:16] = 0.0
+        g = g[None, :, None, :].expand(B, T, H, dk)
+    x["g"] = g.contiguous().float()
+    return x
+
+
+@pytest.mark.parametrize("kernel", ["single", "pair", "pool"])
+@pytest.mark.parametrize("pattern", ["floor", "runs"])
+def test_channel_gate_at_its_bound(gdn, kernel, pattern, monkeypatch):
+    x = _gate_at_bound(prefill_inputs(2, 300, 2, 128, 128, gate="channel", s0_std=0.1, seed=260),
+                       pattern)
+    monkeypatch.setenv("GDN_CHUNK_KERNEL", kernel)
+    got_o, got_s = _gpu(gdn, x)
+    ref_o, ref_s = _ref(x, True)
+    assert torch.isfinite(got_o).all() and torch.isfinite(got_s).all()
+    assert oracle.rel_err(got_o, ref_o) <= TOL
+    assert oracle.rel_err(got_s, ref_s) <= TOL
+    assert gdn.check() == gdn.GDN_OK
+
+
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+def test_second_device_in_the_same_process(gdn, gate):
+    """Kernel attributes (the shared-memory limit) and the SM count belong to a
+    device: a call on cuda:1 after one on cuda:0 in the same process must not
+    rely on settings made while cuda:0 was current."""
+    if torch.cuda.device_count() < 2:
+        pytest.skip("one GPU visible")
+    x = prefill_inputs(2, 300, 3, 128, 128, gate=gate, s0_std=0.1, seed=270)
+    ref_o, ref_s = _ref(x, gate == "channel")
+    for dev_index in (0, 1):
+        dev = torch.device("cuda", dev_index)
+        with torch.cuda.device(dev):
+            args = [x[n].to(dev) for n in ("q", "k", "v", "g", "beta")]
+            out, s = gdn.chunk_fwd(*args, x["s0"].to(dev))
+            torch.cuda.synchronize(dev)
+            assert oracle.rel_err(out.cpu(), ref_o) <= TOL, dev_index
+            assert oracle.rel_err(s.cpu(), ref_s) <= TOL, dev_index
+            assert gdn.check() == gdn.GDN_OK

@@ -83,3 +83,50 @@ def test_long_context_config_sampled_heads(gdn, oracle_threads):
                                   per_channel=False, threads=oracle_threads)
         assert oracle.rel_err(out[:, :, h:h + 1].cpu(), ref_o) <= cfg.tol, h
         assert oracle.rel_err(s[:, h:h + 1].cpu(), ref_s) <= cfg.tol, h
+
+
+@pytest.mark.parametrize("pattern", ["floor", "runs"])
+def test_segments_channel_gate_at_its_bound(gdn, pattern):
+    """Per-channel g at -5 (every token, or runs mixed with g = 0 inside a
+    chunk): the transitions of the segments decay to (near) zero and the
+    factored decay works at the edge of its range."""
+    from tests.test_gpu_chunk import _gate_at_bound
+    x = _gate_at_bound(prefill_inputs(1, 900, 2, 128, 128, gate="channel", s0_std=0.1, seed=320),
+                       pattern)
+    o_seg, s_seg = _run(gdn, x, 3)
+    ref_o, ref_s = oracle.run(x["q"], x["k"], x["v"], x["g"], x["beta"], x["s0"], per_channel=True)
+    assert torch.isfinite(o_seg).all() and torch.isfinite(s_seg).all()
+    assert oracle.rel_err(o_seg, ref_o) <= TOL
+    assert oracle.rel_err(s_seg, ref_s) <= TOL
+
+
+def test_segments_without_decay_run_full_transitions(gdn):
+    """g = 0 and a small beta: the transition of a segment barely decays, so
+    no transition may end early; the segmented result must still be exact."""
+    x = prefill_inputs(1, 1200, 2, 128, 128, gate="scalar", s0_std=0.1, seed=330)
+    x["g"].zero_()
+    x["beta"] = (0.02 * x["beta"]).contiguous()
+    o_seg, s_seg = _run(gdn, x, 4)
+    ref_o, ref_s = oracle.run(x["q"], x["k"], x["v"], x["g"], x["beta"], x["s0"], per_channel=False)
+    assert oracle.rel_err(o_seg, ref_o) <= TOL
+    assert oracle.rel_err(s_seg, ref_s) <= TOL
+
+
+@pytest.mark.parametrize("late", ["beta_above_one", "positive_g"])
+def test_segments_with_tokens_outside_the_contracting_domain(gdn, late):
+    """Fast decay first (the transitions would end after a chunk or two),
+    then tokens outside the domain that makes every step a contraction
+    (beta > 1, or g > 0): the early end must not be taken, and the result
+    must match the oracle."""
+    x = prefill_inputs(1, 1024, 2, 128, 128, gate="scalar", s0_std=0.1, seed=331)
+    g, beta = x["g"].clone(), x["beta"].clone()
+    g[:, :, :] = -3.0
+    if late == "beta_above_one":
+        beta[:, 600:610] = 1.8
+    else:
+        g[:, 600:610] = 0.05
+    x["g"], x["beta"] = g.contiguous(), beta.contiguous()
+    o_seg, s_seg = _run(gdn, x, 3)
+    ref_o, ref_s = oracle.run(x["q"], x["k"], x["v"], x["g"], x["beta"], x["s0"], per_channel=False)
+    assert oracle.rel_err(o_seg, ref_o) <= TOL
+    assert oracle.rel_err(s_seg, ref_s) <= TOL
