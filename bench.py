@@ -628,7 +628,22 @@ def run_prologue(gdn, dev, stream, peaks, world, rank):
     t_pre = max_over_ranks(median_single(
         lambda: gdn.prologue(*args, xd["ring"], xd["pos0"], stream=stream), stream, 20, 3), world)
     b_pre = prologue_bytes(pc.B, pc.T, pc.H, pc.dk, pc.dv, pc.per_channel)
-    del xd, args
+    # The same layer from its raw projections in one call: its default route
+    # (the two passes through scratch) and the fused kernel (the prologue
+    # inside the prefill), against the two calls timed apart.
+    out = torch.empty(pc.B, pc.T, pc.H, pc.dv, dtype=torch.float32, device=dev)
+    s_out = torch.empty(pc.B, pc.H, pc.dk, pc.dv, dtype=torch.float32, device=dev)
+    t_call = max_over_ranks(median_single(
+        lambda: gdn.chunk_fwd_prologue(*args, xd["ring"], xd["pos0"], None, out=out, state_out=s_out,
+                                       stream=stream), stream, 20, 3), world)
+    t_fused = max_over_ranks(median_single(
+        lambda: gdn.chunk_fwd_prologue(*args, xd["ring"], xd["pos0"], None, out=out, state_out=s_out,
+                                       fused=True, stream=stream), stream, 20, 3), world)
+    q, k, v, g, beta = gdn.prologue(*args, xd["ring"], xd["pos0"], stream=stream)
+    t_chunk = max_over_ranks(median_single(
+        lambda: gdn.chunk_fwd(q, k, v, g, beta, None, out=out, state_out=s_out, stream=stream),
+        stream, 20, 3), world)
+    del xd, args, q, k, v, g, beta, out, s_out
 
     dc = DECODE_CFG
     n_in, n_states = 16, 6
@@ -651,6 +666,8 @@ def run_prologue(gdn, dev, stream, peaks, world, rank):
     b_dec = decode_bytes(dc) + dc.B * dc.H * (3 + 1) * C * 4 + dc.H * C * 16
     hbm = peaks["hbm_gbs"]
     return {"prefill_pass_us": _r(t_pre * 1e6), "prefill_pass_frac": _r(b_pre / t_pre / 1e9 / hbm),
+            "layer_call_us": _r(t_call * 1e6), "fused_kernel_us": _r(t_fused * 1e6),
+            "two_calls_us": _r((t_pre + t_chunk) * 1e6),
             "decode_fused_us": _r(t_dec * 1e6), "decode_fused_frac": _r(b_dec / t_dec / 1e9 / hbm)}
 
 

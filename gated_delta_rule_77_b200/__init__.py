@@ -38,7 +38,8 @@ ACT_SILU = 1
 
 SYMBOLS = ("gdn_chunk_fwd", "gdn_chunk_fwd_ex", "gdn_chunk_fwd_segments",
            "gdn_chunk_fwd_segments_noalloc", "gdn_recurrent_step", "gdn_recurrent_step_ex",
-           "gdn_chunk_bwd", "gdn_recurrent_steps", "gdn_recurrent_steps_decoupled", "gdn_state_select", "gdn_prologue", "gdn_recurrent_step_prologue",
+           "gdn_chunk_bwd", "gdn_recurrent_steps", "gdn_recurrent_steps_decoupled", "gdn_state_select",
+           "gdn_prologue", "gdn_recurrent_step_prologue", "gdn_chunk_fwd_prologue",
            "gdn_check", "gdn_status_string")
 
 _lib = None
@@ -76,6 +77,8 @@ def load() -> ctypes.CDLL:
                                  i, i, vp]
     lib.gdn_recurrent_step_prologue.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, fp, fp, vp, i, i, i,
                                                 i, i, i, vp]
+    lib.gdn_chunk_fwd_prologue.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, fp, vp, fp, i, i, i, i,
+                                           i, i, i, i, vp]
     lib.gdn_check.argtypes = [vp]
     lib.gdn_status_string.argtypes = [i]
     lib.gdn_status_string.restype = ctypes.c_char_p
@@ -302,6 +305,38 @@ def recurrent_step_prologue(q_raw, k_raw, v_raw, g_raw, beta_raw, conv_w, ring, 
     if rc != GDN_OK:
         raise GdnError(rc, "gdn_recurrent_step_prologue")
     return out
+
+
+def chunk_fwd_prologue(q_raw, k_raw, v_raw, g_raw, beta_raw, conv_w, ring=None, pos0=None,
+                       state_in=None, *, activation: str = "silu", out=None, state_out=None,
+                       return_state: bool = True, fused: bool = False, stream=None):
+    """The prefill from a layer's raw projections (gdn_chunk_fwd_prologue):
+    the prologue of ``prologue``, then the recurrence -- as two passes
+    through scratch, or with ``fused`` applied inside the prefill kernel while
+    it loads (dk = dv = 128; other shapes take the two passes).  Arguments as
+    ``prologue`` and ``chunk_fwd``; the ring (if given) is read and updated.
+    Returns (out [B,T,H,dv] fp32, final state or None)."""
+    B, T, H, dk = q_raw.shape
+    dv = v_raw.shape[-1]
+    gate = GATE_CHANNEL if g_raw.dim() == 4 else GATE_SCALAR
+    dev = v_raw.device
+    if out is None:
+        out = torch.empty(B, T, H, dv, dtype=torch.float32, device=dev)
+    if state_out is None and return_state:
+        state_out = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
+    _check_cuda(q_raw, k_raw, v_raw, g_raw, beta_raw, conv_w, ring, pos0, state_in, out, state_out)
+    if q_raw.dtype != torch.bfloat16 or v_raw.dtype != torch.bfloat16:
+        raise ValueError("q_raw, k_raw and v_raw must be bf16")
+    if pos0 is not None and pos0.dtype != torch.int32:
+        raise ValueError("pos0 must be int32")
+    rc = load().gdn_chunk_fwd_prologue(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(g_raw),
+                                       _ptr(beta_raw), _ptr(conv_w), _ptr(ring), _ptr(pos0),
+                                       _ptr(state_in), _ptr(out), _ptr(state_out), B, T, H, dk, dv,
+                                       gate, _act_code(activation), int(bool(fused)),
+                                       _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_chunk_fwd_prologue")
+    return out, state_out
 
 
 def check(stream=None) -> int:

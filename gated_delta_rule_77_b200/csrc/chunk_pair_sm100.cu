@@ -57,6 +57,7 @@
 
 #include "chunk_common.cuh"
 #include "gdn_internal.cuh"
+#include "prologue_math.cuh"
 #include "sm100_util.cuh"
 
 #include <cstdlib>
@@ -110,6 +111,12 @@ constexpr uint32_t P_USED = P_G + 32768;
 // Pool form, scalar gate: K*E bf16 [half][64 r][128 B] for the prep's own
 // W^T product (the per-channel X operands' space, unused with a scalar gate).
 constexpr uint32_t P_KE = P_X;
+// Fused prologue, prep CTA, before the X operands are built (same space):
+// q and k history rows [2][3][128] fp32, taps of q | k [256] float4, and the
+// per-channel-chunk sums of squares [16][64] fp32.
+constexpr uint32_t P_PH = P_X;
+constexpr uint32_t P_PW = P_X + 3072;
+constexpr uint32_t P_PS = P_X + 7168;
 
 // ---- CTA 1 (chain) shared memory ----------------------------------------------
 constexpr uint32_t C_IN = 0;                  // 32 KB raw K, Q
@@ -130,13 +137,19 @@ constexpr uint32_t C_LAST = C_GAM + 256;      // 128 f32
 constexpr uint32_t C_BAR = C_LAST + 512;      // tma_kq, tma_v, mma, full, out, full_b, full_c
 constexpr uint32_t C_TMEM = C_BAR + 56;
 constexpr uint32_t C_FETCHED = C_TMEM + 8;    // 3 int: record parts fetched (pool form)
-constexpr uint32_t C_USED = C_FETCHED + 16;
+constexpr uint32_t C_USED_BASE = C_FETCHED + 16;
+// Fused prologue (pool form): v's history rows [3][128] fp32 and taps [128] float4.
+constexpr uint32_t C_HV = C_USED_BASE;
+constexpr uint32_t C_TV = C_HV + 1536;
+constexpr uint32_t C_USED = C_TV + 2048;
 
 constexpr uint32_t SLOT_BYTES = 32768;
 
 // Pool form: task records kept per (batch, head) at once (a ring; >= 4 for
-// progress, see PairParams).
+// progress, see PairParams), and the scratch the records may take before the
+// ring is shortened to kPoolRing slots.
 constexpr int kPoolRing = 8;
+constexpr size_t kPoolScratchBytes = size_t(256) << 20;
 static_assert(kPoolRing >= 4, "the record ring needs at least 4 slots");
 
 // Pool form: one task's record in the global buffer, in three parts that the
@@ -176,9 +189,11 @@ struct PairParams {
     // may rewrite slot c % ring when consumed >= c - ring + 1.  All zero at
     // launch.  The chain publishes consumed = c - 1 while it works on chunk
     // c + 1 (it has read chunk c - 1's record by then).  With ring >= 4 this
-    // cannot deadlock: the unfinished task of lowest index (chunk-major
-    // order) waits only for its chain to reach chunk c - ring + 2, which
-    // needs records of lower index only.
+    // cannot deadlock: a prep CTA publishes its finished record before it
+    // waits for a slot, so every task of lower index than the unfinished one
+    // of lowest index (chunk-major order) has its record published, and that
+    // task waits only for its chain to reach chunk c - ring + 2, which needs
+    // records of lower index only.
     uint8_t* slots;            // [B*H][ring][TASK_BYTES]
     unsigned int* flags;       // [B*H][ring]
     unsigned int* consumed;    // [B*H]
@@ -190,9 +205,89 @@ struct PairParams {
     // wait for chains, so the launch still ends.
     unsigned long long flag_budget_ns;
     long long withheld_task;
+    // Fused input prologue (pool form with PRO): the tensor maps and g, beta
+    // point at the layer's raw projections, and the kernel applies the width-4
+    // causal convolution (history from the ring), the activation, the q/k L2
+    // norm and the gate maps while loading them, as gdn_prologue would.
+    const float* conv_w = nullptr;          // [H, 3D, 4], channels q | k | v
+    const float* conv_ring = nullptr;       // [B, H, 4, 3D] or null: history ring
+    const int* pos0 = nullptr;              // [B] or null (0)
+    const __nv_bfloat16* q_raw = nullptr;   // [B, T, H, D]: history rows
+    const __nv_bfloat16* k_raw = nullptr;
+    const __nv_bfloat16* v_raw = nullptr;
+    bool silu = true;
 };
 
-template <bool CHANNEL, bool POOL>
+// Fused prologue: one 64-token tile of one tensor (bf16, TMA layout: halves
+// of 64 channels `half_stride` bytes apart, [64 tokens][128 B], 128-byte
+// swizzle) becomes the recurrence's input in place: the width-4 causal
+// convolution (tap 3 on the current token; `hist` [3][128] fp32 holds the
+// three tokens before the tile), the activation, the L2 norm over the 128
+// channels when `norm` (x (sum x^2 + 1e-6)^-1/2), bf16 rounding; rows at or
+// past `nvalid` become zero.  Thread t of 256 takes channels 2 (t & 63) and
+// 2 (t & 63) + 1 over tokens 16 (t >> 6) .. + 15, the tap window sliding in
+// registers; a token's sum of squares is the butterfly total of its block's
+// two warps (`ss` 8 x 16 fp32 of shared scratch).  With keep_last, the raw
+// tokens 61-63 replace `hist` (the next consecutive tile's history).  Ends
+// with a proxy fence and a barrier (the tensor core may read the tile next).
+__device__ __forceinline__ void pro_convert_tile(uint8_t* tile, uint32_t half_stride, float* hist,
+                                                 const float4* taps, float* ss, int nvalid, bool silu,
+                                                 bool norm, bool keep_last, int tid) {
+    using namespace prologue_math;
+    const int cp = tid & 63, blk = tid >> 6, lane = tid & 31, warp = tid >> 5;
+    const int c = 2 * cp;
+    uint8_t* col = tile + (c >> 6) * half_stride + ((c & 7) << 1);
+    const uint32_t chunk = (c & 63) >> 3;
+    const float4 w0 = taps[c], w1 = taps[c + 1];
+    const float2 ta = make_float2(w0.x, w1.x), tb = make_float2(w0.y, w1.y);
+    const float2 tc = make_float2(w0.z, w1.z), td = make_float2(w0.w, w1.w);
+    const int r0 = 16 * blk;
+    auto row = [&](int r) -> float2 {
+        if (r >= 0) return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(col + swz(r, chunk)));
+        return make_float2(hist[(3 + r) * D + c], hist[(3 + r) * D + c + 1]);
+    };
+    float2 win[3] = {row(r0 - 3), row(r0 - 2), row(r0 - 1)};
+    float2 y[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float2 x = row(r0 + i);
+        const float2 a = fma2(ta, win[0], fma2(tb, win[1], fma2(tc, win[2], mul2(td, x))));
+        y[i] = r0 + i < nvalid ? act_fn2(a, silu) : make_float2(0.f, 0.f);
+        win[0] = win[1]; win[1] = win[2]; win[2] = x;
+    }
+    if (norm) {
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = fmaf(y[i].x, y[i].x, y[i].y * y[i].y);
+        butterfly_sums16(v, lane);
+        if ((lane & 1) == 0) ss[warp * 16 + butterfly_token(lane)] = v[0];
+    }
+    __syncthreads();                          // every raw row read; the sums in
+    // Lane l computes the inverse norm of token r0 + (l & 15) once; row i
+    // takes it from lane i.
+    float inv_l = 1.f;
+    if (norm) inv_l = rsqrtf(ss[(2 * blk) * 16 + (lane & 15)] + ss[(2 * blk + 1) * 16 + (lane & 15)] + 1e-6f);
+    if (keep_last && blk == 3) {              // raw tokens 61-63: the next tile's history
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {
+            hist[i * D + c] = win[i].x;
+            hist[i * D + c + 1] = win[i].y;
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        float2 o = y[i];
+        if (norm) {
+            const float inv = __shfl_sync(0xffffffffu, inv_l, i);
+            o.x *= inv; o.y *= inv;
+        }
+        *reinterpret_cast<__nv_bfloat162*>(col + swz(r0 + i, chunk)) = __floats2bfloat162_rn(o.x, o.y);
+    }
+    fence_async_smem();
+    __syncthreads();
+}
+
+template <bool CHANNEL, bool POOL, bool PRO = false>
 __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                                           const CUtensorMap& tm_v, const CUtensorMap& tm_o,
                                           const CUtensorMap& tm_g, const PairParams& p)
@@ -337,6 +432,17 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             if (with_beta) bg[1] = p.beta[tk0 + (long)(32 + lane) * H];
             if (!CHANNEL) bg[3] = p.g[tk0 + (long)(32 + lane) * H];
         }
+        if (PRO) {   // raw projections: beta = sigmoid, g = -min(softplus, 5); padding stays 0
+            using namespace prologue_math;
+            if (t0 + lane < T) {
+                if (with_beta) bg[0] = sigmoid_fn(bg[0]);
+                if (!CHANNEL) bg[2] = gate_fn(bg[2]);
+            }
+            if (t0 + 32 + lane < T) {
+                if (with_beta) bg[1] = sigmoid_fn(bg[1]);
+                if (!CHANNEL) bg[3] = gate_fn(bg[3]);
+            }
+        }
     };
     auto gate_scalar = [&](const float (&bg)[4], float* sGam, float* sBeta, float* sEr = nullptr,
                            float* sFj = nullptr, int* sSafe = nullptr) {
@@ -413,6 +519,37 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             }
         };
         int kq_issued = 0;                    // K, Q loads issued (tid 0), for the drain
+        auto item_valid = [&](int j) {   // tokens of item j's chunk inside the sequence
+            int ib, ih, ic;
+            item(j, ib, ih, ic);
+            return T - ic * C < C ? T - ic * C : C;
+        };
+        // Fused prologue: item j's history rows (tokens t0-3 .. t0-1 of q and
+        // k: thread tid takes channel tid & 127 of q (tid < 128) or k, from
+        // the raw inputs, or from the ring before the first token) and the
+        // taps of conv channel tid (q | k), into registers one item ahead.
+        float hq[3] = {0.f, 0.f, 0.f};
+        float4 tq = make_float4(0.f, 0.f, 0.f, 0.f);
+        auto pro_load = [&](int j) {
+            if (!PRO) return;
+            int ib, ih, ic;
+            item(j, ib, ih, ic);
+            const int tn = tid >> 7, ch = tid & 127;
+            const __nv_bfloat16* raw = tn == 0 ? p.q_raw : p.k_raw;
+            const int p0 = p.pos0 ? p.pos0[ib] : 0;
+#pragma unroll
+            for (int i = 0; i < 3; ++i) {
+                const int t = ic * C - 3 + i;
+                float x = 0.f;
+                if (t >= 0) {
+                    x = __bfloat162float(raw[(((long)ib * T + t) * H + ih) * D + ch]);
+                } else if (p.conv_ring && p0 + t >= 0) {
+                    x = p.conv_ring[(((long)ib * H + ih) * 4 + ((p0 + t) & 3)) * (3 * D) + tn * D + ch];
+                }
+                hq[i] = x;
+            }
+            tq = *reinterpret_cast<const float4*>(p.conv_w + ((long)ih * 3 * D + tid) * 4);
+        };
         auto issue_kq = [&](int j) {
             int ib, ih, ic;
             item(j, ib, ih, ic);
@@ -454,9 +591,26 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
         // Wait for a g tile, scan it in place (thread c < 128 runs the 64
         // tokens of channel c in order; a row of a box is 32 channels on 32
         // banks), then read this thread's values.  Every thread calls it.
-        auto scan_g = [&](float (&gn)[4][8]) {
+        auto scan_g = [&](float (&gn)[4][8], int nvalid) {
             ok = ok && mbar_wait(bar_g, g_waited & 1, &g_pair_status_word);
             ++g_waited;
+            if (PRO) {   // raw g: g = -min(softplus, 5) on the chunk's tokens, padding 0; all threads
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int f = tid + NT * j, r = f >> 5, c4 = f & 31;
+                    float4* a = reinterpret_cast<float4*>(smem + P_G + (c4 >> 3) * 8192 + swz(r, c4 & 7));
+                    float4 v = *a;
+                    if (r < nvalid) {
+                        const float2 lo = prologue_math::gate_fn2(make_float2(v.x, v.y));
+                        const float2 hi = prologue_math::gate_fn2(make_float2(v.z, v.w));
+                        v = make_float4(lo.x, lo.y, hi.x, hi.y);
+                    } else {
+                        v = make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+                    *a = v;
+                }
+                __syncthreads();
+            }
             if (tid < D) {
                 uint8_t* col = smem + P_G + (tid >> 5) * 8192 + (tid & 3) * 4;
                 const uint32_t cchunk = (tid & 31) >> 2;
@@ -495,11 +649,14 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
         float gnext[4][8], bgnext[4];
         if (CHANNEL && nitems > 0) {
             if (tid == 0) { issue_g(0); g_issued = 1; }
-            scan_g(gnext);
+            scan_g(gnext, item_valid(0));
             __syncthreads();                      // item 0's g has been read
             if (tid == 0 && nitems > 1) { issue_g(1); g_issued = 2; }
         }
-        if (nitems > 0) beta_load(0, bgnext);
+        if (nitems > 0) {
+            beta_load(0, bgnext);
+            pro_load(0);
+        }
 
         bool next_slot_free = false;           // tid 0: the next item's slot found free
         for (int ci = 0; ci < nitems; ++ci) {
@@ -526,18 +683,47 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             // beta (and a scalar g) were loaded one chunk ahead.
             gate_scalar(bgnext, sGam, sBeta, sEr, sFj, sSafe);
             if (CHANNEL && ci + 1 < nitems) beta_load(ci + 1, bgnext);
+            // (the fused prologue's next history rows and taps are loaded after
+            // this item's conversion, below)
             ok = ok && mbar_wait(bar_tma, ci & 1, &g_pair_status_word);
             kq_waited = ci;
-            if (POOL && tid == 0 && item_chunk >= p.ring) {
+            if (POOL && tid == 0 && item_chunk >= p.ring && !slot_free) {
                 // The slot's previous record (chunk - ring) must have been
                 // read by its chain before anything is stored into it
                 // (usually found so already while the previous item's X ran).
-                if (!slot_free)
-                    ok = ok && flag_wait_until(p.consumed + item_pair, (unsigned)(item_chunk - p.ring + 1),
-                                               &g_pair_status_word);
+                // The previous item's record is published first: a prep CTA
+                // never waits while it holds a finished record, so that the
+                // unfinished task of lowest index always has every earlier
+                // record published (the ring's progress argument).
+                if (copy_pending) {
+                    publish();
+                    copy_pending = false;
+                }
+                ok = ok && flag_wait_until(p.consumed + item_pair, (unsigned)(item_chunk - p.ring + 1),
+                                           &g_pair_status_word);
                 fence_proxy_async_global();
             }
             if (__syncthreads_or(!ok)) break;
+
+            if constexpr (PRO) {
+                // Fused prologue: the raw q and k tiles become the recurrence's
+                // inputs in place, as gdn_prologue computes them (see
+                // pro_convert_tile); the history rows and taps were loaded a
+                // task ahead.
+                float* sH = reinterpret_cast<float*>(smem + P_PH);
+                float4* sW = reinterpret_cast<float4*>(smem + P_PW);
+                float* sS = reinterpret_cast<float*>(smem + P_PS);
+                {
+                    const int tn = tid >> 7, ch = tid & 127;
+#pragma unroll
+                    for (int i = 0; i < 3; ++i) sH[(tn * 3 + i) * D + ch] = hq[i];
+                    sW[tid] = tq;
+                }
+                __syncthreads();
+                const int nvalid = T - item_chunk * C < C ? T - item_chunk * C : C;
+                pro_convert_tile(smem + P_IN + 8192, 16384, sH, sW, sS, nvalid, p.silu, true, false, tid);
+                pro_convert_tile(smem + P_IN, 16384, sH + 3 * D, sW + D, sS, nvalid, p.silu, true, false, tid);
+            }
 
             if (CHANNEL) {
                 // Channel pairs on the paired fp32 instructions.  Tokens
@@ -631,6 +817,10 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                         (int)(flag_acquire(p.consumed + nb * H + nh) - (unsigned)(nc - p.ring + 1)) >= 0;
                 }
             }
+            // Fused prologue: the next task's history rows and taps, loaded
+            // here, where no proxy fence follows soon (a shared-memory proxy
+            // fence waits for the thread's own outstanding global loads).
+            if (PRO && ci + 1 < nitems) pro_load(ci + 1);
             // While X runs: the chain's operands (pool form) and the next
             // chunk's g (the X build of this chunk has read sRef0/1 already).
             if (POOL && CHANNEL) {    // the chain's operands K*E, Q*E and K*D, exp(G_last)
@@ -663,7 +853,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                 }
                 if (tid < D) reinterpret_cast<float*>(gslot + TC_EL)[tid] = __expf(my_last);
             }
-            if (CHANNEL && ci + 1 < nitems) scan_g(gnext);
+            if (CHANNEL && ci + 1 < nitems) scan_g(gnext, item_valid(ci + 1));
             if (POOL && !CHANNEL) {   // the chain's operands Q*E and K*D, exp(G_last); K*E here
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
@@ -981,6 +1171,39 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             fetch_part(0, 1);
             fetch_part(0, 2);
         }
+        // Fused prologue: v's taps (conv channels 2D .. 3D - 1 of this head)
+        // and chunk 0's history rows of v (tokens -3 .. -1: the ring or zero;
+        // thread tid < 128 takes channel tid) once; each later chunk's history
+        // is its predecessor's raw last three tokens, kept by the conversion.
+        float hv[3] = {0.f, 0.f, 0.f};
+        auto pro_load_v = [&](int chunk) {
+            if (!PRO || tid >= D) return;
+            const int p0 = p.pos0 ? p.pos0[b] : 0;
+#pragma unroll
+            for (int i = 0; i < 3; ++i) {
+                const int t = chunk * C - 3 + i;
+                float x = 0.f;
+                if (t >= 0) x = __bfloat162float(p.v_raw[(((long)b * T + t) * H + h) * D + tid]);
+                else if (p.conv_ring && p0 + t >= 0)
+                    x = p.conv_ring[(((long)b * H + h) * 4 + ((p0 + t) & 3)) * (3 * D) + 2 * D + tid];
+                hv[i] = x;
+            }
+        };
+        auto pro_store_v = [&]() {
+            if (!PRO || tid >= D) return;
+            float* sHV = reinterpret_cast<float*>(smem + C_HV);
+#pragma unroll
+            for (int i = 0; i < 3; ++i) sHV[i * D + tid] = hv[i];
+        };
+        if (PRO) {
+            if (tid < D)
+                reinterpret_cast<float4*>(smem + C_TV)[tid] =
+                    *reinterpret_cast<const float4*>(p.conv_w + ((long)h * 3 * D + 2 * D + tid) * 4);
+            if (nchunks > 0) {       // chunk 0's history; later chunks keep their predecessor's
+                pro_load_v(0);
+                pro_store_v();
+            }
+        }
         // A first record that never came: no chunk starts (every thread
         // learns it here, before any wait of the loop).
         const bool started = !POOL || !__syncthreads_or(!ok);
@@ -1086,6 +1309,13 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             ok = ok && mbar_wait(bar_v, ci & 1, &g_pair_status_word);
             v_waited = ci;
             if (__syncthreads_or(!ok)) break;
+            if constexpr (PRO) {
+                // Fused prologue: the raw v tile becomes the recurrence's v in
+                // place (convolution, activation, bf16; no norm).
+                pro_convert_tile(smem + C_V, 8192, reinterpret_cast<float*>(smem + C_HV),
+                                 reinterpret_cast<const float4*>(smem + C_TV), nullptr,
+                                 T - t0 < C ? T - t0 : C, p.silu, false, true, tid);
+            }
 
           if (!W_READY) {
             if (tid == 0) {
@@ -1226,7 +1456,8 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             // previous chunk, before its barriers: their slots may be reused.
             // (Released here, where this thread waits for the products anyway:
             // the release's fence costs the chain nothing.)
-            if (POOL && tid == 32 && ci > 1) flag_release(p.consumed + pair, (unsigned)(ci - 1));
+            if (POOL && p.ring < nchunks && tid == 32 && ci > 1)
+                flag_release(p.consumed + pair, (unsigned)(ci - 1));
             mma_sync();
             if (__syncthreads_or(!ok)) break;
             if (POOL && tid == NT - 32 && ci + 1 < nchunks) fetch_part(ci + 1, 1);   // Q*E consumed
@@ -1335,6 +1566,16 @@ chunk_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     pair_body<CHANNEL, true>(tm_q, tm_k, tm_v, tm_o, tm_g, p);
 }
 
+// The pool form with the layer's input prologue applied while loading.
+template <bool CHANNEL>
+__global__ void __launch_bounds__(NT, 1)
+chunk_pool_prologue_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                           const __grid_constant__ CUtensorMap tm_g, const PairParams p)
+{
+    pair_body<CHANNEL, true, true>(tm_q, tm_k, tm_v, tm_o, tm_g, p);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     // Same entry point for every device; initialised once, thread-safely.
     static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
@@ -1390,45 +1631,27 @@ bool make_map(CUtensorMap* map, const void* base, int H, int T, int B) {
     return r == CUDA_SUCCESS;
 }
 
-template <bool CHANNEL>
-cudaError_t launch_pair(const Problem& p, cudaStream_t stream, int pool_ctas) {
-    {
-        cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(chunk_pair_kernel<CHANNEL>), SMEM_BYTES);
-        if (e == cudaSuccess)
-            e = set_smem_limit(reinterpret_cast<const void*>(chunk_pool_kernel<CHANNEL>), SMEM_BYTES);
-        if (e != cudaSuccess) return e;
+// Pool-form launch shared by the plain and the fused-prologue kernels: the
+// task-record ring from the stream-ordered workspace (flags and counters
+// first, 1 KB aligned, cleared on the stream before the launch), then one
+// cooperative launch of pool_ctas CTAs.  Ring depth: every chunk gets its own
+// slot while all records fit in kPoolScratchBytes (no slot is reused, so
+// nothing waits for a chain); beyond that, as many slots per (batch, head)
+// as fit, at least kPoolRing.  *too_large: the cooperative launch could not
+// fit (only the memset ran).
+template <typename Kernel>
+cudaError_t launch_pool_ring(Kernel kernel, const CUtensorMap& mq, const CUtensorMap& mk,
+                             const CUtensorMap& mv, const CUtensorMap& mo, const CUtensorMap& mg,
+                             PairParams prm, int nbh, int nchunks, int pool_ctas, cudaStream_t stream,
+                             bool* too_large) {
+    *too_large = false;
+    long ring_max = (long)(kPoolScratchBytes / ((size_t)nbh * TASK_BYTES));
+    if (ring_max < kPoolRing) ring_max = kPoolRing;
+    if (const char* r = getenv("GDN_TEST_POOL_RING")) {   // tuning hook: another ring depth (>= 4)
+        const int v = atoi(r);
+        if (v >= 4) ring_max = v;
     }
-    CUtensorMap mq, mk, mv, mo, mg;
-    if (!make_map(&mq, p.q, p.H, p.T, p.B) || !make_map(&mk, p.k, p.H, p.T, p.B) ||
-        !make_map(&mv, p.v, p.H, p.T, p.B) || !make_out_map(&mo, p.out, p.H, p.T, p.B))
-        return cudaErrorInvalidValue;
-    if (CHANNEL) {
-        if (!make_g_map(&mg, p.g, p.H, p.T, p.B)) return cudaErrorInvalidValue;
-    } else {
-        mg = mq;                                   // not read with a scalar gate
-    }
-    PairParams prm{p.g, p.beta, p.state_in, p.state_out, static_cast<float*>(p.out), p.T, p.H, p.B,
-                   nullptr, nullptr, nullptr, 0, kWaitBudgetNs, -1};
-    // Test hooks of the pool form's flag wait (failure detection): a task
-    // whose record is never published, and a short budget for the chains'
-    // flag waits.  Unset in normal use.
-    if (const char* w = getenv("GDN_TEST_WITHHOLD_TASK")) prm.withheld_task = atoll(w);
-    if (const char* b = getenv("GDN_TEST_FLAG_BUDGET_NS")) {
-        const long long ns = atoll(b);
-        if (ns > 0) prm.flag_budget_ns = (unsigned long long)ns;
-    }
-    const int nbh = p.B * p.H;
-    const int nchunks = (p.T + C - 1) / C;
-    if (pool_ctas <= nbh || nchunks == 0) {
-        chunk_pair_kernel<CHANNEL><<<2 * nbh, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mg, prm);
-        return cudaGetLastError();
-    }
-    // Pool form: per (batch, head) a ring of kPoolRing task records, its
-    // flags and its consumed counter, from the stream-ordered workspace
-    // (flags and counters first, 1 KB aligned, cleared on the stream before
-    // the launch).  The scratch is kPoolRing * 99,072 + 4 * (kPoolRing + 1)
-    // bytes per (batch, head), whatever T.
-    const int ring = nchunks < kPoolRing ? nchunks : kPoolRing;
+    const int ring = nchunks < ring_max ? nchunks : (int)ring_max;
     const size_t nslots = (size_t)nbh * ring;
     const size_t counter_words = nslots + (size_t)nbh;
     const size_t flag_bytes = (counter_words * sizeof(unsigned int) + 1023) / 1024 * 1024;
@@ -1453,18 +1676,89 @@ cudaError_t launch_pair(const Problem& p, cudaStream_t stream, int pool_ctas) {
         attr[0].val.cooperative = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, chunk_pool_kernel<CHANNEL>, mq, mk, mv, mo, mg, prm);
-        if (e == cudaErrorCooperativeLaunchTooLarge) {   // fewer SMs free: a cluster per pair
-            (void)cudaGetLastError();
-            prm.slots = nullptr;
-            prm.flags = nullptr;
-            prm.consumed = nullptr;
-            chunk_pair_kernel<CHANNEL><<<2 * nbh, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mg, prm);
-            e = cudaGetLastError();
+        e = cudaLaunchKernelEx(&cfg, kernel, mq, mk, mv, mo, mg, prm);
+        if (e == cudaErrorCooperativeLaunchTooLarge) {
+            if (cudaPeekAtLastError() == cudaErrorCooperativeLaunchTooLarge) (void)cudaGetLastError();
+            *too_large = true;
+            e = cudaSuccess;
         }
     }
     const cudaError_t ef = cudaFreeAsync(ws, stream);
     return e != cudaSuccess ? e : ef;
+}
+
+// Failure-detection test hooks of the pool form's flag wait: a task whose
+// record is never published, and a short budget for the chains' flag waits.
+// Unset in normal use.
+void apply_test_hooks(PairParams& prm) {
+    if (const char* w = getenv("GDN_TEST_WITHHOLD_TASK")) prm.withheld_task = atoll(w);
+    if (const char* b = getenv("GDN_TEST_FLAG_BUDGET_NS")) {
+        const long long ns = atoll(b);
+        if (ns > 0) prm.flag_budget_ns = (unsigned long long)ns;
+    }
+}
+
+template <bool CHANNEL>
+cudaError_t launch_pair(const Problem& p, cudaStream_t stream, int pool_ctas) {
+    {
+        cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(chunk_pair_kernel<CHANNEL>), SMEM_BYTES);
+        if (e == cudaSuccess)
+            e = set_smem_limit(reinterpret_cast<const void*>(chunk_pool_kernel<CHANNEL>), SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+    }
+    CUtensorMap mq, mk, mv, mo, mg;
+    if (!make_map(&mq, p.q, p.H, p.T, p.B) || !make_map(&mk, p.k, p.H, p.T, p.B) ||
+        !make_map(&mv, p.v, p.H, p.T, p.B) || !make_out_map(&mo, p.out, p.H, p.T, p.B))
+        return cudaErrorInvalidValue;
+    if (CHANNEL) {
+        if (!make_g_map(&mg, p.g, p.H, p.T, p.B)) return cudaErrorInvalidValue;
+    } else {
+        mg = mq;                                   // not read with a scalar gate
+    }
+    PairParams prm{p.g, p.beta, p.state_in, p.state_out, static_cast<float*>(p.out), p.T, p.H, p.B,
+                   nullptr, nullptr, nullptr, 0, kWaitBudgetNs, -1};
+    apply_test_hooks(prm);
+    const int nbh = p.B * p.H;
+    const int nchunks = (p.T + C - 1) / C;
+    bool too_large = pool_ctas <= nbh || nchunks == 0;
+    if (!too_large) {
+        cudaError_t e = launch_pool_ring(chunk_pool_kernel<CHANNEL>, mq, mk, mv, mo, mg, prm, nbh, nchunks,
+                                         pool_ctas, stream, &too_large);
+        if (e != cudaSuccess || !too_large) return e;
+    }
+    // The cluster form: a cluster of two CTAs per pair (fewer SMs free, or
+    // the cluster form asked for).
+    chunk_pair_kernel<CHANNEL><<<2 * nbh, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mg, prm);
+    return cudaGetLastError();
+}
+
+template <bool CHANNEL>
+cudaError_t launch_pool_pro(const ProPrefill& a, cudaStream_t stream, bool* too_large) {
+    const PrologueArgs& r = a.pro;
+    cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(chunk_pool_prologue_kernel<CHANNEL>), SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    CUtensorMap mq, mk, mv, mo, mg;
+    if (!make_map(&mq, r.q_raw, r.H, r.T, r.B) || !make_map(&mk, r.k_raw, r.H, r.T, r.B) ||
+        !make_map(&mv, r.v_raw, r.H, r.T, r.B) || !make_out_map(&mo, a.out, r.H, r.T, r.B))
+        return cudaErrorInvalidValue;
+    if (CHANNEL) {
+        if (!make_g_map(&mg, r.g_raw, r.H, r.T, r.B)) return cudaErrorInvalidValue;
+    } else {
+        mg = mq;
+    }
+    PairParams prm{r.g_raw, r.beta_raw, a.state_in, a.state_out, a.out, r.T, r.H, r.B,
+                   nullptr, nullptr, nullptr, 0, kWaitBudgetNs, -1};
+    apply_test_hooks(prm);
+    prm.conv_w = r.conv_w;
+    prm.conv_ring = r.ring;
+    prm.pos0 = r.pos0;
+    prm.q_raw = r.q_raw;
+    prm.k_raw = r.k_raw;
+    prm.v_raw = r.v_raw;
+    prm.silu = r.silu;
+    const int nbh = r.B * r.H;
+    return launch_pool_ring(chunk_pool_prologue_kernel<CHANNEL>, mq, mk, mv, mo, mg, prm, nbh,
+                            (r.T + C - 1) / C, sm_count(), stream, too_large);
 }
 
 }  // namespace
@@ -1472,6 +1766,18 @@ cudaError_t launch_pair(const Problem& p, cudaStream_t stream, int pool_ctas) {
 cudaError_t launch_chunk_pair_sm100(const Problem& p, cudaStream_t stream, int pool_ctas) {
     if (p.io_f32 || !p.out_f32 || p.dk != D || p.dv != D) return cudaErrorNotSupported;
     return p.per_channel ? launch_pair<true>(p, stream, pool_ctas) : launch_pair<false>(p, stream, pool_ctas);
+}
+
+cudaError_t launch_chunk_pool_prologue(const ProPrefill& a, cudaStream_t stream) {
+    const PrologueArgs& r = a.pro;
+    if (r.dk != D || r.dv != D || r.T < 1 || 2 * r.B * r.H > sm_count()) return cudaErrorNotSupported;
+    bool too_large = false;
+    cudaError_t e = r.per_channel ? launch_pool_pro<true>(a, stream, &too_large)
+                                  : launch_pool_pro<false>(a, stream, &too_large);
+    if (e != cudaSuccess) return e;
+    if (too_large) return cudaErrorNotSupported;   // fewer SMs free: the caller runs the two passes
+    if (r.ring) e = launch_prologue_ring(r, stream);   // after the kernel that read it
+    return e;
 }
 
 cudaError_t read_and_clear_pair_status(unsigned int* status) {

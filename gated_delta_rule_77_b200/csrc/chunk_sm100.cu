@@ -87,7 +87,7 @@ constexpr uint32_t R_IN = 0;                 // 32 KB
 constexpr uint32_t OFF_TH = R_IN;            //   8 KB T' hi [64 r][64 m]
 constexpr uint32_t OFF_TL = R_IN + 8192;     //   8 KB T' lo
 constexpr uint32_t OFF_Y = R_IN + 16384;     //   10 KB solve scratch 2 x [32][40] fp32
-constexpr uint32_t OFF_WT = R_IN + 16384;    //   16 KB W^T fp16 [128 i][64 r] (after solve)
+// (R_IN + 26 KB .. 32 KB unused)
 constexpr uint32_t R_V = 32768;              // 16 KB raw V [half][64][128 B]
 constexpr uint32_t R_S = 49152;              // 32 KB S fp16 [j half][128 i][64 j]
 constexpr uint32_t R_X = 81920;              // 112 KB, two uses per chunk:
@@ -98,9 +98,11 @@ constexpr uint32_t OFF_CBH = R_X + 65536;    //   24 KB [half][96][128 B]: rows 
 constexpr uint32_t OFF_CBL = R_X + 90112;    //   24 KB   rows 32-95 K*exp(G_47 - G); one N = 96 B
 constexpr uint32_t CB_HALF = 96 * 128;
 //  (b) after X: derived tiles, P, solve input, U
-constexpr uint32_t OFF_KE = R_X;             //   16 KB K*E bf16  [half][64 r][128 B]
+constexpr uint32_t OFF_KE = R_X;             //   16 KB K*E fp16  [half][64 r][128 B]
+constexpr uint32_t OFF_ZH = R_X;              //   after Y: Z^T = V^T - Y^T bf16 hi [128 j][64 r]
 constexpr uint32_t OFF_OST = R_X;            //   at the chunk's end: 32 KB O fp32 [64 t][128 j] (TMA store)
 constexpr uint32_t OFF_QE = R_X + 16384;     //   16 KB Q*E fp16
+constexpr uint32_t OFF_ZL = R_X + 16384;      //   after Y and the first O products: Z^T lo
 constexpr uint32_t OFF_KDH = R_X + 32768;    //   16 KB K*D bf16 hi
 constexpr uint32_t OFF_KDL = R_X + 49152;    //   16 KB K*D bf16 lo
 constexpr uint32_t OFF_PH = R_X + 65536;     //   8 KB P hi [64 r][64 m]
@@ -131,7 +133,7 @@ constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 
 // ---- TMEM columns (512 allocated) -------------------------------------------
 constexpr uint32_t TM_X = 0;      // X: 128 rows (A rows 0-63, P rows 64-127), N <= 96
-constexpr uint32_t TM_WT = 128;   // W^T: 128 x 64
+constexpr uint32_t TM_YT = 128;   // Y^T = S^T (K*E)^T: 128 x 64
 constexpr uint32_t TM_UT = 192;   // U^T: 128 x 64
 constexpr uint32_t TM_OT = 256;   // O^T: 128 x 64
 constexpr uint32_t TM_SN = 384;   // SN:  128 x 128
@@ -173,9 +175,10 @@ struct Params {
     // tokens it runs (g <= 0 and 0 <= b (K K^T)_rr <= 2, from the diagonal of
     // the product it forms anyway) and, before stopping, beta and g of the
     // tokens it would skip; it never stops once a token is outside.  It then
-    // records how many chunks it ran and writes M = 0 and w only for those
-    // chunks; the correction reads the count.  With decaying gates M falls
-    // below the threshold within a chunk or two.
+    // records how many chunks it ran (negated when it stopped early and
+    // dropped M) and writes M = 0 and w only for those chunks; the correction
+    // reads the count, and the combine skips a dropped M.  With decaying
+    // gates M falls below the threshold within a chunk or two.
     int* trans_len = nullptr;
 };
 
@@ -574,14 +577,37 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     kd[e] = mul2(k2, D2);
                 }
                 const uint32_t o64 = ckh * 8192 + swz(r, ckc);
-                store_bf16x8(smem + OFF_KE + o64, ke);
+                store_f16x8(smem + OFF_KE + o64, ke);
                 store_f16x8(smem + OFF_QE + o64, qe);
                 store_split2(smem + OFF_KDH + o64, smem + OFF_KDL + o64, kd);
             }
         }
-        if (!CHANNEL) {
-            mma_sync();
-            if (__syncthreads_or(!ok)) break;
+        fence_async_smem();                  // K*E, Q*E -> the products below
+        if (!CHANNEL) mma_sync();            // X
+        if (__syncthreads_or(!ok)) break;
+        // Y^T = S^T (K*E)^T and O^T = S^T (Q*E)^T: the state-dependent
+        // products that need only this chunk's derived tiles, issued now, so
+        // that they run during the A/P epilogue.  The corrected values follow
+        // as U = T' (V - (K*E) S) = T' Z (W S = T' (K*E) S), one product after
+        // the solve instead of W^T and U~^T, then U^T -= S^T W^T.
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id_y = idesc_f16(128, 64, true, false);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t a = sdesc_sw128(sbase + R_S + ks * 2048, 16384, 1024);
+                const uint64_t bk = sdesc_sw128(sbase + OFF_KE + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+                mma_bf16(tmem + TM_YT, a, bk, id_y, ks > 0);
+            }
+            if (want_o) {
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint64_t a = sdesc_sw128(sbase + R_S + ks * 2048, 16384, 1024);
+                    const uint64_t bq = sdesc_sw128(sbase + OFF_QE + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+                    mma_bf16(tmem + TM_OT, a, bq, id_y, ks > 0);
+                }
+            }
+            mma_commit(bar_mma);
         }
         // P (rows 64-127, warps of lane quadrants 2 and 3) only where outputs
         // are formed.
@@ -654,6 +680,34 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         // Decay of the state over the whole chunk, per key row (own row).
         const float e_last = __expf(CHANNEL ? sLast[srow] : sGam[C - 1]);
+
+        // Z^T = V^T - Y^T -> bf16 hi + lo [128 j][64 r] over the consumed K*E
+        // and Q*E tiles (thread: value column j = srow, 32 tokens).
+        mma_sync();                          // Y (and the first O products)
+        {
+            float z[32];
+            tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + TM_YT + half * 32, z);
+            tmem_wait_ld();
+            if (!transition) {               // transition CTAs have V = 0
+                const uint8_t* vcol = smem + R_V + (srow >> 6) * 8192 + ((srow & 7) << 1);
+                const uint32_t vchunk = (srow & 63) >> 3;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int r = half * 32 + i;
+                    const float vr = __bfloat162float(
+                        *reinterpret_cast<const __nv_bfloat16*>(vcol + swz(r, vchunk)));
+                    z[i] = vr - z[i];
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) z[i] = -z[i];
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                store_split(smem + OFF_ZH + swz(srow, half * 4 + c), smem + OFF_ZL + swz(srow, half * 4 + c),
+                            &z[8 * c]);
+        }
+        fence_async_smem();
         tc_fence_before();
         __syncthreads();
 
@@ -674,66 +728,29 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             store_split(smem + OFF_TH + swz(r, c), smem + OFF_TL + swz(r, c), tv);
         }
         fence_async_smem();
-        __syncthreads();
-
-        // ---------------------------------------------------- W^T and T'V ------
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id = idesc_bf16(128, 64, true, false);
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const uint32_t tb = part ? OFF_TL : OFF_TH;
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t bt = sdesc_sw128(sbase + tb + ks * 32, 16, 1024);
-                    const uint32_t acc = (part | ks) != 0;
-                    mma_bf16(tmem + TM_WT, sdesc_sw128(sbase + OFF_KE + ks * 2048, 8192, 1024), bt, id, acc);
-                    if (!transition)
-                        mma_bf16(tmem + TM_UT, sdesc_sw128(sbase + R_V + ks * 2048, 8192, 1024), bt, id, acc);
-                }
-            }
-            mma_commit(bar_mma);
-        }
-        mma_sync();
-        if (__syncthreads_or(!ok)) break;
-
-        // W^T -> fp16, MN-major B operand [128 i][64 r].  Thread: row i, 32 r.
-        {
-            float w[32];
-            tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + TM_WT + half * 32, w);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 4; ++c) store_f16x8(smem + OFF_WT + swz(srow, half * 4 + c), &w[8 * c]);
-        }
-        fence_async_smem();
         tc_fence_before();
         __syncthreads();
 
-        // ------------------------------- U^T -= S^T W^T ; O^T = S^T (QE)^T ------
+        // ---------------------------------------------------- U^T = Z^T T'^T ---
+        // bf16 hi + lo on both sides, three products per k-step.
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t id_u = idesc_f16(128, 64, true, true, true);
-            const uint32_t id_o = idesc_f16(128, 64, true, false);
+            const uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t a = sdesc_sw128(sbase + R_S + ks * 2048, 16384, 1024);
-                // Transition CTAs have V = 0: U = -W S starts the accumulator.
-                mma_bf16(tmem + TM_UT, a, sdesc_sw128(sbase + OFF_WT + ks * 2048, 8192, 1024), id_u,
-                         transition ? (ks > 0) : 1);
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t zh = sdesc_sw128(sbase + OFF_ZH + ks * 32, 16, 1024);
+                const uint64_t zl = sdesc_sw128(sbase + OFF_ZL + ks * 32, 16, 1024);
+                const uint64_t th = sdesc_sw128(sbase + OFF_TH + ks * 32, 16, 1024);
+                const uint64_t tl = sdesc_sw128(sbase + OFF_TL + ks * 32, 16, 1024);
+                mma_bf16(tmem + TM_UT, zh, th, id, ks > 0);
+                mma_bf16(tmem + TM_UT, zh, tl, id, 1);
+                mma_bf16(tmem + TM_UT, zl, th, id, 1);
             }
             mma_commit(bar_mma);
-            if (want_o) {
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint64_t a = sdesc_sw128(sbase + R_S + ks * 2048, 16384, 1024);
-                    const uint64_t bq = sdesc_sw128(sbase + OFF_QE + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
-                    mma_bf16(tmem + TM_OT, a, bq, id_o, ks > 0);
-                }
-            }
         }
         mma_sync();
         if (__syncthreads_or(!ok)) break;
-        // Raw K, Q, V, T' and W^T are no longer read: prefetch the next chunk.
+        // Raw K, Q, V, T' and Z are no longer read: prefetch the next chunk.
         if (tid == 0 && ci + 1 < nchunks) {
             issue_loads(ci + 1);
             ++tma_issued;
@@ -867,7 +884,8 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (tid == 0) bulk_wait_all();     // output stores complete before exit
     if (tid == 0 && stopped && tma_issued > tma_waited + 1)   // the next chunk's loads
         mbar_wait(bar_tma, (tma_waited + 1) & 1, &g_status_word);
-    if (tid == 0 && may_stop && ok) p.trans_len[((long)b * p.nseg + seg) * H + h] = chunks_run;
+    if (tid == 0 && may_stop && ok)   // negative: stopped early, M dropped
+        p.trans_len[((long)b * p.nseg + seg) * H + h] = stopped ? -chunks_run : chunks_run;
 
     if (!ok && tid == 0) {
         // Abandoned: drain what this CTA still has in flight (bounded) before
@@ -969,7 +987,7 @@ bool make_map(CUtensorMap* map, const void* base, int H, int T, int B) {
 constexpr int CB_COLS = 32;
 __global__ void __launch_bounds__(256)
 combine_segments_kernel(float* seg_states, const float* trans, const float* state_in,
-                        float* state_out, int H, int nseg, int seg0_true)
+                        float* state_out, int H, int nseg, int seg0_true, const int* trans_len)
 {
     __shared__ __align__(16) float sS[D][CB_COLS];     // current state slice
     const int nslice = D / CB_COLS;
@@ -995,8 +1013,12 @@ combine_segments_kernel(float* seg_states, const float* trans, const float* stat
             acc[4 * q] = v.x; acc[4 * q + 1] = v.y; acc[4 * q + 2] = v.z; acc[4 * q + 3] = v.w;
         }
         const float4* mrow = reinterpret_cast<const float4*>(trans + base + (long)i * D);
+        // No product where M is zero: segment 0 run from the true start, or a
+        // transition that ended early (negative count, see Params::trans_len).
+        const bool no_m = (sg == 0 && seg0_true) ||
+                          (trans_len && sg >= 1 && trans_len[((long)b * nseg + sg) * H + h] < 0);
 #pragma unroll 4
-        for (int k4 = 0; k4 < ((sg == 0 && seg0_true) ? 0 : D / 4); ++k4) {
+        for (int k4 = 0; k4 < (no_m ? 0 : D / 4); ++k4) {
             const float4 m = mrow[k4];
             const float mk[4] = {m.x, m.y, m.z, m.w};
 #pragma unroll
@@ -1057,7 +1079,7 @@ segment_correction_kernel(const float* __restrict__ seg_states, const __half* __
     // Tokens past the chunks the segment's transition ran have w = 0 (it
     // stopped once M had decayed below fp32 resolution): nothing to add.
     const int t_end = min(min(T, t_begin + seg_len),
-                          trans_len ? t_begin + trans_len[((long)b * nseg + seg) * H + h] * C : T);
+                          trans_len ? t_begin + abs(trans_len[((long)b * nseg + seg) * H + h]) * C : T);
     const int tile0 = blockIdx.x * CORR_TILES;
     if (t_begin + tile0 * C >= t_end) return;
     // Tile i's w into stage i & 1 (one commit group; rows past the segment zero).
@@ -1206,7 +1228,7 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
     e = cudaGetLastError();
     if (e == cudaSuccess) {
         combine_segments_kernel<<<p.B * p.H * (D / CB_COLS), 256, 0, stream>>>(
-            seg_states, trans, p.state_in, p.state_out, p.H, nseg, 1);
+            seg_states, trans, p.state_in, p.state_out, p.H, nseg, 1, CHANNEL ? nullptr : trans_len);
         e = cudaGetLastError();
     }
     if (e == cudaSuccess) {
@@ -1285,7 +1307,7 @@ cudaError_t launch_noalloc(const Problem& p, cudaStream_t stream, bool* over_lim
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     combine_segments_kernel<<<p.B * p.H * (D / CB_COLS), 256, 0, stream>>>(
-        seg_states, trans, p.state_in, p.state_out, p.H, nseg, 0);
+        seg_states, trans, p.state_in, p.state_out, p.H, nseg, 0, nullptr);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     Params p2{p.g, p.beta, seg_states, nullptr, nullptr, out, p.T, p.H, p.B, nseg, seg_len, nseg, 1};

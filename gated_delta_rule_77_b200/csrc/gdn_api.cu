@@ -188,6 +188,76 @@ int gdn_recurrent_step_prologue(const void* q_raw, const void* k_raw, const void
     return e == cudaErrorNotSupported ? GDN_ERR_UNSUPPORTED : to_status(e);
 }
 
+int gdn_chunk_fwd_prologue(const void* q_raw, const void* k_raw, const void* v_raw,
+                           const float* g_raw, const float* beta_raw, const float* conv_w, float* ring,
+                           const int* pos0, const float* state_in, void* out, float* state_out, int B,
+                           int T, int H, int dk, int dv, int gate_mode, int activation,
+                           int fused, gdn_stream_t stream_)
+{
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (fused != 0 && fused != 1) return GDN_ERR_INVALID_ARG;
+    const size_t tok = (size_t)(B > 0 ? B : 0) * (size_t)(T > 0 ? T : 0) * (size_t)(H > 0 ? H : 0);
+    const size_t st = (size_t)(B > 0 ? B : 0) * (size_t)(H > 0 ? H : 0) * (size_t)(dk > 0 ? dk : 0) *
+                      (size_t)(dv > 0 ? dv : 0) * 4;
+    // state_out may coincide with state_in exactly (checked below); out and
+    // state_out are outputs that may overlap no input (the ring included).
+    const void* outs[] = {out, state_out};
+    const size_t bytes[] = {tok * (size_t)(dv > 0 ? dv : 0) * 4, state_out ? st : 0};
+    int rc = validate_prologue(q_raw, k_raw, v_raw, g_raw, beta_raw, conv_w, ring, pos0, B, T, H, dk,
+                               dv, gate_mode, activation, outs, bytes, 2);
+    if (rc != GDN_OK) return rc;
+    if (state_in) {
+        if (!aligned16(state_in)) return GDN_ERR_MISALIGNED;
+        const Range rsi = range_of(state_in, st);
+        if (overlaps(rsi, range_of(out, bytes[0]))) return GDN_ERR_INVALID_ARG;
+        if (state_out && state_out != state_in && overlaps(rsi, range_of(state_out, st)))
+            return GDN_ERR_INVALID_ARG;
+        if (ring && overlaps(rsi, range_of(ring, (size_t)B * H * 4 * (2 * (size_t)dk + dv) * 4)))
+            return GDN_ERR_INVALID_ARG;
+    }
+    if (T > (1 << 30)) return GDN_ERR_UNSUPPORTED;
+    if (T == 0) {
+        if (!state_out || state_in == state_out) return GDN_OK;
+        cudaError_t e = state_in
+            ? cudaMemcpyAsync(state_out, state_in, st, cudaMemcpyDeviceToDevice, stream)
+            : cudaMemsetAsync(state_out, 0, st, stream);
+        return to_status(e);
+    }
+    const bool ch = gate_mode == GDN_GATE_CHANNEL;
+    gdn::PrologueArgs pa{static_cast<const __nv_bfloat16*>(q_raw), static_cast<const __nv_bfloat16*>(k_raw),
+                         static_cast<const __nv_bfloat16*>(v_raw), g_raw, beta_raw, conv_w, ring, pos0,
+                         activation == GDN_ACT_SILU, nullptr, nullptr, nullptr, nullptr, nullptr, B, T, H,
+                         dk, dv, ch};
+    cudaError_t e = cudaErrorNotSupported;
+    if (fused) {
+        gdn::ProPrefill fp{pa, state_in, state_out, static_cast<float*>(out)};
+        e = gdn::launch_chunk_pool_prologue(fp, stream);
+        if (e != cudaErrorNotSupported) return to_status(e);
+    }
+    // Route 0, or a shape that is not the fused kernel's (or too few free
+    // SMs): the prologue pass into stream-ordered scratch, then the prefill.
+    const size_t qk = tok * dk * 2, vb = tok * dv * 2, gb = tok * (ch ? (size_t)dk : 1) * 4, bb = tok * 4;
+    auto up16 = [](size_t n) { return (n + 255) / 256 * 256; };
+    uint8_t* ws = nullptr;
+    e = gdn::workspace_alloc(reinterpret_cast<void**>(&ws), 2 * up16(qk) + up16(vb) + up16(gb) + up16(bb),
+                             stream);
+    if (e != cudaSuccess) return to_status(e);
+    pa.q = reinterpret_cast<__nv_bfloat16*>(ws);
+    pa.k = reinterpret_cast<__nv_bfloat16*>(ws + up16(qk));
+    pa.v = reinterpret_cast<__nv_bfloat16*>(ws + 2 * up16(qk));
+    pa.g = reinterpret_cast<float*>(ws + 2 * up16(qk) + up16(vb));
+    pa.beta = reinterpret_cast<float*>(ws + 2 * up16(qk) + up16(vb) + up16(gb));
+    e = gdn::launch_prologue(pa, stream);
+    if (e == cudaSuccess) {
+        gdn::Problem p{pa.q, pa.k, pa.v, pa.g, pa.beta, state_in, state_out, out, B, T, H, dk, dv, ch,
+                       false, true, 0};
+        e = gdn::launch_chunk_sm100(p, stream);
+        if (e == cudaErrorNotSupported) e = gdn::launch_recurrent(p, stream);
+    }
+    const cudaError_t ef = cudaFreeAsync(ws, stream);
+    return to_status(e != cudaSuccess ? e : ef);
+}
+
 static int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g,
                           const float* beta, const float* state_in, void* out, float* state_out,
                           int B, int T, int H, int dk, int dv, int gate_mode, int io_dtype,

@@ -116,6 +116,22 @@ struct PrologueArgs {
 };
 cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream);
 
+// The ring update of a prologue pass alone (slot (pos0 + t) mod 4 takes the
+// raw input of token t for the last min(T, 4) tokens).
+cudaError_t launch_prologue_ring(const PrologueArgs& a, cudaStream_t stream);
+
+// The prefill with the prologue applied while loading the raw projections
+// (pool form, dk = dv = 128, 2 * B * H <= #SMs), then the ring update.
+// cudaErrorNotSupported when that form does not apply (nothing launched but,
+// possibly, a memset of scratch); the caller then runs the two passes.
+struct ProPrefill {
+    PrologueArgs pro;          // raw inputs, taps, ring, pos0, activation (q..beta unused)
+    const float* state_in;     // [B, H, dk, dv] or null
+    float* state_out;          // [B, H, dk, dv] or null
+    float* out;                // [B, T, H, dv] fp32
+};
+cudaError_t launch_chunk_pool_prologue(const ProPrefill& a, cudaStream_t stream);
+
 struct StepPrologueArgs {
     const __nv_bfloat16* q_raw;
     const __nv_bfloat16* k_raw;

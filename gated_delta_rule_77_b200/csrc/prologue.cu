@@ -23,78 +23,14 @@
 
 #include "chunk_common.cuh"
 #include "gdn_internal.cuh"
+#include "prologue_math.cuh"
 
 namespace gdn {
 namespace {
 
 constexpr int TT = 16;   // tokens per CTA of the prefill prologue (a multiple of 8)
 
-__device__ __forceinline__ float ex2_fast(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-constexpr float kLog2eP = 1.4426950408889634f;
-
-// SiLU y / (1 + e^-y) with the hardware 2^x and a fast divide (relative
-// error a few 1e-7, far below the bf16 rounding of the results).  The limits
-// hold: e^-y overflows to inf for y < -88 (result -0), underflows to 0 for
-// large y (result y).
-__device__ __forceinline__ float act_fn(float y, bool silu) {
-    return silu ? __fdividef(y, 1.f + ex2_fast(-y * kLog2eP)) : y;
-}
-__device__ __forceinline__ float sigmoid_fn(float x) { return 1.f / (1.f + expf(-x)); }
-
-// log(1 + u) for u in [0, 1] from log(1 + u) = 2 atanh(s), s = u / (2 + u)
-// in [0, 1/3], and the odd series atanh(s) = s + s^3/3 + s^5/5 + ...; eight
-// terms leave a remainder below (1/3)^16 / 17 < 1.5e-9 of the sum.  Relative
-// accuracy holds down to the smallest u (s ~ u/2), where log1p matters for
-// a gate near 0.
-__device__ __forceinline__ float log1p_unit(float u) {
-    const float s = __fdividef(u, 2.f + u);
-    const float z = s * s;
-    float t = 1.f / 15.f;
-    t = fmaf(t, z, 1.f / 13.f);
-    t = fmaf(t, z, 1.f / 11.f);
-    t = fmaf(t, z, 1.f / 9.f);
-    t = fmaf(t, z, 1.f / 7.f);
-    t = fmaf(t, z, 1.f / 5.f);
-    t = fmaf(t, z, 1.f / 3.f);
-    t = fmaf(t, z, 1.f);
-    return 2.f * s * t;
-}
-
-// g = -min(softplus(x), 5) with softplus(x) = max(x, 0) + log1p(e^-|x|).
-__device__ __forceinline__ float gate_fn(float x) {
-    const float sp = fmaxf(x, 0.f) + log1p_unit(ex2_fast(-fabsf(x) * kLog2eP));
-    return -fminf(sp, 5.f);
-}
-
-// The same two at a time, with paired fp32 (f32x2) arithmetic.
-using chunk::add2;
-using chunk::fma2;
-using chunk::mul2;
-__device__ __forceinline__ float2 gate_fn2(float2 x) {
-    const float2 u = make_float2(ex2_fast(-fabsf(x.x) * kLog2eP), ex2_fast(-fabsf(x.y) * kLog2eP));
-    const float2 s2 = make_float2(__fdividef(u.x, 2.f + u.x), __fdividef(u.y, 2.f + u.y));
-    const float2 z = mul2(s2, s2);
-    float2 t = make_float2(1.f / 15.f, 1.f / 15.f);
-    t = fma2(t, z, make_float2(1.f / 13.f, 1.f / 13.f));
-    t = fma2(t, z, make_float2(1.f / 11.f, 1.f / 11.f));
-    t = fma2(t, z, make_float2(1.f / 9.f, 1.f / 9.f));
-    t = fma2(t, z, make_float2(1.f / 7.f, 1.f / 7.f));
-    t = fma2(t, z, make_float2(1.f / 5.f, 1.f / 5.f));
-    t = fma2(t, z, make_float2(1.f / 3.f, 1.f / 3.f));
-    t = fma2(t, z, make_float2(1.f, 1.f));
-    const float2 l = mul2(mul2(s2, make_float2(2.f, 2.f)), t);
-    return make_float2(-fminf(fmaxf(x.x, 0.f) + l.x, 5.f), -fminf(fmaxf(x.y, 0.f) + l.y, 5.f));
-}
-__device__ __forceinline__ float2 act_fn2(float2 y, bool silu) {
-    if (!silu) return y;
-    const float2 m = mul2(y, make_float2(-kLog2eP, -kLog2eP));
-    const float2 d = add2(make_float2(ex2_fast(m.x), ex2_fast(m.y)), make_float2(1.f, 1.f));
-    return mul2(y, make_float2(__fdividef(1.f, d.x), __fdividef(1.f, d.y)));
-}
+using namespace prologue_math;
 
 // Channels c of q | k | v for token t of row b, head h (bf16 inputs).
 __device__ __forceinline__ float2 raw_pair(const __nv_bfloat16* q, const __nv_bfloat16* k,
@@ -267,19 +203,8 @@ prologue_kernel(const __nv_bfloat16* __restrict__ q_raw, const __nv_bfloat16* __
         float v[TT];
 #pragma unroll
         for (int i = 0; i < TT; ++i) v[i] = fmaf(y[i].x, y[i].x, y[i].y * y[i].y);
-#pragma unroll
-        for (int half = 8, bit = 16; half >= 1; half >>= 1, bit >>= 1) {
-            const bool up = (lane & bit) != 0;
-#pragma unroll
-            for (int i = 0; i < half; ++i) {
-                const float send = up ? v[i] : v[i + half];
-                const float keep = up ? v[i + half] : v[i];
-                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
-            }
-        }
-        v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
-        const int tok = 8 * ((lane >> 4) & 1) + 4 * ((lane >> 3) & 1) + 2 * ((lane >> 2) & 1) + ((lane >> 1) & 1);
-        if ((lane & 1) == 0) s_ss[tensor][warp % QW][tok] = v[0];
+        butterfly_sums16(v, lane);
+        if ((lane & 1) == 0) s_ss[tensor][warp % QW][butterfly_token(lane)] = v[0];
     }
     __syncthreads();
 
@@ -554,6 +479,16 @@ cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream) {
     if (a.dk == 64 && a.dv == 128) return launch_prologue_t<64, 128>(a, stream);
     if (a.dk == 64 && a.dv == 64) return launch_prologue_t<64, 64>(a, stream);
     return cudaErrorNotSupported;
+}
+
+cudaError_t launch_prologue_ring(const PrologueArgs& a, cudaStream_t stream) {
+    if (a.ring == nullptr || a.T < 1) return cudaSuccess;
+    if (a.dk == 128 && a.dv == 128)
+        prologue_ring_kernel<128, 128><<<a.B * a.H, 128, 0, stream>>>(a.q_raw, a.k_raw, a.v_raw, a.ring,
+                                                                      a.pos0, a.T, a.H);
+    else
+        return cudaErrorNotSupported;
+    return cudaGetLastError();
 }
 
 cudaError_t launch_step_prologue(const StepPrologueArgs& a, cudaStream_t stream) {

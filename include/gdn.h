@@ -101,11 +101,12 @@ enum { GDN_IO_BF16 = 0, GDN_IO_F32 = 1 };
  * Scratch: with dk = dv = 128 and 2 * B * H <= the SM count, each chunk's
  * chunk-local results (T' or T and beta, P and the chain's operand tiles:
  * 99,072 bytes) pass from prep CTAs to the state chains through a ring of
- * at most 8 such records per (batch, head): at most
- * B * H * (8 * 99,072 + 36) bytes (about 0.8 MB per (batch, head), whatever
- * T) of stream-ordered scratch on `stream` from the library's pool, freed on
- * `stream` when the call's kernel completes.  If it cannot be had, the call
- * runs the cluster form of the same kernel, which needs none.
+ * such records per (batch, head): one per chunk while all of them fit in
+ * 256 MiB, else as many as fit (at least 8), whatever T -- at most
+ * max(256 MiB, B * H * 8 * 99,072 bytes) plus 4 bytes per record and per
+ * (batch, head) of stream-ordered scratch on `stream` from the library's
+ * pool, freed on `stream` when the call's kernel completes.  If it cannot be
+ * had, the call runs the cluster form of the same kernel, which needs none.
  * After a call that gdn_check reports as GDN_ERR_TIMEOUT, out and state_out
  * are undefined.
  */
@@ -364,6 +365,40 @@ GDN_API int gdn_recurrent_step_prologue(const void* q_raw, const void* k_raw, co
                                         const float* state_in, float* state_out, void* out,
                                         int B, int H, int dk, int dv, int gate_mode,
                                         int activation, gdn_stream_t stream);
+
+/*
+ * gdn_chunk_fwd_prologue -- the chunkwise prefill of a GDN layer from its raw
+ * projections: the prologue above applied while the prefill loads its
+ * inputs, then the recurrence (Atomic-GDN2 model card, section 2.1), as
+ * gdn_prologue followed by gdn_chunk_fwd on its outputs -- without writing
+ * q, k, v, g and beta to memory and reading them back.
+ *
+ *   q_raw .. pos0, activation   as gdn_prologue (the ring is read for the
+ *                               history of token 0 and then updated)
+ *   state_in   [B, H, dk, dv] fp32, or NULL for a zero initial state
+ *   out        [B, T, H, dv] fp32;  state_out [B, H, dk, dv] fp32 or NULL
+ *              (state_out == state_in allowed; out and state_out overlap no
+ *              input and not the ring)
+ *   fused      0: gdn_prologue into stream-ordered scratch
+ *              (B * T * H * (2 dk + dv) * 2 bytes + the gates), then
+ *              gdn_chunk_fwd.  1: with dk = dv = 128 and 2 * B * H <= the SM
+ *              count, the prologue runs inside the prefill's prep-pool
+ *              kernel: the prep tasks convert each chunk's q, k (with the
+ *              three earlier tokens of the convolution) and the gates, the
+ *              state chains convert v, and only the raw projections are
+ *              read; scratch as gdn_chunk_fwd's.  Other shapes (or too few
+ *              free SMs) take route 0.  Route 0 is the faster one on B200 at
+ *              the GDN-2 layer shape (B 8, T 2048, H 8): the conversion in
+ *              the prep tasks costs more than the memory pass it saves.
+ * Outputs agree with the two-call sequence to the rounding of the sums of
+ * squares; errors and scratch failure as gdn_chunk_fwd.
+ */
+GDN_API int gdn_chunk_fwd_prologue(const void* q_raw, const void* k_raw, const void* v_raw,
+                                   const float* g_raw, const float* beta_raw, const float* conv_w,
+                                   float* ring, const int* pos0, const float* state_in, void* out,
+                                   float* state_out, int B, int T, int H, int dk, int dv,
+                                   int gate_mode, int activation, int fused,
+                                   gdn_stream_t stream);
 
 /*
  * gdn_check -- synchronises `stream`, then reports GDN_ERR_TIMEOUT if any

@@ -263,3 +263,90 @@ def test_fused_decode_full_batch_sampled_rows(gdn, oracle_threads):
     assert oracle.rel_err(got[rows].cpu(), ref_o) <= 1e-3
     assert oracle.rel_err(state[rows].cpu(), ref_s) <= 1e-3
     assert torch.equal(ring[rows].cpu(), torch.from_numpy(rring).float())
+
+
+# ---- the prefill with the prologue applied while loading (gdn_chunk_fwd_prologue) ----
+def _fused(gdn, x, s0=None, activation="silu", use_ring=True, use_pos=True, fused=True):
+    ring = _dev(x["ring"]) if use_ring else None
+    out, s_t = gdn.chunk_fwd_prologue(
+        *(_dev(x[n]) for n in ("q_raw", "k_raw", "v_raw", "g_raw", "beta_raw", "conv_w")),
+        ring, _dev(x["pos0"]) if use_pos else None, _dev(s0), activation=activation, fused=fused)
+    torch.cuda.synchronize()
+    return out, s_t, ring
+
+
+@pytest.mark.parametrize("route", ["fused", "two_passes"])
+@pytest.mark.parametrize("gate", ["channel", "scalar"])
+@pytest.mark.parametrize("T", [1, 2, 63, 64, 200, 515])
+def test_fused_prologue_prefill_matches_oracle(gdn, gate, T, route):
+    """The prologue-plus-prefill call, on either route, against the oracle
+    prologue (q, k, v rounded to bf16) followed by the oracle recurrence, with
+    a history ring, random positions (the first tokens' convolution reads the
+    ring) and S0 != 0; lengths from 1 token to several chunks with a ragged
+    tail."""
+    x = prologue_inputs(2, T, 3, 128, 128, gate=gate, seed=60 + T)
+    s0 = torch.randn(2, 3, 128, 128, generator=torch.Generator().manual_seed(61)) * 0.1
+    out, s_t, ring = _fused(gdn, x, s0, fused=route == "fused")
+    rq, rk, rv, rg, rb, rring = _oracle(x)
+    ref_o, ref_s = oracle.run(_bf16(rq), _bf16(rk), _bf16(rv), rg, rb, s0,
+                              per_channel=gate == "channel")
+    assert oracle.rel_err(out.cpu(), ref_o) <= 2e-2
+    assert _err_vs_max(s_t, ref_s) <= 2e-2
+    assert torch.equal(ring.cpu(), torch.from_numpy(rring).float())
+    assert gdn.check() == gdn.GDN_OK
+
+
+@pytest.mark.parametrize("gate", ["channel", "scalar"])
+def test_fused_prologue_prefill_equals_the_two_passes(gdn, gate):
+    """Fused against gdn_prologue then gdn_chunk_fwd on the same inputs: the
+    same arithmetic except the order of the q/k sums of squares, which can
+    flip the bf16 rounding of a q or k element; the output, a small
+    difference of larger terms, then moves by a few 1e-3 of its rms.  Held to
+    half the prefill tolerance, as the other cross-form checks."""
+    x = prologue_inputs(2, 300, 4, 128, 128, gate=gate, seed=62)
+    s0 = torch.randn(2, 4, 128, 128, generator=torch.Generator().manual_seed(63)) * 0.1
+    out_f, s_f, ring_f = _fused(gdn, x, s0)
+    (q, k, v, g, beta), ring_u = _gpu_prologue(gdn, x)
+    out_u, s_u = gdn.chunk_fwd(q, k, v, g, beta, _dev(s0))
+    torch.cuda.synchronize()
+    assert oracle.rel_err(out_f.cpu(), out_u.cpu().double()) <= 1e-2
+    assert _err_vs_max(s_f, s_u.cpu().double().numpy()) <= 1e-2
+    assert torch.equal(ring_f.cpu(), ring_u.cpu())
+
+
+def test_fused_prologue_without_ring_positions_or_activation(gdn):
+    x = prologue_inputs(1, 150, 2, 128, 128, gate="channel", ring=False, seed=64)
+    out, s_t, _ = _fused(gdn, x, activation="none", use_ring=False, use_pos=False)
+    x0 = dict(x)
+    x0["pos0"] = torch.zeros_like(x["pos0"])
+    rq, rk, rv, rg, rb, _ = _oracle(x0, activation="none")
+    ref_o, ref_s = oracle.run(_bf16(rq), _bf16(rk), _bf16(rv), rg, rb, per_channel=True)
+    assert oracle.rel_err(out.cpu(), ref_o) <= 2e-2
+    assert _err_vs_max(s_t, ref_s) <= 2e-2
+
+
+def test_fused_prologue_other_shapes_take_the_two_passes(gdn):
+    """dk = dv = 64 (not the fused kernel's shape) and a pair count above
+    half the SMs run the prologue pass into scratch, then the prefill."""
+    for B, T, H, d in ((1, 130, 2, 64), (2, 70, 40, 128)):
+        x = prologue_inputs(B, T, H, d, d, gate="scalar", seed=65 + H)
+        out, s_t, ring = _fused(gdn, x)
+        rq, rk, rv, rg, rb, rring = _oracle(x)
+        ref_o, ref_s = oracle.run(_bf16(rq), _bf16(rk), _bf16(rv), rg, rb, per_channel=False)
+        assert oracle.rel_err(out.cpu(), ref_o) <= 2e-2, (B, T, H, d)
+        assert _err_vs_max(s_t, ref_s) <= 2e-2, (B, T, H, d)
+        assert torch.equal(ring.cpu(), torch.from_numpy(rring).float())
+
+
+@pytest.mark.parametrize("route", ["fused", "two_passes"])
+def test_fused_prologue_full_layer_size_sampled_rows(gdn, oracle_threads, route):
+    """The GDN-2 layer shape (B8 H8 T2048 d128, per-channel gate) through the
+    prologue-plus-prefill call; rows 0 and 7 against the oracle."""
+    x = prologue_inputs(8, 2048, 8, 128, 128, gate="channel", seed=2)
+    out, s_t, _ = _fused(gdn, x, fused=route == "fused")
+    rows = [0, 7]
+    rq, rk, rv, rg, rb, _ = _oracle(x, rows=rows)
+    ref_o, ref_s = oracle.run(_bf16(rq), _bf16(rk), _bf16(rv), rg, rb, per_channel=True,
+                              threads=oracle_threads)
+    assert oracle.rel_err(out[rows].cpu(), ref_o) <= 2e-2
+    assert _err_vs_max(s_t[rows], ref_s) <= 2e-2
