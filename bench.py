@@ -143,11 +143,19 @@ def ncu_traffic(key: str):
 
 def chunk_path_kernels(cfg, sms: int = 148) -> list:
     """The kernels one gdn_chunk_fwd call launches for a workload (bf16 I/O,
-    d = 128), following the library's choice of path: the segment-parallel
-    path when B*H*4 <= #SMs and T >= 64 chunks, else the prep pool when
-    2*B*H <= #SMs, else one CTA per (batch, head)."""
+    d = 128), following the library's automatic choice: the segment-parallel
+    path when it picks n > 1 segments (scalar gate: n = #SMs // (B*H) from 32
+    chunks, when n >= 3 or n = 2 with 2*B*H >= 0.85 #SMs; per-channel gate:
+    B*H*4 <= #SMs and 64 chunks, n = (#SMs // (B*H) + 1) // 2 >= 3), else the
+    prep pool when 2*B*H <= #SMs, else one CTA per (batch, head)."""
     bh = cfg.B * cfg.H
-    if bh * 4 <= sms and -(-cfg.T // 64) >= 64:
+    nchunks = -(-cfg.T // 64)
+    if cfg.per_channel:
+        seg = nchunks >= 64 and bh * 4 <= sms and (sms // bh + 1) // 2 >= 3
+    else:
+        n = sms // bh
+        seg = nchunks >= 32 and (n >= 3 or (n == 2 and 2 * bh * 100 >= 85 * sms))
+    if seg:
         return ["chunk_fwd_kernel (zero-start + transition CTAs)", "combine_segments_kernel",
                 "segment_correction_kernel"]
     if 2 * bh <= sms:

@@ -1139,19 +1139,35 @@ segment_correction_kernel(const float* __restrict__ seg_states, const __half* __
 }
 
 // Number of time segments per (batch, head).  Segmenting costs a second
-// chunk recursion per segment (the transition) and a correction, so it pays
-// only when the (batch, head) pairs alone leave most SMs idle.  Automatic
-// choice: one segment per SM (B*H*n <= #SMs) where the transitions are
-// expected to end early (scalar gate, cheap_transitions); otherwise the
-// largest n whose B*H*(2n - 1) CTAs fit in one wave; at least 3 segments.
-int choose_segments(int requested, int BH, int nchunks, bool cheap_transitions) {
+// chunk recursion per segment (the transition), a combine and a correction,
+// so it pays only when the (batch, head) pairs alone leave SMs idle.
+// Automatic choice (requested == 0):
+//  * kScalarRule (transitions expected to end early): one zero-start CTA per
+//    SM, n = #SMs / (B*H), from 32 chunks on, when n >= 3, or n = 2 with at
+//    least 85% of the SMs busy.  Measured on B200 (T 8192, B*H = 48):
+//    n = 3 430 us, the prep pool 556 us, n = 2 (96 SMs busy) 611 us; at
+//    B*H = 64 (T 2048) n = 2 took 190 us against 213 us pooled.
+//  * kChannelRule (transitions run in full): the largest n whose
+//    B*H*(2n - 1) CTAs fit in one wave, from B*H*4 <= #SMs and 64 chunks
+//    on, at least 3.
+//  * kNoAllocRule (the fixed-scratch entry, whose transitions run in full
+//    but whose segments each need only two states): n = #SMs / (B*H) from
+//    B*H*4 <= #SMs and 64 chunks on.
+enum SegmentRule { kScalarRule, kChannelRule, kNoAllocRule };
+int choose_segments(int requested, int BH, int nchunks, SegmentRule rule) {
     if (nchunks <= 1 || requested == 1) return 1;
     int n = requested;
     if (n <= 0) {
         const int sms = sm_count();
-        if (nchunks < 64 || BH * 4 > sms) return 1;
-        n = cheap_transitions ? sms / BH : (sms / BH + 1) / 2;
-        if (n < 3) return 1;
+        if (rule == kScalarRule) {
+            n = sms / BH;
+            if (nchunks < 32 || n < 2) return 1;
+            if (n == 2 && 2 * BH * 100 < 85 * sms) return 1;
+        } else {
+            if (nchunks < 64 || BH * 4 > sms) return 1;
+            n = rule == kNoAllocRule ? sms / BH : (sms / BH + 1) / 2;
+            if (n < 3) return 1;
+        }
     }
     return n < nchunks ? n : nchunks;
 }
@@ -1166,8 +1182,8 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
         return cudaErrorInvalidValue;
     float* out = static_cast<float*>(p.out);
     const int nchunks = (p.T + C - 1) / C;
-    int nseg = choose_segments(p.segments, p.B * p.H, nchunks, !CHANNEL);
-    if (nseg <= 1) {
+    int nseg = choose_segments(p.segments, p.B * p.H, nchunks, CHANNEL ? kChannelRule : kScalarRule);
+    auto unsegmented = [&]() -> cudaError_t {
         // Chunk-local work and the state chain on different SMs when two per
         // (batch, head) fit: by default one prep pool over all SMs; a cluster
         // per pair with GDN_CHUNK_KERNEL=pair, one CTA per pair with =single
@@ -1191,7 +1207,8 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
                    1, nchunks * C, 1, 1};
         chunk_fwd_kernel<CHANNEL><<<p.B * p.H, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, mo, prm);
         return cudaGetLastError();
-    }
+    };
+    if (nseg <= 1) return unsegmented();
     // Segment-parallel path in two chunk passes.  One launch runs segment 0
     // from the true initial state and every other segment from a zero state,
     // writing outputs and end states, and, in a second set of CTAs, the
@@ -1209,6 +1226,12 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
     cudaError_t e = workspace_alloc(reinterpret_cast<void**>(&ws),
                                     2 * slab * sizeof(float) + nlen * sizeof(int) + wlen * sizeof(__half),
                                     stream);
+    if (e == cudaErrorMemoryAllocation && p.segments == 0) {
+        // An automatic choice whose scratch cannot be had (nothing was
+        // launched): the unsegmented path, whose own fallback needs none.
+        if (cudaPeekAtLastError() == cudaErrorMemoryAllocation) (void)cudaGetLastError();
+        return unsegmented();
+    }
     if (e != cudaSuccess) return e;
     float* seg_states = ws;
     float* trans = ws + slab;
@@ -1274,7 +1297,7 @@ template <bool CHANNEL>
 cudaError_t launch_noalloc(const Problem& p, cudaStream_t stream, bool* over_limit) {
     *over_limit = false;
     const int nchunks = (p.T + C - 1) / C;
-    int nseg = choose_segments(p.segments, p.B * p.H, nchunks, true);
+    int nseg = choose_segments(p.segments, p.B * p.H, nchunks, kNoAllocRule);
     const int seg_len = ((nchunks + nseg - 1) / nseg) * C;
     if (nseg > 1) nseg = (p.T + seg_len - 1) / seg_len;
     const size_t slab = (size_t)p.B * nseg * p.H * D * D;

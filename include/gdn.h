@@ -98,7 +98,14 @@ enum { GDN_IO_BF16 = 0, GDN_IO_F32 = 1 };
  *   gate_mode GDN_GATE_SCALAR or GDN_GATE_CHANNEL.
  *   T == 0 writes state_out := state_in (or zeros) and returns GDN_OK; the
  *   per-token pointers (q, k, v, g, beta, out) may then be NULL.
- * Scratch: with dk = dv = 128 and 2 * B * H <= the SM count, each chunk's
+ * Path (bf16, dk = dv = 128): the segment-parallel path of
+ * gdn_chunk_fwd_segments where its automatic choice gives n > 1 segments --
+ * scalar gate: n = SMs / (B * H) from T > 1984 (32 chunks), when n >= 3,
+ * or n = 2 with 2 * B * H >= 85% of the SMs; per-channel gate:
+ * B * H * 4 <= SMs and T > 4032 (see gdn_chunk_fwd_segments) -- else the
+ * prep pool when 2 * B * H <= the SM count, else one CTA per (batch, head).
+ * Scratch: the segment path's, as gdn_chunk_fwd_segments (if it cannot be
+ * had, the call runs unsegmented).  In the prep pool each chunk's
  * chunk-local results (T' or T and beta, P and the chain's operand tiles:
  * 99,072 bytes) pass from prep CTAs to the state chains through a ring of
  * such records per (batch, head): one per chunk while all of them fit in
@@ -144,10 +151,16 @@ GDN_API int gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const 
  * true starts instead, since w does not fit its fixed scratch.)
  *   num_segments 0 = automatic (what gdn_chunk_fwd does), 1 = none,
  *                n > 1 = n segments (at most one per 64-token chunk;
- *                dk = dv = 128 only).
- * Scratch: (2 * B * n * H * dk * dv + B * T * H * dk) * 4 bytes,
- * stream-ordered on `stream` from the library's pool (GDN_ERR_NOMEM if it
- * cannot be had).  Other arguments as gdn_chunk_fwd.
+ *                dk = dv = 128 only).  Automatic, scalar gate (transitions
+ *                end once decayed, so they are short): n = SMs / (B * H)
+ *                from 32 chunks on, when n >= 3, or n = 2 with
+ *                2 * B * H >= 85% of the SMs; per-channel gate (transitions
+ *                run in full): from B * H * 4 <= SMs and 64 chunks on, the
+ *                largest n with B * H * (2n - 1) <= SMs, at least 3.
+ * Scratch: 2 * B * n * H * dk * dv * 4 + B * T * H * dk * 2 bytes (plus
+ * 4 bytes per segment), stream-ordered on `stream` from the library's pool
+ * (GDN_ERR_NOMEM if it cannot be had with n given; an automatic choice runs
+ * unsegmented instead).  Other arguments as gdn_chunk_fwd.
  */
 GDN_API int gdn_chunk_fwd_segments(const void* q, const void* k, const void* v, const float* g,
                                    const float* beta, const float* state_in, void* out,
@@ -169,7 +182,8 @@ GDN_API int gdn_chunk_fwd_segments(const void* q, const void* k, const void* v, 
  * that loads libgdn holds until the process exits.
  *
  * Limit: the segmented path needs 2 * B * n * H * dk * dv * 4 bytes for n
- * time segments (n as chosen by gdn_chunk_fwd_segments for num_segments);
+ * time segments (n = num_segments; automatic, n = SMs / (B * H) when
+ * B * H * 4 <= SMs and T > 4032, else 1);
  * with dk = dv = 128 that is B * n * H <= 256.  A larger call returns
  * GDN_ERR_SCRATCH_LIMIT and launches nothing.  With n = 1 no scratch is used.
  * bf16 q, k, v and dk = dv = 128 only (else GDN_ERR_UNSUPPORTED).

@@ -1,6 +1,7 @@
 """Host-side logic of bench.py (CPU only): algorithmic byte / flop accounting,
 the reference arm's JSON line, and the max-over-ranks timing with two gloo
 ranks."""
+import dataclasses
 import json
 import os
 import socket
@@ -33,9 +34,16 @@ def test_algorithmic_bytes_match_the_per_token_head_figures():
 
 
 def test_chunk_path_kernels_follow_the_dispatch_rule():
-    assert len(bench.chunk_path_kernels(CONFIGS[5])) == 3            # 16 pairs: segments
-    assert bench.chunk_path_kernels(CONFIGS[2]) == ["chunk_pool_kernel"]
-    assert bench.chunk_path_kernels(CONFIGS[3]) == ["chunk_pool_kernel"]
+    assert len(bench.chunk_path_kernels(CONFIGS[5])) == 3            # 16 pairs: 9 segments
+    assert bench.chunk_path_kernels(CONFIGS[2]) == ["chunk_pool_kernel"]   # per-channel, 64 pairs
+    assert len(bench.chunk_path_kernels(CONFIGS[3])) == 3            # scalar, 48 pairs: 3 segments
+    scalar = CONFIGS[3]
+    # scalar gate, 2 segments: taken with 64 pairs (128 of 148 SMs), not with 50 (100 SMs)
+    assert len(bench.chunk_path_kernels(dataclasses.replace(scalar, B=4, H=16, T=2048))) == 3
+    assert bench.chunk_path_kernels(dataclasses.replace(scalar, B=5, H=10, T=8192)) == ["chunk_pool_kernel"]
+    # too short for segments (31 chunks), and too many pairs for the pool
+    assert bench.chunk_path_kernels(dataclasses.replace(scalar, B=4, H=12, T=1984)) == ["chunk_pool_kernel"]
+    assert bench.chunk_path_kernels(dataclasses.replace(scalar, B=8, H=12, T=8192)) == ["chunk_fwd_kernel"]
 
 
 def test_decode_accounting_matches_hand_count():
