@@ -2,8 +2,8 @@
 dk = dv = 128) against the fp64 oracle.
 
 Tolerance rule: max|got - ref| <= tol * rms(ref), tol = 2e-2 for bf16 I/O.
-Full-size workloads are checked on sampled (b, h) pairs, which the oracle
-computes exactly like the full problem (pairs are independent).
+Full-size workloads are checked pair by pair: every (b, h) pair is held to
+the rule on its own (the oracle computes pairs independently).
 """
 import numpy as np
 import pytest
@@ -138,16 +138,17 @@ def test_prefill_equals_decode_steps(gdn):
 
 
 @pytest.mark.parametrize("index", [2, 3])
-def test_full_config_sampled_heads(gdn, index, oracle_threads):
+def test_full_config_every_pair(gdn, index, oracle_threads):
+    """The GDN-2 layer workload (64 pairs, per-channel gate, prep pool) and the
+    scalar training workload (48 pairs, S0 != 0, segment path): every (b, h)
+    pair against the oracle, each held to the rule on its own."""
     cfg = CONFIGS[index]
     x = config_inputs(cfg)
     got_o, got_s = _gpu(gdn, x)
     BH = cfg.B * cfg.H
-    heads = sorted({0, BH // 3, BH // 2 + 1, BH - 1})
     ref_o, ref_s = oracle.run(x["q"], x["k"], x["v"], x["g"], x["beta"], x["s0"],
-                              per_channel=cfg.per_channel, heads=heads, threads=oracle_threads)
-    _check_pairs(got_o, got_s, ref_o, ref_s, _pairs(x, heads), cfg.tol)
-    assert torch.isfinite(got_o).all() and torch.isfinite(got_s).all()
+                              per_channel=cfg.per_channel, threads=oracle_threads)
+    _check_pairs(got_o, got_s, ref_o, ref_s, _pairs(x, range(BH)), cfg.tol)
 
 
 @pytest.mark.parametrize("gate", ["scalar", "channel"])

@@ -67,22 +67,26 @@ def test_segments_more_than_chunks_is_capped(gdn):
     assert oracle.rel_err(s_seg, ref_s) <= TOL
 
 
-def test_long_context_config_sampled_heads(gdn, oracle_threads):
+def test_long_context_config_every_head(gdn, oracle_threads):
     """B=1, H=16, T=262,144, scalar gate with 10% g = 0; the default entry point
-    (automatic segmentation).  Two heads are checked in full against the
-    oracle; all outputs must be finite."""
+    (automatic segmentation, 9 segments per head).  Every head against the
+    oracle, each held to the rule on its own (the oracle runs 8 heads at a
+    time to bound its fp64 copies at about 9 GB)."""
     cfg = CONFIGS[5]
     x = config_inputs(cfg)
     dev = torch.device("cuda")
     out, s = gdn.chunk_fwd(*(x[n].to(dev) for n in ("q", "k", "v", "g", "beta")), None)
     torch.cuda.synchronize()
-    assert bool(torch.isfinite(out).all()) and bool(torch.isfinite(s).all())
-    for h in (0, 11):
-        sl = {n: x[n][:, :, h:h + 1].contiguous() for n in ("q", "k", "v", "g", "beta")}
+    out, s = out.cpu(), s.cpu()
+    for h0 in range(0, cfg.H, 8):
+        sl = {n: x[n][:, :, h0:h0 + 8].contiguous() for n in ("q", "k", "v", "g", "beta")}
         ref_o, ref_s = oracle.run(sl["q"], sl["k"], sl["v"], sl["g"], sl["beta"], None,
                                   per_channel=False, threads=oracle_threads)
-        assert oracle.rel_err(out[:, :, h:h + 1].cpu(), ref_o) <= cfg.tol, h
-        assert oracle.rel_err(s[:, h:h + 1].cpu(), ref_s) <= cfg.tol, h
+        for j in range(8):
+            eo = oracle.rel_err(out[:, :, h0 + j], ref_o[:, :, j])
+            es = oracle.rel_err(s[:, h0 + j], ref_s[:, j])
+            assert eo <= cfg.tol and es <= cfg.tol, (h0 + j, eo, es)
+        del ref_o, ref_s, sl
 
 
 @pytest.mark.parametrize("pattern", ["floor", "runs"])
