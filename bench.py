@@ -124,16 +124,20 @@ def source_sha1(names) -> str:
     return h.hexdigest()
 
 
-def ncu_traffic(key: str):
+def ncu_traffic(key: str, kernel: str | None = None):
     """DRAM read + write bytes per launch of a workload's dominant kernel, from
     the committed ncu figures (profiles/traffic.json), or None when the kernel
-    sources changed since that capture (the entry records their sha1)."""
+    sources changed since that capture (the entry records their sha1) or the
+    workload now runs another kernel than the one captured (`kernel`: the
+    dominant kernel's name as chunk_path_kernels gives it)."""
     if not TRAFFIC_FILE.exists():
         return None
     entry = json.loads(TRAFFIC_FILE.read_text()).get(key)
     if not entry:
         return None
     try:
+        if kernel is not None and entry["kernel"].split("<")[0].split(" ")[0] != kernel.split(" ")[0]:
+            return None
         if source_sha1(entry["sources"]) != entry["sources_sha1"]:
             return None
         return float(entry["dram_bytes_per_launch"])
@@ -144,18 +148,14 @@ def ncu_traffic(key: str):
 def chunk_path_kernels(cfg, sms: int = 148) -> list:
     """The kernels one gdn_chunk_fwd call launches for a workload (bf16 I/O,
     d = 128), following the library's automatic choice: the segment-parallel
-    path when it picks n > 1 segments (scalar gate: n = #SMs // (B*H) from 32
-    chunks, when n >= 3 or n = 2 with 2*B*H >= 0.85 #SMs; per-channel gate:
-    B*H*4 <= #SMs and 64 chunks, n = (#SMs // (B*H) + 1) // 2 >= 3), else the
+    path when it picks n > 1 segments (n = #SMs // (B*H) from 32 chunks, when
+    n >= 3, or with a scalar gate n = 2 with 2*B*H >= 0.85 #SMs), else the
     prep pool when 2*B*H <= #SMs, else one CTA per (batch, head)."""
     bh = cfg.B * cfg.H
     nchunks = -(-cfg.T // 64)
-    if cfg.per_channel:
-        seg = nchunks >= 64 and bh * 4 <= sms and (sms // bh + 1) // 2 >= 3
-    else:
-        n = sms // bh
-        seg = nchunks >= 32 and (n >= 3 or (n == 2 and 2 * bh * 100 >= 85 * sms))
-    if seg:
+    n = sms // bh
+    two = n == 2 and not cfg.per_channel and 2 * bh * 100 >= 85 * sms
+    if nchunks >= 32 and (n >= 3 or two):
         return ["chunk_fwd_kernel (zero-start + transition CTAs)", "combine_segments_kernel",
                 "segment_correction_kernel"]
     if 2 * bh <= sms:
@@ -462,7 +462,7 @@ def run_ours(args, rank: int, world: int, local: int):
     nflops = prefill_flops(cfg)
     gbs = nbytes / t_call / 1e9
     roofline = {"bound": "hbm", "achieved": _r(gbs), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": _r(gbs / peaks["hbm_gbs"]), "traffic": ncu_traffic("long_context"),
+                "frac": _r(gbs / peaks["hbm_gbs"]), "traffic": ncu_traffic("long_context", chunk_path_kernels(HEAD_CFG)[0]),
                 "bytes_per_call": nbytes, "kernels": chunk_path_kernels(cfg),
                 "peak_source": peaks["source"]}
     tflops = nflops / t_call / 1e12
@@ -586,7 +586,7 @@ def run_prefill(gdn, cfg, dev, stream, peaks, world, rank, steps: int = 20, warm
     return {"tok_s": _r(cfg.B * cfg.T * world / t), "us": _r(t * 1e6), "GB/s": _r(gbs),
             "frac": _r(gbs / peaks["hbm_gbs"]),
             "tensor_frac": _r(prefill_flops(cfg) / t / 1e12 / peaks["bf16_tflops"]),
-            "traffic": ncu_traffic(key), "kernels": chunk_path_kernels(cfg)}
+            "traffic": ncu_traffic(key, chunk_path_kernels(cfg)[0]), "kernels": chunk_path_kernels(cfg)}
 
 
 def run_decode(gdn, dev, stream, peaks, world, rank, n_steps: int = 1024, n_states: int = 6,

@@ -164,11 +164,11 @@ struct Params {
     // that transition CTAs cover segments trans_first .. nseg - 1.
     int trans_first = 0;
     bool in_first_only = false;
-    // Early end of the transitions (scalar gate; [B, nseg, H] chunks run;
-    // null: run every chunk).  Every step of the recurrence is a contraction
-    // when g <= 0, beta in [0, 1] and |k| = 1 (the model card's input domain,
-    // section 2.1): |I - b k k^T|_2 <= 1 while 0 <= b |k|^2 <= 2, and
-    // |exp(g)| <= 1.  So once max |M_ij| <= kTransitionDrop after a chunk,
+    // Early end of the transitions ([B, nseg, H] chunks run; null: run every
+    // chunk).  Every step of the recurrence is a contraction when g <= 0
+    // (every channel of a per-channel gate), beta in [0, 1] and |k| = 1 (the
+    // model card's input domain, section 2.1): |I - b k k^T|_2 <= 1 while
+    // 0 <= b |k|^2 <= 2, and |Diag(exp(g))|_2 <= 1.  So once max |M_ij| <= kTransitionDrop after a chunk,
     // every later M_t' has |M_t'|_2 <= 128 kTransitionDrop = 2^-53, and
     // dropping it changes an output by at most 2^-53 |S_start|_2 |q| --
     // below fp32 resolution.  A transition CTA checks the domain on the
@@ -308,7 +308,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     int tma_issued = nchunks > 0 ? 1 : 0;   // chunks whose loads were issued (tid 0)
     // Transition CTAs that may stop early: this thread has seen a token
     // outside the contracting domain (sticky), and the chunks run so far.
-    const bool may_stop = !CHANNEL && transition && p.trans_len != nullptr;
+    const bool may_stop = transition && p.trans_len != nullptr;
     bool outside = false;
     bool stopped = false;
     int chunks_run = nchunks;
@@ -372,6 +372,13 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             for (int u = 0; u < 4; ++u)
 #pragma unroll
                 for (int e = 0; e < 8; ++e) gam[u][e] = gnext[u][e];
+            if (may_stop) {   // this thread's 4 tokens x 8 channels of g (0 past T)
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        if (!(gnext[u][e] <= 0.f)) outside = true;
+            }
             // Inclusive scan over the 16 lanes of each 16-token block, then add
             // the totals of the preceding blocks.
 #pragma unroll
@@ -864,13 +871,23 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             for (int w = 1; w < NT / 32; ++w) m = fmaxf(m, sRed[w]);
             if (m <= kTransitionDrop) {
                 // The tokens not run must be inside the domain too: scan their
-                // beta and g (8 bytes a token); unit keys are the caller's
-                // contract.
+                // beta and g (8 bytes a token; 4 + 4 dk with a per-channel
+                // gate); unit keys are the caller's contract.
                 bool bad = false;
-                for (long t = t0 + C + tid; t < t_end; t += NT) {
-                    const long i = ((long)b * T + t) * H + h;
-                    const float bt = p.beta[i], gt = p.g[i];
-                    bad |= !(bt >= 0.f && bt <= 1.f && gt <= 0.f);
+                if (!CHANNEL) {
+                    for (long t = t0 + C + tid; t < t_end; t += NT) {
+                        const long i = ((long)b * T + t) * H + h;
+                        const float bt = p.beta[i], gt = p.g[i];
+                        bad |= !(bt >= 0.f && bt <= 1.f && gt <= 0.f);
+                    }
+                } else {
+                    const long nt = t_end - (t0 + C);
+                    for (long e = tid; e < nt * (D / 4); e += NT) {
+                        const long i = ((long)b * T + t0 + C + e / (D / 4)) * H + h;
+                        const float4 gv = reinterpret_cast<const float4*>(p.g + i * D)[e % (D / 4)];
+                        bad |= !(gv.x <= 0.f && gv.y <= 0.f && gv.z <= 0.f && gv.w <= 0.f);
+                        if (e % (D / 4) == 0) bad |= !(p.beta[i] >= 0.f && p.beta[i] <= 1.f);
+                    }
                 }
                 if (!__syncthreads_or(bad)) {
                     stopped = true;
@@ -1142,31 +1159,31 @@ segment_correction_kernel(const float* __restrict__ seg_states, const __half* __
 // chunk recursion per segment (the transition), a combine and a correction,
 // so it pays only when the (batch, head) pairs alone leave SMs idle.
 // Automatic choice (requested == 0):
-//  * kScalarRule (transitions expected to end early): one zero-start CTA per
-//    SM, n = #SMs / (B*H), from 32 chunks on, when n >= 3, or n = 2 with at
-//    least 85% of the SMs busy.  Measured on B200 (T 8192, B*H = 48):
-//    n = 3 430 us, the prep pool 556 us, n = 2 (96 SMs busy) 611 us; at
-//    B*H = 64 (T 2048) n = 2 took 190 us against 213 us pooled.
-//  * kChannelRule (transitions run in full): the largest n whose
-//    B*H*(2n - 1) CTAs fit in one wave, from B*H*4 <= #SMs and 64 chunks
-//    on, at least 3.
+//  * kDecayRule (the transitions end once decayed, after a chunk or two with
+//    decaying gates): one zero-start CTA per SM, n = #SMs / (B*H), from 32
+//    chunks on, when n >= 3, or (scalar gate) n = 2 with at least 85% of the
+//    SMs busy.  Measured on B200 against the prep pool (us): scalar gate,
+//    T 8192, B*H = 48: n = 3 430, pool 556, n = 2 (96 SMs busy) 611;
+//    B*H = 64, T 2048: n = 2 190, pool 213.  Per-channel gate: B*H = 48,
+//    T 8192: n = 3 641, pool 697; B*H = 32, T 16384: n = 4 808, pool 1347;
+//    B*H = 16, T 65536: n = 9 1551, n = 5 with full transitions 2443; but
+//    B*H = 64, T 2048: n = 2 227-232, pool 225-229 (no gain: the pool keeps
+//    per-channel gates at n = 2).
 //  * kNoAllocRule (the fixed-scratch entry, whose transitions run in full
-//    but whose segments each need only two states): n = #SMs / (B*H) from
+//    and whose segments need two states each): n = #SMs / (B*H) from
 //    B*H*4 <= #SMs and 64 chunks on.
-enum SegmentRule { kScalarRule, kChannelRule, kNoAllocRule };
-int choose_segments(int requested, int BH, int nchunks, SegmentRule rule) {
+enum SegmentRule { kDecayRule, kNoAllocRule };
+int choose_segments(int requested, int BH, int nchunks, SegmentRule rule, bool channel) {
     if (nchunks <= 1 || requested == 1) return 1;
     int n = requested;
     if (n <= 0) {
         const int sms = sm_count();
-        if (rule == kScalarRule) {
-            n = sms / BH;
+        n = sms / BH;
+        if (rule == kDecayRule) {
             if (nchunks < 32 || n < 2) return 1;
-            if (n == 2 && 2 * BH * 100 < 85 * sms) return 1;
-        } else {
-            if (nchunks < 64 || BH * 4 > sms) return 1;
-            n = rule == kNoAllocRule ? sms / BH : (sms / BH + 1) / 2;
-            if (n < 3) return 1;
+            if (n == 2 && (channel || 2 * BH * 100 < 85 * sms)) return 1;
+        } else if (nchunks < 64 || n < 4) {
+            return 1;
         }
     }
     return n < nchunks ? n : nchunks;
@@ -1182,7 +1199,7 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
         return cudaErrorInvalidValue;
     float* out = static_cast<float*>(p.out);
     const int nchunks = (p.T + C - 1) / C;
-    int nseg = choose_segments(p.segments, p.B * p.H, nchunks, CHANNEL ? kChannelRule : kScalarRule);
+    int nseg = choose_segments(p.segments, p.B * p.H, nchunks, kDecayRule, CHANNEL);
     auto unsegmented = [&]() -> cudaError_t {
         // Chunk-local work and the state chain on different SMs when two per
         // (batch, head) fit: by default one prep pool over all SMs; a cluster
@@ -1251,7 +1268,7 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
     e = cudaGetLastError();
     if (e == cudaSuccess) {
         combine_segments_kernel<<<p.B * p.H * (D / CB_COLS), 256, 0, stream>>>(
-            seg_states, trans, p.state_in, p.state_out, p.H, nseg, 1, CHANNEL ? nullptr : trans_len);
+            seg_states, trans, p.state_in, p.state_out, p.H, nseg, 1, trans_len);
         e = cudaGetLastError();
     }
     if (e == cudaSuccess) {
@@ -1259,7 +1276,7 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
         if (e == cudaSuccess) {
             const int groups = (seg_len / C + CORR_TILES - 1) / CORR_TILES;
             segment_correction_kernel<<<dim3(groups, (nseg - 1) * p.H, p.B), 256, sizeof(CorrSmem), stream>>>(
-                seg_states, wbuf, out, p.T, p.H, nseg, seg_len, 1, CHANNEL ? nullptr : trans_len);
+                seg_states, wbuf, out, p.T, p.H, nseg, seg_len, 1, trans_len);
             e = cudaGetLastError();
         }
     }
@@ -1297,7 +1314,7 @@ template <bool CHANNEL>
 cudaError_t launch_noalloc(const Problem& p, cudaStream_t stream, bool* over_limit) {
     *over_limit = false;
     const int nchunks = (p.T + C - 1) / C;
-    int nseg = choose_segments(p.segments, p.B * p.H, nchunks, kNoAllocRule);
+    int nseg = choose_segments(p.segments, p.B * p.H, nchunks, kNoAllocRule, CHANNEL);
     const int seg_len = ((nchunks + nseg - 1) / nseg) * C;
     if (nseg > 1) nseg = (p.T + seg_len - 1) / seg_len;
     const size_t slab = (size_t)p.B * nseg * p.H * D * D;

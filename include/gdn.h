@@ -99,11 +99,10 @@ enum { GDN_IO_BF16 = 0, GDN_IO_F32 = 1 };
  *   T == 0 writes state_out := state_in (or zeros) and returns GDN_OK; the
  *   per-token pointers (q, k, v, g, beta, out) may then be NULL.
  * Path (bf16, dk = dv = 128): the segment-parallel path of
- * gdn_chunk_fwd_segments where its automatic choice gives n > 1 segments --
- * scalar gate: n = SMs / (B * H) from T > 1984 (32 chunks), when n >= 3,
- * or n = 2 with 2 * B * H >= 85% of the SMs; per-channel gate:
- * B * H * 4 <= SMs and T > 4032 (see gdn_chunk_fwd_segments) -- else the
- * prep pool when 2 * B * H <= the SM count, else one CTA per (batch, head).
+ * gdn_chunk_fwd_segments where its automatic choice gives n > 1 segments
+ * (n = SMs / (B * H) from T > 1984, i.e. 32 chunks, when n >= 3, or with a
+ * scalar gate n = 2 with 2 * B * H >= 85% of the SMs), else the prep pool when
+ * 2 * B * H <= the SM count, else one CTA per (batch, head).
  * Scratch: the segment path's, as gdn_chunk_fwd_segments (if it cannot be
  * had, the call runs unsegmented).  In the prep pool each chunk's
  * chunk-local results (T' or T and beta, P and the chain's operand tiles:
@@ -151,12 +150,12 @@ GDN_API int gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const 
  * true starts instead, since w does not fit its fixed scratch.)
  *   num_segments 0 = automatic (what gdn_chunk_fwd does), 1 = none,
  *                n > 1 = n segments (at most one per 64-token chunk;
- *                dk = dv = 128 only).  Automatic, scalar gate (transitions
- *                end once decayed, so they are short): n = SMs / (B * H)
- *                from 32 chunks on, when n >= 3, or n = 2 with
- *                2 * B * H >= 85% of the SMs; per-channel gate (transitions
- *                run in full): from B * H * 4 <= SMs and 64 chunks on, the
- *                largest n with B * H * (2n - 1) <= SMs, at least 3.
+ *                dk = dv = 128 only).  Automatic: n = SMs / (B * H) from
+ *                32 chunks on, when n >= 3, or with a scalar gate n = 2
+ *                with 2 * B * H >= 85% of the SMs.  A segment's transition ends once every entry
+ *                has decayed below 2^-60 while every token it covers is in
+ *                the contracting domain (g <= 0, 0 <= beta <= 1, unit k);
+ *                with decaying gates that is after a chunk or two.
  * Scratch: 2 * B * n * H * dk * dv * 4 + B * T * H * dk * 2 bytes (plus
  * 4 bytes per segment), stream-ordered on `stream` from the library's pool
  * (GDN_ERR_NOMEM if it cannot be had with n given; an automatic choice runs

@@ -35,7 +35,8 @@ def test_algorithmic_bytes_match_the_per_token_head_figures():
 
 def test_chunk_path_kernels_follow_the_dispatch_rule():
     assert len(bench.chunk_path_kernels(CONFIGS[5])) == 3            # 16 pairs: 9 segments
-    assert bench.chunk_path_kernels(CONFIGS[2]) == ["chunk_pool_kernel"]   # per-channel, 64 pairs
+    assert bench.chunk_path_kernels(CONFIGS[2]) == ["chunk_pool_kernel"]   # per-channel, n = 2: pool
+    assert len(bench.chunk_path_kernels(dataclasses.replace(CONFIGS[2], B=4, H=12))) == 3   # n = 3
     assert len(bench.chunk_path_kernels(CONFIGS[3])) == 3            # scalar, 48 pairs: 3 segments
     scalar = CONFIGS[3]
     # scalar gate, 2 segments: taken with 64 pairs (128 of 148 SMs), not with 50 (100 SMs)

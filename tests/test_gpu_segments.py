@@ -104,33 +104,64 @@ def test_segments_channel_gate_at_its_bound(gdn, pattern):
     assert oracle.rel_err(s_seg, ref_s) <= TOL
 
 
-def test_segments_without_decay_run_full_transitions(gdn):
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+def test_segments_without_decay_run_full_transitions(gdn, gate):
     """g = 0 and a small beta: the transition of a segment barely decays, so
     no transition may end early; the segmented result must still be exact."""
-    x = prefill_inputs(1, 1200, 2, 128, 128, gate="scalar", s0_std=0.1, seed=330)
+    x = prefill_inputs(1, 1200, 2, 128, 128, gate=gate, s0_std=0.1, seed=330)
     x["g"].zero_()
     x["beta"] = (0.02 * x["beta"]).contiguous()
     o_seg, s_seg = _run(gdn, x, 4)
-    ref_o, ref_s = oracle.run(x["q"], x["k"], x["v"], x["g"], x["beta"], x["s0"], per_channel=False)
+    ref_o, ref_s = oracle.run(x["q"], x["k"], x["v"], x["g"], x["beta"], x["s0"],
+                              per_channel=gate == "channel")
     assert oracle.rel_err(o_seg, ref_o) <= TOL
     assert oracle.rel_err(s_seg, ref_s) <= TOL
 
 
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
 @pytest.mark.parametrize("late", ["beta_above_one", "positive_g"])
-def test_segments_with_tokens_outside_the_contracting_domain(gdn, late):
+def test_segments_with_tokens_outside_the_contracting_domain(gdn, gate, late):
     """Fast decay first (the transitions would end after a chunk or two),
     then tokens outside the domain that makes every step a contraction
-    (beta > 1, or g > 0): the early end must not be taken, and the result
-    must match the oracle."""
-    x = prefill_inputs(1, 1024, 2, 128, 128, gate="scalar", s0_std=0.1, seed=331)
+    (beta > 1, or g > 0 -- in one channel of a per-channel gate): the early
+    end must not be taken, and the result must match the oracle."""
+    x = prefill_inputs(1, 1024, 2, 128, 128, gate=gate, s0_std=0.1, seed=331)
     g, beta = x["g"].clone(), x["beta"].clone()
-    g[:, :, :] = -3.0
+    g[...] = -3.0
     if late == "beta_above_one":
         beta[:, 600:610] = 1.8
-    else:
+    elif gate == "scalar":
         g[:, 600:610] = 0.05
+    else:
+        g[:, 600:610, :, 77] = 0.05
     x["g"], x["beta"] = g.contiguous(), beta.contiguous()
     o_seg, s_seg = _run(gdn, x, 3)
-    ref_o, ref_s = oracle.run(x["q"], x["k"], x["v"], x["g"], x["beta"], x["s0"], per_channel=False)
+    ref_o, ref_s = oracle.run(x["q"], x["k"], x["v"], x["g"], x["beta"], x["s0"],
+                              per_channel=gate == "channel")
+    assert oracle.rel_err(o_seg, ref_o) <= TOL
+    assert oracle.rel_err(s_seg, ref_s) <= TOL
+
+
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+@pytest.mark.parametrize("what", ["beta", "g"])
+def test_segments_outside_the_domain_in_a_chunk_they_run(gdn, gate, what):
+    """A token outside the domain inside the first chunk of every segment
+    (token 5 of each: beta = 2.5, so beta |k|^2 > 2, or g = +0.05 -- in one
+    channel of a per-channel gate), where the transition runs rather than
+    skips it: the in-kernel checks on run tokens must keep the transitions
+    in full."""
+    x = prefill_inputs(1, 960, 2, 128, 128, gate=gate, s0_std=0.1, seed=332)
+    beta, g = x["beta"].clone(), x["g"].clone()
+    for t in (5, 325, 645):                   # 3 segments of 320 tokens
+        if what == "beta":
+            beta[:, t] = 2.5
+        elif gate == "scalar":
+            g[:, t] = 0.05
+        else:
+            g[:, t, :, 77] = 0.05
+    x["beta"], x["g"] = beta.contiguous(), g.contiguous()
+    o_seg, s_seg = _run(gdn, x, 3)
+    ref_o, ref_s = oracle.run(x["q"], x["k"], x["v"], x["g"], x["beta"], x["s0"],
+                              per_channel=gate == "channel")
     assert oracle.rel_err(o_seg, ref_o) <= TOL
     assert oracle.rel_err(s_seg, ref_s) <= TOL
