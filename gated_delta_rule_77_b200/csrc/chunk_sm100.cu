@@ -101,6 +101,7 @@ constexpr uint32_t CB_HALF = 96 * 128;
 constexpr uint32_t OFF_KE = R_X;             //   16 KB K*E fp16  [half][64 r][128 B]
 constexpr uint32_t OFF_ZH = R_X;              //   after Y: Z^T = V^T - Y^T bf16 hi [128 j][64 r]
 constexpr uint32_t OFF_OST = R_X;            //   at the chunk's end: 32 KB O fp32 [64 t][128 j] (TMA store)
+constexpr uint32_t OFF_OST_LATE = R_X + 81920;  // scalar gate: the same, over A / T / U (see finish_chunk)
 constexpr uint32_t OFF_QE = R_X + 16384;     //   16 KB Q*E fp16
 constexpr uint32_t OFF_ZL = R_X + 16384;      //   after Y and the first O products: Z^T lo
 constexpr uint32_t OFF_KDH = R_X + 32768;    //   16 KB K*D bf16 hi
@@ -120,8 +121,8 @@ constexpr uint32_t SM_LAST = SM_REF1 + 512;   // 128 f32: G at token 63
 constexpr uint32_t SM_ER = SM_LAST + 512;     // 64 f32: exp(G_r - G_31)  (scalar gate)
 constexpr uint32_t SM_FJ = SM_ER + 256;       // 64 f32: exp(G_31 - G_j)
 constexpr uint32_t SM_SAFE = SM_FJ + 256;     // int: product form in range
-constexpr uint32_t SM_BAR = SM_SAFE + 16;     // 3 mbarriers: loads, products, products into O
-constexpr uint32_t SM_TMEM = SM_BAR + 24;     // TMEM base address
+constexpr uint32_t SM_BAR = SM_SAFE + 16;     // 4 mbarriers: loads, products, products into O, SN
+constexpr uint32_t SM_TMEM = SM_BAR + 32;     // TMEM base address
 constexpr uint32_t SM_RED = SM_TMEM + 16;     // 8 f32: per-warp max |M| (transition CTAs)
 constexpr uint32_t SMEM_USED = SM_RED + 32;
 
@@ -208,6 +209,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t bar_tma = sbase + SM_BAR;
     const uint32_t bar_mma = sbase + SM_BAR + 8;
     const uint32_t bar_out = sbase + SM_BAR + 16;   // O^T products, committed apart
+    const uint32_t bar_sn = sbase + SM_BAR + 24;    // SN, committed apart
     uint32_t* sTmemBase = reinterpret_cast<uint32_t*>(smem + SM_TMEM);
     float* sRed = reinterpret_cast<float*>(smem + SM_RED);
 
@@ -251,6 +253,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         mbar_init(bar_tma, 1);
         mbar_init(bar_mma, 1);
         mbar_init(bar_out, 1);
+        mbar_init(bar_sn, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -358,6 +361,115 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     float gnext[4][8], bgnext[4];
     if (CHANNEL && nchunks > 0) load_gate(0, gnext);
     if (nchunks > 0) load_beta(0, bgnext);
+
+    // With a scalar gate the next chunk's X product reads only the raw K and Q
+    // (R_IN), so the state step of chunk c can follow the issue of chunk
+    // c + 1's X (see finish_chunk).
+    constexpr bool LATE = !CHANNEL;
+    constexpr uint32_t OST = LATE ? OFF_OST_LATE : OFF_OST;
+    float e_last = 1.f;       // E_last of the chunk whose state step is due
+    uint32_t sn_phase = 0;
+    int pending = -1;         // LATE: the chunk whose state step is due
+    // The state update and output of chunk cj: S <- Diag(E_last) S + SN, its
+    // fp16 copy for the next chunk's products, O (or w) to shared memory and
+    // one TMA store, and a transition's early end.  0: go on, 1: abandoned
+    // (a bounded wait ran out), 2: the transition ended early.  With a scalar
+    // gate (LATE) it runs one chunk late, after the next chunk's gate prep and
+    // the issue of its X product, so that those overlap the SN and O products;
+    // its O goes to a staging tile clear of the next chunk's derived tiles.
+    auto finish_chunk = [&](int cj) -> int {
+        const int tj0 = t_begin + cj * C;
+        ok = ok && mbar_wait(bar_sn, sn_phase, &g_status_word);
+        sn_phase ^= 1;
+        tc_fence_after();
+        float o[32];
+        {
+            const uint32_t lb = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+            {
+                float sn0[32], sn1[32];
+                tmem_ld32(lb + TM_SN + half * 64, sn0);
+                tmem_ld32(lb + TM_SN + half * 64 + 32, sn1);
+                tmem_wait_ld();
+                const float2 e2 = make_float2(e_last, e_last);
+#pragma unroll
+                for (int c = 0; c < 32; c += 2) {
+                    const float2 a = fma2(e2, make_float2(s[c], s[c + 1]), make_float2(sn0[c], sn0[c + 1]));
+                    const float2 z = fma2(e2, make_float2(s[32 + c], s[33 + c]), make_float2(sn1[c], sn1[c + 1]));
+                    s[c] = a.x; s[c + 1] = a.y; s[32 + c] = z.x; s[33 + c] = z.y;
+                }
+            }
+            write_state_f16();
+            if (want_o) {
+                ok = ok && mbar_wait(bar_out, cj & 1, &g_status_word);
+                tc_fence_after();
+                tmem_ld32(lb + TM_OT + half * 32, o);
+                tmem_wait_ld();
+                // O^T (lane = value column) -> [token][column] fp32 over the
+                // consumed K*E / Q*E tiles; one TMA store per chunk, rows past
+                // T dropped.  Thread stores would hold up the next proxy fence.
+                if (transition) {   // w in fp16
+                    __half* sh = reinterpret_cast<__half*>(smem + OST) + half * 32 * D + srow;
+#pragma unroll
+                    for (int r = 0; r < 32; ++r) sh[r * D] = __float2half_rn(o[r]);
+                } else {
+                    float* so = reinterpret_cast<float*>(smem + OST) + half * 32 * D + srow;
+#pragma unroll
+                    for (int r = 0; r < 32; ++r) so[r * D] = o[r];
+                }
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        if (may_stop) {   // this chunk's max |M| (or +inf outside the domain), per warp
+            float m = 0.f;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) m = fmaxf(m, fabsf(s[c]));
+            if (outside) m = __int_as_float(0x7f800000);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (lane == 0) sRed[warp] = m;
+        }
+        if (__syncthreads_or(!ok)) return 1;
+        if (want_o && tid == 0) {
+            tma_store_4d(tm_store, sbase + OST, 0, h, tj0, b);
+            bulk_commit();
+        }
+        if (may_stop && cj + 1 < nchunks) {
+            // Read by every thread between this barrier and the next chunk's
+            // first one; rewritten only at the next chunk's end.
+            float m = sRed[0];
+#pragma unroll
+            for (int w = 1; w < NT / 32; ++w) m = fmaxf(m, sRed[w]);
+            if (m <= kTransitionDrop) {
+                // The tokens not run must be inside the domain too: scan their
+                // beta and g (8 bytes a token; 4 + 4 dk with a per-channel
+                // gate); unit keys are the caller's contract.
+                bool bad = false;
+                if (!CHANNEL) {
+                    for (long t = tj0 + C + tid; t < t_end; t += NT) {
+                        const long i = ((long)b * T + t) * H + h;
+                        const float bt = p.beta[i], gt = p.g[i];
+                        bad |= !(bt >= 0.f && bt <= 1.f && gt <= 0.f);
+                    }
+                } else {
+                    const long nt = t_end - (tj0 + C);
+                    for (long e = tid; e < nt * (D / 4); e += NT) {
+                        const long i = ((long)b * T + tj0 + C + e / (D / 4)) * H + h;
+                        const float4 gv = reinterpret_cast<const float4*>(p.g + i * D)[e % (D / 4)];
+                        bad |= !(gv.x <= 0.f && gv.y <= 0.f && gv.z <= 0.f && gv.w <= 0.f);
+                        if (e % (D / 4) == 0) bad |= !(p.beta[i] >= 0.f && p.beta[i] <= 1.f);
+                    }
+                }
+                if (!__syncthreads_or(bad)) {
+                    stopped = true;
+                    chunks_run = cj + 1;
+                    return 2;
+                }
+                outside = true;   // some later token is outside: run every chunk
+            }
+        }
+        return 0;
+    };
 
     for (int ci = 0; ci < nchunks; ++ci) {
         const int t0 = t_begin + ci * C;
@@ -541,6 +653,14 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             mma_sync();
             if (__syncthreads_or(!ok)) break;
         }
+        if (LATE && ci > 0) {
+            const int r = finish_chunk(ci - 1);
+            pending = -1;
+            if (r != 0) {
+                if (r == 2) mma_sync();      // ended early: this chunk's X is in flight
+                break;
+            }
+        }
         if (ci + 1 < nchunks) load_beta(ci + 1, bgnext);
 
         // ------------------------------- derived tiles; A and P from X ----------
@@ -591,6 +711,9 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         fence_async_smem();                  // K*E, Q*E -> the products below
         if (!CHANNEL) mma_sync();            // X
+        // LATE: the previous chunk's output store has read its staging tile,
+        // which the A/P epilogue below overwrites.
+        if (LATE && tid == 0) bulk_wait_read_all();
         if (__syncthreads_or(!ok)) break;
         // Y^T = S^T (K*E)^T and O^T = S^T (Q*E)^T: the state-dependent
         // products that need only this chunk's derived tiles, issued now, so
@@ -686,7 +809,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
         }
         // Decay of the state over the whole chunk, per key row (own row).
-        const float e_last = __expf(CHANNEL ? sLast[srow] : sGam[C - 1]);
+        e_last = __expf(CHANNEL ? sLast[srow] : sGam[C - 1]);
 
         // Z^T = V^T - Y^T -> bf16 hi + lo [128 j][64 r] over the consumed K*E
         // and Q*E tiles (thread: value column j = srow, 32 tokens).
@@ -792,7 +915,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 mma_bf16(tmem + TM_SN, kdh, ul, id_s, 1);
                 mma_bf16(tmem + TM_SN, kdl, uh, id_s, 1);
             }
-            mma_commit(bar_mma);
+            mma_commit(bar_sn);
             if (want_o) {
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
@@ -807,97 +930,14 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 mma_commit(bar_out);
             }
         }
-        mma_sync();
-        if (__syncthreads_or(!ok)) break;
-
-        // ---------------------------------------------------- state and output --
-        float o[32];
-        {
-            const uint32_t lb = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-            {
-                float sn0[32], sn1[32];
-                tmem_ld32(lb + TM_SN + half * 64, sn0);
-                tmem_ld32(lb + TM_SN + half * 64 + 32, sn1);
-                tmem_wait_ld();
-                const float2 e2 = make_float2(e_last, e_last);
-#pragma unroll
-                for (int c = 0; c < 32; c += 2) {
-                    const float2 a = fma2(e2, make_float2(s[c], s[c + 1]), make_float2(sn0[c], sn0[c + 1]));
-                    const float2 z = fma2(e2, make_float2(s[32 + c], s[33 + c]), make_float2(sn1[c], sn1[c + 1]));
-                    s[c] = a.x; s[c + 1] = a.y; s[32 + c] = z.x; s[33 + c] = z.y;
-                }
-            }
-            write_state_f16();
-            if (want_o) {
-                ok = ok && mbar_wait(bar_out, ci & 1, &g_status_word);
-                tc_fence_after();
-                tmem_ld32(lb + TM_OT + half * 32, o);
-                tmem_wait_ld();
-                // O^T (lane = value column) -> [token][column] fp32 over the
-                // consumed K*E / Q*E tiles; one TMA store per chunk, rows past
-                // T dropped.  Thread stores would hold up the next proxy fence.
-                if (transition) {   // w in fp16
-                    __half* sh = reinterpret_cast<__half*>(smem + OFF_OST) + half * 32 * D + srow;
-#pragma unroll
-                    for (int r = 0; r < 32; ++r) sh[r * D] = __float2half_rn(o[r]);
-                } else {
-                    float* so = reinterpret_cast<float*>(smem + OFF_OST) + half * 32 * D + srow;
-#pragma unroll
-                    for (int r = 0; r < 32; ++r) so[r * D] = o[r];
-                }
-            }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        if (may_stop) {   // this chunk's max |M| (or +inf outside the domain), per warp
-            float m = 0.f;
-#pragma unroll
-            for (int c = 0; c < 64; ++c) m = fmaxf(m, fabsf(s[c]));
-            if (outside) m = __int_as_float(0x7f800000);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            if (lane == 0) sRed[warp] = m;
-        }
-        if (__syncthreads_or(!ok)) break;
-        if (want_o && tid == 0) {
-            tma_store_4d(tm_store, sbase + OFF_OST, 0, h, t0, b);
-            bulk_commit();
-        }
-        if (may_stop && ci + 1 < nchunks) {
-            // Read by every thread between this barrier and the next chunk's
-            // first one; rewritten only at the next chunk's end.
-            float m = sRed[0];
-#pragma unroll
-            for (int w = 1; w < NT / 32; ++w) m = fmaxf(m, sRed[w]);
-            if (m <= kTransitionDrop) {
-                // The tokens not run must be inside the domain too: scan their
-                // beta and g (8 bytes a token; 4 + 4 dk with a per-channel
-                // gate); unit keys are the caller's contract.
-                bool bad = false;
-                if (!CHANNEL) {
-                    for (long t = t0 + C + tid; t < t_end; t += NT) {
-                        const long i = ((long)b * T + t) * H + h;
-                        const float bt = p.beta[i], gt = p.g[i];
-                        bad |= !(bt >= 0.f && bt <= 1.f && gt <= 0.f);
-                    }
-                } else {
-                    const long nt = t_end - (t0 + C);
-                    for (long e = tid; e < nt * (D / 4); e += NT) {
-                        const long i = ((long)b * T + t0 + C + e / (D / 4)) * H + h;
-                        const float4 gv = reinterpret_cast<const float4*>(p.g + i * D)[e % (D / 4)];
-                        bad |= !(gv.x <= 0.f && gv.y <= 0.f && gv.z <= 0.f && gv.w <= 0.f);
-                        if (e % (D / 4) == 0) bad |= !(p.beta[i] >= 0.f && p.beta[i] <= 1.f);
-                    }
-                }
-                if (!__syncthreads_or(bad)) {
-                    stopped = true;
-                    chunks_run = ci + 1;
-                    break;
-                }
-                outside = true;   // some later token is outside: run every chunk
-            }
+        if (LATE) {
+            pending = ci;                // its state and output: next iteration
+        } else {
+            const int r = finish_chunk(ci);
+            if (r != 0) break;
         }
     }
+    if (LATE && pending >= 0 && ok) finish_chunk(pending);
     if (tid == 0) bulk_wait_all();     // output stores complete before exit
     if (tid == 0 && stopped && tma_issued > tma_waited + 1)   // the next chunk's loads
         mbar_wait(bar_tma, (tma_waited + 1) & 1, &g_status_word);
