@@ -686,7 +686,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             // (the fused prologue's next history rows and taps are loaded after
             // this item's conversion, below)
             ok = ok && mbar_wait(bar_tma, ci & 1, &g_pair_status_word);
-            kq_waited = ci;
+            if (ok) kq_waited = ci;   // else drained at exit
             if (POOL && tid == 0 && item_chunk >= p.ring && !slot_free) {
                 // The slot's previous record (chunk - ring) must have been
                 // read by its chain before anything is stored into it
@@ -1034,8 +1034,8 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
         if (tid == 0) {
             bulk_wait_all();                 // own copies complete before exit
             if (POOL && pending_flag) publish();
-            if (!ok && kq_issued > kq_waited + 1)
-                mbar_wait(bar_tma, (kq_waited + 1) & 1, &g_pair_status_word);
+            for (int i = kq_waited + 1; !ok && i < kq_issued; ++i)   // K/Q tiles still in flight
+                mbar_wait(bar_tma, i & 1, &g_pair_status_word);
             for (int i = g_waited; !ok && i < g_issued; ++i)   // g tiles still in flight
                 mbar_wait(bar_g, i & 1, &g_pair_status_word);
         }
@@ -1223,7 +1223,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                 gate_scalar(bgnext, sGam, nullptr);
             }
             ok = ok && mbar_wait(bar_kq, ci & 1, &g_pair_status_word);
-            kq_waited = ci;
+            if (ok) kq_waited = ci;   // else drained at exit
             if (__syncthreads_or(!ok)) break;
 
             // K*E (bf16), Q*E (fp16), K*D (bf16 hi + lo), on channel pairs.
@@ -1286,7 +1286,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             if (tid == 0 || (POOL && CHANNEL)) {   // pool, per-channel: every thread reads T
                 ok = ok && (POOL ? mbar_wait(bar_full, ci & 1, &g_pair_status_word)
                                  : mbar_wait_cluster(bar_full, ci & 1, &g_pair_status_word));
-                full_waited = ci;
+                if (ok) full_waited = ci;   // else drained at exit
             }
             if (POOL && CHANNEL && ok) {   // T' = T Diag(beta) as bf16 hi + lo (lower triangle)
                 const float* sTc = reinterpret_cast<const float*>(smem + C_TF);
@@ -1307,7 +1307,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                 fence_async_smem();
             }
             ok = ok && mbar_wait(bar_v, ci & 1, &g_pair_status_word);
-            v_waited = ci;
+            if (ok) v_waited = ci;   // else drained at exit
             if (__syncthreads_or(!ok)) break;
             if constexpr (PRO) {
                 // Fused prologue: the raw v tile becomes the recurrence's v in
@@ -1351,7 +1351,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
           }
             if (POOL && !W_READY && tid == 0) {   // Q*E of this chunk, for the O products below
                 ok = ok && mbar_wait(bar_full_b, ci & 1, &g_pair_status_word);
-                b_waited = ci;
+                if (ok) b_waited = ci;   // else drained at exit
             }
             fence_async_smem();
             tc_fence_before();
@@ -1383,7 +1383,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                 mma_commit(bar_mma);
                 if (W_READY) {           // Q*E of this chunk, for the O products below
                     ok = ok && mbar_wait(bar_full_b, ci & 1, &g_pair_status_word);
-                    b_waited = ci;
+                    if (ok) b_waited = ci;   // else drained at exit
                 }
               if (ok) {
 #pragma unroll
@@ -1413,7 +1413,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             }
             if (POOL && tid == 0) {          // P and K*D of this chunk, for the products below
                 ok = ok && mbar_wait(bar_full_c, ci & 1, &g_pair_status_word);
-                c_waited = ci;
+                if (ok) c_waited = ci;   // else drained at exit
             }
             fence_async_smem();
             tc_fence_before();
@@ -1513,8 +1513,8 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
         if (tid == 0) bulk_wait_all();       // output stores complete before exit
         const bool failed = __syncthreads_or(!ok);
         if (tid == 0 && failed) {   // drain this CTA's own loads and products (bounded)
-            if (!POOL && kq_issued > kq_waited + 1) mbar_wait(bar_kq, (kq_waited + 1) & 1, &g_pair_status_word);
-            if (v_issued > v_waited + 1) mbar_wait(bar_v, (v_waited + 1) & 1, &g_pair_status_word);
+            for (int i = kq_waited + 1; !POOL && i < kq_issued; ++i) mbar_wait(bar_kq, i & 1, &g_pair_status_word);
+            for (int i = v_waited + 1; i < v_issued; ++i) mbar_wait(bar_v, i & 1, &g_pair_status_word);
             if (POOL) {   // record parts still in flight (at most one of each)
                 const int waited[3] = {full_waited, b_waited, c_waited};
                 const uint32_t bars[3] = {bar_full, bar_full_b, bar_full_c};

@@ -98,11 +98,11 @@ constexpr uint32_t OFF_CBH = R_X + 65536;    //   24 KB [half][96][128 B]: rows 
 constexpr uint32_t OFF_CBL = R_X + 90112;    //   24 KB   rows 32-95 K*exp(G_47 - G); one N = 96 B
 constexpr uint32_t CB_HALF = 96 * 128;
 //  (b) after X: derived tiles, P, solve input, U
-constexpr uint32_t OFF_KE = R_X;             //   16 KB K*E fp16  [half][64 r][128 B]
+constexpr uint32_t OFF_KE = R_X;             //   16 KB K*E fp16 [half][K*E 64 r | Q*E 64 r][128 B]:
 constexpr uint32_t OFF_ZH = R_X;              //   after Y: Z^T = V^T - Y^T bf16 hi [128 j][64 r]
 constexpr uint32_t OFF_OST = R_X;            //   at the chunk's end: 32 KB O fp32 [64 t][128 j] (TMA store)
 constexpr uint32_t OFF_OST_LATE = R_X + 81920;  // scalar gate: the same, over A / T / U (see finish_chunk)
-constexpr uint32_t OFF_QE = R_X + 16384;     //   16 KB Q*E fp16
+constexpr uint32_t OFF_QE = R_X + 8192;      //   16 KB Q*E fp16   one N = 128 B operand of Y and O
 constexpr uint32_t OFF_ZL = R_X + 16384;      //   after Y and the first O products: Z^T lo
 constexpr uint32_t OFF_KDH = R_X + 32768;    //   16 KB K*D bf16 hi
 constexpr uint32_t OFF_KDL = R_X + 49152;    //   16 KB K*D bf16 lo
@@ -135,8 +135,8 @@ constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 // ---- TMEM columns (512 allocated) -------------------------------------------
 constexpr uint32_t TM_X = 0;      // X: 128 rows (A rows 0-63, P rows 64-127), N <= 96
 constexpr uint32_t TM_YT = 128;   // Y^T = S^T (K*E)^T: 128 x 64
-constexpr uint32_t TM_UT = 192;   // U^T: 128 x 64
-constexpr uint32_t TM_OT = 256;   // O^T: 128 x 64
+constexpr uint32_t TM_OT = 192;   // O^T: 128 x 64 (next to Y^T: one N = 128 product forms both)
+constexpr uint32_t TM_UT = 256;   // U^T: 128 x 64
 constexpr uint32_t TM_SN = 384;   // SN:  128 x 128
 
 // One launch covers B x nseg x H (batch, time segment, head) problems, and
@@ -563,7 +563,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
         }
         ok = ok && mbar_wait(bar_tma, ci & 1, &g_status_word);
-        tma_waited = ci;
+        if (ok) tma_waited = ci;    // else the exit path drains these loads
         if (tid == 0) bulk_wait_read_all();   // the previous output store has read OFF_OST
         if (__syncthreads_or(!ok)) break;
 
@@ -704,8 +704,9 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     kd[e] = mul2(k2, D2);
                 }
                 const uint32_t o64 = ckh * 8192 + swz(r, ckc);
-                store_f16x8(smem + OFF_KE + o64, ke);
-                store_f16x8(smem + OFF_QE + o64, qe);
+                const uint32_t o128 = ckh * 16384 + swz(r, ckc);
+                store_f16x8(smem + OFF_KE + o128, ke);
+                store_f16x8(smem + OFF_QE + o128, qe);
                 store_split2(smem + OFF_KDH + o64, smem + OFF_KDL + o64, kd);
             }
         }
@@ -720,22 +721,17 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // that they run during the A/P epilogue.  The corrected values follow
         // as U = T' (V - (K*E) S) = T' Z (W S = T' (K*E) S), one product after
         // the solve instead of W^T and U~^T, then U^T -= S^T W^T.
+        // With outputs, one N = 128 product over [K*E; Q*E] forms Y^T (TMEM
+        // columns TM_YT ..) and O^T (TM_OT = TM_YT + 64 ..) together.
+        static_assert(TM_OT == TM_YT + 64, "Y^T and O^T side by side");
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t id_y = idesc_f16(128, 64, true, false);
+            const uint32_t id_y = idesc_f16(128, want_o ? 128 : 64, true, false);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint64_t a = sdesc_sw128(sbase + R_S + ks * 2048, 16384, 1024);
-                const uint64_t bk = sdesc_sw128(sbase + OFF_KE + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+                const uint64_t bk = sdesc_sw128(sbase + OFF_KE + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
                 mma_bf16(tmem + TM_YT, a, bk, id_y, ks > 0);
-            }
-            if (want_o) {
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint64_t a = sdesc_sw128(sbase + R_S + ks * 2048, 16384, 1024);
-                    const uint64_t bq = sdesc_sw128(sbase + OFF_QE + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
-                    mma_bf16(tmem + TM_OT, a, bq, id_y, ks > 0);
-                }
             }
             mma_commit(bar_mma);
         }
