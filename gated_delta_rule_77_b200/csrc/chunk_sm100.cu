@@ -136,7 +136,7 @@ constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 constexpr uint32_t TM_X = 0;      // X: 128 rows (A rows 0-63, P rows 64-127), N <= 96
 constexpr uint32_t TM_YT = 128;   // Y^T = S^T (K*E)^T: 128 x 64
 constexpr uint32_t TM_OT = 192;   // O^T: 128 x 64 (next to Y^T: one N = 128 product forms both)
-constexpr uint32_t TM_UT = 256;   // U^T: 128 x 64
+constexpr uint32_t TM_UT = 256;   // U^T: 128 x 128, Z^T hi T'^T (hi + lo) side by side (summed on load)
 constexpr uint32_t TM_SN = 384;   // SN:  128 x 128
 
 // One launch covers B x nseg x H (batch, time segment, head) problems, and
@@ -861,15 +861,18 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // bf16 hi + lo on both sides, three products per k-step.
         if (tid == 0) {
             tc_fence_after();
+            // Z^T hi times [T' hi; T' lo] (one N = 128 operand: T' lo follows
+            // T' hi) into columns TM_UT .. + 127, Z^T lo times T' hi into the
+            // first 64; the epilogue adds the two halves.
+            static_assert(OFF_TL == OFF_TH + 8192, "T' hi and lo as one operand");
+            const uint32_t id2 = idesc_bf16(128, 128, false, false);
             const uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
                 const uint64_t zh = sdesc_sw128(sbase + OFF_ZH + ks * 32, 16, 1024);
                 const uint64_t zl = sdesc_sw128(sbase + OFF_ZL + ks * 32, 16, 1024);
                 const uint64_t th = sdesc_sw128(sbase + OFF_TH + ks * 32, 16, 1024);
-                const uint64_t tl = sdesc_sw128(sbase + OFF_TL + ks * 32, 16, 1024);
-                mma_bf16(tmem + TM_UT, zh, th, id, ks > 0);
-                mma_bf16(tmem + TM_UT, zh, tl, id, 1);
+                mma_bf16(tmem + TM_UT, zh, th, id2, ks > 0);
                 mma_bf16(tmem + TM_UT, zl, th, id, 1);
             }
             mma_commit(bar_mma);
@@ -884,9 +887,12 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
         // U^T -> bf16 hi + lo [128 j][64 r] (K-major B of SN, K-major A of O^T).
         {
-            float u[32];
+            float u[32], u2[32];
             tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + TM_UT + half * 32, u);
+            tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + TM_UT + 64 + half * 32, u2);
             tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) u[i] += u2[i];
 #pragma unroll
             for (int c = 0; c < 4; ++c)
                 store_split(smem + OFF_UH + swz(srow, half * 4 + c), smem + OFF_UL + swz(srow, half * 4 + c),
