@@ -37,20 +37,22 @@
 // compute mode): a value is carried as a bf16 hi part plus a bf16 lo part
 // and a product takes three bf16 MMAs (hi*hi + hi*lo + lo*hi).  Here that is
 // applied to the operands that need it: the factored operands of A and P,
-// T', P, U and K*D.  The state copy S, W and Q*E, whose magnitudes stay
+// T', P, U, Z and K*D.  The state copy S, K*E and Q*E, whose magnitudes stay
 // moderate, are fp16 operands (4x finer than bf16).  Accumulation is fp32 in
 // TMEM and the output is written in fp32.
 //
 // Products (all 128-row tcgen05.mma; transposed forms put the 128-wide key or
 // value dimension on M):
-//   X   = [K*F;Q*F] (K/F)^T        M = 2C rows, N = 32 / 64 -> A and P (raw)
-//   W^T = (K*E)^T T'^T             M = dk, N = C, K = C
-//   U^T = V^T T'^T - S^T W^T       M = dv, N = C, K = C then dk
-//   O^T = S^T (Q*E)^T + U^T P^T    M = dv, N = C
-//   SN  = (K*D)^T U                M = dk, N = dv, K = C
+//   X       = [K*F;Q*F] (K/F)^T       M = 2C rows, N = 64 / 96 -> A and P (raw)
+//   [Y|O]^T = S^T [K*E; Q*E]^T        M = dv, N = 2C (Y^T = S^T (K*E)^T, O^T = S^T (Q*E)^T)
+//   U^T     = Z^T T'^T, Z = V - Y      M = dv, N = C, K = C  (U = T' V - W S with W S = T' Y)
+//   O^T    += U^T P^T                  M = dv, N = C
+//   SN      = (K*D)^T U                M = dk, N = dv, K = C
 //
-// This version runs the phases of a chunk one after another in one CTA per
-// (batch, head); the next chunk's TMA loads overlap the end of the chunk.
+// The phases of a chunk run one after another in one CTA per (batch, head,
+// segment); with a scalar gate the state step of chunk c runs after chunk
+// c + 1's gate scan and X issue (see finish_chunk), and the next chunk's TMA
+// loads overlap the end of the chunk.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
