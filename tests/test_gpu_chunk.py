@@ -158,7 +158,11 @@ def test_single_cta_pair_and_pool_kernels_agree(gdn, gate, T, monkeypatch):
     SM, state chain on the other) and the prep-pool kernel (chains fed by
     prep CTAs on every other SM through a global slot buffer) compute the same
     chunk algebra.  With 4 pairs and few chunks, most prep CTAs of the pool
-    get no task at all."""
+    get no task at all.  The forms do not share an arithmetic order (the
+    gate's prefix sums, T' = T Diag(beta) formed on different sides, the
+    one-CTA kernel's U from Z = V - Y), so a bf16 operand can round the other
+    way and they agree to the bf16 operands' error (tol / 2), not bit for bit;
+    each form on its own is bit-for-bit repeatable (test_every_form_is_repeatable)."""
     x = prefill_inputs(2, T, 2, 128, 128, gate=gate, s0_std=0.1, seed=230 + T)
     got = {}
     for kernel in ("single", "pair", "pool"):
@@ -266,3 +270,27 @@ def test_second_device_in_the_same_process(gdn, gate):
             assert oracle.rel_err(out.cpu(), ref_o) <= TOL, dev_index
             assert oracle.rel_err(s.cpu(), ref_s) <= TOL, dev_index
             assert gdn.check() == gdn.GDN_OK
+
+
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+@pytest.mark.parametrize("form", ["single", "pair", "pool", "segments"])
+def test_every_form_is_repeatable(gdn, gate, form, monkeypatch):
+    """Two calls on the same inputs give the same bits, in every form of the
+    prefill (no form reads a record, a slot or a staged tile before it is
+    complete, and no reduction depends on timing).  A race between a producer
+    and its consumer shows up here as a difference."""
+    x = prefill_inputs(2, 700, 3, 128, 128, gate=gate, s0_std=0.1, seed=270)
+    dev = torch.device("cuda")
+    args = [x[n].to(dev) for n in ("q", "k", "v", "g", "beta")]
+    s0 = x["s0"].to(dev)
+    if form != "segments":
+        monkeypatch.setenv("GDN_CHUNK_KERNEL", form)
+    seg = 3 if form == "segments" else 1
+    runs = []
+    for _ in range(3):
+        out, s = gdn.chunk_fwd(*args, s0, segments=seg)
+        torch.cuda.synchronize()
+        runs.append((out.cpu(), s.cpu()))
+    assert gdn.check() == gdn.GDN_OK
+    for out, s in runs[1:]:
+        assert torch.equal(out, runs[0][0]) and torch.equal(s, runs[0][1])

@@ -350,3 +350,14 @@ def test_fused_prologue_full_layer_size_sampled_rows(gdn, oracle_threads, route)
                               threads=oracle_threads)
     assert oracle.rel_err(out[rows].cpu(), ref_o) <= 2e-2
     assert _err_vs_max(s_t[rows], ref_s) <= 2e-2
+
+
+@pytest.mark.parametrize("gate", ["channel", "scalar"])
+def test_fused_prologue_prefill_is_repeatable(gdn, gate):
+    """The fused route twice on the same inputs (the ring restored in
+    between): the same bits, outputs, final state and ring alike."""
+    x = prologue_inputs(2, 300, 4, 128, 128, gate=gate, seed=66)
+    s0 = torch.randn(2, 4, 128, 128, generator=torch.Generator().manual_seed(67)) * 0.1
+    runs = [_fused(gdn, x, s0) for _ in range(2)]
+    for a, b in zip(runs[0], runs[1]):
+        assert torch.equal(a.cpu(), b.cpu())
