@@ -80,13 +80,13 @@ constexpr uint32_t P_IN = 0;                  // 32 KB raw K, Q [half][K 64 | Q 
 constexpr uint32_t P_X = 32768;               // 112 KB:
 constexpr uint32_t P_AH = P_X;                //   X operands (per-channel): 32 KB
 constexpr uint32_t P_AL = P_X + 32768;        //   32 KB
-// B operand of X, hi and lo, [64-channel half][96 rows][128 B]: rows 0-31 =
-// K/F of tokens 0-31 (reference 15), rows 32-95 = K*exp(G_47 - G) of tokens
-// 0-63, so that one N = 96 product per k-step covers both (fewer operand
-// reads from shared memory than separate N = 32 and N = 64 products).
-constexpr uint32_t P_CBH = P_X + 65536;       //   24 KB
-constexpr uint32_t P_CBL = P_X + 90112;       //   24 KB
-constexpr uint32_t CB_HALF = 96 * 128;
+// B operand of X, [64-channel half][hi rows 0-95 | lo rows 0-95][128 B]:
+// rows 0-31 = K/F of tokens 0-31 (reference 15), rows 32-95 = K*exp(G_47 - G)
+// of tokens 0-63, so that one N = 96 product per k-step covers both; hi and
+// lo back to back make [hi; lo] one N = 192 operand (A hi times both in one
+// product, see the X issue).
+constexpr uint32_t P_CB = P_X + 65536;        //   48 KB
+constexpr uint32_t CB_HALF = 96 * 128;        //   one of hi / lo of one channel half
 constexpr uint32_t P_A = P_X + 32768;         //   16 KB A fp32 (fidx layout)
 constexpr uint32_t P_T = P_X + 49152;         //   16 KB T fp32 (tidx layout)
 constexpr uint32_t P_Y = P_X + 65536;         //   10 KB solve scratch 2 x [32][40]
@@ -333,7 +333,7 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
         for (int i = 0; i < (rank == 0 ? 4 : 7); ++i) mbar_init(bar0 + 8 * i, 1);
         fence_mbar_init();
     }
-    const uint32_t tmem_cols = rank == 0 ? 128 : 512;
+    const uint32_t tmem_cols = rank == 0 ? 256 : 512;   // prep: X with its hi / lo halves
     if (warp == 0) {
         tmem_alloc(sbase + (rank == 0 ? P_TMEM : C_TMEM), tmem_cols);
         tmem_relinquish();
@@ -767,11 +767,11 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                     store_split2(smem + P_AH + o128, smem + P_AL + o128, kr);
                     store_split2(smem + P_AH + o128q, smem + P_AL + o128q, qr);
                     if (u < 2) {
-                        const uint32_t o32 = ckh * CB_HALF + swz(r, ckc);
-                        store_split2(smem + P_CBH + o32, smem + P_CBL + o32, kc);
+                        const uint32_t o32 = ckh * 2 * CB_HALF + swz(r, ckc);
+                        store_split2(smem + P_CB + o32, smem + P_CB + CB_HALF + o32, kc);
                     }
-                    const uint32_t o64 = ckh * CB_HALF + swz(32 + r, ckc);
-                    store_split2(smem + P_CBH + o64, smem + P_CBL + o64, kc1);
+                    const uint32_t o64 = ckh * 2 * CB_HALF + swz(32 + r, ckc);
+                    store_split2(smem + P_CB + o64, smem + P_CB + CB_HALF + o64, kc1);
                 }
                 fence_async_smem();
                 __syncthreads();
@@ -779,17 +779,19 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
             if (tid == 0) {
                 tc_fence_after();
                 if (CHANNEL) {
+                    // A hi times [B hi; B lo] (N = 192) into TM_X .. + 191, A lo
+                    // times B hi into the first 96 columns; the epilogue adds
+                    // the two 96-column halves.
+                    const uint32_t id2 = idesc_bf16(128, 192, false, false);
                     const uint32_t id = idesc_bf16(128, 96, false, false);
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {
                         const uint32_t ka = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        const uint32_t kb = (ks >> 2) * CB_HALF + (ks & 3) * 32;
+                        const uint32_t kb = (ks >> 2) * 2 * CB_HALF + (ks & 3) * 32;
                         const uint64_t ah = sdesc_sw128(sbase + P_AH + ka, 16, 1024);
                         const uint64_t al = sdesc_sw128(sbase + P_AL + ka, 16, 1024);
-                        const uint64_t bh = sdesc_sw128(sbase + P_CBH + kb, 16, 1024);
-                        const uint64_t bl = sdesc_sw128(sbase + P_CBL + kb, 16, 1024);
-                        mma_bf16(tmem + TM_X, ah, bh, id, ks > 0);
-                        mma_bf16(tmem + TM_X, ah, bl, id, 1);
+                        const uint64_t bh = sdesc_sw128(sbase + P_CB + kb, 16, 1024);
+                        mma_bf16(tmem + TM_X, ah, bh, id2, ks > 0);
                         mma_bf16(tmem + TM_X, al, bh, id, 1);
                     }
                 } else {
@@ -897,15 +899,22 @@ __device__ __forceinline__ void pair_body(const CUtensorMap& tm_q, const CUtenso
                 const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
                 bool zero = false;
                 if (CHANNEL) {
-                    if (r < 32) {
-                        if (half == 0) tmem_ld32(lane_base + TM_X, x); else zero = true;
-                    } else {
-                        tmem_ld32(lane_base + TM_X + 32 + half * 32, x);
+                    float x2[32];
+                    const uint32_t col = r < 32 ? 0u : 32u + half * 32u;
+                    zero = r < 32 && half != 0;
+                    if (!zero) {
+                        tmem_ld32(lane_base + TM_X + col, x);
+                        tmem_ld32(lane_base + TM_X + 96 + col, x2);
+                    }
+                    tmem_wait_ld();
+                    if (!zero) {
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) x[jj] += x2[jj];
                     }
                 } else {
                     tmem_ld32(lane_base + TM_X + half * 32, x);
+                    tmem_wait_ld();
                 }
-                tmem_wait_ld();
                 if (zero) {
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) x[jj] = 0.f;
