@@ -99,3 +99,16 @@ def test_max_over_ranks_gloo_two_ranks():
         assert p.exitcode == 0
     got = sorted(q.get(timeout=10) for _ in range(2))
     assert got == [(0, 11.0), (1, 11.0)]
+
+
+def test_traffic_figures_follow_the_kernel_and_its_sources(monkeypatch):
+    """bench.py reports an ncu traffic figure only for the kernel it was
+    captured on and only while the kernel's sources hash as at the capture."""
+    entry = json.loads(bench.TRAFFIC_FILE.read_text())["decode"]
+    assert bench.ncu_traffic("decode") == float(entry["dram_bytes_per_launch"])
+    assert bench.ncu_traffic("no_such_workload") is None
+    layer = json.loads(bench.TRAFFIC_FILE.read_text())["gdn2_layer"]
+    assert bench.ncu_traffic("gdn2_layer", "chunk_pool_kernel") == float(layer["dram_bytes_per_launch"])
+    assert bench.ncu_traffic("gdn2_layer", "chunk_fwd_kernel (zero-start + transition CTAs)") is None
+    monkeypatch.setattr(bench, "source_sha1", lambda names: "0" * 40)
+    assert bench.ncu_traffic("decode") is None
